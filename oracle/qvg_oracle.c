@@ -316,6 +316,12 @@ void ref_group_quant(const float* R, int64_t N, int d, int G,
                 if (r[j] < lo) lo = r[j];
                 if (r[j] > hi) hi = r[j];
             }
+            /* READING: a minimum or maximum of -0 is taken as +0 (adding +0
+             * maps -0 to +0 and leaves every other value unchanged), so the
+             * stored bytes never depend on which of two equal zeros is met
+             * first. */
+            lo = lo + 0.0f;
+            hi = hi + 0.0f;
             zc = ref_e4m3_encode(lo);
             m = ref_e4m3_decode(zc);
             span = hi - m;
@@ -367,6 +373,7 @@ int ref_quantize(int K, int T, int G, int iters, int dtype, const void* X,
     float *R, *R2, *C;
     if (K < 1 || K > 256 || T < 0 || G < 4 || G % 4 || d % G || d % 4 || N < 1 || H < 1 || iters < 0)
         return -1;
+    if (T > 0 && iters < 1) return -1;     /* assignments need one assign step */
     if (T > 0 && init == NULL && N < K) return -1;
     R = (float*)malloc((size_t)(N * d) * sizeof(float));
     R2 = (float*)malloc((size_t)(N * d) * sizeof(float));

@@ -41,6 +41,15 @@ def test_group_quant_grid_values_are_exact(ora):
     assert q == [2, 0, 3, 1, 1, 3, 0, 2]
 
 
+def test_signed_zero_extremes_are_canonical(ora):
+    """A group whose minimum or maximum is -0 stores the same bytes as +0."""
+    a = ora.group_quant(np.array([[-0.0, 0.0, 0.0, -0.0]], np.float32), 4)
+    b = ora.group_quant(np.array([[0.0, 0.0, 0.0, 0.0]], np.float32), 4)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+    assert a[1][0, 0] == 0 and a[2][0, 0] == 0
+
+
 def test_constant_group_has_zero_scale(ora):
     codes, scale, zero = ora.group_quant(np.full((1, 8), 1.5, np.float32), 8)
     assert scale[0, 0] == 0 and ora.e4m3_decode(zero)[0, 0] == 1.5 and np.all(codes == 0)
@@ -169,7 +178,7 @@ def test_smoothing_lowers_error_vs_rtn(ora):
 
 def test_invalid_arguments_rejected(ora):
     X = np.zeros((1, 8, 16), np.float32)
-    for kw in (dict(K=0), dict(K=257), dict(G=6), dict(G=32), dict(K=9, T=1)):
+    for kw in (dict(K=0), dict(K=257), dict(G=6), dict(G=32), dict(K=9, T=1), dict(iters=0)):
         args = dict(K=4, T=1, G=8, iters=2)
         args.update(kw)
         with pytest.raises(ValueError):
