@@ -1,0 +1,370 @@
+#!/usr/bin/env python
+"""Benchmark of the QVG 2-bit KV-cache codec on B200.
+
+One step = the whole hot path over one batch of synthetic KV: k-means
+semantic-aware smoothing with T progressive residual stages + 2-bit group
+quantisation of every block (qvg_quantize), then the fused reconstruction of
+every block (qvg_dequantize).  Default workload: the LongCat-scale cache --
+48 layers x 32 heads x {K, V} = 3,072 blocks of 38,000 tokens (25 frames of
+38x40 latents), d = 128, bf16 (29.9 GB), K = 256, T = 2, G = 64, 10 Lloyd
+iterations.  The metric is KV GB/s: uncompressed bf16 KV bytes / step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload longcat|chunk]
+    python bench.py --impl reference ...   # the oracle on the host cores
+
+Multi-GPU (torchrun, one process per GPU): every rank compresses and
+reconstructs its own cache of the same size (weak scaling, no collective on
+the data path); time = max over ranks of the device-timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV GB/s: fused dequant + k-means/2-bit quantize, as % of B200 HBM roofline"
+
+WORKLOADS = {
+    "longcat": dict(layers=48, heads=32, frames=25, gh=38, gw=40, K=256, T=2, G=64, iters=10,
+                    desc="LongCat-scale full cache: 48 layers x 32 heads x K/V, 38,000 tokens "
+                         "(25 frames x 38x40), d=128, bf16; K=256, T=2, G=64, 10 Lloyd iterations"),
+    "chunk": dict(layers=1, heads=12, frames=3, gh=30, gw=52, K=256, T=2, G=64, iters=8,
+                  desc="Self-Forcing-scale chunk: 1 layer x 12 heads x K/V, 4,680 tokens "
+                       "(3 frames x 30x52), d=128, bf16; K=256, T=2, G=64, 8 Lloyd iterations"),
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sus=p["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.rows, self.proc = index, [], None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm = [float(r[1]) for r in self.rows if len(r) >= 9 and r[1].replace('.', '', 1).isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) >= 9 and r[2].replace('.', '', 1).isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in self.rows if len(r) >= 9 for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle arm
+def oracle_sample(wl, tokens: int, seed: int = 99):
+    """Time the oracle's quantise + dequantise of one block of `tokens` tokens
+    of the workload's shape on the host cores.  Returns (seconds, bytes, threads)."""
+    import numpy as np
+    from bit_kv_cache_qvg_b200 import synth
+    from oracle import oracle as o
+    o.build()
+    frames = max(1, math.ceil(tokens / (wl["gh"] * wl["gw"])))
+    X = synth.block_batch(1, synth.KVShape(frames, wl["gh"], wl["gw"]), seed=seed, kinds=[1])[:, :tokens]
+    Xb = X.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
+    t0 = time.perf_counter()
+    p = o.quantize(Xb, K=wl["K"], T=wl["T"], G=wl["G"], iters=wl["iters"])
+    o.dequantize(p, K=wl["K"], T=wl["T"], G=wl["G"], N=tokens, H=1, d=128)
+    dt = time.perf_counter() - t0
+    return dt, tokens * 128 * 2, o.get_threads()
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    tokens = args.ref_tokens
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, nbytes, threads = oracle_sample(wl, tokens, seed=1000 + i)
+        if i >= args.warmup:
+            times.append(dt)
+    t = sum(times) / len(times)
+    v = nbytes / t / 1e9
+    sample = f"one V block of {tokens} tokens of the workload's shape per step (quantise + dequantise)"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl["desc"], "reference": "C oracle (fp64 k-means) on host cores"},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+# ---------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="longcat", choices=sorted(WORKLOADS))
+    ap.add_argument("--layers", type=int, default=None, help="override the layer count")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=4750)
+    ap.add_argument("--cpu-tokens", type=int, default=9500)
+    args = ap.parse_args()
+    wl = dict(WORKLOADS[args.workload])
+    if args.layers:
+        wl["layers"] = args.layers
+        wl["desc"] += f" [{args.layers} layers]"
+
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    from bit_kv_cache_qvg_b200 import build, qvg, synth
+    if rank == 0 or world == 1:
+        build.build()
+    if dist is not None:
+        dist.barrier()
+    qvg.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+
+    L, Hh = wl["layers"], wl["heads"]
+    N = wl["frames"] * wl["gh"] * wl["gw"]
+    U = L * 2 * Hh                      # blocks: layer x {K, V} x head
+    K, T, G, I = wl["K"], wl["T"], wl["G"], wl["iters"]
+    cfg = qvg.config(K=K, T=T, group_size=G, iters=I)
+
+    # inputs resident in HBM (generated per layer on the device, seeded per rank)
+    X = torch.empty((U, N, 128), dtype=torch.bfloat16, device=dev)
+    for l in range(L):
+        kinds = [0] * Hh + [1] * Hh
+        X[l * 2 * Hh:(l + 1) * 2 * Hh] = synth.block_batch(
+            2 * Hh, synth.KVShape(wl["frames"], wl["gh"], wl["gw"]), seed=synth.unit_seed(rank, l, 0, 0),
+            kinds=kinds, device=dev)
+    packed = qvg.alloc_packed(cfg, N, U, device=dev)
+    ws = qvg.alloc_workspace(cfg, N, U, device=dev)
+    Y = torch.empty_like(X)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        qvg.quantize(X, cfg, out=packed, workspace=ws, stream=stream)
+        qvg.dequantize(packed, Y, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if qvg.workspace_status(ws) != 0:
+        raise SystemExit("device-side wait timed out during warm-up")
+
+    # timed region: inputs (29.9 GB for the default workload) exceed L2, no flush needed
+    qvg.profile_reset()
+    qvg.profile_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+    qvg.profile_enable(False)
+    launches = qvg.profile_launches()
+    kernels = qvg.profile_report()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    kv_bytes = U * N * 128 * 2
+    value = kv_bytes * world / (ms / 1e3) / 1e9
+
+    # roofline of the kernels (algorithmic work per launch / mean launch time)
+    E = U * N * 128
+    esz = 2
+    deq_bytes_per_elem = 2 / 8 + 2 / G + T / 128 + esz * T * K / N + 2
+    roof = {}
+    if "qvg_dequant_fused" in kernels:
+        k = kernels["qvg_dequant_fused"]
+        t_launch = k["ms"] / max(k["timed"], 1) / 1e3
+        per_launch = deq_bytes_per_elem * E
+        roof["qvg_dequant_fused"] = {"bound": "hbm", "achieved": per_launch / t_launch / 1e9,
+                                     "peak": peaks["hbm"], "unit": "GB/s",
+                                     "frac": per_launch / t_launch / 1e9 / peaks["hbm"], "traffic": None,
+                                     "alg_bytes_per_launch": per_launch}
+    for name in ("qvg_kmeans_assign", "qvg_assign_exact"):
+        if name in kernels and kernels[name]["timed"]:
+            k = kernels[name]
+            flops_total = 2.0 * K * 128 * N * U * T * I * args.steps
+            # an assign launch covers one batch of blocks for one Lloyd iteration
+            per_launch = flops_total / k["timed"]
+            t_launch = k["ms"] / k["timed"] / 1e3
+            ach = per_launch / t_launch / 1e12
+            roof[name] = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+                          "frac": ach / peaks["bf16_sus"], "traffic": None,
+                          "alg_flops_per_launch": per_launch}
+    top = max(kernels.items(), key=lambda kv: kv[1]["ms"])[0] if kernels else None
+    dominant = roof.get(top) if top in roof else (next(iter(roof.values())) if roof else None)
+    if dominant is not None:
+        dominant = dict(dominant, kernel=top if top in roof else next(iter(roof)))
+
+    # quantise-path roofline: max(F / P_bf16, B / BW)
+    q_ms = sum(v["ms"] for n, v in kernels.items() if n != "qvg_dequant_fused") / args.steps
+    F = 2.0 * K * I * T * E
+    B = E * 2 + packed.nbytes()
+    q_roof_ms = max(F / (peaks["bf16_sus"] * 1e12), B / (peaks["hbm"] * 1e9)) * 1e3
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl["desc"], "blocks_per_gpu": U, "tokens_per_block": N,
+                   "uncompressed_bytes_per_gpu": kv_bytes, "packed_bytes_per_gpu": packed.nbytes(),
+                   "l2": "inputs larger than L2 (no flush needed)" if kv_bytes > 126e6 else "L2 flushed",
+                   "parallelism": f"weak: {world} rank(s), independent caches"},
+        "roofline": dominant,
+        "rooflines": roof,
+        "quantize_path": {"ms_per_step": q_ms, "roofline_ms": q_roof_ms, "frac": q_roof_ms / q_ms if q_ms else None,
+                          "peak_source": peaks["source"]},
+        "kernels": kernels,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+
+    # end to end through the public API with host buffers (pinned), per layer
+    if not args.no_e2e:
+        result["e2e"] = e2e(args, qvg, cfg, X, Y, packed, ws, L, Hh, N, dev, world, dist)
+    if rank == 0 and not args.no_cpu_baseline:
+        dt, nbytes, threads = oracle_sample(wl, args.cpu_tokens)
+        result["cpu_baseline"] = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                  "sample": f"one V block of {args.cpu_tokens} tokens of the workload's shape "
+                                            f"(quantise + dequantise), {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(result))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e(args, qvg, cfg, X, Y, packed, ws, L, Hh, N, dev, world, dist):
+    """Same step, but every layer's K/V arrive from pinned host memory and every
+    layer's reconstruction returns to pinned host memory inside the timed
+    region; copies overlap the codec on separate streams."""
+    import psutil
+    import torch
+    layer_bytes = 2 * Hh * N * 128 * 2
+    avail = psutil.virtual_memory().available
+    nh = int(max(1, min(L, (0.25 * avail) // (2 * layer_bytes))))
+    Xh = [torch.empty((2 * Hh, N, 128), dtype=torch.bfloat16, pin_memory=True) for _ in range(nh)]
+    Yh = [torch.empty((2 * Hh, N, 128), dtype=torch.bfloat16, pin_memory=True) for _ in range(nh)]
+    for i in range(nh):
+        Xh[i].copy_(X[i * 2 * Hh:(i + 1) * 2 * Hh])
+    comp = torch.cuda.current_stream(dev)
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    U = X.shape[0]
+    # The packed layout is [T][H][...]; per-layer slices of assign/centroids are
+    # strided over T, so each layer gets its own contiguous packed buffers.
+    lp = [qvg.alloc_packed(cfg, N, 2 * Hh, device=dev) for _ in range(2)]
+    lws = qvg.alloc_workspace(cfg, N, 2 * Hh, device=dev)
+
+    def step():
+        done_in = []
+        for l in range(L):
+            s = slice(l * 2 * Hh, (l + 1) * 2 * Hh)
+            with torch.cuda.stream(h2d):
+                X[s].copy_(Xh[l % nh], non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(h2d)
+            done_in.append(e)
+        for l in range(L):
+            s = slice(l * 2 * Hh, (l + 1) * 2 * Hh)
+            comp.wait_event(done_in[l])
+            p = lp[l % 2]
+            qvg.quantize(X[s], cfg, out=p, workspace=lws, stream=comp)
+            qvg.dequantize(p, Y[s], stream=comp)
+            e = torch.cuda.Event()
+            e.record(comp)
+            d2h.wait_event(e)
+            with torch.cuda.stream(d2h):
+                Yh[l % nh].copy_(Y[s], non_blocking=True)
+        comp.wait_stream(d2h)
+        comp.wait_stream(h2d)
+
+    step()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0.record(comp)
+    for _ in range(args.steps):
+        step()
+    ev1.record(comp)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    nbytes = U * N * 128 * 2
+    return {"value": nbytes * world / (ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+            "host_layers_distinct": nh, "api": "qvg_quantize + qvg_dequantize per layer (64 blocks)"}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,468 @@
+// kernel_assign_tc.cu -- qvg_kmeans_assign: the k-means assignment step of
+// semantic-aware smoothing (m.163.com article on Quant VideoGen, section 三)
+// as a tensor-core contraction on sm_100a.
+//
+// For a tile of 128 tokens R (bf16) and the block's K <= 256 centroids C
+// (bf16), tcgen05.mma (kind::f16, M=128, N=Kpad, fp32 accumulate) computes the
+// 128 x Kpad dot products r_i . c_k into tensor memory.  The epilogue warps
+// read them back with tcgen05.ld and form the screening values
+// g_ik = |c_k|^2 - 2 r_i . c_k (argmin_k g_ik = argmin_k |r_i - c_k|^2),
+// keeping the smallest two per token.  If the runner-up lies within the
+// rounding-error bound of the minimum, the token is appended to a per-block
+// list that an exact fp64 pass (qvg_assign_exact in list mode) decides;
+// otherwise the minimum's index is the assignment.
+//
+// Data movement: the centroid table is loaded once per CTA with TMA (128-byte
+// swizzle, K-major), token tiles stream through a 3-stage TMA ring; no
+// multicast.  Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (one
+// elected thread) and TMEM owner, warps 2-9 = epilogue (two warps per TMEM
+// lane quarter, each owning half of the centroid columns).  Two TMEM
+// accumulators (2 x 256 columns) let the epilogue of tile i overlap the MMAs
+// of tile i+1.  Every mbarrier wait is bounded; on timeout the kernel records
+// an error in the status word, drains, frees TMEM and returns.
+#include <cuda.h>
+#include <cstdio>
+
+#include "qvg_common.cuh"
+#include "qvg_launch.h"
+
+namespace qvg {
+namespace {
+
+constexpr int kTcThreads = 320;     // 10 warps
+constexpr int kStages = 3;
+constexpr int kTileM = 128;
+constexpr int kAStageBytes = kTileM * kD * 2;     // 32 KB: two 16 KB K-halves
+constexpr int kAHalfBytes = kTileM * 128;         // 128 rows x 128 B
+#ifdef QVG_TC_DEBUG
+constexpr uint64_t kWaitLimitNs = 50000000ull;     // 50 ms in the self-checking build
+#else
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s of wall time per wait
+#endif
+constexpr uint32_t kStatusTimeout = 1u;
+
+struct __align__(8) TcSmemBarriers {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t b_full;
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for the phase of `parity` to complete: gives up after
+// kWaitLimitNs of wall time and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((it & 63u) == 0u) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kWaitLimitNs) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), leading offset unused (1), descriptor version 1.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;                 // LBO (16-byte units)
+  d |= (uint64_t)(1024 >> 4) << 32;       // SBO
+  d |= (uint64_t)1 << 46;                 // version
+  d |= (uint64_t)2 << 61;                 // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor: kind::f16, A = B = bf16, D = f32, both K-major.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns -> 32 registers per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+struct TcParams {
+  const float* rnorm2;      // [W][N]
+  const float* cn;          // [W][K]
+  uint8_t* pi;              // [W][N]
+  uint32_t* list;           // [W][N]
+  uint32_t* list_count;     // [W]
+  uint32_t* status;         // workspace status word
+  unsigned long long* flagged;
+  int64_t N;
+  int K;
+  int Npad;                 // K rounded up to 16 (MMA N)
+  int tiles_per_unit;
+  int tiles_per_cta;
+  float gamma;              // relative error bound of the tensor-core dot products
+};
+
+#ifdef QVG_TC_DEBUG
+// Self-checking build: where each role gave up, and how far each got.
+//   [0..3]  producer: empty-wait gave up at tile+1, b_full drain
+//   [4..7]  mma: b_full, tmem_empty, full wait gave up at tile+1
+//   [8..11] epilogue: tmem_full wait gave up at tile+1
+//   [16] tiles produced, [17] tiles issued to MMA, [18] tiles consumed
+__device__ uint32_t g_tc_dbg[32];
+#define TC_DBG(i, v) do { if (blockIdx.x == 0 && blockIdx.y == 0) atomicMax(&g_tc_dbg[i], (uint32_t)(v)); } while (0)
+#else
+#define TC_DBG(i, v) do { } while (0)
+#endif
+
+__device__ __forceinline__ int aborted(const TcSmemBarriers* b) {
+  return *reinterpret_cast<const volatile int*>(&b->abort_flag);
+}
+__device__ __forceinline__ void set_abort(TcSmemBarriers* b) {
+  *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
+}
+
+__device__ __forceinline__ float key_with_index(float g, int k) {
+  return __int_as_float((__float_as_int(g) & ~0xFF) | k);
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmC,
+                  const TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int u = blockIdx.y;
+  const int t_begin = blockIdx.x * p.tiles_per_cta;
+  const int t_end = min(p.tiles_per_unit, t_begin + p.tiles_per_cta);
+  if (t_begin >= t_end) return;
+  const int ntiles = t_end - t_begin;
+
+  const int Npad = p.Npad;
+  uint8_t* sB = smem;                                           // 2 x Npad x 128 B
+  uint8_t* sA = smem + 2 * Npad * 128;                          // kStages x 32 KB (1024-aligned)
+  float* cn_s = reinterpret_cast<float*>(sA + kStages * kAStageBytes);   // [256]
+  float* mbuf = cn_s + kMaxK;                                   // [2 acc][2 vals][128 rows]
+  TcSmemBarriers* bars = reinterpret_cast<TcSmemBarriers*>(mbuf + 2 * 2 * kTileM);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&bars->full[s], 1); mbar_init(&bars->empty[s], 1); }
+    mbar_init(&bars->b_full, 1);
+    for (int a = 0; a < 2; ++a) { mbar_init(&bars->tmem_full[a], 1); mbar_init(&bars->tmem_empty[a], 8); }
+    bars->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(&bars->tmem_base)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  for (int k = threadIdx.x; k < kMaxK; k += blockDim.x)
+    cn_s[k] = k < p.K ? p.cn[(int64_t)u * p.K + k] : __int_as_float(0x7f800000);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      mbar_expect_tx(&bars->b_full, (uint32_t)(2 * Npad * 128));
+      tma_load_3d(sB, &tmC, 0, 0, u, &bars->b_full);
+      tma_load_3d(sB + Npad * 128, &tmC, 64, 0, u, &bars->b_full);
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+        if (!mbar_wait(&bars->empty[s], ph ^ 1u) || aborted(bars)) { TC_DBG(0, i + 1); set_abort(bars); break; }
+        uint8_t* a = sA + s * kAStageBytes;
+        const int row = (t_begin + i) * kTileM;
+        mbar_expect_tx(&bars->full[s], (uint32_t)kAStageBytes);
+        tma_load_3d(a, &tmR, 0, row, u, &bars->full[s]);
+        tma_load_3d(a + kAHalfBytes, &tmR, 64, row, u, &bars->full[s]);
+        ++issued;
+        TC_DBG(16, issued);
+      }
+      if (aborted(bars)) {        // drain: wait (bounded) for the loads in flight
+        for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+          mbar_wait(&bars->full[i % kStages], (uint32_t)(i / kStages) & 1u);
+        mbar_wait(&bars->b_full, 0);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(kTileM, Npad);
+      const uint32_t b_addr = smem_u32(sB);
+      bool ok = mbar_wait(&bars->b_full, 0);
+      if (!ok) TC_DBG(4, 1);
+      int issued = 0;
+      for (int i = 0; ok && i < ntiles; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+        const int acc = i & 1;
+        const uint32_t aph = (uint32_t)(i >> 1) & 1u;
+        if (!mbar_wait(&bars->tmem_empty[acc], aph ^ 1u)) { TC_DBG(5, i + 1); ok = false; break; }
+        if (!mbar_wait(&bars->full[s], ph)) { TC_DBG(6, i + 1); ok = false; break; }
+        if (aborted(bars)) { TC_DBG(7, i + 1); ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(sA + s * kAStageBytes);
+        const uint32_t d_tmem = tmem + (uint32_t)(acc * 256);
+#pragma unroll
+        for (int k = 0; k < kD / 16; ++k) {
+          const uint32_t koff = (uint32_t)((k & 3) * 32);
+          const uint64_t ad = umma_desc_sw128(a_addr + (k >> 2) * kAHalfBytes + koff);
+          const uint64_t bd = umma_desc_sw128(b_addr + (k >> 2) * Npad * 128 + koff);
+          umma_bf16(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&bars->empty[s]);
+        umma_commit(&bars->tmem_full[acc]);
+        ++issued;
+        TC_DBG(17, issued);
+      }
+      if (!ok) {
+        set_abort(bars);
+        if (issued > 0) mbar_wait(&bars->tmem_full[(issued - 1) & 1], (uint32_t)((issued - 1) >> 1) & 1u);
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..9)
+    const int q = warp & 3;                  // TMEM lane quarter this warp may access
+    const int hc = (warp - 2) >> 2;          // centroid-column half
+    const int row = q * 32 + lane;
+    const int ncol = Npad > 128 ? Npad - 128 : 0;
+    const int cols = hc == 0 ? min(Npad, 128) : ncol;
+    for (int i = 0; i < ntiles; ++i) {
+      const int acc = i & 1;
+      const uint32_t aph = (uint32_t)(i >> 1) & 1u;
+      const bool ok = !aborted(bars) && mbar_wait(&bars->tmem_full[acc], aph);
+      if (!ok) { TC_DBG(8, i + 1); set_abort(bars); }
+      else if (lane == 0 && warp == 2) TC_DBG(18, i + 1);
+      tc_fence_after();
+      float v1 = __int_as_float(0x7f800000), v2 = v1;
+      if (ok) {
+        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256 + hc * 128);
+        for (int c0 = 0; c0 < cols; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tbase + (uint32_t)c0, r);
+          const int kb = hc * 128 + c0;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float g = __fmaf_rn(-2.0f, __uint_as_float(r[e]), cn_s[kb + e]);
+            const float key = key_with_index(g, kb + e);
+            v2 = fminf(v2, fmaxf(v1, key));
+            v1 = fminf(v1, key);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->tmem_empty[acc]);
+      float* mb = mbuf + acc * 2 * kTileM;
+      if (hc == 1) { mb[row] = v1; mb[kTileM + row] = v2; }
+      named_bar_sync(1, 256);
+      if (hc == 0) {
+        const float o1 = mb[row], o2 = mb[kTileM + row];
+        const float w1 = fminf(v1, o1);
+        const float w2 = fminf(fmaxf(v1, o1), fminf(v2, o2));
+        const int64_t tok = (int64_t)(t_begin + i) * kTileM + row;
+        const bool valid = tok < p.N && !aborted(bars);
+        const int64_t gi = (int64_t)u * p.N + tok;
+        bool flag = false;
+        if (valid) {
+          // error bound of the screening values (see qvg_assign_exact) plus the
+          // 2^-15 relative perturbation of the index bits in both keys
+          const float rn2 = p.rnorm2[gi];
+          const float nr = sqrtf(fmaxf(rn2, 0.0f)) * 1.0001f;
+          const float cb = 1.02f * nr + sqrtf(fmaxf(rn2 + w1, 0.0f));
+          const float E = 2.0f * p.gamma * nr * cb + 1.2e-7f * cb * cb + 1.2e-7f * fabsf(w1) + 1e-30f;
+          const float margin = 2.0f * E + 6.2e-5f * (fabsf(w1) + fabsf(w2));
+          flag = !(w2 - w1 > margin);
+          if (!flag) p.pi[gi] = (uint8_t)(__float_as_int(w1) & 0xFF);
+        }
+        // every lane of the warp takes part in the list append
+        const unsigned fm = __ballot_sync(0xffffffffu, flag);
+        if (fm) {
+          const int leader = __ffs(fm) - 1;
+          uint32_t base = 0;
+          if (lane == leader) {
+            base = atomicAdd(&p.list_count[u], (uint32_t)__popc(fm));
+            atomicAdd(p.flagged, (unsigned long long)__popc(fm));
+          }
+          base = __shfl_sync(0xffffffffu, base, leader);
+          if (flag) p.list[(int64_t)u * p.N + base + __popc(fm & ((1u << lane) - 1u))] = (uint32_t)tok;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (aborted(bars) && threadIdx.x == 0) atomicOr(p.status, kStatusTimeout);
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// 3-D bf16 map over [W][rows][128]: box = 64 channels (128 B, swizzled) x box_rows x 1.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int W, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)W};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)rows * kD * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t assign_tc_smem_bytes(int K) {
+  const int Npad = (K + 15) & ~15;
+  return 1024 + 2 * (size_t)Npad * 128 + (size_t)kStages * kAStageBytes + kMaxK * 4 + 2 * 2 * kTileM * 4 +
+         sizeof(TcSmemBarriers);
+}
+
+cudaError_t launch_assign_tc(const AssignTcParams& a, cudaStream_t s) {
+  CUtensorMap mR, mC;
+  const int Npad = (a.K + 15) & ~15;
+  if (!make_map(&mR, a.R, a.N, a.W, kTileM) || !make_map(&mC, a.C, a.K, a.W, Npad))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.rnorm2 = a.rnorm2; p.cn = a.cn; p.pi = a.pi; p.list = a.list; p.list_count = a.list_count;
+  p.status = a.status; p.flagged = a.flagged; p.N = a.N; p.K = a.K; p.Npad = Npad;
+  p.tiles_per_unit = (int)((a.N + kTileM - 1) / kTileM);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int splits = sms / a.W;
+  if (splits < 1) splits = 1;
+  p.tiles_per_cta = (p.tiles_per_unit + splits - 1) / splits;
+  if (p.tiles_per_cta < 2) p.tiles_per_cta = 2;
+  splits = (p.tiles_per_unit + p.tiles_per_cta - 1) / p.tiles_per_cta;
+  p.gamma = a.gamma;
+  const size_t smem = assign_tc_smem_bytes(a.K);
+  cudaError_t e = cudaFuncSetAttribute(qvg_kmeans_assign, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+#ifdef QVG_TC_DEBUG
+  {
+    uint32_t z[32] = {};
+    cudaMemcpyToSymbol(g_tc_dbg, z, sizeof(z));
+  }
+#endif
+  qvg_kmeans_assign<<<dim3((unsigned)splits, (unsigned)a.W), kTcThreads, smem, s>>>(mR, mC, p);
+#ifdef QVG_TC_DEBUG
+  {
+    cudaError_t le = cudaDeviceSynchronize();
+    uint32_t h[32] = {};
+    cudaMemcpyFromSymbol(h, g_tc_dbg, sizeof(h));
+    fprintf(stderr, "[tc-debug] grid=(%d,%d) tiles/cta=%d Npad=%d smem=%zu err=%s dbg:", splits, a.W,
+            p.tiles_per_cta, Npad, smem, cudaGetErrorString(le));
+    for (int i = 0; i < 20; ++i) fprintf(stderr, " %u", h[i]);
+    fprintf(stderr, "\n");
+  }
+#endif
+  return cudaGetLastError();
+}
+
+}  // namespace qvg

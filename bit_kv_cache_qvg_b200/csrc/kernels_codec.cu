@@ -1,0 +1,440 @@
+// kernels_codec.cu -- memory-bound codec kernels for sm_100a:
+//   * qvg_dequant_fused: unpack 2-bit codes, dequantise with the E4M3 group
+//     scale and zero point, add every stage's centroid in reverse stage order,
+//     write the storage dtype -- one pass, values kept in registers (m.163.com
+//     article on Quant VideoGen, section 五, fused dequantisation kernel;
+//     gist.science/de, Technische Zusammenfassung 2C "Fused Kernel").
+//   * qvg_residual / qvg_residual_quant: R(t) = round(R(t-1) - C(t)[pi(t)])
+//     (section 三, centroid subtraction), and for the last stage the per-group
+//     min/max 2-bit quantisation with E4M3 scale and zero point (section 五).
+//
+// Thread layout shared by all three: 8 threads per token, thread j owns the
+// two 8-channel chunks j and j+8 (channels 8j..8j+7 and 64+8j..64+8j+7).  The
+// 8 threads of a token therefore read and write 128 contiguous bytes per
+// instruction (coalesced), read centroid rows from shared memory without bank
+// conflicts, and a group of G channels is reduced with xor-shuffles over
+// G/8 threads.
+#include "qvg_common.cuh"
+#include "qvg_launch.h"
+
+namespace qvg {
+namespace {
+
+// ---------------------------------------------------------------- 8-value IO
+template <int DT> struct Vec8;
+
+template <> struct Vec8<kBF16> {
+  __device__ static __forceinline__ void load(const void* p, float (&v)[8]) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] = __uint_as_float(x[e] << 16);
+      v[2 * e + 1] = __uint_as_float(x[e] & 0xFFFF0000u);
+    }
+  }
+  // Round 8 fp32 values to bf16 (nearest even) and store 16 bytes.
+  __device__ static __forceinline__ void store(void* p, const float (&v)[8]) {
+    uint32_t x[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+      x[e] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(x[0], x[1], x[2], x[3]);
+  }
+  // Round to bf16 and return the rounded values as fp32.
+  __device__ static __forceinline__ void round(float (&v)[8]) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
+  }
+};
+
+template <> struct Vec8<kFP32> {
+  __device__ static __forceinline__ void load(const void* p, float (&v)[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0];
+    const float4 b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  __device__ static __forceinline__ void store(void* p, const float (&v)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+  __device__ static __forceinline__ void round(float (&)[8]) {}
+};
+
+// ---------------------------------------------------------------- dequant
+constexpr int kDqThreads = 512;
+constexpr int kDqTokPerIter = kDqThreads / 8;   // 64 tokens per block iteration
+constexpr int kDqUnroll = 4;                    // tokens per thread per iteration
+
+// TT = number of stages when it is <= 4 (all assignment loads issued up front),
+// or -1 for the generic runtime-T loop.
+template <int DT, int TT>
+__global__ void __launch_bounds__(kDqThreads)
+qvg_dequant_fused(const DequantParams p, const int splits) {
+  constexpr int ESZ = Store<DT>::bytes;
+  constexpr int TR = TT < 0 ? 1 : (TT == 0 ? 1 : TT);
+  extern __shared__ __align__(16) unsigned char smem[];
+
+  const int unit = blockIdx.x / splits;
+  const int part = blockIdx.x % splits;
+  const int h = unit % p.H;
+  const int c = unit / p.H;
+  int64_t o_c = 0, n_c = p.N;
+  if (p.chunk_off != nullptr) {
+    o_c = p.chunk_off[c];
+    n_c = p.chunk_off[c + 1] - o_c;
+  }
+  const int64_t per = (n_c + splits - 1) / splits;
+  const int64_t i_begin = (int64_t)part * per;
+  const int64_t i_end = min(n_c, i_begin + per);
+  const int K = p.K, T = TT < 0 ? p.T : TT, G = p.G;
+  const int64_t tab_elems = (int64_t)K * kD;
+  const char* tables = static_cast<const char*>(p.centroids) + (int64_t)c * T * p.H * tab_elems * ESZ;
+
+  // Stage the first t_smem tables of this (chunk, head) in shared memory.
+  for (int t = 0; t < p.t_smem; ++t) {
+    const uint4* src = reinterpret_cast<const uint4*>(tables + ((int64_t)t * p.H + h) * tab_elems * ESZ);
+    uint4* dst = reinterpret_cast<uint4*>(smem + (size_t)t * tab_elems * ESZ);
+    const int n16 = (int)(tab_elems * ESZ / 16);
+    for (int x = threadIdx.x; x < n16; x += blockDim.x) dst[x] = src[x];
+  }
+  __syncthreads();
+  if (i_begin >= i_end) return;
+
+  const int j = threadIdx.x & 7;
+  const int tl = threadIdx.x >> 3;
+  const int ng = kD / G;
+  const int g0 = (8 * j) / G, g1 = (64 + 8 * j) / G;
+  const int64_t row0 = (int64_t)p.H * o_c + (int64_t)h * n_c;
+  const uint8_t* codes = p.codes + row0 * (kD / 4);
+  const uint8_t* sc = p.scale + row0 * ng;
+  const uint8_t* zr = p.zero + row0 * ng;
+  const uint8_t* asg = p.assign + (int64_t)T * p.H * o_c + (int64_t)h * n_c;
+  const int64_t asg_t = (int64_t)p.H * n_c;
+  char* Y = static_cast<char*>(p.Y) + ((int64_t)h * p.y_head_stride + o_c) * kD * ESZ;
+
+  for (int64_t base = i_begin + tl; base < i_end; base += kDqTokPerIter * kDqUnroll) {
+    int64_t tok[kDqUnroll];
+    uint32_t q0[kDqUnroll], q1[kDqUnroll];
+    uint8_t s0b[kDqUnroll], m0b[kDqUnroll], s1b[kDqUnroll], m1b[kDqUnroll];
+    int kk[kDqUnroll][TR];
+    // issue every load of the iteration first
+#pragma unroll
+    for (int u = 0; u < kDqUnroll; ++u) {
+      tok[u] = base + u * kDqTokPerIter;
+      const int64_t i = tok[u] < i_end ? tok[u] : base;
+      q0[u] = *reinterpret_cast<const uint16_t*>(codes + i * (kD / 4) + 2 * j);
+      q1[u] = *reinterpret_cast<const uint16_t*>(codes + i * (kD / 4) + 16 + 2 * j);
+      s0b[u] = sc[i * ng + g0]; m0b[u] = zr[i * ng + g0];
+      s1b[u] = sc[i * ng + g1]; m1b[u] = zr[i * ng + g1];
+      if (TT > 0) {
+#pragma unroll
+        for (int t = 0; t < TR; ++t) kk[u][t] = asg[t * asg_t + i];
+      }
+    }
+    // then finish the tokens one at a time (16 values live per thread)
+#pragma unroll
+    for (int u = 0; u < kDqUnroll; ++u) {
+      float y0[8], y1[8];
+      const float s0 = e4m3_to_f32(s0b[u]), m0 = e4m3_to_f32(m0b[u]);
+      const float s1 = e4m3_to_f32(s1b[u]), m1 = e4m3_to_f32(m1b[u]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        // s*q + m is exact in fp32 (E4M3 operands, q <= 3)
+        y0[e] = __fmaf_rn(s0, (float)((q0[u] >> (2 * e)) & 3u), m0);
+        y1[e] = __fmaf_rn(s1, (float)((q1[u] >> (2 * e)) & 3u), m1);
+      }
+      const int64_t i = tok[u] < i_end ? tok[u] : base;
+      // centroids of stage T, T-1, ..., 1, in that order
+#pragma unroll
+      for (int tt = 0; tt < (TT < 0 ? kMaxT : (TT == 0 ? 0 : TR)); ++tt) {
+        const int t = T - 1 - tt;
+        if (TT < 0 && t < 0) break;
+        int k = TT > 0 ? kk[u][t] : (int)asg[t * asg_t + i];
+        k = k < K ? k : K - 1;
+        const char* rowp = (t < p.t_smem)
+            ? reinterpret_cast<const char*>(smem) + ((int64_t)t * tab_elems + (int64_t)k * kD) * ESZ
+            : tables + (((int64_t)t * p.H + h) * tab_elems + (int64_t)k * kD) * ESZ;
+        float c0[8], c1[8];
+        Vec8<DT>::load(rowp + 8 * j * ESZ, c0);
+        Vec8<DT>::load(rowp + (64 + 8 * j) * ESZ, c1);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          y0[e] = __fadd_rn(y0[e], c0[e]);
+          y1[e] = __fadd_rn(y1[e], c1[e]);
+        }
+      }
+      if (tok[u] < i_end) {
+        char* yr = Y + tok[u] * kD * ESZ;
+        Vec8<DT>::store(yr + 8 * j * ESZ, y0);
+        Vec8<DT>::store(yr + (64 + 8 * j) * ESZ, y1);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- residual / quant
+constexpr int kRqThreads = 512;
+constexpr int kRqTokPerIter = kRqThreads / 8;
+
+__device__ __forceinline__ float grp_min(float v, int G) {
+  if (G >= 16) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  if (G >= 32) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+  if (G >= 64) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+  return v;
+}
+__device__ __forceinline__ float grp_max(float v, int G) {
+  if (G >= 16) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  if (G >= 32) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+  if (G >= 64) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+  return v;
+}
+
+// Quantise one 8-channel chunk given its group's (lo, hi); returns the 16-bit
+// packed codes and the scale/zero bytes.
+__device__ __forceinline__ uint32_t quant_chunk(const float (&r)[8], float lo, float hi,
+                                                uint8_t& sc_out, uint8_t& zc_out) {
+  lo = __fadd_rn(lo, 0.0f);             // -0 -> +0
+  hi = __fadd_rn(hi, 0.0f);
+  const uint8_t zc = f32_to_e4m3(lo);
+  const float m = e4m3_to_f32(zc);
+  const float span = __fsub_rn(hi, m);
+  const uint8_t scb = f32_to_e4m3(__fdiv_rn(span, 3.0f));
+  const float s = e4m3_to_f32(scb);
+  uint32_t packed = 0;
+  if (s != 0.0f) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      int q = __float2int_rn(__fdiv_rn(__fsub_rn(r[e], m), s));
+      q = q < 0 ? 0 : (q > 3 ? 3 : q);
+      packed |= (uint32_t)q << (2 * e);
+    }
+  }
+  sc_out = scb;
+  zc_out = zc;
+  return packed;
+}
+
+template <int DT, bool QUANT, bool HAS_C>
+__global__ void __launch_bounds__(kRqThreads)
+qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
+  constexpr int ESZ = Store<DT>::bytes;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int u = blockIdx.y;
+  const int64_t t0 = (int64_t)blockIdx.x * per_block;
+  const int64_t t1 = min(p.N, t0 + per_block);
+  if (HAS_C) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(p.C) + (int64_t)u * p.K * kD * ESZ);
+    uint4* dst = reinterpret_cast<uint4*>(smem);
+    const int n16 = p.K * kD * ESZ / 16;
+    for (int x = threadIdx.x; x < n16; x += blockDim.x) dst[x] = src[x];
+    __syncthreads();
+  }
+  const int j = threadIdx.x & 7;
+  const int ng = kD / p.G;
+  const int G = p.G;
+  const char* Rin = static_cast<const char*>(p.R_in) + (int64_t)u * p.N * kD * ESZ;
+  // The loop bound is uniform across the warp (4 tokens per warp per
+  // iteration) so that the group shuffles below always run on all 32 lanes;
+  // lanes past the end work on a valid token and store nothing.
+  const int64_t warp_tok = (threadIdx.x >> 5) * 4;
+  for (int64_t ib = t0 + warp_tok; ib < t1; ib += kRqTokPerIter) {
+    const int64_t iv = ib + ((threadIdx.x >> 3) & 3);
+    const bool valid = iv < t1;
+    const int64_t i = valid ? iv : ib;
+    float r0[8], r1[8];
+    Vec8<DT>::load(Rin + (i * kD + 8 * j) * ESZ, r0);
+    Vec8<DT>::load(Rin + (i * kD + 64 + 8 * j) * ESZ, r1);
+    if (HAS_C) {
+      int k = p.pi[(int64_t)u * p.N + i];
+      k = k < p.K ? k : p.K - 1;
+      float c0[8], c1[8];
+      const char* crow = reinterpret_cast<const char*>(smem) + (int64_t)k * kD * ESZ;
+      Vec8<DT>::load(crow + 8 * j * ESZ, c0);
+      Vec8<DT>::load(crow + (64 + 8 * j) * ESZ, c1);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        r0[e] = __fsub_rn(r0[e], c0[e]);
+        r1[e] = __fsub_rn(r1[e], c1[e]);
+      }
+      Vec8<DT>::round(r0);
+      Vec8<DT>::round(r1);
+    }
+    if (!QUANT) {
+      if (valid && p.R_out != nullptr) {
+        char* Ro = static_cast<char*>(p.R_out) + ((int64_t)u * p.N + i) * kD * ESZ;
+        Vec8<DT>::store(Ro + 8 * j * ESZ, r0);
+        Vec8<DT>::store(Ro + (64 + 8 * j) * ESZ, r1);
+      }
+      float s2 = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        s2 = __fmaf_rn(r0[e], r0[e], s2);
+        s2 = __fmaf_rn(r1[e], r1[e], s2);
+      }
+      s2 += __shfl_xor_sync(0xffffffffu, s2, 1);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, 4);
+      if (valid && j == 0 && p.rnorm2 != nullptr) p.rnorm2[(int64_t)u * p.N + i] = s2;
+    } else {
+      float lo0 = r0[0], hi0 = r0[0], lo1 = r1[0], hi1 = r1[0];
+#pragma unroll
+      for (int e = 1; e < 8; ++e) {
+        lo0 = fminf(lo0, r0[e]); hi0 = fmaxf(hi0, r0[e]);
+        lo1 = fminf(lo1, r1[e]); hi1 = fmaxf(hi1, r1[e]);
+      }
+      if (G == 128) {
+        lo0 = lo1 = fminf(lo0, lo1);
+        hi0 = hi1 = fmaxf(hi0, hi1);
+      }
+      const int Gs = G > 64 ? 64 : G;
+      lo0 = grp_min(lo0, Gs); hi0 = grp_max(hi0, Gs);
+      lo1 = grp_min(lo1, Gs); hi1 = grp_max(hi1, Gs);
+      uint8_t s0, z0, s1, z1;
+      const uint32_t q0 = quant_chunk(r0, lo0, hi0, s0, z0);
+      const uint32_t q1 = quant_chunk(r1, lo1, hi1, s1, z1);
+      if (!valid) continue;
+      const int64_t row = (int64_t)u * p.N + i;
+      uint8_t* cr = p.codes + row * (kD / 4);
+      *reinterpret_cast<uint16_t*>(cr + 2 * j) = (uint16_t)q0;
+      *reinterpret_cast<uint16_t*>(cr + 16 + 2 * j) = (uint16_t)q1;
+      if ((8 * j) % G == 0) {
+        p.scale[row * ng + (8 * j) / G] = s0;
+        p.zero[row * ng + (8 * j) / G] = z0;
+      }
+      if (G < 128 && (64 + 8 * j) % G == 0) {
+        p.scale[row * ng + (64 + 8 * j) / G] = s1;
+        p.zero[row * ng + (64 + 8 * j) / G] = z1;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- centroid init
+template <int DT>
+__global__ void __launch_bounds__(256)
+qvg_init_centroids(const void* src, int64_t src_unit_stride, void* C, float* cn, int K) {
+  constexpr int ESZ = Store<DT>::bytes;
+  const int u = blockIdx.y;
+  const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (k >= K) return;
+  const char* s = static_cast<const char*>(src) + ((int64_t)u * src_unit_stride + (int64_t)k * kD) * ESZ;
+  char* d = static_cast<char*>(C) + ((int64_t)u * K + k) * kD * ESZ;
+  double acc = 0.0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int jj = lane * 4 + e;
+    float v;
+    if (DT == kBF16) {
+      const uint16_t b = reinterpret_cast<const uint16_t*>(s)[jj];
+      reinterpret_cast<uint16_t*>(d)[jj] = b;
+      v = bf16_bits_to_f32(b);
+    } else {
+      v = reinterpret_cast<const float*>(s)[jj];
+      reinterpret_cast<float*>(d)[jj] = v;
+    }
+    acc = __dadd_rn(acc, __dmul_rn((double)v, (double)v));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc = __dadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+  if (lane == 0) cn[(int64_t)u * K + k] = __double2float_rn(acc);
+}
+
+template <typename F>
+cudaError_t set_smem(F* f, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+}  // namespace
+
+template <int DT, int TT>
+static cudaError_t launch_dq(const DequantParams& p, int blocks, int splits, size_t smem, cudaStream_t s) {
+  cudaError_t e = set_smem(qvg_dequant_fused<DT, TT>, smem);
+  if (e != cudaSuccess) return e;
+  qvg_dequant_fused<DT, TT><<<blocks, kDqThreads, smem, s>>>(p, splits);
+  return cudaGetLastError();
+}
+
+template <int DT>
+static cudaError_t launch_dq_t(const DequantParams& p, int blocks, int splits, size_t smem, cudaStream_t s) {
+  switch (p.T) {
+    case 0: return launch_dq<DT, 0>(p, blocks, splits, smem, s);
+    case 1: return launch_dq<DT, 1>(p, blocks, splits, smem, s);
+    case 2: return launch_dq<DT, 2>(p, blocks, splits, smem, s);
+    case 3: return launch_dq<DT, 3>(p, blocks, splits, smem, s);
+    case 4: return launch_dq<DT, 4>(p, blocks, splits, smem, s);
+    default: return launch_dq<DT, -1>(p, blocks, splits, smem, s);
+  }
+}
+
+cudaError_t launch_dequant(const DequantParams& p, int dtype, cudaStream_t s) {
+  const int esz = dtype == kBF16 ? 2 : 4;
+  const size_t smem = (size_t)p.t_smem * p.K * kD * esz;
+  const int units = p.n_chunks * p.H;
+  if (units == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // split blocks along tokens until the grid covers the GPU at least twice
+  int splits = (2 * sms + units - 1) / units;
+  const int64_t ntok = p.chunk_off ? 0 : p.N;
+  if (ntok > 0) {
+    const int64_t max_splits = (ntok + 255) / 256;
+    if (splits > max_splits) splits = (int)max_splits;
+  } else if (splits > 8) {
+    splits = 8;
+  }
+  if (splits < 1) splits = 1;
+  const int blocks = units * splits;
+  return dtype == kBF16 ? launch_dq_t<kBF16>(p, blocks, splits, smem, s)
+                        : launch_dq_t<kFP32>(p, blocks, splits, smem, s);
+}
+
+template <int DT, bool Q, bool C>
+static cudaError_t launch_rq(const ResidualParams& p, dim3 grid, int64_t per, size_t smem, cudaStream_t s) {
+  cudaError_t e = set_smem(qvg_residual_quant<DT, Q, C>, smem);
+  if (e != cudaSuccess) return e;
+  qvg_residual_quant<DT, Q, C><<<grid, kRqThreads, smem, s>>>(p, per);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_residual(const ResidualParams& p, int dtype, bool quant, cudaStream_t s) {
+  const int esz = dtype == kBF16 ? 2 : 4;
+  const bool has_c = p.C != nullptr;
+  const size_t smem = has_c ? (size_t)p.K * kD * esz : 0;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // Enough blocks for two waves over the SMs; each block stages the table once.
+  int64_t splits = (2 * (int64_t)sms + p.W - 1) / p.W;
+  const int64_t min_tok = 256;
+  if (splits * min_tok > p.N) splits = (p.N + min_tok - 1) / min_tok;
+  if (splits < 1) splits = 1;
+  const int64_t per = (p.N + splits - 1) / splits;
+  const dim3 grid((unsigned)splits, (unsigned)p.W);
+  if (dtype == kBF16) {
+    if (quant) return has_c ? launch_rq<kBF16, true, true>(p, grid, per, smem, s)
+                            : launch_rq<kBF16, true, false>(p, grid, per, smem, s);
+    return has_c ? launch_rq<kBF16, false, true>(p, grid, per, smem, s)
+                 : launch_rq<kBF16, false, false>(p, grid, per, smem, s);
+  }
+  if (quant) return has_c ? launch_rq<kFP32, true, true>(p, grid, per, smem, s)
+                          : launch_rq<kFP32, true, false>(p, grid, per, smem, s);
+  return has_c ? launch_rq<kFP32, false, true>(p, grid, per, smem, s)
+               : launch_rq<kFP32, false, false>(p, grid, per, smem, s);
+}
+
+cudaError_t launch_init_centroids(const void* src, int64_t src_unit_stride, void* C,
+                                  float* cn, int W, int K, int dtype, cudaStream_t s) {
+  const dim3 grid((unsigned)((K + 7) / 8), (unsigned)W);
+  if (dtype == kBF16) qvg_init_centroids<kBF16><<<grid, 256, 0, s>>>(src, src_unit_stride, C, cn, K);
+  else qvg_init_centroids<kFP32><<<grid, 256, 0, s>>>(src, src_unit_stride, C, cn, K);
+  return cudaGetLastError();
+}
+
+}  // namespace qvg

@@ -1,0 +1,544 @@
+// qvg_api.cu -- host side of libqvg.so: argument checks, workspace planning,
+// the progressive-residual stage loop, and the streaming cache.  Every
+// arithmetic step of the codec runs in the kernels; this file only
+// schedules them (m.163.com article on Quant VideoGen, sections 三-五;
+// gist.science/de, Technische Zusammenfassung 2A-2C).
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <mutex>
+#include <string>
+#include <vector>
+#include <cstdlib>
+#include <cstring>
+#include <cstdint>
+
+#include "qvg.h"
+#include "qvg_launch.h"
+
+using namespace qvg;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+int esize(int dtype) { return dtype == kFP32 ? 4 : 2; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Layout of the caller's workspace for a batch of W units.
+struct Plan {
+  int W = 0;
+  int nseg = 0;
+  int nR = 0;
+  size_t off_R[2] = {0, 0};
+  size_t off_rnorm = 0, off_cn = 0, off_list = 0, off_listcnt = 0;
+  size_t off_partial = 0, off_counts = 0, off_status = 0, total = 0;
+};
+
+Plan make_plan(const qvg_config& c, int64_t N, int W, int dtype) {
+  Plan p;
+  p.W = W;
+  p.nseg = (int)((N + kSeg - 1) / kSeg);
+  p.nR = c.T >= 3 ? 2 : (c.T == 2 ? 1 : 0);
+  const size_t esz = (size_t)esize(dtype);
+  size_t o = 0;
+  p.off_status = o;                       o = align_up(o + 16);
+  for (int b = 0; b < p.nR; ++b) { p.off_R[b] = o; o = align_up(o + (size_t)W * N * kD * esz); }
+  p.off_rnorm = o;                        o = align_up(o + (size_t)W * N * sizeof(float));
+  p.off_cn = o;                           o = align_up(o + (size_t)W * kMaxK * sizeof(float));
+  p.off_list = o;                         o = align_up(o + (size_t)W * N * sizeof(uint32_t));
+  p.off_listcnt = o;                      o = align_up(o + (size_t)W * sizeof(uint32_t));
+  p.off_partial = o;                      o = align_up(o + (size_t)W * p.nseg * c.K * kD * sizeof(double));
+  p.off_counts = o;                       o = align_up(o + (size_t)W * p.nseg * c.K * sizeof(int));
+  p.total = o;
+  return p;
+}
+
+int preferred_batch(int64_t N, int H, int dtype) {
+  if (const char* env = std::getenv("QVG_BATCH_UNITS")) {
+    const int w = std::atoi(env);
+    if (w > 0) return std::min(w, H);
+  }
+  // Keep the stage inputs of one batch within about 48 MB so that the
+  // repeated passes of the Lloyd iterations are served from L2.
+  const double budget = 48.0 * 1024.0 * 1024.0;
+  int w = (int)std::floor(budget / ((double)N * kD * esize(dtype)));
+  return std::max(1, std::min(w, H));
+}
+
+// Relative error bound assumed for the tensor-core dot products of 128
+// bf16 x bf16 products accumulated in fp32 (2^-14, 128x the unit roundoff).
+constexpr float kTcGamma = 6.103515625e-05f;
+
+// QVG_ASSIGN_PATH=exact routes bf16 blocks through the CUDA-core exact
+// assignment as well (diagnostics; the results are identical).
+bool assign_path_tc() {
+  const char* e = std::getenv("QVG_ASSIGN_PATH");
+  return !(e != nullptr && std::strcmp(e, "exact") == 0);
+}
+
+bool g_supported(int G) { return G == 8 || G == 16 || G == 32 || G == 64 || G == 128; }
+
+qvg_status check_config(const qvg_config* c, int64_t N, int32_t H, int32_t d, qvg_dtype dtype) {
+  if (c == nullptr) return QVG_ERR_INVALID_ARG;
+  if (dtype != QVG_BF16 && dtype != QVG_FP32) return QVG_ERR_INVALID_ARG;
+  if (c->bits != 2 || c->K < 1 || c->K > 256 || c->T < 0) return QVG_ERR_INVALID_ARG;
+  if (c->group_size < 4 || c->group_size % 4 != 0 || d < 4 || d % c->group_size != 0)
+    return QVG_ERR_INVALID_ARG;
+  if (N < 0 || H < 1) return QVG_ERR_INVALID_ARG;
+  if (d != kD || !g_supported(c->group_size) || c->T > kMaxT) return QVG_ERR_UNSUPPORTED;
+  return QVG_OK;
+}
+
+qvg_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QVG_OK : QVG_ERR_CUDA; }
+
+
+// ---------------------------------------------------------------- diagnostics
+// Launch counts per kernel (always kept) and, when enabled, device time per
+// kernel from CUDA events recorded on the launching stream around each launch.
+enum Kind {
+  K_DEQUANT, K_RESIDUAL, K_RESIDUAL_QUANT, K_ROWNORM, K_INIT, K_ASSIGN_EXACT, K_ASSIGN_TC,
+  K_RECHECK, K_UPD_PARTIAL, K_UPD_FINAL, K_NKINDS
+};
+const char* const kKindNames[K_NKINDS] = {
+  "qvg_dequant_fused", "qvg_residual", "qvg_residual_quant", "qvg_row_norms", "qvg_init_centroids",
+  "qvg_assign_exact", "qvg_kmeans_assign", "qvg_assign_recheck", "qvg_update_partial",
+  "qvg_update_finalize"};
+
+struct Profiler {
+  std::mutex mu;
+  std::atomic<bool> timing{false};
+  std::atomic<long long> launches[K_NKINDS];
+  std::vector<int> kinds;
+  std::vector<cudaEvent_t> ev;     // pairs
+  std::vector<cudaEvent_t> pool;
+  double ms[K_NKINDS] = {};
+  long long timed[K_NKINDS] = {};
+  Profiler() { for (auto& l : launches) l = 0; }
+};
+Profiler& prof() {
+  static Profiler p;
+  return p;
+}
+
+cudaEvent_t pool_event(Profiler& p) {
+  if (!p.pool.empty()) { cudaEvent_t e = p.pool.back(); p.pool.pop_back(); return e; }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+template <class F>
+cudaError_t plaunch(Kind k, cudaStream_t s, F&& f) {
+  Profiler& p = prof();
+  p.launches[k]++;
+  if (!p.timing.load(std::memory_order_relaxed)) return f();
+  cudaEvent_t a, b;
+  {
+    std::lock_guard<std::mutex> g(p.mu);
+    a = pool_event(p);
+    b = pool_event(p);
+  }
+  cudaEventRecord(a, s);
+  const cudaError_t e = f();
+  cudaEventRecord(b, s);
+  std::lock_guard<std::mutex> g(p.mu);
+  p.kinds.push_back((int)k);
+  p.ev.push_back(a);
+  p.ev.push_back(b);
+  return e;
+}
+
+#define QVG_TRY(expr)                                    \
+  do {                                                   \
+    cudaError_t qvg_e_ = (expr);                         \
+    if (qvg_e_ != cudaSuccess) return QVG_ERR_CUDA;      \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* qvg_status_string(qvg_status s) {
+  switch (s) {
+    case QVG_OK: return "ok";
+    case QVG_ERR_INVALID_ARG: return "invalid argument";
+    case QVG_ERR_UNSUPPORTED: return "unsupported configuration";
+    case QVG_ERR_NO_MEMORY: return "out of device memory";
+    case QVG_ERR_CUDA: return "CUDA error";
+    case QVG_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case QVG_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case QVG_ERR_CAPACITY: return "cache capacity exceeded";
+  }
+  return "unknown status";
+}
+
+const char* qvg_version(void) { return "qvg-b200 sm_100a"; }
+
+size_t qvg_packed_bytes(const qvg_config* c, int64_t N, int32_t H, int32_t d, qvg_dtype dtype) {
+  if (c == nullptr || c->bits != 2 || c->K < 1 || c->K > 256 || c->T < 0 || c->group_size < 4 ||
+      c->group_size % 4 != 0 || d < 4 || d % c->group_size != 0 || N < 0 || H < 1 ||
+      (dtype != QVG_BF16 && dtype != QVG_FP32))
+    return 0;
+  const size_t esz = (size_t)esize(dtype);
+  const size_t codes = (size_t)H * N * d * c->bits / 8;
+  const size_t scales = 2 * (size_t)H * N * (d / c->group_size);
+  const size_t assign = (size_t)c->T * H * N;
+  const size_t cents = (size_t)c->T * H * c->K * d * esz;
+  return codes + scales + assign + cents;
+}
+
+size_t qvg_workspace_bytes(const qvg_config* c, int64_t N, int32_t H, int32_t d, qvg_dtype dtype) {
+  if (check_config(c, N, H, d, dtype) != QVG_OK || N < 1) return 0;
+  return make_plan(*c, N, preferred_batch(N, H, dtype), dtype).total;
+}
+
+qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, int64_t N,
+                        int32_t H, int32_t d, const void* init, const qvg_packed* out,
+                        void* workspace, size_t ws_bytes, qvg_stream_t stream_) {
+  qvg_status st = check_config(cfg, N, H, d, dtype);
+  if (st != QVG_OK) return st;
+  const qvg_config c = *cfg;
+  const bool warm = init != nullptr;
+  const int iters = warm ? c.warm_iters : c.iters;
+  if (N < 1 || X == nullptr || out == nullptr || workspace == nullptr) return QVG_ERR_INVALID_ARG;
+  if (out->codes == nullptr || out->scale == nullptr || out->zero == nullptr) return QVG_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(init, 16) || !aligned(out->centroids, 16) || !aligned(out->codes, 2) ||
+      !aligned(workspace, kAlign))
+    return QVG_ERR_INVALID_ARG;
+  if (c.T > 0) {
+    if (out->assign == nullptr || out->centroids == nullptr || iters < 1) return QVG_ERR_INVALID_ARG;
+    if (!warm && N < c.K) return QVG_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  const int dt = (int)dtype;
+  const size_t esz = (size_t)esize(dt);
+
+  int W = preferred_batch(N, H, dt);
+  Plan plan = make_plan(c, N, W, dt);
+  while (plan.total > ws_bytes && W > 1) plan = make_plan(c, N, --W, dt);
+  if (plan.total > ws_bytes) return QVG_ERR_WORKSPACE_TOO_SMALL;
+
+  char* ws = static_cast<char*>(workspace);
+  float* rnorm = reinterpret_cast<float*>(ws + plan.off_rnorm);
+  float* cn = reinterpret_cast<float*>(ws + plan.off_cn);
+  uint32_t* list = reinterpret_cast<uint32_t*>(ws + plan.off_list);
+  uint32_t* list_count = reinterpret_cast<uint32_t*>(ws + plan.off_listcnt);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + plan.off_status);
+  unsigned long long* flagged = reinterpret_cast<unsigned long long*>(ws + plan.off_status + 8);
+  // bf16 blocks take the tensor-core assignment; fp32 blocks the exact CUDA-core one
+  const bool use_tc = dt == kBF16 && assign_path_tc();
+  const int ng = kD / c.group_size;
+
+  for (int u0 = 0; u0 < H; u0 += W) {
+    const int w = std::min(W, H - u0);
+    const char* Xu = static_cast<const char*>(X) + (size_t)u0 * N * kD * esz;
+    ResidualParams rq{};
+    rq.N = N; rq.W = w; rq.K = c.K; rq.G = c.group_size;
+    rq.codes = out->codes + (size_t)u0 * N * (kD / 4);
+    rq.scale = out->scale + (size_t)u0 * N * ng;
+    rq.zero = out->zero + (size_t)u0 * N * ng;
+    if (c.T == 0) {
+      rq.R_in = Xu;
+      QVG_TRY(plaunch(K_RESIDUAL_QUANT, s, [&] { return launch_residual(rq, dt, true, s); }));
+      continue;
+    }
+    const void* Rin = Xu;
+    for (int t = 0; t < c.T; ++t) {
+      char* Ct = static_cast<char*>(out->centroids) + ((size_t)t * H + u0) * c.K * kD * esz;
+      uint8_t* pit = out->assign + ((size_t)t * H + u0) * N;
+      if (t == 0) {   // squared row norms of X for the assignment error bound
+        ResidualParams nq = rq;
+        nq.R_in = Xu; nq.C = nullptr; nq.R_out = nullptr; nq.rnorm2 = rnorm;
+        QVG_TRY(plaunch(K_ROWNORM, s, [&] { return launch_residual(nq, dt, false, s); }));
+      }
+      if (warm) {
+        const char* src = static_cast<const char*>(init) + ((size_t)t * H + u0) * c.K * kD * esz;
+        QVG_TRY(plaunch(K_INIT, s, [&] { return launch_init_centroids(src, (int64_t)c.K * kD, Ct, cn, w, c.K, dt, s); }));
+      } else {
+        QVG_TRY(plaunch(K_INIT, s, [&] { return launch_init_centroids(Rin, N * kD, Ct, cn, w, c.K, dt, s); }));
+      }
+      for (int it = 0; it < iters; ++it) {
+        AssignParams ap{};
+        ap.R = Rin; ap.rnorm2 = rnorm; ap.C = Ct; ap.cn = cn; ap.pi = pit;
+        ap.list = nullptr; ap.list_count = nullptr; ap.N = N; ap.W = w; ap.K = c.K;
+        if (use_tc) {
+          // tensor-core screening; listed near-ties are decided exactly next
+          QVG_TRY(cudaMemsetAsync(list_count, 0, (size_t)w * sizeof(uint32_t), s));
+          AssignTcParams tp{};
+          tp.R = Rin; tp.rnorm2 = rnorm; tp.C = Ct; tp.cn = cn; tp.pi = pit; tp.list = list;
+          tp.list_count = list_count; tp.status = status; tp.flagged = flagged;
+          tp.N = N; tp.W = w; tp.K = c.K; tp.gamma = kTcGamma;
+          QVG_TRY(plaunch(K_ASSIGN_TC, s, [&] { return launch_assign_tc(tp, s); }));
+          ap.list = list; ap.list_count = list_count;
+          QVG_TRY(plaunch(K_RECHECK, s, [&] { return launch_assign_exact(ap, dt, s); }));
+        } else {
+          QVG_TRY(plaunch(K_ASSIGN_EXACT, s, [&] { return launch_assign_exact(ap, dt, s); }));
+        }
+        UpdateParams up{};
+        up.R = Rin; up.pi = pit; up.C = Ct; up.cn = cn; up.N = N; up.W = w; up.K = c.K;
+        up.nseg = plan.nseg;
+        up.partial = reinterpret_cast<double*>(ws + plan.off_partial);
+        up.counts = reinterpret_cast<int*>(ws + plan.off_counts);
+        QVG_TRY(plaunch(K_UPD_PARTIAL, s, [&] { return launch_update_partial(up, dt, s); }));
+        QVG_TRY(plaunch(K_UPD_FINAL, s, [&] { return launch_update_finalize(up, dt, s); }));
+      }
+      ResidualParams rp = rq;
+      rp.R_in = Rin; rp.C = Ct; rp.pi = pit;
+      if (t + 1 < c.T) {
+        void* Rout = ws + plan.off_R[t % 2];
+        rp.R_out = Rout; rp.rnorm2 = rnorm;
+        QVG_TRY(plaunch(K_RESIDUAL, s, [&] { return launch_residual(rp, dt, false, s); }));
+        Rin = Rout;
+      } else {
+        QVG_TRY(plaunch(K_RESIDUAL_QUANT, s, [&] { return launch_residual(rp, dt, true, s); }));
+      }
+    }
+  }
+  return QVG_OK;
+}
+
+qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packed, qvg_dtype dtype,
+                          int64_t N, int32_t H, int32_t d, void* Y, qvg_stream_t stream_) {
+  qvg_status st = check_config(cfg, N, H, d, dtype);
+  if (st != QVG_OK) return st;
+  if (packed == nullptr || Y == nullptr || packed->codes == nullptr || packed->scale == nullptr ||
+      packed->zero == nullptr)
+    return QVG_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (packed->assign == nullptr || packed->centroids == nullptr)) return QVG_ERR_INVALID_ARG;
+  if (!aligned(Y, 16) || !aligned(packed->centroids, 16) || !aligned(packed->codes, 2)) return QVG_ERR_INVALID_ARG;
+  if (N == 0) return QVG_OK;
+  const int dt = (int)dtype;
+  const size_t table = (size_t)cfg->K * kD * esize(dt);
+  DequantParams p{};
+  p.codes = packed->codes; p.scale = packed->scale; p.zero = packed->zero;
+  p.assign = packed->assign; p.centroids = packed->centroids; p.Y = Y;
+  p.chunk_off = nullptr; p.N = N; p.y_head_stride = N; p.n_chunks = 1; p.H = H;
+  p.K = cfg->K; p.T = cfg->T; p.G = cfg->group_size;
+  p.t_smem = std::min<int>(cfg->T, (int)((160 * 1024) / table));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  return cuda_status(plaunch(K_DEQUANT, s, [&] { return launch_dequant(p, dt, s); }));
+}
+
+int64_t qvg_workspace_flagged(void* workspace, size_t ws_bytes, qvg_stream_t stream_) {
+  if (workspace == nullptr || ws_bytes < 16) return -1;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  unsigned long long n = 0;
+  if (cudaMemcpyAsync(&n, static_cast<char*>(workspace) + 8, sizeof(n), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess || cudaMemsetAsync(static_cast<char*>(workspace) + 8, 0, 8, s) != cudaSuccess)
+    return -1;
+  return (int64_t)n;
+}
+
+qvg_status qvg_workspace_status(void* workspace, size_t ws_bytes, qvg_stream_t stream_) {
+  if (workspace == nullptr || ws_bytes < 16) return QVG_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  uint32_t word = 0;
+  QVG_TRY(cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s));
+  QVG_TRY(cudaStreamSynchronize(s));
+  QVG_TRY(cudaMemsetAsync(workspace, 0, 4, s));
+  return word == 0 ? QVG_OK : QVG_ERR_DEVICE_TIMEOUT;
+}
+
+
+void qvg_profile_enable(int enable) { prof().timing = enable != 0; }
+
+void qvg_profile_reset(void) {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  for (auto& l : p.launches) l = 0;
+  for (int k = 0; k < K_NKINDS; ++k) { p.ms[k] = 0.0; p.timed[k] = 0; }
+  for (cudaEvent_t e : p.ev) p.pool.push_back(e);
+  p.ev.clear();
+  p.kinds.clear();
+}
+
+int64_t qvg_profile_launches(void) {
+  Profiler& p = prof();
+  long long n = 0;
+  for (auto& l : p.launches) n += l.load();
+  return n;
+}
+
+int qvg_profile_report(char* buf, size_t buf_bytes) {
+  Profiler& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  if (!p.ev.empty()) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    for (size_t i = 0; i < p.kinds.size(); ++i) {
+      float t = 0.0f;
+      if (cudaEventElapsedTime(&t, p.ev[2 * i], p.ev[2 * i + 1]) == cudaSuccess) {
+        p.ms[p.kinds[i]] += t;
+        p.timed[p.kinds[i]] += 1;
+      }
+    }
+    for (cudaEvent_t e : p.ev) p.pool.push_back(e);
+    p.ev.clear();
+    p.kinds.clear();
+  }
+  std::string out = "{";
+  bool first = true;
+  for (int k = 0; k < K_NKINDS; ++k) {
+    const long long n = p.launches[k].load();
+    if (n == 0 && p.timed[k] == 0) continue;
+    char item[256];
+    std::snprintf(item, sizeof(item), "%s\"%s\": {\"launches\": %lld, \"timed\": %lld, \"ms\": %.6f}",
+                  first ? "" : ", ", kKindNames[k], n, p.timed[k], p.ms[k]);
+    out += item;
+    first = false;
+  }
+  out += "}";
+  if (buf == nullptr || buf_bytes < out.size() + 1) return (int)out.size() + 1;
+  std::memcpy(buf, out.c_str(), out.size() + 1);
+  return 0;
+}
+
+// ---------------------------------------------------------------- cache
+struct qvg_cache {
+  qvg_config cfg{};
+  int dtype = 0, H = 0;
+  int64_t max_tokens = 0;
+  int max_chunks = 0;
+  uint8_t* codes = nullptr;
+  uint8_t* scale = nullptr;
+  uint8_t* zero = nullptr;
+  uint8_t* assign = nullptr;
+  char* tables = nullptr;
+  int64_t* d_off = nullptr;     // device copy of the chunk offsets
+  int64_t* h_off = nullptr;     // pinned host offsets [max_chunks + 1]
+  int n_chunks = 0;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  size_t bytes = 0;
+};
+
+static void cache_free(qvg_cache* c) {
+  if (c == nullptr) return;
+  cudaFree(c->codes); cudaFree(c->scale); cudaFree(c->zero); cudaFree(c->assign);
+  cudaFree(c->tables); cudaFree(c->d_off); cudaFree(c->ws);
+  cudaFreeHost(c->h_off);
+  delete c;
+}
+
+qvg_status qvg_cache_create(const qvg_config* cfg, qvg_dtype dtype, int32_t H, int32_t d,
+                            int64_t max_tokens, int32_t max_chunks, qvg_cache** out) {
+  if (out == nullptr) return QVG_ERR_INVALID_ARG;
+  *out = nullptr;
+  qvg_status st = check_config(cfg, max_tokens, H, d, dtype);
+  if (st != QVG_OK) return st;
+  if (max_tokens < 1 || max_chunks < 1) return QVG_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (cfg->iters < 1 || cfg->warm_iters < 1)) return QVG_ERR_INVALID_ARG;
+  qvg_cache* c = new qvg_cache();
+  c->cfg = *cfg; c->dtype = (int)dtype; c->H = H; c->max_tokens = max_tokens; c->max_chunks = max_chunks;
+  const size_t esz = (size_t)esize(c->dtype);
+  const int ng = kD / cfg->group_size;
+  const size_t n_codes = (size_t)H * max_tokens * (kD / 4);
+  const size_t n_sc = (size_t)H * max_tokens * ng;
+  const size_t n_as = std::max<size_t>(1, (size_t)cfg->T * H * max_tokens);
+  const size_t n_tab = std::max<size_t>(16, (size_t)max_chunks * cfg->T * H * cfg->K * kD * esz);
+  bool ok = cudaMalloc(&c->codes, n_codes) == cudaSuccess && cudaMalloc(&c->scale, n_sc) == cudaSuccess &&
+            cudaMalloc(&c->zero, n_sc) == cudaSuccess && cudaMalloc(&c->assign, n_as) == cudaSuccess &&
+            cudaMalloc(&c->tables, n_tab) == cudaSuccess &&
+            cudaMalloc(&c->d_off, sizeof(int64_t) * ((size_t)max_chunks + 1)) == cudaSuccess &&
+            cudaMemset(c->d_off, 0, sizeof(int64_t) * ((size_t)max_chunks + 1)) == cudaSuccess &&
+            cudaMallocHost(&c->h_off, sizeof(int64_t) * ((size_t)max_chunks + 1)) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    cache_free(c);
+    return QVG_ERR_NO_MEMORY;
+  }
+  c->bytes = n_codes + 2 * n_sc + n_as + n_tab + sizeof(int64_t) * ((size_t)max_chunks + 1);
+  c->h_off[0] = 0;
+  c->n_chunks = 0;
+  *out = c;
+  return QVG_OK;
+}
+
+static void chunk_view(const qvg_cache* c, int chunk, qvg_packed* v) {
+  const int64_t o = c->h_off[chunk];
+  const size_t esz = (size_t)esize(c->dtype);
+  const int ng = kD / c->cfg.group_size;
+  v->codes = c->codes + (size_t)c->H * o * (kD / 4);
+  v->scale = c->scale + (size_t)c->H * o * ng;
+  v->zero = c->zero + (size_t)c->H * o * ng;
+  v->assign = c->assign + (size_t)c->cfg.T * c->H * o;
+  v->centroids = c->tables + (size_t)chunk * c->cfg.T * c->H * c->cfg.K * kD * esz;
+}
+
+qvg_status qvg_append_chunk(qvg_cache* c, const void* X, int64_t n, qvg_stream_t stream_) {
+  if (c == nullptr || X == nullptr || n < 1) return QVG_ERR_INVALID_ARG;
+  const int chunk = c->n_chunks;
+  if (chunk >= c->max_chunks || c->h_off[chunk] + n > c->max_tokens) return QVG_ERR_CAPACITY;
+  if (chunk == 0 && c->cfg.T > 0 && n < c->cfg.K) return QVG_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  const size_t need = qvg_workspace_bytes(&c->cfg, n, c->H, kD, (qvg_dtype)c->dtype);
+  if (need > c->ws_bytes) {
+    if (c->ws) {
+      QVG_TRY(cudaStreamSynchronize(s));
+      cudaFree(c->ws);
+      c->ws = nullptr;
+      c->ws_bytes = 0;
+    }
+    if (cudaMalloc(&c->ws, need) != cudaSuccess) { cudaGetLastError(); return QVG_ERR_NO_MEMORY; }
+    QVG_TRY(cudaMemsetAsync(c->ws, 0, 16, s));
+    c->ws_bytes = need;
+  }
+  qvg_packed v;
+  chunk_view(c, chunk, &v);
+  const void* init = nullptr;
+  if (chunk > 0) {
+    qvg_packed prev;
+    chunk_view(c, chunk - 1, &prev);
+    init = prev.centroids;
+  }
+  qvg_status st = qvg_quantize(&c->cfg, X, (qvg_dtype)c->dtype, n, c->H, kD, init, &v, c->ws,
+                               c->ws_bytes, stream_);
+  if (st != QVG_OK) return st;
+  c->h_off[chunk + 1] = c->h_off[chunk] + n;
+  // The new end offset travels to the device in stream order (pinned source,
+  // written once and never changed afterwards).
+  QVG_TRY(cudaMemcpyAsync(c->d_off + chunk + 1, &c->h_off[chunk + 1], sizeof(int64_t),
+                          cudaMemcpyHostToDevice, s));
+  c->n_chunks = chunk + 1;
+  return QVG_OK;
+}
+
+qvg_status qvg_cache_dequantize(const qvg_cache* c, void* Y, qvg_stream_t stream_) {
+  if (c == nullptr || Y == nullptr) return QVG_ERR_INVALID_ARG;
+  const int n_chunks = c->n_chunks;
+  if (n_chunks == 0) return QVG_OK;
+  const size_t table = (size_t)c->cfg.K * kD * esize(c->dtype);
+  DequantParams p{};
+  p.codes = c->codes; p.scale = c->scale; p.zero = c->zero; p.assign = c->assign;
+  p.centroids = c->tables; p.Y = Y; p.chunk_off = c->d_off; p.N = 0;
+  p.y_head_stride = c->h_off[n_chunks]; p.n_chunks = n_chunks; p.H = c->H;
+  p.K = c->cfg.K; p.T = c->cfg.T; p.G = c->cfg.group_size;
+  p.t_smem = std::min<int>(c->cfg.T, (int)((160 * 1024) / table));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  return cuda_status(plaunch(K_DEQUANT, s, [&] { return launch_dequant(p, c->dtype, s); }));
+}
+
+int64_t qvg_cache_tokens(const qvg_cache* c) { return c ? c->h_off[c->n_chunks] : 0; }
+int32_t qvg_cache_chunks(const qvg_cache* c) { return c ? c->n_chunks : 0; }
+
+qvg_status qvg_cache_chunk_view(const qvg_cache* c, int32_t chunk, qvg_packed* view,
+                                int64_t* first_token, int64_t* n_tokens) {
+  if (c == nullptr || view == nullptr || chunk < 0 || chunk >= c->n_chunks)
+    return QVG_ERR_INVALID_ARG;
+  chunk_view(c, chunk, view);
+  if (first_token) *first_token = c->h_off[chunk];
+  if (n_tokens) *n_tokens = c->h_off[chunk + 1] - c->h_off[chunk];
+  return QVG_OK;
+}
+
+size_t qvg_cache_device_bytes(const qvg_cache* c) { return c ? c->bytes + c->ws_bytes : 0; }
+
+void qvg_cache_destroy(qvg_cache* c) {
+  if (c == nullptr) return;
+  cudaDeviceSynchronize();
+  cache_free(c);
+}
+
+}  // extern "C"

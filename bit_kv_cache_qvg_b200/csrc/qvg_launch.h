@@ -1,0 +1,102 @@
+// qvg_launch.h -- host-side launchers of the sm_100a kernels (internal to
+// libqvg.so; the public surface is include/qvg.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qvg_common.cuh"
+
+namespace qvg {
+
+// ---- codec kernels (kernels_codec.cu)
+
+// Fused reconstruction of a set of (chunk, head) blocks.
+cudaError_t launch_dequant(const DequantParams& p, int dtype, cudaStream_t s);
+
+// Residual pass over W units of N tokens:
+//   r = round_S(R_in - C[pi])   (or r = R_in when C == nullptr)
+// then either
+//   quant == false: R_out = r (if R_out != nullptr) and rnorm2 = |r|^2 (fp32)
+//   quant == true : 2-bit group quantisation of r into codes/scale/zero.
+struct ResidualParams {
+  const void* R_in;        // [W][N][d] storage dtype
+  const void* C;           // [W][K][d] or nullptr
+  const uint8_t* pi;       // [W][N]
+  void* R_out;             // [W][N][d] or nullptr
+  float* rnorm2;           // [W][N] or nullptr
+  uint8_t* codes;          // [W][N][d/4]
+  uint8_t* scale;          // [W][N][d/G]
+  uint8_t* zero;           // [W][N][d/G]
+  int64_t N;
+  int W;
+  int K;
+  int G;
+};
+cudaError_t launch_residual(const ResidualParams& p, int dtype, bool quant, cudaStream_t s);
+
+// C[u] = rows of src[u] (first K rows of a stage input, or given tables);
+// cn[u][k] = |c_k|^2 rounded to fp32 from an fp64 sum.
+cudaError_t launch_init_centroids(const void* src, int64_t src_unit_stride, void* C,
+                                  float* cn, int W, int K, int dtype, cudaStream_t s);
+
+// ---- k-means kernels (kernels_kmeans.cu)
+
+struct AssignParams {
+  const void* R;               // [W][N][d]
+  const float* rnorm2;         // [W][N]
+  const void* C;               // [W][K][d]
+  const float* cn;             // [W][K]
+  uint8_t* pi;                 // [W][N]
+  const uint32_t* list;        // [W][N] rows to (re)assign, or nullptr = every row
+  const uint32_t* list_count;  // [W]
+  int64_t N;
+  int W;
+  int K;
+};
+// Exact assignment: fp32 screening distances, exact fp64 distances for every
+// centroid within the screening error bound, lowest index on exact ties.
+cudaError_t launch_assign_exact(const AssignParams& p, int dtype, cudaStream_t s);
+
+// Tensor-core assignment (kernel_assign_tc.cu): tcgen05 screening GEMM with a
+// top-2 epilogue; tokens whose runner-up is within the error bound are listed
+// for the exact pass (launch_assign_exact in list mode).  bf16 only.
+struct AssignTcParams {
+  const void* R;               // [W][N][d] bf16
+  const float* rnorm2;         // [W][N]
+  const void* C;               // [W][K][d] bf16
+  const float* cn;             // [W][K]
+  uint8_t* pi;                 // [W][N]
+  uint32_t* list;              // [W][N]
+  uint32_t* list_count;        // [W], zero on entry
+  uint32_t* status;            // workspace status word
+  unsigned long long* flagged; // running total of listed tokens
+  int64_t N;
+  int W;
+  int K;
+  float gamma;
+};
+cudaError_t launch_assign_tc(const AssignTcParams& p, cudaStream_t s);
+size_t assign_tc_smem_bytes(int K);
+
+constexpr int kSeg = 2048;   // tokens per update segment
+
+struct UpdateParams {
+  const void* R;        // [W][N][d]
+  const uint8_t* pi;    // [W][N]
+  double* partial;      // [W][nseg][K][d]
+  int* counts;          // [W][nseg][K]
+  void* C;              // [W][K][d]  (updated in place)
+  float* cn;            // [W][K]
+  int64_t N;
+  int W;
+  int K;
+  int nseg;
+};
+// Per-segment fp64 cluster sums (tokens ascending) ...
+cudaError_t launch_update_partial(const UpdateParams& p, int dtype, cudaStream_t s);
+// ... then a fixed-order reduction over segments, mean, one rounding to the
+// storage dtype.
+cudaError_t launch_update_finalize(const UpdateParams& p, int dtype, cudaStream_t s);
+
+}  // namespace qvg

@@ -1,0 +1,225 @@
+/*
+ * qvg.h -- C ABI of the B200 (sm_100a) implementation of the Quant VideoGen
+ * (QVG) 2-bit KV-cache codec.
+ *
+ * The method (arXiv:2602.02958, as described by the m.163.com article on
+ * Quant VideoGen, sections 三-五, and by gist.science/de, "Technische
+ * Zusammenfassung" 2A-2C):
+ *   1. semantic-aware smoothing: k-means over the tokens of a block, each
+ *      token minus its centroid leaves a small, even residual (section 三);
+ *   2. progressive residual quantisation: T such stages, R(0) = X, stage t
+ *      gives centroids C(t), uint8 assignments pi(t) and R(t) (section 四);
+ *   3. the final residual R(T) is quantised per group of G channels to 2-bit
+ *      codes with FP8 E4M3 group scales (section 五);
+ *   4. reconstruction runs in reverse: dequantise R(T), then add back the
+ *      centroids of stage T, T-1, ..., 1, in one fused kernel (sections 四,
+ *      五; "Fused Kernel" in Technische Zusammenfassung 2C);
+ *   5. in streaming generation each chunk's k-means starts from the previous
+ *      chunk's centroids (streaming centroid cache, section 五).
+ *
+ * Conventions for every call below:
+ *   - "device" pointers are CUDA global-memory pointers on the current
+ *     device; the caller owns them and keeps them alive until the work queued
+ *     on `stream` has finished.  Only a qvg_cache owns memory.
+ *   - Work is queued asynchronously on `stream` (0 = legacy default stream);
+ *     a call returns once the work is queued.  Errors found while queueing
+ *     (bad arguments, launch failures) are returned; a device-side timeout of
+ *     a bounded wait is reported by the next call on the same workspace or
+ *     cache as QVG_ERR_DEVICE_TIMEOUT (see qvg_workspace_status).
+ *   - Nothing is thrown across the ABI; all entry points are thread-compatible
+ *     (distinct workspaces/caches may be used from distinct threads).
+ *   - Tensor layouts are row-major.  H is the number of independent blocks
+ *     in one call (heads, or heads x layers x K/V), N the tokens per block,
+ *     d the channels per token (head dimension).
+ *   - Supported by the kernels: d = 128; G in {8, 16, 32, 64, 128};
+ *     bits = 2; 1 <= K <= 256; 0 <= T <= 8.  Other values that the method
+ *     allows return QVG_ERR_UNSUPPORTED.
+ */
+#ifndef QVG_H_
+#define QVG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QVG_API __attribute__((visibility("default")))
+#else
+#define QVG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle (cudaStream_t). */
+typedef struct CUstream_st* qvg_stream_t;
+
+typedef enum {
+    QVG_OK = 0,
+    QVG_ERR_INVALID_ARG = 1,         /* argument outside the method's domain */
+    QVG_ERR_UNSUPPORTED = 2,         /* allowed by the method, not by these kernels */
+    QVG_ERR_NO_MEMORY = 3,           /* a qvg_cache allocation failed */
+    QVG_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed */
+    QVG_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device-side wait gave up */
+    QVG_ERR_WORKSPACE_TOO_SMALL = 6, /* ws_bytes below qvg_workspace_bytes(...) for one block */
+    QVG_ERR_CAPACITY = 7             /* a qvg_cache is full (tokens or chunks) */
+} qvg_status;
+
+/* Storage dtype of X, of the centroid tables and of the reconstruction. */
+typedef enum { QVG_BF16 = 0, QVG_FP32 = 1 } qvg_dtype;
+
+typedef struct {
+    int32_t K;          /* centroids per block and stage (section 七 uses 256, stored as uint8) */
+    int32_t T;          /* progressive residual stages (section 四); 0 = plain per-group RTN */
+    int32_t group_size; /* G: contiguous channels of one token that share a scale */
+    int32_t bits;       /* code width; 2 (INT2) */
+    int32_t iters;      /* Lloyd iterations of a cold start (no initial centroids) */
+    int32_t warm_iters; /* Lloyd iterations when started from given centroids */
+} qvg_config;
+
+/* The packed (compressed) form of H blocks of N tokens.  All DEVICE
+ * pointers, caller-owned, written by qvg_quantize, read by qvg_dequantize.
+ *   codes     [H][N][d*bits/8]  2-bit codes, channel j of a token at bits
+ *                               2*(j%4) of byte j/4 of the token's row
+ *   scale     [H][N][d/G]       E4M3 bytes: group step s
+ *   zero      [H][N][d/G]       E4M3 bytes: group zero point m (the rounded
+ *                               group minimum); value = s*q + m
+ *   assign    [T][H][N]         uint8 centroid index of each token per stage
+ *   centroids [T][H][K][d]      centroid tables in the storage dtype
+ * With T = 0, assign and centroids are not accessed (may be NULL). */
+typedef struct {
+    uint8_t* codes;
+    uint8_t* scale;
+    uint8_t* zero;
+    uint8_t* assign;
+    void* centroids;
+} qvg_packed;
+
+/* Human-readable name of a status code (static string). */
+QVG_API const char* qvg_status_string(qvg_status s);
+
+/* Library build string, e.g. "qvg-b200 sm_100a". */
+QVG_API const char* qvg_version(void);
+
+/* Bytes of the packed form: H*N*d*bits/8 + 2*H*N*d/G + T*H*N +
+ * T*H*K*d*sizeof(S).  This equals bits-per-element x H*N*d/8 with
+ * bits-per-element = bits + 16/G + 8T/d + 8*sizeof(S)*T*K/N.  Returns 0 for
+ * invalid arguments.  Host-only, no CUDA call. */
+QVG_API size_t qvg_packed_bytes(const qvg_config* cfg, int64_t N, int32_t H, int32_t d,
+                        qvg_dtype dtype);
+
+/* Device scratch bytes qvg_quantize needs to process `H` blocks of N tokens
+ * in the library's preferred batch.  Any ws_bytes >= qvg_workspace_bytes(cfg,
+ * N, 1, d, dtype) works (the call then processes fewer blocks at a time).
+ * Returns 0 for invalid arguments.  Host-only, no CUDA call. */
+QVG_API size_t qvg_workspace_bytes(const qvg_config* cfg, int64_t N, int32_t H, int32_t d,
+                           qvg_dtype dtype);
+
+/* Compress H independent blocks X[H][N][d] (pre-RoPE K, or V, in `dtype`;
+ * section 五 caches keys before the rotary embedding) into `out`.
+ *   init_centroids: NULL for a cold start, in which every stage's k-means
+ *     starts from the first K tokens of its input and runs cfg->iters Lloyd
+ *     iterations; or DEVICE [T][H][K][d] tables in `dtype` (e.g. the previous
+ *     chunk's final centroids, section 五), with cfg->warm_iters iterations.
+ *   Each Lloyd iteration: assign every token to the centroid at the least
+ *     squared Euclidean distance (ties to the lowest index), then replace
+ *     every non-empty centroid by the mean of its tokens rounded to `dtype`
+ *     (an empty one keeps its value).  The stored pi(t) and C(t) are those of
+ *     the last iteration.  R(t) = round(R(t-1) - C(t)[pi(t)]).
+ *   The last residual is quantised per group g of G channels of a token:
+ *     m = E4M3(min), s = E4M3((max - m)/3), q = clamp(rint((r - m)/s), 0, 3),
+ *     (q = 0 when s = 0); E4M3 rounds to nearest even and saturates at 448.
+ *   workspace: DEVICE scratch of ws_bytes bytes (see qvg_workspace_bytes),
+ *     256-byte aligned, not shared with concurrent calls.
+ * Errors: INVALID_ARG for NULL pointers, K < 1 or K > 256, T < 0, bits != 2,
+ * G not dividing d or not a multiple of 4, N < 1, H < 1, N < K on a cold
+ * start with T > 0, iters < 1 (or warm_iters < 1 when warm) with T > 0;
+ * UNSUPPORTED for d != 128, G outside {8,16,32,64,128}, T > 8;
+ * WORKSPACE_TOO_SMALL; CUDA; DEVICE_TIMEOUT. */
+QVG_API qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype,
+                        int64_t N, int32_t H, int32_t d, const void* init_centroids,
+                        const qvg_packed* out, void* workspace, size_t ws_bytes,
+                        qvg_stream_t stream);
+
+/* Reconstruct Y[H][N][d] (DEVICE, `dtype`) from `packed` in one fused kernel:
+ * y = s*q + m, then + C(T)[pi_T], + C(T-1)[pi_(T-1)], ..., + C(1)[pi_1], each
+ * an fp32 add in that order, then one rounding to `dtype`.  Assignment
+ * values >= K are clamped to K-1.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+QVG_API qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packed, qvg_dtype dtype,
+                          int64_t N, int32_t H, int32_t d, void* Y, qvg_stream_t stream);
+
+/* Status word of a workspace after the work queued on it has completed
+ * (synchronises `stream`): QVG_OK, or QVG_ERR_DEVICE_TIMEOUT if a bounded
+ * device-side wait in a kernel gave up (its outputs are then invalid).
+ * Clears the word. */
+QVG_API qvg_status qvg_workspace_status(void* workspace, size_t ws_bytes, qvg_stream_t stream);
+
+/* Tokens whose tensor-core assignment was a near-tie and was decided by
+ * the exact fp64 pass, summed over the calls that used this workspace since
+ * the last read (synchronises `stream`; resets the count).  -1 on error.
+ * No counterpart in the method: a diagnostic of the assignment kernels. */
+QVG_API int64_t qvg_workspace_flagged(void* workspace, size_t ws_bytes, qvg_stream_t stream);
+
+/* ------------------------------------------------------------------ */
+/* Diagnostics (no counterpart in the method; used by the benchmark).    */
+/* ------------------------------------------------------------------ */
+
+/* Turn per-kernel device timing on or off (process-wide).  When on, every
+ * kernel launch is bracketed by two CUDA events on its stream. */
+QVG_API void qvg_profile_enable(int enable);
+
+/* Zero the launch counters and timing totals. */
+QVG_API void qvg_profile_reset(void);
+
+/* Kernel launches issued by this library since the last reset. */
+QVG_API int64_t qvg_profile_launches(void);
+
+/* Write a JSON object {"kernel": {"launches": n, "timed": m, "ms": t}, ...}
+ * into buf (NUL-terminated).  Synchronises the device if timed launches are
+ * pending.  Returns 0, or the needed size if buf is NULL or too small, or -1
+ * on a CUDA error. */
+QVG_API int qvg_profile_report(char* buf, size_t buf_bytes);
+
+/* ------------------------------------------------------------------ */
+/* Streaming cache (section 五, streaming centroid cache).               */
+/* A library-owned, append-only compressed KV cache for H blocks (heads). */
+/* Each appended chunk is quantised as one block per head; chunk c > 0    */
+/* warm-starts every stage's k-means from chunk c-1's final centroids.    */
+/* ------------------------------------------------------------------ */
+typedef struct qvg_cache qvg_cache;
+
+/* Allocate a cache for up to max_tokens tokens per head in up to max_chunks
+ * chunks (device memory on the current device).  Errors: INVALID_ARG,
+ * UNSUPPORTED, NO_MEMORY. */
+QVG_API qvg_status qvg_cache_create(const qvg_config* cfg, qvg_dtype dtype, int32_t H, int32_t d,
+                            int64_t max_tokens, int32_t max_chunks, qvg_cache** out);
+
+/* Compress and append one chunk X_chunk[H][N_chunk][d] (DEVICE, cache dtype).
+ * Chunk 0 runs a cold start (needs N_chunk >= K when T > 0) with cfg->iters;
+ * later chunks warm-start with cfg->warm_iters.  Errors: INVALID_ARG,
+ * CAPACITY, CUDA, NO_MEMORY. */
+QVG_API qvg_status qvg_append_chunk(qvg_cache* cache, const void* X_chunk, int64_t N_chunk,
+                            qvg_stream_t stream);
+
+/* Reconstruct the whole cache into Y[H][tokens][d] (DEVICE, cache dtype), one
+ * fused launch over every (chunk, head) block. */
+QVG_API qvg_status qvg_cache_dequantize(const qvg_cache* cache, void* Y, qvg_stream_t stream);
+
+QVG_API int64_t qvg_cache_tokens(const qvg_cache* cache);   /* tokens per head so far */
+QVG_API int32_t qvg_cache_chunks(const qvg_cache* cache);   /* chunks so far */
+
+/* Packed view of chunk `chunk` (DEVICE pointers into the cache, valid until
+ * qvg_cache_destroy; layouts as qvg_packed with H blocks of *n_tokens
+ * tokens); *first_token is the chunk's first token index. */
+QVG_API qvg_status qvg_cache_chunk_view(const qvg_cache* cache, int32_t chunk, qvg_packed* view,
+                                int64_t* first_token, int64_t* n_tokens);
+
+/* Bytes of device memory the cache holds (packed storage + workspace). */
+QVG_API size_t qvg_cache_device_bytes(const qvg_cache* cache);
+
+QVG_API void qvg_cache_destroy(qvg_cache* cache);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QVG_H_ */

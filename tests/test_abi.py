@@ -1,0 +1,104 @@
+"""CPU checks of the C ABI: the library loads, exports every function that
+include/qvg.h declares, and its host-only functions (sizes, argument checks)
+behave as declared.  No kernel is launched here."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def q():
+    from bit_kv_cache_qvg_b200 import build
+    build.build()
+    from bit_kv_cache_qvg_b200 import qvg
+    qvg.lib()
+    return qvg
+
+
+def _declared():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            names |= set(re.findall(r"QVG_API[^;(]*?\b(qvg_\w+)\s*\(", src, re.S))
+    return names
+
+
+def test_library_exports_every_declared_symbol(q):
+    declared = _declared()
+    assert len(declared) >= 15
+    L = C.CDLL(q.LIB_PATH)
+    for name in declared:
+        assert hasattr(L, name), name
+    assert declared == set(q.exported_symbols())
+
+
+def test_version_and_status_strings(q):
+    assert q.lib().qvg_version().decode().startswith("qvg-b200")
+    assert q.status_string(0) == "ok"
+    assert q.status_string(6) == "workspace too small"
+
+
+@pytest.mark.parametrize("K,T,G,N,H,dtype", [
+    (16, 1, 16, 512, 1, 1), (256, 2, 64, 4680, 12, 0), (256, 2, 64, 38000, 32, 0),
+    (64, 4, 32, 38000, 32, 0), (256, 0, 64, 100, 3, 0), (7, 3, 8, 1000, 5, 1),
+])
+def test_packed_bytes_matches_oracle_closed_form(q, ora, K, T, G, N, H, dtype):
+    cfg = q.config(K=K, T=T, group_size=G)
+    assert q.packed_bytes(cfg, N, H, 128, dtype) == ora.packed_bytes(K, T, G, N, H, 128, dtype=dtype)
+
+
+def test_workspace_bytes_positive_and_monotone(q):
+    cfg = q.config(K=256, T=2, group_size=64)
+    one = q.workspace_bytes(cfg, 38000, 1)
+    many = q.workspace_bytes(cfg, 38000, 64)
+    assert 0 < one <= many
+    assert q.workspace_bytes(q.config(K=0), 100, 1) == 0
+
+
+def _quantize_status(q, cfg, N=512, H=1, d=128, dtype=0, init=None, X=0x1000, ws=0x10000,
+                     ws_bytes=1 << 30, packed=None):
+    p = packed or q._Packed(0x2000, 0x3000, 0x4000, 0x5000, 0x6000)
+    return q.lib().qvg_quantize(C.byref(cfg), X, dtype, N, H, d, init, C.byref(p), ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(K=0), 1), (dict(K=257), 1), (dict(T=-1), 1), (dict(bits=3), 1),
+    (dict(group_size=6), 1), (dict(group_size=48), 1), (dict(iters=0), 1),
+    (dict(group_size=4), 2), (dict(T=9), 2),
+])
+def test_quantize_rejects_bad_config_without_touching_the_gpu(q, kw, expect):
+    args = dict(K=16, T=1, group_size=16, iters=4)
+    args.update(kw)
+    assert _quantize_status(q, q.config(**args)) == expect
+
+
+def test_quantize_rejects_bad_shapes_and_pointers(q):
+    cfg = q.config(K=16, T=1, group_size=16, iters=4)
+    assert _quantize_status(q, cfg, d=64) == 2                  # kernels are d = 128
+    assert _quantize_status(q, cfg, N=8) == 1                   # N < K on a cold start
+    assert _quantize_status(q, cfg, H=0) == 1
+    assert _quantize_status(q, cfg, X=None) == 1
+    assert _quantize_status(q, cfg, X=0x1001) == 1              # misaligned X
+    assert _quantize_status(q, cfg, ws=None) == 1
+    assert _quantize_status(q, cfg, dtype=7) == 1
+    assert _quantize_status(q, cfg, ws_bytes=16) == 6           # workspace too small
+    assert _quantize_status(q, cfg, packed=q._Packed(0x2000, 0x3000, 0x4000, None, None)) == 1
+
+
+def test_dequantize_and_cache_reject_bad_arguments(q):
+    cfg = q.config(K=16, T=1, group_size=16, iters=4)
+    p = q._Packed(0x2000, 0x3000, 0x4000, 0x5000, 0x6000)
+    L = q.lib()
+    assert L.qvg_dequantize(C.byref(cfg), C.byref(p), 0, 10, 1, 128, None, None) == 1
+    assert L.qvg_dequantize(C.byref(cfg), None, 0, 10, 1, 128, 0x1000, None) == 1
+    assert L.qvg_dequantize(C.byref(q.config(K=300)), C.byref(p), 0, 10, 1, 128, 0x1000, None) == 1
+    h = C.c_void_p()
+    assert L.qvg_cache_create(C.byref(cfg), 0, 1, 128, 0, 4, C.byref(h)) == 1
+    assert L.qvg_cache_create(C.byref(cfg), 0, 1, 96, 100, 4, C.byref(h)) == 2
+    assert L.qvg_append_chunk(None, 0x1000, 10, None) == 1
+    assert L.qvg_cache_tokens(None) == 0 and L.qvg_cache_chunks(None) == 0
