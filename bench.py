@@ -143,6 +143,7 @@ def main():
     ap.add_argument("--workload", default="longcat", choices=sorted(WORKLOADS))
     ap.add_argument("--layers", type=int, default=None, help="override the layer count")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=4750)
     ap.add_argument("--cpu-tokens", type=int, default=9500)
@@ -195,7 +196,8 @@ def main():
     packed = qvg.alloc_packed(cfg, N, U, device=dev)
     ws = qvg.alloc_workspace(cfg, N, U, device=dev)
     Y = torch.empty_like(X)
-    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(dev)     # a side stream: CUDA graphs are captured on one
 
     def step():
         qvg.quantize(X, cfg, out=packed, workspace=ws, stream=stream)
@@ -207,29 +209,68 @@ def main():
     if qvg.workspace_status(ws) != 0:
         raise SystemExit("device-side wait timed out during warm-up")
 
+    # One step is captured as a CUDA graph (every launch of the library is a
+    # stream operation); the timed region replays it.
+    graph = None
+    if not args.eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        with torch.cuda.stream(stream):
+            graph.replay()
+        torch.cuda.synchronize()
+
     # timed region: inputs (29.9 GB for the default workload) exceed L2, no flush needed
-    qvg.profile_reset()
-    qvg.profile_enable(True)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize()
         ev0.record(stream)
-        for _ in range(args.steps):
-            step()
+        with torch.cuda.stream(stream):       # replay() launches on the current stream
+            for _ in range(args.steps):
+                if graph is not None:
+                    graph.replay()
+                else:
+                    step()
         ev1.record(stream)
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
-    qvg.profile_enable(False)
-    launches = qvg.profile_launches()
-    kernels = qvg.profile_report()
     ms = ev0.elapsed_time(ev1) / args.steps
     if dist is not None:
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
+    if qvg.workspace_status(ws) != 0:
+        raise SystemExit("device-side wait timed out in the timed region")
+
+    # per-kernel device time: one more step, captured with a CUDA event recorded
+    # on the launching stream before and after every kernel, then replayed
+    qvg.workspace_flagged(ws)           # reset the near-tie counter
+    qvg.profile_reset()
+    qvg.profile_enable(True)
+    if graph is not None:
+        pgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(pgraph, stream=stream):
+            step()                      # the event pairs become graph nodes
+        qvg.profile_enable(False)
+        pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pe0.record(stream)
+        with torch.cuda.stream(stream):
+            pgraph.replay()
+        pe1.record(stream)
+    else:
+        pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pe0.record(stream)
+        step()
+        pe1.record(stream)
+    torch.cuda.synchronize()
+    qvg.profile_enable(False)
+    launches = qvg.profile_launches() * args.steps
+    kernels = qvg.profile_report()
+    eager_ms = pe0.elapsed_time(pe1)
+    flagged = qvg.workspace_flagged(ws)
     kv_bytes = U * N * 128 * 2
     value = kv_bytes * world / (ms / 1e3) / 1e9
 
@@ -238,7 +279,7 @@ def main():
     esz = 2
     deq_bytes_per_elem = 2 / 8 + 2 / G + T / 128 + esz * T * K / N + 2
     roof = {}
-    if "qvg_dequant_fused" in kernels:
+    if "qvg_dequant_fused" in kernels and kernels["qvg_dequant_fused"]["ms"] > 0:
         k = kernels["qvg_dequant_fused"]
         t_launch = k["ms"] / max(k["timed"], 1) / 1e3
         per_launch = deq_bytes_per_elem * E
@@ -247,9 +288,9 @@ def main():
                                      "frac": per_launch / t_launch / 1e9 / peaks["hbm"], "traffic": None,
                                      "alg_bytes_per_launch": per_launch}
     for name in ("qvg_kmeans_assign", "qvg_assign_exact"):
-        if name in kernels and kernels[name]["timed"]:
+        if name in kernels and kernels[name]["timed"] and kernels[name]["ms"] > 0:
             k = kernels[name]
-            flops_total = 2.0 * K * 128 * N * U * T * I * args.steps
+            flops_total = 2.0 * K * 128 * N * U * T * I
             # an assign launch covers one batch of blocks for one Lloyd iteration
             per_launch = flops_total / k["timed"]
             t_launch = k["ms"] / k["timed"] / 1e3
@@ -263,7 +304,7 @@ def main():
         dominant = dict(dominant, kernel=top if top in roof else next(iter(roof)))
 
     # quantise-path roofline: max(F / P_bf16, B / BW)
-    q_ms = sum(v["ms"] for n, v in kernels.items() if n != "qvg_dequant_fused") / args.steps
+    q_ms = sum(v["ms"] for n, v in kernels.items() if n != "qvg_dequant_fused")
     F = 2.0 * K * I * T * E
     B = E * 2 + packed.nbytes()
     q_roof_ms = max(F / (peaks["bf16_sus"] * 1e12), B / (peaks["hbm"] * 1e9)) * 1e3
@@ -282,6 +323,10 @@ def main():
                           "peak_source": peaks["source"]},
         "kernels": kernels,
         "gpu_launches": launches,
+        "profiled_step_ms_with_kernel_events": eager_ms,
+        "timed_region": "CUDA graph replay of the step" if graph is not None else "eager launches",
+        "near_tie_tokens_per_step": flagged if flagged >= 0 else None,
+        "token_assignments_per_step": U * N * T * I,
         "clocks": clk.summary(),
     }
 

@@ -119,6 +119,22 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// Descriptor of a K-major operand without swizzle: 8x16-byte core matrices,
+// the two 8-element K halves 128 bytes apart (LBO), 8-row groups 256 bytes
+// apart (SBO).
+__device__ __forceinline__ uint64_t umma_desc_noswz(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)(128 >> 4) << 16;        // LBO
+  d |= (uint64_t)(256 >> 4) << 32;        // SBO
+  d |= (uint64_t)1 << 46;                 // version
+  return d;                               // layout type 0: no swizzle
+}
+// Byte offset of element (row, k), k < 16, in that layout.
+__device__ __forceinline__ int noswz_offset(int row, int k) {
+  return (row >> 3) * 256 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2;
+}
+
 // Instruction descriptor: kind::f16, A = B = bf16, D = f32, both K-major.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
@@ -170,13 +186,13 @@ struct TcParams {
   const float* rnorm2;      // [W][N]
   const float* cn;          // [W][K]
   uint8_t* pi;              // [W][N]
-  uint32_t* list;           // [W][N]
+  uint2* list;              // [W][N] {token, mask of 32-centroid chunks holding the candidates}
   uint32_t* list_count;     // [W]
   uint32_t* status;         // workspace status word
   unsigned long long* flagged;
   int64_t N;
   int K;
-  int Npad;                 // K rounded up to 16 (MMA N)
+  int Npad;                 // K rounded up to 32 (MMA N)
   int tiles_per_unit;
   int tiles_per_cta;
   float gamma;              // relative error bound of the tensor-core dot products
@@ -201,6 +217,12 @@ __device__ __forceinline__ void set_abort(TcSmemBarriers* b) {
   *reinterpret_cast<volatile int*>(&b->abort_flag) = 1;
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ float key_with_index(float g, int k) {
   return __int_as_float((__float_as_int(g) & ~0xFF) | k);
 }
@@ -219,9 +241,10 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
   const int Npad = p.Npad;
   uint8_t* sB = smem;                                           // 2 x Npad x 128 B
   uint8_t* sA = smem + 2 * Npad * 128;                          // kStages x 32 KB (1024-aligned)
-  float* cn_s = reinterpret_cast<float*>(sA + kStages * kAStageBytes);   // [256]
-  float* mbuf = cn_s + kMaxK;                                   // [2 acc][2 vals][128 rows]
-  TcSmemBarriers* bars = reinterpret_cast<TcSmemBarriers*>(mbuf + 2 * 2 * kTileM);
+  uint8_t* sAx = sA + kStages * kAStageBytes;                   // 128 x 16 bf16: [1 1 1 0 ...]
+  uint8_t* sBx = sAx + kTileM * 32;                             // Npad x 16 bf16: -|c|^2/2 in 3 pieces
+  float* mbuf = reinterpret_cast<float*>(sBx + Npad * 32);      // [2 acc][2 halves][6 vals][128 rows]
+  TcSmemBarriers* bars = reinterpret_cast<TcSmemBarriers*>(mbuf + 2 * 12 * kTileM);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -237,8 +260,33 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
                      smem_u32(&bars->tmem_base)));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  for (int k = threadIdx.x; k < kMaxK; k += blockDim.x)
-    cn_s[k] = k < p.K ? p.cn[(int64_t)u * p.K + k] : __int_as_float(0x7f800000);
+  // Extra K step of the MMA: A rows [1, 1, 1, 0, ...] times B rows
+  // [b0, b1, b2, 0, ...] with b0 + b1 + b2 = -|c_k|^2 / 2 (three bf16 pieces
+  // of the fp32 value; the most negative bf16 for padded centroids) adds -|c_k|^2/2 to every
+  // dot product, so the accumulator holds r.c_k - |c_k|^2/2.
+  for (int x = threadIdx.x; x < kTileM * 16; x += blockDim.x) {
+    const int r = x >> 4, k = x & 15;
+    *reinterpret_cast<uint16_t*>(sAx + noswz_offset(r, k)) = k < 3 ? (uint16_t)0x3F80 : (uint16_t)0;
+  }
+  for (int x = threadIdx.x; x < Npad * 16; x += blockDim.x) {
+    const int c = x >> 4, k = x & 15;
+    uint16_t bits = 0;
+    if (k < 3) {
+      if (c >= p.K) {
+        bits = k == 0 ? (uint16_t)0xFF7F : (uint16_t)0;           // -3.39e38: never the maximum
+      } else {
+        const float v = -0.5f * p.cn[(int64_t)u * p.K + c];
+        const __nv_bfloat16 b0 = __float2bfloat16_rn(v);
+        const float r1 = __fsub_rn(v, __bfloat162float(b0));
+        const __nv_bfloat16 b1 = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 b2 = __float2bfloat16_rn(__fsub_rn(r1, __bfloat162float(b1)));
+        const __nv_bfloat16 pick = k == 0 ? b0 : (k == 1 ? b1 : b2);
+        bits = *reinterpret_cast<const uint16_t*>(&pick);
+      }
+    }
+    *reinterpret_cast<uint16_t*>(sBx + noswz_offset(c, k)) = bits;
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -274,6 +322,7 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_bf16(kTileM, Npad);
       const uint32_t b_addr = smem_u32(sB);
+      const uint32_t ax_addr = smem_u32(sAx), bx_addr = smem_u32(sBx);
       bool ok = mbar_wait(&bars->b_full, 0);
       if (!ok) TC_DBG(4, 1);
       int issued = 0;
@@ -295,6 +344,7 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
           const uint64_t bd = umma_desc_sw128(b_addr + (k >> 2) * Npad * 128 + koff);
           umma_bf16(d_tmem, ad, bd, idesc, k > 0 ? 1u : 0u);
         }
+        umma_bf16(d_tmem, umma_desc_noswz(ax_addr), umma_desc_noswz(bx_addr), idesc, 1u);
         umma_commit(&bars->empty[s]);
         umma_commit(&bars->tmem_full[acc]);
         ++issued;
@@ -310,68 +360,122 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int hc = (warp - 2) >> 2;          // centroid-column half
     const int row = q * 32 + lane;
+    const bool mine = (lane >> 4) == hc;     // rows this thread decides after the merge
     const int ncol = Npad > 128 ? Npad - 128 : 0;
     const int cols = hc == 0 ? min(Npad, 128) : ncol;
+    const float kInf = __int_as_float(0x7f800000);
+    float rn2_next = 0.0f;
+    {
+      const int64_t tok = (int64_t)t_begin * kTileM + row;
+      if (mine && tok < p.N) rn2_next = p.rnorm2[(int64_t)u * p.N + tok];
+    }
     for (int i = 0; i < ntiles; ++i) {
       const int acc = i & 1;
       const uint32_t aph = (uint32_t)(i >> 1) & 1u;
+      const float rn2 = rn2_next;
+      {   // prefetch the next tile's squared row norm
+        const int64_t tok = (int64_t)(t_begin + i + 1) * kTileM + row;
+        if (mine && i + 1 < ntiles && tok < p.N) rn2_next = p.rnorm2[(int64_t)u * p.N + tok];
+      }
       const bool ok = !aborted(bars) && mbar_wait(&bars->tmem_full[acc], aph);
       if (!ok) { TC_DBG(8, i + 1); set_abort(bars); }
       else if (lane == 0 && warp == 2) TC_DBG(18, i + 1);
       tc_fence_after();
-      float v1 = __int_as_float(0x7f800000), v2 = v1;
+      // Top two of h_k = r.c_k - |c_k|^2/2 (the largest h is the nearest
+      // centroid), each value carrying its column index in its 8 low bits;
+      // columns are taken in pairs, four independent chains.  The largest key
+      // of every 32-column chunk is kept too: it tells the exact pass which
+      // chunks can hold a near-tie candidate.
+      const float kNegBig = -3.0e38f;
+      float c1[4] = {kNegBig, kNegBig, kNegBig, kNegBig}, c2[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
+      float cmax[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
       if (ok) {
         const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256 + hc * 128);
-        for (int c0 = 0; c0 < cols; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(tbase + (uint32_t)c0, r);
-          const int kb = hc * 128 + c0;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float g = __fmaf_rn(-2.0f, __uint_as_float(r[e]), cn_s[kb + e]);
-            const float key = key_with_index(g, kb + e);
-            v2 = fminf(v2, fmaxf(v1, key));
-            v1 = fminf(v1, key);
+        for (int ci = 0; ci < 4; ++ci) {
+          const int c0 = ci * 32;
+          if (c0 < cols) {
+            uint32_t r[32];
+            tmem_ld32(tbase + (uint32_t)c0, r);
+            const int kb = hc * 128 + c0;
+            float m0 = kNegBig, m1 = kNegBig;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float ka = key_with_index(__uint_as_float(r[e]), kb + e);
+              const float kb2 = key_with_index(__uint_as_float(r[e + 1]), kb + e + 1);
+              const float kc = key_with_index(__uint_as_float(r[e + 2]), kb + e + 2);
+              const float kd = key_with_index(__uint_as_float(r[e + 3]), kb + e + 3);
+              const float hi0 = fmaxf(ka, kb2), lo0 = fminf(ka, kb2);
+              const float hi1 = fmaxf(kc, kd), lo1 = fminf(kc, kd);
+              const int ch0 = (e >> 1) & 3, ch1 = ((e >> 1) + 1) & 3;
+              c2[ch0] = max3f(fminf(c1[ch0], hi0), c2[ch0], lo0);
+              c1[ch0] = fmaxf(c1[ch0], hi0);
+              c2[ch1] = max3f(fminf(c1[ch1], hi1), c2[ch1], lo1);
+              c1[ch1] = fmaxf(c1[ch1], hi1);
+              if ((e & 4) == 0) m0 = max3f(m0, hi0, hi1); else m1 = max3f(m1, hi0, hi1);
+            }
+            cmax[ci] = fmaxf(m0, m1);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->tmem_empty[acc]);
-      float* mb = mbuf + acc * 2 * kTileM;
-      if (hc == 1) { mb[row] = v1; mb[kTileM + row] = v2; }
+      float v1 = fmaxf(c1[0], c1[1]), v2 = max3f(fminf(c1[0], c1[1]), c2[0], c2[1]);
+      const float u1 = fmaxf(c1[2], c1[3]), u2 = max3f(fminf(c1[2], c1[3]), c2[2], c2[3]);
+      v2 = max3f(fminf(v1, u1), v2, u2);
+      v1 = fmaxf(v1, u1);
+      float* mb = mbuf + acc * 12 * kTileM;      // [hc][v1, v2, chunk max 0..3][row]
+      mb[(hc * 6 + 0) * kTileM + row] = v1;
+      mb[(hc * 6 + 1) * kTileM + row] = v2;
+#pragma unroll
+      for (int ci = 0; ci < 4; ++ci) mb[(hc * 6 + 2 + ci) * kTileM + row] = cmax[ci];
       named_bar_sync(1, 256);
-      if (hc == 0) {
-        const float o1 = mb[row], o2 = mb[kTileM + row];
-        const float w1 = fminf(v1, o1);
-        const float w2 = fminf(fmaxf(v1, o1), fminf(v2, o2));
-        const int64_t tok = (int64_t)(t_begin + i) * kTileM + row;
-        const bool valid = tok < p.N && !aborted(bars);
-        const int64_t gi = (int64_t)u * p.N + tok;
-        bool flag = false;
-        if (valid) {
-          // error bound of the screening values (see qvg_assign_exact) plus the
-          // 2^-15 relative perturbation of the index bits in both keys
-          const float rn2 = p.rnorm2[gi];
-          const float nr = sqrtf(fmaxf(rn2, 0.0f)) * 1.0001f;
-          const float cb = 1.02f * nr + sqrtf(fmaxf(rn2 + w1, 0.0f));
-          const float E = 2.0f * p.gamma * nr * cb + 1.2e-7f * cb * cb + 1.2e-7f * fabsf(w1) + 1e-30f;
-          const float margin = 2.0f * E + 6.2e-5f * (fabsf(w1) + fabsf(w2));
-          flag = !(w2 - w1 > margin);
-          if (!flag) p.pi[gi] = (uint8_t)(__float_as_int(w1) & 0xFF);
-        }
-        // every lane of the warp takes part in the list append
-        const unsigned fm = __ballot_sync(0xffffffffu, flag);
-        if (fm) {
-          const int leader = __ffs(fm) - 1;
-          uint32_t base = 0;
-          if (lane == leader) {
-            base = atomicAdd(&p.list_count[u], (uint32_t)__popc(fm));
-            atomicAdd(p.flagged, (unsigned long long)__popc(fm));
+      // each half decides 16 of the warp's 32 rows
+      const int oh = 1 - hc;
+      const float o1 = mb[(oh * 6 + 0) * kTileM + row], o2 = mb[(oh * 6 + 1) * kTileM + row];
+      const float w1 = fmaxf(v1, o1);
+      const float w2 = max3f(fminf(v1, o1), v2, o2);
+      const int64_t tok = (int64_t)(t_begin + i) * kTileM + row;
+      const bool valid = mine && tok < p.N && !aborted(bars);
+      const int64_t gi = (int64_t)u * p.N + tok;
+      bool flag = false;
+      uint32_t chunks = 0;
+      if (valid) {
+        // Error bound of h (fp32 tensor-core sums of 128 exact products and the
+        // three pieces of -|c|^2/2): gamma * (|r| |c| + |c|^2 / 2) for every
+        // centroid at least as near as the nearest, |c| <= |r| + sqrt(D_min);
+        // plus the 2^-15 relative perturbation of the index bits of both keys.
+        const float nr = sqrtf(fmaxf(rn2, 0.0f)) * 1.0001f;
+        const float cb = 1.02f * nr + sqrtf(fmaxf(rn2 - 2.0f * w1, 0.0f));
+        const float E = p.gamma * (nr * cb + 0.5f * cb * cb) + 6.0e-8f * cb * cb + 1e-30f;
+        const float margin = 2.0f * E + 3.1e-5f * (fabsf(w1) + fabsf(w2));
+        flag = !(w1 - w2 > margin);
+        if (!flag) {
+          p.pi[gi] = (uint8_t)(__float_as_int(w1) & 0xFF);
+        } else {
+          // chunks whose largest key reaches the threshold (with the index-bit
+          // perturbation of that key allowed for) hold every candidate
+          const float thr = w1 - margin;
+          const float thr_key = thr - 6.2e-5f * (fabsf(w1) + fabsf(thr));
+#pragma unroll
+          for (int ci = 0; ci < 4; ++ci) {
+            if (cmax[ci] >= thr_key) chunks |= 1u << (hc * 4 + ci);
+            if (mb[(oh * 6 + 2 + ci) * kTileM + row] >= thr_key) chunks |= 1u << (oh * 4 + ci);
           }
-          base = __shfl_sync(0xffffffffu, base, leader);
-          if (flag) p.list[(int64_t)u * p.N + base + __popc(fm & ((1u << lane) - 1u))] = (uint32_t)tok;
         }
+      }
+      // every lane of the warp takes part in the list append
+      const unsigned fm = __ballot_sync(0xffffffffu, flag);
+      if (fm) {
+        const int leader = __ffs(fm) - 1;
+        uint32_t base = 0;
+        if (lane == leader) {
+          base = atomicAdd(&p.list_count[u], (uint32_t)__popc(fm));
+          atomicAdd(p.flagged, (unsigned long long)__popc(fm));
+        }
+        base = __shfl_sync(0xffffffffu, base, leader);
+        if (flag) p.list[(int64_t)u * p.N + base + __popc(fm & ((1u << lane) - 1u))] = make_uint2((uint32_t)tok, chunks);
       }
     }
   }
@@ -418,23 +522,22 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int W, int box_row
 }  // namespace
 
 size_t assign_tc_smem_bytes(int K) {
-  const int Npad = (K + 15) & ~15;
-  return 1024 + 2 * (size_t)Npad * 128 + (size_t)kStages * kAStageBytes + kMaxK * 4 + 2 * 2 * kTileM * 4 +
+  const int Npad = (K + 31) & ~31;
+  return 1024 + 2 * (size_t)Npad * 128 + (size_t)kStages * kAStageBytes + kTileM * 32 + (size_t)Npad * 32 +
+         2 * 12 * kTileM * 4 +
          sizeof(TcSmemBarriers);
 }
 
 cudaError_t launch_assign_tc(const AssignTcParams& a, cudaStream_t s) {
   CUtensorMap mR, mC;
-  const int Npad = (a.K + 15) & ~15;
+  const int Npad = (a.K + 31) & ~31;
   if (!make_map(&mR, a.R, a.N, a.W, kTileM) || !make_map(&mC, a.C, a.K, a.W, Npad))
     return cudaErrorInvalidValue;
   TcParams p{};
   p.rnorm2 = a.rnorm2; p.cn = a.cn; p.pi = a.pi; p.list = a.list; p.list_count = a.list_count;
   p.status = a.status; p.flagged = a.flagged; p.N = a.N; p.K = a.K; p.Npad = Npad;
   p.tiles_per_unit = (int)((a.N + kTileM - 1) / kTileM);
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   int splits = sms / a.W;
   if (splits < 1) splits = 1;
   p.tiles_per_cta = (p.tiles_per_unit + splits - 1) / splits;
@@ -442,7 +545,7 @@ cudaError_t launch_assign_tc(const AssignTcParams& a, cudaStream_t s) {
   splits = (p.tiles_per_unit + p.tiles_per_cta - 1) / p.tiles_per_cta;
   p.gamma = a.gamma;
   const size_t smem = assign_tc_smem_bytes(a.K);
-  cudaError_t e = cudaFuncSetAttribute(qvg_kmeans_assign, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(qvg_kmeans_assign), smem);
   if (e != cudaSuccess) return e;
 #ifdef QVG_TC_DEBUG
   {

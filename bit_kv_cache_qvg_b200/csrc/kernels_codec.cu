@@ -66,16 +66,29 @@ template <> struct Vec8<kFP32> {
 
 // ---------------------------------------------------------------- dequant
 constexpr int kDqThreads = 512;
-constexpr int kDqTokPerIter = kDqThreads / 8;   // 64 tokens per block iteration
-constexpr int kDqUnroll = 4;                    // tokens per thread per iteration
+constexpr int kDqTokPerIter = kDqThreads / 8;   // 64 tokens per block row of threads
+constexpr int kDqUnroll = 4;                    // tokens per thread per tile
+constexpr int kDqTile = kDqTokPerIter * kDqUnroll;   // 256 tokens per tile
+constexpr int kDqStages = 3;                    // codes ring depth
+constexpr int kDqTileBytes = kDqTile * (kD / 4);     // 8 KB of codes per tile
 
-// TT = number of stages when it is <= 4 (all assignment loads issued up front),
-// or -1 for the generic runtime-T loop.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// TT = number of stages when it is <= 4 (the tile's assignments are fetched
+// one tile ahead into registers), or -1 for the generic runtime-T loop.
 template <int DT, int TT>
 __global__ void __launch_bounds__(kDqThreads)
 qvg_dequant_fused(const DequantParams p, const int splits) {
   constexpr int ESZ = Store<DT>::bytes;
-  constexpr int TR = TT < 0 ? 1 : (TT == 0 ? 1 : TT);
+  constexpr int TR = TT <= 0 ? 1 : TT;
   extern __shared__ __align__(16) unsigned char smem[];
 
   const int unit = blockIdx.x / splits;
@@ -92,17 +105,9 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
   const int64_t i_end = min(n_c, i_begin + per);
   const int K = p.K, T = TT < 0 ? p.T : TT, G = p.G;
   const int64_t tab_elems = (int64_t)K * kD;
+  const size_t tab_bytes = (size_t)tab_elems * ESZ;
   const char* tables = static_cast<const char*>(p.centroids) + (int64_t)c * T * p.H * tab_elems * ESZ;
-
-  // Stage the first t_smem tables of this (chunk, head) in shared memory.
-  for (int t = 0; t < p.t_smem; ++t) {
-    const uint4* src = reinterpret_cast<const uint4*>(tables + ((int64_t)t * p.H + h) * tab_elems * ESZ);
-    uint4* dst = reinterpret_cast<uint4*>(smem + (size_t)t * tab_elems * ESZ);
-    const int n16 = (int)(tab_elems * ESZ / 16);
-    for (int x = threadIdx.x; x < n16; x += blockDim.x) dst[x] = src[x];
-  }
-  __syncthreads();
-  if (i_begin >= i_end) return;
+  uint8_t* cring = smem + (size_t)p.t_smem * tab_bytes;       // codes ring (16-byte aligned)
 
   const int j = threadIdx.x & 7;
   const int tl = threadIdx.x >> 3;
@@ -115,49 +120,83 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
   const uint8_t* asg = p.assign + (int64_t)T * p.H * o_c + (int64_t)h * n_c;
   const int64_t asg_t = (int64_t)p.H * n_c;
   char* Y = static_cast<char*>(p.Y) + ((int64_t)h * p.y_head_stride + o_c) * kD * ESZ;
+  const int64_t ntile = i_end > i_begin ? (i_end - i_begin + kDqTile - 1) / kDqTile : 0;
+  if (ntile == 0) return;                                     // uniform over the block
 
-  for (int64_t base = i_begin + tl; base < i_end; base += kDqTokPerIter * kDqUnroll) {
-    int64_t tok[kDqUnroll];
-    uint32_t q0[kDqUnroll], q1[kDqUnroll];
-    uint8_t s0b[kDqUnroll], m0b[kDqUnroll], s1b[kDqUnroll], m1b[kDqUnroll];
-    int kk[kDqUnroll][TR];
-    // issue every load of the iteration first
+  // codes of tile t -> ring slot t % kDqStages: one 16-byte async copy per thread
+  auto issue = [&](int64_t t) {
+    if (t < ntile) {
+      const int64_t tok0 = i_begin + t * kDqTile;
+      const int64_t nbytes = min((int64_t)kDqTile, i_end - tok0) * (kD / 4);
+      if ((int64_t)threadIdx.x * 16 < nbytes)
+        cp_async16(cring + (t % kDqStages) * kDqTileBytes + threadIdx.x * 16,
+                   codes + tok0 * (kD / 4) + threadIdx.x * 16);
+    }
+    cp_async_commit();
+  };
+  issue(0);
+  issue(1);
+
+  // Stage the first t_smem tables of this (chunk, head) in shared memory.
+  for (int t = 0; t < p.t_smem; ++t) {
+    const uint4* src = reinterpret_cast<const uint4*>(tables + ((int64_t)t * p.H + h) * tab_bytes);
+    uint4* dst = reinterpret_cast<uint4*>(smem + (size_t)t * tab_bytes);
+    const int n16 = (int)(tab_bytes / 16);
+    for (int x = threadIdx.x; x < n16; x += blockDim.x) dst[x] = src[x];
+  }
+
+  // per-token bytes of a tile: scale/zero of both groups, assignments (TT <= 4)
+  uint32_t sz[kDqUnroll], ka[kDqUnroll];
+  auto fetch_small = [&](int64_t t, uint32_t (&s_out)[kDqUnroll], uint32_t (&k_out)[kDqUnroll]) {
 #pragma unroll
     for (int u = 0; u < kDqUnroll; ++u) {
-      tok[u] = base + u * kDqTokPerIter;
-      const int64_t i = tok[u] < i_end ? tok[u] : base;
-      q0[u] = *reinterpret_cast<const uint16_t*>(codes + i * (kD / 4) + 2 * j);
-      q1[u] = *reinterpret_cast<const uint16_t*>(codes + i * (kD / 4) + 16 + 2 * j);
-      s0b[u] = sc[i * ng + g0]; m0b[u] = zr[i * ng + g0];
-      s1b[u] = sc[i * ng + g1]; m1b[u] = zr[i * ng + g1];
+      int64_t i = i_begin + t * kDqTile + tl + u * kDqTokPerIter;
+      if (t >= ntile || i >= i_end) i = i_begin;
+      s_out[u] = (uint32_t)sc[i * ng + g0] | ((uint32_t)zr[i * ng + g0] << 8) |
+                 ((uint32_t)sc[i * ng + g1] << 16) | ((uint32_t)zr[i * ng + g1] << 24);
+      uint32_t kw = 0;
       if (TT > 0) {
 #pragma unroll
-        for (int t = 0; t < TR; ++t) kk[u][t] = asg[t * asg_t + i];
+        for (int tt = 0; tt < TR; ++tt) kw |= (uint32_t)asg[tt * asg_t + i] << (8 * tt);
       }
+      k_out[u] = kw;
     }
-    // then finish the tokens one at a time (16 values live per thread)
+  };
+  fetch_small(0, sz, ka);
+
+  for (int64_t t = 0; t < ntile; ++t) {
+    issue(t + 2);
+    cp_async_wait<2>();          // this thread's copies of tile t have landed
+    __syncthreads();             // everyone's have (and the tables are staged)
+    uint32_t sz_n[kDqUnroll], ka_n[kDqUnroll];
+    fetch_small(t + 1, sz_n, ka_n);
+    const uint8_t* ct = cring + (t % kDqStages) * kDqTileBytes;
 #pragma unroll
     for (int u = 0; u < kDqUnroll; ++u) {
+      const int r = tl + u * kDqTokPerIter;                // token within the tile
+      const int64_t tok = i_begin + t * kDqTile + r;
+      const uint32_t q0 = *reinterpret_cast<const uint16_t*>(ct + r * (kD / 4) + 2 * j);
+      const uint32_t q1 = *reinterpret_cast<const uint16_t*>(ct + r * (kD / 4) + 16 + 2 * j);
+      const float s0 = e4m3_to_f32((uint8_t)(sz[u] & 0xFF)), m0 = e4m3_to_f32((uint8_t)((sz[u] >> 8) & 0xFF));
+      const float s1 = e4m3_to_f32((uint8_t)((sz[u] >> 16) & 0xFF)), m1 = e4m3_to_f32((uint8_t)(sz[u] >> 24));
       float y0[8], y1[8];
-      const float s0 = e4m3_to_f32(s0b[u]), m0 = e4m3_to_f32(m0b[u]);
-      const float s1 = e4m3_to_f32(s1b[u]), m1 = e4m3_to_f32(m1b[u]);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         // s*q + m is exact in fp32 (E4M3 operands, q <= 3)
-        y0[e] = __fmaf_rn(s0, (float)((q0[u] >> (2 * e)) & 3u), m0);
-        y1[e] = __fmaf_rn(s1, (float)((q1[u] >> (2 * e)) & 3u), m1);
+        y0[e] = __fmaf_rn(s0, (float)((q0 >> (2 * e)) & 3u), m0);
+        y1[e] = __fmaf_rn(s1, (float)((q1 >> (2 * e)) & 3u), m1);
       }
-      const int64_t i = tok[u] < i_end ? tok[u] : base;
+      const int64_t ii = tok < i_end ? tok : i_begin;
       // centroids of stage T, T-1, ..., 1, in that order
 #pragma unroll
       for (int tt = 0; tt < (TT < 0 ? kMaxT : (TT == 0 ? 0 : TR)); ++tt) {
-        const int t = T - 1 - tt;
-        if (TT < 0 && t < 0) break;
-        int k = TT > 0 ? kk[u][t] : (int)asg[t * asg_t + i];
+        const int st = T - 1 - tt;
+        if (TT < 0 && st < 0) break;
+        int k = TT > 0 ? (int)((ka[u] >> (8 * st)) & 0xFF) : (int)asg[st * asg_t + ii];
         k = k < K ? k : K - 1;
-        const char* rowp = (t < p.t_smem)
-            ? reinterpret_cast<const char*>(smem) + ((int64_t)t * tab_elems + (int64_t)k * kD) * ESZ
-            : tables + (((int64_t)t * p.H + h) * tab_elems + (int64_t)k * kD) * ESZ;
+        const char* rowp = (st < p.t_smem)
+            ? reinterpret_cast<const char*>(smem) + ((int64_t)st * tab_elems + (int64_t)k * kD) * ESZ
+            : tables + (((int64_t)st * p.H + h) * tab_elems + (int64_t)k * kD) * ESZ;
         float c0[8], c1[8];
         Vec8<DT>::load(rowp + 8 * j * ESZ, c0);
         Vec8<DT>::load(rowp + (64 + 8 * j) * ESZ, c1);
@@ -167,13 +206,17 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
           y1[e] = __fadd_rn(y1[e], c1[e]);
         }
       }
-      if (tok[u] < i_end) {
-        char* yr = Y + tok[u] * kD * ESZ;
+      if (tok < i_end) {
+        char* yr = Y + tok * kD * ESZ;
         Vec8<DT>::store(yr + 8 * j * ESZ, y0);
         Vec8<DT>::store(yr + (64 + 8 * j) * ESZ, y1);
       }
     }
+#pragma unroll
+    for (int u = 0; u < kDqUnroll; ++u) { sz[u] = sz_n[u]; ka[u] = ka_n[u]; }
+    __syncthreads();             // ring slot t % kDqStages is free again
   }
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------- residual / quant
@@ -346,8 +389,7 @@ qvg_init_centroids(const void* src, int64_t src_unit_stride, void* C, float* cn,
 
 template <typename F>
 cudaError_t set_smem(F* f, size_t bytes) {
-  if (bytes <= 48 * 1024) return cudaSuccess;
-  return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  return ensure_dynamic_smem(reinterpret_cast<const void*>(f), bytes);
 }
 
 }  // namespace
@@ -374,12 +416,10 @@ static cudaError_t launch_dq_t(const DequantParams& p, int blocks, int splits, s
 
 cudaError_t launch_dequant(const DequantParams& p, int dtype, cudaStream_t s) {
   const int esz = dtype == kBF16 ? 2 : 4;
-  const size_t smem = (size_t)p.t_smem * p.K * kD * esz;
+  const size_t smem = (size_t)p.t_smem * p.K * kD * esz + (size_t)kDqStages * kDqTileBytes;
   const int units = p.n_chunks * p.H;
   if (units == 0) return cudaSuccess;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   // split blocks along tokens until the grid covers the GPU at least twice
   int splits = (2 * sms + units - 1) / units;
   const int64_t ntok = p.chunk_off ? 0 : p.N;
@@ -407,9 +447,7 @@ cudaError_t launch_residual(const ResidualParams& p, int dtype, bool quant, cuda
   const int esz = dtype == kBF16 ? 2 : 4;
   const bool has_c = p.C != nullptr;
   const size_t smem = has_c ? (size_t)p.K * kD * esz : 0;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   // Enough blocks for two waves over the SMs; each block stages the table once.
   int64_t splits = (2 * (int64_t)sms + p.W - 1) / p.W;
   const int64_t min_tok = 256;

@@ -19,6 +19,35 @@
 
 using namespace qvg;
 
+namespace qvg {
+
+int device_sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int n = 148;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, size_t>> done;
+  std::lock_guard<std::mutex> g(mu);
+  for (auto& d : done)
+    if (d.first == kernel && d.second >= bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done.emplace_back(kernel, bytes);
+  return e;
+}
+
+}  // namespace qvg
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -34,7 +63,8 @@ struct Plan {
   int nR = 0;
   size_t off_R[2] = {0, 0};
   size_t off_rnorm = 0, off_cn = 0, off_list = 0, off_listcnt = 0;
-  size_t off_partial = 0, off_counts = 0, off_status = 0, total = 0;
+  size_t off_partial = 0, off_ncontrib = 0, off_dcount = 0, off_S = 0, off_n = 0, off_pi = 0;
+  size_t off_status = 0, total = 0;
 };
 
 Plan make_plan(const qvg_config& c, int64_t N, int W, int dtype) {
@@ -48,10 +78,14 @@ Plan make_plan(const qvg_config& c, int64_t N, int W, int dtype) {
   for (int b = 0; b < p.nR; ++b) { p.off_R[b] = o; o = align_up(o + (size_t)W * N * kD * esz); }
   p.off_rnorm = o;                        o = align_up(o + (size_t)W * N * sizeof(float));
   p.off_cn = o;                           o = align_up(o + (size_t)W * kMaxK * sizeof(float));
-  p.off_list = o;                         o = align_up(o + (size_t)W * N * sizeof(uint32_t));
+  p.off_list = o;                         o = align_up(o + (size_t)W * N * 8);
   p.off_listcnt = o;                      o = align_up(o + (size_t)W * sizeof(uint32_t));
   p.off_partial = o;                      o = align_up(o + (size_t)W * p.nseg * c.K * kD * sizeof(double));
-  p.off_counts = o;                       o = align_up(o + (size_t)W * p.nseg * c.K * sizeof(int));
+  p.off_ncontrib = o;                     o = align_up(o + (size_t)W * p.nseg * c.K * sizeof(int));
+  p.off_dcount = o;                       o = align_up(o + (size_t)W * p.nseg * c.K * sizeof(int));
+  p.off_S = o;                            o = align_up(o + (size_t)W * c.K * kD * sizeof(double));
+  p.off_n = o;                            o = align_up(o + (size_t)W * c.K * sizeof(long long));
+  p.off_pi = o;                           o = align_up(o + (size_t)W * N);
   p.total = o;
   return p;
 }
@@ -68,9 +102,10 @@ int preferred_batch(int64_t N, int H, int dtype) {
   return std::max(1, std::min(w, H));
 }
 
-// Relative error bound assumed for the tensor-core dot products of 128
-// bf16 x bf16 products accumulated in fp32 (2^-14, 128x the unit roundoff).
-constexpr float kTcGamma = 6.103515625e-05f;
+// Relative error bound assumed for the tensor-core sums (128 exact bf16 x bf16
+// products plus three bf16 pieces of -|c|^2/2, accumulated in fp32 over nine
+// MMA steps): 2^-16, about 7x a bound of two fp32 ulps per step.
+constexpr float kTcGamma = 1.52587890625e-05f;   // 2^-16
 
 // QVG_ASSIGN_PATH=exact routes bf16 blocks through the CUDA-core exact
 // assignment as well (diagnostics; the results are identical).
@@ -141,9 +176,14 @@ cudaError_t plaunch(Kind k, cudaStream_t s, F&& f) {
     a = pool_event(p);
     b = pool_event(p);
   }
-  cudaEventRecord(a, s);
+  // Inside a stream capture the events must be external record nodes to be
+  // timed when the graph replays.
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cs);
+  const unsigned flags = cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : 0u;
+  cudaEventRecordWithFlags(a, s, flags);
   const cudaError_t e = f();
-  cudaEventRecord(b, s);
+  cudaEventRecordWithFlags(b, s, flags);
   std::lock_guard<std::mutex> g(p.mu);
   p.kinds.push_back((int)k);
   p.ev.push_back(a);
@@ -224,7 +264,7 @@ qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, i
   char* ws = static_cast<char*>(workspace);
   float* rnorm = reinterpret_cast<float*>(ws + plan.off_rnorm);
   float* cn = reinterpret_cast<float*>(ws + plan.off_cn);
-  uint32_t* list = reinterpret_cast<uint32_t*>(ws + plan.off_list);
+  uint2* list = reinterpret_cast<uint2*>(ws + plan.off_list);
   uint32_t* list_count = reinterpret_cast<uint32_t*>(ws + plan.off_listcnt);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + plan.off_status);
   unsigned long long* flagged = reinterpret_cast<unsigned long long*>(ws + plan.off_status + 8);
@@ -260,28 +300,38 @@ qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, i
       } else {
         QVG_TRY(plaunch(K_INIT, s, [&] { return launch_init_centroids(Rin, N * kD, Ct, cn, w, c.K, dt, s); }));
       }
+      // The assignment of iteration `it` goes to pit or to the spare buffer, so
+      // that the last iteration's lands in pit and the previous one is kept
+      // for the incremental update.
+      uint8_t* spare = reinterpret_cast<uint8_t*>(ws + plan.off_pi);
       for (int it = 0; it < iters; ++it) {
+        uint8_t* pi_new = ((iters - 1 - it) % 2 == 0) ? pit : spare;
+        uint8_t* pi_old = it == 0 ? nullptr : (pi_new == pit ? spare : pit);
         AssignParams ap{};
-        ap.R = Rin; ap.rnorm2 = rnorm; ap.C = Ct; ap.cn = cn; ap.pi = pit;
+        ap.R = Rin; ap.rnorm2 = rnorm; ap.C = Ct; ap.cn = cn; ap.pi = pi_new;
         ap.list = nullptr; ap.list_count = nullptr; ap.N = N; ap.W = w; ap.K = c.K;
         if (use_tc) {
           // tensor-core screening; listed near-ties are decided exactly next
           QVG_TRY(cudaMemsetAsync(list_count, 0, (size_t)w * sizeof(uint32_t), s));
           AssignTcParams tp{};
-          tp.R = Rin; tp.rnorm2 = rnorm; tp.C = Ct; tp.cn = cn; tp.pi = pit; tp.list = list;
+          tp.R = Rin; tp.rnorm2 = rnorm; tp.C = Ct; tp.cn = cn; tp.pi = pi_new; tp.list = list;
           tp.list_count = list_count; tp.status = status; tp.flagged = flagged;
           tp.N = N; tp.W = w; tp.K = c.K; tp.gamma = kTcGamma;
           QVG_TRY(plaunch(K_ASSIGN_TC, s, [&] { return launch_assign_tc(tp, s); }));
-          ap.list = list; ap.list_count = list_count;
-          QVG_TRY(plaunch(K_RECHECK, s, [&] { return launch_assign_exact(ap, dt, s); }));
+          QVG_TRY(plaunch(K_RECHECK, s, [&] {
+            return launch_assign_candidates(Rin, Ct, c.K, N, w, list, list_count, pi_new, s);
+          }));
         } else {
           QVG_TRY(plaunch(K_ASSIGN_EXACT, s, [&] { return launch_assign_exact(ap, dt, s); }));
         }
         UpdateParams up{};
-        up.R = Rin; up.pi = pit; up.C = Ct; up.cn = cn; up.N = N; up.W = w; up.K = c.K;
-        up.nseg = plan.nseg;
+        up.R = Rin; up.pi = pi_new; up.pi_old = pi_old; up.C = Ct; up.cn = cn;
+        up.N = N; up.W = w; up.K = c.K; up.nseg = plan.nseg;
         up.partial = reinterpret_cast<double*>(ws + plan.off_partial);
-        up.counts = reinterpret_cast<int*>(ws + plan.off_counts);
+        up.ncontrib = reinterpret_cast<int*>(ws + plan.off_ncontrib);
+        up.dcount = reinterpret_cast<int*>(ws + plan.off_dcount);
+        up.S = reinterpret_cast<double*>(ws + plan.off_S);
+        up.n = reinterpret_cast<long long*>(ws + plan.off_n);
         QVG_TRY(plaunch(K_UPD_PARTIAL, s, [&] { return launch_update_partial(up, dt, s); }));
         QVG_TRY(plaunch(K_UPD_FINAL, s, [&] { return launch_update_finalize(up, dt, s); }));
       }
@@ -308,7 +358,7 @@ qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packed, qvg_d
       packed->zero == nullptr)
     return QVG_ERR_INVALID_ARG;
   if (cfg->T > 0 && (packed->assign == nullptr || packed->centroids == nullptr)) return QVG_ERR_INVALID_ARG;
-  if (!aligned(Y, 16) || !aligned(packed->centroids, 16) || !aligned(packed->codes, 2)) return QVG_ERR_INVALID_ARG;
+  if (!aligned(Y, 16) || !aligned(packed->centroids, 16) || !aligned(packed->codes, 16)) return QVG_ERR_INVALID_ARG;
   if (N == 0) return QVG_OK;
   const int dt = (int)dtype;
   const size_t table = (size_t)cfg->K * kD * esize(dt);

@@ -9,6 +9,13 @@
 
 namespace qvg {
 
+// ---- launch helpers (qvg_api.cu)
+// SM count of the current device (cached per device).
+int device_sm_count();
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` (the
+// attribute call is made once per kernel and size; later calls are cached).
+cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes);
+
 // ---- codec kernels (kernels_codec.cu)
 
 // Fused reconstruction of a set of (chunk, head) blocks.
@@ -67,7 +74,7 @@ struct AssignTcParams {
   const void* C;               // [W][K][d] bf16
   const float* cn;             // [W][K]
   uint8_t* pi;                 // [W][N]
-  uint32_t* list;              // [W][N]
+  uint2* list;                 // [W][N] listed tokens: {token, mask of candidate 32-centroid chunks}
   uint32_t* list_count;        // [W], zero on entry
   uint32_t* status;            // workspace status word
   unsigned long long* flagged; // running total of listed tokens
@@ -77,26 +84,39 @@ struct AssignTcParams {
   float gamma;
 };
 cudaError_t launch_assign_tc(const AssignTcParams& p, cudaStream_t s);
+// Exact decision of the listed tokens: sequential fp64 squared distances to
+// every centroid of the listed 32-centroid chunks (all chunks when the mask is
+// empty), the least one wins, ties to the lowest index.
+cudaError_t launch_assign_candidates(const void* R, const void* C, int K, int64_t N, int W,
+                                     const uint2* list, const uint32_t* list_count, uint8_t* pi,
+                                     cudaStream_t s);
 size_t assign_tc_smem_bytes(int K);
 
 constexpr int kSeg = 2048;   // tokens per update segment
 
 struct UpdateParams {
   const void* R;        // [W][N][d]
-  const uint8_t* pi;    // [W][N]
-  double* partial;      // [W][nseg][K][d]
-  int* counts;          // [W][nseg][K]
-  void* C;              // [W][K][d]  (updated in place)
+  const uint8_t* pi;    // [W][N] assignment of this iteration
+  const uint8_t* pi_old;// [W][N] assignment of the previous iteration, or nullptr (full sums)
+  double* partial;      // [W][nseg][K][d] per-segment sums of the contributions
+  int* ncontrib;        // [W][nseg][K]   contributions per segment (0 = partial not written)
+  int* dcount;          // [W][nseg][K]   change of the member count per segment
+  double* S;            // [W][K][d]      running fp64 sums of the members
+  long long* n;         // [W][K]         member counts
+  void* C;              // [W][K][d]      centroids (updated in place)
   float* cn;            // [W][K]
   int64_t N;
   int W;
   int K;
   int nseg;
 };
-// Per-segment fp64 cluster sums (tokens ascending) ...
+// Per-segment fp64 sums of the contributions of the segment's tokens in
+// centroid order (stable counting sort): with pi_old == nullptr every token
+// adds its row to its centroid; otherwise a token whose centroid changed adds
+// its row to the new centroid and subtracts it from the old one.
 cudaError_t launch_update_partial(const UpdateParams& p, int dtype, cudaStream_t s);
-// ... then a fixed-order reduction over segments, mean, one rounding to the
-// storage dtype.
+// Running sums S += segment sums (segments in order), counts n += changes,
+// then every non-empty centroid = round(S / n) in the storage dtype.
 cudaError_t launch_update_finalize(const UpdateParams& p, int dtype, cudaStream_t s);
 
 }  // namespace qvg

@@ -141,7 +141,8 @@ QVG_API qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype 
                         const qvg_packed* out, void* workspace, size_t ws_bytes,
                         qvg_stream_t stream);
 
-/* Reconstruct Y[H][N][d] (DEVICE, `dtype`) from `packed` in one fused kernel:
+/* Reconstruct Y[H][N][d] (DEVICE, `dtype`, 16-byte aligned) from `packed`
+ * (codes and centroids 16-byte aligned) in one fused kernel:
  * y = s*q + m, then + C(T)[pi_T], + C(T-1)[pi_(T-1)], ..., + C(1)[pi_1], each
  * an fp32 add in that order, then one rounding to `dtype`.  Assignment
  * values >= K are clamped to K-1.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
