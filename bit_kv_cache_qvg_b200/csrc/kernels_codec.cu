@@ -64,6 +64,53 @@ template <> struct Vec8<kFP32> {
   __device__ static __forceinline__ void round(float (&)[8]) {}
 };
 
+// ---------------------------------------------------------------- packed pairs
+// Two fp32 values in one 64-bit register, operated on with the f32x2
+// instructions (each lane of the pair rounded as a separate fp32 operation).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  return ((uint64_t)__float_as_uint(hi) << 32) | (uint64_t)__float_as_uint(lo);
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+template <int DT> struct Pair4;
+template <> struct Pair4<kBF16> {
+  // y[e] += channels (2e, 2e+1) of 8 bf16 centroid values
+  __device__ static __forceinline__ void add(const void* p, uint64_t (&y)[4]) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] = add2(y[e], ((uint64_t)(x[e] & 0xFFFF0000u) << 32) | (uint64_t)(x[e] << 16));
+  }
+  __device__ static __forceinline__ void store(void* p, const uint64_t (&y)[4]) {
+    uint32_t x[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float((uint32_t)y[e]), __uint_as_float((uint32_t)(y[e] >> 32)));
+      x[e] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(x[0], x[1], x[2], x[3]);
+  }
+};
+template <> struct Pair4<kFP32> {
+  __device__ static __forceinline__ void add(const void* p, uint64_t (&y)[4]) {
+    const ulonglong2 a = reinterpret_cast<const ulonglong2*>(p)[0];
+    const ulonglong2 b = reinterpret_cast<const ulonglong2*>(p)[1];
+    y[0] = add2(y[0], a.x); y[1] = add2(y[1], a.y); y[2] = add2(y[2], b.x); y[3] = add2(y[3], b.y);
+  }
+  __device__ static __forceinline__ void store(void* p, const uint64_t (&y)[4]) {
+    reinterpret_cast<ulonglong2*>(p)[0] = make_ulonglong2(y[0], y[1]);
+    reinterpret_cast<ulonglong2*>(p)[1] = make_ulonglong2(y[2], y[3]);
+  }
+};
+
 // ---------------------------------------------------------------- dequant
 constexpr int kDqThreads = 512;
 constexpr int kDqTokPerIter = kDqThreads / 8;   // 64 tokens per block row of threads
@@ -108,6 +155,12 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
   const size_t tab_bytes = (size_t)tab_elems * ESZ;
   const char* tables = static_cast<const char*>(p.centroids) + (int64_t)c * T * p.H * tab_elems * ESZ;
   uint8_t* cring = smem + (size_t)p.t_smem * tab_bytes;       // codes ring (16-byte aligned)
+  // byte of four 2-bit codes -> the four codes as floats (channel order)
+  float4* qlut = reinterpret_cast<float4*>(cring + kDqStages * kDqTileBytes);
+  if (threadIdx.x < 256) {
+    const uint32_t b = threadIdx.x;
+    qlut[b] = make_float4((float)(b & 3u), (float)((b >> 2) & 3u), (float)((b >> 4) & 3u), (float)(b >> 6));
+  }
 
   const int j = threadIdx.x & 7;
   const int tl = threadIdx.x >> 3;
@@ -179,12 +232,17 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
       const uint32_t q1 = *reinterpret_cast<const uint16_t*>(ct + r * (kD / 4) + 16 + 2 * j);
       const float s0 = e4m3_to_f32((uint8_t)(sz[u] & 0xFF)), m0 = e4m3_to_f32((uint8_t)((sz[u] >> 8) & 0xFF));
       const float s1 = e4m3_to_f32((uint8_t)((sz[u] >> 16) & 0xFF)), m1 = e4m3_to_f32((uint8_t)(sz[u] >> 24));
-      float y0[8], y1[8];
+      // y = s*q + m (exact in fp32: E4M3 operands, q <= 3), two channels per op
+      uint64_t y0[4], y1[4];
+      const uint64_t s0p = pack2(s0, s0), m0p = pack2(m0, m0), s1p = pack2(s1, s1), m1p = pack2(m1, m1);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        // s*q + m is exact in fp32 (E4M3 operands, q <= 3)
-        y0[e] = __fmaf_rn(s0, (float)((q0 >> (2 * e)) & 3u), m0);
-        y1[e] = __fmaf_rn(s1, (float)((q1 >> (2 * e)) & 3u), m1);
+      for (int bq = 0; bq < 2; ++bq) {
+        const float4 a = qlut[(q0 >> (8 * bq)) & 0xFFu];
+        const float4 b = qlut[(q1 >> (8 * bq)) & 0xFFu];
+        y0[2 * bq] = fma2(s0p, pack2(a.x, a.y), m0p);
+        y0[2 * bq + 1] = fma2(s0p, pack2(a.z, a.w), m0p);
+        y1[2 * bq] = fma2(s1p, pack2(b.x, b.y), m1p);
+        y1[2 * bq + 1] = fma2(s1p, pack2(b.z, b.w), m1p);
       }
       const int64_t ii = tok < i_end ? tok : i_begin;
       // centroids of stage T, T-1, ..., 1, in that order
@@ -197,19 +255,13 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
         const char* rowp = (st < p.t_smem)
             ? reinterpret_cast<const char*>(smem) + ((int64_t)st * tab_elems + (int64_t)k * kD) * ESZ
             : tables + (((int64_t)st * p.H + h) * tab_elems + (int64_t)k * kD) * ESZ;
-        float c0[8], c1[8];
-        Vec8<DT>::load(rowp + 8 * j * ESZ, c0);
-        Vec8<DT>::load(rowp + (64 + 8 * j) * ESZ, c1);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          y0[e] = __fadd_rn(y0[e], c0[e]);
-          y1[e] = __fadd_rn(y1[e], c1[e]);
-        }
+        Pair4<DT>::add(rowp + 8 * j * ESZ, y0);
+        Pair4<DT>::add(rowp + (64 + 8 * j) * ESZ, y1);
       }
       if (tok < i_end) {
         char* yr = Y + tok * kD * ESZ;
-        Vec8<DT>::store(yr + 8 * j * ESZ, y0);
-        Vec8<DT>::store(yr + (64 + 8 * j) * ESZ, y1);
+        Pair4<DT>::store(yr + 8 * j * ESZ, y0);
+        Pair4<DT>::store(yr + (64 + 8 * j) * ESZ, y1);
       }
     }
 #pragma unroll
@@ -237,7 +289,11 @@ __device__ __forceinline__ float grp_max(float v, int G) {
 }
 
 // Quantise one 8-channel chunk given its group's (lo, hi); returns the 16-bit
-// packed codes and the scale/zero bytes.
+// packed codes and the scale/zero bytes.  q = clamp(rint(fl((r - m) / s)), 0, 3)
+// with IEEE rounding of the divide: the quotient is first formed as
+// (r - m) * (1/s), which is within 3 ulp of fl((r - m) / s); only when it lies
+// within 2^-19 of 0.5, 1.5 or 2.5 (the only boundaries that change a clamped
+// code) is the correctly rounded divide evaluated.
 __device__ __forceinline__ uint32_t quant_chunk(const float (&r)[8], float lo, float hi,
                                                 uint8_t& sc_out, uint8_t& zc_out) {
   lo = __fadd_rn(lo, 0.0f);             // -0 -> +0
@@ -249,9 +305,24 @@ __device__ __forceinline__ uint32_t quant_chunk(const float (&r)[8], float lo, f
   const float s = e4m3_to_f32(scb);
   uint32_t packed = 0;
   if (s != 0.0f) {
+    const float inv = __frcp_rn(s);
+    float d[8], t[8];
+    uint32_t near = 0;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      int q = __float2int_rn(__fdiv_rn(__fsub_rn(r[e], m), s));
+      d[e] = __fsub_rn(r[e], m);
+      t[e] = __fmul_rn(d[e], inv);
+      const float fl = floorf(t[e]);
+      if (fl >= 0.0f && fl <= 2.0f && fabsf(__fsub_rn(t[e], fl) - 0.5f) < 1.9073486328125e-06f) near |= 1u << e;
+    }
+    if (near) {                          // rare: quotients next to a rounding boundary
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if ((near >> e) & 1u) t[e] = __fdiv_rn(d[e], s);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      int q = __float2int_rn(t[e]);
       q = q < 0 ? 0 : (q > 3 ? 3 : q);
       packed |= (uint32_t)q << (2 * e);
     }
@@ -416,7 +487,7 @@ static cudaError_t launch_dq_t(const DequantParams& p, int blocks, int splits, s
 
 cudaError_t launch_dequant(const DequantParams& p, int dtype, cudaStream_t s) {
   const int esz = dtype == kBF16 ? 2 : 4;
-  const size_t smem = (size_t)p.t_smem * p.K * kD * esz + (size_t)kDqStages * kDqTileBytes;
+  const size_t smem = (size_t)p.t_smem * p.K * kD * esz + (size_t)kDqStages * kDqTileBytes + 256 * 16;
   const int units = p.n_chunks * p.H;
   if (units == 0) return cudaSuccess;
   const int sms = device_sm_count();

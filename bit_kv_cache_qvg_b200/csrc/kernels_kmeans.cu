@@ -240,7 +240,7 @@ constexpr int kUpThreads = 512;
 constexpr int kUpWarps = kUpThreads / 32;
 constexpr int kTokPerWarp = kSeg / kUpWarps;      // 128
 constexpr int kRounds = kTokPerWarp / 32;         // 4
-constexpr int kBatch = 16;                        // rows in flight per warp
+constexpr int kBatch = 8;                         // rows in flight per warp
 
 // Exact widening of a bf16 / fp32 value to fp64 with integer operations (the
 // exponent is rebiased, the significand shifted); zero, subnormal, infinite
@@ -293,7 +293,7 @@ __device__ __forceinline__ void load4(const char* row, int lane, float (&v)[4]) 
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kUpThreads)
+__global__ void __launch_bounds__(kUpThreads, 2)
 qvg_update_partial(const UpdateParams p) {
   constexpr int ESZ = Store<DT>::bytes;
   constexpr int kMaxC = 2 * kSeg;                  // contributions per segment
@@ -320,6 +320,15 @@ qvg_update_partial(const UpdateParams p) {
   // 1. Stable per-warp ranks of the contributions.  Warp w owns tokens
   //    [w*128, w*128+128); its contributions are taken in a fixed order:
   //    pass 0 = subtractions (old centroid), pass 1 = additions (new centroid).
+  // the warp's 128 assignments (and the previous ones), loaded up front:
+  // round r of lane l is token w*128 + r*32 + l
+  uint8_t an[kRounds], ao[kRounds];
+#pragma unroll
+  for (int r = 0; r < kRounds; ++r) {
+    const int tok = warp * kTokPerWarp + r * 32 + lane;
+    an[r] = tok < seg_len ? pn[tok] : 0;
+    ao[r] = (po != nullptr && tok < seg_len) ? po[tok] : 0;
+  }
   int key[2][kRounds], rank[2][kRounds];
 #pragma unroll
   for (int ps = 0; ps < 2; ++ps) {
@@ -329,10 +338,10 @@ qvg_update_partial(const UpdateParams p) {
       bool valid = tok < seg_len;
       int k = 0;
       if (valid) {
-        const int kn = pn[tok];
+        const int kn = an[r];
         if (po == nullptr) { valid = ps == 1; k = kn; }
         else {
-          const int ko = po[tok];
+          const int ko = ao[r];
           valid = ko != kn;
           k = ps == 0 ? ko : kn;
         }

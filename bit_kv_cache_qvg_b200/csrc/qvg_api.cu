@@ -90,22 +90,23 @@ Plan make_plan(const qvg_config& c, int64_t N, int W, int dtype) {
   return p;
 }
 
-int preferred_batch(int64_t N, int H, int dtype) {
+int preferred_batch(const qvg_config& c, int64_t N, int H, int dtype) {
   if (const char* env = std::getenv("QVG_BATCH_UNITS")) {
     const int w = std::atoi(env);
     if (w > 0) return std::min(w, H);
   }
-  // Keep the stage inputs of one batch within about 48 MB so that the
-  // repeated passes of the Lloyd iterations are served from L2.
-  const double budget = 48.0 * 1024.0 * 1024.0;
-  int w = (int)std::floor(budget / ((double)N * kD * esize(dtype)));
-  return std::max(1, std::min(w, H));
+  // As many blocks per launch as a 2 GiB workspace holds (at most 128): wide
+  // launches keep every SM busy and amortise the per-launch pipeline fill.
+  const double budget = 2.0 * 1024.0 * 1024.0 * 1024.0;
+  const double per_unit = (double)make_plan(c, N, 1, dtype).total;
+  int w = (int)std::floor(budget / per_unit);
+  return std::max(1, std::min(std::min(w, 128), H));
 }
 
 // Relative error bound assumed for the tensor-core sums (128 exact bf16 x bf16
 // products plus three bf16 pieces of -|c|^2/2, accumulated in fp32 over nine
 // MMA steps): 2^-16, about 7x a bound of two fp32 ulps per step.
-constexpr float kTcGamma = 1.52587890625e-05f;   // 2^-16
+constexpr float kTcGamma = 1.52587890625e-05f;
 
 // QVG_ASSIGN_PATH=exact routes bf16 blocks through the CUDA-core exact
 // assignment as well (diagnostics; the results are identical).
@@ -232,7 +233,7 @@ size_t qvg_packed_bytes(const qvg_config* c, int64_t N, int32_t H, int32_t d, qv
 
 size_t qvg_workspace_bytes(const qvg_config* c, int64_t N, int32_t H, int32_t d, qvg_dtype dtype) {
   if (check_config(c, N, H, d, dtype) != QVG_OK || N < 1) return 0;
-  return make_plan(*c, N, preferred_batch(N, H, dtype), dtype).total;
+  return make_plan(*c, N, preferred_batch(*c, N, H, dtype), dtype).total;
 }
 
 qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, int64_t N,
@@ -256,7 +257,7 @@ qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, i
   const int dt = (int)dtype;
   const size_t esz = (size_t)esize(dt);
 
-  int W = preferred_batch(N, H, dt);
+  int W = preferred_batch(c, N, H, dt);
   Plan plan = make_plan(c, N, W, dt);
   while (plan.total > ws_bytes && W > 1) plan = make_plan(c, N, --W, dt);
   if (plan.total > ws_bytes) return QVG_ERR_WORKSPACE_TOO_SMALL;
