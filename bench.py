@@ -52,6 +52,28 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, source="fallback")
 
 
+def load_traffic():
+    """DRAM bytes per launch from the committed ncu table (profiles/dram_traffic.md):
+    {kernel: (bytes, blocks_per_launch)} for rows whose source hash still matches."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    out = {}
+    if not os.path.exists(path):
+        return out
+    for line in open(path):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) < 6 or not cells[0].startswith("qvg_"):
+            continue
+        name, src, digest, blocks, nbytes = cells[:5]
+        try:
+            cur = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:16]
+            if cur == digest:
+                out[name] = (float(nbytes), float(blocks))
+        except (OSError, ValueError):
+            pass
+    return out
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -279,13 +301,22 @@ def main():
     esz = 2
     deq_bytes_per_elem = 2 / 8 + 2 / G + T / 128 + esz * T * K / N + 2
     roof = {}
+    traffic = load_traffic()
+
+    def traffic_for(name, blocks_per_launch):
+        if name not in traffic:
+            return None
+        nbytes, blocks = traffic[name]
+        return nbytes * blocks_per_launch / blocks
+
     if "qvg_dequant_fused" in kernels and kernels["qvg_dequant_fused"]["ms"] > 0:
         k = kernels["qvg_dequant_fused"]
         t_launch = k["ms"] / max(k["timed"], 1) / 1e3
         per_launch = deq_bytes_per_elem * E
         roof["qvg_dequant_fused"] = {"bound": "hbm", "achieved": per_launch / t_launch / 1e9,
                                      "peak": peaks["hbm"], "unit": "GB/s",
-                                     "frac": per_launch / t_launch / 1e9 / peaks["hbm"], "traffic": None,
+                                     "frac": per_launch / t_launch / 1e9 / peaks["hbm"],
+                                     "traffic": traffic_for("qvg_dequant_fused", U / k["timed"]),
                                      "alg_bytes_per_launch": per_launch}
     for name in ("qvg_kmeans_assign", "qvg_assign_exact"):
         if name in kernels and kernels[name]["timed"] and kernels[name]["ms"] > 0:
@@ -296,7 +327,8 @@ def main():
             t_launch = k["ms"] / k["timed"] / 1e3
             ach = per_launch / t_launch / 1e12
             roof[name] = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
-                          "frac": ach / peaks["bf16_sus"], "traffic": None,
+                          "frac": ach / peaks["bf16_sus"],
+                          "traffic": traffic_for(name, U * T * I / k["timed"]),
                           "alg_flops_per_launch": per_launch}
     top = max(kernels.items(), key=lambda kv: kv[1]["ms"])[0] if kernels else None
     dominant = roof.get(top) if top in roof else (next(iter(roof.values())) if roof else None)
