@@ -1,0 +1,73 @@
+// qvg_static_scratch.cu -- qvg_quantize_static: the compression call of
+// qvg_quantize, run on a scratch area that the library reserves once per
+// device in a static __device__ array, so that the call allocates nothing.
+//
+// Who needs it: a caller that must not touch the CUDA allocator while it
+// runs, and has no workspace of its own to lend.  A cudaMalloc or cudaFree
+// can synchronise the whole device, stalling every stream of the process.
+// It can fail under memory pressure in the middle of a generation.  And a
+// caching allocator elsewhere in the process may already hold the free
+// memory that a raw allocation would need.  Such a caller (for example a
+// per-chunk hook of a decoding loop) can call this entry with device
+// buffers it already owns for the input and the outputs, and nothing else.
+//
+// The reserve is kStaticScratchBytes (32 MiB) of global memory.  It holds
+// the k-means working set of as many blocks per wave as fit, and at least
+// one: about 80,000 tokens per block at bf16, K = 256, T = 2.  A call whose
+// single block needs more is rejected before any work is queued.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "qvg.h"
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+constexpr int kMaxDevices = 64;
+
+// One reserve per device (a __device__ variable has one instance per device
+// on which the library's device code is loaded).  256-byte alignment is the
+// alignment qvg_quantize requires of a workspace.
+__device__ __align__(256) unsigned char g_qvg_static_scratch[kStaticScratchBytes];
+
+std::mutex g_setup_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the reserve on the current device, looked up once per
+// device (the lookup may load this file's device code on first use).
+qvg_status scratch_on_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QVG_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return QVG_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_qvg_static_scratch) != cudaSuccess || p == nullptr) return QVG_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return QVG_OK;
+}
+
+}  // namespace
+
+extern "C" QVG_API qvg_status qvg_quantize_static(const qvg_config* cfg, const void* X, qvg_dtype dtype,
+                                                  int64_t N, int32_t H, int32_t d,
+                                                  const void* init_centroids, const qvg_packed* out,
+                                                  qvg_stream_t stream) {
+  // One block's working set must fit in the reserve (a zero size means the
+  // arguments are invalid; qvg_quantize then reports which).
+  const size_t one_block = qvg_workspace_bytes(cfg, N, 1, d, dtype);
+  if (one_block > kStaticScratchBytes) return QVG_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  const qvg_status st = scratch_on_current_device(&scratch);
+  if (st != QVG_OK) return st;
+  // The workspace contract: the 16-byte status word and near-tie counter at
+  // the start must read zero when the work begins.  Nothing else in the
+  // scratch needs initialising (every other region is written before read).
+  if (cudaMemsetAsync(scratch, 0, 16, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return QVG_ERR_CUDA;
+  return qvg_quantize(cfg, X, dtype, N, H, d, init_centroids, out, scratch, kStaticScratchBytes, stream);
+}

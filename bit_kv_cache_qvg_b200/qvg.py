@@ -57,6 +57,8 @@ _SIGS = {
     "qvg_workspace_bytes": (C.c_size_t, [C.POINTER(Config), C.c_int64, C.c_int32, C.c_int32, C.c_int]),
     "qvg_quantize": (C.c_int, [C.POINTER(Config), C.c_void_p, C.c_int, C.c_int64, C.c_int32, C.c_int32,
                                C.c_void_p, C.POINTER(_Packed), C.c_void_p, C.c_size_t, C.c_void_p]),
+    "qvg_quantize_static": (C.c_int, [C.POINTER(Config), C.c_void_p, C.c_int, C.c_int64, C.c_int32,
+                                      C.c_int32, C.c_void_p, C.POINTER(_Packed), C.c_void_p]),
     "qvg_dequantize": (C.c_int, [C.POINTER(Config), C.POINTER(_Packed), C.c_int, C.c_int64, C.c_int32,
                                  C.c_int32, C.c_void_p, C.c_void_p]),
     "qvg_workspace_status": (C.c_int, [C.c_void_p, C.c_size_t, C.c_void_p]),
@@ -190,6 +192,22 @@ def quantize(X: torch.Tensor, cfg: Config, init: Optional[torch.Tensor] = None,
     st = lib().qvg_quantize(C.byref(cfg), _ptr(X), dt, N, H, d, _ptr(init), C.byref(ps),
                             _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "qvg_quantize")
+    return out
+
+
+def quantize_static(X: torch.Tensor, cfg: Config, init: Optional[torch.Tensor] = None,
+                    out: Optional[Packed] = None, stream=None) -> Packed:
+    """qvg_quantize_static on X [H][N][d]: no workspace argument; the library's
+    per-device static reserve is the scratch (calls must not overlap)."""
+    if X.dim() != 3 or not X.is_contiguous():
+        raise QvgError(1, "X must be a contiguous [H][N][d] tensor")
+    H, N, d = X.shape
+    dt = _DTYPES[X.dtype]
+    if out is None:
+        out = alloc_packed(cfg, N, H, d, dt, X.device)
+    ps = out.struct()
+    st = lib().qvg_quantize_static(C.byref(cfg), _ptr(X), dt, N, H, d, _ptr(init), C.byref(ps), _stream(stream))
+    _check(st, "qvg_quantize_static")
     return out
 
 

@@ -161,6 +161,34 @@ QVG_API qvg_status qvg_workspace_status(void* workspace, size_t ws_bytes, qvg_st
  * No counterpart in the method: a diagnostic of the assignment kernels. */
 QVG_API int64_t qvg_workspace_flagged(void* workspace, size_t ws_bytes, qvg_stream_t stream);
 
+/* qvg_quantize without a caller workspace and without any allocation.
+ * The method has no counterpart of this call: it is a library-usage variant
+ * for callers that must not allocate device memory while they run (a
+ * cudaMalloc/cudaFree can synchronise the device and stall every stream,
+ * can fail under memory pressure mid-generation, or can find the memory
+ * held by another allocator in the process) and have no workspace to lend.
+ * The scratch is a 32 MiB reserve in a static __device__ array, one per
+ * device, whose address is looked up on the first call on each device.
+ * That first call may load the library's device code, so make it before
+ * any stream capture begins.
+ * Arguments, layouts, results and errors are those of qvg_quantize, less
+ * the workspace; each call first zeroes the reserve's 16-byte status word
+ * and near-tie counter (on `stream`), then queues the same kernels.
+ * Limits: the reserve must hold one block's working set, about 80,000
+ * tokens per block at bf16 with K = 256, T = 2 (qvg_workspace_bytes with
+ * H = 1 gives the exact need); a larger block returns WORKSPACE_TOO_SMALL
+ * before anything is queued.  Blocks beyond what one wave holds run in
+ * further waves, as in qvg_quantize.
+ * Concurrency: every call on a device uses the same reserve, so two calls
+ * whose work can overlap on the device (different streams, or threads
+ * without ordering between them) race and corrupt each other's results;
+ * order them on one stream, or use qvg_quantize with separate workspaces.
+ * A device-side timeout of this path is recorded in the reserve only; it is
+ * not reported to the caller. */
+QVG_API qvg_status qvg_quantize_static(const qvg_config* cfg, const void* X, qvg_dtype dtype,
+                               int64_t N, int32_t H, int32_t d, const void* init_centroids,
+                               const qvg_packed* out, qvg_stream_t stream);
+
 /* ------------------------------------------------------------------ */
 /* Diagnostics (no counterpart in the method; used by the benchmark).    */
 /* ------------------------------------------------------------------ */
