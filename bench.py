@@ -330,10 +330,9 @@ def main():
                           "frac": ach / peaks["bf16_sus"],
                           "traffic": traffic_for(name, U * T * I / k["timed"]),
                           "alg_flops_per_launch": per_launch}
-    top = max(kernels.items(), key=lambda kv: kv[1]["ms"])[0] if kernels else None
-    dominant = roof.get(top) if top in roof else (next(iter(roof.values())) if roof else None)
-    if dominant is not None:
-        dominant = dict(dominant, kernel=top if top in roof else next(iter(roof)))
+    # the dominant kernel: the one with a roofline that takes the most time
+    top = max(roof, key=lambda n: kernels[n]["ms"]) if roof else None
+    dominant = dict(roof[top], kernel=top) if top else None
 
     # quantise-path roofline: max(F / P_bf16, B / BW)
     q_ms = sum(v["ms"] for n, v in kernels.items() if n != "qvg_dequant_fused")

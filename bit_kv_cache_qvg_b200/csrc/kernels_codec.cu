@@ -43,10 +43,16 @@ template <> struct Vec8<kBF16> {
     }
     *reinterpret_cast<uint4*>(p) = make_uint4(x[0], x[1], x[2], x[3]);
   }
-  // Round to bf16 and return the rounded values as fp32.
+  // Round to bf16 (nearest even, two values per conversion) and return the
+  // rounded values as fp32.
   __device__ static __forceinline__ void round(float (&v)[8]) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+      const uint32_t x = *reinterpret_cast<const uint32_t*>(&b);
+      v[2 * e] = __uint_as_float(x << 16);
+      v[2 * e + 1] = __uint_as_float(x & 0xFFFF0000u);
+    }
   }
 };
 
@@ -288,48 +294,64 @@ __device__ __forceinline__ float grp_max(float v, int G) {
   return v;
 }
 
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// min and max of 8 values
+__device__ __forceinline__ void minmax8(const float (&r)[8], float& lo, float& hi) {
+  lo = min3f(min3f(r[0], r[1], r[2]), min3f(r[3], r[4], r[5]), fminf(r[6], r[7]));
+  hi = max3f(max3f(r[0], r[1], r[2]), max3f(r[3], r[4], r[5]), fmaxf(r[6], r[7]));
+}
+
 // Quantise one 8-channel chunk given its group's (lo, hi); returns the 16-bit
 // packed codes and the scale/zero bytes.  q = clamp(rint(fl((r - m) / s)), 0, 3)
-// with IEEE rounding of the divide: the quotient is first formed as
-// (r - m) * (1/s), which is within 3 ulp of fl((r - m) / s); only when it lies
-// within 2^-19 of 0.5, 1.5 or 2.5 (the only boundaries that change a clamped
-// code) is the correctly rounded divide evaluated.
+// with IEEE rounding of the divide.  The quotient is first formed as
+// (r - m) * (1/s), within 3 ulp of fl((r - m) / s).  Clamping to [0, 3]
+// before rounding gives the same code (the boundaries -0.5 and 3.5 clamp to
+// the same code on both sides), and rounding to nearest even is an add and a
+// subtract of 1.5 * 2^23.  Only a clamped quotient that lies within 2^-19 of
+// 0.5, 1.5 or 2.5 can round differently from the exact one; a chunk holding
+// such a value is redone with the correctly rounded divide.  The codes are
+// packed with fused multiply-adds by 4^e, exact in fp32.
 __device__ __forceinline__ uint32_t quant_chunk(const float (&r)[8], float lo, float hi,
                                                 uint8_t& sc_out, uint8_t& zc_out) {
-  lo = __fadd_rn(lo, 0.0f);             // -0 -> +0
+  constexpr float kRound = 12582912.0f;     // 1.5 * 2^23
+  constexpr float kNear = 0.5f - 1.9073486328125e-06f;
+  lo = __fadd_rn(lo, 0.0f);                 // -0 -> +0
   hi = __fadd_rn(hi, 0.0f);
   const uint8_t zc = f32_to_e4m3(lo);
   const float m = e4m3_to_f32(zc);
   const float span = __fsub_rn(hi, m);
   const uint8_t scb = f32_to_e4m3(__fdiv_rn(span, 3.0f));
   const float s = e4m3_to_f32(scb);
-  uint32_t packed = 0;
-  if (s != 0.0f) {
-    const float inv = __frcp_rn(s);
-    float d[8], t[8];
-    uint32_t near = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      d[e] = __fsub_rn(r[e], m);
-      t[e] = __fmul_rn(d[e], inv);
-      const float fl = floorf(t[e]);
-      if (fl >= 0.0f && fl <= 2.0f && fabsf(__fsub_rn(t[e], fl) - 0.5f) < 1.9073486328125e-06f) near |= 1u << e;
-    }
-    if (near) {                          // rare: quotients next to a rounding boundary
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if ((near >> e) & 1u) t[e] = __fdiv_rn(d[e], s);
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      int q = __float2int_rn(t[e]);
-      q = q < 0 ? 0 : (q > 3 ? 3 : q);
-      packed |= (uint32_t)q << (2 * e);
-    }
-  }
   sc_out = scb;
   zc_out = zc;
-  return packed;
+  if (s == 0.0f) return 0u;
+  const float inv = __frcp_rn(s);
+  float pk = 0.0f, dev = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float t = fminf(fmaxf(__fmul_rn(__fsub_rn(r[e], m), inv), 0.0f), 3.0f);
+    const float q = __fsub_rn(__fadd_rn(t, kRound), kRound);
+    dev = fmaxf(dev, fabsf(__fsub_rn(t, q)));
+    pk = __fmaf_rn(q, (float)(1 << (2 * e)), pk);
+  }
+  if (dev > kNear) {                        // rare: a quotient next to a rounding boundary
+    pk = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float t = fminf(fmaxf(__fdiv_rn(__fsub_rn(r[e], m), s), 0.0f), 3.0f);
+      pk = __fmaf_rn(__fsub_rn(__fadd_rn(t, kRound), kRound), (float)(1 << (2 * e)), pk);
+    }
+  }
+  return __float_as_uint(__fadd_rn(pk, 8388608.0f)) & 0xFFFFu;   // 2^23: integer in the low bits
 }
 
 template <int DT, bool QUANT, bool HAS_C>
@@ -347,6 +369,17 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
     for (int x = threadIdx.x; x < n16; x += blockDim.x) dst[x] = src[x];
     __syncthreads();
   }
+  // largest |value| per channel of the values this pass hands to the next
+  // k-means (fixed-point scale of the centroid sums), when asked for
+  __shared__ uint32_t s_chmax[kD];
+  const bool want_max = !QUANT && p.chmax != nullptr;
+  if (want_max) {
+    for (int x = threadIdx.x; x < kD; x += blockDim.x) s_chmax[x] = 0u;
+    __syncthreads();
+  }
+  float mx0[8], mx1[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) { mx0[e] = 0.0f; mx1[e] = 0.0f; }
   const int j = threadIdx.x & 7;
   const int ng = kD / p.G;
   const int G = p.G;
@@ -393,13 +426,17 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
       s2 += __shfl_xor_sync(0xffffffffu, s2, 2);
       s2 += __shfl_xor_sync(0xffffffffu, s2, 4);
       if (valid && j == 0 && p.rnorm2 != nullptr) p.rnorm2[(int64_t)u * p.N + i] = s2;
-    } else {
-      float lo0 = r0[0], hi0 = r0[0], lo1 = r1[0], hi1 = r1[0];
+      if (want_max) {
 #pragma unroll
-      for (int e = 1; e < 8; ++e) {
-        lo0 = fminf(lo0, r0[e]); hi0 = fmaxf(hi0, r0[e]);
-        lo1 = fminf(lo1, r1[e]); hi1 = fmaxf(hi1, r1[e]);
+        for (int e = 0; e < 8; ++e) {
+          mx0[e] = fmaxf(mx0[e], fabsf(r0[e]));
+          mx1[e] = fmaxf(mx1[e], fabsf(r1[e]));
+        }
       }
+    } else {
+      float lo0, hi0, lo1, hi1;
+      minmax8(r0, lo0, hi0);
+      minmax8(r1, lo1, hi1);
       if (G == 128) {
         lo0 = lo1 = fminf(lo0, lo1);
         hi0 = hi1 = fmaxf(hi0, hi1);
@@ -424,6 +461,27 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
         p.zero[row * ng + (64 + 8 * j) / G] = z1;
       }
     }
+  }
+  if (want_max) {
+    // lanes j, j+8, j+16, j+24 hold the same channels (invalid lanes repeat a
+    // valid token, so they never raise a maximum)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      mx0[e] = fmaxf(mx0[e], __shfl_xor_sync(0xffffffffu, mx0[e], 8));
+      mx0[e] = fmaxf(mx0[e], __shfl_xor_sync(0xffffffffu, mx0[e], 16));
+      mx1[e] = fmaxf(mx1[e], __shfl_xor_sync(0xffffffffu, mx1[e], 8));
+      mx1[e] = fmaxf(mx1[e], __shfl_xor_sync(0xffffffffu, mx1[e], 16));
+    }
+    if ((threadIdx.x & 31) < 8) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        atomicMax(&s_chmax[8 * j + e], __float_as_uint(mx0[e]));
+        atomicMax(&s_chmax[64 + 8 * j + e], __float_as_uint(mx1[e]));
+      }
+    }
+    __syncthreads();
+    for (int x = threadIdx.x; x < kD; x += blockDim.x)
+      if (s_chmax[x] != 0u) atomicMax(&p.chmax[(int64_t)u * kD + x], s_chmax[x]);
   }
 }
 
@@ -519,8 +577,9 @@ cudaError_t launch_residual(const ResidualParams& p, int dtype, bool quant, cuda
   const bool has_c = p.C != nullptr;
   const size_t smem = has_c ? (size_t)p.K * kD * esz : 0;
   const int sms = device_sm_count();
-  // Enough blocks for two waves over the SMs; each block stages the table once.
-  int64_t splits = (2 * (int64_t)sms + p.W - 1) / p.W;
+  // About eight blocks per SM (four waves at two resident blocks per SM), so
+  // that the last wave is short; each block stages the table once.
+  int64_t splits = (8 * (int64_t)sms + p.W - 1) / p.W;
   const int64_t min_tok = 256;
   if (splits * min_tok > p.N) splits = (p.N + min_tok - 1) / min_tok;
   if (splits < 1) splits = 1;

@@ -7,12 +7,11 @@
 //     ascending order, separate subtract / multiply / add) for every centroid
 //     whose screening value lies within the rounding-error bound of the
 //     minimum; ties go to the lowest index.
-//   * qvg_kmeans_update: per 2048-token segment a stable counting sort of the
-//     tokens by centroid, fp64 sums of each centroid's tokens in ascending
-//     order, then a fixed-order reduction over segments, the mean (one fp64
-//     divide) and one rounding to the storage dtype; an empty centroid keeps
-//     its value.  The reduction order never depends on scheduling, so the
-//     result is deterministic.
+//   * qvg_kmeans_update: exact centroid sums in 64-bit fixed point (so the
+//     order of the adds cannot change them), the mean (one fp64 divide) and
+//     one rounding to the storage dtype; an empty centroid keeps its value.
+//     After the first iteration only the tokens whose assignment changed are
+//     read.
 #include "qvg_common.cuh"
 #include "qvg_launch.h"
 
@@ -236,336 +235,304 @@ qvg_assign_candidates(const void* R, const void* C, const int K, const int64_t N
 }
 
 // ---------------------------------------------------------------- update
-constexpr int kUpThreads = 512;
-constexpr int kUpWarps = kUpThreads / 32;
-constexpr int kTokPerWarp = kSeg / kUpWarps;      // 128
-constexpr int kRounds = kTokPerWarp / 32;         // 4
-constexpr int kBatch = 8;                         // rows in flight per warp
+// Centroid sums in 64-bit fixed point.  For channel c of the stage input let
+// m_c be its largest magnitude over the block, e_c = floor(log2 m_c), and
+// L_c = e_c + k - 62 with 2^k > N.  A value is converted to the integer
+// v / 2^L_c, which is exact for every value that is a multiple of 2^L_c:
+// all bf16 values within 39 binades of m_c when N < 2^16 (fp32: 23 binades).
+// No sum of the block's integers can leave the int64 range, integer addition
+// is associative, so the sums are exact and do not depend on the order in
+// which tokens are added -- the update may use atomics and still be
+// deterministic -- and S * 2^L_c equals the fp64 sum taken in any order
+// whenever that sum is itself exact.  The mean is one fp64 divide of the sum
+// (converted exactly, or rounded once if it needs more than 53 bits) by the
+// member count, rounded once to the storage dtype.
+//
+// Three launches per iteration:
+//   bucket    (one CTA per block): the block's entries -- every token on the
+//             first iteration; later, every token whose assignment changed,
+//             once for the centroid it joined (+) and once for the one it left
+//             (-) -- are counted per centroid and written to a list bucketed by
+//             centroid; per-centroid offsets and member-count changes go to
+//             global memory (on the first iteration the running sums are
+//             cleared here).
+//   sum       (several CTAs per block): each warp walks a contiguous piece of
+//             the list, gathers rows two batches ahead, converts them to fixed
+//             point and accumulates them in registers while the centroid stays
+//             the same; each run is added to the running sums with 64-bit
+//             integer atomics (exact, so the order does not matter).
+//   centroids (a warp per centroid): every centroid with entries gets its new
+//             count and, if non-empty, its mean and squared norm.
+constexpr int kBucketThreads = 1024;
+constexpr int kScan = 8;              // assignments per thread per scan step (loads in flight)
+constexpr int kSumThreads = 256;
+constexpr int kSumWarps = kSumThreads / 32;
+constexpr int kSumSlices = 8;         // sum CTAs per block
+constexpr int kSumBatch = 8;          // rows per batch; two batches in flight per warp
 
-// Exact widening of a bf16 / fp32 value to fp64 with integer operations (the
-// exponent is rebiased, the significand shifted); zero, subnormal, infinite
-// and NaN inputs take the conversion instruction.
-__device__ __forceinline__ double widen_bf16(uint32_t b) {
-  const uint32_t e = (b >> 7) & 0xFFu;
-  if (e == 0u || e == 0xFFu) return (double)__uint_as_float(b << 16);
-  const unsigned long long bits = ((unsigned long long)(b & 0x8000u) << 48) |
-                                  ((unsigned long long)(e + 896u) << 52) |
-                                  ((unsigned long long)(b & 0x7Fu) << 45);
-  return __longlong_as_double((long long)bits);
-}
-__device__ __forceinline__ double widen_f32(uint32_t f) {
-  const uint32_t e = (f >> 23) & 0xFFu;
-  if (e == 0u || e == 0xFFu) return (double)__uint_as_float(f);
-  const unsigned long long bits = ((unsigned long long)(f & 0x80000000u) << 32) |
-                                  ((unsigned long long)(e + 896u) << 52) |
-                                  ((unsigned long long)(f & 0x7FFFFFu) << 29);
-  return __longlong_as_double((long long)bits);
+// List entry: token (bits 0-22), centroid (23-30), subtract flag (31).
+constexpr uint32_t kEntTok = 0x7FFFFFu;
+constexpr int kEntKShift = 23;
+constexpr uint32_t kEntSub = 1u << 31;
+constexpr uint32_t kEntNone = 0xFFFFFFFFu;   // never a real entry (token 2^23-1 is out of range)
+
+// L_c of a channel from the bits of its largest magnitude (0 for an all-zero
+// channel), clamped so that 2^-L_c is a normal float.
+__device__ __forceinline__ int fix_exponent(uint32_t maxbits, int log2n) {
+  const int e = maxbits == 0u ? 0 : (int)((maxbits >> 23) & 0xFFu) - 127;
+  const int L = e + log2n - 62;
+  return L < -126 ? -126 : L;
 }
 
-// Lane's four channels of a row as raw 32-bit words (bf16 pairs or fp32).
-template <int DT>
-__device__ __forceinline__ void load4raw(const char* row, int lane, uint32_t (&w)[4]) {
-  if (DT == kBF16) {
-    const uint2 x = *reinterpret_cast<const uint2*>(row + lane * 8);
-    w[0] = x.x & 0xFFFFu; w[1] = x.x >> 16; w[2] = x.y & 0xFFFFu; w[3] = x.y >> 16;
-  } else {
-    const uint4 x = *reinterpret_cast<const uint4*>(row + lane * 16);
-    w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+// Assignments of tokens c + j*blockDim.x + threadIdx.x, j < kScan: new (kn)
+// and previous (ko; -1 on a full pass).  Past the end both read -1, so
+// kn == ko marks "nothing to do" for unchanged and missing tokens alike.
+__device__ __forceinline__ void load_assignments(const uint8_t* piu, const uint8_t* pio, int64_t N, int64_t c,
+                                                 int (&kn)[kScan], int (&ko)[kScan]) {
+#pragma unroll
+  for (int j = 0; j < kScan; ++j) {
+    const int64_t t = c + (int64_t)j * blockDim.x + threadIdx.x;
+    kn[j] = t < N ? (int)piu[t] : -1;
+    ko[j] = (t < N && pio != nullptr) ? (int)pio[t] : -1;
   }
 }
-template <int DT>
-__device__ __forceinline__ double widen(uint32_t w) {
-  return DT == kBF16 ? widen_bf16(w) : widen_f32(w);
+
+// Warp-aggregated shared-memory add of `v` to counter[key] (lanes with the
+// same key are combined; `key` < 0 takes part in no add).  Returns, for
+// returning adds, the slot of this lane: old value + rank among its peers.
+__device__ __forceinline__ int warp_add(int* counter, int key, int v, bool want_slot) {
+  const unsigned peers = __match_any_sync(0xffffffffu, key);
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(peers) - 1;
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  int base = 0;
+  if (key >= 0 && lane == leader) base = atomicAdd(counter + key, v * __popc(peers));
+  if (want_slot) base = __shfl_sync(0xffffffffu, base, leader);
+  return base + rank;
 }
 
 template <int DT>
-__device__ __forceinline__ void load4(const char* row, int lane, float (&v)[4]) {
-  if (DT == kBF16) {
-    const uint2 w = *reinterpret_cast<const uint2*>(row + lane * 8);
+__global__ void __launch_bounds__(kBucketThreads, 1)
+qvg_update_bucket(const UpdateParams p) {
+  __shared__ int hist[kMaxK];
+  __shared__ int dcnt[kMaxK];
+  __shared__ int cursor[kMaxK];
+  const int u = blockIdx.x;
+  const int K = p.K;
+  const int64_t N = p.N;
+  const bool full = p.pi_old == nullptr;
+  for (int x = threadIdx.x; x < kMaxK; x += blockDim.x) { hist[x] = 0; dcnt[x] = 0; }
+  if (full) {                                  // the running sums restart from zero
+    longlong2* S = reinterpret_cast<longlong2*>(p.S + (int64_t)u * K * kD);
+    for (int x = threadIdx.x; x < K * kD / 2; x += blockDim.x) S[x] = make_longlong2(0, 0);
+  }
+  __syncthreads();
+  const uint8_t* piu = p.pi + (int64_t)u * N;
+  const uint8_t* pio = full ? nullptr : p.pi_old + (int64_t)u * N;
+  const int64_t step = (int64_t)kScan * blockDim.x;
+  for (int64_t c = 0; c < N; c += step) {
+    int kn[kScan], ko[kScan];
+    load_assignments(piu, pio, N, c, kn, ko);
+#pragma unroll
+    for (int j = 0; j < kScan; ++j) {
+      const bool ch = kn[j] != ko[j];
+      warp_add(hist, ch ? kn[j] : -1, 1, false);
+      if (!full) {
+        warp_add(hist, ch ? ko[j] : -1, 1, false);
+        warp_add(dcnt, ch ? kn[j] : -1, 1, false);
+        warp_add(dcnt, ch ? ko[j] : -1, -1, false);
+      }
+    }
+  }
+  __syncthreads();
+  // exclusive prefix over the counts (warp 0; 8 per lane)
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int v[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { v[i] = lane * 8 + i < K ? hist[lane * 8 + i] : 0; sum += v[i]; }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    int run = incl - sum;
+    int* off_u = p.off + (int64_t)u * (K + 1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = lane * 8 + i;
+      if (k < K) { cursor[k] = run; off_u[k] = run; }
+      run += v[i];
+    }
+    if (lane == 31) off_u[K] = run;
+  }
+  for (int k = threadIdx.x; k < K; k += blockDim.x)
+    p.cnt[(int64_t)u * K + k] = full ? hist[k] : dcnt[k];
+  __syncthreads();
+  uint32_t* list = p.list + (int64_t)u * 2 * N;    // capacity 2N entries per block
+  for (int64_t c = 0; c < N; c += step) {
+    int kn[kScan], ko[kScan];
+    load_assignments(piu, pio, N, c, kn, ko);
+#pragma unroll
+    for (int j = 0; j < kScan; ++j) {
+      const bool ch = kn[j] != ko[j];
+      const uint32_t t = (uint32_t)(c + (int64_t)j * blockDim.x + threadIdx.x);
+      const int sa = warp_add(cursor, ch ? kn[j] : -1, 1, true);
+      if (ch) list[sa] = t | ((uint32_t)kn[j] << kEntKShift);
+      if (!full) {
+        const int sb = warp_add(cursor, ch ? ko[j] : -1, 1, true);
+        if (ch) list[sb] = t | ((uint32_t)ko[j] << kEntKShift) | kEntSub;
+      }
+    }
+  }
+}
+
+template <int DT> struct RowPart;                 // a lane's 4 channels of a row, raw
+template <> struct RowPart<kBF16> {
+  uint2 w;
+  __device__ __forceinline__ void load(const char* row, int lane) {
+    w = *reinterpret_cast<const uint2*>(row + lane * 8);
+  }
+  __device__ __forceinline__ void get(float (&v)[4]) const {
     v[0] = __uint_as_float(w.x << 16);
     v[1] = __uint_as_float(w.x & 0xFFFF0000u);
     v[2] = __uint_as_float(w.y << 16);
     v[3] = __uint_as_float(w.y & 0xFFFF0000u);
-  } else {
-    const float4 w = *reinterpret_cast<const float4*>(row + lane * 16);
-    v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
   }
-}
+};
+template <> struct RowPart<kFP32> {
+  float4 w;
+  __device__ __forceinline__ void load(const char* row, int lane) {
+    w = *reinterpret_cast<const float4*>(row + lane * 16);
+  }
+  __device__ __forceinline__ void get(float (&v)[4]) const { v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w; }
+};
 
 template <int DT>
-__global__ void __launch_bounds__(kUpThreads, 2)
-qvg_update_partial(const UpdateParams p) {
+__global__ void __launch_bounds__(kSumThreads, 2)
+qvg_update_sum(const UpdateParams p) {
   constexpr int ESZ = Store<DT>::bytes;
-  constexpr int kMaxC = 2 * kSeg;                  // contributions per segment
-  __shared__ uint16_t hist[kUpWarps][kMaxK];      // per-warp counts, then offsets
-  __shared__ int tot[kMaxK];
-  __shared__ int start[kMaxK];
-  __shared__ int dsum[kMaxK];
-  __shared__ uint16_t sorted[kMaxC];              // token | 0x8000 when subtracted
-  __shared__ uint8_t sorted_k[kMaxC];
-  __shared__ int wsum[kMaxK / 32];
-  __shared__ double2 piece[kUpWarps][kD / 2];     // first run of each warp when it continues a centroid
-
-  const int u = blockIdx.y, sgi = blockIdx.x;
+  const int u = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t seg0 = (int64_t)sgi * kSeg;
-  const int seg_len = (int)min((int64_t)kSeg, p.N - seg0);
-  const uint8_t* pn = p.pi + (int64_t)u * p.N + seg0;
-  const uint8_t* po = p.pi_old ? p.pi_old + (int64_t)u * p.N + seg0 : nullptr;
+  const int64_t N = p.N;
+  const int E = p.off[(int64_t)u * (p.K + 1) + p.K];
+  // this warp's piece of the block's list
+  const int64_t part = (int64_t)blockIdx.x * kSumWarps + warp, parts = (int64_t)gridDim.x * kSumWarps;
+  const int e0 = (int)(E * part / parts), e1 = (int)(E * (part + 1) / parts);
+  if (e0 >= e1) return;
+  float to_fix[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    to_fix[e] = __int_as_float((127 - fix_exponent(p.chmax[(int64_t)u * kD + 4 * lane + e], p.log2n)) << 23);
+  const uint32_t* list = p.list + (int64_t)u * 2 * N;
+  const char* Ru = static_cast<const char*>(p.R) + (int64_t)u * N * kD * ESZ;
+  long long* Su = p.S + (int64_t)u * p.K * kD + 4 * lane;
+  const int nb = (e1 - e0 + kSumBatch - 1) / kSumBatch;
+  long long run[4] = {0, 0, 0, 0};
+  int run_k = -1;
+  uint32_t grp = e0 + lane < e1 ? list[e0 + lane] : kEntNone;          // 32 consecutive entries, one per lane
+  uint32_t grp_next = e0 + 32 + lane < e1 ? list[e0 + 32 + lane] : kEntNone;
+  RowPart<DT> ra[kSumBatch], rb[kSumBatch];
+  uint32_t ea[kSumBatch], eb[kSumBatch];
 
-  for (int x = threadIdx.x; x < kUpWarps * kMaxK; x += blockDim.x) (&hist[0][0])[x] = 0;
-  for (int x = threadIdx.x; x < kMaxK; x += blockDim.x) dsum[x] = 0;
-  __syncthreads();
-
-  // 1. Stable per-warp ranks of the contributions.  Warp w owns tokens
-  //    [w*128, w*128+128); its contributions are taken in a fixed order:
-  //    pass 0 = subtractions (old centroid), pass 1 = additions (new centroid).
-  // the warp's 128 assignments (and the previous ones), loaded up front:
-  // round r of lane l is token w*128 + r*32 + l
-  uint8_t an[kRounds], ao[kRounds];
-#pragma unroll
-  for (int r = 0; r < kRounds; ++r) {
-    const int tok = warp * kTokPerWarp + r * 32 + lane;
-    an[r] = tok < seg_len ? pn[tok] : 0;
-    ao[r] = (po != nullptr && tok < seg_len) ? po[tok] : 0;
-  }
-  int key[2][kRounds], rank[2][kRounds];
-#pragma unroll
-  for (int ps = 0; ps < 2; ++ps) {
-#pragma unroll
-    for (int r = 0; r < kRounds; ++r) {
-      const int tok = warp * kTokPerWarp + r * 32 + lane;
-      bool valid = tok < seg_len;
-      int k = 0;
-      if (valid) {
-        const int kn = an[r];
-        if (po == nullptr) { valid = ps == 1; k = kn; }
-        else {
-          const int ko = ao[r];
-          valid = ko != kn;
-          k = ps == 0 ? ko : kn;
-        }
-      }
-      key[ps][r] = valid ? k : 0x10000 + lane;           // invalid keys never match
-      const unsigned mask = __match_any_sync(0xffffffffu, key[ps][r]);
-      const int before = __popc(mask & ((1u << lane) - 1u));
-      const int base = valid ? hist[warp][k] : 0;
-      __syncwarp();
-      if (valid && before == 0) {
-        hist[warp][k] = (uint16_t)(base + __popc(mask));
-        atomicAdd(&dsum[k], ps == 0 ? -__popc(mask) : __popc(mask));
-      }
-      __syncwarp();
-      rank[ps][r] = base + before;
+  auto fetch = [&](int b, RowPart<DT>(&rows)[kSumBatch], uint32_t(&ent)[kSumBatch]) {
+    if ((b & 3) == 0 && b > 0) {
+      grp = grp_next;
+      const int nxt = e0 + (b / 4 + 1) * 32 + lane;
+      grp_next = nxt < e1 ? list[nxt] : kEntNone;
     }
-  }
-  __syncthreads();
-
-  // 2. Exclusive prefix over (k, w): offsets of each warp's run of centroid k.
-  if (threadIdx.x < kMaxK) {
-    const int k = threadIdx.x;
-    int run = 0;
-    for (int w = 0; w < kUpWarps; ++w) {
-      const int c = hist[w][k];
-      hist[w][k] = (uint16_t)run;
-      run += c;
-    }
-    tot[k] = run;
-    int v = run;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, v, off);
-      if (lane >= off) v += o;
-    }
-    if (lane == 31) wsum[k >> 5] = v;
-    start[k] = v - run;
-  }
-  __syncthreads();
-  if (threadIdx.x < kMaxK) {
-    const int k = threadIdx.x;
-    int add = 0;
-    for (int w = 0; w < (k >> 5); ++w) add += wsum[w];
-    start[k] += add;
-    if (k < p.K) {
-      const int64_t o = ((int64_t)u * p.nseg + sgi) * p.K + k;
-      p.ncontrib[o] = tot[k];
-      p.dcount[o] = dsum[k];
-    }
-  }
-  __syncthreads();
-  const int total = start[kMaxK - 1] + tot[kMaxK - 1];
-
-  // 3. Scatter into centroid order (stable within a centroid).
-#pragma unroll
-  for (int ps = 0; ps < 2; ++ps) {
-#pragma unroll
-    for (int r = 0; r < kRounds; ++r) {
-      const int k = key[ps][r];
-      if (k < 0x10000) {
-        const int tok = warp * kTokPerWarp + r * 32 + lane;
-        const int pos = start[k] + hist[warp][k] + rank[ps][r];
-        sorted[pos] = (uint16_t)(tok | (ps == 0 ? 0x8000 : 0));
-        sorted_k[pos] = (uint8_t)k;
-      }
-    }
-  }
-  __syncthreads();
-
-  // 4. Each warp sums an equal share of the sorted contributions (lane owns 4
-  //    channels) run by run.  A run holding all of a centroid's contributions
-  //    is written out directly; a warp's first run that continues a centroid
-  //    from the previous warp is parked in shared memory; a last run that
-  //    continues into the next warp is completed by this warp after the
-  //    barrier, adding the parked pieces in warp order.
-  const char* R = static_cast<const char*>(p.R) + ((int64_t)u * p.N + seg0) * kD * ESZ;
-  double* part = p.partial + ((int64_t)u * p.nseg + sgi) * p.K * kD;
-  const int share = (total + kUpWarps - 1) / kUpWarps;
-  const int r0 = min(total, warp * share);
-  const int r1 = min(total, r0 + share);
-  int cur = -1, cur_begin = r0;
-  double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-  int own_k = -1;
-  double o0 = 0.0, o1 = 0.0, o2 = 0.0, o3 = 0.0;
-  auto emit = [&](int k, int run_begin, int run_end) {
-    const int cb = start[k], ce = start[k] + tot[k];
-    if (cb >= run_begin && ce <= run_end) {            // all of the centroid's contributions
-      double2* dst = reinterpret_cast<double2*>(part + (int64_t)k * kD + lane * 4);
-      dst[0] = make_double2(a0, a1);
-      dst[1] = make_double2(a2, a3);
-    } else if (cb < run_begin) {                        // continues a centroid: park it
-      piece[warp][lane * 2] = make_double2(a0, a1);
-      piece[warp][lane * 2 + 1] = make_double2(a2, a3);
-    } else {                                            // starts here, continues past r1
-      own_k = k; o0 = a0; o1 = a1; o2 = a2; o3 = a3;
+    for (int r = 0; r < kSumBatch; ++r) {
+      ent[r] = __shfl_sync(0xffffffffu, grp, (b & 3) * 8 + r);
+      if (ent[r] != kEntNone) rows[r].load(Ru + (int64_t)(ent[r] & kEntTok) * kD * ESZ, lane);
     }
   };
-  for (int b = r0; b < r1; b += kBatch) {
-    uint32_t v[kBatch][4];
-    int kk[kBatch];
-    bool neg[kBatch];
+  auto flush = [&]() {
+    if (run_k >= 0) {
+      long long* a = Su + (int64_t)run_k * kD;
 #pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      const int pos = min(b + q, r1 - 1);
-      kk[q] = sorted_k[pos];
-      const int e = sorted[pos];
-      neg[q] = (e & 0x8000) != 0;
-      load4raw<DT>(R + (int64_t)(e & 0x7FFF) * kD * ESZ, lane, v[q]);
+      for (int e = 0; e < 4; ++e)
+        atomicAdd(reinterpret_cast<unsigned long long*>(a + e), (unsigned long long)run[e]);
     }
+  };
+  auto consume = [&](const RowPart<DT>(&rows)[kSumBatch], const uint32_t(&ent)[kSumBatch]) {
 #pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-      if (b + q < r1) {
-        if (kk[q] != cur) {
-          if (cur >= 0) emit(cur, cur_begin, b + q);
-          cur = kk[q];
-          cur_begin = b + q;
-          a0 = a1 = a2 = a3 = 0.0;
-        }
-        // a subtraction adds the negated value (a sign flip, exact)
-        const double x0 = widen<DT>(v[q][0]), x1 = widen<DT>(v[q][1]);
-        const double x2 = widen<DT>(v[q][2]), x3 = widen<DT>(v[q][3]);
-        a0 = __dadd_rn(a0, neg[q] ? -x0 : x0);
-        a1 = __dadd_rn(a1, neg[q] ? -x1 : x1);
-        a2 = __dadd_rn(a2, neg[q] ? -x2 : x2);
-        a3 = __dadd_rn(a3, neg[q] ? -x3 : x3);
+    for (int r = 0; r < kSumBatch; ++r) {
+      if (ent[r] == kEntNone) break;               // warp-uniform
+      const int k = (int)((ent[r] >> kEntKShift) & 0xFFu);
+      if (k != run_k) {
+        flush();
+        run_k = k;
+        run[0] = run[1] = run[2] = run[3] = 0;
+      }
+      float v[4];
+      rows[r].get(v);
+      const bool neg = (ent[r] & kEntSub) != 0u;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const long long q = __float2ll_rn(__fmul_rn(v[e], to_fix[e]));
+        run[e] += neg ? -q : q;
       }
     }
-  }
-  if (cur >= 0) emit(cur, cur_begin, r1);
-  __syncthreads();
-  if (own_k >= 0) {
-    const int last_w = min(kUpWarps - 1, (start[own_k] + tot[own_k] - 1) / share);
-    for (int w = warp + 1; w <= last_w; ++w) {
-      const double2 x = piece[w][lane * 2], y = piece[w][lane * 2 + 1];
-      o0 = __dadd_rn(o0, x.x); o1 = __dadd_rn(o1, x.y);
-      o2 = __dadd_rn(o2, y.x); o3 = __dadd_rn(o3, y.y);
+  };
+  fetch(0, ra, ea);
+  for (int b = 0; b < nb; b += 2) {
+    if (b + 1 < nb) fetch(b + 1, rb, eb);
+    consume(ra, ea);
+    if (b + 1 < nb) {
+      if (b + 2 < nb) fetch(b + 2, ra, ea);
+      consume(rb, eb);
     }
-    double2* dst = reinterpret_cast<double2*>(part + (int64_t)own_k * kD + lane * 4);
-    dst[0] = make_double2(o0, o1);
-    dst[1] = make_double2(o2, o3);
   }
+  flush();
 }
 
-// Running sums += segment sums (segments in order), counts += changes, then
-// the mean of every non-empty centroid, rounded once to the storage dtype.
+// A warp per centroid: new count; for a non-empty centroid the mean of the
+// exact sum, rounded once to the storage dtype, and its squared norm.
 template <int DT>
 __global__ void __launch_bounds__(256)
-qvg_update_finalize(const UpdateParams p) {
+qvg_update_centroids(const UpdateParams p) {
   const int u = blockIdx.y;
   const int k = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (k >= p.K) return;
-  const int64_t seg_stride = (int64_t)p.K * kD;
-  const int* nc = p.ncontrib + (int64_t)u * p.nseg * p.K + k;
-  const int* dc = p.dcount + (int64_t)u * p.nseg * p.K + k;
-  const double* part = p.partial + ((int64_t)u * p.nseg * p.K + k) * kD + lane * 4;
-  double2* Sk = reinterpret_cast<double2*>(p.S + ((int64_t)u * p.K + k) * kD + lane * 4);
   const bool full = p.pi_old == nullptr;
-  double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-  long long n = 0;
-  if (!full) {
-    const double2 x = Sk[0], y = Sk[1];
-    a0 = x.x; a1 = x.y; a2 = y.x; a3 = y.y;
-    n = p.n[(int64_t)u * p.K + k];
-  }
-  bool any = false;
-  for (int s0 = 0; s0 < p.nseg; s0 += 32) {
-    const int sl = s0 + lane;
-    const int c = sl < p.nseg ? nc[(int64_t)sl * p.K] : 0;
-    int d = sl < p.nseg ? dc[(int64_t)sl * p.K] : 0;
-    unsigned m = __ballot_sync(0xffffffffu, c > 0);
-    any |= m != 0;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-    n += d;
-    // segments in ascending order, four loads in flight
-    while (m) {
-      int idx[4];
-      double2 x[4], y[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        idx[q] = m ? __ffs(m) - 1 : -1;
-        if (m) m &= m - 1;
-        if (idx[q] >= 0) {
-          const double2* src = reinterpret_cast<const double2*>(part + (int64_t)(s0 + idx[q]) * seg_stride);
-          x[q] = src[0];
-          y[q] = src[1];
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (idx[q] >= 0) {
-          a0 = __dadd_rn(a0, x[q].x); a1 = __dadd_rn(a1, x[q].y);
-          a2 = __dadd_rn(a2, y[q].x); a3 = __dadd_rn(a3, y[q].y);
-        }
-      }
-    }
-  }
-  if (full || any) {
-    Sk[0] = make_double2(a0, a1);
-    Sk[1] = make_double2(a2, a3);
-    if (lane == 0) p.n[(int64_t)u * p.K + k] = n;
-  }
-  if (n <= 0 || !(full || any)) return;   // empty keeps its centroid; unchanged needs no update
+  const int* off_u = p.off + (int64_t)u * (p.K + 1);
+  if (!full && off_u[k + 1] == off_u[k]) return;   // no entries: unchanged
+  int n = p.cnt[(int64_t)u * p.K + k];
+  if (!full) n += p.n[(int64_t)u * p.K + k];
+  if (lane == 0) p.n[(int64_t)u * p.K + k] = n;
+  if (n <= 0) return;                                // an empty centroid keeps its value
+  const longlong2* Sg = reinterpret_cast<const longlong2*>(p.S + ((int64_t)u * p.K + k) * kD + 4 * lane);
+  const longlong2 a = Sg[0], b = Sg[1];
+  const long long sum[4] = {a.x, a.y, b.x, b.y};
   const double dn = (double)n;
-  const double a[4] = {a0, a1, a2, a3};
   double sq = 0.0;
+  double mean[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int L = fix_exponent(p.chmax[(int64_t)u * kD + 4 * lane + e], p.log2n);
+    const double scale = __longlong_as_double((long long)(1023 + L) << 52);
+    mean[e] = __ddiv_rn(__dmul_rn(__ll2double_rn(sum[e]), scale), dn);
+  }
   if (DT == kBF16) {
-    uint16_t b[4];
+    uint16_t h[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      b[e] = f64_to_bf16_rne(__ddiv_rn(a[e], dn));
-      const double c = (double)bf16_bits_to_f32(b[e]);
+      h[e] = f64_to_bf16_rne(mean[e]);
+      const double c = (double)bf16_bits_to_f32(h[e]);
       sq = __dadd_rn(sq, __dmul_rn(c, c));
     }
     uint2 w;
-    w.x = (uint32_t)b[0] | ((uint32_t)b[1] << 16);
-    w.y = (uint32_t)b[2] | ((uint32_t)b[3] << 16);
+    w.x = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
+    w.y = (uint32_t)h[2] | ((uint32_t)h[3] << 16);
     *reinterpret_cast<uint2*>(static_cast<char*>(p.C) + (((int64_t)u * p.K + k) * kD + lane * 4) * 2) = w;
   } else {
     float f[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      f[e] = __double2float_rn(__ddiv_rn(a[e], dn));
+      f[e] = __double2float_rn(mean[e]);
       sq = __dadd_rn(sq, __dmul_rn((double)f[e], (double)f[e]));
     }
     *reinterpret_cast<float4*>(static_cast<char*>(p.C) + (((int64_t)u * p.K + k) * kD + lane * 4) * 4) =
@@ -622,17 +589,23 @@ cudaError_t launch_assign_candidates(const void* R, const void* C, int K, int64_
   return cudaGetLastError();
 }
 
-cudaError_t launch_update_partial(const UpdateParams& p, int dtype, cudaStream_t s) {
-  const dim3 g1((unsigned)p.nseg, (unsigned)p.W);
-  if (dtype == kBF16) qvg_update_partial<kBF16><<<g1, kUpThreads, 0, s>>>(p);
-  else qvg_update_partial<kFP32><<<g1, kUpThreads, 0, s>>>(p);
+cudaError_t launch_update_bucket(const UpdateParams& p, int dtype, cudaStream_t s) {
+  if (dtype == kBF16) qvg_update_bucket<kBF16><<<(unsigned)p.W, kBucketThreads, 0, s>>>(p);
+  else qvg_update_bucket<kFP32><<<(unsigned)p.W, kBucketThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_update_finalize(const UpdateParams& p, int dtype, cudaStream_t s) {
-  const dim3 g2((unsigned)((p.K + 7) / 8), (unsigned)p.W);
-  if (dtype == kBF16) qvg_update_finalize<kBF16><<<g2, 256, 0, s>>>(p);
-  else qvg_update_finalize<kFP32><<<g2, 256, 0, s>>>(p);
+cudaError_t launch_update_sum(const UpdateParams& p, int dtype, cudaStream_t s) {
+  const dim3 grid((unsigned)kSumSlices, (unsigned)p.W);
+  if (dtype == kBF16) qvg_update_sum<kBF16><<<grid, kSumThreads, 0, s>>>(p);
+  else qvg_update_sum<kFP32><<<grid, kSumThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_update_centroids(const UpdateParams& p, int dtype, cudaStream_t s) {
+  const dim3 grid((unsigned)((p.K + 7) / 8), (unsigned)p.W);
+  if (dtype == kBF16) qvg_update_centroids<kBF16><<<grid, 256, 0, s>>>(p);
+  else qvg_update_centroids<kFP32><<<grid, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -59,18 +59,16 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // Layout of the caller's workspace for a batch of W units.
 struct Plan {
   int W = 0;
-  int nseg = 0;
   int nR = 0;
   size_t off_R[2] = {0, 0};
   size_t off_rnorm = 0, off_cn = 0, off_list = 0, off_listcnt = 0;
-  size_t off_partial = 0, off_ncontrib = 0, off_dcount = 0, off_S = 0, off_n = 0, off_pi = 0;
+  size_t off_chmax = 0, off_off = 0, off_cnt = 0, off_S = 0, off_n = 0, off_pi = 0;
   size_t off_status = 0, total = 0;
 };
 
 Plan make_plan(const qvg_config& c, int64_t N, int W, int dtype) {
   Plan p;
   p.W = W;
-  p.nseg = (int)((N + kSeg - 1) / kSeg);
   p.nR = c.T >= 3 ? 2 : (c.T == 2 ? 1 : 0);
   const size_t esz = (size_t)esize(dtype);
   size_t o = 0;
@@ -80,11 +78,11 @@ Plan make_plan(const qvg_config& c, int64_t N, int W, int dtype) {
   p.off_cn = o;                           o = align_up(o + (size_t)W * kMaxK * sizeof(float));
   p.off_list = o;                         o = align_up(o + (size_t)W * N * 8);
   p.off_listcnt = o;                      o = align_up(o + (size_t)W * sizeof(uint32_t));
-  p.off_partial = o;                      o = align_up(o + (size_t)W * p.nseg * c.K * kD * sizeof(double));
-  p.off_ncontrib = o;                     o = align_up(o + (size_t)W * p.nseg * c.K * sizeof(int));
-  p.off_dcount = o;                       o = align_up(o + (size_t)W * p.nseg * c.K * sizeof(int));
-  p.off_S = o;                            o = align_up(o + (size_t)W * c.K * kD * sizeof(double));
-  p.off_n = o;                            o = align_up(o + (size_t)W * c.K * sizeof(long long));
+  p.off_chmax = o;                        o = align_up(o + (size_t)W * kD * sizeof(uint32_t));
+  p.off_off = o;                          o = align_up(o + (size_t)W * (c.K + 1) * sizeof(int));
+  p.off_cnt = o;                          o = align_up(o + (size_t)W * c.K * sizeof(int));
+  p.off_S = o;                            o = align_up(o + (size_t)W * c.K * kD * sizeof(long long));
+  p.off_n = o;                            o = align_up(o + (size_t)W * c.K * sizeof(int));
   p.off_pi = o;                           o = align_up(o + (size_t)W * N);
   p.total = o;
   return p;
@@ -95,12 +93,13 @@ int preferred_batch(const qvg_config& c, int64_t N, int H, int dtype) {
     const int w = std::atoi(env);
     if (w > 0) return std::min(w, H);
   }
-  // As many blocks per launch as a 2 GiB workspace holds (at most 128): wide
-  // launches keep every SM busy and amortise the per-launch pipeline fill.
+  // As many blocks per launch as a 2 GiB workspace holds, at most one per SM:
+  // the tensor-core assignment runs one CTA per block, so a wave of exactly
+  // one block per SM keeps every SM busy; other kernels split blocks further.
   const double budget = 2.0 * 1024.0 * 1024.0 * 1024.0;
   const double per_unit = (double)make_plan(c, N, 1, dtype).total;
   int w = (int)std::floor(budget / per_unit);
-  return std::max(1, std::min(std::min(w, 128), H));
+  return std::max(1, std::min(std::min(w, qvg::device_sm_count()), H));
 }
 
 // Relative error bound assumed for the tensor-core sums (128 exact bf16 x bf16
@@ -124,6 +123,7 @@ qvg_status check_config(const qvg_config* c, int64_t N, int32_t H, int32_t d, qv
   if (c->group_size < 4 || c->group_size % 4 != 0 || d < 4 || d % c->group_size != 0)
     return QVG_ERR_INVALID_ARG;
   if (N < 0 || H < 1) return QVG_ERR_INVALID_ARG;
+  if (N >= (int64_t(1) << 23)) return QVG_ERR_UNSUPPORTED;   // token indices are 23-bit in the update
   if (d != kD || !g_supported(c->group_size) || c->T > kMaxT) return QVG_ERR_UNSUPPORTED;
   return QVG_OK;
 }
@@ -136,12 +136,12 @@ qvg_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QVG_OK : QVG_E
 // kernel from CUDA events recorded on the launching stream around each launch.
 enum Kind {
   K_DEQUANT, K_RESIDUAL, K_RESIDUAL_QUANT, K_ROWNORM, K_INIT, K_ASSIGN_EXACT, K_ASSIGN_TC,
-  K_RECHECK, K_UPD_PARTIAL, K_UPD_FINAL, K_NKINDS
+  K_RECHECK, K_UPD_BUCKET, K_UPD_SUM, K_UPD_CENT, K_NKINDS
 };
 const char* const kKindNames[K_NKINDS] = {
   "qvg_dequant_fused", "qvg_residual", "qvg_residual_quant", "qvg_row_norms", "qvg_init_centroids",
-  "qvg_assign_exact", "qvg_kmeans_assign", "qvg_assign_recheck", "qvg_update_partial",
-  "qvg_update_finalize"};
+  "qvg_assign_exact", "qvg_kmeans_assign", "qvg_assign_recheck", "qvg_update_bucket", "qvg_update_sum",
+  "qvg_update_centroids"};
 
 struct Profiler {
   std::mutex mu;
@@ -269,6 +269,9 @@ qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, i
   uint32_t* list_count = reinterpret_cast<uint32_t*>(ws + plan.off_listcnt);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws + plan.off_status);
   unsigned long long* flagged = reinterpret_cast<unsigned long long*>(ws + plan.off_status + 8);
+  uint32_t* chmax = reinterpret_cast<uint32_t*>(ws + plan.off_chmax);
+  int log2n = 0;                      // smallest k with 2^k > N (fixed-point scale of the sums)
+  while (log2n < 62 && (int64_t(1) << log2n) <= N) ++log2n;
   // bf16 blocks take the tensor-core assignment; fp32 blocks the exact CUDA-core one
   const bool use_tc = dt == kBF16 && assign_path_tc();
   const int ng = kD / c.group_size;
@@ -290,9 +293,10 @@ qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, i
     for (int t = 0; t < c.T; ++t) {
       char* Ct = static_cast<char*>(out->centroids) + ((size_t)t * H + u0) * c.K * kD * esz;
       uint8_t* pit = out->assign + ((size_t)t * H + u0) * N;
-      if (t == 0) {   // squared row norms of X for the assignment error bound
+      if (t == 0) {   // squared row norms of X (assignment error bound), channel maxima (update scale)
         ResidualParams nq = rq;
-        nq.R_in = Xu; nq.C = nullptr; nq.R_out = nullptr; nq.rnorm2 = rnorm;
+        nq.R_in = Xu; nq.C = nullptr; nq.R_out = nullptr; nq.rnorm2 = rnorm; nq.chmax = chmax;
+        QVG_TRY(cudaMemsetAsync(chmax, 0, (size_t)w * kD * sizeof(uint32_t), s));
         QVG_TRY(plaunch(K_ROWNORM, s, [&] { return launch_residual(nq, dt, false, s); }));
       }
       if (warm) {
@@ -326,21 +330,23 @@ qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, i
           QVG_TRY(plaunch(K_ASSIGN_EXACT, s, [&] { return launch_assign_exact(ap, dt, s); }));
         }
         UpdateParams up{};
-        up.R = Rin; up.pi = pi_new; up.pi_old = pi_old; up.C = Ct; up.cn = cn;
-        up.N = N; up.W = w; up.K = c.K; up.nseg = plan.nseg;
-        up.partial = reinterpret_cast<double*>(ws + plan.off_partial);
-        up.ncontrib = reinterpret_cast<int*>(ws + plan.off_ncontrib);
-        up.dcount = reinterpret_cast<int*>(ws + plan.off_dcount);
-        up.S = reinterpret_cast<double*>(ws + plan.off_S);
-        up.n = reinterpret_cast<long long*>(ws + plan.off_n);
-        QVG_TRY(plaunch(K_UPD_PARTIAL, s, [&] { return launch_update_partial(up, dt, s); }));
-        QVG_TRY(plaunch(K_UPD_FINAL, s, [&] { return launch_update_finalize(up, dt, s); }));
+        up.R = Rin; up.pi = pi_new; up.pi_old = pi_old; up.chmax = chmax; up.C = Ct; up.cn = cn;
+        up.N = N; up.W = w; up.K = c.K; up.log2n = log2n;
+        up.list = reinterpret_cast<uint32_t*>(list);   // the near-tie list is consumed by now
+        up.off = reinterpret_cast<int*>(ws + plan.off_off);
+        up.cnt = reinterpret_cast<int*>(ws + plan.off_cnt);
+        up.S = reinterpret_cast<long long*>(ws + plan.off_S);
+        up.n = reinterpret_cast<int*>(ws + plan.off_n);
+        QVG_TRY(plaunch(K_UPD_BUCKET, s, [&] { return launch_update_bucket(up, dt, s); }));
+        QVG_TRY(plaunch(K_UPD_SUM, s, [&] { return launch_update_sum(up, dt, s); }));
+        QVG_TRY(plaunch(K_UPD_CENT, s, [&] { return launch_update_centroids(up, dt, s); }));
       }
       ResidualParams rp = rq;
       rp.R_in = Rin; rp.C = Ct; rp.pi = pit;
       if (t + 1 < c.T) {
         void* Rout = ws + plan.off_R[t % 2];
-        rp.R_out = Rout; rp.rnorm2 = rnorm;
+        rp.R_out = Rout; rp.rnorm2 = rnorm; rp.chmax = chmax;
+        QVG_TRY(cudaMemsetAsync(chmax, 0, (size_t)w * kD * sizeof(uint32_t), s));
         QVG_TRY(plaunch(K_RESIDUAL, s, [&] { return launch_residual(rp, dt, false, s); }));
         Rin = Rout;
       } else {

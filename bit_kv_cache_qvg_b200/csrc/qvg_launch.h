@@ -32,6 +32,8 @@ struct ResidualParams {
   const uint8_t* pi;       // [W][N]
   void* R_out;             // [W][N][d] or nullptr
   float* rnorm2;           // [W][N] or nullptr
+  uint32_t* chmax;         // [W][d] or nullptr: atomic max of the bits of |value| per channel
+                           // of the values read (no C) or written (with C); starts at zero
   uint8_t* codes;          // [W][N][d/4]
   uint8_t* scale;          // [W][N][d/G]
   uint8_t* zero;           // [W][N][d/G]
@@ -92,31 +94,30 @@ cudaError_t launch_assign_candidates(const void* R, const void* C, int K, int64_
                                      cudaStream_t s);
 size_t assign_tc_smem_bytes(int K);
 
-constexpr int kSeg = 2048;   // tokens per update segment
-
 struct UpdateParams {
-  const void* R;        // [W][N][d]
-  const uint8_t* pi;    // [W][N] assignment of this iteration
-  const uint8_t* pi_old;// [W][N] assignment of the previous iteration, or nullptr (full sums)
-  double* partial;      // [W][nseg][K][d] per-segment sums of the contributions
-  int* ncontrib;        // [W][nseg][K]   contributions per segment (0 = partial not written)
-  int* dcount;          // [W][nseg][K]   change of the member count per segment
-  double* S;            // [W][K][d]      running fp64 sums of the members
-  long long* n;         // [W][K]         member counts
-  void* C;              // [W][K][d]      centroids (updated in place)
-  float* cn;            // [W][K]
+  const void* R;          // [W][N][d] stage input
+  const uint8_t* pi;      // [W][N] assignment of this iteration
+  const uint8_t* pi_old;  // [W][N] assignment of the previous iteration, or nullptr (full sums)
+  const uint32_t* chmax;  // [W][d] bits of the largest |value| of each channel of R
+  uint32_t* list;         // [W][2N] scratch: entries bucketed by centroid
+  int* off;               // [W][K+1] scratch: bucket offsets
+  int* cnt;               // [W][K]   scratch: member counts (first iteration) or their changes
+  long long* S;           // [W][K][d] running member sums in fixed point (units of 2^L_c)
+  int* n;                 // [W][K]    member counts
+  void* C;                // [W][K][d] centroids (updated in place)
+  float* cn;              // [W][K]    squared centroid norms
   int64_t N;
   int W;
   int K;
-  int nseg;
+  int log2n;              // smallest k with 2^k > N
 };
-// Per-segment fp64 sums of the contributions of the segment's tokens in
-// centroid order (stable counting sort): with pi_old == nullptr every token
-// adds its row to its centroid; otherwise a token whose centroid changed adds
-// its row to the new centroid and subtracts it from the old one.
-cudaError_t launch_update_partial(const UpdateParams& p, int dtype, cudaStream_t s);
-// Running sums S += segment sums (segments in order), counts n += changes,
-// then every non-empty centroid = round(S / n) in the storage dtype.
-cudaError_t launch_update_finalize(const UpdateParams& p, int dtype, cudaStream_t s);
+// Exact fixed-point centroid sums: with pi_old == nullptr every token adds its
+// row to its centroid; otherwise a token whose centroid changed adds its row
+// to the new centroid and subtracts it from the old one.  Then every changed,
+// non-empty centroid = round(S / n) in the storage dtype, and its |c|^2.
+// Three launches: bucket the entries by centroid, sum them, recompute centroids.
+cudaError_t launch_update_bucket(const UpdateParams& p, int dtype, cudaStream_t s);
+cudaError_t launch_update_sum(const UpdateParams& p, int dtype, cudaStream_t s);
+cudaError_t launch_update_centroids(const UpdateParams& p, int dtype, cudaStream_t s);
 
 }  // namespace qvg

@@ -13,7 +13,7 @@
 //
 // The reserve is kStaticScratchBytes (32 MiB) of global memory.  It holds
 // the k-means working set of as many blocks per wave as fit, and at least
-// one: about 80,000 tokens per block at bf16, K = 256, T = 2.  A call whose
+// one: about 120,000 tokens per block at bf16, K = 256, T = 2.  A call whose
 // single block needs more is rejected before any work is queued.
 #include <cuda_runtime.h>
 

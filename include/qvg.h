@@ -32,7 +32,7 @@
  *     in one call (heads, or heads x layers x K/V), N the tokens per block,
  *     d the channels per token (head dimension).
  *   - Supported by the kernels: d = 128; G in {8, 16, 32, 64, 128};
- *     bits = 2; 1 <= K <= 256; 0 <= T <= 8.  Other values that the method
+ *     bits = 2; 1 <= K <= 256; 0 <= T <= 8; N < 2^23.  Other values that the method
  *     allows return QVG_ERR_UNSUPPORTED.
  */
 #ifndef QVG_H_
@@ -134,7 +134,7 @@ QVG_API size_t qvg_workspace_bytes(const qvg_config* cfg, int64_t N, int32_t H, 
  * Errors: INVALID_ARG for NULL pointers, K < 1 or K > 256, T < 0, bits != 2,
  * G not dividing d or not a multiple of 4, N < 1, H < 1, N < K on a cold
  * start with T > 0, iters < 1 (or warm_iters < 1 when warm) with T > 0;
- * UNSUPPORTED for d != 128, G outside {8,16,32,64,128}, T > 8;
+ * UNSUPPORTED for d != 128, G outside {8,16,32,64,128}, T > 8, N >= 2^23;
  * WORKSPACE_TOO_SMALL; CUDA; DEVICE_TIMEOUT. */
 QVG_API qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype,
                         int64_t N, int32_t H, int32_t d, const void* init_centroids,
@@ -174,7 +174,7 @@ QVG_API int64_t qvg_workspace_flagged(void* workspace, size_t ws_bytes, qvg_stre
  * Arguments, layouts, results and errors are those of qvg_quantize, less
  * the workspace; each call first zeroes the reserve's 16-byte status word
  * and near-tie counter (on `stream`), then queues the same kernels.
- * Limits: the reserve must hold one block's working set, about 80,000
+ * Limits: the reserve must hold one block's working set, about 120,000
  * tokens per block at bf16 with K = 256, T = 2 (qvg_workspace_bytes with
  * H = 1 gives the exact need); a larger block returns WORKSPACE_TOO_SMALL
  * before anything is queued.  Blocks beyond what one wave holds run in

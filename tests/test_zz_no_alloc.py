@@ -66,7 +66,7 @@ def test_static_reserve_warm_start_matches(q):
 
 def test_static_reserve_rejects_block_too_large(q):
     cfg = q.config(K=256, T=2, group_size=64, iters=1)
-    N = 120_000                           # one block's working set exceeds the 32 MiB reserve
+    N = 200_000                           # one block's working set exceeds the 32 MiB reserve
     assert q.workspace_bytes(cfg, N, 1) > 32 << 20
     X = torch.zeros((1, N, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(q.QvgError) as e:
