@@ -16,10 +16,10 @@
 // swizzle, K-major), token tiles stream through a 3-stage TMA ring; no
 // multicast.  Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (one
 // elected thread) and TMEM owner, warps 2-9 = epilogue (two warps per TMEM
-// lane quarter, each owning half of the centroid columns).  Two TMEM
-// accumulators (2 x 256 columns) let the epilogue of tile i overlap the MMAs
-// of tile i+1.  Every mbarrier wait is bounded; on timeout the kernel records
-// an error in the status word, drains, frees TMEM and returns.
+// lane quarter, taking alternate tiles).  Two TMEM accumulators (2 x 256
+// columns) let the epilogue of tile i overlap the MMAs of tile i+1.  Every
+// mbarrier wait is bounded; on timeout the kernel records an error in the
+// status word, drains, frees TMEM and returns.
 #include <cuda.h>
 #include <cstdio>
 
@@ -163,8 +163,9 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// 32 lanes x 32 consecutive 32-bit columns -> 32 registers per thread.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// 32 lanes x 32 consecutive 32-bit columns -> 32 registers per thread
+// (asynchronous: the registers are valid after tmem_wait_ld).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -175,12 +176,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// Wait for this thread's tensor-memory loads; the buffer's registers pass
+// through the asm so that no use of them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+        "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+        "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+        "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 struct TcParams {
   const float* rnorm2;      // [W][N]
@@ -243,15 +253,14 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
   uint8_t* sA = smem + 2 * Npad * 128;                          // kStages x 32 KB (1024-aligned)
   uint8_t* sAx = sA + kStages * kAStageBytes;                   // 128 x 16 bf16: [1 1 1 0 ...]
   uint8_t* sBx = sAx + kTileM * 32;                             // Npad x 16 bf16: -|c|^2/2 in 3 pieces
-  float* mbuf = reinterpret_cast<float*>(sBx + Npad * 32);      // [2 acc][2 halves][6 vals][128 rows]
-  TcSmemBarriers* bars = reinterpret_cast<TcSmemBarriers*>(mbuf + 2 * 12 * kTileM);
+  TcSmemBarriers* bars = reinterpret_cast<TcSmemBarriers*>(sBx + Npad * 32);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&bars->full[s], 1); mbar_init(&bars->empty[s], 1); }
     mbar_init(&bars->b_full, 1);
-    for (int a = 0; a < 2; ++a) { mbar_init(&bars->tmem_full[a], 1); mbar_init(&bars->tmem_empty[a], 8); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&bars->tmem_full[a], 1); mbar_init(&bars->tmem_empty[a], 4); }
     bars->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -357,87 +366,91 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
     }
   } else {
     // ---------------- epilogue (warps 2..9)
-    const int q = warp & 3;                  // TMEM lane quarter this warp may access
-    const int hc = (warp - 2) >> 2;          // centroid-column half
+    // Warp (q, h) may read TMEM lane quarter q = warp % 4 (its 32 rows) and
+    // owns accumulator h: it takes the tiles i with i % 2 == h, all columns.
+    // The two warps of a quarter share an SM sub-partition and alternate
+    // tiles, so each decides its rows alone (no exchange between warps).
+    const int q = warp & 3;
+    const int hc = (warp - 2) >> 2;
     const int row = q * 32 + lane;
-    const bool mine = (lane >> 4) == hc;     // rows this thread decides after the merge
-    const int ncol = Npad > 128 ? Npad - 128 : 0;
-    const int cols = hc == 0 ? min(Npad, 128) : ncol;
-    const float kInf = __int_as_float(0x7f800000);
+    const int nch = Npad >> 5;                 // 32-column chunks (>= 1)
     float rn2_next = 0.0f;
     {
-      const int64_t tok = (int64_t)t_begin * kTileM + row;
-      if (mine && tok < p.N) rn2_next = p.rnorm2[(int64_t)u * p.N + tok];
+      const int64_t tok = (int64_t)(t_begin + hc) * kTileM + row;
+      if (hc < ntiles && tok < p.N) rn2_next = p.rnorm2[(int64_t)u * p.N + tok];
     }
-    for (int i = 0; i < ntiles; ++i) {
-      const int acc = i & 1;
+    for (int i = hc; i < ntiles; i += 2) {
+      const int acc = hc;
       const uint32_t aph = (uint32_t)(i >> 1) & 1u;
       const float rn2 = rn2_next;
-      {   // prefetch the next tile's squared row norm
-        const int64_t tok = (int64_t)(t_begin + i + 1) * kTileM + row;
-        if (mine && i + 1 < ntiles && tok < p.N) rn2_next = p.rnorm2[(int64_t)u * p.N + tok];
+      {   // prefetch the squared row norm of this warp's next tile
+        const int64_t tok = (int64_t)(t_begin + i + 2) * kTileM + row;
+        if (i + 2 < ntiles && tok < p.N) rn2_next = p.rnorm2[(int64_t)u * p.N + tok];
       }
       const bool ok = !aborted(bars) && mbar_wait(&bars->tmem_full[acc], aph);
       if (!ok) { TC_DBG(8, i + 1); set_abort(bars); }
       else if (lane == 0 && warp == 2) TC_DBG(18, i + 1);
       tc_fence_after();
       // Top two of h_k = r.c_k - |c_k|^2/2 (the largest h is the nearest
-      // centroid), each value carrying its column index in its 8 low bits;
-      // columns are taken in pairs, four independent chains.  The largest key
-      // of every 32-column chunk is kept too: it tells the exact pass which
-      // chunks can hold a near-tie candidate.
+      // centroid), each value carrying its column index in its 8 low bits.
+      // Columns are taken in quads (top two of the quad by a small network),
+      // merged into four independent chains.  The largest key of every
+      // 32-column chunk is kept too: it tells the exact pass which chunks can
+      // hold a near-tie candidate.  The next chunk's tensor-memory load is in
+      // flight while the current one is processed.
       const float kNegBig = -3.0e38f;
       float c1[4] = {kNegBig, kNegBig, kNegBig, kNegBig}, c2[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
-      float cmax[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
+      float cmax[8];
+#pragma unroll
+      for (int ci = 0; ci < 8; ++ci) cmax[ci] = kNegBig;
       if (ok) {
-        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256 + hc * 128);
+        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
+        uint32_t ra[32], rb[32];
+        tmem_ld32_async(tbase, ra);
+        tmem_wait_ld(ra);
+        auto chunk = [&](const uint32_t (&r)[32], int ci) {
+          const int kb = ci * 32;
+          float m0 = kNegBig, m1 = kNegBig;
 #pragma unroll
-        for (int ci = 0; ci < 4; ++ci) {
-          const int c0 = ci * 32;
-          if (c0 < cols) {
-            uint32_t r[32];
-            tmem_ld32(tbase + (uint32_t)c0, r);
-            const int kb = hc * 128 + c0;
-            float m0 = kNegBig, m1 = kNegBig;
+          for (int e = 0; e < 32; e += 4) {
+            const float ka = key_with_index(__uint_as_float(r[e]), kb + e);
+            const float kb2 = key_with_index(__uint_as_float(r[e + 1]), kb + e + 1);
+            const float kc = key_with_index(__uint_as_float(r[e + 2]), kb + e + 2);
+            const float kd = key_with_index(__uint_as_float(r[e + 3]), kb + e + 3);
+            const float h1 = fmaxf(ka, kb2), l1 = fminf(ka, kb2);
+            const float h2 = fmaxf(kc, kd), l2 = fminf(kc, kd);
+            const float qt = fmaxf(h1, h2);
+            const float qs = max3f(fminf(h1, h2), l1, l2);
+            const int ch = (e >> 2) & 3;
+            c2[ch] = max3f(fminf(c1[ch], qt), c2[ch], qs);
+            c1[ch] = fmaxf(c1[ch], qt);
+            if ((e & 4) == 0) m0 = fmaxf(m0, qt); else m1 = fmaxf(m1, qt);
+          }
+          cmax[ci] = fmaxf(m0, m1);
+        };
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float ka = key_with_index(__uint_as_float(r[e]), kb + e);
-              const float kb2 = key_with_index(__uint_as_float(r[e + 1]), kb + e + 1);
-              const float kc = key_with_index(__uint_as_float(r[e + 2]), kb + e + 2);
-              const float kd = key_with_index(__uint_as_float(r[e + 3]), kb + e + 3);
-              const float hi0 = fmaxf(ka, kb2), lo0 = fminf(ka, kb2);
-              const float hi1 = fmaxf(kc, kd), lo1 = fminf(kc, kd);
-              const int ch0 = (e >> 1) & 3, ch1 = ((e >> 1) + 1) & 3;
-              c2[ch0] = max3f(fminf(c1[ch0], hi0), c2[ch0], lo0);
-              c1[ch0] = fmaxf(c1[ch0], hi0);
-              c2[ch1] = max3f(fminf(c1[ch1], hi1), c2[ch1], lo1);
-              c1[ch1] = fmaxf(c1[ch1], hi1);
-              if ((e & 4) == 0) m0 = max3f(m0, hi0, hi1); else m1 = max3f(m1, hi0, hi1);
-            }
-            cmax[ci] = fmaxf(m0, m1);
+        for (int ci = 0; ci < 8; ci += 2) {
+          if (ci < nch) {
+            if (ci + 1 < nch) tmem_ld32_async(tbase + (uint32_t)((ci + 1) * 32), rb);
+            chunk(ra, ci);
+            tmem_wait_ld(rb);
+          }
+          if (ci + 1 < nch) {
+            if (ci + 2 < nch) tmem_ld32_async(tbase + (uint32_t)((ci + 2) * 32), ra);
+            chunk(rb, ci + 1);
+            tmem_wait_ld(ra);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->tmem_empty[acc]);
-      float v1 = fmaxf(c1[0], c1[1]), v2 = max3f(fminf(c1[0], c1[1]), c2[0], c2[1]);
+      float w1 = fmaxf(c1[0], c1[1]), w2 = max3f(fminf(c1[0], c1[1]), c2[0], c2[1]);
       const float u1 = fmaxf(c1[2], c1[3]), u2 = max3f(fminf(c1[2], c1[3]), c2[2], c2[3]);
-      v2 = max3f(fminf(v1, u1), v2, u2);
-      v1 = fmaxf(v1, u1);
-      float* mb = mbuf + acc * 12 * kTileM;      // [hc][v1, v2, chunk max 0..3][row]
-      mb[(hc * 6 + 0) * kTileM + row] = v1;
-      mb[(hc * 6 + 1) * kTileM + row] = v2;
-#pragma unroll
-      for (int ci = 0; ci < 4; ++ci) mb[(hc * 6 + 2 + ci) * kTileM + row] = cmax[ci];
-      named_bar_sync(1, 256);
-      // each half decides 16 of the warp's 32 rows
-      const int oh = 1 - hc;
-      const float o1 = mb[(oh * 6 + 0) * kTileM + row], o2 = mb[(oh * 6 + 1) * kTileM + row];
-      const float w1 = fmaxf(v1, o1);
-      const float w2 = max3f(fminf(v1, o1), v2, o2);
+      w2 = max3f(fminf(w1, u1), w2, u2);
+      w1 = fmaxf(w1, u1);
       const int64_t tok = (int64_t)(t_begin + i) * kTileM + row;
-      const bool valid = mine && tok < p.N && !aborted(bars);
+      const bool valid = ok && tok < p.N && !aborted(bars);
       const int64_t gi = (int64_t)u * p.N + tok;
       bool flag = false;
       uint32_t chunks = 0;
@@ -459,10 +472,8 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
           const float thr = w1 - margin;
           const float thr_key = thr - 6.2e-5f * (fabsf(w1) + fabsf(thr));
 #pragma unroll
-          for (int ci = 0; ci < 4; ++ci) {
-            if (cmax[ci] >= thr_key) chunks |= 1u << (hc * 4 + ci);
-            if (mb[(oh * 6 + 2 + ci) * kTileM + row] >= thr_key) chunks |= 1u << (oh * 4 + ci);
-          }
+          for (int ci = 0; ci < 8; ++ci)
+            if (cmax[ci] >= thr_key) chunks |= 1u << ci;
         }
       }
       // every lane of the warp takes part in the list append
@@ -524,7 +535,6 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int W, int box_row
 size_t assign_tc_smem_bytes(int K) {
   const int Npad = (K + 31) & ~31;
   return 1024 + 2 * (size_t)Npad * 128 + (size_t)kStages * kAStageBytes + kTileM * 32 + (size_t)Npad * 32 +
-         2 * 12 * kTileM * 4 +
          sizeof(TcSmemBarriers);
 }
 

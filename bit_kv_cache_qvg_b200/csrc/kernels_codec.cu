@@ -310,47 +310,68 @@ __device__ __forceinline__ void minmax8(const float (&r)[8], float& lo, float& h
   hi = max3f(max3f(r[0], r[1], r[2]), max3f(r[3], r[4], r[5]), fmaxf(r[6], r[7]));
 }
 
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float lo_of(uint64_t x) { return __uint_as_float((uint32_t)x); }
+__device__ __forceinline__ float hi_of(uint64_t x) { return __uint_as_float((uint32_t)(x >> 32)); }
+
+// E4M3 code -> value and -> correctly rounded reciprocal (0 where the value
+// is 0 or NaN), built once per block in shared memory.
+struct E4m3Tables {
+  float dec[256];
+  float rcp[256];
+};
+
 // Quantise one 8-channel chunk given its group's (lo, hi); returns the 16-bit
 // packed codes and the scale/zero bytes.  q = clamp(rint(fl((r - m) / s)), 0, 3)
-// with IEEE rounding of the divide.  The quotient is first formed as
-// (r - m) * (1/s), within 3 ulp of fl((r - m) / s).  Clamping to [0, 3]
-// before rounding gives the same code (the boundaries -0.5 and 3.5 clamp to
-// the same code on both sides), and rounding to nearest even is an add and a
-// subtract of 1.5 * 2^23.  Only a clamped quotient that lies within 2^-19 of
-// 0.5, 1.5 or 2.5 can round differently from the exact one; a chunk holding
-// such a value is redone with the correctly rounded divide.  The codes are
-// packed with fused multiply-adds by 4^e, exact in fp32.
-__device__ __forceinline__ uint32_t quant_chunk(const float (&r)[8], float lo, float hi,
+// and s = E4M3(fl(span / 3)), every quotient the IEEE fp32 one: it is formed
+// as q0 = x * y with y = RN(1/divisor), then corrected once,
+// q = fma(fma(-divisor, q0, x), y, q0) (Markstein's method), which returns
+// the IEEE quotient for every E4M3 divisor and every normal quotient (an
+// exhaustive host check covers all fp32 inputs); a subnormal quotient gives
+// code 0 and E4M3 0 either way.  Clamping to [0, 3] before rounding gives the
+// same code (the boundaries -0.5 and 3.5 clamp to the same code on both
+// sides); rounding to nearest even is an add and a subtract of 1.5 * 2^23;
+// the codes are packed with fused multiply-adds by 4^e, exact in fp32.  Pairs
+// of channels go through the packed f32x2 instructions (each lane one IEEE
+// fp32 operation).
+__device__ __forceinline__ uint32_t quant_chunk(const float (&r)[8], float lo, float hi, const E4m3Tables& tab,
                                                 uint8_t& sc_out, uint8_t& zc_out) {
+  constexpr float kThird = 0x1.555556p-2f;  // RN(1/3)
   constexpr float kRound = 12582912.0f;     // 1.5 * 2^23
-  constexpr float kNear = 0.5f - 1.9073486328125e-06f;
   lo = __fadd_rn(lo, 0.0f);                 // -0 -> +0
   hi = __fadd_rn(hi, 0.0f);
   const uint8_t zc = f32_to_e4m3(lo);
-  const float m = e4m3_to_f32(zc);
+  const float m = tab.dec[zc];
   const float span = __fsub_rn(hi, m);
-  const uint8_t scb = f32_to_e4m3(__fdiv_rn(span, 3.0f));
-  const float s = e4m3_to_f32(scb);
+  const float t0 = __fmul_rn(span, kThird);
+  const uint8_t scb = f32_to_e4m3(__fmaf_rn(__fmaf_rn(-3.0f, t0, span), kThird, t0));
+  const float s = tab.dec[scb];
   sc_out = scb;
   zc_out = zc;
   if (s == 0.0f) return 0u;
-  const float inv = __frcp_rn(s);
-  float pk = 0.0f, dev = 0.0f;
+  const float y = tab.rcp[scb];
+  const uint64_t m2 = pack2(m, m), y2 = pack2(y, y), ns2 = pack2(-s, -s), k2 = pack2(kRound, kRound);
+  uint64_t pk2 = 0;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float t = fminf(fmaxf(__fmul_rn(__fsub_rn(r[e], m), inv), 0.0f), 3.0f);
-    const float q = __fsub_rn(__fadd_rn(t, kRound), kRound);
-    dev = fmaxf(dev, fabsf(__fsub_rn(t, q)));
-    pk = __fmaf_rn(q, (float)(1 << (2 * e)), pk);
+  for (int e = 0; e < 8; e += 2) {
+    const uint64_t d2 = sub2(pack2(r[e], r[e + 1]), m2);
+    const uint64_t q02 = mul2(d2, y2);
+    const uint64_t t2 = fma2(fma2(ns2, q02, d2), y2, q02);
+    const float ta = fminf(fmaxf(lo_of(t2), 0.0f), 3.0f);
+    const float tb = fminf(fmaxf(hi_of(t2), 0.0f), 3.0f);
+    const uint64_t q2 = sub2(add2(pack2(ta, tb), k2), k2);
+    pk2 = fma2(q2, pack2((float)(1 << (2 * e)), (float)(1 << (2 * e + 2))), pk2);
   }
-  if (dev > kNear) {                        // rare: a quotient next to a rounding boundary
-    pk = 0.0f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float t = fminf(fmaxf(__fdiv_rn(__fsub_rn(r[e], m), s), 0.0f), 3.0f);
-      pk = __fmaf_rn(__fsub_rn(__fadd_rn(t, kRound), kRound), (float)(1 << (2 * e)), pk);
-    }
-  }
+  const float pk = __fadd_rn(lo_of(pk2), hi_of(pk2));
   return __float_as_uint(__fadd_rn(pk, 8388608.0f)) & 0xFFFFu;   // 2^23: integer in the low bits
 }
 
@@ -367,6 +388,16 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
     uint4* dst = reinterpret_cast<uint4*>(smem);
     const int n16 = p.K * kD * ESZ / 16;
     for (int x = threadIdx.x; x < n16; x += blockDim.x) dst[x] = src[x];
+    __syncthreads();
+  }
+  // E4M3 decode and reciprocal tables for the quantiser
+  __shared__ E4m3Tables s_tab;
+  if (QUANT) {
+    for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+      const float v = e4m3_to_f32((uint8_t)c);
+      s_tab.dec[c] = v;
+      s_tab.rcp[c] = (v == 0.0f || v != v) ? 0.0f : __frcp_rn(v);
+    }
     __syncthreads();
   }
   // largest |value| per channel of the values this pass hands to the next
@@ -445,8 +476,8 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
       lo0 = grp_min(lo0, Gs); hi0 = grp_max(hi0, Gs);
       lo1 = grp_min(lo1, Gs); hi1 = grp_max(hi1, Gs);
       uint8_t s0, z0, s1, z1;
-      const uint32_t q0 = quant_chunk(r0, lo0, hi0, s0, z0);
-      const uint32_t q1 = quant_chunk(r1, lo1, hi1, s1, z1);
+      const uint32_t q0 = quant_chunk(r0, lo0, hi0, s_tab, s0, z0);
+      const uint32_t q1 = quant_chunk(r1, lo1, hi1, s_tab, s1, z1);
       if (!valid) continue;
       const int64_t row = (int64_t)u * p.N + i;
       uint8_t* cr = p.codes + row * (kD / 4);
