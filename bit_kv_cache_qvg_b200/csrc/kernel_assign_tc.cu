@@ -233,9 +233,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
-__device__ __forceinline__ float key_with_index(float g, int k) {
-  return __int_as_float((__float_as_int(g) & ~0xFF) | k);
-}
 
 __global__ void __launch_bounds__(kTcThreads, 1)
 qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmC,
@@ -408,18 +405,27 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
         uint32_t ra[32], rb[32];
         tmem_ld32_async(tbase, ra);
         tmem_wait_ld(ra);
+        // Keys are formed in two steps so that each is one logic operation:
+        // the position within the quad (0-3, held in registers) replaces the
+        // 8 low bits of every value, and the quad's column (a multiple of 4,
+        // an immediate) is or-ed into the quad's maximum only -- the runner-up
+        // value needs no index.
+        uint32_t pos1, pos2, pos3;
+        asm("mov.b32 %0, 1;" : "=r"(pos1));
+        asm("mov.b32 %0, 2;" : "=r"(pos2));
+        asm("mov.b32 %0, 3;" : "=r"(pos3));
         auto chunk = [&](const uint32_t (&r)[32], int ci) {
           const int kb = ci * 32;
           float m0 = kNegBig, m1 = kNegBig;
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
-            const float ka = key_with_index(__uint_as_float(r[e]), kb + e);
-            const float kb2 = key_with_index(__uint_as_float(r[e + 1]), kb + e + 1);
-            const float kc = key_with_index(__uint_as_float(r[e + 2]), kb + e + 2);
-            const float kd = key_with_index(__uint_as_float(r[e + 3]), kb + e + 3);
+            const float ka = __uint_as_float(r[e] & 0xFFFFFF00u);
+            const float kb2 = __uint_as_float((r[e + 1] & 0xFFFFFF00u) | pos1);
+            const float kc = __uint_as_float((r[e + 2] & 0xFFFFFF00u) | pos2);
+            const float kd = __uint_as_float((r[e + 3] & 0xFFFFFF00u) | pos3);
             const float h1 = fmaxf(ka, kb2), l1 = fminf(ka, kb2);
             const float h2 = fmaxf(kc, kd), l2 = fminf(kc, kd);
-            const float qt = fmaxf(h1, h2);
+            const float qt = __uint_as_float(__float_as_uint(fmaxf(h1, h2)) | (uint32_t)(kb + e));
             const float qs = max3f(fminf(h1, h2), l1, l2);
             const int ch = (e >> 2) & 3;
             c2[ch] = max3f(fminf(c1[ch], qt), c2[ch], qs);

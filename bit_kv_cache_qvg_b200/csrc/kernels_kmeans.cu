@@ -268,7 +268,6 @@ constexpr int kScan = 8;              // assignments per thread per scan step (l
 constexpr int kSumThreads = 256;
 constexpr int kSumWarps = kSumThreads / 32;
 constexpr int kSumSlices = 8;         // sum CTAs per block
-constexpr int kSumBatch = 8;          // rows per batch; two batches in flight per warp
 
 // List entry: token (bits 0-22), centroid (23-30), subtract flag (31).
 constexpr uint32_t kEntTok = 0x7FFFFFu;
@@ -316,7 +315,8 @@ __global__ void __launch_bounds__(kBucketThreads, 1)
 qvg_update_bucket(const UpdateParams p) {
   __shared__ int hist[kMaxK];
   __shared__ int dcnt[kMaxK];
-  __shared__ int cursor[kMaxK];
+  __shared__ int cursor[kMaxK];      // next slot for an added row (from the bucket's start, upward)
+  __shared__ int cursor_sub[kMaxK];  // next slot for a removed row (from the bucket's end, downward)
   const int u = blockIdx.x;
   const int K = p.K;
   const int64_t N = p.N;
@@ -336,6 +336,7 @@ qvg_update_bucket(const UpdateParams p) {
 #pragma unroll
     for (int j = 0; j < kScan; ++j) {
       const bool ch = kn[j] != ko[j];
+      if (!__any_sync(0xffffffffu, ch)) continue;   // no entry in these 32 tokens (warp-uniform)
       warp_add(hist, ch ? kn[j] : -1, 1, false);
       if (!full) {
         warp_add(hist, ch ? ko[j] : -1, 1, false);
@@ -362,7 +363,7 @@ qvg_update_bucket(const UpdateParams p) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int k = lane * 8 + i;
-      if (k < K) { cursor[k] = run; off_u[k] = run; }
+      if (k < K) { cursor[k] = run; cursor_sub[k] = -(run + v[i]); off_u[k] = run; }
       run += v[i];
     }
     if (lane == 31) off_u[K] = run;
@@ -377,42 +378,45 @@ qvg_update_bucket(const UpdateParams p) {
 #pragma unroll
     for (int j = 0; j < kScan; ++j) {
       const bool ch = kn[j] != ko[j];
+      if (!__any_sync(0xffffffffu, ch)) continue;   // warp-uniform
       const uint32_t t = (uint32_t)(c + (int64_t)j * blockDim.x + threadIdx.x);
       const int sa = warp_add(cursor, ch ? kn[j] : -1, 1, true);
       if (ch) list[sa] = t | ((uint32_t)kn[j] << kEntKShift);
       if (!full) {
-        const int sb = warp_add(cursor, ch ? ko[j] : -1, 1, true);
+        // cursor_sub holds minus the end of the free region: slot = end - 1 - rank
+        const int sb = -warp_add(cursor_sub, ch ? ko[j] : -1, 1, true) - 1;
         if (ch) list[sb] = t | ((uint32_t)ko[j] << kEntKShift) | kEntSub;
       }
     }
   }
 }
 
-template <int DT> struct RowPart;                 // a lane's 4 channels of a row, raw
-template <> struct RowPart<kBF16> {
-  uint2 w;
-  __device__ __forceinline__ void load(const char* row, int lane) {
-    w = *reinterpret_cast<const uint2*>(row + lane * 8);
-  }
-  __device__ __forceinline__ void get(float (&v)[4]) const {
-    v[0] = __uint_as_float(w.x << 16);
-    v[1] = __uint_as_float(w.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(w.y << 16);
-    v[3] = __uint_as_float(w.y & 0xFFFF0000u);
-  }
-};
-template <> struct RowPart<kFP32> {
-  float4 w;
-  __device__ __forceinline__ void load(const char* row, int lane) {
-    w = *reinterpret_cast<const float4*>(row + lane * 16);
-  }
-  __device__ __forceinline__ void get(float (&v)[4]) const { v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w; }
-};
+__device__ __forceinline__ void cp_async_row(void* smem_dst, const void* gsrc, int bytes) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  if (bytes == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_groups() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Each warp walks its piece of the list with a ring of kSumRing rows in
+// shared memory filled by cp.async (every lane copies, and later reads back,
+// its own 4 channels of each row), so that many rows are in flight without
+// holding registers.  Within a bucket the added rows come first and the
+// removed rows last, so a run (same centroid, same sign) is summed in
+// registers and applied with its sign when it ends.
+constexpr int kSumRing = 16;
 
 template <int DT>
-__global__ void __launch_bounds__(kSumThreads, 2)
+__global__ void __launch_bounds__(kSumThreads, 4)
 qvg_update_sum(const UpdateParams p) {
   constexpr int ESZ = Store<DT>::bytes;
+  constexpr int LANE_BYTES = 4 * ESZ;            // a lane's 4 channels
+  constexpr int ROW = kD * ESZ;
+  extern __shared__ __align__(16) unsigned char smem[];
   const int u = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t N = p.N;
@@ -420,72 +424,80 @@ qvg_update_sum(const UpdateParams p) {
   // this warp's piece of the block's list
   const int64_t part = (int64_t)blockIdx.x * kSumWarps + warp, parts = (int64_t)gridDim.x * kSumWarps;
   const int e0 = (int)(E * part / parts), e1 = (int)(E * (part + 1) / parts);
-  if (e0 >= e1) return;
+  const int n = e1 - e0;
+  if (n <= 0) return;
   float to_fix[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e)
     to_fix[e] = __int_as_float((127 - fix_exponent(p.chmax[(int64_t)u * kD + 4 * lane + e], p.log2n)) << 23);
-  const uint32_t* list = p.list + (int64_t)u * 2 * N;
-  const char* Ru = static_cast<const char*>(p.R) + (int64_t)u * N * kD * ESZ;
+  const uint32_t* list = p.list + (int64_t)u * 2 * N + e0;
+  const char* Ru = static_cast<const char*>(p.R) + (int64_t)u * N * ROW + lane * LANE_BYTES;
+  unsigned char* ring = smem + (size_t)warp * kSumRing * ROW + lane * LANE_BYTES;
   long long* Su = p.S + (int64_t)u * p.K * kD + 4 * lane;
-  const int nb = (e1 - e0 + kSumBatch - 1) / kSumBatch;
-  long long run[4] = {0, 0, 0, 0};
-  int run_k = -1;
-  uint32_t grp = e0 + lane < e1 ? list[e0 + lane] : kEntNone;          // 32 consecutive entries, one per lane
-  uint32_t grp_next = e0 + 32 + lane < e1 ? list[e0 + 32 + lane] : kEntNone;
-  RowPart<DT> ra[kSumBatch], rb[kSumBatch];
-  uint32_t ea[kSumBatch], eb[kSumBatch];
 
-  auto fetch = [&](int b, RowPart<DT>(&rows)[kSumBatch], uint32_t(&ent)[kSumBatch]) {
-    if ((b & 3) == 0 && b > 0) {
-      grp = grp_next;
-      const int nxt = e0 + (b / 4 + 1) * 32 + lane;
-      grp_next = nxt < e1 ? list[nxt] : kEntNone;
-    }
+  // entries in groups of 32 (one per lane); two groups held, the next loaded
+  // one group ahead of the issue pointer
+  uint32_t ge0 = lane < n ? list[lane] : kEntNone;
+  uint32_t ge1 = 32 + lane < n ? list[32 + lane] : kEntNone;
 #pragma unroll
-    for (int r = 0; r < kSumBatch; ++r) {
-      ent[r] = __shfl_sync(0xffffffffu, grp, (b & 3) * 8 + r);
-      if (ent[r] != kEntNone) rows[r].load(Ru + (int64_t)(ent[r] & kEntTok) * kD * ESZ, lane);
+  for (int r = 0; r < kSumRing; ++r) {
+    if (r < n) {
+      const uint32_t ent = __shfl_sync(0xffffffffu, ge0, r);
+      cp_async_row(ring + r * ROW, Ru + (int64_t)(ent & kEntTok) * ROW, LANE_BYTES);
     }
-  };
+    cp_async_commit_group();
+  }
+  long long run[4] = {0, 0, 0, 0};
+  uint32_t run_key = 0xFFFFFFFFu;                 // (centroid, sign) of the open run
   auto flush = [&]() {
-    if (run_k >= 0) {
-      long long* a = Su + (int64_t)run_k * kD;
+    if (run_key != 0xFFFFFFFFu) {
+      long long* a = Su + (int64_t)(run_key & 0xFFu) * kD;
+      const bool neg = (run_key & 0x100u) != 0u;
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        atomicAdd(reinterpret_cast<unsigned long long*>(a + e), (unsigned long long)run[e]);
+        atomicAdd(reinterpret_cast<unsigned long long*>(a + e), (unsigned long long)(neg ? -run[e] : run[e]));
     }
   };
-  auto consume = [&](const RowPart<DT>(&rows)[kSumBatch], const uint32_t(&ent)[kSumBatch]) {
-#pragma unroll
-    for (int r = 0; r < kSumBatch; ++r) {
-      if (ent[r] == kEntNone) break;               // warp-uniform
-      const int k = (int)((ent[r] >> kEntKShift) & 0xFFu);
-      if (k != run_k) {
-        flush();
-        run_k = k;
-        run[0] = run[1] = run[2] = run[3] = 0;
-      }
-      float v[4];
-      rows[r].get(v);
-      const bool neg = (ent[r] & kEntSub) != 0u;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const long long q = __float2ll_rn(__fmul_rn(v[e], to_fix[e]));
-        run[e] += neg ? -q : q;
+  for (int j = 0; j < n; ++j) {
+    cp_async_wait_groups<kSumRing - 1>();
+    if ((j & 31) == 0 && j >= 32) {                // entering group g = j/32: fetch group g+1
+      const int nxt = j + 32 + lane;
+      const uint32_t x = nxt < n ? list[nxt] : kEntNone;
+      if (((j >> 5) + 1) & 1) ge1 = x; else ge0 = x;
+    }
+    const uint32_t ent = __shfl_sync(0xffffffffu, (j >> 5) & 1 ? ge1 : ge0, j & 31);
+    float v[4];
+    {
+      const unsigned char* src = ring + (j % kSumRing) * ROW;
+      if (DT == kBF16) {
+        const uint2 w = *reinterpret_cast<const uint2*>(src);
+        v[0] = __uint_as_float(w.x << 16);
+        v[1] = __uint_as_float(w.x & 0xFFFF0000u);
+        v[2] = __uint_as_float(w.y << 16);
+        v[3] = __uint_as_float(w.y & 0xFFFF0000u);
+      } else {
+        const float4 w = *reinterpret_cast<const float4*>(src);
+        v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
       }
     }
-  };
-  fetch(0, ra, ea);
-  for (int b = 0; b < nb; b += 2) {
-    if (b + 1 < nb) fetch(b + 1, rb, eb);
-    consume(ra, ea);
-    if (b + 1 < nb) {
-      if (b + 2 < nb) fetch(b + 2, ra, ea);
-      consume(rb, eb);
+    const uint32_t key = ent >> kEntKShift;       // centroid and sign
+    if (key != run_key) {                          // warp-uniform
+      flush();
+      run_key = key;
+      run[0] = run[1] = run[2] = run[3] = 0;
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) run[e] += __float2ll_rn(__fmul_rn(v[e], to_fix[e]));
+    // refill the slot just read with the row kSumRing ahead
+    const int ip = j + kSumRing;
+    if (ip < n) {
+      const uint32_t e2 = __shfl_sync(0xffffffffu, (ip >> 5) & 1 ? ge1 : ge0, ip & 31);
+      cp_async_row(ring + (j % kSumRing) * ROW, Ru + (int64_t)(e2 & kEntTok) * ROW, LANE_BYTES);
+    }
+    cp_async_commit_group();
   }
   flush();
+  cp_async_wait_groups<0>();
 }
 
 // A warp per centroid: new count; for a non-empty centroid the mean of the
@@ -597,8 +609,13 @@ cudaError_t launch_update_bucket(const UpdateParams& p, int dtype, cudaStream_t 
 
 cudaError_t launch_update_sum(const UpdateParams& p, int dtype, cudaStream_t s) {
   const dim3 grid((unsigned)kSumSlices, (unsigned)p.W);
-  if (dtype == kBF16) qvg_update_sum<kBF16><<<grid, kSumThreads, 0, s>>>(p);
-  else qvg_update_sum<kFP32><<<grid, kSumThreads, 0, s>>>(p);
+  const size_t smem = (size_t)kSumWarps * kSumRing * kD * (dtype == kBF16 ? 2 : 4);
+  const void* fn = dtype == kBF16 ? reinterpret_cast<const void*>(qvg_update_sum<kBF16>)
+                                  : reinterpret_cast<const void*>(qvg_update_sum<kFP32>);
+  const cudaError_t e = ensure_dynamic_smem(fn, smem);
+  if (e != cudaSuccess) return e;
+  if (dtype == kBF16) qvg_update_sum<kBF16><<<grid, kSumThreads, smem, s>>>(p);
+  else qvg_update_sum<kFP32><<<grid, kSumThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
