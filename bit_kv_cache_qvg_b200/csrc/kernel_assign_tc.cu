@@ -425,7 +425,8 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
             const float kd = __uint_as_float((r[e + 3] & 0xFFFFFF00u) | pos3);
             const float h1 = fmaxf(ka, kb2), l1 = fminf(ka, kb2);
             const float h2 = fmaxf(kc, kd), l2 = fminf(kc, kd);
-            const float qt = __uint_as_float(__float_as_uint(fmaxf(h1, h2)) | (uint32_t)(kb + e));
+            // bits 2-7 of the key are zero here, so adding the quad's column is an or
+            const float qt = __uint_as_float(__float_as_uint(fmaxf(h1, h2)) + (uint32_t)(kb + e));
             const float qs = max3f(fminf(h1, h2), l1, l2);
             const int ch = (e >> 2) & 3;
             c2[ch] = max3f(fminf(c1[ch], qt), c2[ch], qs);

@@ -71,77 +71,73 @@ template <> struct Vec8<kFP32> {
 };
 
 // ---------------------------------------------------------------- packed pairs
-// Two fp32 values in one 64-bit register, operated on with the f32x2
-// instructions (each lane of the pair rounded as a separate fp32 operation).
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-  return ((uint64_t)__float_as_uint(hi) << 32) | (uint64_t)__float_as_uint(lo);
+// Two fp32 values operated on with the f32x2 instructions (float2 intrinsics:
+// each lane of the pair is rounded as a separate IEEE fp32 operation).
+__device__ __forceinline__ float2 f2(float lo, float hi) { return make_float2(lo, hi); }
+// the two bf16 values of a 32-bit word (low half first) as fp32
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-template <int DT> struct Pair4;
-template <> struct Pair4<kBF16> {
-  // y[e] += channels (2e, 2e+1) of 8 bf16 centroid values
-  __device__ static __forceinline__ void add(const void* p, uint64_t (&y)[4]) {
-    const uint4 w = *reinterpret_cast<const uint4*>(p);
-    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) y[e] = add2(y[e], ((uint64_t)(x[e] & 0xFFFF0000u) << 32) | (uint64_t)(x[e] << 16));
+
+// ---------------------------------------------------------------- dequant
+// Eight lanes per token: lane l of the eight owns channels 8l..8l+7 and
+// 64+8l..64+8l+7 (bytes 2l, 2l+1, 16+2l, 17+2l of the token's 32-byte code
+// row); for each centroid row the eight lanes read 128 contiguous bytes per
+// half, so the shared-memory tables are read without bank conflicts, and
+// they write two coalesced 128-byte halves of the output row.  Each group of
+// eight lanes walks kDqU tokens per step and loads the next step's codes,
+// scale/zero bytes and assignments while it computes the current one.  E4M3
+// bytes are decoded through a 256-entry shared table; a nibble of codes (two
+// channels) maps to a pair of floats through a 16-entry table.
+constexpr int kDqThreads = 768;
+constexpr int kDqWarps = kDqThreads / 32;
+constexpr int kDqStreams = 4 * kDqWarps;        // token streams per block (8 lanes each)
+
+// tokens per half-warp per step (fewer when more assignment bytes are in flight)
+template <int TT> constexpr int dq_unroll() { return (TT < 0 || TT >= 3) ? 2 : 4; }
+
+template <int DT> struct Oct;                   // a lane's 8 channels of a row
+template <> struct Oct<kBF16> {
+  __device__ static __forceinline__ void add(const char* row, float2 (&y)[4]) {
+    const uint4 w = *reinterpret_cast<const uint4*>(row);
+    y[0] = __fadd2_rn(y[0], bf16x2_to_f2(w.x));
+    y[1] = __fadd2_rn(y[1], bf16x2_to_f2(w.y));
+    y[2] = __fadd2_rn(y[2], bf16x2_to_f2(w.z));
+    y[3] = __fadd2_rn(y[3], bf16x2_to_f2(w.w));
   }
-  __device__ static __forceinline__ void store(void* p, const uint64_t (&y)[4]) {
+  __device__ static __forceinline__ void store(char* row, const float2 (&y)[4]) {
     uint32_t x[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float((uint32_t)y[e]), __uint_as_float((uint32_t)(y[e] >> 32)));
+      const __nv_bfloat162 b = __float22bfloat162_rn(y[e]);
       x[e] = *reinterpret_cast<const uint32_t*>(&b);
     }
-    *reinterpret_cast<uint4*>(p) = make_uint4(x[0], x[1], x[2], x[3]);
+    *reinterpret_cast<uint4*>(row) = make_uint4(x[0], x[1], x[2], x[3]);
   }
 };
-template <> struct Pair4<kFP32> {
-  __device__ static __forceinline__ void add(const void* p, uint64_t (&y)[4]) {
-    const ulonglong2 a = reinterpret_cast<const ulonglong2*>(p)[0];
-    const ulonglong2 b = reinterpret_cast<const ulonglong2*>(p)[1];
-    y[0] = add2(y[0], a.x); y[1] = add2(y[1], a.y); y[2] = add2(y[2], b.x); y[3] = add2(y[3], b.y);
+template <> struct Oct<kFP32> {
+  __device__ static __forceinline__ void add(const char* row, float2 (&y)[4]) {
+    const float4 a = reinterpret_cast<const float4*>(row)[0];
+    const float4 b = reinterpret_cast<const float4*>(row)[1];
+    y[0] = __fadd2_rn(y[0], f2(a.x, a.y));
+    y[1] = __fadd2_rn(y[1], f2(a.z, a.w));
+    y[2] = __fadd2_rn(y[2], f2(b.x, b.y));
+    y[3] = __fadd2_rn(y[3], f2(b.z, b.w));
   }
-  __device__ static __forceinline__ void store(void* p, const uint64_t (&y)[4]) {
-    reinterpret_cast<ulonglong2*>(p)[0] = make_ulonglong2(y[0], y[1]);
-    reinterpret_cast<ulonglong2*>(p)[1] = make_ulonglong2(y[2], y[3]);
+  __device__ static __forceinline__ void store(char* row, const float2 (&y)[4]) {
+    reinterpret_cast<float4*>(row)[0] = make_float4(y[0].x, y[0].y, y[1].x, y[1].y);
+    reinterpret_cast<float4*>(row)[1] = make_float4(y[2].x, y[2].y, y[3].x, y[3].y);
   }
 };
 
-// ---------------------------------------------------------------- dequant
-constexpr int kDqThreads = 512;
-constexpr int kDqTokPerIter = kDqThreads / 8;   // 64 tokens per block row of threads
-constexpr int kDqUnroll = 4;                    // tokens per thread per tile
-constexpr int kDqTile = kDqTokPerIter * kDqUnroll;   // 256 tokens per tile
-constexpr int kDqStages = 3;                    // codes ring depth
-constexpr int kDqTileBytes = kDqTile * (kD / 4);     // 8 KB of codes per tile
-
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                   static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
-               "l"(gsrc)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// TT = number of stages when it is <= 4 (the tile's assignments are fetched
-// one tile ahead into registers), or -1 for the generic runtime-T loop.
+// TT = number of stages when it is <= 4 (assignments fetched a step ahead
+// with the codes), or -1 for the generic runtime-T loop.
 template <int DT, int TT>
-__global__ void __launch_bounds__(kDqThreads)
+__global__ void __launch_bounds__(kDqThreads, 1)
 qvg_dequant_fused(const DequantParams p, const int splits) {
   constexpr int ESZ = Store<DT>::bytes;
   constexpr int TR = TT <= 0 ? 1 : TT;
+  constexpr int kDqU = dq_unroll<TT>();
   extern __shared__ __align__(16) unsigned char smem[];
 
   const int unit = blockIdx.x / splits;
@@ -160,121 +156,125 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
   const int64_t tab_elems = (int64_t)K * kD;
   const size_t tab_bytes = (size_t)tab_elems * ESZ;
   const char* tables = static_cast<const char*>(p.centroids) + (int64_t)c * T * p.H * tab_elems * ESZ;
-  uint8_t* cring = smem + (size_t)p.t_smem * tab_bytes;       // codes ring (16-byte aligned)
-  // byte of four 2-bit codes -> the four codes as floats (channel order)
-  float4* qlut = reinterpret_cast<float4*>(cring + kDqStages * kDqTileBytes);
-  if (threadIdx.x < 256) {
-    const uint32_t b = threadIdx.x;
-    qlut[b] = make_float4((float)(b & 3u), (float)((b >> 2) & 3u), (float)((b >> 4) & 3u), (float)(b >> 6));
-  }
-
-  const int j = threadIdx.x & 7;
-  const int tl = threadIdx.x >> 3;
-  const int ng = kD / G;
-  const int g0 = (8 * j) / G, g1 = (64 + 8 * j) / G;
-  const int64_t row0 = (int64_t)p.H * o_c + (int64_t)h * n_c;
-  const uint8_t* codes = p.codes + row0 * (kD / 4);
-  const uint8_t* sc = p.scale + row0 * ng;
-  const uint8_t* zr = p.zero + row0 * ng;
-  const uint8_t* asg = p.assign + (int64_t)T * p.H * o_c + (int64_t)h * n_c;
-  const int64_t asg_t = (int64_t)p.H * n_c;
-  char* Y = static_cast<char*>(p.Y) + ((int64_t)h * p.y_head_stride + o_c) * kD * ESZ;
-  const int64_t ntile = i_end > i_begin ? (i_end - i_begin + kDqTile - 1) / kDqTile : 0;
-  if (ntile == 0) return;                                     // uniform over the block
-
-  // codes of tile t -> ring slot t % kDqStages: one 16-byte async copy per thread
-  auto issue = [&](int64_t t) {
-    if (t < ntile) {
-      const int64_t tok0 = i_begin + t * kDqTile;
-      const int64_t nbytes = min((int64_t)kDqTile, i_end - tok0) * (kD / 4);
-      if ((int64_t)threadIdx.x * 16 < nbytes)
-        cp_async16(cring + (t % kDqStages) * kDqTileBytes + threadIdx.x * 16,
-                   codes + tok0 * (kD / 4) + threadIdx.x * 16);
-    }
-    cp_async_commit();
-  };
-  issue(0);
-  issue(1);
-
-  // Stage the first t_smem tables of this (chunk, head) in shared memory.
+  float* dec = reinterpret_cast<float*>(smem + (size_t)p.t_smem * tab_bytes);   // E4M3 byte -> value
+  float2* nlut = reinterpret_cast<float2*>(dec + 256);                          // nibble -> two codes
+  if (i_end <= i_begin) return;                                                 // uniform over the block
+  for (int x = threadIdx.x; x < 256; x += blockDim.x) dec[x] = e4m3_to_f32((uint8_t)x);
+  if (threadIdx.x < 16) nlut[threadIdx.x] = make_float2((float)(threadIdx.x & 3u), (float)(threadIdx.x >> 2));
   for (int t = 0; t < p.t_smem; ++t) {
     const uint4* src = reinterpret_cast<const uint4*>(tables + ((int64_t)t * p.H + h) * tab_bytes);
     uint4* dst = reinterpret_cast<uint4*>(smem + (size_t)t * tab_bytes);
     const int n16 = (int)(tab_bytes / 16);
     for (int x = threadIdx.x; x < n16; x += blockDim.x) dst[x] = src[x];
   }
+  __syncthreads();
 
-  // per-token bytes of a tile: scale/zero of both groups, assignments (TT <= 4)
-  uint32_t sz[kDqUnroll], ka[kDqUnroll];
-  auto fetch_small = [&](int64_t t, uint32_t (&s_out)[kDqUnroll], uint32_t (&k_out)[kDqUnroll]) {
+  const int ql = threadIdx.x & 7;                // lane within the token's eight
+  const int stream = threadIdx.x >> 3;           // this group's token stream
+  const int ng = kD / G;
+  const int g0 = (8 * ql) / G, g1 = (64 + 8 * ql) / G;   // groups of the two 8-channel halves
+  const int nt = (int)(i_end - i_begin);         // tokens of this block (< 2^31)
+  const int64_t row0 = (int64_t)p.H * o_c + (int64_t)h * n_c + i_begin;
+  // per-lane base pointers; a token t of the block is an int offset from them
+  const uint16_t* cbp = reinterpret_cast<const uint16_t*>(p.codes + row0 * (kD / 4)) + ql;
+  const uint8_t* scp = p.scale + row0 * ng;
+  const uint8_t* zrp = p.zero + row0 * ng;
+  const uint8_t* ap = p.assign + (int64_t)T * p.H * o_c + (int64_t)h * n_c + i_begin;
+  const int64_t asg_t = (int64_t)p.H * n_c;
+  char* yp = static_cast<char*>(p.Y) + ((int64_t)h * p.y_head_stride + o_c + i_begin) * kD * ESZ + 8 * ql * ESZ;
+  const int step = kDqStreams * kDqU;
+
+  // codes (two 16-bit words), scale/zero bytes of both halves and (TT > 0)
+  // assignments of tokens t0..t0+kDqU-1 (past the block's end: token 0 again;
+  // nothing is stored for those)
+  auto load = [&](int t0, uint32_t (&cb)[kDqU], uint32_t (&sz)[kDqU], uint32_t (&ka)[kDqU]) {
 #pragma unroll
-    for (int u = 0; u < kDqUnroll; ++u) {
-      int64_t i = i_begin + t * kDqTile + tl + u * kDqTokPerIter;
-      if (t >= ntile || i >= i_end) i = i_begin;
-      s_out[u] = (uint32_t)sc[i * ng + g0] | ((uint32_t)zr[i * ng + g0] << 8) |
-                 ((uint32_t)sc[i * ng + g1] << 16) | ((uint32_t)zr[i * ng + g1] << 24);
+    for (int u = 0; u < kDqU; ++u) {
+      const int t = t0 + u < nt ? t0 + u : 0;
+      cb[u] = (uint32_t)cbp[t * (kD / 8)] | ((uint32_t)cbp[t * (kD / 8) + 8] << 16);
+      sz[u] = (uint32_t)scp[t * ng + g0] | ((uint32_t)zrp[t * ng + g0] << 8) |
+              ((uint32_t)scp[t * ng + g1] << 16) | ((uint32_t)zrp[t * ng + g1] << 24);
       uint32_t kw = 0;
       if (TT > 0) {
 #pragma unroll
-        for (int tt = 0; tt < TR; ++tt) kw |= (uint32_t)asg[tt * asg_t + i] << (8 * tt);
+        for (int tt = 0; tt < TR; ++tt) kw |= (uint32_t)ap[tt * asg_t + t] << (8 * tt);
       }
-      k_out[u] = kw;
+      ka[u] = kw;
     }
   };
-  fetch_small(0, sz, ka);
-
-  for (int64_t t = 0; t < ntile; ++t) {
-    issue(t + 2);
-    cp_async_wait<2>();          // this thread's copies of tile t have landed
-    __syncthreads();             // everyone's have (and the tables are staged)
-    uint32_t sz_n[kDqUnroll], ka_n[kDqUnroll];
-    fetch_small(t + 1, sz_n, ka_n);
-    const uint8_t* ct = cring + (t % kDqStages) * kDqTileBytes;
+  uint32_t cb[kDqU], sz[kDqU], ka[kDqU];
+  int t0 = stream * kDqU;
+  load(t0, cb, sz, ka);
+  for (; t0 < nt; t0 += step) {
+    uint32_t cb_n[kDqU], sz_n[kDqU], ka_n[kDqU];
+    load(t0 + step, cb_n, sz_n, ka_n);
 #pragma unroll
-    for (int u = 0; u < kDqUnroll; ++u) {
-      const int r = tl + u * kDqTokPerIter;                // token within the tile
-      const int64_t tok = i_begin + t * kDqTile + r;
-      const uint32_t q0 = *reinterpret_cast<const uint16_t*>(ct + r * (kD / 4) + 2 * j);
-      const uint32_t q1 = *reinterpret_cast<const uint16_t*>(ct + r * (kD / 4) + 16 + 2 * j);
-      const float s0 = e4m3_to_f32((uint8_t)(sz[u] & 0xFF)), m0 = e4m3_to_f32((uint8_t)((sz[u] >> 8) & 0xFF));
-      const float s1 = e4m3_to_f32((uint8_t)((sz[u] >> 16) & 0xFF)), m1 = e4m3_to_f32((uint8_t)(sz[u] >> 24));
+    for (int u = 0; u < kDqU; ++u) {
+      const int t = t0 + u;
       // y = s*q + m (exact in fp32: E4M3 operands, q <= 3), two channels per op
-      uint64_t y0[4], y1[4];
-      const uint64_t s0p = pack2(s0, s0), m0p = pack2(m0, m0), s1p = pack2(s1, s1), m1p = pack2(m1, m1);
+      float2 y0[4], y1[4];
+      {
+        const float s0 = dec[sz[u] & 0xFFu], m0 = dec[(sz[u] >> 8) & 0xFFu];
+        const float s1 = dec[(sz[u] >> 16) & 0xFFu], m1 = dec[sz[u] >> 24];
+        const float2 sp0 = f2(s0, s0), mp0 = f2(m0, m0), sp1 = f2(s1, s1), mp1 = f2(m1, m1);
 #pragma unroll
-      for (int bq = 0; bq < 2; ++bq) {
-        const float4 a = qlut[(q0 >> (8 * bq)) & 0xFFu];
-        const float4 b = qlut[(q1 >> (8 * bq)) & 0xFFu];
-        y0[2 * bq] = fma2(s0p, pack2(a.x, a.y), m0p);
-        y0[2 * bq + 1] = fma2(s0p, pack2(a.z, a.w), m0p);
-        y1[2 * bq] = fma2(s1p, pack2(b.x, b.y), m1p);
-        y1[2 * bq + 1] = fma2(s1p, pack2(b.z, b.w), m1p);
+        for (int e = 0; e < 4; ++e) {
+          y0[e] = __ffma2_rn(sp0, nlut[(cb[u] >> (4 * e)) & 0xFu], mp0);
+          y1[e] = __ffma2_rn(sp1, nlut[(cb[u] >> (16 + 4 * e)) & 0xFu], mp1);
+        }
       }
-      const int64_t ii = tok < i_end ? tok : i_begin;
       // centroids of stage T, T-1, ..., 1, in that order
 #pragma unroll
       for (int tt = 0; tt < (TT < 0 ? kMaxT : (TT == 0 ? 0 : TR)); ++tt) {
         const int st = T - 1 - tt;
         if (TT < 0 && st < 0) break;
-        int k = TT > 0 ? (int)((ka[u] >> (8 * st)) & 0xFF) : (int)asg[st * asg_t + ii];
-        k = k < K ? k : K - 1;
-        const char* rowp = (st < p.t_smem)
-            ? reinterpret_cast<const char*>(smem) + ((int64_t)st * tab_elems + (int64_t)k * kD) * ESZ
-            : tables + (((int64_t)st * p.H + h) * tab_elems + (int64_t)k * kD) * ESZ;
-        Pair4<DT>::add(rowp + 8 * j * ESZ, y0);
-        Pair4<DT>::add(rowp + (64 + 8 * j) * ESZ, y1);
+        int k = TT > 0 ? (int)((ka[u] >> (8 * st)) & 0xFFu) : (int)ap[st * asg_t + (t < nt ? t : 0)];
+        k = min(k, K - 1);
+        // shared and global rows on separate paths, so that the shared one is
+        // addressed as shared memory (st < t_smem is uniform over the block)
+        if (st < p.t_smem) {
+          const char* r = reinterpret_cast<const char*>(smem) + (st * (int)tab_elems + k * kD + 8 * ql) * ESZ;
+          Oct<DT>::add(r, y0);
+          Oct<DT>::add(r + 64 * ESZ, y1);
+        } else {
+          const char* r = tables + (((int64_t)st * p.H + h) * tab_elems + (int64_t)k * kD + 8 * ql) * ESZ;
+          Oct<DT>::add(r, y0);
+          Oct<DT>::add(r + 64 * ESZ, y1);
+        }
       }
-      if (tok < i_end) {
-        char* yr = Y + tok * kD * ESZ;
-        Pair4<DT>::store(yr + 8 * j * ESZ, y0);
-        Pair4<DT>::store(yr + (64 + 8 * j) * ESZ, y1);
+      if (t < nt) {
+        char* yr = yp + (int64_t)t * (kD * ESZ);
+        Oct<DT>::store(yr, y0);
+        Oct<DT>::store(yr + 64 * ESZ, y1);
       }
     }
 #pragma unroll
-    for (int u = 0; u < kDqUnroll; ++u) { sz[u] = sz_n[u]; ka[u] = ka_n[u]; }
-    __syncthreads();             // ring slot t % kDqStages is free again
+    for (int u = 0; u < kDqU; ++u) { cb[u] = cb_n[u]; sz[u] = sz_n[u]; ka[u] = ka_n[u]; }
   }
-  cp_async_wait<0>();
+}
+
+template <int DT>
+static cudaError_t launch_dq_t(const DequantParams& p, int blocks, int splits, size_t smem, cudaStream_t s) {
+  const void* fn;
+  switch (p.T) {
+    case 0: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 0>); break;
+    case 1: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 1>); break;
+    case 2: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 2>); break;
+    case 3: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 3>); break;
+    case 4: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 4>); break;
+    default: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, -1>); break;
+  }
+  cudaError_t e = ensure_dynamic_smem(fn, smem);
+  if (e != cudaSuccess) return e;
+  switch (p.T) {
+    case 0: qvg_dequant_fused<DT, 0><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+    case 1: qvg_dequant_fused<DT, 1><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+    case 2: qvg_dequant_fused<DT, 2><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+    case 3: qvg_dequant_fused<DT, 3><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+    case 4: qvg_dequant_fused<DT, 4><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+    default: qvg_dequant_fused<DT, -1><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+  }
+  return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- residual / quant
@@ -309,19 +309,6 @@ __device__ __forceinline__ void minmax8(const float (&r)[8], float& lo, float& h
   lo = min3f(min3f(r[0], r[1], r[2]), min3f(r[3], r[4], r[5]), fminf(r[6], r[7]));
   hi = max3f(max3f(r[0], r[1], r[2]), max3f(r[3], r[4], r[5]), fmaxf(r[6], r[7]));
 }
-
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ float lo_of(uint64_t x) { return __uint_as_float((uint32_t)x); }
-__device__ __forceinline__ float hi_of(uint64_t x) { return __uint_as_float((uint32_t)(x >> 32)); }
 
 // E4M3 code -> value and -> correctly rounded reciprocal (0 where the value
 // is 0 or NaN), built once per block in shared memory.
@@ -359,19 +346,18 @@ __device__ __forceinline__ uint32_t quant_chunk(const float (&r)[8], float lo, f
   zc_out = zc;
   if (s == 0.0f) return 0u;
   const float y = tab.rcp[scb];
-  const uint64_t m2 = pack2(m, m), y2 = pack2(y, y), ns2 = pack2(-s, -s), k2 = pack2(kRound, kRound);
-  uint64_t pk2 = 0;
+  const float2 nm2 = f2(-m, -m), y2 = f2(y, y), ns2 = f2(-s, -s), k2 = f2(kRound, kRound), nk2 = f2(-kRound, -kRound);
+  float2 pk2 = f2(0.0f, 0.0f);
 #pragma unroll
   for (int e = 0; e < 8; e += 2) {
-    const uint64_t d2 = sub2(pack2(r[e], r[e + 1]), m2);
-    const uint64_t q02 = mul2(d2, y2);
-    const uint64_t t2 = fma2(fma2(ns2, q02, d2), y2, q02);
-    const float ta = fminf(fmaxf(lo_of(t2), 0.0f), 3.0f);
-    const float tb = fminf(fmaxf(hi_of(t2), 0.0f), 3.0f);
-    const uint64_t q2 = sub2(add2(pack2(ta, tb), k2), k2);
-    pk2 = fma2(q2, pack2((float)(1 << (2 * e)), (float)(1 << (2 * e + 2))), pk2);
+    const float2 d2 = __fadd2_rn(f2(r[e], r[e + 1]), nm2);
+    const float2 q02 = __fmul2_rn(d2, y2);
+    const float2 t2 = __ffma2_rn(__ffma2_rn(ns2, q02, d2), y2, q02);
+    const float2 tc = f2(fminf(fmaxf(t2.x, 0.0f), 3.0f), fminf(fmaxf(t2.y, 0.0f), 3.0f));
+    const float2 q2 = __fadd2_rn(__fadd2_rn(tc, k2), nk2);
+    pk2 = __ffma2_rn(q2, f2((float)(1 << (2 * e)), (float)(1 << (2 * e + 2))), pk2);
   }
-  const float pk = __fadd_rn(lo_of(pk2), hi_of(pk2));
+  const float pk = __fadd_rn(pk2.x, pk2.y);
   return __float_as_uint(__fadd_rn(pk, 8388608.0f)) & 0xFFFFu;   // 2^23: integer in the low bits
 }
 
@@ -554,37 +540,19 @@ cudaError_t set_smem(F* f, size_t bytes) {
 
 }  // namespace
 
-template <int DT, int TT>
-static cudaError_t launch_dq(const DequantParams& p, int blocks, int splits, size_t smem, cudaStream_t s) {
-  cudaError_t e = set_smem(qvg_dequant_fused<DT, TT>, smem);
-  if (e != cudaSuccess) return e;
-  qvg_dequant_fused<DT, TT><<<blocks, kDqThreads, smem, s>>>(p, splits);
-  return cudaGetLastError();
-}
-
-template <int DT>
-static cudaError_t launch_dq_t(const DequantParams& p, int blocks, int splits, size_t smem, cudaStream_t s) {
-  switch (p.T) {
-    case 0: return launch_dq<DT, 0>(p, blocks, splits, smem, s);
-    case 1: return launch_dq<DT, 1>(p, blocks, splits, smem, s);
-    case 2: return launch_dq<DT, 2>(p, blocks, splits, smem, s);
-    case 3: return launch_dq<DT, 3>(p, blocks, splits, smem, s);
-    case 4: return launch_dq<DT, 4>(p, blocks, splits, smem, s);
-    default: return launch_dq<DT, -1>(p, blocks, splits, smem, s);
-  }
-}
-
 cudaError_t launch_dequant(const DequantParams& p, int dtype, cudaStream_t s) {
   const int esz = dtype == kBF16 ? 2 : 4;
-  const size_t smem = (size_t)p.t_smem * p.K * kD * esz + (size_t)kDqStages * kDqTileBytes + 256 * 16;
+  const size_t smem = (size_t)p.t_smem * p.K * kD * esz + 256 * sizeof(float) + 16 * sizeof(float2);
   const int units = p.n_chunks * p.H;
   if (units == 0) return cudaSuccess;
   const int sms = device_sm_count();
-  // split blocks along tokens until the grid covers the GPU at least twice
-  int splits = (2 * sms + units - 1) / units;
+  // One resident block per SM: split blocks along tokens until the grid is
+  // about four waves, so that the last one is short and every block stages
+  // its tables once for a few thousand tokens.
+  int splits = (4 * sms + units - 1) / units;
   const int64_t ntok = p.chunk_off ? 0 : p.N;
   if (ntok > 0) {
-    const int64_t max_splits = (ntok + 255) / 256;
+    const int64_t max_splits = (ntok + 1023) / 1024;
     if (splits > max_splits) splits = (int)max_splits;
   } else if (splits > 8) {
     splits = 8;

@@ -402,23 +402,26 @@ __device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async
 template <int N>
 __device__ __forceinline__ void cp_async_wait_groups() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Each warp walks its piece of the list with a ring of kSumRing rows in
+// Each warp walks its piece of the list two rows at a time, one per
+// half-warp (16 lanes x 8 channels), with a ring of kSumRing row pairs in
 // shared memory filled by cp.async (every lane copies, and later reads back,
-// its own 4 channels of each row), so that many rows are in flight without
+// its own 8 channels of a row), so that many rows are in flight without
 // holding registers.  Within a bucket the added rows come first and the
 // removed rows last, so a run (same centroid, same sign) is summed in
-// registers and applied with its sign when it ends.
+// registers and applied with its sign when it ends; each half-warp keeps its
+// own run.
 constexpr int kSumRing = 16;
 
 template <int DT>
-__global__ void __launch_bounds__(kSumThreads, 4)
+__global__ void __launch_bounds__(kSumThreads, 3)
 qvg_update_sum(const UpdateParams p) {
   constexpr int ESZ = Store<DT>::bytes;
-  constexpr int LANE_BYTES = 4 * ESZ;            // a lane's 4 channels
+  constexpr int LANE_BYTES = 8 * ESZ;            // a lane's 8 channels
   constexpr int ROW = kD * ESZ;
   extern __shared__ __align__(16) unsigned char smem[];
   const int u = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = lane >> 4, hl = lane & 15;    // row of the pair, lane within the half
   const int64_t N = p.N;
   const int E = p.off[(int64_t)u * (p.K + 1) + p.K];
   // this warp's piece of the block's list
@@ -426,74 +429,90 @@ qvg_update_sum(const UpdateParams p) {
   const int e0 = (int)(E * part / parts), e1 = (int)(E * (part + 1) / parts);
   const int n = e1 - e0;
   if (n <= 0) return;
-  float to_fix[4];
+  const int npairs = (n + 1) >> 1;
+  float to_fix[8];
 #pragma unroll
-  for (int e = 0; e < 4; ++e)
-    to_fix[e] = __int_as_float((127 - fix_exponent(p.chmax[(int64_t)u * kD + 4 * lane + e], p.log2n)) << 23);
+  for (int e = 0; e < 8; ++e)
+    to_fix[e] = __int_as_float((127 - fix_exponent(p.chmax[(int64_t)u * kD + 8 * hl + e], p.log2n)) << 23);
   const uint32_t* list = p.list + (int64_t)u * 2 * N + e0;
-  const char* Ru = static_cast<const char*>(p.R) + (int64_t)u * N * ROW + lane * LANE_BYTES;
-  unsigned char* ring = smem + (size_t)warp * kSumRing * ROW + lane * LANE_BYTES;
-  long long* Su = p.S + (int64_t)u * p.K * kD + 4 * lane;
+  const char* Ru = static_cast<const char*>(p.R) + (int64_t)u * N * ROW + hl * LANE_BYTES;
+  unsigned char* ring = smem + (size_t)warp * kSumRing * 2 * ROW + half * ROW + hl * LANE_BYTES;
+  long long* Su = p.S + (int64_t)u * p.K * kD + 8 * hl;
 
-  // entries in groups of 32 (one per lane); two groups held, the next loaded
-  // one group ahead of the issue pointer
+  // entries in groups of 32 (16 pairs), one per lane; two groups held, the
+  // next loaded one group ahead of the issue pointer
   uint32_t ge0 = lane < n ? list[lane] : kEntNone;
   uint32_t ge1 = 32 + lane < n ? list[32 + lane] : kEntNone;
+  auto issue = [&](int jp, int slot) {           // rows 2jp and 2jp+1 into ring slot
+    const int r = 2 * jp + half;                  // this half's row (entry index)
+    const uint32_t ent = __shfl_sync(0xffffffffu, (r >> 5) & 1 ? ge1 : ge0, r & 31);
+    if (r < n) {
+      const char* src = Ru + (int64_t)(ent & kEntTok) * ROW;
+      unsigned char* dst = ring + slot * 2 * ROW;
+      if (DT == kBF16) {
+        cp_async_row(dst, src, 16);
+      } else {
+        cp_async_row(dst, src, 16);
+        cp_async_row(dst + 16, src + 16, 16);
+      }
+    }
+  };
 #pragma unroll
   for (int r = 0; r < kSumRing; ++r) {
-    if (r < n) {
-      const uint32_t ent = __shfl_sync(0xffffffffu, ge0, r);
-      cp_async_row(ring + r * ROW, Ru + (int64_t)(ent & kEntTok) * ROW, LANE_BYTES);
-    }
+    if (r < npairs) issue(r, r);
     cp_async_commit_group();
   }
-  long long run[4] = {0, 0, 0, 0};
-  uint32_t run_key = 0xFFFFFFFFu;                 // (centroid, sign) of the open run
+  long long run[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) run[e] = 0;
+  uint32_t run_key = 0xFFFFFFFFu;                 // (centroid, sign) of this half's open run
   auto flush = [&]() {
     if (run_key != 0xFFFFFFFFu) {
       long long* a = Su + (int64_t)(run_key & 0xFFu) * kD;
       const bool neg = (run_key & 0x100u) != 0u;
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
+      for (int e = 0; e < 8; ++e)
         atomicAdd(reinterpret_cast<unsigned long long*>(a + e), (unsigned long long)(neg ? -run[e] : run[e]));
     }
   };
-  for (int j = 0; j < n; ++j) {
+  for (int jp = 0; jp < npairs; ++jp) {
     cp_async_wait_groups<kSumRing - 1>();
-    if ((j & 31) == 0 && j >= 32) {                // entering group g = j/32: fetch group g+1
-      const int nxt = j + 32 + lane;
+    if ((jp & 15) == 0 && jp >= 16) {              // entering group g = jp/16: fetch group g+1
+      const int nxt = 2 * jp + 32 + lane;
       const uint32_t x = nxt < n ? list[nxt] : kEntNone;
-      if (((j >> 5) + 1) & 1) ge1 = x; else ge0 = x;
+      if (((jp >> 4) + 1) & 1) ge1 = x; else ge0 = x;
     }
-    const uint32_t ent = __shfl_sync(0xffffffffu, (j >> 5) & 1 ? ge1 : ge0, j & 31);
-    float v[4];
-    {
-      const unsigned char* src = ring + (j % kSumRing) * ROW;
+    const int r = 2 * jp + half;
+    const uint32_t ent = __shfl_sync(0xffffffffu, (r >> 5) & 1 ? ge1 : ge0, r & 31);
+    const int slot = jp % kSumRing;
+    if (r < n) {
+      float v[8];
+      const unsigned char* src = ring + slot * 2 * ROW;
       if (DT == kBF16) {
-        const uint2 w = *reinterpret_cast<const uint2*>(src);
-        v[0] = __uint_as_float(w.x << 16);
-        v[1] = __uint_as_float(w.x & 0xFFFF0000u);
-        v[2] = __uint_as_float(w.y << 16);
-        v[3] = __uint_as_float(w.y & 0xFFFF0000u);
-      } else {
-        const float4 w = *reinterpret_cast<const float4*>(src);
-        v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
-      }
-    }
-    const uint32_t key = ent >> kEntKShift;       // centroid and sign
-    if (key != run_key) {                          // warp-uniform
-      flush();
-      run_key = key;
-      run[0] = run[1] = run[2] = run[3] = 0;
-    }
+        const uint4 w = *reinterpret_cast<const uint4*>(src);
+        const uint32_t x[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) run[e] += __float2ll_rn(__fmul_rn(v[e], to_fix[e]));
-    // refill the slot just read with the row kSumRing ahead
-    const int ip = j + kSumRing;
-    if (ip < n) {
-      const uint32_t e2 = __shfl_sync(0xffffffffu, (ip >> 5) & 1 ? ge1 : ge0, ip & 31);
-      cp_async_row(ring + (j % kSumRing) * ROW, Ru + (int64_t)(e2 & kEntTok) * ROW, LANE_BYTES);
+        for (int e = 0; e < 4; ++e) {
+          v[2 * e] = __uint_as_float(x[e] << 16);
+          v[2 * e + 1] = __uint_as_float(x[e] & 0xFFFF0000u);
+        }
+      } else {
+        const float4 a = reinterpret_cast<const float4*>(src)[0];
+        const float4 b = reinterpret_cast<const float4*>(src)[1];
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+      }
+      const uint32_t key = ent >> kEntKShift;     // centroid and sign
+      if (key != run_key) {
+        flush();
+        run_key = key;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) run[e] = 0;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) run[e] += __float2ll_rn(__fmul_rn(v[e], to_fix[e]));
     }
+    // refill the slot just read with the pair kSumRing ahead
+    if (jp + kSumRing < npairs) issue(jp + kSumRing, slot);
     cp_async_commit_group();
   }
   flush();
@@ -609,7 +628,7 @@ cudaError_t launch_update_bucket(const UpdateParams& p, int dtype, cudaStream_t 
 
 cudaError_t launch_update_sum(const UpdateParams& p, int dtype, cudaStream_t s) {
   const dim3 grid((unsigned)kSumSlices, (unsigned)p.W);
-  const size_t smem = (size_t)kSumWarps * kSumRing * kD * (dtype == kBF16 ? 2 : 4);
+  const size_t smem = (size_t)kSumWarps * kSumRing * 2 * kD * (dtype == kBF16 ? 2 : 4);
   const void* fn = dtype == kBF16 ? reinterpret_cast<const void*>(qvg_update_sum<kBF16>)
                                   : reinterpret_cast<const void*>(qvg_update_sum<kFP32>);
   const cudaError_t e = ensure_dynamic_smem(fn, smem);
