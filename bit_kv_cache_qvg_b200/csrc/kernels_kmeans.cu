@@ -90,10 +90,10 @@ qvg_assign_exact(const AssignParams p) {
     const char* rrow = Rg + i * kD * ESZ;
     if (DT == kBF16) {
       const uint2 w = *reinterpret_cast<const uint2*>(rrow + lane * 8);
-      rw[4 * lane + 0] = __uint_as_float(w.x << 16);
-      rw[4 * lane + 1] = __uint_as_float(w.x & 0xFFFF0000u);
-      rw[4 * lane + 2] = __uint_as_float(w.y << 16);
-      rw[4 * lane + 3] = __uint_as_float(w.y & 0xFFFF0000u);
+      rw[4 * lane + 0] = (double)__uint_as_float(w.x << 16);
+      rw[4 * lane + 1] = (double)__uint_as_float(w.x & 0xFFFF0000u);
+      rw[4 * lane + 2] = (double)__uint_as_float(w.y << 16);
+      rw[4 * lane + 3] = (double)__uint_as_float(w.y & 0xFFFF0000u);
     } else {
       const float4 w = *reinterpret_cast<const float4*>(rrow + lane * 16);
       rw[4 * lane + 0] = w.x; rw[4 * lane + 1] = w.y; rw[4 * lane + 2] = w.z; rw[4 * lane + 3] = w.w;
@@ -150,20 +150,21 @@ qvg_assign_exact(const AssignParams p) {
 constexpr int kCandWarps = 8;
 
 // Exact squared distance, fp64, channels in ascending order (one subtract,
-// multiply and add per channel), centroid row read from global memory.
+// multiply and add per channel), token row as fp64 in shared memory, centroid
+// row read from global memory.
 template <int DT>
-__device__ __forceinline__ double exact_dist(const float* rw, const char* crow) {
+__device__ __forceinline__ double exact_dist(const double* rw, const char* crow) {
   double D = 0.0;
 #pragma unroll 2
   for (int j0 = 0; j0 < kD; j0 += 8) {
-    float c[8];
+    double c[8];
     if (DT == kBF16) {
       const uint4 w = *reinterpret_cast<const uint4*>(crow + j0 * 2);
       const uint32_t x[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        c[2 * e] = __uint_as_float(x[e] << 16);
-        c[2 * e + 1] = __uint_as_float(x[e] & 0xFFFF0000u);
+        c[2 * e] = (double)__uint_as_float(x[e] << 16);
+        c[2 * e + 1] = (double)__uint_as_float(x[e] & 0xFFFF0000u);
       }
     } else {
       const float4 a = *reinterpret_cast<const float4*>(crow + j0 * 4);
@@ -172,7 +173,7 @@ __device__ __forceinline__ double exact_dist(const float* rw, const char* crow) 
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const double diff = __dsub_rn((double)rw[j0 + e], (double)c[e]);
+      const double diff = __dsub_rn(rw[j0 + e], c[e]);
       D = __dadd_rn(D, __dmul_rn(diff, diff));
     }
   }
@@ -184,12 +185,12 @@ __global__ void __launch_bounds__(kCandWarps * 32)
 qvg_assign_candidates(const void* R, const void* C, const int K, const int64_t N, const uint2* list,
                       const uint32_t* list_count, uint8_t* pi) {
   constexpr int ESZ = Store<DT>::bytes;
-  __shared__ float rbuf[kCandWarps][kD];
+  __shared__ double rbuf[kCandWarps][kD];
   const int u = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n_rows = min((int64_t)list_count[u], N);
   const int64_t stride = (int64_t)gridDim.x * kCandWarps;
-  float* rw = rbuf[warp];
+  double* rw = rbuf[warp];
   const char* Ru = static_cast<const char*>(R) + (int64_t)u * N * kD * ESZ;
   const char* Cu = static_cast<const char*>(C) + (int64_t)u * K * kD * ESZ;
   const uint32_t all = (K + 31) / 32 >= 32 ? 0xFFFFFFFFu : ((1u << ((K + 31) / 32)) - 1u);
@@ -202,10 +203,10 @@ qvg_assign_candidates(const void* R, const void* C, const int K, const int64_t N
     const char* rrow = Ru + tok * kD * ESZ;
     if (DT == kBF16) {
       const uint2 w = *reinterpret_cast<const uint2*>(rrow + lane * 8);
-      rw[4 * lane + 0] = __uint_as_float(w.x << 16);
-      rw[4 * lane + 1] = __uint_as_float(w.x & 0xFFFF0000u);
-      rw[4 * lane + 2] = __uint_as_float(w.y << 16);
-      rw[4 * lane + 3] = __uint_as_float(w.y & 0xFFFF0000u);
+      rw[4 * lane + 0] = (double)__uint_as_float(w.x << 16);
+      rw[4 * lane + 1] = (double)__uint_as_float(w.x & 0xFFFF0000u);
+      rw[4 * lane + 2] = (double)__uint_as_float(w.y << 16);
+      rw[4 * lane + 3] = (double)__uint_as_float(w.y & 0xFFFF0000u);
     } else {
       const float4 w = *reinterpret_cast<const float4*>(rrow + lane * 16);
       rw[4 * lane + 0] = w.x; rw[4 * lane + 1] = w.y; rw[4 * lane + 2] = w.z; rw[4 * lane + 3] = w.w;
@@ -336,12 +337,16 @@ qvg_update_bucket(const UpdateParams p) {
 #pragma unroll
     for (int j = 0; j < kScan; ++j) {
       const bool ch = kn[j] != ko[j];
-      if (!__any_sync(0xffffffffu, ch)) continue;   // no entry in these 32 tokens (warp-uniform)
-      warp_add(hist, ch ? kn[j] : -1, 1, false);
-      if (!full) {
-        warp_add(hist, ch ? ko[j] : -1, 1, false);
-        warp_add(dcnt, ch ? kn[j] : -1, 1, false);
-        warp_add(dcnt, ch ? ko[j] : -1, -1, false);
+      if (full) {
+        // every token has an entry; neighbours often share a centroid, so
+        // lanes with the same key are combined into one add
+        warp_add(hist, ch ? kn[j] : -1, 1, false);
+      } else if (ch) {
+        // few tokens change: plain adds by the lanes that did
+        atomicAdd(hist + kn[j], 1);
+        atomicAdd(hist + ko[j], 1);
+        atomicAdd(dcnt + kn[j], 1);
+        atomicAdd(dcnt + ko[j], -1);
       }
     }
   }
@@ -378,14 +383,14 @@ qvg_update_bucket(const UpdateParams p) {
 #pragma unroll
     for (int j = 0; j < kScan; ++j) {
       const bool ch = kn[j] != ko[j];
-      if (!__any_sync(0xffffffffu, ch)) continue;   // warp-uniform
       const uint32_t t = (uint32_t)(c + (int64_t)j * blockDim.x + threadIdx.x);
-      const int sa = warp_add(cursor, ch ? kn[j] : -1, 1, true);
-      if (ch) list[sa] = t | ((uint32_t)kn[j] << kEntKShift);
-      if (!full) {
-        // cursor_sub holds minus the end of the free region: slot = end - 1 - rank
-        const int sb = -warp_add(cursor_sub, ch ? ko[j] : -1, 1, true) - 1;
-        if (ch) list[sb] = t | ((uint32_t)ko[j] << kEntKShift) | kEntSub;
+      if (full) {
+        const int sa = warp_add(cursor, ch ? kn[j] : -1, 1, true);
+        if (ch) list[sa] = t | ((uint32_t)kn[j] << kEntKShift);
+      } else if (ch) {
+        list[atomicAdd(cursor + kn[j], 1)] = t | ((uint32_t)kn[j] << kEntKShift);
+        // cursor_sub holds minus the end of the free region: slot = end - 1 - (count so far)
+        list[-atomicAdd(cursor_sub + ko[j], 1) - 1] = t | ((uint32_t)ko[j] << kEntKShift) | kEntSub;
       }
     }
   }
