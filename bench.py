@@ -115,6 +115,23 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- multi-rank helpers
+def max_over_ranks(dist, ms: float, device) -> float:
+    """The step time every rank agrees on: the maximum over ranks (one
+    all-reduce; no collective on the data path)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(bytes_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job GB/s: every rank processes its own cache of the same size."""
+    return bytes_per_rank * world / (ms / 1e3) / 1e9
+
+
 # ---------------------------------------------------------------- oracle arm
 def oracle_sample(wl, tokens: int, seed: int = 99):
     """Time the oracle's quantise + dequantise of one block of `tokens` tokens
@@ -259,11 +276,7 @@ def main():
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
-    ms = ev0.elapsed_time(ev1) / args.steps
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(dist, ev0.elapsed_time(ev1) / args.steps, dev)
     if qvg.workspace_status(ws) != 0:
         raise SystemExit("device-side wait timed out in the timed region")
 
@@ -294,7 +307,7 @@ def main():
     eager_ms = pe0.elapsed_time(pe1)
     flagged = qvg.workspace_flagged(ws)
     kv_bytes = U * N * 128 * 2
-    value = kv_bytes * world / (ms / 1e3) / 1e9
+    value = weak_scaling_value(kv_bytes, world, ms)
 
     # roofline of the kernels (algorithmic work per launch / mean launch time)
     E = U * N * 128
@@ -431,13 +444,9 @@ def e2e(args, qvg, cfg, X, Y, packed, ws, L, Hh, N, dev, world, dist):
         step()
     ev1.record(comp)
     torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1) / args.steps
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(dist, ev0.elapsed_time(ev1) / args.steps, dev)
     nbytes = U * N * 128 * 2
-    return {"value": nbytes * world / (ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+    return {"value": weak_scaling_value(nbytes, world, ms), "unit": "GB/s", "ms_per_step": ms,
             "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
             "host_layers_distinct": nh, "api": "qvg_quantize + qvg_dequantize per layer (64 blocks)"}
 

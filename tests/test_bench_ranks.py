@@ -1,0 +1,52 @@
+"""The multi-rank path of bench.py on CPU: two gloo ranks (one process each)
+agree on the slowest rank's step time and report whole-job throughput for
+weak scaling (every rank compresses its own cache; no data-path collective)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms = bench.max_over_ranks(dist, 10.0 + 5.0 * rank, torch.device("cpu"))
+        out[rank] = (ms, bench.weak_scaling_value(1e9, world, ms))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_slowest_time():
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        port = _free_port()
+        mp.start_processes(_rank, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
+        res = dict(out)
+    assert res[0][0] == pytest.approx(15.0) and res[1][0] == pytest.approx(15.0)
+    # 2 ranks x 1 GB in 15 ms
+    assert res[0][1] == pytest.approx(2e9 / 15e-3 / 1e9)
+
+
+def test_single_rank_needs_no_collective():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(None, 12.5, torch.device("cpu")) == 12.5
+    assert bench.weak_scaling_value(2e9, 1, 1000.0) == pytest.approx(2.0)
