@@ -196,7 +196,7 @@ struct TcParams {
   const float* rnorm2;      // [W][N]
   const float* cn;          // [W][K]
   uint8_t* pi;              // [W][N]
-  uint2* list;              // [W][N] {token, mask of 32-centroid chunks holding the candidates}
+  uint2* list;              // [W][N] {token, mask of 8-centroid groups holding the candidates}
   uint32_t* list_count;     // [W]
   uint32_t* status;         // workspace status word
   unsigned long long* flagged;
@@ -392,14 +392,14 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
       // centroid), each value carrying its column index in its 8 low bits.
       // Columns are taken in quads (top two of the quad by a small network),
       // merged into four independent chains.  The largest key of every
-      // 32-column chunk is kept too: it tells the exact pass which chunks can
-      // hold a near-tie candidate.  The next chunk's tensor-memory load is in
-      // flight while the current one is processed.
+      // 8-column group is kept too: it tells the exact pass which groups can
+      // hold a near-tie candidate.  The next 32-column chunk's tensor-memory
+      // load is in flight while the current one is processed.
       const float kNegBig = -3.0e38f;
       float c1[4] = {kNegBig, kNegBig, kNegBig, kNegBig}, c2[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
-      float cmax[8];
+      float gmax[32];
 #pragma unroll
-      for (int ci = 0; ci < 8; ++ci) cmax[ci] = kNegBig;
+      for (int g = 0; g < 32; ++g) gmax[g] = kNegBig;
       if (ok) {
         const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
         uint32_t ra[32], rb[32];
@@ -416,7 +416,7 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
         asm("mov.b32 %0, 3;" : "=r"(pos3));
         auto chunk = [&](const uint32_t (&r)[32], int ci) {
           const int kb = ci * 32;
-          float m0 = kNegBig, m1 = kNegBig;
+          float qprev = kNegBig;
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             const float ka = __uint_as_float(r[e] & 0xFFFFFF00u);
@@ -431,9 +431,9 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
             const int ch = (e >> 2) & 3;
             c2[ch] = max3f(fminf(c1[ch], qt), c2[ch], qs);
             c1[ch] = fmaxf(c1[ch], qt);
-            if ((e & 4) == 0) m0 = fmaxf(m0, qt); else m1 = fmaxf(m1, qt);
+            // largest key of each 8-column group (two quads)
+            if ((e & 4) == 0) qprev = qt; else gmax[ci * 4 + (e >> 3)] = fmaxf(qprev, qt);
           }
-          cmax[ci] = fmaxf(m0, m1);
         };
 #pragma unroll
         for (int ci = 0; ci < 8; ci += 2) {
@@ -460,7 +460,7 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
       const bool valid = ok && tok < p.N && !aborted(bars);
       const int64_t gi = (int64_t)u * p.N + tok;
       bool flag = false;
-      uint32_t chunks = 0;
+      uint32_t groups = 0;
       if (valid) {
         // Error bound of h (fp32 tensor-core sums of 128 exact products and the
         // three pieces of -|c|^2/2): gamma * (|r| |c| + |c|^2 / 2) for every
@@ -474,13 +474,13 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
         if (!flag) {
           p.pi[gi] = (uint8_t)(__float_as_int(w1) & 0xFF);
         } else {
-          // chunks whose largest key reaches the threshold (with the index-bit
+          // groups whose largest key reaches the threshold (with the index-bit
           // perturbation of that key allowed for) hold every candidate
           const float thr = w1 - margin;
           const float thr_key = thr - 6.2e-5f * (fabsf(w1) + fabsf(thr));
 #pragma unroll
-          for (int ci = 0; ci < 8; ++ci)
-            if (cmax[ci] >= thr_key) chunks |= 1u << ci;
+          for (int g = 0; g < 32; ++g)
+            if (gmax[g] >= thr_key) groups |= 1u << g;
         }
       }
       // every lane of the warp takes part in the list append
@@ -493,7 +493,7 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
           atomicAdd(p.flagged, (unsigned long long)__popc(fm));
         }
         base = __shfl_sync(0xffffffffu, base, leader);
-        if (flag) p.list[(int64_t)u * p.N + base + __popc(fm & ((1u << lane) - 1u))] = make_uint2((uint32_t)tok, chunks);
+        if (flag) p.list[(int64_t)u * p.N + base + __popc(fm & ((1u << lane) - 1u))] = make_uint2((uint32_t)tok, groups);
       }
     }
   }

@@ -193,13 +193,13 @@ qvg_assign_candidates(const void* R, const void* C, const int K, const int64_t N
   double* rw = rbuf[warp];
   const char* Ru = static_cast<const char*>(R) + (int64_t)u * N * kD * ESZ;
   const char* Cu = static_cast<const char*>(C) + (int64_t)u * K * kD * ESZ;
-  const uint32_t all = (K + 31) / 32 >= 32 ? 0xFFFFFFFFu : ((1u << ((K + 31) / 32)) - 1u);
+  const uint32_t all = (K + 7) / 8 >= 32 ? 0xFFFFFFFFu : ((1u << ((K + 7) / 8)) - 1u);
   for (int64_t e = (int64_t)blockIdx.x * kCandWarps + warp; e < n_rows; e += stride) {
     const uint2 ent = list[(int64_t)u * N + e];
     const int64_t tok = ent.x;
     if (tok >= N) continue;                    // warp-uniform; never true for listed tokens
-    uint32_t chunks = ent.y & all;
-    if (chunks == 0) chunks = all;
+    uint32_t groups = ent.y & all;
+    if (groups == 0) groups = all;
     const char* rrow = Ru + tok * kD * ESZ;
     if (DT == kBF16) {
       const uint2 w = *reinterpret_cast<const uint2*>(rrow + lane * 8);
@@ -214,12 +214,19 @@ qvg_assign_candidates(const void* R, const void* C, const int K, const int64_t N
     __syncwarp();
     double bestD = __longlong_as_double(0x7ff0000000000000ll);
     int bestK = 0x7fffffff;
-    // chunks in ascending order; lane takes centroid 32*chunk + lane
-    while (chunks) {
-      const int c = __ffs(chunks) - 1;
-      chunks &= chunks - 1;
-      const int k = c * 32 + lane;
-      if (k < K) {
+    // groups in ascending order, four per round: lane l takes centroid
+    // 8*g + (l % 8) of the (l / 8)-th group of the round, so each lane meets
+    // its centroids in ascending order
+    while (groups) {
+      int gsel = -1;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int g = groups ? __ffs(groups) - 1 : -1;
+        if (groups) groups &= groups - 1;
+        if (q == (lane >> 3)) gsel = g;
+      }
+      const int k = gsel * 8 + (lane & 7);
+      if (gsel >= 0 && k < K) {
         const double D = exact_dist<DT>(rw, Cu + (int64_t)k * kD * ESZ);
         if (D < bestD) { bestD = D; bestK = k; }
       }

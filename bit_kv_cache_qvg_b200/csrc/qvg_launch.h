@@ -76,7 +76,7 @@ struct AssignTcParams {
   const void* C;               // [W][K][d] bf16
   const float* cn;             // [W][K]
   uint8_t* pi;                 // [W][N]
-  uint2* list;                 // [W][N] listed tokens: {token, mask of candidate 32-centroid chunks}
+  uint2* list;                 // [W][N] listed tokens: {token, mask of candidate 8-centroid groups}
   uint32_t* list_count;        // [W], zero on entry
   uint32_t* status;            // workspace status word
   unsigned long long* flagged; // running total of listed tokens
@@ -87,7 +87,7 @@ struct AssignTcParams {
 };
 cudaError_t launch_assign_tc(const AssignTcParams& p, cudaStream_t s);
 // Exact decision of the listed tokens: sequential fp64 squared distances to
-// every centroid of the listed 32-centroid chunks (all chunks when the mask is
+// every centroid of the listed 8-centroid groups (all groups when the mask is
 // empty), the least one wins, ties to the lowest index.
 cudaError_t launch_assign_candidates(const void* R, const void* C, int K, int64_t N, int W,
                                      const uint2* list, const uint32_t* list_count, uint8_t* pi,
