@@ -85,16 +85,18 @@ __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
 // row); for each centroid row the eight lanes read 128 contiguous bytes per
 // half, so the shared-memory tables are read without bank conflicts, and
 // they write two coalesced 128-byte halves of the output row.  Each group of
-// eight lanes walks kDqU tokens per step and loads the next step's codes,
-// scale/zero bytes and assignments while it computes the current one.  E4M3
+// eight lanes walks kDqU tokens per step and keeps the codes, scale/zero bytes
+// and assignments of the next kDqDepth steps in flight.  E4M3
 // bytes are decoded through a 256-entry shared table; a nibble of codes (two
 // channels) maps to a pair of floats through a 16-entry table.
 constexpr int kDqThreads = 768;
 constexpr int kDqWarps = kDqThreads / 32;
 constexpr int kDqStreams = 4 * kDqWarps;        // token streams per block (8 lanes each)
 
-// tokens per half-warp per step (fewer when more assignment bytes are in flight)
-template <int TT> constexpr int dq_unroll() { return (TT < 0 || TT >= 3) ? 2 : 4; }
+// tokens per stream per step, and steps whose loads are in flight (fewer
+// when more assignment bytes are held per token)
+template <int TT> constexpr int dq_unroll() { return 2; }
+template <int TT> constexpr int dq_depth() { return (TT < 0 || TT >= 3) ? 3 : 4; }
 
 template <int DT> struct Oct;                   // a lane's 8 channels of a row
 template <> struct Oct<kBF16> {
@@ -138,6 +140,7 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
   constexpr int ESZ = Store<DT>::bytes;
   constexpr int TR = TT <= 0 ? 1 : TT;
   constexpr int kDqU = dq_unroll<TT>();
+  constexpr int kDqDepth = dq_depth<TT>();
   extern __shared__ __align__(16) unsigned char smem[];
 
   const int unit = blockIdx.x / splits;
@@ -202,15 +205,10 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
       ka[u] = kw;
     }
   };
-  uint32_t cb[kDqU], sz[kDqU], ka[kDqU];
-  int t0 = stream * kDqU;
-  load(t0, cb, sz, ka);
-  for (; t0 < nt; t0 += step) {
-    uint32_t cb_n[kDqU], sz_n[kDqU], ka_n[kDqU];
-    load(t0 + step, cb_n, sz_n, ka_n);
+  auto process = [&](int tb, const uint32_t (&cb)[kDqU], const uint32_t (&sz)[kDqU], const uint32_t (&ka)[kDqU]) {
 #pragma unroll
     for (int u = 0; u < kDqU; ++u) {
-      const int t = t0 + u;
+      const int t = tb + u;
       // y = s*q + m (exact in fp32: E4M3 operands, q <= 3), two channels per op
       float2 y0[4], y1[4];
       {
@@ -248,8 +246,20 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
         Oct<DT>::store(yr + 64 * ESZ, y1);
       }
     }
+  };
+  // kDqDepth steps of per-token bytes in flight: step d of a round is loaded
+  // kDqDepth steps before it is processed
+  uint32_t cb[kDqDepth][kDqU], sz[kDqDepth][kDqU], ka[kDqDepth][kDqU];
+  const int t_first = stream * kDqU;
 #pragma unroll
-    for (int u = 0; u < kDqU; ++u) { cb[u] = cb_n[u]; sz[u] = sz_n[u]; ka[u] = ka_n[u]; }
+  for (int d = 0; d < kDqDepth; ++d) load(t_first + d * step, cb[d], sz[d], ka[d]);
+  for (int t0 = t_first; t0 < nt; t0 += kDqDepth * step) {
+#pragma unroll
+    for (int d = 0; d < kDqDepth; ++d) {
+      const int tb = t0 + d * step;
+      if (tb < nt) process(tb, cb[d], sz[d], ka[d]);
+      load(tb + kDqDepth * step, cb[d], sz[d], ka[d]);
+    }
   }
 }
 
