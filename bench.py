@@ -10,7 +10,14 @@ every block (qvg_dequantize).  Default workload: the LongCat-scale cache --
 iterations.  The metric is KV GB/s: uncompressed bf16 KV bytes / step time.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload longcat|chunk]
+    python bench.py --workload stream      # streaming cache, one line of its own
     python bench.py --impl reference ...   # the oracle on the host cores
+
+The stream workload appends 234 chunks (700 frames of 30x52 tokens, 3 frames
+per chunk) of 32 heads x {K, V} to one cache with warm-started k-means and
+dequantises the whole cache after every chunk; its line reports the median
+per-chunk append latency, a cold-start control, and dequant GB/s against the
+cache length.
 
 Multi-GPU (torchrun, one process per GPU): every rank compresses and
 reconstructs its own cache of the same size (weak scaling, no collective on
@@ -32,6 +39,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "KV GB/s: fused dequant + k-means/2-bit quantize, as % of B200 HBM roofline"
+STREAM_METRIC = "streaming append: per-chunk quantize latency (warm start), with whole-cache dequant GB/s"
 
 WORKLOADS = {
     "longcat": dict(layers=48, heads=32, frames=25, gh=38, gw=40, K=256, T=2, G=64, iters=10,
@@ -40,6 +48,12 @@ WORKLOADS = {
     "chunk": dict(layers=1, heads=12, frames=3, gh=30, gw=52, K=256, T=2, G=64, iters=8,
                   desc="Self-Forcing-scale chunk: 1 layer x 12 heads x K/V, 4,680 tokens "
                        "(3 frames x 30x52), d=128, bf16; K=256, T=2, G=64, 8 Lloyd iterations"),
+    "stream": dict(layers=1, heads=32, frames=700, chunk_frames=3, gh=30, gw=52, K=256, T=2, G=64,
+                   iters=10, warm_iters=3,
+                   desc="Streaming long generation: 1 layer x 32 heads x K/V, 700 frames of 30x52 "
+                        "tokens appended in chunks of 3 frames (4,680 tokens; last chunk 1 frame), "
+                        "up to 1,092,000 tokens, d=128, bf16; K=256, T=2, G=64; warm start 3 "
+                        "Lloyd iterations vs 10 cold; whole cache dequantised after every chunk"),
 }
 
 
@@ -150,8 +164,47 @@ def oracle_sample(wl, tokens: int, seed: int = 99):
     return dt, tokens * 128 * 2, o.get_threads()
 
 
+def oracle_stream_sample(wl, chunks: int, seed: int = 7):
+    """Time the oracle's warm-started append of `chunks` chunks of one V block
+    (the first chunk, cold, is untimed).  Returns (seconds per chunk, threads)."""
+    import numpy as np
+    import torch
+    from bit_kv_cache_qvg_b200 import synth
+    from oracle import oracle as o
+    o.build()
+    s = synth.PrototypeStream(1, wl["gh"], wl["gw"], kinds=[1], seed=seed)
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    K, T, G = wl["K"], wl["T"], wl["G"]
+    prev = o.quantize(bits(s.next(wl["chunk_frames"])), K=K, T=T, G=G, iters=wl["iters"])
+    t = 0.0
+    for _ in range(chunks):
+        X = bits(s.next(wl["chunk_frames"]))
+        t0 = time.perf_counter()
+        prev = o.quantize(X, K=K, T=T, G=G, iters=wl["warm_iters"], init=prev["centroids"])
+        t += time.perf_counter() - t0
+    return t / chunks, o.get_threads()
+
+
 def run_reference(args, wl, rank, world):
     if rank != 0:
+        return
+    if "chunk_frames" in wl:
+        times = []
+        for i in range(args.warmup + args.steps):
+            dt, threads = oracle_stream_sample(wl, 1, seed=1000 + i)
+            if i >= args.warmup:
+                times.append(dt)
+        v = sum(times) / len(times) * 1e3 * 2 * wl["heads"]
+        sample = ("one V block: a cold first chunk (untimed) then one warm-started 4,680-token append per "
+                  f"step; ms scaled by the {2 * wl['heads']} blocks of a chunk")
+        print(json.dumps({
+            "impl": "reference", "metric": STREAM_METRIC, "value": v, "unit": "ms", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl["desc"], "reference": "C oracle (fp64 k-means) on host cores"},
+            "cpu_baseline": {"value": v, "unit": "ms", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
         return
     tokens = args.ref_tokens
     times = []
@@ -186,11 +239,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=4750)
     ap.add_argument("--cpu-tokens", type=int, default=9500)
+    ap.add_argument("--frames", type=int, default=None, help="override the frame count")
     args = ap.parse_args()
     wl = dict(WORKLOADS[args.workload])
     if args.layers:
         wl["layers"] = args.layers
         wl["desc"] += f" [{args.layers} layers]"
+    if args.frames:
+        wl["frames"] = args.frames
+        wl["desc"] += f" [{args.frames} frames]"
 
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -218,6 +275,12 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
+    if "chunk_frames" in wl:
+        run_stream(args, wl, qvg, synth, dev, dist, rank, world, local, peaks)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     L, Hh = wl["layers"], wl["heads"]
     N = wl["frames"] * wl["gh"] * wl["gw"]
@@ -387,6 +450,217 @@ def main():
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def stream_chunks(wl):
+    """Token counts of the stream's chunks: chunk_frames frames each, the last
+    chunk takes what is left of the frame count."""
+    cf, hw, F = wl["chunk_frames"], wl["gh"] * wl["gw"], wl["frames"]
+    return [min(cf, F - f) * hw for f in range(0, F, cf)]
+
+
+def dequant_alg_bytes(U, n, chunks, K, T, G, esz=2):
+    """Algorithmic bytes of one fused dequant of U blocks of n tokens spread
+    over `chunks` chunks: codes + E4M3 scale/zero + assignments read, output
+    written, and every chunk's T centroid tables read once."""
+    return U * n * 128 * (2 / 8 + 2 / G + T / 128 + esz) + chunks * T * U * K * 128 * esz
+
+
+def run_stream(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
+    """Streaming cache: chunks appended by qvg_append_chunk (warm start from
+    the previous chunk's centroids), the whole cache fused-dequantised after
+    every chunk.  Every append and every dequant is bracketed by CUDA events on
+    the launching stream.  A second pass quantises the same chunks cold (first-K
+    init, `iters` Lloyd iterations) as the control."""
+    import torch
+    Hh = wl["heads"]
+    U = 2 * Hh
+    K, T, G = wl["K"], wl["T"], wl["G"]
+    sizes = stream_chunks(wl)
+    total, nch = sum(sizes), len(sizes)
+    cfg = qvg.config(K=K, T=T, group_size=G, iters=wl["iters"], warm_iters=wl["warm_iters"])
+    cold_cfg = qvg.config(K=K, T=T, group_size=G, iters=wl["iters"], warm_iters=wl["iters"])
+    kinds = [0] * Hh + [1] * Hh
+    seed = synth.unit_seed(rank, 0, 0, 0)
+    stream = torch.cuda.Stream(dev)
+    ybuf = torch.empty(U * total * 128, dtype=torch.bfloat16, device=dev)
+    quality_at = sorted({1, 2, nch // 2, nch - 2})
+
+    def events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    # warm-up: W chunks through a throwaway cache (kernel load, workspace sizing)
+    gen = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=kinds, seed=seed + 1, device=dev)
+    wcache = qvg.Cache(cfg, U, sum(sizes[:max(args.warmup, 1)]), max(args.warmup, 1))
+    with torch.cuda.stream(stream):
+        for c in range(max(args.warmup, 1)):
+            wcache.append(gen.next(sizes[c] // (wl["gh"] * wl["gw"])), stream=stream)
+            wcache.dequantize(ybuf[:U * wcache.tokens * 128].view(U, wcache.tokens, 128), stream=stream)
+    torch.cuda.synchronize()
+    wcache.close()
+
+    # pass 1: the streaming cache
+    cache = qvg.Cache(cfg, U, total, nch)
+    gen = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=kinds, seed=seed, device=dev)
+    ea, eb, da, db = events(nch), events(nch), events(nch), events(nch)
+    kept = {}
+    with ClockSampler(local) as clk:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for c, n in enumerate(sizes):
+                X = gen.next(n // (wl["gh"] * wl["gw"]))
+                if c in quality_at:
+                    kept[c] = X
+                ea[c].record(stream)
+                cache.append(X, stream=stream)
+                eb[c].record(stream)
+                tok = cache.tokens
+                da[c].record(stream)
+                cache.dequantize(ybuf[:U * tok * 128].view(U, tok, 128), stream=stream)
+                db[c].record(stream)
+        torch.cuda.synchronize()
+    append_ms = [ea[c].elapsed_time(eb[c]) for c in range(nch)]
+    deq_ms = [da[c].elapsed_time(db[c]) for c in range(nch)]
+    cum = [sum(sizes[:c + 1]) for c in range(nch)]
+
+    def rel_mse(Y, X):
+        d = Y.float() - X.float()
+        return float((d * d).sum() / (X.float() ** 2).sum())
+
+    warm_q = {}
+    with torch.cuda.stream(stream):
+        for c, X in kept.items():
+            warm_q[c] = rel_mse(qvg.dequantize(cache.chunk(c), stream=stream), X)
+    del kept
+
+    # pass 2: the same chunks quantised cold, one by one
+    gen = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=kinds, seed=seed, device=dev)
+    packed = qvg.alloc_packed(cold_cfg, max(sizes), U, device=dev)
+    ws = qvg.alloc_workspace(cold_cfg, max(sizes), U, device=dev)
+    ca, cb = events(nch), events(nch)
+    cold_q = {}
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for c, n in enumerate(sizes):
+            X = gen.next(n // (wl["gh"] * wl["gw"]))
+            p = packed if n == max(sizes) else qvg.alloc_packed(cold_cfg, n, U, device=dev)
+            ca[c].record(stream)
+            qvg.quantize(X, cold_cfg, out=p, workspace=ws, stream=stream)
+            cb[c].record(stream)
+            if c in quality_at:
+                cold_q[c] = rel_mse(qvg.dequantize(p, stream=stream), X)
+    torch.cuda.synchronize()
+    cold_ms = [ca[c].elapsed_time(cb[c]) for c in range(nch)]
+
+    full = [c for c in range(1, nch) if sizes[c] == sizes[0]]
+    med_warm = statistics.median(append_ms[c] for c in full)
+    med_cold = statistics.median(cold_ms[c] for c in full)
+    value = max_over_ranks(dist, med_warm, dev)
+
+    def gbs(c):
+        return dequant_alg_bytes(U, cum[c], c + 1, K, T, G) / (deq_ms[c] / 1e3) / 1e9
+
+    picks = sorted({0, 9, 19, 49, 99, 149, 199, nch - 1} & set(range(nch)))
+    last = nch - 1
+    ach = gbs(last)
+    result = {
+        "metric": STREAM_METRIC, "value": value, "unit": "ms", "n_gpus": world, "steps": nch,
+        "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl["desc"], "blocks": U, "chunks": nch, "chunk_tokens": sizes[0],
+                   "last_chunk_tokens": sizes[-1], "cache_tokens": total,
+                   "l2": "every chunk's input (76.7 MB) is freshly generated; dequant outputs up to "
+                         f"{U * total * 256 / 1e9:.1f} GB exceed L2",
+                   "parallelism": f"weak: {world} rank(s), independent caches"},
+        "append_ms": {"median_warm": med_warm, "median_cold_control": med_cold,
+                      "cold_over_warm": med_cold / med_warm, "first_chunk_cold": append_ms[0],
+                      "last_chunk": append_ms[-1], "min_warm": min(append_ms[c] for c in full),
+                      "max_warm": max(append_ms[c] for c in full)},
+        "dequant_vs_length": [{"chunks": c + 1, "tokens": cum[c], "ms": deq_ms[c], "GB/s": gbs(c)}
+                              for c in picks],
+        "relative_mse": {"warm": {str(c): warm_q[c] for c in sorted(warm_q)},
+                         "cold": {str(c): cold_q[c] for c in sorted(cold_q)}},
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": ach / peaks["hbm"], "traffic": None, "kernel": "qvg_dequant_fused",
+                     "at": f"full cache, {total} tokens x {U} blocks, {nch} chunks",
+                     "alg_bytes_per_launch": dequant_alg_bytes(U, total, nch, K, T, G)},
+        "gpu_launches": None,
+        "clocks": clk.summary(),
+    }
+    qvg.profile_reset()
+    qvg.profile_enable(True)
+    with torch.cuda.stream(stream):
+        cache.dequantize(ybuf[:U * total * 128].view(U, total, 128), stream=stream)
+    torch.cuda.synchronize()
+    qvg.profile_enable(False)
+    result["gpu_launches"] = {"per_dequant": qvg.profile_launches(), "per_append": None}
+    # one more append into a scratch cache counts the launches of one warm append
+    scache = qvg.Cache(cfg, U, 2 * sizes[0], 2)
+    g2 = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=kinds, seed=seed + 2, device=dev)
+    with torch.cuda.stream(stream):
+        scache.append(g2.next(wl["chunk_frames"]), stream=stream)
+        torch.cuda.synchronize()
+        qvg.profile_reset()
+        qvg.profile_enable(True)
+        scache.append(g2.next(wl["chunk_frames"]), stream=stream)
+        torch.cuda.synchronize()
+        qvg.profile_enable(False)
+    result["gpu_launches"]["per_append"] = qvg.profile_launches()
+    result["kernels_warm_append"] = qvg.profile_report()
+    scache.close()
+    result["gpu_launches"] = nch * (result["gpu_launches"]["per_dequant"] + result["gpu_launches"]["per_append"])
+    if rank == 0 and not args.no_e2e:
+        result["e2e"] = stream_e2e(args, wl, qvg, synth, cfg, sizes, dev, stream)
+    if rank == 0 and not args.no_cpu_baseline:
+        dt, threads = oracle_stream_sample(wl, 1)
+        result["cpu_baseline"] = {"value": dt * 1e3 * U, "unit": "ms", "cores": threads, "kind": "oracle",
+                                  "sample": f"one warm-started {sizes[0]}-token append of one V block "
+                                            f"({dt:.1f} s), scaled by the {U} blocks of a chunk"}
+    cache.close()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+def stream_e2e(args, wl, qvg, synth, cfg, sizes, dev, stream, chunks=40):
+    """Per-chunk latency through the public API with host buffers: the chunk
+    arrives from pinned host memory, is appended, and its packed form (codes,
+    scale, zero, assignments, centroids) returns to pinned host memory."""
+    import torch
+    Hh = wl["heads"]
+    U = 2 * Hh
+    n = sizes[0]
+    chunks = min(chunks, len([s for s in sizes if s == n]))
+    cache = qvg.Cache(cfg, U, chunks * n, chunks)
+    gen = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=[0] * Hh + [1] * Hh, seed=12345, device=dev)
+    Xh = torch.empty((U, n, 128), dtype=torch.bfloat16, pin_memory=True)
+    Xd = torch.empty((U, n, 128), dtype=torch.bfloat16, device=dev)
+    out_h = None
+    times = []
+    for c in range(chunks):
+        Xh.copy_(gen.next(wl["chunk_frames"]))
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            Xd.copy_(Xh, non_blocking=True)
+            cache.append(Xd, stream=stream)
+            p = cache.chunk(c)
+            parts = (p.codes, p.scale, p.zero, p.assign, p.centroids)
+            if out_h is None:
+                out_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in parts]
+            for h, t in zip(out_h, parts):
+                h.copy_(t, non_blocking=True)
+            e1.record(stream)
+        torch.cuda.synchronize()
+        if c > 0:
+            times.append(e0.elapsed_time(e1))
+    cache.close()
+    d2h = sum(h.numel() * h.element_size() for h in out_h)
+    return {"value": statistics.median(times), "unit": "ms", "h2d_bytes_per_step": U * n * 256,
+            "d2h_bytes_per_step": d2h, "chunks_timed": len(times),
+            "api": "qvg_append_chunk with the chunk from pinned host memory and its packed form back"}
 
 
 def e2e(args, qvg, cfg, X, Y, packed, ws, L, Hh, N, dev, world, dist):
