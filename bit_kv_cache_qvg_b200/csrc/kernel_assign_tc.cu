@@ -206,6 +206,7 @@ struct TcParams {
   int tiles_per_unit;
   int tiles_per_cta;
   float gamma;              // relative error bound of the tensor-core dot products
+  uint32_t unit;            // always 1: the multiplier that puts the column add on the FMA pipe
 };
 
 #ifdef QVG_TC_DEBUG
@@ -391,10 +392,12 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
       // Top two of h_k = r.c_k - |c_k|^2/2 (the largest h is the nearest
       // centroid), each value carrying its column index in its 8 low bits.
       // Columns are taken in quads (top two of the quad by a small network),
-      // merged into four independent chains.  The largest key of every
-      // 8-column group is kept too: it tells the exact pass which groups can
-      // hold a near-tie candidate.  The next 32-column chunk's tensor-memory
-      // load is in flight while the current one is processed.
+      // two quads make an 8-column group (its maximum is kept: it tells the
+      // exact pass which groups can hold a near-tie candidate), and groups
+      // are merged into four independent chains.  The next 32-column chunk's
+      // tensor-memory load is in flight while the current one is processed.
+      // The epilogue is bound by the integer/logic pipe, so each key is one
+      // lop3 and the column add runs as an integer multiply-add on the FMA pipe.
       const float kNegBig = -3.0e38f;
       float c1[4] = {kNegBig, kNegBig, kNegBig, kNegBig}, c2[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
       float gmax[32];
@@ -405,34 +408,45 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
         uint32_t ra[32], rb[32];
         tmem_ld32_async(tbase, ra);
         tmem_wait_ld(ra);
-        // Keys are formed in two steps so that each is one logic operation:
-        // the position within the quad (0-3, held in registers) replaces the
-        // 8 low bits of every value, and the quad's column (a multiple of 4,
-        // an immediate) is or-ed into the quad's maximum only -- the runner-up
-        // value needs no index.
+        // The position within the quad (0-3, held in registers) replaces the
+        // 8 low bits of every value; the quad's column (a multiple of 4) is
+        // added to the quad's maximum only -- the runner-up needs no index.
         uint32_t pos1, pos2, pos3;
         asm("mov.b32 %0, 1;" : "=r"(pos1));
         asm("mov.b32 %0, 2;" : "=r"(pos2));
         asm("mov.b32 %0, 3;" : "=r"(pos3));
+        const uint32_t unit = p.unit;
+        auto key = [](uint32_t v, uint32_t pos) {
+          uint32_t k;
+          asm("lop3.b32 %0, %1, 0xFFFFFF00, %2, 0xEA;" : "=r"(k) : "r"(v), "r"(pos));  // (v & ~0xFF) | pos
+          return __uint_as_float(k);
+        };
+        auto quad = [&](const uint32_t (&r)[32], int e, int col, float& qt, float& qs) {
+          uint32_t ka_u;
+          asm("and.b32 %0, %1, 0xFFFFFF00;" : "=r"(ka_u) : "r"(r[e]));
+          const float ka = __uint_as_float(ka_u);
+          const float kb2 = key(r[e + 1], pos1), kc = key(r[e + 2], pos2), kd = key(r[e + 3], pos3);
+          const float h1 = fmaxf(ka, kb2), l1 = fminf(ka, kb2);
+          const float h2 = fmaxf(kc, kd), l2 = fminf(kc, kd);
+          // bits 2-7 of the key are zero here, so adding the quad's column is an or
+          uint32_t qt_u;
+          asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(qt_u) : "r"(unit), "r"((uint32_t)col),
+              "r"(__float_as_uint(fmaxf(h1, h2))));
+          qt = __uint_as_float(qt_u);
+          qs = max3f(fminf(h1, h2), l1, l2);
+        };
         auto chunk = [&](const uint32_t (&r)[32], int ci) {
-          const int kb = ci * 32;
-          float qprev = kNegBig;
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float ka = __uint_as_float(r[e] & 0xFFFFFF00u);
-            const float kb2 = __uint_as_float((r[e + 1] & 0xFFFFFF00u) | pos1);
-            const float kc = __uint_as_float((r[e + 2] & 0xFFFFFF00u) | pos2);
-            const float kd = __uint_as_float((r[e + 3] & 0xFFFFFF00u) | pos3);
-            const float h1 = fmaxf(ka, kb2), l1 = fminf(ka, kb2);
-            const float h2 = fmaxf(kc, kd), l2 = fminf(kc, kd);
-            // bits 2-7 of the key are zero here, so adding the quad's column is an or
-            const float qt = __uint_as_float(__float_as_uint(fmaxf(h1, h2)) + (uint32_t)(kb + e));
-            const float qs = max3f(fminf(h1, h2), l1, l2);
-            const int ch = (e >> 2) & 3;
-            c2[ch] = max3f(fminf(c1[ch], qt), c2[ch], qs);
-            c1[ch] = fmaxf(c1[ch], qt);
-            // largest key of each 8-column group (two quads)
-            if ((e & 4) == 0) qprev = qt; else gmax[ci * 4 + (e >> 3)] = fmaxf(qprev, qt);
+          for (int e = 0; e < 32; e += 8) {
+            float ta, sa, tb, sb;
+            quad(r, e, ci * 32 + e, ta, sa);
+            quad(r, e + 4, ci * 32 + e + 4, tb, sb);
+            const float gt = fmaxf(ta, tb);
+            const float gs = max3f(fminf(ta, tb), sa, sb);
+            const int ch = e >> 3;
+            gmax[ci * 4 + ch] = gt;
+            c2[ch] = max3f(fminf(c1[ch], gt), c2[ch], gs);
+            c1[ch] = fmaxf(c1[ch], gt);
           }
         };
 #pragma unroll
@@ -561,6 +575,7 @@ cudaError_t launch_assign_tc(const AssignTcParams& a, cudaStream_t s) {
   if (p.tiles_per_cta < 2) p.tiles_per_cta = 2;
   splits = (p.tiles_per_unit + p.tiles_per_cta - 1) / p.tiles_per_cta;
   p.gamma = a.gamma;
+  p.unit = 1;
   const size_t smem = assign_tc_smem_bytes(a.K);
   cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(qvg_kmeans_assign), smem);
   if (e != cudaSuccess) return e;
