@@ -419,9 +419,9 @@ __device__ __forceinline__ void cp_async_wait_groups() { asm volatile("cp.async.
 // shared memory filled by cp.async (every lane copies, and later reads back,
 // its own 8 channels of a row), so that many rows are in flight without
 // holding registers.  Within a bucket the added rows come first and the
-// removed rows last, so a run (same centroid, same sign) is summed in
-// registers and applied with its sign when it ends; each half-warp keeps its
-// own run.
+// removed rows last, so a run (one centroid, its added rows then its removed
+// rows, with their signs) is summed in registers and applied when it ends;
+// each half-warp keeps its own run.
 constexpr int kSumRing = 16;
 
 template <int DT>
@@ -449,7 +449,10 @@ qvg_update_sum(const UpdateParams p) {
   const uint32_t* list = p.list + (int64_t)u * 2 * N + e0;
   const char* Ru = static_cast<const char*>(p.R) + (int64_t)u * N * ROW + hl * LANE_BYTES;
   unsigned char* ring = smem + (size_t)warp * kSumRing * 2 * ROW + half * ROW + hl * LANE_BYTES;
-  long long* Su = p.S + (int64_t)u * p.K * kD + 8 * hl;
+  // S keeps channel c at (c % 8) * 16 + c / 8, so that the adds of a
+  // half-warp (lane hl owns channels 8*hl ... 8*hl + 7) to one channel slot e
+  // land on 128 contiguous bytes
+  long long* Su = p.S + (int64_t)u * p.K * kD + hl;
 
   // entries in groups of 32 (16 pairs), one per lane; two groups held, the
   // next loaded one group ahead of the issue pointer
@@ -477,14 +480,12 @@ qvg_update_sum(const UpdateParams p) {
   long long run[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) run[e] = 0;
-  uint32_t run_key = 0xFFFFFFFFu;                 // (centroid, sign) of this half's open run
+  uint32_t run_key = 0xFFFFFFFFu;                 // centroid of this half's open run
   auto flush = [&]() {
     if (run_key != 0xFFFFFFFFu) {
-      long long* a = Su + (int64_t)(run_key & 0xFFu) * kD;
-      const bool neg = (run_key & 0x100u) != 0u;
+      long long* a = Su + (int64_t)run_key * kD;
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        atomicAdd(reinterpret_cast<unsigned long long*>(a + e), (unsigned long long)(neg ? -run[e] : run[e]));
+      for (int e = 0; e < 8; ++e) atomicAdd(reinterpret_cast<unsigned long long*>(a + 16 * e), (unsigned long long)run[e]);
     }
   };
   for (int jp = 0; jp < npairs; ++jp) {
@@ -513,7 +514,10 @@ qvg_update_sum(const UpdateParams p) {
         const float4 b = reinterpret_cast<const float4*>(src)[1];
         v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
       }
-      const uint32_t key = ent >> kEntKShift;     // centroid and sign
+      // A run is one centroid: its added rows, then its removed rows (the
+      // bucket order), summed with their signs and applied once.
+      const uint32_t key = (ent >> kEntKShift) & 0xFFu;
+      const float sg = (ent & kEntSub) ? -1.0f : 1.0f;
       if (key != run_key) {
         flush();
         run_key = key;
@@ -521,7 +525,7 @@ qvg_update_sum(const UpdateParams p) {
         for (int e = 0; e < 8; ++e) run[e] = 0;
       }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) run[e] += __float2ll_rn(__fmul_rn(v[e], to_fix[e]));
+      for (int e = 0; e < 8; ++e) run[e] += __float2ll_rn(__fmul_rn(__fmul_rn(v[e], sg), to_fix[e]));
     }
     // refill the slot just read with the pair kSumRing ahead
     if (jp + kSumRing < npairs) issue(jp + kSumRing, slot);
@@ -547,9 +551,9 @@ qvg_update_centroids(const UpdateParams p) {
   if (!full) n += p.n[(int64_t)u * p.K + k];
   if (lane == 0) p.n[(int64_t)u * p.K + k] = n;
   if (n <= 0) return;                                // an empty centroid keeps its value
-  const longlong2* Sg = reinterpret_cast<const longlong2*>(p.S + ((int64_t)u * p.K + k) * kD + 4 * lane);
-  const longlong2 a = Sg[0], b = Sg[1];
-  const long long sum[4] = {a.x, a.y, b.x, b.y};
+  // channel c = 4 * lane + e sits at (c % 8) * 16 + c / 8 of the centroid's sums
+  const long long* Sg = p.S + ((int64_t)u * p.K + k) * kD + (4 * (lane & 1)) * 16 + (lane >> 1);
+  const long long sum[4] = {Sg[0], Sg[16], Sg[32], Sg[48]};
   const double dn = (double)n;
   double sq = 0.0;
   double mean[4];

@@ -102,7 +102,7 @@ struct UpdateParams {
   uint32_t* list;         // [W][2N] scratch: entries bucketed by centroid
   int* off;               // [W][K+1] scratch: bucket offsets
   int* cnt;               // [W][K]   scratch: member counts (first iteration) or their changes
-  long long* S;           // [W][K][d] running member sums in fixed point (units of 2^L_c)
+  long long* S;           // [W][K][d] running member sums in fixed point (units of 2^L_c); channel c at (c % 8) * 16 + c / 8
   int* n;                 // [W][K]    member counts
   void* C;                // [W][K][d] centroids (updated in place)
   float* cn;              // [W][K]    squared centroid norms
