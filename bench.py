@@ -344,8 +344,13 @@ def main():
         raise SystemExit("device-side wait timed out in the timed region")
 
     # per-kernel device time: one more step, captured with a CUDA event recorded
-    # on the launching stream before and after every kernel, then replayed
+    # on the launching stream before and after every kernel, then replayed.
+    # It runs its waves one at a time on one stream, so that every launch is
+    # timed alone (with two waves in flight an event pair would also count
+    # the time a launch queues behind the other wave's kernels).
     qvg.workspace_flagged(ws)           # reset the near-tie counter
+    lanes_env = os.environ.get("QVG_WAVE_LANES")
+    os.environ["QVG_WAVE_LANES"] = "1"
     qvg.profile_reset()
     qvg.profile_enable(True)
     if graph is not None:
@@ -365,6 +370,10 @@ def main():
         pe1.record(stream)
     torch.cuda.synchronize()
     qvg.profile_enable(False)
+    if lanes_env is None:
+        del os.environ["QVG_WAVE_LANES"]
+    else:
+        os.environ["QVG_WAVE_LANES"] = lanes_env
     launches = qvg.profile_launches() * args.steps
     kernels = qvg.profile_report()
     eager_ms = pe0.elapsed_time(pe1)
@@ -432,6 +441,7 @@ def main():
         "gpu_launches": launches,
         "profiled_step_ms_with_kernel_events": eager_ms,
         "timed_region": "CUDA graph replay of the step" if graph is not None else "eager launches",
+        "per_kernel_times": "one more step with an event pair around every launch, waves one at a time",
         "near_tie_tokens_per_step": flagged if flagged >= 0 else None,
         "token_assignments_per_step": U * N * T * I,
         "clocks": clk.summary(),

@@ -102,6 +102,33 @@ int preferred_batch(const qvg_config& c, int64_t N, int H, int dtype) {
   return std::max(1, std::min(std::min(w, qvg::device_sm_count()), H));
 }
 
+// Waves of blocks are independent, so consecutive waves run on two streams
+// ("lanes"), each with its own workspace: the latency-bound update kernels of
+// one wave then overlap the other wave's tensor-core assignment.
+// QVG_WAVE_LANES=1 keeps every wave on the caller's stream.
+int wave_lanes(int H, int W) {
+  if (H <= W) return 1;
+  if (const char* env = std::getenv("QVG_WAVE_LANES")) {
+    if (std::atoi(env) == 1) return 1;
+  }
+  return 2;
+}
+
+// The second lane's stream, one per device, created on first use.
+cudaStream_t side_stream() {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  std::lock_guard<std::mutex> g(mu);
+  if (streams[dev] == nullptr && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    streams[dev] = nullptr;
+  }
+  return streams[dev];
+}
+
 // Relative error bound assumed for the tensor-core sums (128 exact bf16 x bf16
 // products plus three bf16 pieces of -|c|^2/2, accumulated in fp32 over nine
 // MMA steps): 2^-16, about 7x a bound of two fp32 ulps per step.
@@ -233,12 +260,17 @@ size_t qvg_packed_bytes(const qvg_config* c, int64_t N, int32_t H, int32_t d, qv
 
 size_t qvg_workspace_bytes(const qvg_config* c, int64_t N, int32_t H, int32_t d, qvg_dtype dtype) {
   if (check_config(c, N, H, d, dtype) != QVG_OK || N < 1) return 0;
-  return make_plan(*c, N, preferred_batch(*c, N, H, dtype), dtype).total;
+  const int W = preferred_batch(*c, N, H, dtype);
+  return (size_t)wave_lanes(H, W) * make_plan(*c, N, W, dtype).total;
 }
 
-qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, int64_t N,
-                        int32_t H, int32_t d, const void* init, const qvg_packed* out,
-                        void* workspace, size_t ws_bytes, qvg_stream_t stream_) {
+}  // extern "C"
+
+namespace qvg {
+
+qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, int64_t N, int32_t H,
+                         int32_t d, const void* init, const qvg_packed* out, void* workspace,
+                         size_t ws_bytes, qvg_stream_t stream_, int max_lanes) {
   qvg_status st = check_config(cfg, N, H, d, dtype);
   if (st != QVG_OK) return st;
   const qvg_config c = *cfg;
@@ -258,26 +290,34 @@ qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, i
   const size_t esz = (size_t)esize(dt);
 
   int W = preferred_batch(c, N, H, dt);
+  int lanes = std::min(max_lanes, wave_lanes(H, W));
   Plan plan = make_plan(c, N, W, dt);
-  while (plan.total > ws_bytes && W > 1) plan = make_plan(c, N, --W, dt);
+  while ((size_t)lanes * plan.total > ws_bytes && W > 1) {
+    plan = make_plan(c, N, --W, dt);
+    lanes = std::min(max_lanes, wave_lanes(H, W));
+  }
+  if ((size_t)lanes * plan.total > ws_bytes) lanes = 1;
   if (plan.total > ws_bytes) return QVG_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s1 = lanes > 1 ? side_stream() : s;
+  if (s1 == nullptr) { lanes = 1; s1 = s; }
 
-  char* ws = static_cast<char*>(workspace);
-  float* rnorm = reinterpret_cast<float*>(ws + plan.off_rnorm);
-  float* cn = reinterpret_cast<float*>(ws + plan.off_cn);
-  uint2* list = reinterpret_cast<uint2*>(ws + plan.off_list);
-  uint32_t* list_count = reinterpret_cast<uint32_t*>(ws + plan.off_listcnt);
-  uint32_t* status = reinterpret_cast<uint32_t*>(ws + plan.off_status);
-  unsigned long long* flagged = reinterpret_cast<unsigned long long*>(ws + plan.off_status + 8);
-  uint32_t* chmax = reinterpret_cast<uint32_t*>(ws + plan.off_chmax);
+  // the status word and the near-tie counter are shared by both lanes
+  char* const ws0 = static_cast<char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws0 + plan.off_status);
+  unsigned long long* flagged = reinterpret_cast<unsigned long long*>(ws0 + plan.off_status + 8);
   int log2n = 0;                      // smallest k with 2^k > N (fixed-point scale of the sums)
   while (log2n < 62 && (int64_t(1) << log2n) <= N) ++log2n;
   // bf16 blocks take the tensor-core assignment; fp32 blocks the exact CUDA-core one
   const bool use_tc = dt == kBF16 && assign_path_tc();
   const int ng = kD / c.group_size;
 
-  for (int u0 = 0; u0 < H; u0 += W) {
-    const int w = std::min(W, H - u0);
+  // one wave: blocks u0 .. u0+w-1 on stream s with workspace ws
+  auto run_wave = [&](int u0, int w, cudaStream_t s, char* ws) -> qvg_status {
+    float* rnorm = reinterpret_cast<float*>(ws + plan.off_rnorm);
+    float* cn = reinterpret_cast<float*>(ws + plan.off_cn);
+    uint2* list = reinterpret_cast<uint2*>(ws + plan.off_list);
+    uint32_t* list_count = reinterpret_cast<uint32_t*>(ws + plan.off_listcnt);
+    uint32_t* chmax = reinterpret_cast<uint32_t*>(ws + plan.off_chmax);
     const char* Xu = static_cast<const char*>(X) + (size_t)u0 * N * kD * esz;
     ResidualParams rq{};
     rq.N = N; rq.W = w; rq.K = c.K; rq.G = c.group_size;
@@ -287,7 +327,7 @@ qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, i
     if (c.T == 0) {
       rq.R_in = Xu;
       QVG_TRY(plaunch(K_RESIDUAL_QUANT, s, [&] { return launch_residual(rq, dt, true, s); }));
-      continue;
+      return QVG_OK;
     }
     const void* Rin = Xu;
     for (int t = 0; t < c.T; ++t) {
@@ -353,8 +393,46 @@ qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, i
         QVG_TRY(plaunch(K_RESIDUAL_QUANT, s, [&] { return launch_residual(rp, dt, true, s); }));
       }
     }
+    return QVG_OK;
+  };
+
+  if (lanes == 1) {
+    for (int u0 = 0; u0 < H; u0 += W) {
+      st = run_wave(u0, std::min(W, H - u0), s, ws0);
+      if (st != QVG_OK) return st;
+    }
+    return QVG_OK;
   }
-  return QVG_OK;
+  // Two lanes: the side stream joins after the caller's stream reaches this
+  // call, and the caller's stream waits for the side stream at the end (also
+  // on an error, so that a stream capture stays joined).
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    if (fork) cudaEventDestroy(fork);
+    return QVG_ERR_CUDA;
+  }
+  st = QVG_OK;
+  if (cudaEventRecord(fork, s) != cudaSuccess || cudaStreamWaitEvent(s1, fork, 0) != cudaSuccess) st = QVG_ERR_CUDA;
+  for (int u0 = 0, wv = 0; st == QVG_OK && u0 < H; u0 += W, ++wv) {
+    const int lane = wv & 1;
+    st = run_wave(u0, std::min(W, H - u0), lane ? s1 : s, ws0 + (size_t)lane * plan.total);
+  }
+  if (cudaEventRecord(join, s1) != cudaSuccess || cudaStreamWaitEvent(s, join, 0) != cudaSuccess) st = QVG_ERR_CUDA;
+  cudaEventDestroy(fork);
+  cudaEventDestroy(join);
+  return st;
+}
+
+}  // namespace qvg
+
+extern "C" {
+
+qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, int64_t N,
+                        int32_t H, int32_t d, const void* init, const qvg_packed* out,
+                        void* workspace, size_t ws_bytes, qvg_stream_t stream_) {
+  return qvg::quantize_impl(cfg, X, dtype, N, H, d, init, out, workspace, ws_bytes, stream_, 2);
 }
 
 qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packed, qvg_dtype dtype,

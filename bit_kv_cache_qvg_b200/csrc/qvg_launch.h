@@ -5,11 +5,17 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "qvg.h"
 #include "qvg_common.cuh"
 
 namespace qvg {
 
 // ---- launch helpers (qvg_api.cu)
+// qvg_quantize with at most `max_lanes` waves of blocks in flight at once
+// (1: every wave on the caller's stream, with no side stream and no events).
+qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, int64_t N, int32_t H,
+                         int32_t d, const void* init, const qvg_packed* out, void* workspace,
+                         size_t ws_bytes, qvg_stream_t stream, int max_lanes);
 // SM count of the current device (cached per device).
 int device_sm_count();
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` (the

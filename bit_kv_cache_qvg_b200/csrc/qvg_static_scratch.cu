@@ -21,6 +21,7 @@
 #include <mutex>
 
 #include "qvg.h"
+#include "qvg_launch.h"
 
 namespace {
 
@@ -69,5 +70,6 @@ extern "C" QVG_API qvg_status qvg_quantize_static(const qvg_config* cfg, const v
   // scratch needs initialising (every other region is written before read).
   if (cudaMemsetAsync(scratch, 0, 16, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return QVG_ERR_CUDA;
-  return qvg_quantize(cfg, X, dtype, N, H, d, init_centroids, out, scratch, kStaticScratchBytes, stream);
+  // One wave at a time on the caller's stream: no side stream, no events.
+  return qvg::quantize_impl(cfg, X, dtype, N, H, d, init_centroids, out, scratch, kStaticScratchBytes, stream, 1);
 }

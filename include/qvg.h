@@ -109,9 +109,12 @@ QVG_API size_t qvg_packed_bytes(const qvg_config* cfg, int64_t N, int32_t H, int
                         qvg_dtype dtype);
 
 /* Device scratch bytes qvg_quantize needs to process `H` blocks of N tokens
- * in the library's preferred batch.  Any ws_bytes >= qvg_workspace_bytes(cfg,
- * N, 1, d, dtype) works (the call then processes fewer blocks at a time).
- * Returns 0 for invalid arguments.  Host-only, no CUDA call. */
+ * in the library's preferred batch: one wave of up to one block per SM, or
+ * two waves in flight when H needs more than one wave.  Any ws_bytes >=
+ * qvg_workspace_bytes(cfg, N, 1, d, dtype) works (the call then processes
+ * fewer blocks at a time, one wave at a time if two do not fit).
+ * Returns 0 for invalid arguments.  Host-only apart from reading the SM
+ * count of the current device. */
 QVG_API size_t qvg_workspace_bytes(const qvg_config* cfg, int64_t N, int32_t H, int32_t d,
                            qvg_dtype dtype);
 
@@ -131,6 +134,11 @@ QVG_API size_t qvg_workspace_bytes(const qvg_config* cfg, int64_t N, int32_t H, 
  *     (q = 0 when s = 0); E4M3 rounds to nearest even and saturates at 448.
  *   workspace: DEVICE scratch of ws_bytes bytes (see qvg_workspace_bytes),
  *     256-byte aligned, not shared with concurrent calls.
+ *   Streams: the work is ordered after the work queued on `stream` before
+ *     the call, and `stream` waits for all of it at the end.  When two waves
+ *     of blocks fit in the workspace, every other wave runs on a second
+ *     stream that the library creates once per device, joined to `stream` by
+ *     events (a stream capture of `stream` captures both).
  * Errors: INVALID_ARG for NULL pointers, K < 1 or K > 256, T < 0, bits != 2,
  * G not dividing d or not a multiple of 4, N < 1, H < 1, N < K on a cold
  * start with T > 0, iters < 1 (or warm_iters < 1 when warm) with T > 0;

@@ -217,3 +217,27 @@ def test_tensor_core_and_exact_assignment_agree(q, monkeypatch):
     print(f"near-tie tokens decided exactly: {flagged} of {total} ({flagged / total:.4%})")
     assert 0 <= flagged < 0.2 * total
     assert q.workspace_status(ws) == 0
+
+
+@pytest.mark.gpu
+def test_waves_on_two_streams_match_one_wave(q, monkeypatch):
+    """Blocks in several waves -- alternating between the caller's stream and
+    the library's second stream, or all on one stream -- give the same packed
+    stream as one wave holding every block (waves are independent)."""
+    from bit_kv_cache_qvg_b200 import synth
+    X = synth.block_batch(6, synth.KVShape(3, 30, 52), seed=91, kinds=[0, 1] * 3, device="cuda")
+    H, N = X.shape[0], X.shape[1]
+    cfg = q.config(K=256, T=2, group_size=64, iters=4)
+    one_wave = packed_np(q.quantize(X, cfg, workspace=q.alloc_workspace(cfg, N, H)))
+    # room for two one-block waves: six waves, alternating lanes
+    ws = torch.zeros(2 * q.workspace_bytes(cfg, N, 1), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        two_lanes = packed_np(q.quantize(X, cfg, workspace=ws, stream=stream))
+    assert q.workspace_status(ws, stream=stream) == 0
+    monkeypatch.setenv("QVG_WAVE_LANES", "1")
+    one_lane = packed_np(q.quantize(X, cfg, workspace=ws))
+    torch.cuda.synchronize()
+    for k in one_wave:
+        np.testing.assert_array_equal(two_lanes[k], one_wave[k])
+        np.testing.assert_array_equal(one_lane[k], one_wave[k])
