@@ -54,6 +54,10 @@ WORKLOADS = {
                         "tokens appended in chunks of 3 frames (4,680 tokens; last chunk 1 frame), "
                         "up to 1,092,000 tokens, d=128, bf16; K=256, T=2, G=64; warm start 3 "
                         "Lloyd iterations vs 10 cold; whole cache dequantised after every chunk"),
+    "sweep": dict(layers=1, heads=32, frames=25, gh=38, gw=40, K=256, T=2, G=64, iters=10, sweep=True,
+                  desc="Design sweep on one layer: 32 heads x K/V, 38,000 tokens (25 frames x 38x40), "
+                       "d=128, bf16; T in {0,1,2,3,4} x G in {16,32,64} x K in {64,256}, 10 Lloyd "
+                       "iterations (T=0: plain per-group 2-bit rounding)"),
 }
 
 
@@ -275,6 +279,12 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
+    if wl.get("sweep"):
+        run_sweep(args, wl, qvg, synth, dev, dist, rank, world, peaks)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     if "chunk_frames" in wl:
         run_stream(args, wl, qvg, synth, dev, dist, rank, world, local, peaks)
         if dist is not None:
@@ -474,6 +484,87 @@ def dequant_alg_bytes(U, n, chunks, K, T, G, esz=2):
     over `chunks` chunks: codes + E4M3 scale/zero + assignments read, output
     written, and every chunk's T centroid tables read once."""
     return U * n * 128 * (2 / 8 + 2 / G + T / 128 + esz) + chunks * T * U * K * 128 * esz
+
+
+def bits_per_element(K, T, G, N, d=128, bits=2, esz=2):
+    """Closed form of the packed size per element: the code, the two E4M3
+    bytes of each group, T uint8 assignments per token and T centroid tables
+    of K x d values per block."""
+    return bits + 16.0 / G + 8.0 * T / d + 8.0 * esz * T * K / N
+
+
+def compression_ratio(K, T, G, N, d=128, bits=2, esz=2):
+    return 8.0 * esz / bits_per_element(K, T, G, N, d, bits, esz)
+
+
+def run_sweep(args, wl, qvg, synth, dev, dist, rank, world, peaks):
+    """Design sweep over (T, G, K) on one layer of the LongCat shape: per point
+    the reconstruction error of K and V blocks, the compression ratio (packed
+    bytes, checked against its closed form), and the quantise and dequantise
+    rates, each timed with CUDA events on the launching stream."""
+    import torch
+    Hh = wl["heads"]
+    U = 2 * Hh
+    N = wl["frames"] * wl["gh"] * wl["gw"]
+    kinds = [0] * Hh + [1] * Hh
+    X = synth.block_batch(U, synth.KVShape(wl["frames"], wl["gh"], wl["gw"]), seed=synth.unit_seed(rank, 0, 0, 0),
+                          kinds=kinds, device=dev)
+    Y = torch.empty_like(X)
+    kv_bytes = U * N * 128 * 2
+    stream = torch.cuda.Stream(dev)
+    xx = [float((X[h].float() ** 2).sum()) for h in range(U)]
+
+    def rel_err(lo, hi):
+        num = sum(float(((Y[h].float() - X[h].float()) ** 2).sum()) for h in range(lo, hi))
+        return num / sum(xx[lo:hi])
+
+    points = []
+    grid = [(0, G, 0) for G in (16, 32, 64)] + [(T, G, K) for T in (1, 2, 3, 4) for G in (16, 32, 64)
+                                               for K in (64, 256)]
+    for T, G, K in grid:
+        cfg = qvg.config(K=max(K, 1), T=T, group_size=G, iters=wl["iters"])
+        packed = qvg.alloc_packed(cfg, N, U, device=dev)
+        ws = qvg.alloc_workspace(cfg, N, U, device=dev)
+        with torch.cuda.stream(stream):
+            qvg.quantize(X, cfg, out=packed, workspace=ws, stream=stream)     # warm-up
+            qvg.dequantize(packed, Y, stream=stream)
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            tq = td = 0.0
+            for _ in range(args.steps):
+                e[0].record(stream)
+                qvg.quantize(X, cfg, out=packed, workspace=ws, stream=stream)
+                e[1].record(stream)
+                qvg.dequantize(packed, Y, stream=stream)
+                e[2].record(stream)
+                torch.cuda.synchronize()
+                tq += e[0].elapsed_time(e[1])
+                td += e[1].elapsed_time(e[2])
+        tq /= args.steps
+        td /= args.steps
+        if qvg.workspace_status(ws) != 0:
+            raise SystemExit("device-side wait timed out in the sweep")
+        nbytes = packed.nbytes()
+        ratio = kv_bytes / nbytes
+        closed = compression_ratio(K, T, G, N)
+        points.append({"T": T, "G": G, "K": K if T else None, "rel_mse_K": rel_err(0, Hh), "rel_mse_V": rel_err(Hh, U),
+                       "packed_bytes": nbytes, "compression": ratio, "compression_closed_form": closed,
+                       "closed_form_matches": abs(ratio - closed) < 1e-9 * closed,
+                       "quantize_ms": tq, "quantize_GBps": kv_bytes / (tq / 1e3) / 1e9,
+                       "dequant_ms": td, "dequant_GBps": dequant_alg_bytes(U, N, 1, K, T, G) / (td / 1e3) / 1e9})
+        del packed, ws
+    head = next(p for p in points if (p["T"], p["G"], p["K"]) == (wl["T"], wl["G"], wl["K"]))
+    result = {
+        "metric": "design sweep: reconstruction error, compression ratio and per-pass rate over T, G, K",
+        "value": head["quantize_GBps"], "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": 1,
+        "ms_per_step": head["quantize_ms"] + head["dequant_ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl["desc"], "blocks": U, "tokens_per_block": N,
+                   "value_is": f"quantise rate at T={wl['T']}, G={wl['G']}, K={wl['K']}",
+                   "l2": "inputs larger than L2 (no flush needed)"},
+        "points": points,
+    }
+    if rank == 0:
+        print(json.dumps(result))
 
 
 def run_stream(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):

@@ -31,3 +31,23 @@ def test_dequant_bytes():
     b1 = bench.dequant_alg_bytes(64, 4680, 1, 256, 2, 64)
     b2 = bench.dequant_alg_bytes(64, 4680, 2, 256, 2, 64)
     assert b2 - b1 == 2 * 64 * 256 * 128 * 2
+
+
+def test_sweep_closed_form_matches_library_packed_size():
+    """The sweep's closed-form compression ratio is the library's packed size
+    (codes, E4M3 scale and zero, uint8 assignments, bf16 centroid tables)."""
+    from bit_kv_cache_qvg_b200 import qvg
+    for T, G, K, N in [(0, 16, 1, 38000), (1, 64, 256, 38000), (2, 64, 256, 38000), (4, 16, 64, 4680),
+                       (3, 32, 256, 1000)]:
+        cfg = qvg.config(K=K, T=T, group_size=G)
+        packed = qvg.packed_bytes(cfg, N, 1)
+        ratio = N * 128 * 2 / packed
+        assert abs(ratio - bench.compression_ratio(K, T, G, N)) < 1e-9 * ratio
+
+
+def test_sweep_grid_covers_the_design_space():
+    wl = bench.WORKLOADS["sweep"]
+    assert wl["frames"] * wl["gh"] * wl["gw"] == 38000 and wl["heads"] == 32
+    # the headline operating point: 2 bits + 0.25 (two E4M3 bytes per 64) +
+    # 0.125 (two uint8 assignments per 128 channels) + 0.2156 (two bf16 tables)
+    assert abs(bench.bits_per_element(256, 2, 64, 38000) - (2 + 0.25 + 0.125 + 16 * 2 * 256 / 38000)) < 1e-12
