@@ -180,21 +180,54 @@ __device__ __forceinline__ double exact_dist(const double* rw, const char* crow)
   return D;
 }
 
+// Every listed token of the wave is dealt out over all warps of the grid
+// (one resident wave of CTAs): the listed tokens are unevenly spread over the
+// blocks, so a split per block would leave most warps idle while a few walk a
+// long list.  Each CTA forms the prefix of the blocks' list counts, and a warp
+// finds the block of its entry by binary search.
+constexpr int kCandMaxWave = 1024;
+
 template <int DT>
 __global__ void __launch_bounds__(kCandWarps * 32)
-qvg_assign_candidates(const void* R, const void* C, const int K, const int64_t N, const uint2* list,
+qvg_assign_candidates(const void* R, const void* C, const int K, const int64_t N, const int W, const uint2* list,
                       const uint32_t* list_count, uint8_t* pi) {
   constexpr int ESZ = Store<DT>::bytes;
   __shared__ double rbuf[kCandWarps][kD];
-  const int u = blockIdx.y;
+  __shared__ int64_t s_pre[kCandMaxWave + 1];    // s_pre[u] = listed entries of blocks 0 .. u-1
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n_rows = min((int64_t)list_count[u], N);
+  if (warp == 0) {
+    const int per = (W + 31) / 32;
+    const int b0 = min(W, lane * per), b1 = min(W, b0 + per);
+    int64_t sum = 0;
+    for (int u = b0; u < b1; ++u) sum += min((int64_t)list_count[u], N);
+    int64_t incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int64_t o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    int64_t run = incl - sum;
+    for (int u = b0; u < b1; ++u) {
+      s_pre[u] = run;
+      run += min((int64_t)list_count[u], N);
+    }
+    if (lane == 31) s_pre[W] = incl;
+  }
+  __syncthreads();
+  const int64_t total = s_pre[W];
   const int64_t stride = (int64_t)gridDim.x * kCandWarps;
   double* rw = rbuf[warp];
-  const char* Ru = static_cast<const char*>(R) + (int64_t)u * N * kD * ESZ;
-  const char* Cu = static_cast<const char*>(C) + (int64_t)u * K * kD * ESZ;
   const uint32_t all = (K + 7) / 8 >= 32 ? 0xFFFFFFFFu : ((1u << ((K + 7) / 8)) - 1u);
-  for (int64_t e = (int64_t)blockIdx.x * kCandWarps + warp; e < n_rows; e += stride) {
+  for (int64_t g = (int64_t)blockIdx.x * kCandWarps + warp; g < total; g += stride) {
+    int lo = 0, hi = W - 1;                      // the last block u with s_pre[u] <= g
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pre[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    const int u = lo;
+    const int64_t e = g - s_pre[u];
+    const char* Ru = static_cast<const char*>(R) + (int64_t)u * N * kD * ESZ;
+    const char* Cu = static_cast<const char*>(C) + (int64_t)u * K * kD * ESZ;
     const uint2 ent = list[(int64_t)u * N + e];
     const int64_t tok = ent.x;
     if (tok >= N) continue;                    // warp-uniform; never true for listed tokens
@@ -221,9 +254,9 @@ qvg_assign_candidates(const void* R, const void* C, const int K, const int64_t N
       int gsel = -1;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const int g = groups ? __ffs(groups) - 1 : -1;
+        const int g8 = groups ? __ffs(groups) - 1 : -1;
         if (groups) groups &= groups - 1;
-        if (q == (lane >> 3)) gsel = g;
+        if (q == (lane >> 3)) gsel = g8;
       }
       const int k = gsel * 8 + (lane & 7);
       if (gsel >= 0 && k < K) {
@@ -629,10 +662,10 @@ cudaError_t launch_assign_exact(const AssignParams& p, int dtype, cudaStream_t s
 cudaError_t launch_assign_candidates(const void* R, const void* C, int K, int64_t N, int W,
                                      const uint2* list, const uint32_t* list_count, uint8_t* pi,
                                      cudaStream_t s) {
-  // listed tokens are few and unevenly spread over the blocks: up to 32 CTAs
-  // per block, those past a block's count return at once
-  const dim3 grid(32u, (unsigned)W);
-  qvg_assign_candidates<kBF16><<<grid, kCandWarps * 32, 0, s>>>(R, C, K, N, list, list_count, pi);
+  // one resident wave: four 8-warp CTAs per SM deal out the wave's listed tokens
+  if (W < 1 || W > kCandMaxWave) return cudaErrorInvalidValue;
+  const unsigned grid = (unsigned)(4 * device_sm_count());
+  qvg_assign_candidates<kBF16><<<grid, kCandWarps * 32, 0, s>>>(R, C, K, N, W, list, list_count, pi);
   return cudaGetLastError();
 }
 
