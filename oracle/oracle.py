@@ -60,6 +60,8 @@ def lib():
         L.ref_objective.restype = f64
         L.ref_objective.argtypes = [vp, i64, i32, vp, vp]
         L.ref_update.argtypes = [vp, i64, i32, vp, i32, i32, vp]
+        L.ref_exact_sum.restype = f64
+        L.ref_exact_sum.argtypes = [vp, i64]
         L.ref_kmeans.argtypes = [vp, i64, i32, i32, i32, i32, vp, vp, vp]
         L.ref_residual.argtypes = [vp, i64, i32, vp, vp, i32, vp]
         L.ref_group_quant.argtypes = [vp, i64, i32, i32, vp, vp, vp]
@@ -134,6 +136,12 @@ def objective(R, Cc, pi) -> float:
     R, Cc = _f32(R), _f32(Cc)
     pi = np.ascontiguousarray(pi, dtype=np.uint8)
     return float(lib().ref_objective(_p(R), R.shape[0], R.shape[1], _p(Cc), _p(pi)))
+
+
+def exact_sum(x) -> float:
+    """The exact sum of fp32 values, rounded once to fp64 (the update's sum)."""
+    x = _f32(x).ravel()
+    return float(lib().ref_exact_sum(_p(x), x.size))
 
 
 def update(R, pi, Cc, dtype=BF16) -> np.ndarray:

@@ -237,28 +237,123 @@ double ref_objective(const float* R, int64_t N, int d, const float* C,
     return J;
 }
 
-/* Update step: c_k = round_S( (sum_{pi_i = k} r_i) / n_k ), sums in fp64 over
- * tokens in ascending order, one fp64 divide, one rounding to S.  A cluster
- * with no members keeps its previous centroid (READING). */
+/* Exact sum of fp32 values.  Every fp32 value is an integer multiple of
+ * 2^-149 (the smallest subnormal), and |v| < 2^128, so v * 2^149 is an
+ * integer below 2^277; a sum of fewer than 2^40 of them fits a signed 320-bit
+ * two's-complement integer (five 64-bit words, least significant first). */
+typedef struct { uint64_t w[5]; } exact_sum;
+
+static void exact_add(exact_sum* a, float v)
+{
+    int e, sh, k;
+    uint64_t mag, lo, hi, carry;
+    int neg;
+    double m;
+    if (v == 0.0f) return;
+    m = frexp((double)v, &e);            /* v = m 2^e, 0.5 <= |m| < 1 */
+    neg = m < 0.0;
+    mag = (uint64_t)ldexp(neg ? -m : m, 24);   /* 24-bit integer significand, exact */
+    sh = e - 24 + 149;                   /* v * 2^149 = mag * 2^sh */
+    if (sh < 0) { mag >>= -sh; sh = 0; } /* subnormals: the low bits are zero */
+    /* the shifted magnitude as a 128-bit pair at word sh/64 */
+    k = sh / 64;
+    lo = mag << (sh % 64);
+    hi = (sh % 64) ? mag >> (64 - sh % 64) : 0;
+    if (!neg) {
+        uint64_t t = a->w[k] + lo;
+        carry = t < lo;
+        a->w[k] = t;
+        if (k + 1 < 5) {
+            uint64_t t2 = a->w[k + 1] + hi;
+            uint64_t c2 = t2 < hi;
+            t2 += carry;
+            c2 += t2 < carry;
+            a->w[k + 1] = t2;
+            carry = c2;
+            for (k += 2; k < 5 && carry; ++k) { a->w[k] += 1; carry = a->w[k] == 0; }
+        }
+    } else {
+        uint64_t borrow = a->w[k] < lo;
+        a->w[k] -= lo;
+        if (k + 1 < 5) {
+            uint64_t b2 = a->w[k + 1] < hi;
+            a->w[k + 1] -= hi;
+            b2 += a->w[k + 1] < borrow;
+            a->w[k + 1] -= borrow;
+            borrow = b2;
+            for (k += 2; k < 5 && borrow; ++k) { borrow = a->w[k] == 0; a->w[k] -= 1; }
+        }
+    }
+}
+
+/* The exact sum rounded once to the nearest double (ties to even). */
+static double exact_to_double(const exact_sum* a)
+{
+    uint64_t w[5];
+    int i, neg = (a->w[4] >> 63) != 0, top = -1;
+    uint64_t sig = 0, rest_nonzero = 0, half;
+    double r;
+    for (i = 0; i < 5; ++i) w[i] = a->w[i];
+    if (neg) {                           /* two's complement negate */
+        uint64_t carry = 1;
+        for (i = 0; i < 5; ++i) { w[i] = ~w[i] + carry; carry = carry && w[i] == 0; }
+    }
+    for (i = 319; i >= 0; --i)
+        if ((w[i / 64] >> (i % 64)) & 1) { top = i; break; }
+    if (top < 0) return 0.0;
+    if (top <= 52) {                     /* fits 53 bits: exact */
+        sig = w[0];
+        r = ldexp((double)sig, -149);
+        return neg ? -r : r;
+    }
+    /* bits top-52 .. top form the significand; the bits below round it */
+    for (i = 0; i < 53; ++i) {
+        const int b = top - 52 + i;
+        sig |= ((w[b / 64] >> (b % 64)) & 1) << i;
+    }
+    half = (w[(top - 53) / 64] >> ((top - 53) % 64)) & 1;
+    for (i = 0; i < top - 53; ++i)
+        if ((w[i / 64] >> (i % 64)) & 1) { rest_nonzero = 1; break; }
+    if (half && (rest_nonzero || (sig & 1))) sig += 1;   /* may carry to 2^53: still exact in a double */
+    r = ldexp((double)sig, top - 52 - 149);
+    return neg ? -r : r;
+}
+
+/* Update step ([163] 三: each group's centroid is the mean of its tokens):
+ * c_k = round_S( RN64( RN64(sum_{pi_i = k} r_i) / n_k ) ), where the sum is
+ * formed exactly and rounded once to fp64, then one fp64 divide and one
+ * rounding to S (READING: the plain mean, with one rounding per step).  A
+ * cluster with no members keeps its previous centroid (READING). */
 void ref_update(const float* R, int64_t N, int d, const uint8_t* pi, int K,
                 int dtype, float* C)
 {
-    double* sums = (double*)calloc((size_t)K * d, sizeof(double));
+    exact_sum* sums = (exact_sum*)calloc((size_t)K * d, sizeof(exact_sum));
     int64_t* cnt = (int64_t*)calloc((size_t)K, sizeof(int64_t));
     int64_t i;
     int k, j;
     for (i = 0; i < N; ++i) {
         k = pi[i];
         cnt[k] += 1;
-        for (j = 0; j < d; ++j) sums[(int64_t)k * d + j] = sums[(int64_t)k * d + j] + (double)R[i * d + j];
+        for (j = 0; j < d; ++j) exact_add(&sums[(int64_t)k * d + j], R[i * d + j]);
     }
     for (k = 0; k < K; ++k) {
         if (cnt[k] == 0) continue;
         for (j = 0; j < d; ++j)
-            C[(int64_t)k * d + j] = store_round(sums[(int64_t)k * d + j] / (double)cnt[k], dtype);
+            C[(int64_t)k * d + j] = store_round(exact_to_double(&sums[(int64_t)k * d + j]) / (double)cnt[k], dtype);
     }
     free(sums);
     free(cnt);
+}
+
+/* The exact sum of n fp32 values, rounded once to fp64 (exposed for the
+ * tests that pin the update). */
+double ref_exact_sum(const float* x, int64_t n)
+{
+    exact_sum a;
+    int64_t i;
+    memset(&a, 0, sizeof(a));
+    for (i = 0; i < n; ++i) exact_add(&a, x[i]);
+    return exact_to_double(&a);
 }
 
 /* Lloyd's iteration run exactly `iters` times, each an assignment followed by

@@ -136,3 +136,40 @@ def test_sqdist_is_fp64_sum_in_channel_order(ora):
     c = np.zeros(4, np.float32)
     # fp64: 1e16 + 1 -> 1e16 (1 lost), + 1e16, + 1 -> 2e16 exactly as ordered
     assert ora.sqdist(r, c) == ((1e16 + 1.0) + 1e16) + 1.0
+
+
+@pytest.mark.parametrize("family", ["normal", "wide", "cancel", "subnormal"])
+def test_update_sum_is_the_correctly_rounded_exact_sum(ora, family):
+    """The update's per-channel sum is the exact sum of the members rounded
+    once to fp64 -- pinned against Python's correctly rounded math.fsum."""
+    import math
+    rng = np.random.default_rng({"normal": 1, "wide": 2, "cancel": 3, "subnormal": 4}[family])
+    for _ in range(300):
+        n = int(rng.integers(1, 300))
+        if family == "normal":
+            x = rng.standard_normal(n).astype(np.float32)
+        elif family == "wide":
+            x = (rng.standard_normal(n) * np.exp2(rng.integers(-140, 120, n))).astype(np.float32)
+        elif family == "cancel":
+            b = (rng.standard_normal(n) * np.float32(1e30)).astype(np.float32)
+            x = rng.permutation(np.concatenate([b, -b, rng.standard_normal(3).astype(np.float32)]))
+        else:
+            x = (rng.integers(-5, 6, n) * np.float32(2.0 ** -149)).astype(np.float32)
+        assert ora.exact_sum(x) == math.fsum(float(v) for v in x)
+
+
+def test_update_mean_survives_cancellation(ora):
+    """Members 2^100, 1, -2^100 in one channel: an fp64 running sum would lose
+    the 1; the mean is 1/3, rounded to bf16 (and to fp32)."""
+    import torch
+    X = np.zeros((3, 4), np.float32)
+    X[:, 0] = [2.0 ** 100, 1.0, -(2.0 ** 100)]
+    X[:, 1] = [1.0, 2.0, 4.0]
+    pi = np.zeros(3, np.uint8)
+    C0 = np.full((1, 4), 7.0, np.float32)
+    third_bf16 = float(torch.tensor(1.0 / 3.0, dtype=torch.float64).to(torch.bfloat16).float())
+    Cb = ora.update(X, pi, C0, dtype=BF16)
+    assert Cb[0, 0] == np.float32(third_bf16)
+    assert Cb[0, 1] == np.float32(float(torch.tensor(7.0 / 3.0, dtype=torch.float64).to(torch.bfloat16).float()))
+    Cf = ora.update(X, pi, C0, dtype=FP32)
+    assert Cf[0, 0] == np.float32(1.0 / 3.0)
