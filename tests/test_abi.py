@@ -102,3 +102,20 @@ def test_dequantize_and_cache_reject_bad_arguments(q):
     assert L.qvg_cache_create(C.byref(cfg), 0, 1, 96, 100, 4, C.byref(h)) == 2
     assert L.qvg_append_chunk(None, 0x1000, 10, None) == 1
     assert L.qvg_cache_tokens(None) == 0 and L.qvg_cache_chunks(None) == 0
+
+
+def test_workspace_covers_two_waves_when_blocks_exceed_one(q, monkeypatch):
+    """Host logic of the wave lanes: a wave holds up to one block per SM (the
+    SM count the library reads; 148 on this part, the fallback without a
+    device); when the blocks need more than one wave the workspace holds two
+    waves, one per lane; QVG_WAVE_LANES=1 asks for one wave."""
+    cfg = q.config(K=256, T=2, group_size=64)
+    N = 38000
+    sizes = {H: q.workspace_bytes(cfg, N, H) for H in range(1, 400)}
+    # past one wave the size no longer grows with H: W is the largest one-wave batch
+    W = min(H for H in sizes if sizes[H] == sizes[399]) - 1
+    assert all(sizes[H] < sizes[H + 1] for H in range(1, W))
+    assert sizes[W + 1] == 2 * sizes[W]
+    assert all(sizes[H] == 2 * sizes[W] for H in range(W + 1, 400))
+    monkeypatch.setenv("QVG_WAVE_LANES", "1")
+    assert q.workspace_bytes(cfg, N, W + 1) == sizes[W]
