@@ -687,17 +687,17 @@ def run_stream(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
                      "frac": ach / peaks["hbm"], "traffic": None, "kernel": "qvg_dequant_fused",
                      "at": f"full cache, {total} tokens x {U} blocks, {nch} chunks",
                      "alg_bytes_per_launch": dequant_alg_bytes(U, total, nch, K, T, G)},
-        "gpu_launches": None,
         "clocks": clk.summary(),
     }
+    # launches of the library's kernels: one whole-cache dequant, and one warm
+    # append into a scratch cache (its profile is also the kernel breakdown)
     qvg.profile_reset()
     qvg.profile_enable(True)
     with torch.cuda.stream(stream):
         cache.dequantize(ybuf[:U * total * 128].view(U, total, 128), stream=stream)
     torch.cuda.synchronize()
     qvg.profile_enable(False)
-    result["gpu_launches"] = {"per_dequant": qvg.profile_launches(), "per_append": None}
-    # one more append into a scratch cache counts the launches of one warm append
+    per_dequant = qvg.profile_launches()
     scache = qvg.Cache(cfg, U, 2 * sizes[0], 2)
     g2 = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=kinds, seed=seed + 2, device=dev)
     with torch.cuda.stream(stream):
@@ -708,10 +708,12 @@ def run_stream(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
         scache.append(g2.next(wl["chunk_frames"]), stream=stream)
         torch.cuda.synchronize()
         qvg.profile_enable(False)
-    result["gpu_launches"]["per_append"] = qvg.profile_launches()
+    per_append = qvg.profile_launches()
     result["kernels_warm_append"] = qvg.profile_report()
     scache.close()
-    result["gpu_launches"] = nch * (result["gpu_launches"]["per_dequant"] + result["gpu_launches"]["per_append"])
+    # every chunk of the timed pass: one append and one whole-cache dequant
+    result["gpu_launches"] = nch * (per_dequant + per_append)
+    result["gpu_launches_per_chunk"] = {"append": per_append, "dequant": per_dequant}
     if rank == 0 and not args.no_e2e:
         result["e2e"] = stream_e2e(args, wl, qvg, synth, cfg, sizes, dev, stream)
     if rank == 0 and not args.no_cpu_baseline:
