@@ -11,6 +11,7 @@ iterations.  The metric is KV GB/s: uncompressed bf16 KV bytes / step time.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload longcat|chunk]
     python bench.py --workload stream      # streaming cache, one line of its own
+    python bench.py --workload sweep       # design sweep over T, G, K, one line
     python bench.py --impl reference ...   # the oracle on the host cores
 
 The stream workload appends 234 chunks (700 frames of 30x52 tokens, 3 frames
