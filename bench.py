@@ -41,6 +41,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "KV GB/s: fused dequant + k-means/2-bit quantize, as % of B200 HBM roofline"
 STREAM_METRIC = "streaming append: per-chunk quantize latency (warm start), with whole-cache dequant GB/s"
+SWEEP_METRIC = "design sweep: reconstruction error, compression ratio and per-pass rate over T, G, K"
 
 WORKLOADS = {
     "longcat": dict(layers=48, heads=32, frames=25, gh=38, gw=40, K=256, T=2, G=64, iters=10,
@@ -152,9 +153,10 @@ def weak_scaling_value(bytes_per_rank: float, world: int, ms: float) -> float:
 
 
 # ---------------------------------------------------------------- oracle arm
-def oracle_sample(wl, tokens: int, seed: int = 99):
-    """Time the oracle's quantise + dequantise of one block of `tokens` tokens
-    of the workload's shape on the host cores.  Returns (seconds, bytes, threads)."""
+def oracle_sample(wl, tokens: int, seed: int = 99, dequant: bool = True):
+    """Time the oracle's quantise (+ dequantise unless `dequant` is False) of
+    one block of `tokens` tokens of the workload's shape on the host cores.
+    Returns (seconds, bytes, threads)."""
     import numpy as np
     from bit_kv_cache_qvg_b200 import synth
     from oracle import oracle as o
@@ -164,7 +166,8 @@ def oracle_sample(wl, tokens: int, seed: int = 99):
     Xb = X.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
     t0 = time.perf_counter()
     p = o.quantize(Xb, K=wl["K"], T=wl["T"], G=wl["G"], iters=wl["iters"])
-    o.dequantize(p, K=wl["K"], T=wl["T"], G=wl["G"], N=tokens, H=1, d=128)
+    if dequant:
+        o.dequantize(p, K=wl["K"], T=wl["T"], G=wl["G"], N=tokens, H=1, d=128)
     dt = time.perf_counter() - t0
     return dt, tokens * 128 * 2, o.get_threads()
 
@@ -212,16 +215,19 @@ def run_reference(args, wl, rank, world):
         }))
         return
     tokens = args.ref_tokens
+    sweep = bool(wl.get("sweep"))          # the sweep's value is the quantise rate
     times = []
     for i in range(args.warmup + args.steps):
-        dt, nbytes, threads = oracle_sample(wl, tokens, seed=1000 + i)
+        dt, nbytes, threads = oracle_sample(wl, tokens, seed=1000 + i, dequant=not sweep)
         if i >= args.warmup:
             times.append(dt)
     t = sum(times) / len(times)
     v = nbytes / t / 1e9
-    sample = f"one V block of {tokens} tokens of the workload's shape per step (quantise + dequantise)"
+    sample = (f"one V block of {tokens} tokens of the workload's shape per step "
+              + (f"(quantise at T={wl['T']}, G={wl['G']}, K={wl['K']})" if sweep else "(quantise + dequantise)"))
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": SWEEP_METRIC if sweep else METRIC, "value": v, "unit": "GB/s",
+        "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl["desc"], "reference": "C oracle (fp64 k-means) on host cores"},
@@ -555,7 +561,7 @@ def run_sweep(args, wl, qvg, synth, dev, dist, rank, world, peaks):
         del packed, ws
     head = next(p for p in points if (p["T"], p["G"], p["K"]) == (wl["T"], wl["G"], wl["K"]))
     result = {
-        "metric": "design sweep: reconstruction error, compression ratio and per-pass rate over T, G, K",
+        "metric": SWEEP_METRIC,
         "value": head["quantize_GBps"], "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": 1,
         "ms_per_step": head["quantize_ms"] + head["dequant_ms"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",

@@ -1,6 +1,8 @@
-"""Host logic of the streaming bench line: the chunk schedule of a long
-generation (700 frames in chunks of 3, the last chunk of 1 frame) and the
-algorithmic bytes of one fused dequant of the growing cache."""
+"""Host logic of the bench's extra workloads: the streaming line's chunk
+schedule (700 frames in chunks of 3, the last chunk of 1 frame) and the
+algorithmic bytes of one fused dequant of the growing cache; the design
+sweep's closed-form compression ratio; and the oracle reference arm of both
+lines (run on the host cores)."""
 import os
 import sys
 
@@ -8,6 +10,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
+import pytest  # noqa: E402
 
 
 def test_chunk_schedule():
@@ -51,3 +54,20 @@ def test_sweep_grid_covers_the_design_space():
     # the headline operating point: 2 bits + 0.25 (two E4M3 bytes per 64) +
     # 0.125 (two uint8 assignments per 128 channels) + 0.2156 (two bf16 tables)
     assert abs(bench.bits_per_element(256, 2, 64, 38000) - (2 + 0.25 + 0.125 + 16 * 2 * 256 / 38000)) < 1e-12
+
+
+@pytest.mark.parametrize("workload", ["stream", "sweep"])
+def test_reference_arm_prints_one_line(workload):
+    """--impl reference runs the oracle on the host cores and prints the
+    workload's own metric with the reference keys (no GPU involved)."""
+    import json
+    import subprocess
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                          workload, "--steps", "1", "--warmup", "0", "--ref-tokens", "1600"],
+                         capture_output=True, text=True, timeout=600, check=True).stdout.strip().splitlines()
+    line = json.loads(out[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["metric"] == (bench.STREAM_METRIC if workload == "stream" else bench.SWEEP_METRIC)
+    for key in ("unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "cpu_baseline", "e2e"):
+        assert key in line
+    assert line["cpu_baseline"]["kind"] == "oracle"
