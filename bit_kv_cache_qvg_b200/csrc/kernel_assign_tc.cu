@@ -235,6 +235,10 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 }
 
 
+// NCH > 0 fixes the number of 32-column chunks at compile time (8 for
+// K = 256), so the epilogue's chunk guards fold away; NCH = 0 reads it from
+// the padded centroid count.
+template <int NCH>
 __global__ void __launch_bounds__(kTcThreads, 1)
 qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmC,
                   const TcParams p) {
@@ -371,7 +375,7 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
     const int q = warp & 3;
     const int hc = (warp - 2) >> 2;
     const int row = q * 32 + lane;
-    const int nch = Npad >> 5;                 // 32-column chunks (>= 1)
+    const int nch = NCH > 0 ? NCH : (Npad >> 5);   // 32-column chunks (>= 1)
     float rn2_next = 0.0f;
     {
       const int64_t tok = (int64_t)(t_begin + hc) * kTileM + row;
@@ -577,7 +581,10 @@ cudaError_t launch_assign_tc(const AssignTcParams& a, cudaStream_t s) {
   p.gamma = a.gamma;
   p.unit = 1;
   const size_t smem = assign_tc_smem_bytes(a.K);
-  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(qvg_kmeans_assign), smem);
+  const bool full = Npad == 256;
+  const void* fn = full ? reinterpret_cast<const void*>(qvg_kmeans_assign<8>)
+                        : reinterpret_cast<const void*>(qvg_kmeans_assign<0>);
+  cudaError_t e = ensure_dynamic_smem(fn, smem);
   if (e != cudaSuccess) return e;
 #ifdef QVG_TC_DEBUG
   {
@@ -585,7 +592,10 @@ cudaError_t launch_assign_tc(const AssignTcParams& a, cudaStream_t s) {
     cudaMemcpyToSymbol(g_tc_dbg, z, sizeof(z));
   }
 #endif
-  qvg_kmeans_assign<<<dim3((unsigned)splits, (unsigned)a.W), kTcThreads, smem, s>>>(mR, mC, p);
+  if (full)
+    qvg_kmeans_assign<8><<<dim3((unsigned)splits, (unsigned)a.W), kTcThreads, smem, s>>>(mR, mC, p);
+  else
+    qvg_kmeans_assign<0><<<dim3((unsigned)splits, (unsigned)a.W), kTcThreads, smem, s>>>(mR, mC, p);
 #ifdef QVG_TC_DEBUG
   {
     cudaError_t le = cudaDeviceSynchronize();
