@@ -354,7 +354,7 @@ __device__ __forceinline__ uint32_t quant_chunk(const float (&r)[8], float lo, f
   const float s = tab.dec[scb];
   sc_out = scb;
   zc_out = zc;
-  if (s == 0.0f) return 0u;
+  // s = 0 needs no branch: y = 0 makes every quotient +-0, hence code 0
   const float y = tab.rcp[scb];
   const float2 nm2 = f2(-m, -m), y2 = f2(y, y), ns2 = f2(-s, -s), k2 = f2(kRound, kRound), nk2 = f2(-kRound, -kRound);
   float2 pk2 = f2(0.0f, 0.0f);
@@ -371,7 +371,10 @@ __device__ __forceinline__ uint32_t quant_chunk(const float (&r)[8], float lo, f
   return __float_as_uint(__fadd_rn(pk, 8388608.0f)) & 0xFFFFu;   // 2^23: integer in the low bits
 }
 
-template <int DT, bool QUANT, bool HAS_C>
+// GT > 0 fixes the group size at compile time (the quantising pass is
+// instantiated for every supported G, so its group reductions and stores fold
+// to straight-line code); GT = 0 reads it from the parameters.
+template <int DT, bool QUANT, bool HAS_C, int GT>
 __global__ void __launch_bounds__(kRqThreads)
 qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
   constexpr int ESZ = Store<DT>::bytes;
@@ -408,8 +411,8 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
 #pragma unroll
   for (int e = 0; e < 8; ++e) { mx0[e] = 0.0f; mx1[e] = 0.0f; }
   const int j = threadIdx.x & 7;
-  const int ng = kD / p.G;
-  const int G = p.G;
+  const int G = GT > 0 ? GT : p.G;
+  const int ng = kD / G;
   const char* Rin = static_cast<const char*>(p.R_in) + (int64_t)u * p.N * kD * ESZ;
   // The loop bound is uniform across the warp (4 tokens per warp per
   // iteration) so that the group shuffles below always run on all 32 lanes;
@@ -573,12 +576,27 @@ cudaError_t launch_dequant(const DequantParams& p, int dtype, cudaStream_t s) {
                         : launch_dq_t<kFP32>(p, blocks, splits, smem, s);
 }
 
+template <int DT, bool Q, bool C, int GT>
+static cudaError_t launch_rq_g(const ResidualParams& p, dim3 grid, int64_t per, size_t smem, cudaStream_t s) {
+  cudaError_t e = set_smem(qvg_residual_quant<DT, Q, C, GT>, smem);
+  if (e != cudaSuccess) return e;
+  qvg_residual_quant<DT, Q, C, GT><<<grid, kRqThreads, smem, s>>>(p, per);
+  return cudaGetLastError();
+}
+
+// The quantising pass takes the instance of its group size; the others do
+// not use G.
 template <int DT, bool Q, bool C>
 static cudaError_t launch_rq(const ResidualParams& p, dim3 grid, int64_t per, size_t smem, cudaStream_t s) {
-  cudaError_t e = set_smem(qvg_residual_quant<DT, Q, C>, smem);
-  if (e != cudaSuccess) return e;
-  qvg_residual_quant<DT, Q, C><<<grid, kRqThreads, smem, s>>>(p, per);
-  return cudaGetLastError();
+  if (!Q) return launch_rq_g<DT, Q, C, 0>(p, grid, per, smem, s);
+  switch (p.G) {
+    case 8: return launch_rq_g<DT, Q, C, 8>(p, grid, per, smem, s);
+    case 16: return launch_rq_g<DT, Q, C, 16>(p, grid, per, smem, s);
+    case 32: return launch_rq_g<DT, Q, C, 32>(p, grid, per, smem, s);
+    case 64: return launch_rq_g<DT, Q, C, 64>(p, grid, per, smem, s);
+    case 128: return launch_rq_g<DT, Q, C, 128>(p, grid, per, smem, s);
+    default: return launch_rq_g<DT, Q, C, 0>(p, grid, per, smem, s);
+  }
 }
 
 cudaError_t launch_residual(const ResidualParams& p, int dtype, bool quant, cudaStream_t s) {
