@@ -245,16 +245,21 @@ typedef struct { uint64_t w[5]; } exact_sum;
 
 static void exact_add(exact_sum* a, float v)
 {
-    int e, sh, k;
+    int sh, k, ex;
     uint64_t mag, lo, hi, carry;
     int neg;
-    double m;
+    uint32_t bits;
     if (v == 0.0f) return;
-    m = frexp((double)v, &e);            /* v = m 2^e, 0.5 <= |m| < 1 */
-    neg = m < 0.0;
-    mag = (uint64_t)ldexp(neg ? -m : m, 24);   /* 24-bit integer significand, exact */
-    sh = e - 24 + 149;                   /* v * 2^149 = mag * 2^sh */
-    if (sh < 0) { mag >>= -sh; sh = 0; } /* subnormals: the low bits are zero */
+    memcpy(&bits, &v, sizeof(bits));     /* IEEE binary32: sign, 8-bit exponent, 23-bit fraction */
+    neg = (int)(bits >> 31);
+    ex = (int)((bits >> 23) & 0xFF);
+    mag = bits & 0x7FFFFFu;
+    if (ex == 0) {
+        sh = 0;                          /* subnormal: v = fraction * 2^-149 */
+    } else {
+        mag |= 0x800000u;                /* normal: v = (2^23 + fraction) * 2^(ex - 150) */
+        sh = ex - 1;                     /* v * 2^149 = mag * 2^sh */
+    }
     /* the shifted magnitude as a 128-bit pair at word sh/64 */
     k = sh / 64;
     lo = mag << (sh % 64);
@@ -298,8 +303,8 @@ static double exact_to_double(const exact_sum* a)
         uint64_t carry = 1;
         for (i = 0; i < 5; ++i) { w[i] = ~w[i] + carry; carry = carry && w[i] == 0; }
     }
-    for (i = 319; i >= 0; --i)
-        if ((w[i / 64] >> (i % 64)) & 1) { top = i; break; }
+    for (i = 4; i >= 0; --i)             /* the highest set bit */
+        if (w[i]) { top = 64 * i + 63 - __builtin_clzll(w[i]); break; }
     if (top < 0) return 0.0;
     if (top <= 52) {                     /* fits 53 bits: exact */
         sig = w[0];
@@ -312,8 +317,11 @@ static double exact_to_double(const exact_sum* a)
         sig |= ((w[b / 64] >> (b % 64)) & 1) << i;
     }
     half = (w[(top - 53) / 64] >> ((top - 53) % 64)) & 1;
-    for (i = 0; i < top - 53; ++i)
-        if ((w[i / 64] >> (i % 64)) & 1) { rest_nonzero = 1; break; }
+    {                                    /* any set bit below bit top - 53 */
+        const int b = top - 53, wb = b / 64, ob = b % 64;
+        for (i = 0; i < wb; ++i) rest_nonzero |= w[i] != 0;
+        if (ob) rest_nonzero |= (w[wb] & ((1ull << ob) - 1ull)) != 0;
+    }
     if (half && (rest_nonzero || (sig & 1))) sig += 1;   /* may carry to 2^53: still exact in a double */
     r = ldexp((double)sig, top - 52 - 149);
     return neg ? -r : r;
@@ -331,11 +339,12 @@ void ref_update(const float* R, int64_t N, int d, const uint8_t* pi, int K,
     int64_t* cnt = (int64_t*)calloc((size_t)K, sizeof(int64_t));
     int64_t i;
     int k, j;
-    for (i = 0; i < N; ++i) {
-        k = pi[i];
-        cnt[k] += 1;
-        for (j = 0; j < d; ++j) exact_add(&sums[(int64_t)k * d + j], R[i * d + j]);
-    }
+    for (i = 0; i < N; ++i) cnt[pi[i]] += 1;
+    /* Channels are independent and exact sums do not depend on the order of
+     * the adds, so the channels may be summed by different threads. */
+#pragma omp parallel for schedule(static) private(i)
+    for (j = 0; j < d; ++j)
+        for (i = 0; i < N; ++i) exact_add(&sums[(int64_t)pi[i] * d + j], R[i * d + j]);
     for (k = 0; k < K; ++k) {
         if (cnt[k] == 0) continue;
         for (j = 0; j < d; ++j)
