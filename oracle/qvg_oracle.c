@@ -22,8 +22,9 @@
  *
  * Arithmetic rules: build with -O2 -ffp-contract=off and no fast-math, so that
  * every multiply and add below is one IEEE operation in the written order.
- * Distances and centroid sums are fp64.  Residuals and quantisation use fp32
- * operations, as the data is stored in 16/32-bit floats.
+ * Distances are fp64.  Centroid sums are exact (a wide integer), rounded once
+ * to fp64 before the divide.  Residuals and quantisation use fp32 operations,
+ * as the data is stored in 16/32-bit floats.
  *
  * Parity status: every function here is pinned by the tests under tests/
  * (format round trips against library casts, closed forms, worked examples,
