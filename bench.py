@@ -152,6 +152,20 @@ def weak_scaling_value(bytes_per_rank: float, world: int, ms: float) -> float:
     return bytes_per_rank * world / (ms / 1e3) / 1e9
 
 
+def shard_units(n: int, world: int, rank: int):
+    """Contiguous share [first, last) of n units (heads) for `rank` of
+    `world`; the shares partition [0, n) and differ in size by at most one."""
+    base, extra = divmod(n, world)
+    first = rank * base + min(rank, extra)
+    return first, first + base + (1 if rank < extra else 0)
+
+
+def strong_scaling_value(total_bytes: float, ms: float) -> float:
+    """Whole-job GB/s when the ranks share one cache: its bytes over the
+    slowest rank's time."""
+    return total_bytes / (ms / 1e3) / 1e9
+
+
 # ---------------------------------------------------------------- oracle arm
 def oracle_sample(wl, tokens: int, seed: int = 99, dequant: bool = True):
     """Time the oracle's quantise (+ dequantise unless `dequant` is False) of
@@ -251,6 +265,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=4750)
     ap.add_argument("--cpu-tokens", type=int, default=9500)
     ap.add_argument("--frames", type=int, default=None, help="override the frame count")
+    ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
+                    help="weak: every rank its own cache; strong: the ranks share one cache by heads")
     args = ap.parse_args()
     wl = dict(WORKLOADS[args.workload])
     if args.layers:
@@ -299,19 +315,29 @@ def main():
             dist.destroy_process_group()
         return
 
-    L, Hh = wl["layers"], wl["heads"]
+    L, Hh_all = wl["layers"], wl["heads"]
     N = wl["frames"] * wl["gh"] * wl["gw"]
+    strong = args.scaling == "strong"
+    # weak: every rank holds a whole cache; strong: heads h0 .. h1-1 of one cache
+    h0, h1 = shard_units(Hh_all, world, rank) if strong else (0, Hh_all)
+    if h1 <= h0:
+        raise SystemExit("strong scaling needs at least one head per rank")
+    Hh = h1 - h0                        # heads on this rank
     U = L * 2 * Hh                      # blocks: layer x {K, V} x head
     K, T, G, I = wl["K"], wl["T"], wl["G"], wl["iters"]
     cfg = qvg.config(K=K, T=T, group_size=G, iters=I)
 
-    # inputs resident in HBM (generated per layer on the device, seeded per rank)
+    # inputs resident in HBM, generated per layer on the device: seeded per
+    # rank for weak scaling, per cache (the same on every rank) for strong
     X = torch.empty((U, N, 128), dtype=torch.bfloat16, device=dev)
     for l in range(L):
-        kinds = [0] * Hh + [1] * Hh
-        X[l * 2 * Hh:(l + 1) * 2 * Hh] = synth.block_batch(
-            2 * Hh, synth.KVShape(wl["frames"], wl["gh"], wl["gw"]), seed=synth.unit_seed(rank, l, 0, 0),
-            kinds=kinds, device=dev)
+        kinds = [0] * Hh_all + [1] * Hh_all
+        layer = synth.block_batch(
+            2 * Hh_all, synth.KVShape(wl["frames"], wl["gh"], wl["gw"]),
+            seed=synth.unit_seed(0 if strong else rank, l, 0, 0), kinds=kinds, device=dev)
+        X[l * 2 * Hh:l * 2 * Hh + Hh] = layer[h0:h1]                   # K heads
+        X[l * 2 * Hh + Hh:(l + 1) * 2 * Hh] = layer[Hh_all + h0:Hh_all + h1]   # V heads
+        del layer
     packed = qvg.alloc_packed(cfg, N, U, device=dev)
     ws = qvg.alloc_workspace(cfg, N, U, device=dev)
     Y = torch.empty_like(X)
@@ -396,7 +422,8 @@ def main():
     eager_ms = pe0.elapsed_time(pe1)
     flagged = qvg.workspace_flagged(ws)
     kv_bytes = U * N * 128 * 2
-    value = weak_scaling_value(kv_bytes, world, ms)
+    total_bytes = L * 2 * Hh_all * N * 128 * 2
+    value = strong_scaling_value(total_bytes, ms) if strong else weak_scaling_value(kv_bytes, world, ms)
 
     # roofline of the kernels (algorithmic work per launch / mean launch time)
     E = U * N * 128
@@ -444,12 +471,14 @@ def main():
 
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong" if strong else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl["desc"], "blocks_per_gpu": U, "tokens_per_block": N,
                    "uncompressed_bytes_per_gpu": kv_bytes, "packed_bytes_per_gpu": packed.nbytes(),
                    "l2": "inputs larger than L2 (no flush needed)" if kv_bytes > 126e6 else "L2 flushed",
-                   "parallelism": f"weak: {world} rank(s), independent caches"},
+                   "parallelism": (f"strong: {world} rank(s) share one cache by heads (rank 0: heads {h0}-{h1 - 1})"
+                                   if strong else f"weak: {world} rank(s), independent caches")},
         "roofline": dominant,
         "rooflines": roof,
         "quantize_path": {"ms_per_step": q_ms, "roofline_ms": q_roof_ms, "frac": q_roof_ms / q_ms if q_ms else None,
@@ -466,7 +495,8 @@ def main():
 
     # end to end through the public API with host buffers (pinned), per layer
     if not args.no_e2e:
-        result["e2e"] = e2e(args, qvg, cfg, X, Y, packed, ws, L, Hh, N, dev, world, dist)
+        result["e2e"] = e2e(args, qvg, cfg, X, Y, packed, ws, L, Hh, N, dev, world, dist,
+                            total_bytes=total_bytes if strong else None)
     if rank == 0 and not args.no_cpu_baseline:
         dt, nbytes, threads = oracle_sample(wl, args.cpu_tokens)
         result["cpu_baseline"] = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
@@ -773,7 +803,7 @@ def stream_e2e(args, wl, qvg, synth, cfg, sizes, dev, stream, chunks=40):
             "api": "qvg_append_chunk with the chunk from pinned host memory and its packed form back"}
 
 
-def e2e(args, qvg, cfg, X, Y, packed, ws, L, Hh, N, dev, world, dist):
+def e2e(args, qvg, cfg, X, Y, packed, ws, L, Hh, N, dev, world, dist, total_bytes=None):
     """Same step, but every layer's K/V arrive from pinned host memory and every
     layer's reconstruction returns to pinned host memory inside the timed
     region; copies overlap the codec on separate streams."""
@@ -830,7 +860,8 @@ def e2e(args, qvg, cfg, X, Y, packed, ws, L, Hh, N, dev, world, dist):
     torch.cuda.synchronize()
     ms = max_over_ranks(dist, ev0.elapsed_time(ev1) / args.steps, dev)
     nbytes = U * N * 128 * 2
-    return {"value": weak_scaling_value(nbytes, world, ms), "unit": "GB/s", "ms_per_step": ms,
+    value = strong_scaling_value(total_bytes, ms) if total_bytes else weak_scaling_value(nbytes, world, ms)
+    return {"value": value, "unit": "GB/s", "ms_per_step": ms,
             "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
             "host_layers_distinct": nh, "api": "qvg_quantize + qvg_dequantize per layer (64 blocks)"}
 

@@ -50,3 +50,20 @@ def test_single_rank_needs_no_collective():
     import bench
     assert bench.max_over_ranks(None, 12.5, torch.device("cpu")) == 12.5
     assert bench.weak_scaling_value(2e9, 1, 1000.0) == pytest.approx(2.0)
+
+
+def test_head_shards_partition_every_cache():
+    """Strong scaling shares one cache by heads: the ranks' contiguous shares
+    cover every head exactly once and differ in size by at most one."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    for H in (1, 7, 12, 32):
+        for world in range(1, H + 1):
+            shares = [bench.shard_units(H, world, r) for r in range(world)]
+            assert shares[0][0] == 0 and shares[-1][1] == H
+            assert all(shares[r][1] == shares[r + 1][0] for r in range(world - 1))
+            sizes = [b - a for a, b in shares]
+            assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+    # whole-job rate: the one cache's bytes over the slowest rank's time
+    assert bench.strong_scaling_value(2e9, 1000.0) == 2.0
