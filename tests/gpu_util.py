@@ -1,5 +1,5 @@
 """Shared helpers of the GPU parity tests: move packed outputs between the
-CUDA path and the oracle, and judge agreement with the tolerances of the
+CUDA path and the oracle, and assess agreement with the tolerances of the
 codec's contract (bit-exact dequantisation; >= 99.9 % agreement of
 assignments and codes, disagreements only at near-ties; reconstruction MSE
 within 1 % and max error <= 1e-2 x group scale where codes agree)."""
@@ -45,7 +45,7 @@ def e4m3_values(b: np.ndarray) -> np.ndarray:
 
 
 def compare_quantize(ora, X_np, gpu: dict, ref: dict, K, T, G, iters, dtype, init=None):
-    """Judge GPU quantisation against the oracle's.  Returns a report dict."""
+    """Compare GPU quantisation with the oracle's.  Returns a report dict."""
     H, N, d = X_np.shape
     rep = {}
     exact = all(np.array_equal(gpu[k], ref[k]) for k in ("codes", "scale", "zero", "assign", "centroids"))
