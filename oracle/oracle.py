@@ -65,16 +65,17 @@ def lib():
         L.ref_kmeans.argtypes = [vp, i64, i32, i32, i32, i32, vp, vp, vp]
         L.ref_residual.argtypes = [vp, i64, i32, vp, vp, i32, vp]
         L.ref_group_quant.argtypes = [vp, i64, i32, i32, vp, vp, vp]
+        L.ref_group_quant_sym.argtypes = [vp, i64, i32, i32, vp, vp]
         L.ref_quantize.restype = i32
-        L.ref_quantize.argtypes = [i32, i32, i32, i32, i32, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]
+        L.ref_quantize.argtypes = [i32, i32, i32, i32, i32, i32, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]
         L.ref_dequantize.restype = i32
-        L.ref_dequantize.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, i32, i32, vp]
+        L.ref_dequantize.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, i32, i32, vp]
         L.ref_kv_cache_bytes.restype = f64
         L.ref_kv_cache_bytes.argtypes = [i64, i64, i64, i64]
         L.ref_bits_per_element.restype = f64
-        L.ref_bits_per_element.argtypes = [i32, i32, i32, i32, i64, i32, i32]
+        L.ref_bits_per_element.argtypes = [i32, i32, i32, i32, i64, i32, i32, i32]
         L.ref_packed_bytes.restype = i64
-        L.ref_packed_bytes.argtypes = [i32, i32, i32, i32, i64, i32, i32, i32]
+        L.ref_packed_bytes.argtypes = [i32, i32, i32, i32, i64, i32, i32, i32, i32]
         _lib = L
     return _lib
 
@@ -182,43 +183,55 @@ def group_quant(R, G):
     return codes, scale, zero
 
 
+def group_quant_sym(R, G):
+    """Symmetric mode: one E4M3 scale per group; returns (codes, scale)."""
+    R = _f32(R)
+    N, d = R.shape
+    codes = np.empty((N, d // 4), np.uint8)
+    scale = np.empty((N, d // G), np.uint8)
+    lib().ref_group_quant_sym(_p(R), N, d, G, _p(codes), _p(scale))
+    return codes, scale
+
+
 # ---------------------------------------------------------------- codec
 def _dt(X):
     return FP32 if X.dtype == np.float32 else BF16
 
 
-def quantize(X, K, T, G, iters, init=None):
+def quantize(X, K, T, G, iters, init=None, scale_mode=0):
     """X: [H][N][d] uint16 (bf16 bits) or float32.  Returns a dict of the
-    packed arrays in the codec's layouts."""
+    packed arrays in the codec's layouts (scale_mode 1: one E4M3 scale per
+    group; ``zero`` is then an empty array)."""
     X = np.ascontiguousarray(X)
     dtype = _dt(X)
     H, N, d = X.shape
     out = dict(
         codes=np.zeros((H, N, d // 4), np.uint8),
         scale=np.zeros((H, N, d // G), np.uint8),
-        zero=np.zeros((H, N, d // G), np.uint8),
+        zero=np.zeros((H, N, d // G) if scale_mode == 0 else (0,), np.uint8),
         assign=np.zeros((T, H, N), np.uint8),
         centroids=np.zeros((T, H, K, d), X.dtype),
     )
     if init is not None:
         init = np.ascontiguousarray(init, dtype=X.dtype)
         assert init.shape == (T, H, K, d)
-    rc = lib().ref_quantize(K, T, G, iters, dtype, _p(X), N, H, d,
+    rc = lib().ref_quantize(K, T, G, iters, dtype, scale_mode, _p(X), N, H, d,
                             _p(init) if init is not None else None,
-                            _p(out["codes"]), _p(out["scale"]), _p(out["zero"]),
+                            _p(out["codes"]), _p(out["scale"]), _p(out["zero"]) if scale_mode == 0 else None,
                             _p(out["assign"]), _p(out["centroids"]))
     if rc != 0:
         raise ValueError("oracle quantize rejected its arguments")
     return out
 
 
-def dequantize(packed, K, T, G, N, H, d, dtype=BF16) -> np.ndarray:
+def dequantize(packed, K, T, G, N, H, d, dtype=BF16, scale_mode=0) -> np.ndarray:
     Y = np.empty((H, N, d), np.float32 if dtype == FP32 else np.uint16)
     cen = np.ascontiguousarray(packed["centroids"])
-    rc = lib().ref_dequantize(K, T, G, dtype,
+    zero = np.ascontiguousarray(packed["zero"]) if scale_mode == 0 else None
+    rc = lib().ref_dequantize(K, T, G, dtype, scale_mode,
                               _p(np.ascontiguousarray(packed["codes"])),
                               _p(np.ascontiguousarray(packed["scale"])),
-                              _p(np.ascontiguousarray(packed["zero"])),
+                              _p(zero) if zero is not None else None,
                               _p(np.ascontiguousarray(packed["assign"])),
                               _p(cen), N, H, d, _p(Y))
     if rc != 0:
@@ -231,9 +244,9 @@ def kv_cache_bytes(L, tokens, hidden, nbytes) -> float:
     return float(lib().ref_kv_cache_bytes(L, tokens, hidden, nbytes))
 
 
-def bits_per_element(K, T, G, N, d, bits=2, dtype=BF16) -> float:
-    return float(lib().ref_bits_per_element(K, T, G, bits, N, d, dtype))
+def bits_per_element(K, T, G, N, d, bits=2, dtype=BF16, scale_mode=0) -> float:
+    return float(lib().ref_bits_per_element(K, T, G, bits, N, d, dtype, scale_mode))
 
 
-def packed_bytes(K, T, G, N, H, d, bits=2, dtype=BF16) -> int:
-    return int(lib().ref_packed_bytes(K, T, G, bits, N, H, d, dtype))
+def packed_bytes(K, T, G, N, H, d, bits=2, dtype=BF16, scale_mode=0) -> int:
+    return int(lib().ref_packed_bytes(K, T, G, bits, N, H, d, dtype, scale_mode))

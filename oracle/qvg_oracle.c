@@ -450,12 +450,55 @@ void ref_group_quant(const float* R, int64_t N, int d, int G,
     }
 }
 
+/* Symmetric variant: ONE FP8 E4M3 scale per group ([163] 五 names only
+ * "FP8 E4M3 group scales"; with one byte per group the closed form gives the
+ * 6.94-7.05x of [163] 六 at T = 1, G = 64, and the 6.40x of plain rounding at
+ * G = 16, see ref_bits_per_element).  READING: standard symmetric signed
+ * INT2, the scale being the group's largest magnitude over the largest
+ * positive code (2^(b-1) - 1 = 1):
+ *   s = E4M3(max |r|),  q = clamp(rint(r / s), -2, 1),  stored u = q + 2,
+ * with an IEEE fp32 divide, ties to even, and q = 0 when s = 0.  The value
+ * of u is s * (u - 2).  Codes are packed as in ref_group_quant. */
+void ref_group_quant_sym(const float* R, int64_t N, int d, int G,
+                         uint8_t* codes, uint8_t* scale)
+{
+    int64_t i;
+    int g, j, ng = d / G;
+    memset(codes, 0, (size_t)(N * (d / 4)));
+    for (i = 0; i < N; ++i) {
+        for (g = 0; g < ng; ++g) {
+            const float* r = R + i * d + (int64_t)g * G;
+            float amax = 0.0f, s;
+            uint8_t sc;
+            for (j = 0; j < G; ++j) {
+                float a = fabsf(r[j]);
+                if (a > amax) amax = a;
+            }
+            sc = ref_e4m3_encode(amax);
+            s = ref_e4m3_decode(sc);
+            scale[i * ng + g] = sc;
+            for (j = 0; j < G; ++j) {
+                int ch = g * G + j, q = 0;
+                if (s != 0.0f) {
+                    float t = r[j] / s;
+                    float rt = rintf(t);
+                    if (rt < -2.0f) rt = -2.0f;
+                    if (rt > 1.0f) rt = 1.0f;
+                    q = (int)rt;
+                }
+                codes[i * (d / 4) + ch / 4] |= (uint8_t)((q + 2) << (2 * (ch % 4)));
+            }
+        }
+    }
+}
+
 /* ------------------------------------------------------------------ */
 /* Whole codec.  Layouts (all row-major):                                */
 /*   X          [H][N][d]   in S (bf16 bits or fp32)                      */
 /*   init       [T][H][K][d] in S, or NULL for the cold start              */
 /*   codes      [H][N][d/4]                                               */
-/*   scale,zero [H][N][d/G] E4M3 bytes                                    */
+/*   scale,zero [H][N][d/G] E4M3 bytes (zero unused, may be NULL, in the */
+/*              symmetric mode: scale_mode = 1)                           */
 /*   assign     [T][H][N]   uint8                                         */
 /*   centroids  [T][H][K][d] in S                                         */
 /* Progressive residual quantisation ([163] 四; [de] 2B; [pt] 2B):       */
@@ -468,8 +511,8 @@ void ref_group_quant(const float* R, int64_t N, int d, int G,
 /* centroids (READING).                                                   */
 /* Returns 0 on success, -1 on invalid arguments.                          */
 /* ------------------------------------------------------------------ */
-int ref_quantize(int K, int T, int G, int iters, int dtype, const void* X,
-                 int64_t N, int H, int d, const void* init,
+int ref_quantize(int K, int T, int G, int iters, int dtype, int scale_mode,
+                 const void* X, int64_t N, int H, int d, const void* init,
                  uint8_t* codes, uint8_t* scale, uint8_t* zero,
                  uint8_t* assign, void* centroids)
 {
@@ -478,6 +521,7 @@ int ref_quantize(int K, int T, int G, int iters, int dtype, const void* X,
     float *R, *R2, *C;
     if (K < 1 || K > 256 || T < 0 || G < 4 || G % 4 || d % G || d % 4 || N < 1 || H < 1 || iters < 0)
         return -1;
+    if (scale_mode != 0 && scale_mode != 1) return -1;
     if (T > 0 && iters < 1) return -1;     /* assignments need one assign step */
     if (T > 0 && init == NULL && N < K) return -1;
     R = (float*)malloc((size_t)(N * d) * sizeof(float));
@@ -496,8 +540,12 @@ int ref_quantize(int K, int T, int G, int iters, int dtype, const void* X,
             ref_residual(R, N, d, C, pi, dtype, R2);
             tmp = R; R = R2; R2 = tmp;
         }
-        ref_group_quant(R, N, d, G, codes + (int64_t)h * N * (d / 4),
-                        scale + (int64_t)h * N * (d / G), zero + (int64_t)h * N * (d / G));
+        if (scale_mode == 1)
+            ref_group_quant_sym(R, N, d, G, codes + (int64_t)h * N * (d / 4),
+                                scale + (int64_t)h * N * (d / G));
+        else
+            ref_group_quant(R, N, d, G, codes + (int64_t)h * N * (d / 4),
+                            scale + (int64_t)h * N * (d / G), zero + (int64_t)h * N * (d / G));
     }
     free(R);
     free(R2);
@@ -506,11 +554,12 @@ int ref_quantize(int K, int T, int G, int iters, int dtype, const void* X,
 }
 
 /* Reconstruction in reverse order ([163] 四, 五; [de] 2B "Rekonstruktion"):
- * y = s*q + m, then the centroid of stage T, T-1, ..., 1 is added, each an
- * fp32 add, and the sum is rounded once to S.  s*q + m is exact in fp32:
- * s and m are E4M3 values (4 significant bits, bits between 2^-9 and 2^8)
- * and q <= 3, so the sum spans fewer than 24 bits. */
-int ref_dequantize(int K, int T, int G, int dtype, const uint8_t* codes,
+ * y = s*q + m (symmetric mode: y = s*(u - 2)), then the centroid of stage
+ * T, T-1, ..., 1 is added, each an fp32 add, and the sum is rounded once to
+ * S.  The first value is exact in fp32: s and m are E4M3 values (4
+ * significant bits, bits between 2^-9 and 2^8) and q <= 3, so it spans fewer
+ * than 24 bits. */
+int ref_dequantize(int K, int T, int G, int dtype, int scale_mode, const uint8_t* codes,
                    const uint8_t* scale, const uint8_t* zero,
                    const uint8_t* assign, const void* centroids,
                    int64_t N, int H, int d, void* Y)
@@ -520,6 +569,7 @@ int ref_dequantize(int K, int T, int G, int dtype, const uint8_t* codes,
     float* C;
     float* row;
     if (K < 1 || K > 256 || T < 0 || G < 4 || G % 4 || d % G || d % 4 || N < 0 || H < 1) return -1;
+    if (scale_mode != 0 && scale_mode != 1) return -1;
     ng = d / G;
     C = (float*)malloc((size_t)(T > 0 ? T : 1) * K * d * sizeof(float));
     row = (float*)malloc((size_t)d * sizeof(float));
@@ -532,8 +582,13 @@ int ref_dequantize(int K, int T, int G, int dtype, const uint8_t* codes,
             for (j = 0; j < d; ++j) {
                 int q = (codes[tok * (d / 4) + j / 4] >> (2 * (j % 4))) & 3;
                 float s = ref_e4m3_decode(scale[tok * ng + j / G]);
-                float m = ref_e4m3_decode(zero[tok * ng + j / G]);
-                float y = (float)((double)s * (double)q + (double)m);
+                float y;
+                if (scale_mode == 1) {
+                    y = (float)((double)s * (double)(q - 2));
+                } else {
+                    float m = ref_e4m3_decode(zero[tok * ng + j / G]);
+                    y = (float)((double)s * (double)q + (double)m);
+                }
                 for (t = T - 1; t >= 0; --t) {
                     int k = assign[((int64_t)t * H + h) * N + i];
                     y = y + C[((int64_t)t * K + k) * d + j];
@@ -561,22 +616,23 @@ double ref_kv_cache_bytes(int64_t L, int64_t tokens, int64_t hidden, int64_t byt
 }
 
 /* Bits per cached element of the codec: b code bits, two E4M3 bytes per
- * group of G, one uint8 assignment per token per stage (8T/d per element),
- * and T centroid tables of K x d values in S amortised over the N tokens
- * of a block. */
-double ref_bits_per_element(int K, int T, int G, int bits, int64_t N, int d, int dtype)
+ * group of G (one in the symmetric mode), one uint8 assignment per token per
+ * stage (8T/d per element), and T centroid tables of K x d values in S
+ * amortised over the N tokens of a block. */
+double ref_bits_per_element(int K, int T, int G, int bits, int64_t N, int d, int dtype, int scale_mode)
 {
     double sc = dtype == REF_FP32 ? 32.0 : 16.0;
-    return (double)bits + 16.0 / G + 8.0 * T / d + sc * T * K / (double)N;
+    double per_group = scale_mode == 1 ? 8.0 : 16.0;
+    return (double)bits + per_group / G + 8.0 * T / d + sc * T * K / (double)N;
 }
 
 /* Bytes of the packed stream for H blocks of N tokens, summed array by
  * array over the layouts above. */
-int64_t ref_packed_bytes(int K, int T, int G, int bits, int64_t N, int H, int d, int dtype)
+int64_t ref_packed_bytes(int K, int T, int G, int bits, int64_t N, int H, int d, int dtype, int scale_mode)
 {
     int64_t esz = dtype == REF_FP32 ? 4 : 2;
     int64_t codes = (int64_t)H * N * d * bits / 8;
-    int64_t scales = 2 * (int64_t)H * N * (d / G);
+    int64_t scales = (scale_mode == 1 ? 1 : 2) * (int64_t)H * N * (d / G);
     int64_t assign = (int64_t)T * H * N;
     int64_t cents = (int64_t)T * H * K * d * esz;
     return codes + scales + assign + cents;

@@ -67,3 +67,31 @@ def test_compression_and_codes_share_match_pages(ora):
     cr1 = 16 / ora.bits_per_element(256, 1, 64, 38000, 128)
     assert cr2 == pytest.approx(6.176, abs=2e-3) and cr1 == pytest.approx(6.611, abs=2e-3)
     assert cr1 < GOLD["compression_qvg"]["min"]
+
+
+def test_one_scale_per_group_reproduces_the_pages_ratios(ora):
+    """With ONE E4M3 byte per group (the symmetric mode) the closed form at
+    K = 256 and a 38,000-token block lands inside both of the pages' ranges:
+    the QVG point (T = 1, G = 64) in 6.94-7.05x, the QVG-Pro point (T = 4,
+    G = 16) in 4.97-5.20x, and plain rounding (T = 0, G = 16) gives exactly the
+    6.40x the pages quote for their round-to-nearest baseline (section 六).
+    The scale-and-zero layout reaches the QVG range only at G = 128."""
+    bpe = lambda T, G, m: ora.bits_per_element(256, T, G, 38000, 128, scale_mode=m)
+    qvg, pro, rtn = 16 / bpe(1, 64, 1), 16 / bpe(4, 16, 1), 16 / bpe(0, 16, 1)
+    assert GOLD["compression_qvg"]["min"] <= qvg <= GOLD["compression_qvg"]["max"]
+    assert GOLD["compression_qvg_pro"]["min"] <= pro <= GOLD["compression_qvg_pro"]["max"]
+    assert rtn == GOLD["compression_rtn_baseline"]["value"]
+    # written out: 2 + 8/64 + 8/128 + 16*256/38000 bits per element
+    assert bpe(1, 64, 1) == pytest.approx(2 + 0.125 + 0.0625 + 16 * 256 / 38000, rel=1e-12)
+    assert 16 / bpe(1, 64, 0) < GOLD["compression_qvg"]["min"]
+    assert GOLD["compression_qvg"]["min"] <= 16 / bpe(1, 128, 0) <= GOLD["compression_qvg"]["max"]
+    # the 2-bit codes hold more than 65 % of QVG memory
+    assert 2 / bpe(1, 64, 1) > GOLD["codes_share_of_memory_min"]["value"]
+
+
+def test_symmetric_packed_bytes_equal_the_arrays_quantize_writes(ora):
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((3, 40, 32)).astype(np.float32)
+    p = ora.quantize(X, K=8, T=2, G=16, iters=2, scale_mode=1)
+    assert p["zero"].size == 0
+    assert sum(a.nbytes for a in p.values()) == ora.packed_bytes(8, 2, 16, 40, 3, 32, dtype=1, scale_mode=1)

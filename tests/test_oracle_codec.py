@@ -183,3 +183,53 @@ def test_invalid_arguments_rejected(ora):
         args.update(kw)
         with pytest.raises(ValueError):
             ora.quantize(X, **args)
+
+
+def _e4m3_byte(x):
+    import torch
+    return int(torch.tensor([x], dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)[0])
+
+
+def test_symmetric_group_worked_examples(ora):
+    """One E4M3 scale per group: s = E4M3(max |r|), q = clamp(rint(r/s), -2, 1),
+    stored u = q + 2 at bits 2*(j mod 4).  Hand-worked groups of four:
+      [0.3, -0.9, 1.2, 0.05]: s = E4M3(1.2) = 1.25 (0x3A); r/s = 0.24, -0.72,
+        0.96, 0.04 -> q = 0, -1, 1, 0 -> u = 2, 1, 3, 2 -> byte 0xB6;
+      [-1, 0.5, -0.5, 1]: s = 1; r/s = -1, 0.5, -0.5, 1 -> ties to even give
+        q = -1, 0, 0, 1 -> u = 1, 2, 2, 3 -> byte 0xE9;
+      zeros: s = 0, every u = 2 -> byte 0xAA;
+      [1000, -3, 0, 2]: s saturates at 448 (0x7E); 1000/448 -> 2 -> clamp 1."""
+    R = np.array([[0.3, -0.9, 1.2, 0.05], [-1.0, 0.5, -0.5, 1.0], [0, 0, 0, 0], [1000, -3, 0, 2]], np.float32)
+    codes, scale = ora.group_quant_sym(R, 4)
+    assert scale[:, 0].tolist() == [0x3A, _e4m3_byte(1.0), 0x00, 0x7E]
+    assert scale[0, 0] == _e4m3_byte(1.25)
+    assert codes[:, 0].tolist() == [0xB6, 0xE9, 0xAA, 3 | (2 << 2) | (2 << 4) | (2 << 6)]
+
+
+def test_symmetric_error_bound_and_round_trip(ora):
+    """|r - s (u - 2)| <= s/2 for every value (|r| <= 1.0625 s after E4M3
+    rounding of the group maximum, inside the [-1.5 s, 1.5 s] the levels
+    cover), and the oracle's dequantisation of a T = 0 stream is s (u - 2)."""
+    rng = np.random.default_rng(7)
+    X = (rng.standard_normal((1, 300, 128)) * np.exp(rng.standard_normal((1, 300, 1)))).astype(np.float32)
+    p = ora.quantize(X, K=1, T=0, G=32, iters=0, scale_mode=1)
+    Y = ora.dequantize(p, K=1, T=0, G=32, N=300, H=1, d=128, dtype=1, scale_mode=1)
+    s = np.repeat(ora.e4m3_decode(p["scale"][0]), 32, axis=-1).astype(np.float64)
+    j = np.arange(128)
+    u = (p["codes"][0][:, j // 4] >> (2 * (j % 4))) & 3
+    np.testing.assert_array_equal(Y[0], (s * (u - 2)).astype(np.float32))
+    assert np.all(np.abs(X[0] - Y[0]) <= s / 2 * (1 + 2 ** -22))
+    assert (u != 0).all()                      # q = -2 needs r/s < -1.5: never reached
+
+
+def test_symmetric_dequant_hand_tables(ora):
+    """T = 1, K = 2, G = 4, d = 4: y = s (u - 2) + C[pi], one fp32 add."""
+    packed = dict(codes=np.array([[[0xB6]], [[0xAA]]], np.uint8).reshape(1, 2, 1),
+                  scale=np.array([[[0x3A], [0x38]]], np.uint8),
+                  zero=np.zeros((0,), np.uint8),
+                  assign=np.array([[[1, 0]]], np.uint8),
+                  centroids=np.array([[[[1, 2, 3, 4], [10, 20, 30, 40]]]], np.float32))
+    Y = ora.dequantize(packed, K=2, T=1, G=4, N=2, H=1, d=4, dtype=1, scale_mode=1)
+    # token 0: u = 2, 1, 3, 2 with s = 1.25, plus centroid 1; token 1: zeros plus centroid 0
+    np.testing.assert_array_equal(Y[0, 0], np.array([10, 20 - 1.25, 30 + 1.25, 40], np.float32))
+    np.testing.assert_array_equal(Y[0, 1], np.array([1, 2, 3, 4], np.float32))
