@@ -153,11 +153,10 @@ def weak_scaling_value(bytes_per_rank: float, world: int, ms: float) -> float:
 
 
 def shard_units(n: int, world: int, rank: int):
-    """Contiguous share [first, last) of n units (heads) for `rank` of
-    `world`; the shares partition [0, n) and differ in size by at most one."""
-    base, extra = divmod(n, world)
-    first = rank * base + min(rank, extra)
-    return first, first + base + (1 if rank < extra else 0)
+    """Contiguous share [first, last) of n heads for `rank` of `world` (the
+    package's head sharding; the shares partition [0, n))."""
+    from bit_kv_cache_qvg_b200.shard import shard_units as _shard
+    return _shard(n, world, rank)
 
 
 def strong_scaling_value(total_bytes: float, ms: float) -> float:
@@ -629,7 +628,8 @@ def run_stream(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
 
     # warm-up: W chunks through a throwaway cache (kernel load, workspace sizing)
     gen = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=kinds, seed=seed + 1, device=dev)
-    wcache = qvg.Cache(cfg, U, sum(sizes[:max(args.warmup, 1)]), max(args.warmup, 1))
+    wcache = qvg.Cache(cfg, U, sum(sizes[:max(args.warmup, 1)]), max(args.warmup, 1),
+                       max_chunk_tokens=max(sizes))
     with torch.cuda.stream(stream):
         for c in range(max(args.warmup, 1)):
             wcache.append(gen.next(sizes[c] // (wl["gh"] * wl["gw"])), stream=stream)
@@ -638,7 +638,7 @@ def run_stream(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
     wcache.close()
 
     # pass 1: the streaming cache
-    cache = qvg.Cache(cfg, U, total, nch)
+    cache = qvg.Cache(cfg, U, total, nch, max_chunk_tokens=max(sizes))
     gen = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=kinds, seed=seed, device=dev)
     ea, eb, da, db = events(nch), events(nch), events(nch), events(nch)
     kept = {}
@@ -735,7 +735,7 @@ def run_stream(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
     torch.cuda.synchronize()
     qvg.profile_enable(False)
     per_dequant = qvg.profile_launches()
-    scache = qvg.Cache(cfg, U, 2 * sizes[0], 2)
+    scache = qvg.Cache(cfg, U, 2 * sizes[0], 2, max_chunk_tokens=sizes[0])
     g2 = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=kinds, seed=seed + 2, device=dev)
     with torch.cuda.stream(stream):
         scache.append(g2.next(wl["chunk_frames"]), stream=stream)
@@ -772,7 +772,7 @@ def stream_e2e(args, wl, qvg, synth, cfg, sizes, dev, stream, chunks=40):
     U = 2 * Hh
     n = sizes[0]
     chunks = min(chunks, len([s for s in sizes if s == n]))
-    cache = qvg.Cache(cfg, U, chunks * n, chunks)
+    cache = qvg.Cache(cfg, U, chunks * n, chunks, max_chunk_tokens=n)
     gen = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=[0] * Hh + [1] * Hh, seed=12345, device=dev)
     Xh = torch.empty((U, n, 128), dtype=torch.bfloat16, pin_memory=True)
     Xd = torch.empty((U, n, 128), dtype=torch.bfloat16, device=dev)

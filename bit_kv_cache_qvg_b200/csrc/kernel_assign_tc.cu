@@ -5,12 +5,13 @@
 // For a tile of 128 tokens R (bf16) and the block's K <= 256 centroids C
 // (bf16), tcgen05.mma (kind::f16, M=128, N=Kpad, fp32 accumulate) computes the
 // 128 x Kpad dot products r_i . c_k into tensor memory.  The epilogue warps
-// read them back with tcgen05.ld and form the screening values
-// g_ik = |c_k|^2 - 2 r_i . c_k (argmin_k g_ik = argmin_k |r_i - c_k|^2),
-// keeping the smallest two per token.  If the runner-up lies within the
-// rounding-error bound of the minimum, the token is appended to a per-block
-// list that an exact fp64 pass (qvg_assign_exact in list mode) decides;
-// otherwise the minimum's index is the assignment.
+// read them back with tcgen05.ld as h_ik = r_i . c_k - |c_k|^2/2 (a ninth MMA
+// K-step adds the bias; argmax_k h_ik = argmin_k |r_i - c_k|^2) and keep, per
+// token, the maxima of the 32 eight-column groups and of the 8 position
+// classes within a group.  If a second group or a second position class comes
+// within the rounding-error bound of the maximum, the token is appended to a
+// per-block list that an exact fp64 pass (qvg_assign_candidates) decides;
+// otherwise the maximum's column is the assignment.
 //
 // Data movement: the centroid table is loaded once per CTA with TMA (128-byte
 // swizzle, K-major), token tiles stream through a 3-stage TMA ring; no
@@ -21,7 +22,6 @@
 // mbarrier wait is bounded; on timeout the kernel records an error in the
 // status word, drains, frees TMEM and returns.
 #include <cuda.h>
-#include <cstdio>
 
 #include "qvg_common.cuh"
 #include "qvg_launch.h"
@@ -34,11 +34,7 @@ constexpr int kStages = 3;
 constexpr int kTileM = 128;
 constexpr int kAStageBytes = kTileM * kD * 2;     // 32 KB: two 16 KB K-halves
 constexpr int kAHalfBytes = kTileM * 128;         // 128 rows x 128 B
-#ifdef QVG_TC_DEBUG
-constexpr uint64_t kWaitLimitNs = 50000000ull;     // 50 ms in the self-checking build
-#else
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s of wall time per wait
-#endif
 constexpr uint32_t kStatusTimeout = 1u;
 
 struct __align__(8) TcSmemBarriers {
@@ -76,8 +72,8 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Bounded wait for the phase of `parity` to complete: gives up after
-// kWaitLimitNs of wall time and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// `limit_ns` of wall time and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   const uint32_t addr = smem_u32(bar);
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
@@ -93,7 +89,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if ((it & 63u) == 0u) {
       const uint64_t now = globaltimer_ns();
       if (t0 == 0) t0 = now;
-      else if (now - t0 > kWaitLimitNs) return false;
+      else if (now - t0 > limit_ns) return false;
     }
   }
 }
@@ -206,20 +202,14 @@ struct TcParams {
   int tiles_per_unit;
   int tiles_per_cta;
   float gamma;              // relative error bound of the tensor-core dot products
-  uint32_t unit;            // always 1: the multiplier that puts the column add on the FMA pipe
+  // Test hook of the bounded waits (fault injection on the host side): the
+  // CTA of block 0, tile range 0 waits at most `hook_wait_ns` and, when
+  // `hook_withhold` >= 0, its producer stops before issuing that tile, so
+  // that the waits on it run out.  Off: hook_withhold = -1, hook_wait_ns = 0.
+  int hook_withhold;
+  uint64_t hook_wait_ns;
 };
 
-#ifdef QVG_TC_DEBUG
-// Self-checking build: where each role gave up, and how far each got.
-//   [0..3]  producer: empty-wait gave up at tile+1, b_full drain
-//   [4..7]  mma: b_full, tmem_empty, full wait gave up at tile+1
-//   [8..11] epilogue: tmem_full wait gave up at tile+1
-//   [16] tiles produced, [17] tiles issued to MMA, [18] tiles consumed
-__device__ uint32_t g_tc_dbg[32];
-#define TC_DBG(i, v) do { if (blockIdx.x == 0 && blockIdx.y == 0) atomicMax(&g_tc_dbg[i], (uint32_t)(v)); } while (0)
-#else
-#define TC_DBG(i, v) do { } while (0)
-#endif
 
 __device__ __forceinline__ int aborted(const TcSmemBarriers* b) {
   return *reinterpret_cast<const volatile int*>(&b->abort_flag);
@@ -303,6 +293,11 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
+  // The test hook applies to the CTA of block 0 that starts at tile 0 only.
+  const bool hooked = p.hook_wait_ns != 0 && u == 0 && blockIdx.x == 0;
+  const uint64_t wait_ns = hooked ? p.hook_wait_ns : kWaitLimitNs;
+  const int withhold = hooked ? p.hook_withhold : -1;
+
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0) {
@@ -310,22 +305,23 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
       tma_load_3d(sB, &tmC, 0, 0, u, &bars->b_full);
       tma_load_3d(sB + Npad * 128, &tmC, 64, 0, u, &bars->b_full);
       int issued = 0;
+      bool stopped = false;
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % kStages;
         const uint32_t ph = (uint32_t)(i / kStages) & 1u;
-        if (!mbar_wait(&bars->empty[s], ph ^ 1u) || aborted(bars)) { TC_DBG(0, i + 1); set_abort(bars); break; }
+        if (!mbar_wait(&bars->empty[s], ph ^ 1u, wait_ns) || aborted(bars)) { set_abort(bars); stopped = true; break; }
+        if (i == withhold) { stopped = true; break; }   // test hook: this tile is never loaded
         uint8_t* a = sA + s * kAStageBytes;
         const int row = (t_begin + i) * kTileM;
         mbar_expect_tx(&bars->full[s], (uint32_t)kAStageBytes);
         tma_load_3d(a, &tmR, 0, row, u, &bars->full[s]);
         tma_load_3d(a + kAHalfBytes, &tmR, 64, row, u, &bars->full[s]);
         ++issued;
-        TC_DBG(16, issued);
       }
-      if (aborted(bars)) {        // drain: wait (bounded) for the loads in flight
+      if (stopped) {              // drain: wait (bounded) for the loads in flight
         for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-          mbar_wait(&bars->full[i % kStages], (uint32_t)(i / kStages) & 1u);
-        mbar_wait(&bars->b_full, 0);
+          mbar_wait(&bars->full[i % kStages], (uint32_t)(i / kStages) & 1u, wait_ns);
+        mbar_wait(&bars->b_full, 0, wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -334,17 +330,16 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
       const uint32_t idesc = umma_idesc_bf16(kTileM, Npad);
       const uint32_t b_addr = smem_u32(sB);
       const uint32_t ax_addr = smem_u32(sAx), bx_addr = smem_u32(sBx);
-      bool ok = mbar_wait(&bars->b_full, 0);
-      if (!ok) TC_DBG(4, 1);
+      bool ok = mbar_wait(&bars->b_full, 0, wait_ns);
       int issued = 0;
       for (int i = 0; ok && i < ntiles; ++i) {
         const int s = i % kStages;
         const uint32_t ph = (uint32_t)(i / kStages) & 1u;
         const int acc = i & 1;
         const uint32_t aph = (uint32_t)(i >> 1) & 1u;
-        if (!mbar_wait(&bars->tmem_empty[acc], aph ^ 1u)) { TC_DBG(5, i + 1); ok = false; break; }
-        if (!mbar_wait(&bars->full[s], ph)) { TC_DBG(6, i + 1); ok = false; break; }
-        if (aborted(bars)) { TC_DBG(7, i + 1); ok = false; break; }
+        if (!mbar_wait(&bars->tmem_empty[acc], aph ^ 1u, wait_ns)) { ok = false; break; }
+        if (!mbar_wait(&bars->full[s], ph, wait_ns)) { ok = false; break; }
+        if (aborted(bars)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_u32(sA + s * kAStageBytes);
         const uint32_t d_tmem = tmem + (uint32_t)(acc * 256);
@@ -359,11 +354,11 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
         umma_commit(&bars->empty[s]);
         umma_commit(&bars->tmem_full[acc]);
         ++issued;
-        TC_DBG(17, issued);
       }
       if (!ok) {
         set_abort(bars);
-        if (issued > 0) mbar_wait(&bars->tmem_full[(issued - 1) & 1], (uint32_t)((issued - 1) >> 1) & 1u);
+        // the last MMAs issued must finish before the CTA frees tensor memory
+        if (issued > 0) mbar_wait(&bars->tmem_full[(issued - 1) & 1], (uint32_t)((issued - 1) >> 1) & 1u, wait_ns);
       }
     }
   } else {
@@ -389,68 +384,42 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
         const int64_t tok = (int64_t)(t_begin + i + 2) * kTileM + row;
         if (i + 2 < ntiles && tok < p.N) rn2_next = p.rnorm2[(int64_t)u * p.N + tok];
       }
-      const bool ok = !aborted(bars) && mbar_wait(&bars->tmem_full[acc], aph);
-      if (!ok) { TC_DBG(8, i + 1); set_abort(bars); }
-      else if (lane == 0 && warp == 2) TC_DBG(18, i + 1);
+      const bool ok = !aborted(bars) && mbar_wait(&bars->tmem_full[acc], aph, wait_ns);
+      if (!ok) set_abort(bars);
       tc_fence_after();
-      // Top two of h_k = r.c_k - |c_k|^2/2 (the largest h is the nearest
-      // centroid), each value carrying its column index in its 8 low bits.
-      // Columns are taken in quads (top two of the quad by a small network),
-      // two quads make an 8-column group (its maximum is kept: it tells the
-      // exact pass which groups can hold a near-tie candidate), and groups
-      // are merged into four independent chains.  The next 32-column chunk's
-      // tensor-memory load is in flight while the current one is processed.
-      // The epilogue is bound by the integer/logic pipe, so each key is one
-      // lop3 and the column add runs as an integer multiply-add on the FMA pipe.
+      // h_k = r.c_k - |c_k|^2/2; the largest h is the nearest centroid.  Column
+      // k = 8g + j lies in group g (8 consecutive columns) and position class
+      // j.  The maxima of the 32 groups and of the 8 position classes are
+      // kept; they are exact maxima of the accumulator values, formed with
+      // three-input max instructions (about one per value).  A column other
+      // than the winner w lies outside w's group or outside w's position
+      // class, so the larger of the best other group and the best other
+      // position class is exactly the runner-up value.  The next 32-column
+      // chunk's tensor-memory load is in flight while the current one is
+      // processed.
       const float kNegBig = -3.0e38f;
-      float c1[4] = {kNegBig, kNegBig, kNegBig, kNegBig}, c2[4] = {kNegBig, kNegBig, kNegBig, kNegBig};
-      float gmax[32];
+      float gmax[32], pmax[8];
 #pragma unroll
       for (int g = 0; g < 32; ++g) gmax[g] = kNegBig;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) pmax[j] = kNegBig;
       if (ok) {
         const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
         uint32_t ra[32], rb[32];
         tmem_ld32_async(tbase, ra);
         tmem_wait_ld(ra);
-        // The position within the quad (0-3, held in registers) replaces the
-        // 8 low bits of every value; the quad's column (a multiple of 4) is
-        // added to the quad's maximum only -- the runner-up needs no index.
-        uint32_t pos1, pos2, pos3;
-        asm("mov.b32 %0, 1;" : "=r"(pos1));
-        asm("mov.b32 %0, 2;" : "=r"(pos2));
-        asm("mov.b32 %0, 3;" : "=r"(pos3));
-        const uint32_t unit = p.unit;
-        auto key = [](uint32_t v, uint32_t pos) {
-          uint32_t k;
-          asm("lop3.b32 %0, %1, 0xFFFFFF00, %2, 0xEA;" : "=r"(k) : "r"(v), "r"(pos));  // (v & ~0xFF) | pos
-          return __uint_as_float(k);
-        };
-        auto quad = [&](const uint32_t (&r)[32], int e, int col, float& qt, float& qs) {
-          uint32_t ka_u;
-          asm("and.b32 %0, %1, 0xFFFFFF00;" : "=r"(ka_u) : "r"(r[e]));
-          const float ka = __uint_as_float(ka_u);
-          const float kb2 = key(r[e + 1], pos1), kc = key(r[e + 2], pos2), kd = key(r[e + 3], pos3);
-          const float h1 = fmaxf(ka, kb2), l1 = fminf(ka, kb2);
-          const float h2 = fmaxf(kc, kd), l2 = fminf(kc, kd);
-          // bits 2-7 of the key are zero here, so adding the quad's column is an or
-          uint32_t qt_u;
-          asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(qt_u) : "r"(unit), "r"((uint32_t)col),
-              "r"(__float_as_uint(fmaxf(h1, h2))));
-          qt = __uint_as_float(qt_u);
-          qs = max3f(fminf(h1, h2), l1, l2);
-        };
         auto chunk = [&](const uint32_t (&r)[32], int ci) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
-            float ta, sa, tb, sb;
-            quad(r, e, ci * 32 + e, ta, sa);
-            quad(r, e + 4, ci * 32 + e + 4, tb, sb);
-            const float gt = fmaxf(ta, tb);
-            const float gs = max3f(fminf(ta, tb), sa, sb);
-            const int ch = e >> 3;
-            gmax[ci * 4 + ch] = gt;
-            c2[ch] = max3f(fminf(c1[ch], gt), c2[ch], gs);
-            c1[ch] = fmaxf(c1[ch], gt);
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r[e + j]);
+            gmax[ci * 4 + (e >> 3)] = max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            pmax[j] = max3f(pmax[j], __uint_as_float(r[j]), __uint_as_float(r[8 + j]));
+            pmax[j] = max3f(pmax[j], __uint_as_float(r[16 + j]), __uint_as_float(r[24 + j]));
           }
         };
 #pragma unroll
@@ -470,35 +439,36 @@ qvg_kmeans_assign(const __grid_constant__ CUtensorMap tmR, const __grid_constant
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->tmem_empty[acc]);
-      float w1 = fmaxf(c1[0], c1[1]), w2 = max3f(fminf(c1[0], c1[1]), c2[0], c2[1]);
-      const float u1 = fmaxf(c1[2], c1[3]), u2 = max3f(fminf(c1[2], c1[3]), c2[2], c2[3]);
-      w2 = max3f(fminf(w1, u1), w2, u2);
-      w1 = fmaxf(w1, u1);
       const int64_t tok = (int64_t)(t_begin + i) * kTileM + row;
       const bool valid = ok && tok < p.N && !aborted(bars);
       const int64_t gi = (int64_t)u * p.N + tok;
       bool flag = false;
       uint32_t groups = 0;
       if (valid) {
-        // Error bound of h (fp32 tensor-core sums of 128 exact products and the
-        // three pieces of -|c|^2/2): gamma * (|r| |c| + |c|^2 / 2) for every
-        // centroid at least as near as the nearest, |c| <= |r| + sqrt(D_min);
-        // plus the 2^-15 relative perturbation of the index bits of both keys.
+        const float M = max3f(max3f(pmax[0], pmax[1], pmax[2]), max3f(pmax[3], pmax[4], pmax[5]),
+                              fmaxf(pmax[6], pmax[7]));
+        // Error bound E of every h that can compete (fp32 tensor-core sums of
+        // 128 exact products and the three pieces of -|c|^2/2):
+        // gamma * (|r| |c| + |c|^2 / 2), where |c| <= |r| + sqrt(D_min) for
+        // every centroid at least as near as the nearest.  A column whose h is
+        // below thr = M - 2E cannot be the exact maximum; the extra
+        // 2^-23 |M| covers the rounding of thr itself.
         const float nr = sqrtf(fmaxf(rn2, 0.0f)) * 1.0001f;
-        const float cb = 1.02f * nr + sqrtf(fmaxf(rn2 - 2.0f * w1, 0.0f));
+        const float cb = 1.02f * nr + sqrtf(fmaxf(rn2 - 2.0f * M, 0.0f));
         const float E = p.gamma * (nr * cb + 0.5f * cb * cb) + 6.0e-8f * cb * cb + 1e-30f;
-        const float margin = 2.0f * E + 3.1e-5f * (fabsf(w1) + fabsf(w2));
-        flag = !(w1 - w2 > margin);
-        if (!flag) {
-          p.pi[gi] = (uint8_t)(__float_as_int(w1) & 0xFF);
-        } else {
-          // groups whose largest key reaches the threshold (with the index-bit
-          // perturbation of that key allowed for) hold every candidate
-          const float thr = w1 - margin;
-          const float thr_key = thr - 6.2e-5f * (fabsf(w1) + fabsf(thr));
+        const float thr = M - (2.0f * E + 1.2e-7f * fabsf(M));
+        uint32_t mp = 0;
 #pragma unroll
-          for (int g = 0; g < 32; ++g)
-            if (gmax[g] >= thr_key) groups |= 1u << g;
+        for (int j = 0; j < 8; ++j) mp |= pmax[j] >= thr ? (1u << j) : 0u;
+#pragma unroll
+        for (int g = 0; g < 32; ++g) groups |= gmax[g] >= thr ? (1u << g) : 0u;
+        // one group and one position class reach thr: the winner is certain
+        // (both masks hold M's column unless M is not a number)
+        const bool unique = mp != 0u && groups != 0u && (mp & (mp - 1u)) == 0u && (groups & (groups - 1u)) == 0u;
+        if (unique) {
+          p.pi[gi] = (uint8_t)(8 * (__ffs(groups) - 1) + (__ffs(mp) - 1));
+        } else {
+          flag = true;   // the groups that reach thr hold every candidate
         }
       }
       // every lane of the warp takes part in the list append
@@ -579,34 +549,18 @@ cudaError_t launch_assign_tc(const AssignTcParams& a, cudaStream_t s) {
   if (p.tiles_per_cta < 2) p.tiles_per_cta = 2;
   splits = (p.tiles_per_unit + p.tiles_per_cta - 1) / p.tiles_per_cta;
   p.gamma = a.gamma;
-  p.unit = 1;
+  p.hook_withhold = a.hook_withhold;
+  p.hook_wait_ns = a.hook_wait_ns;
   const size_t smem = assign_tc_smem_bytes(a.K);
   const bool full = Npad == 256;
   const void* fn = full ? reinterpret_cast<const void*>(qvg_kmeans_assign<8>)
                         : reinterpret_cast<const void*>(qvg_kmeans_assign<0>);
   cudaError_t e = ensure_dynamic_smem(fn, smem);
   if (e != cudaSuccess) return e;
-#ifdef QVG_TC_DEBUG
-  {
-    uint32_t z[32] = {};
-    cudaMemcpyToSymbol(g_tc_dbg, z, sizeof(z));
-  }
-#endif
   if (full)
     qvg_kmeans_assign<8><<<dim3((unsigned)splits, (unsigned)a.W), kTcThreads, smem, s>>>(mR, mC, p);
   else
     qvg_kmeans_assign<0><<<dim3((unsigned)splits, (unsigned)a.W), kTcThreads, smem, s>>>(mR, mC, p);
-#ifdef QVG_TC_DEBUG
-  {
-    cudaError_t le = cudaDeviceSynchronize();
-    uint32_t h[32] = {};
-    cudaMemcpyFromSymbol(h, g_tc_dbg, sizeof(h));
-    fprintf(stderr, "[tc-debug] grid=(%d,%d) tiles/cta=%d Npad=%d smem=%zu err=%s dbg:", splits, a.W,
-            p.tiles_per_cta, Npad, smem, cudaGetErrorString(le));
-    for (int i = 0; i < 20; ++i) fprintf(stderr, " %u", h[i]);
-    fprintf(stderr, "\n");
-  }
-#endif
   return cudaGetLastError();
 }
 

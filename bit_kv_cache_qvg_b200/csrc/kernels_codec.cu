@@ -134,7 +134,7 @@ template <> struct Oct<kFP32> {
 
 // TT = number of stages when it is <= 4 (assignments fetched a step ahead
 // with the codes), or -1 for the generic runtime-T loop.
-template <int DT, int TT>
+template <int DT, int TT, bool SYM>
 __global__ void __launch_bounds__(kDqThreads, 1)
 qvg_dequant_fused(const DequantParams p, const int splits) {
   constexpr int ESZ = Store<DT>::bytes;
@@ -195,8 +195,11 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
     for (int u = 0; u < kDqU; ++u) {
       const int t = t0 + u < nt ? t0 + u : 0;
       cb[u] = (uint32_t)cbp[t * (kD / 8)] | ((uint32_t)cbp[t * (kD / 8) + 8] << 16);
-      sz[u] = (uint32_t)scp[t * ng + g0] | ((uint32_t)zrp[t * ng + g0] << 8) |
-              ((uint32_t)scp[t * ng + g1] << 16) | ((uint32_t)zrp[t * ng + g1] << 24);
+      if (SYM)
+        sz[u] = (uint32_t)scp[t * ng + g0] | ((uint32_t)scp[t * ng + g1] << 16);
+      else
+        sz[u] = (uint32_t)scp[t * ng + g0] | ((uint32_t)zrp[t * ng + g0] << 8) |
+                ((uint32_t)scp[t * ng + g1] << 16) | ((uint32_t)zrp[t * ng + g1] << 24);
       uint32_t kw = 0;
       if (TT > 0) {
 #pragma unroll
@@ -209,11 +212,13 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
 #pragma unroll
     for (int u = 0; u < kDqU; ++u) {
       const int t = tb + u;
-      // y = s*q + m (exact in fp32: E4M3 operands, q <= 3), two channels per op
+      // y = s*q + m (exact in fp32: E4M3 operands, q <= 3), two channels per
+      // op; the symmetric mode is the same with m = -2s (y = s*(u - 2))
       float2 y0[4], y1[4];
       {
-        const float s0 = dec[sz[u] & 0xFFu], m0 = dec[(sz[u] >> 8) & 0xFFu];
-        const float s1 = dec[(sz[u] >> 16) & 0xFFu], m1 = dec[sz[u] >> 24];
+        const float s0 = dec[sz[u] & 0xFFu], s1 = dec[(sz[u] >> 16) & 0xFFu];
+        const float m0 = SYM ? -2.0f * s0 : dec[(sz[u] >> 8) & 0xFFu];
+        const float m1 = SYM ? -2.0f * s1 : dec[sz[u] >> 24];
         const float2 sp0 = f2(s0, s0), mp0 = f2(m0, m0), sp1 = f2(s1, s1), mp1 = f2(m1, m1);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -263,26 +268,26 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
   }
 }
 
-template <int DT>
+template <int DT, bool SYM>
 static cudaError_t launch_dq_t(const DequantParams& p, int blocks, int splits, size_t smem, cudaStream_t s) {
   const void* fn;
   switch (p.T) {
-    case 0: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 0>); break;
-    case 1: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 1>); break;
-    case 2: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 2>); break;
-    case 3: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 3>); break;
-    case 4: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 4>); break;
-    default: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, -1>); break;
+    case 0: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 0, SYM>); break;
+    case 1: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 1, SYM>); break;
+    case 2: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 2, SYM>); break;
+    case 3: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 3, SYM>); break;
+    case 4: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, 4, SYM>); break;
+    default: fn = reinterpret_cast<const void*>(qvg_dequant_fused<DT, -1, SYM>); break;
   }
   cudaError_t e = ensure_dynamic_smem(fn, smem);
   if (e != cudaSuccess) return e;
   switch (p.T) {
-    case 0: qvg_dequant_fused<DT, 0><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
-    case 1: qvg_dequant_fused<DT, 1><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
-    case 2: qvg_dequant_fused<DT, 2><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
-    case 3: qvg_dequant_fused<DT, 3><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
-    case 4: qvg_dequant_fused<DT, 4><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
-    default: qvg_dequant_fused<DT, -1><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+    case 0: qvg_dequant_fused<DT, 0, SYM><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+    case 1: qvg_dequant_fused<DT, 1, SYM><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+    case 2: qvg_dequant_fused<DT, 2, SYM><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+    case 3: qvg_dequant_fused<DT, 3, SYM><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+    case 4: qvg_dequant_fused<DT, 4, SYM><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
+    default: qvg_dequant_fused<DT, -1, SYM><<<blocks, kDqThreads, smem, s>>>(p, splits); break;
   }
   return cudaGetLastError();
 }
@@ -371,10 +376,40 @@ __device__ __forceinline__ uint32_t quant_chunk(const float (&r)[8], float lo, f
   return __float_as_uint(__fadd_rn(pk, 8388608.0f)) & 0xFFFFu;   // 2^23: integer in the low bits
 }
 
+// The symmetric mode (one E4M3 byte per group): s = E4M3(max |r|),
+// q = clamp(rint(fl(r / s)), -2, 1), stored u = q + 2, packed as in
+// quant_chunk.  The quotient is the IEEE one by the same Markstein
+// correction (the divisor is again an E4M3 value); rounding to nearest even
+// is the add and subtract of 1.5 * 2^23 (exact for |q| <= 2), and u = q + 2
+// is added after rounding.  s = 0 makes every quotient +-0, hence u = 2.
+__device__ __forceinline__ uint32_t quant_chunk_sym(const float (&r)[8], float lo, float hi, const E4m3Tables& tab,
+                                                    uint8_t& sc_out) {
+  constexpr float kRound = 12582912.0f;     // 1.5 * 2^23
+  const float amax = fmaxf(fabsf(lo), fabsf(hi));
+  const uint8_t scb = f32_to_e4m3(amax);
+  const float s = tab.dec[scb];
+  sc_out = scb;
+  const float y = tab.rcp[scb];
+  const float2 y2 = f2(y, y), ns2 = f2(-s, -s), k2 = f2(kRound, kRound), nk2 = f2(-kRound, -kRound);
+  const float2 two2 = f2(2.0f, 2.0f);
+  float2 pk2 = f2(0.0f, 0.0f);
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    const float2 d2 = f2(r[e], r[e + 1]);
+    const float2 q02 = __fmul2_rn(d2, y2);
+    const float2 t2 = __ffma2_rn(__ffma2_rn(ns2, q02, d2), y2, q02);
+    const float2 tc = f2(fminf(fmaxf(t2.x, -2.0f), 1.0f), fminf(fmaxf(t2.y, -2.0f), 1.0f));
+    const float2 u2 = __fadd2_rn(__fadd2_rn(__fadd2_rn(tc, k2), nk2), two2);
+    pk2 = __ffma2_rn(u2, f2((float)(1 << (2 * e)), (float)(1 << (2 * e + 2))), pk2);
+  }
+  const float pk = __fadd_rn(pk2.x, pk2.y);
+  return __float_as_uint(__fadd_rn(pk, 8388608.0f)) & 0xFFFFu;   // 2^23: integer in the low bits
+}
+
 // GT > 0 fixes the group size at compile time (the quantising pass is
 // instantiated for every supported G, so its group reductions and stores fold
 // to straight-line code); GT = 0 reads it from the parameters.
-template <int DT, bool QUANT, bool HAS_C, int GT>
+template <int DT, bool QUANT, bool HAS_C, int GT, bool SYM>
 __global__ void __launch_bounds__(kRqThreads)
 qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
   constexpr int ESZ = Store<DT>::bytes;
@@ -400,16 +435,19 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
     __syncthreads();
   }
   // largest |value| per channel of the values this pass hands to the next
-  // k-means (fixed-point scale of the centroid sums), when asked for
+  // k-means (fixed-point scale of the centroid sums), and the smallest
+  // nonzero |value| (whether every value fits that fixed point), when asked
   __shared__ uint32_t s_chmax[kD];
+  __shared__ uint32_t s_chmin[kD];
   const bool want_max = !QUANT && p.chmax != nullptr;
   if (want_max) {
-    for (int x = threadIdx.x; x < kD; x += blockDim.x) s_chmax[x] = 0u;
+    for (int x = threadIdx.x; x < kD; x += blockDim.x) { s_chmax[x] = 0u; s_chmin[x] = 0u; }
     __syncthreads();
   }
-  float mx0[8], mx1[8];
+  const float kInf = __int_as_float(0x7f800000);
+  float mx0[8], mx1[8], mn0[8], mn1[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) { mx0[e] = 0.0f; mx1[e] = 0.0f; }
+  for (int e = 0; e < 8; ++e) { mx0[e] = 0.0f; mx1[e] = 0.0f; mn0[e] = kInf; mn1[e] = kInf; }
   const int j = threadIdx.x & 7;
   const int G = GT > 0 ? GT : p.G;
   const int ng = kD / G;
@@ -461,6 +499,8 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
         for (int e = 0; e < 8; ++e) {
           mx0[e] = fmaxf(mx0[e], fabsf(r0[e]));
           mx1[e] = fmaxf(mx1[e], fabsf(r1[e]));
+          mn0[e] = fminf(mn0[e], r0[e] != 0.0f ? fabsf(r0[e]) : kInf);
+          mn1[e] = fminf(mn1[e], r1[e] != 0.0f ? fabsf(r1[e]) : kInf);
         }
       }
     } else {
@@ -474,9 +514,9 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
       const int Gs = G > 64 ? 64 : G;
       lo0 = grp_min(lo0, Gs); hi0 = grp_max(hi0, Gs);
       lo1 = grp_min(lo1, Gs); hi1 = grp_max(hi1, Gs);
-      uint8_t s0, z0, s1, z1;
-      const uint32_t q0 = quant_chunk(r0, lo0, hi0, s_tab, s0, z0);
-      const uint32_t q1 = quant_chunk(r1, lo1, hi1, s_tab, s1, z1);
+      uint8_t s0, z0 = 0, s1, z1 = 0;
+      const uint32_t q0 = SYM ? quant_chunk_sym(r0, lo0, hi0, s_tab, s0) : quant_chunk(r0, lo0, hi0, s_tab, s0, z0);
+      const uint32_t q1 = SYM ? quant_chunk_sym(r1, lo1, hi1, s_tab, s1) : quant_chunk(r1, lo1, hi1, s_tab, s1, z1);
       if (!valid) continue;
       const int64_t row = (int64_t)u * p.N + i;
       uint8_t* cr = p.codes + row * (kD / 4);
@@ -484,11 +524,11 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
       *reinterpret_cast<uint16_t*>(cr + 16 + 2 * j) = (uint16_t)q1;
       if ((8 * j) % G == 0) {
         p.scale[row * ng + (8 * j) / G] = s0;
-        p.zero[row * ng + (8 * j) / G] = z0;
+        if (!SYM) p.zero[row * ng + (8 * j) / G] = z0;
       }
       if (G < 128 && (64 + 8 * j) % G == 0) {
         p.scale[row * ng + (64 + 8 * j) / G] = s1;
-        p.zero[row * ng + (64 + 8 * j) / G] = z1;
+        if (!SYM) p.zero[row * ng + (64 + 8 * j) / G] = z1;
       }
     }
   }
@@ -501,17 +541,28 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
       mx0[e] = fmaxf(mx0[e], __shfl_xor_sync(0xffffffffu, mx0[e], 16));
       mx1[e] = fmaxf(mx1[e], __shfl_xor_sync(0xffffffffu, mx1[e], 8));
       mx1[e] = fmaxf(mx1[e], __shfl_xor_sync(0xffffffffu, mx1[e], 16));
+      mn0[e] = fminf(mn0[e], __shfl_xor_sync(0xffffffffu, mn0[e], 8));
+      mn0[e] = fminf(mn0[e], __shfl_xor_sync(0xffffffffu, mn0[e], 16));
+      mn1[e] = fminf(mn1[e], __shfl_xor_sync(0xffffffffu, mn1[e], 8));
+      mn1[e] = fminf(mn1[e], __shfl_xor_sync(0xffffffffu, mn1[e], 16));
     }
+    // the smallest nonzero magnitude is kept as 0x7FFFFFFF minus its bits, so
+    // that an atomic maximum finds it and zero means "no nonzero value"
+    auto inv = [](float m) { return m == __int_as_float(0x7f800000) ? 0u : 0x7FFFFFFFu - __float_as_uint(m); };
     if ((threadIdx.x & 31) < 8) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         atomicMax(&s_chmax[8 * j + e], __float_as_uint(mx0[e]));
         atomicMax(&s_chmax[64 + 8 * j + e], __float_as_uint(mx1[e]));
+        atomicMax(&s_chmin[8 * j + e], inv(mn0[e]));
+        atomicMax(&s_chmin[64 + 8 * j + e], inv(mn1[e]));
       }
     }
     __syncthreads();
-    for (int x = threadIdx.x; x < kD; x += blockDim.x)
+    for (int x = threadIdx.x; x < kD; x += blockDim.x) {
       if (s_chmax[x] != 0u) atomicMax(&p.chmax[(int64_t)u * kD + x], s_chmax[x]);
+      if (s_chmin[x] != 0u) atomicMax(&p.chmin[(int64_t)u * kD + x], s_chmin[x]);
+    }
   }
 }
 
@@ -572,31 +623,40 @@ cudaError_t launch_dequant(const DequantParams& p, int dtype, cudaStream_t s) {
   }
   if (splits < 1) splits = 1;
   const int blocks = units * splits;
-  return dtype == kBF16 ? launch_dq_t<kBF16>(p, blocks, splits, smem, s)
-                        : launch_dq_t<kFP32>(p, blocks, splits, smem, s);
+  if (p.sym)
+    return dtype == kBF16 ? launch_dq_t<kBF16, true>(p, blocks, splits, smem, s)
+                          : launch_dq_t<kFP32, true>(p, blocks, splits, smem, s);
+  return dtype == kBF16 ? launch_dq_t<kBF16, false>(p, blocks, splits, smem, s)
+                        : launch_dq_t<kFP32, false>(p, blocks, splits, smem, s);
 }
 
-template <int DT, bool Q, bool C, int GT>
+template <int DT, bool Q, bool C, int GT, bool SYM>
 static cudaError_t launch_rq_g(const ResidualParams& p, dim3 grid, int64_t per, size_t smem, cudaStream_t s) {
-  cudaError_t e = set_smem(qvg_residual_quant<DT, Q, C, GT>, smem);
+  cudaError_t e = set_smem(qvg_residual_quant<DT, Q, C, GT, SYM>, smem);
   if (e != cudaSuccess) return e;
-  qvg_residual_quant<DT, Q, C, GT><<<grid, kRqThreads, smem, s>>>(p, per);
+  qvg_residual_quant<DT, Q, C, GT, SYM><<<grid, kRqThreads, smem, s>>>(p, per);
   return cudaGetLastError();
 }
 
-// The quantising pass takes the instance of its group size; the others do
-// not use G.
+template <int DT, bool Q, bool C, bool SYM>
+static cudaError_t launch_rq_mode(const ResidualParams& p, dim3 grid, int64_t per, size_t smem, cudaStream_t s) {
+  switch (p.G) {
+    case 8: return launch_rq_g<DT, Q, C, 8, SYM>(p, grid, per, smem, s);
+    case 16: return launch_rq_g<DT, Q, C, 16, SYM>(p, grid, per, smem, s);
+    case 32: return launch_rq_g<DT, Q, C, 32, SYM>(p, grid, per, smem, s);
+    case 64: return launch_rq_g<DT, Q, C, 64, SYM>(p, grid, per, smem, s);
+    case 128: return launch_rq_g<DT, Q, C, 128, SYM>(p, grid, per, smem, s);
+    default: return launch_rq_g<DT, Q, C, 0, SYM>(p, grid, per, smem, s);
+  }
+}
+
+// The quantising pass takes the instance of its group size and scale mode;
+// the others use neither.
 template <int DT, bool Q, bool C>
 static cudaError_t launch_rq(const ResidualParams& p, dim3 grid, int64_t per, size_t smem, cudaStream_t s) {
-  if (!Q) return launch_rq_g<DT, Q, C, 0>(p, grid, per, smem, s);
-  switch (p.G) {
-    case 8: return launch_rq_g<DT, Q, C, 8>(p, grid, per, smem, s);
-    case 16: return launch_rq_g<DT, Q, C, 16>(p, grid, per, smem, s);
-    case 32: return launch_rq_g<DT, Q, C, 32>(p, grid, per, smem, s);
-    case 64: return launch_rq_g<DT, Q, C, 64>(p, grid, per, smem, s);
-    case 128: return launch_rq_g<DT, Q, C, 128>(p, grid, per, smem, s);
-    default: return launch_rq_g<DT, Q, C, 0>(p, grid, per, smem, s);
-  }
+  if (!Q) return launch_rq_g<DT, Q, C, 0, false>(p, grid, per, smem, s);
+  return p.sym ? launch_rq_mode<DT, Q, C, true>(p, grid, per, smem, s)
+               : launch_rq_mode<DT, Q, C, false>(p, grid, per, smem, s);
 }
 
 cudaError_t launch_residual(const ResidualParams& p, int dtype, bool quant, cudaStream_t s) {

@@ -285,7 +285,9 @@ qvg_assign_candidates(const void* R, const void* C, const int K, const int64_t N
 // is associative, so the sums are exact and do not depend on the order in
 // which tokens are added -- the update may use atomics and still be
 // deterministic -- and S * 2^L_c equals the fp64 sum taken in any order
-// whenever that sum is itself exact.  The mean is one fp64 divide of the sum
+// whenever that sum is itself exact.  (A channel with a value below the
+// window takes an exact 320-bit sum in the centroid kernel instead; see
+// exact_member_sum.)  The mean is one fp64 divide of the sum
 // (converted exactly, or rounded once if it needs more than 53 bits) by the
 // member count, rounded once to the storage dtype.
 //
@@ -327,13 +329,16 @@ __device__ __forceinline__ int fix_exponent(uint32_t maxbits, int log2n) {
 // Assignments of tokens c + j*blockDim.x + threadIdx.x, j < kScan: new (kn)
 // and previous (ko; -1 on a full pass).  Past the end both read -1, so
 // kn == ko marks "nothing to do" for unchanged and missing tokens alike.
+// Indices are clamped to K - 1: every stored assignment is below K, but after
+// a device-side timeout the assignments of the abandoned tiles were never
+// written, and the clamp keeps every later access of this call in bounds.
 __device__ __forceinline__ void load_assignments(const uint8_t* piu, const uint8_t* pio, int64_t N, int64_t c,
-                                                 int (&kn)[kScan], int (&ko)[kScan]) {
+                                                 int K, int (&kn)[kScan], int (&ko)[kScan]) {
 #pragma unroll
   for (int j = 0; j < kScan; ++j) {
     const int64_t t = c + (int64_t)j * blockDim.x + threadIdx.x;
-    kn[j] = t < N ? (int)piu[t] : -1;
-    ko[j] = (t < N && pio != nullptr) ? (int)pio[t] : -1;
+    kn[j] = t < N ? min((int)piu[t], K - 1) : -1;
+    ko[j] = (t < N && pio != nullptr) ? min((int)pio[t], K - 1) : -1;
   }
 }
 
@@ -373,7 +378,7 @@ qvg_update_bucket(const UpdateParams p) {
   const int64_t step = (int64_t)kScan * blockDim.x;
   for (int64_t c = 0; c < N; c += step) {
     int kn[kScan], ko[kScan];
-    load_assignments(piu, pio, N, c, kn, ko);
+    load_assignments(piu, pio, N, c, K, kn, ko);
 #pragma unroll
     for (int j = 0; j < kScan; ++j) {
       const bool ch = kn[j] != ko[j];
@@ -419,7 +424,7 @@ qvg_update_bucket(const UpdateParams p) {
   uint32_t* list = p.list + (int64_t)u * 2 * N;    // capacity 2N entries per block
   for (int64_t c = 0; c < N; c += step) {
     int kn[kScan], ko[kScan];
-    load_assignments(piu, pio, N, c, kn, ko);
+    load_assignments(piu, pio, N, c, K, kn, ko);
 #pragma unroll
     for (int j = 0; j < kScan; ++j) {
       const bool ch = kn[j] != ko[j];
@@ -568,6 +573,135 @@ qvg_update_sum(const UpdateParams p) {
   cp_async_wait_groups<0>();
 }
 
+// ---------------------------------------------------------------- sums beyond the fixed-point window
+// A channel whose smallest nonzero |value| in the block has a quantum below
+// 2^L_c (more than about 39 binades under the channel's largest magnitude for
+// bf16) does not fit the 64-bit fixed point.  For such a channel the centroid
+// kernel forms each member sum exactly from scratch, in a 320-bit
+// two's-complement integer (ten 32-bit limbs, least significant first) that
+// counts units of 2^-149: every fp32 or bf16 value is a whole number of units
+// below 2^277, and fewer than 2^23 of them sum to less than 2^300.
+constexpr int kWideLimbs = 10;
+struct Wide320 {
+  uint32_t w[kWideLimbs];
+};
+
+__device__ __forceinline__ void wide_clear(Wide320& a) {
+#pragma unroll
+  for (int j = 0; j < kWideLimbs; ++j) a.w[j] = 0u;
+}
+
+// a += b, or a -= b when `sub`, limb by limb with the carry (borrow) in 64 bits.
+__device__ __forceinline__ void wide_accumulate(Wide320& a, const Wide320& b, bool sub) {
+  uint64_t c = 0;
+#pragma unroll
+  for (int j = 0; j < kWideLimbs; ++j) {
+    if (!sub) {
+      const uint64_t t = (uint64_t)a.w[j] + b.w[j] + c;
+      a.w[j] = (uint32_t)t;
+      c = t >> 32;
+    } else {
+      const uint64_t t = (uint64_t)a.w[j] - b.w[j] - c;
+      a.w[j] = (uint32_t)t;
+      c = (t >> 63) & 1u;
+    }
+  }
+}
+
+// a += v for an fp32 value v (bf16 values are widened exactly): |v| is
+// M * 2^(P - 149) with M the significand (implicit bit included) and P the
+// biased exponent minus one (zero for subnormals), so M lands at bit P.
+__device__ __forceinline__ void wide_add_value(Wide320& a, float v) {
+  const uint32_t bits = __float_as_uint(v);
+  const uint32_t E = (bits >> 23) & 0xFFu;
+  const uint32_t M = E ? ((bits & 0x7FFFFFu) | 0x800000u) : (bits & 0x7FFFFFu);
+  if (M == 0u) return;
+  const int P = E ? (int)E - 1 : 0;
+  const int L0 = P >> 5, sh = P & 31;
+  Wide320 b;
+#pragma unroll
+  for (int j = 0; j < kWideLimbs; ++j)
+    b.w[j] = j == L0 ? (M << sh) : (j == L0 + 1 && sh ? (M >> (32 - sh)) : 0u);
+  wide_accumulate(a, b, (bits >> 31) != 0u);
+}
+
+// The integer's value (units of 2^-149) rounded once to the nearest double,
+// ties to even.
+__device__ __forceinline__ double wide_to_double(Wide320 a) {
+  const bool neg = (a.w[kWideLimbs - 1] >> 31) != 0u;
+  if (neg) {                                   // magnitude: ~a + 1
+    uint64_t c = 1;
+#pragma unroll
+    for (int j = 0; j < kWideLimbs; ++j) {
+      const uint64_t t = (uint64_t)(~a.w[j]) + c;
+      a.w[j] = (uint32_t)t;
+      c = t >> 32;
+    }
+  }
+  int top = -1;                                // highest set bit
+#pragma unroll
+  for (int j = kWideLimbs - 1; j >= 0; --j)
+    if (top < 0 && a.w[j] != 0u) top = 32 * j + 31 - __clz(a.w[j]);
+  if (top < 0) return 0.0;
+  // the 64 bits [start, start + 64) of the magnitude (bits below 0 read as 0)
+  auto window = [&](int start) {
+    uint64_t r = 0;
+#pragma unroll
+    for (int j = 0; j < kWideLimbs; ++j) {
+      const int pos = 32 * j - start;          // where limb j's bit 0 lands
+      if (pos > -32 && pos < 64) r |= pos >= 0 ? ((uint64_t)a.w[j] << pos) : ((uint64_t)a.w[j] >> (-pos));
+    }
+    return r;
+  };
+  double mag;
+  if (top <= 52) {                             // fewer than 54 bits: exact
+    mag = __dmul_rn((double)window(0), 0x1p-149);
+  } else {
+    const int start = top - 63;                // bit 63 of the window is the top bit
+    const uint64_t w = window(start);
+    bool sticky = false;                       // any set bit below `start`
+#pragma unroll
+    for (int j = 0; j < kWideLimbs; ++j) {
+      const int lo = 32 * j;
+      if (lo + 32 <= start) sticky |= a.w[j] != 0u;
+      else if (lo < start) sticky |= (a.w[j] & ((1u << (start - lo)) - 1u)) != 0u;
+    }
+    uint64_t mant = w >> 11;                   // 53 bits
+    const uint64_t rest = w & 0x7FFull;
+    int e2 = start + 11 - 149;                 // the value is mant * 2^e2
+    if (rest > 0x400ull || (rest == 0x400ull && (sticky || (mant & 1ull)))) ++mant;
+    if (mant == (1ull << 53)) { mant >>= 1; ++e2; }
+    mag = __dmul_rn((double)mant, __longlong_as_double((long long)(1023 + e2) << 52));
+  }
+  return neg ? -mag : mag;
+}
+
+// The exact sum of channel c over the tokens of block u assigned to
+// centroid k, rounded once to fp64 (the whole warp scans the assignments).
+template <int DT>
+__device__ double exact_member_sum(const UpdateParams& p, int u, int k, int c) {
+  constexpr int ESZ = Store<DT>::bytes;
+  const int lane = threadIdx.x & 31;
+  const uint8_t* piu = p.pi + (int64_t)u * p.N;
+  const char* Ru = static_cast<const char*>(p.R) + (int64_t)u * p.N * kD * ESZ;
+  Wide320 acc;
+  wide_clear(acc);
+  for (int64_t i = lane; i < p.N; i += 32) {
+    if ((int)piu[i] != k) continue;
+    const float v = DT == kBF16 ? bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(Ru)[i * kD + c])
+                                : reinterpret_cast<const float*>(Ru)[i * kD + c];
+    wide_add_value(acc, v);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    Wide320 o;
+#pragma unroll
+    for (int j = 0; j < kWideLimbs; ++j) o.w[j] = __shfl_xor_sync(0xffffffffu, acc.w[j], off);
+    wide_accumulate(acc, o, false);
+  }
+  return wide_to_double(acc);
+}
+
 // A warp per centroid: new count; for a non-empty centroid the mean of the
 // exact sum, rounded once to the storage dtype, and its squared norm.
 template <int DT>
@@ -590,11 +724,34 @@ qvg_update_centroids(const UpdateParams p) {
   const double dn = (double)n;
   double sq = 0.0;
   double mean[4];
+  uint32_t wide = 0;                     // this lane's channels outside the fixed-point window
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const int L = fix_exponent(p.chmax[(int64_t)u * kD + 4 * lane + e], p.log2n);
     const double scale = __longlong_as_double((long long)(1023 + L) << 52);
     mean[e] = __ddiv_rn(__dmul_rn(__ll2double_rn(sum[e]), scale), dn);
+    // the quantum of the smallest nonzero value, 2^(e_min - p) with p the
+    // stored fraction bits, must be at least 2^L for the sum to be exact
+    const uint32_t inv = p.chmin[(int64_t)u * kD + 4 * lane + e];
+    if (inv != 0u) {
+      const uint32_t mb = 0x7FFFFFFFu - inv;
+      const int emin = (int)((mb >> 23) & 0xFFu) == 0 ? -126 : (int)((mb >> 23) & 0xFFu) - 127;
+      if (emin - (DT == kBF16 ? 7 : 23) < L) wide |= 1u << e;
+    }
+  }
+  // rare: exact sums for those channels (every lane of the warp takes part)
+  unsigned any = __ballot_sync(0xffffffffu, wide != 0u);
+  while (any) {
+    const int src = __ffs(any) - 1;
+    any &= any - 1u;
+    const uint32_t wb = __shfl_sync(0xffffffffu, wide, src);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if ((wb >> e) & 1u) {
+        const double exact = exact_member_sum<DT>(p, u, k, 4 * src + e);
+        if (lane == src) mean[e] = __ddiv_rn(exact, dn);
+      }
+    }
   }
   if (DT == kBF16) {
     uint16_t h[4];

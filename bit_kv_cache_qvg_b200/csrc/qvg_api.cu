@@ -34,6 +34,20 @@ int device_sm_count() {
   return cached[dev];
 }
 
+bool fault_injected(const char* what) {
+  const char* env = std::getenv("QVG_FAULT_INJECT");
+  if (env == nullptr || *env == '\0') return false;
+  const size_t n = std::strlen(what);
+  for (const char* p = env; *p;) {
+    const char* e = std::strchr(p, ',');
+    const size_t len = e ? (size_t)(e - p) : std::strlen(p);
+    if (len == n && std::strncmp(p, what, n) == 0) return true;
+    if (e == nullptr) break;
+    p = e + 1;
+  }
+  return false;
+}
+
 cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
   static std::mutex mu;
@@ -44,6 +58,37 @@ cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes) {
   const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e == cudaSuccess) done.emplace_back(kernel, bytes);
   return e;
+}
+
+// The sticky status word at `word` (device memory: the first 4 bytes of a
+// workspace, of a cache's workspace or of the static reserve), read without
+// waiting for the GPU: only when every operation queued on `s` has completed
+// and `s` is not being captured into a graph.  While earlier work is still in
+// flight its outcome is not known yet and the result is QVG_OK; a later call,
+// or the status query of the object, reports it.
+qvg_status peek_sticky(const void* word, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) { cudaGetLastError(); return QVG_OK; }
+  if (cs != cudaStreamCaptureStatusNone) return QVG_OK;
+  const cudaError_t q = cudaStreamQuery(s);
+  if (q == cudaErrorNotReady) return QVG_OK;
+  if (q != cudaSuccess) return QVG_ERR_CUDA;
+  uint32_t w = 0;
+  if (cudaMemcpyAsync(&w, word, sizeof(w), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return QVG_ERR_CUDA;
+  return w == 0 ? QVG_OK : QVG_ERR_DEVICE_TIMEOUT;
+}
+
+// Read and clear a sticky status word after the work queued on `s` has
+// completed (synchronises `s`).
+qvg_status take_sticky(void* word, cudaStream_t s) {
+  uint32_t w = 0;
+  if (cudaMemcpyAsync(&w, word, sizeof(w), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess || cudaMemsetAsync(word, 0, sizeof(w), s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return QVG_ERR_CUDA;
+  return w == 0 ? QVG_OK : QVG_ERR_DEVICE_TIMEOUT;
 }
 
 }  // namespace qvg
@@ -78,7 +123,7 @@ Plan make_plan(const qvg_config& c, int64_t N, int W, int dtype) {
   p.off_cn = o;                           o = align_up(o + (size_t)W * kMaxK * sizeof(float));
   p.off_list = o;                         o = align_up(o + (size_t)W * N * 8);
   p.off_listcnt = o;                      o = align_up(o + (size_t)W * sizeof(uint32_t));
-  p.off_chmax = o;                        o = align_up(o + (size_t)W * kD * sizeof(uint32_t));
+  p.off_chmax = o;                        o = align_up(o + 2 * (size_t)W * kD * sizeof(uint32_t));  // max, then min
   p.off_off = o;                          o = align_up(o + (size_t)W * (c.K + 1) * sizeof(int));
   p.off_cnt = o;                          o = align_up(o + (size_t)W * c.K * sizeof(int));
   p.off_S = o;                            o = align_up(o + (size_t)W * c.K * kD * sizeof(long long));
@@ -147,6 +192,7 @@ qvg_status check_config(const qvg_config* c, int64_t N, int32_t H, int32_t d, qv
   if (c == nullptr) return QVG_ERR_INVALID_ARG;
   if (dtype != QVG_BF16 && dtype != QVG_FP32) return QVG_ERR_INVALID_ARG;
   if (c->bits != 2 || c->K < 1 || c->K > 256 || c->T < 0) return QVG_ERR_INVALID_ARG;
+  if (c->scale_mode != QVG_SCALE_ASYM && c->scale_mode != QVG_SCALE_SYM) return QVG_ERR_INVALID_ARG;
   if (c->group_size < 4 || c->group_size % 4 != 0 || d < 4 || d % c->group_size != 0)
     return QVG_ERR_INVALID_ARG;
   if (N < 0 || H < 1) return QVG_ERR_INVALID_ARG;
@@ -156,6 +202,7 @@ qvg_status check_config(const qvg_config* c, int64_t N, int32_t H, int32_t d, qv
 }
 
 qvg_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QVG_OK : QVG_ERR_CUDA; }
+
 
 
 // ---------------------------------------------------------------- diagnostics
@@ -248,11 +295,12 @@ const char* qvg_version(void) { return "qvg-b200 sm_100a"; }
 size_t qvg_packed_bytes(const qvg_config* c, int64_t N, int32_t H, int32_t d, qvg_dtype dtype) {
   if (c == nullptr || c->bits != 2 || c->K < 1 || c->K > 256 || c->T < 0 || c->group_size < 4 ||
       c->group_size % 4 != 0 || d < 4 || d % c->group_size != 0 || N < 0 || H < 1 ||
-      (dtype != QVG_BF16 && dtype != QVG_FP32))
+      (dtype != QVG_BF16 && dtype != QVG_FP32) ||
+      (c->scale_mode != QVG_SCALE_ASYM && c->scale_mode != QVG_SCALE_SYM))
     return 0;
   const size_t esz = (size_t)esize(dtype);
   const size_t codes = (size_t)H * N * d * c->bits / 8;
-  const size_t scales = 2 * (size_t)H * N * (d / c->group_size);
+  const size_t scales = (c->scale_mode == QVG_SCALE_SYM ? 1 : 2) * (size_t)H * N * (d / c->group_size);
   const size_t assign = (size_t)c->T * H * N;
   const size_t cents = (size_t)c->T * H * c->K * d * esz;
   return codes + scales + assign + cents;
@@ -277,7 +325,8 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
   const bool warm = init != nullptr;
   const int iters = warm ? c.warm_iters : c.iters;
   if (N < 1 || X == nullptr || out == nullptr || workspace == nullptr) return QVG_ERR_INVALID_ARG;
-  if (out->codes == nullptr || out->scale == nullptr || out->zero == nullptr) return QVG_ERR_INVALID_ARG;
+  const bool sym = c.scale_mode == QVG_SCALE_SYM;
+  if (out->codes == nullptr || out->scale == nullptr || (out->zero == nullptr && !sym)) return QVG_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(init, 16) || !aligned(out->centroids, 16) || !aligned(out->codes, 2) ||
       !aligned(workspace, kAlign))
     return QVG_ERR_INVALID_ARG;
@@ -288,6 +337,11 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
   const int dt = (int)dtype;
   const size_t esz = (size_t)esize(dt);
+  if (make_plan(c, N, 1, dt).total > ws_bytes) return QVG_ERR_WORKSPACE_TOO_SMALL;
+  // a timeout recorded by earlier (completed) work on this workspace is
+  // reported before anything is queued; qvg_workspace_status clears it
+  st = peek_sticky(workspace, s);
+  if (st != QVG_OK) return st;
 
   int W = preferred_batch(c, N, H, dt);
   int lanes = std::min(max_lanes, wave_lanes(H, W));
@@ -310,6 +364,9 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
   // bf16 blocks take the tensor-core assignment; fp32 blocks the exact CUDA-core one
   const bool use_tc = dt == kBF16 && assign_path_tc();
   const int ng = kD / c.group_size;
+  // QVG_FAULT_INJECT=timeout: the tensor-core assignment's first CTA withholds
+  // a tile load and waits 1 ms, so that its bounded waits run out (tests only)
+  const bool hook_timeout = fault_injected("timeout");
 
   // one wave: blocks u0 .. u0+w-1 on stream s with workspace ws
   auto run_wave = [&](int u0, int w, cudaStream_t s, char* ws) -> qvg_status {
@@ -318,12 +375,13 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
     uint2* list = reinterpret_cast<uint2*>(ws + plan.off_list);
     uint32_t* list_count = reinterpret_cast<uint32_t*>(ws + plan.off_listcnt);
     uint32_t* chmax = reinterpret_cast<uint32_t*>(ws + plan.off_chmax);
+    uint32_t* chmin = chmax + (size_t)plan.W * kD;
     const char* Xu = static_cast<const char*>(X) + (size_t)u0 * N * kD * esz;
     ResidualParams rq{};
-    rq.N = N; rq.W = w; rq.K = c.K; rq.G = c.group_size;
+    rq.N = N; rq.W = w; rq.K = c.K; rq.G = c.group_size; rq.sym = sym ? 1 : 0;
     rq.codes = out->codes + (size_t)u0 * N * (kD / 4);
     rq.scale = out->scale + (size_t)u0 * N * ng;
-    rq.zero = out->zero + (size_t)u0 * N * ng;
+    rq.zero = sym ? nullptr : out->zero + (size_t)u0 * N * ng;
     if (c.T == 0) {
       rq.R_in = Xu;
       QVG_TRY(plaunch(K_RESIDUAL_QUANT, s, [&] { return launch_residual(rq, dt, true, s); }));
@@ -335,8 +393,8 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
       uint8_t* pit = out->assign + ((size_t)t * H + u0) * N;
       if (t == 0) {   // squared row norms of X (assignment error bound), channel maxima (update scale)
         ResidualParams nq = rq;
-        nq.R_in = Xu; nq.C = nullptr; nq.R_out = nullptr; nq.rnorm2 = rnorm; nq.chmax = chmax;
-        QVG_TRY(cudaMemsetAsync(chmax, 0, (size_t)w * kD * sizeof(uint32_t), s));
+        nq.R_in = Xu; nq.C = nullptr; nq.R_out = nullptr; nq.rnorm2 = rnorm; nq.chmax = chmax; nq.chmin = chmin;
+        QVG_TRY(cudaMemsetAsync(chmax, 0, 2 * (size_t)plan.W * kD * sizeof(uint32_t), s));
         QVG_TRY(plaunch(K_ROWNORM, s, [&] { return launch_residual(nq, dt, false, s); }));
       }
       if (warm) {
@@ -362,6 +420,8 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
           tp.R = Rin; tp.rnorm2 = rnorm; tp.C = Ct; tp.cn = cn; tp.pi = pi_new; tp.list = list;
           tp.list_count = list_count; tp.status = status; tp.flagged = flagged;
           tp.N = N; tp.W = w; tp.K = c.K; tp.gamma = kTcGamma;
+          tp.hook_withhold = -1; tp.hook_wait_ns = 0;
+          if (hook_timeout) { tp.hook_withhold = 0; tp.hook_wait_ns = 1000000ull; }   // 1 ms
           QVG_TRY(plaunch(K_ASSIGN_TC, s, [&] { return launch_assign_tc(tp, s); }));
           QVG_TRY(plaunch(K_RECHECK, s, [&] {
             return launch_assign_candidates(Rin, Ct, c.K, N, w, list, list_count, pi_new, s);
@@ -370,7 +430,7 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
           QVG_TRY(plaunch(K_ASSIGN_EXACT, s, [&] { return launch_assign_exact(ap, dt, s); }));
         }
         UpdateParams up{};
-        up.R = Rin; up.pi = pi_new; up.pi_old = pi_old; up.chmax = chmax; up.C = Ct; up.cn = cn;
+        up.R = Rin; up.pi = pi_new; up.pi_old = pi_old; up.chmax = chmax; up.chmin = chmin; up.C = Ct; up.cn = cn;
         up.N = N; up.W = w; up.K = c.K; up.log2n = log2n;
         up.list = reinterpret_cast<uint32_t*>(list);   // the near-tie list is consumed by now
         up.off = reinterpret_cast<int*>(ws + plan.off_off);
@@ -385,8 +445,8 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
       rp.R_in = Rin; rp.C = Ct; rp.pi = pit;
       if (t + 1 < c.T) {
         void* Rout = ws + plan.off_R[t % 2];
-        rp.R_out = Rout; rp.rnorm2 = rnorm; rp.chmax = chmax;
-        QVG_TRY(cudaMemsetAsync(chmax, 0, (size_t)w * kD * sizeof(uint32_t), s));
+        rp.R_out = Rout; rp.rnorm2 = rnorm; rp.chmax = chmax; rp.chmin = chmin;
+        QVG_TRY(cudaMemsetAsync(chmax, 0, 2 * (size_t)plan.W * kD * sizeof(uint32_t), s));
         QVG_TRY(plaunch(K_RESIDUAL, s, [&] { return launch_residual(rp, dt, false, s); }));
         Rin = Rout;
       } else {
@@ -401,7 +461,8 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
       st = run_wave(u0, std::min(W, H - u0), s, ws0);
       if (st != QVG_OK) return st;
     }
-    return QVG_OK;
+    // QVG_FAULT_INJECT=stream: report the stream error a failed launch would
+    return fault_injected("stream") ? QVG_ERR_CUDA : QVG_OK;
   }
   // Two lanes: the side stream joins after the caller's stream reaches this
   // call, and the caller's stream waits for the side stream at the end (also
@@ -422,6 +483,7 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
   if (cudaEventRecord(join, s1) != cudaSuccess || cudaStreamWaitEvent(s, join, 0) != cudaSuccess) st = QVG_ERR_CUDA;
   cudaEventDestroy(fork);
   cudaEventDestroy(join);
+  if (st == QVG_OK && fault_injected("stream")) st = QVG_ERR_CUDA;
   return st;
 }
 
@@ -440,7 +502,7 @@ qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packed, qvg_d
   qvg_status st = check_config(cfg, N, H, d, dtype);
   if (st != QVG_OK) return st;
   if (packed == nullptr || Y == nullptr || packed->codes == nullptr || packed->scale == nullptr ||
-      packed->zero == nullptr)
+      (packed->zero == nullptr && cfg->scale_mode != QVG_SCALE_SYM))
     return QVG_ERR_INVALID_ARG;
   if (cfg->T > 0 && (packed->assign == nullptr || packed->centroids == nullptr)) return QVG_ERR_INVALID_ARG;
   if (!aligned(Y, 16) || !aligned(packed->centroids, 16) || !aligned(packed->codes, 16)) return QVG_ERR_INVALID_ARG;
@@ -451,10 +513,12 @@ qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packed, qvg_d
   p.codes = packed->codes; p.scale = packed->scale; p.zero = packed->zero;
   p.assign = packed->assign; p.centroids = packed->centroids; p.Y = Y;
   p.chunk_off = nullptr; p.N = N; p.y_head_stride = N; p.n_chunks = 1; p.H = H;
-  p.K = cfg->K; p.T = cfg->T; p.G = cfg->group_size;
+  p.K = cfg->K; p.T = cfg->T; p.G = cfg->group_size; p.sym = cfg->scale_mode == QVG_SCALE_SYM;
   p.t_smem = std::min<int>(cfg->T, (int)((160 * 1024) / table));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
-  return cuda_status(plaunch(K_DEQUANT, s, [&] { return launch_dequant(p, dt, s); }));
+  st = cuda_status(plaunch(K_DEQUANT, s, [&] { return launch_dequant(p, dt, s); }));
+  if (st == QVG_OK && fault_injected("stream")) st = QVG_ERR_CUDA;
+  return st;
 }
 
 int64_t qvg_workspace_flagged(void* workspace, size_t ws_bytes, qvg_stream_t stream_) {
@@ -469,12 +533,7 @@ int64_t qvg_workspace_flagged(void* workspace, size_t ws_bytes, qvg_stream_t str
 
 qvg_status qvg_workspace_status(void* workspace, size_t ws_bytes, qvg_stream_t stream_) {
   if (workspace == nullptr || ws_bytes < 16) return QVG_ERR_INVALID_ARG;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
-  uint32_t word = 0;
-  QVG_TRY(cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s));
-  QVG_TRY(cudaStreamSynchronize(s));
-  QVG_TRY(cudaMemsetAsync(workspace, 0, 4, s));
-  return word == 0 ? QVG_OK : QVG_ERR_DEVICE_TIMEOUT;
+  return take_sticky(workspace, reinterpret_cast<cudaStream_t>(stream_));
 }
 
 
@@ -535,6 +594,7 @@ struct qvg_cache {
   qvg_config cfg{};
   int dtype = 0, H = 0;
   int64_t max_tokens = 0;
+  int64_t max_chunk_tokens = 0;
   int max_chunks = 0;
   uint8_t* codes = nullptr;
   uint8_t* scale = nullptr;
@@ -558,33 +618,46 @@ static void cache_free(qvg_cache* c) {
 }
 
 qvg_status qvg_cache_create(const qvg_config* cfg, qvg_dtype dtype, int32_t H, int32_t d,
-                            int64_t max_tokens, int32_t max_chunks, qvg_cache** out) {
+                            int64_t max_tokens, int32_t max_chunks, int64_t max_chunk_tokens,
+                            qvg_cache** out) {
   if (out == nullptr) return QVG_ERR_INVALID_ARG;
   *out = nullptr;
   qvg_status st = check_config(cfg, max_tokens, H, d, dtype);
   if (st != QVG_OK) return st;
-  if (max_tokens < 1 || max_chunks < 1) return QVG_ERR_INVALID_ARG;
+  if (max_tokens < 1 || max_chunks < 1 || max_chunk_tokens < 0) return QVG_ERR_INVALID_ARG;
+  if (max_chunk_tokens == 0 || max_chunk_tokens > max_tokens) max_chunk_tokens = max_tokens;
   if (cfg->T > 0 && (cfg->iters < 1 || cfg->warm_iters < 1)) return QVG_ERR_INVALID_ARG;
+  if (cfg->T > 0 && max_chunk_tokens < cfg->K) return QVG_ERR_INVALID_ARG;   // chunk 0 needs K tokens
+  // QVG_FAULT_INJECT=alloc: every device allocation of the cache fails
+  if (fault_injected("alloc")) return QVG_ERR_NO_MEMORY;
+  // the workspace of the largest chunk: any smaller chunk fits in it
+  const size_t ws_bytes = qvg_workspace_bytes(cfg, max_chunk_tokens, H, d, dtype);
+  if (ws_bytes == 0) return QVG_ERR_INVALID_ARG;
   qvg_cache* c = new qvg_cache();
   c->cfg = *cfg; c->dtype = (int)dtype; c->H = H; c->max_tokens = max_tokens; c->max_chunks = max_chunks;
+  c->max_chunk_tokens = max_chunk_tokens;
   const size_t esz = (size_t)esize(c->dtype);
   const int ng = kD / cfg->group_size;
   const size_t n_codes = (size_t)H * max_tokens * (kD / 4);
   const size_t n_sc = (size_t)H * max_tokens * ng;
+  const size_t n_zero = cfg->scale_mode == QVG_SCALE_SYM ? 16 : n_sc;   // no zero points when symmetric
   const size_t n_as = std::max<size_t>(1, (size_t)cfg->T * H * max_tokens);
   const size_t n_tab = std::max<size_t>(16, (size_t)max_chunks * cfg->T * H * cfg->K * kD * esz);
   bool ok = cudaMalloc(&c->codes, n_codes) == cudaSuccess && cudaMalloc(&c->scale, n_sc) == cudaSuccess &&
-            cudaMalloc(&c->zero, n_sc) == cudaSuccess && cudaMalloc(&c->assign, n_as) == cudaSuccess &&
+            cudaMalloc(&c->zero, n_zero) == cudaSuccess && cudaMalloc(&c->assign, n_as) == cudaSuccess &&
             cudaMalloc(&c->tables, n_tab) == cudaSuccess &&
             cudaMalloc(&c->d_off, sizeof(int64_t) * ((size_t)max_chunks + 1)) == cudaSuccess &&
             cudaMemset(c->d_off, 0, sizeof(int64_t) * ((size_t)max_chunks + 1)) == cudaSuccess &&
-            cudaMallocHost(&c->h_off, sizeof(int64_t) * ((size_t)max_chunks + 1)) == cudaSuccess;
+            cudaMallocHost(&c->h_off, sizeof(int64_t) * ((size_t)max_chunks + 1)) == cudaSuccess &&
+            cudaMalloc(&c->ws, ws_bytes) == cudaSuccess && cudaMemset(c->ws, 0, 16) == cudaSuccess &&
+            cudaDeviceSynchronize() == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     cache_free(c);
     return QVG_ERR_NO_MEMORY;
   }
-  c->bytes = n_codes + 2 * n_sc + n_as + n_tab + sizeof(int64_t) * ((size_t)max_chunks + 1);
+  c->ws_bytes = ws_bytes;
+  c->bytes = n_codes + n_sc + n_zero + n_as + n_tab + sizeof(int64_t) * ((size_t)max_chunks + 1);
   c->h_off[0] = 0;
   c->n_chunks = 0;
   *out = c;
@@ -597,7 +670,7 @@ static void chunk_view(const qvg_cache* c, int chunk, qvg_packed* v) {
   const int ng = kD / c->cfg.group_size;
   v->codes = c->codes + (size_t)c->H * o * (kD / 4);
   v->scale = c->scale + (size_t)c->H * o * ng;
-  v->zero = c->zero + (size_t)c->H * o * ng;
+  v->zero = c->cfg.scale_mode == QVG_SCALE_SYM ? nullptr : c->zero + (size_t)c->H * o * ng;
   v->assign = c->assign + (size_t)c->cfg.T * c->H * o;
   v->centroids = c->tables + (size_t)chunk * c->cfg.T * c->H * c->cfg.K * kD * esz;
 }
@@ -605,21 +678,11 @@ static void chunk_view(const qvg_cache* c, int chunk, qvg_packed* v) {
 qvg_status qvg_append_chunk(qvg_cache* c, const void* X, int64_t n, qvg_stream_t stream_) {
   if (c == nullptr || X == nullptr || n < 1) return QVG_ERR_INVALID_ARG;
   const int chunk = c->n_chunks;
-  if (chunk >= c->max_chunks || c->h_off[chunk] + n > c->max_tokens) return QVG_ERR_CAPACITY;
+  if (chunk >= c->max_chunks || c->h_off[chunk] + n > c->max_tokens || n > c->max_chunk_tokens)
+    return QVG_ERR_CAPACITY;
   if (chunk == 0 && c->cfg.T > 0 && n < c->cfg.K) return QVG_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
-  const size_t need = qvg_workspace_bytes(&c->cfg, n, c->H, kD, (qvg_dtype)c->dtype);
-  if (need > c->ws_bytes) {
-    if (c->ws) {
-      QVG_TRY(cudaStreamSynchronize(s));
-      cudaFree(c->ws);
-      c->ws = nullptr;
-      c->ws_bytes = 0;
-    }
-    if (cudaMalloc(&c->ws, need) != cudaSuccess) { cudaGetLastError(); return QVG_ERR_NO_MEMORY; }
-    QVG_TRY(cudaMemsetAsync(c->ws, 0, 16, s));
-    c->ws_bytes = need;
-  }
+  // the workspace was sized at creation for the largest chunk: no allocation here
   qvg_packed v;
   chunk_view(c, chunk, &v);
   const void* init = nullptr;
@@ -649,10 +712,12 @@ qvg_status qvg_cache_dequantize(const qvg_cache* c, void* Y, qvg_stream_t stream
   p.codes = c->codes; p.scale = c->scale; p.zero = c->zero; p.assign = c->assign;
   p.centroids = c->tables; p.Y = Y; p.chunk_off = c->d_off; p.N = 0;
   p.y_head_stride = c->h_off[n_chunks]; p.n_chunks = n_chunks; p.H = c->H;
-  p.K = c->cfg.K; p.T = c->cfg.T; p.G = c->cfg.group_size;
+  p.K = c->cfg.K; p.T = c->cfg.T; p.G = c->cfg.group_size; p.sym = c->cfg.scale_mode == QVG_SCALE_SYM;
   p.t_smem = std::min<int>(c->cfg.T, (int)((160 * 1024) / table));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
-  return cuda_status(plaunch(K_DEQUANT, s, [&] { return launch_dequant(p, c->dtype, s); }));
+  qvg_status st = cuda_status(plaunch(K_DEQUANT, s, [&] { return launch_dequant(p, c->dtype, s); }));
+  if (st == QVG_OK && fault_injected("stream")) st = QVG_ERR_CUDA;
+  return st;
 }
 
 int64_t qvg_cache_tokens(const qvg_cache* c) { return c ? c->h_off[c->n_chunks] : 0; }
@@ -669,6 +734,11 @@ qvg_status qvg_cache_chunk_view(const qvg_cache* c, int32_t chunk, qvg_packed* v
 }
 
 size_t qvg_cache_device_bytes(const qvg_cache* c) { return c ? c->bytes + c->ws_bytes : 0; }
+
+qvg_status qvg_cache_status(qvg_cache* c, qvg_stream_t stream_) {
+  if (c == nullptr || c->ws == nullptr) return QVG_ERR_INVALID_ARG;
+  return take_sticky(c->ws, reinterpret_cast<cudaStream_t>(stream_));
+}
 
 void qvg_cache_destroy(qvg_cache* c) {
   if (c == nullptr) return;

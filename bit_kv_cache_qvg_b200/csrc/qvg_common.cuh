@@ -99,6 +99,7 @@ struct DequantParams {
   int T;
   int G;
   int t_smem;                 // stages whose tables are staged in shared memory
+  int sym;                    // 1: one scale byte per group, value s*(u - 2); zero unused
 };
 
 }  // namespace qvg

@@ -18,6 +18,16 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
                          size_t ws_bytes, qvg_stream_t stream, int max_lanes);
 // SM count of the current device (cached per device).
 int device_sm_count();
+// Host-side fault injection for tests: true when the comma-separated list in
+// the environment variable QVG_FAULT_INJECT names `what` ("alloc", "stream",
+// "timeout").  Read on every call; unset in normal use.
+bool fault_injected(const char* what);
+// The sticky status word of a workspace, cache or static reserve (its first
+// four bytes): peek_sticky reads it without waiting (QVG_OK while work queued
+// on `s` is still running or `s` is being captured); take_sticky waits for
+// `s`, reads it and clears it.
+qvg_status peek_sticky(const void* word, cudaStream_t s);
+qvg_status take_sticky(void* word, cudaStream_t s);
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` (the
 // attribute call is made once per kernel and size; later calls are cached).
 cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes);
@@ -40,13 +50,16 @@ struct ResidualParams {
   float* rnorm2;           // [W][N] or nullptr
   uint32_t* chmax;         // [W][d] or nullptr: atomic max of the bits of |value| per channel
                            // of the values read (no C) or written (with C); starts at zero
+  uint32_t* chmin;         // [W][d], used with chmax: atomic max of 0x7FFFFFFF minus the bits of
+                           // the smallest nonzero |value| per channel (0: none); starts at zero
   uint8_t* codes;          // [W][N][d/4]
   uint8_t* scale;          // [W][N][d/G]
-  uint8_t* zero;           // [W][N][d/G]
+  uint8_t* zero;           // [W][N][d/G] (unused when sym)
   int64_t N;
   int W;
   int K;
   int G;
+  int sym;                 // 1: one E4M3 scale per group (symmetric signed INT2)
 };
 cudaError_t launch_residual(const ResidualParams& p, int dtype, bool quant, cudaStream_t s);
 
@@ -90,6 +103,8 @@ struct AssignTcParams {
   int W;
   int K;
   float gamma;
+  int hook_withhold;           // test hook (QVG_FAULT_INJECT=timeout): tile the hooked CTA never loads, or -1
+  uint64_t hook_wait_ns;       // test hook: wait limit of the hooked CTA, or 0 (hook off)
 };
 cudaError_t launch_assign_tc(const AssignTcParams& p, cudaStream_t s);
 // Exact decision of the listed tokens: sequential fp64 squared distances to
@@ -105,6 +120,7 @@ struct UpdateParams {
   const uint8_t* pi;      // [W][N] assignment of this iteration
   const uint8_t* pi_old;  // [W][N] assignment of the previous iteration, or nullptr (full sums)
   const uint32_t* chmax;  // [W][d] bits of the largest |value| of each channel of R
+  const uint32_t* chmin;  // [W][d] 0x7FFFFFFF minus the bits of the smallest nonzero |value| (0: none)
   uint32_t* list;         // [W][2N] scratch: entries bucketed by centroid
   int* off;               // [W][K+1] scratch: bucket offsets
   int* cnt;               // [W][K]   scratch: member counts (first iteration) or their changes

@@ -15,6 +15,13 @@
 // the k-means working set of as many blocks per wave as fit, and at least
 // one: about 120,000 tokens per block at bf16, K = 256, T = 2.  A call whose
 // single block needs more is rejected before any work is queued.
+//
+// Its first 16 bytes are the workspace status word and near-tie counter.  A
+// __device__ array starts zeroed when the module loads, and no kernel needs
+// those bytes to be zero (the status word is only ever set, the counter only
+// ever added to), so a call queues no clearing of its own: a timeout that a
+// bounded device-side wait records stays in the word until
+// qvg_static_status reads and clears it.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -40,12 +47,15 @@ void* g_scratch_ptr[kMaxDevices] = {};
 // device (the lookup may load this file's device code on first use).
 qvg_status scratch_on_current_device(void** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return QVG_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return QVG_ERR_CUDA; }
   if (dev < 0 || dev >= kMaxDevices) return QVG_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_setup_mu);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_qvg_static_scratch) != cudaSuccess || p == nullptr) return QVG_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_qvg_static_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();       // leave no error pending for a later launch check
+      return QVG_ERR_CUDA;
+    }
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];
@@ -58,18 +68,23 @@ extern "C" QVG_API qvg_status qvg_quantize_static(const qvg_config* cfg, const v
                                                   int64_t N, int32_t H, int32_t d,
                                                   const void* init_centroids, const qvg_packed* out,
                                                   qvg_stream_t stream) {
-  // One block's working set must fit in the reserve (a zero size means the
-  // arguments are invalid; qvg_quantize then reports which).
+  // One block's working set must fit in the reserve.  A zero size means the
+  // arguments are invalid: qvg::quantize_impl then reports which, before it
+  // queues anything.
   const size_t one_block = qvg_workspace_bytes(cfg, N, 1, d, dtype);
   if (one_block > kStaticScratchBytes) return QVG_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;
   const qvg_status st = scratch_on_current_device(&scratch);
   if (st != QVG_OK) return st;
-  // The workspace contract: the 16-byte status word and near-tie counter at
-  // the start must read zero when the work begins.  Nothing else in the
-  // scratch needs initialising (every other region is written before read).
-  if (cudaMemsetAsync(scratch, 0, 16, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return QVG_ERR_CUDA;
-  // One wave at a time on the caller's stream: no side stream, no events.
+  // The same checks and kernels as qvg_quantize, one wave at a time on the
+  // caller's stream (no side stream, no events); a timeout recorded in the
+  // reserve by earlier, completed work is returned before anything is queued.
   return qvg::quantize_impl(cfg, X, dtype, N, H, d, init_centroids, out, scratch, kStaticScratchBytes, stream, 1);
+}
+
+extern "C" QVG_API qvg_status qvg_static_status(qvg_stream_t stream) {
+  void* scratch = nullptr;
+  const qvg_status st = scratch_on_current_device(&scratch);
+  if (st != QVG_OK) return st;
+  return qvg::take_sticky(scratch, reinterpret_cast<cudaStream_t>(stream));
 }

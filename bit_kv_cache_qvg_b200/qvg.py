@@ -33,13 +33,17 @@ class QvgError(RuntimeError):
         super().__init__(f"{what}: {STATUS.get(status, status)}" if what else STATUS.get(status, str(status)))
 
 
+ASYM, SYM = 0, 1     # qvg_scale_mode: scale and zero point per group, or one scale per group
+
+
 class Config(C.Structure):
     _fields_ = [("K", C.c_int32), ("T", C.c_int32), ("group_size", C.c_int32),
-                ("bits", C.c_int32), ("iters", C.c_int32), ("warm_iters", C.c_int32)]
+                ("bits", C.c_int32), ("iters", C.c_int32), ("warm_iters", C.c_int32),
+                ("scale_mode", C.c_int32)]
 
     def __repr__(self):
         return (f"Config(K={self.K}, T={self.T}, group_size={self.group_size}, bits={self.bits}, "
-                f"iters={self.iters}, warm_iters={self.warm_iters})")
+                f"iters={self.iters}, warm_iters={self.warm_iters}, scale_mode={self.scale_mode})")
 
 
 class _Packed(C.Structure):
@@ -64,7 +68,9 @@ _SIGS = {
     "qvg_workspace_status": (C.c_int, [C.c_void_p, C.c_size_t, C.c_void_p]),
     "qvg_workspace_flagged": (C.c_int64, [C.c_void_p, C.c_size_t, C.c_void_p]),
     "qvg_cache_create": (C.c_int, [C.POINTER(Config), C.c_int, C.c_int32, C.c_int32, C.c_int64, C.c_int32,
-                                   C.POINTER(C.c_void_p)]),
+                                   C.c_int64, C.POINTER(C.c_void_p)]),
+    "qvg_cache_status": (C.c_int, [C.c_void_p, C.c_void_p]),
+    "qvg_static_status": (C.c_int, [C.c_void_p]),
     "qvg_append_chunk": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p]),
     "qvg_cache_dequantize": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p]),
     "qvg_cache_tokens": (C.c_int64, [C.c_void_p]),
@@ -119,8 +125,24 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else t.data_ptr()
 
 
-def config(K=256, T=2, group_size=64, iters=10, warm_iters=3, bits=2) -> Config:
-    return Config(K, T, group_size, bits, iters, warm_iters)
+def config(K=256, T=2, group_size=64, iters=10, warm_iters=3, bits=2, scale_mode=ASYM) -> Config:
+    return Config(K, T, group_size, bits, iters, warm_iters, scale_mode)
+
+
+# Named operating points.  With one E4M3 scale per group the closed-form
+# compression at K = 256 on a 38,000-token block is 6.97x for "qvg" and
+# 5.03x for "qvg-pro" (the m.163.com article on Quant VideoGen, section 六,
+# reports 6.94-7.05x and 4.97-5.20x; section 七 names G = 64 the best
+# trade-off and G = 16 the high-quality setting).  The pages do not print the
+# settings themselves: these are the ones the closed form admits.
+PRESETS = {
+    "qvg": dict(K=256, T=1, group_size=64, scale_mode=SYM),
+    "qvg-pro": dict(K=256, T=4, group_size=16, scale_mode=SYM),
+}
+
+
+def preset(name: str, iters=10, warm_iters=3) -> Config:
+    return config(iters=iters, warm_iters=warm_iters, **PRESETS[name])
 
 
 @dataclass
@@ -138,7 +160,7 @@ class Packed:
     dtype: int
 
     def struct(self) -> _Packed:
-        return _Packed(_ptr(self.codes), _ptr(self.scale), _ptr(self.zero),
+        return _Packed(_ptr(self.codes), _ptr(self.scale), _ptr(self.zero) if self.zero.numel() else None,
                        _ptr(self.assign) if self.assign.numel() else None,
                        _ptr(self.centroids) if self.centroids.numel() else None)
 
@@ -161,7 +183,7 @@ def alloc_packed(cfg: Config, N: int, H: int, d: int = 128, dtype: int = BF16, d
     return Packed(
         codes=torch.empty((H, N, d // 4), **u8),
         scale=torch.empty((H, N, d // G), **u8),
-        zero=torch.empty((H, N, d // G), **u8),
+        zero=torch.empty((H, N, d // G) if cfg.scale_mode == ASYM else (0,), **u8),
         assign=torch.empty((T, H, N), **u8),
         centroids=torch.empty((T, H, K, d), dtype=_TORCH[dtype], device=device),
         cfg=cfg, N=N, H=H, d=d, dtype=dtype)
@@ -250,6 +272,11 @@ def workspace_status(workspace: torch.Tensor, stream=None) -> int:
     return int(lib().qvg_workspace_status(_ptr(workspace), workspace.numel(), _stream(stream)))
 
 
+def static_status(stream=None) -> int:
+    """qvg_static_status: read and clear the static reserve's status word."""
+    return int(lib().qvg_static_status(_stream(stream)))
+
+
 class _DevView:
     """__cuda_array_interface__ wrapper of a raw device pointer (for views)."""
 
@@ -271,11 +298,12 @@ class Cache:
     warm-started from the previous chunk's centroids; dequantise all."""
 
     def __init__(self, cfg: Config, H: int, max_tokens: int, max_chunks: int, d: int = 128,
-                 dtype: int = BF16):
+                 dtype: int = BF16, max_chunk_tokens: int = 0):
         self.cfg, self.H, self.d, self.dtype = cfg, H, d, dtype
+        self._h = C.c_void_p()
         h = C.c_void_p()
-        _check(lib().qvg_cache_create(C.byref(cfg), dtype, H, d, max_tokens, max_chunks, C.byref(h)),
-               "qvg_cache_create")
+        _check(lib().qvg_cache_create(C.byref(cfg), dtype, H, d, max_tokens, max_chunks, max_chunk_tokens,
+                                      C.byref(h)), "qvg_cache_create")
         self._h = h
 
     def append(self, X: torch.Tensor, stream=None):
@@ -294,6 +322,10 @@ class Cache:
     def device_bytes(self) -> int:
         return int(lib().qvg_cache_device_bytes(self._h))
 
+    def status(self, stream=None) -> int:
+        """qvg_cache_status: read and clear the cache's device status word."""
+        return int(lib().qvg_cache_status(self._h, _stream(stream)))
+
     def dequantize(self, Y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         if Y is None:
             Y = torch.empty((self.H, self.tokens, self.d), dtype=_TORCH[self.dtype], device="cuda")
@@ -310,7 +342,7 @@ class Cache:
         G, T, K = cfg.group_size, cfg.T, cfg.K
         return Packed(codes=_view(v.codes, (H, N, d // 4), torch.uint8),
                       scale=_view(v.scale, (H, N, d // G), torch.uint8),
-                      zero=_view(v.zero, (H, N, d // G), torch.uint8),
+                      zero=_view(v.zero, (H, N, d // G) if cfg.scale_mode == ASYM else (0,), torch.uint8),
                       assign=_view(v.assign, (T, H, N), torch.uint8),
                       centroids=_view(v.centroids, (T, H, K, d), _TORCH[self.dtype]),
                       cfg=cfg, N=N, H=H, d=d, dtype=self.dtype)

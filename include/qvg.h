@@ -23,9 +23,28 @@
  *     on `stream` has finished.  Only a qvg_cache owns memory.
  *   - Work is queued asynchronously on `stream` (0 = legacy default stream);
  *     a call returns once the work is queued.  Errors found while queueing
- *     (bad arguments, launch failures) are returned; a device-side timeout of
- *     a bounded wait is reported by the next call on the same workspace or
- *     cache as QVG_ERR_DEVICE_TIMEOUT (see qvg_workspace_status).
+ *     (bad arguments, launch failures) are returned.
+ *   - Device-side timeouts: every wait of the tensor-core kernel on another
+ *     of its warps is bounded (2 s); a wait that runs out records
+ *     QVG_ERR_DEVICE_TIMEOUT in the sticky status word of the workspace,
+ *     cache or static reserve the call used, the kernel drains and returns,
+ *     and that call's outputs are invalid.  The next qvg_quantize,
+ *     qvg_append_chunk or qvg_quantize_static on the same workspace, cache or
+ *     reserve returns QVG_ERR_DEVICE_TIMEOUT without queueing anything, when
+ *     the earlier work has completed by the time of the call (the check never
+ *     waits for the GPU: it reads the word only when the stream is idle and
+ *     not being captured).  qvg_workspace_status, qvg_cache_status and
+ *     qvg_static_status wait for the stream, read the word and clear it.
+ *   - Fault injection for tests (host side; unset in normal use): the
+ *     environment variable QVG_FAULT_INJECT holds a comma-separated list of
+ *       alloc    every device allocation of qvg_cache_create fails
+ *                (QVG_ERR_NO_MEMORY, nothing allocated);
+ *       stream   qvg_quantize, qvg_dequantize and qvg_cache_dequantize report
+ *                QVG_ERR_CUDA after queueing, as a failed launch would (an
+ *                append then leaves the cache unchanged);
+ *       timeout  the first CTA of the tensor-core assignment withholds one
+ *                tile load and its waits give up after 1 ms, so that the
+ *                bounded waits run out and record a device-side timeout.
  *   - Nothing is thrown across the ABI; all entry points are thread-compatible
  *     (distinct workspaces/caches may be used from distinct threads).
  *   - Tensor layouts are row-major.  H is the number of independent blocks
@@ -68,6 +87,23 @@ typedef enum {
 /* Storage dtype of X, of the centroid tables and of the reconstruction. */
 typedef enum { QVG_BF16 = 0, QVG_FP32 = 1 } qvg_dtype;
 
+/* How a group of G residual values is scaled (section 五 of the m.163.com
+ * article: INT2 codes with FP8 E4M3 group scales).
+ *   QVG_SCALE_ASYM  two E4M3 bytes per group, scale s and zero point m:
+ *                   m = E4M3(min), s = E4M3((max - m)/3),
+ *                   q = clamp(rint((r - m)/s), 0, 3); value s*q + m.
+ *   QVG_SCALE_SYM   one E4M3 byte per group (symmetric signed INT2):
+ *                   s = E4M3(max |r|), q = clamp(rint(r/s), -2, 1), stored
+ *                   u = q + 2; value s*(u - 2).  With it the closed-form
+ *                   compression at K = 256 on a 38,000-token block is 6.97x
+ *                   at T = 1, G = 64 (the pages' QVG range 6.94-7.05x,
+ *                   section 六) and 5.03x at T = 4, G = 16 (QVG-Pro,
+ *                   4.97-5.20x); plain rounding at G = 16 gives the 6.40x the
+ *                   pages quote for their round-to-nearest baseline.
+ * In both, divides are IEEE fp32, rint and E4M3 round to nearest even (E4M3
+ * saturates at 448), and q = 0 when s = 0. */
+typedef enum { QVG_SCALE_ASYM = 0, QVG_SCALE_SYM = 1 } qvg_scale_mode;
+
 typedef struct {
     int32_t K;          /* centroids per block and stage (section 七 uses 256, stored as uint8) */
     int32_t T;          /* progressive residual stages (section 四); 0 = plain per-group RTN */
@@ -75,6 +111,7 @@ typedef struct {
     int32_t bits;       /* code width; 2 (INT2) */
     int32_t iters;      /* Lloyd iterations of a cold start (no initial centroids) */
     int32_t warm_iters; /* Lloyd iterations when started from given centroids */
+    int32_t scale_mode; /* qvg_scale_mode */
 } qvg_config;
 
 /* The packed (compressed) form of H blocks of N tokens.  All DEVICE
@@ -83,7 +120,8 @@ typedef struct {
  *                               2*(j%4) of byte j/4 of the token's row
  *   scale     [H][N][d/G]       E4M3 bytes: group step s
  *   zero      [H][N][d/G]       E4M3 bytes: group zero point m (the rounded
- *                               group minimum); value = s*q + m
+ *                               group minimum); value = s*q + m.  Not used
+ *                               (may be NULL) with QVG_SCALE_SYM
  *   assign    [T][H][N]         uint8 centroid index of each token per stage
  *   centroids [T][H][K][d]      centroid tables in the storage dtype
  * With T = 0, assign and centroids are not accessed (may be NULL). */
@@ -101,9 +139,12 @@ QVG_API const char* qvg_status_string(qvg_status s);
 /* Library build string, e.g. "qvg-b200 sm_100a". */
 QVG_API const char* qvg_version(void);
 
-/* Bytes of the packed form: H*N*d*bits/8 + 2*H*N*d/G + T*H*N +
- * T*H*K*d*sizeof(S).  This equals bits-per-element x H*N*d/8 with
- * bits-per-element = bits + 16/G + 8T/d + 8*sizeof(S)*T*K/N.  Returns 0 for
+/* Bytes of the packed form (the storage that section 五 of the m.163.com
+ * article lists: INT2 codes, FP8 E4M3 group scales, uint8 assignment vectors,
+ * and the centroid tables of every stage): H*N*d*bits/8 + z*H*N*d/G + T*H*N +
+ * T*H*K*d*sizeof(S), with z = 2 scale bytes per group (QVG_SCALE_ASYM) or 1
+ * (QVG_SCALE_SYM).  This equals bits-per-element x H*N*d/8 with
+ * bits-per-element = bits + 8z/G + 8T/d + 8*sizeof(S)*T*K/N.  Returns 0 for
  * invalid arguments.  Host-only, no CUDA call. */
 QVG_API size_t qvg_packed_bytes(const qvg_config* cfg, int64_t N, int32_t H, int32_t d,
                         qvg_dtype dtype);
@@ -129,9 +170,8 @@ QVG_API size_t qvg_workspace_bytes(const qvg_config* cfg, int64_t N, int32_t H, 
  *     every non-empty centroid by the mean of its tokens rounded to `dtype`
  *     (an empty one keeps its value).  The stored pi(t) and C(t) are those of
  *     the last iteration.  R(t) = round(R(t-1) - C(t)[pi(t)]).
- *   The last residual is quantised per group g of G channels of a token:
- *     m = E4M3(min), s = E4M3((max - m)/3), q = clamp(rint((r - m)/s), 0, 3),
- *     (q = 0 when s = 0); E4M3 rounds to nearest even and saturates at 448.
+ *   The last residual is quantised per group g of G channels of a token as
+ *     cfg->scale_mode says (qvg_scale_mode above).
  *   workspace: DEVICE scratch of ws_bytes bytes (see qvg_workspace_bytes),
  *     256-byte aligned, not shared with concurrent calls.
  *   Streams: the work is ordered after the work queued on `stream` before
@@ -139,7 +179,8 @@ QVG_API size_t qvg_workspace_bytes(const qvg_config* cfg, int64_t N, int32_t H, 
  *     of blocks fit in the workspace, every other wave runs on a second
  *     stream that the library creates once per device, joined to `stream` by
  *     events (a stream capture of `stream` captures both).
- * Errors: INVALID_ARG for NULL pointers, K < 1 or K > 256, T < 0, bits != 2,
+ * Errors: INVALID_ARG for NULL pointers (zero may be NULL with
+ * QVG_SCALE_SYM), scale_mode not a qvg_scale_mode, K < 1 or K > 256, T < 0, bits != 2,
  * G not dividing d or not a multiple of 4, N < 1, H < 1, N < K on a cold
  * start with T > 0, iters < 1 (or warm_iters < 1 when warm) with T > 0;
  * UNSUPPORTED for d != 128, G outside {8,16,32,64,128}, T > 8, N >= 2^23;
@@ -150,8 +191,12 @@ QVG_API qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype 
                         qvg_stream_t stream);
 
 /* Reconstruct Y[H][N][d] (DEVICE, `dtype`, 16-byte aligned) from `packed`
- * (codes and centroids 16-byte aligned) in one fused kernel:
- * y = s*q + m, then + C(T)[pi_T], + C(T-1)[pi_(T-1)], ..., + C(1)[pi_1], each
+ * (codes and centroids 16-byte aligned) in one fused kernel (the reverse-order
+ * reconstruction of the m.163.com article, sections 四 and 五: dequantise the
+ * final residual, then add back the centroid of every stage, last stage
+ * first; "Fused Kernel" in gist.science/de, Technische Zusammenfassung 2C):
+ * y = s*q + m (s*(u - 2) with QVG_SCALE_SYM), then + C(T)[pi_T],
+ * + C(T-1)[pi_(T-1)], ..., + C(1)[pi_1], each
  * an fp32 add in that order, then one rounding to `dtype`.  Assignment
  * values >= K are clamped to K-1.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
 QVG_API qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packed, qvg_dtype dtype,
@@ -159,8 +204,8 @@ QVG_API qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packe
 
 /* Status word of a workspace after the work queued on it has completed
  * (synchronises `stream`): QVG_OK, or QVG_ERR_DEVICE_TIMEOUT if a bounded
- * device-side wait in a kernel gave up (its outputs are then invalid).
- * Clears the word. */
+ * device-side wait in a kernel gave up (the outputs of that call are then
+ * invalid).  Clears the word, after which calls on the workspace proceed. */
 QVG_API qvg_status qvg_workspace_status(void* workspace, size_t ws_bytes, qvg_stream_t stream);
 
 /* Tokens whose tensor-core assignment was a near-tie and was decided by
@@ -179,9 +224,12 @@ QVG_API int64_t qvg_workspace_flagged(void* workspace, size_t ws_bytes, qvg_stre
  * device, whose address is looked up on the first call on each device.
  * That first call may load the library's device code, so make it before
  * any stream capture begins.
+ * The reserve's device address is looked up once per device and kept for
+ * the life of the process; after a cudaDeviceReset of a device this entry
+ * must not be called on that device again.
  * Arguments, layouts, results and errors are those of qvg_quantize, less
- * the workspace; each call first zeroes the reserve's 16-byte status word
- * and near-tie counter (on `stream`), then queues the same kernels.
+ * the workspace; the same kernels are queued, one wave at a time on
+ * `stream`.
  * Limits: the reserve must hold one block's working set, about 120,000
  * tokens per block at bf16 with K = 256, T = 2 (qvg_workspace_bytes with
  * H = 1 gives the exact need); a larger block returns WORKSPACE_TOO_SMALL
@@ -191,11 +239,18 @@ QVG_API int64_t qvg_workspace_flagged(void* workspace, size_t ws_bytes, qvg_stre
  * whose work can overlap on the device (different streams, or threads
  * without ordering between them) race and corrupt each other's results;
  * order them on one stream, or use qvg_quantize with separate workspaces.
- * A device-side timeout of this path is recorded in the reserve only; it is
- * not reported to the caller. */
+ * A device-side timeout is recorded in the reserve's status word, returned
+ * by the next call (as for a workspace, see the conventions above) and read
+ * and cleared by qvg_static_status. */
 QVG_API qvg_status qvg_quantize_static(const qvg_config* cfg, const void* X, qvg_dtype dtype,
                                int64_t N, int32_t H, int32_t d, const void* init_centroids,
                                const qvg_packed* out, qvg_stream_t stream);
+
+/* Status word of the current device's static reserve after the work queued
+ * on `stream` has completed (synchronises `stream`): QVG_OK, or
+ * QVG_ERR_DEVICE_TIMEOUT if a bounded wait of a qvg_quantize_static call gave
+ * up.  Clears the word.  No counterpart in the method (as qvg_quantize_static). */
+QVG_API qvg_status qvg_static_status(qvg_stream_t stream);
 
 /* ------------------------------------------------------------------ */
 /* Diagnostics (no counterpart in the method; used by the benchmark).    */
@@ -226,17 +281,30 @@ QVG_API int qvg_profile_report(char* buf, size_t buf_bytes);
 typedef struct qvg_cache qvg_cache;
 
 /* Allocate a cache for up to max_tokens tokens per head in up to max_chunks
- * chunks (device memory on the current device).  Errors: INVALID_ARG,
- * UNSUPPORTED, NO_MEMORY. */
+ * chunks of at most max_chunk_tokens tokens each (0 = max_tokens): the
+ * packed storage, the centroid tables of every chunk, and the k-means
+ * workspace of the largest chunk, all device memory on the current device
+ * (synchronises the device).  Errors: INVALID_ARG (also max_chunk_tokens < K
+ * with T > 0), UNSUPPORTED, NO_MEMORY (nothing is left allocated). */
 QVG_API qvg_status qvg_cache_create(const qvg_config* cfg, qvg_dtype dtype, int32_t H, int32_t d,
-                            int64_t max_tokens, int32_t max_chunks, qvg_cache** out);
+                            int64_t max_tokens, int32_t max_chunks, int64_t max_chunk_tokens,
+                            qvg_cache** out);
 
 /* Compress and append one chunk X_chunk[H][N_chunk][d] (DEVICE, cache dtype).
  * Chunk 0 runs a cold start (needs N_chunk >= K when T > 0) with cfg->iters;
- * later chunks warm-start with cfg->warm_iters.  Errors: INVALID_ARG,
- * CAPACITY, CUDA, NO_MEMORY. */
+ * later chunks warm-start with cfg->warm_iters.  Allocates nothing and does
+ * not wait for the GPU: the workspace was sized at qvg_cache_create.  On an
+ * error the cache is unchanged.  Errors: INVALID_ARG, CAPACITY (more tokens
+ * or chunks than the cache holds, or N_chunk > max_chunk_tokens), CUDA,
+ * DEVICE_TIMEOUT (see the conventions above; qvg_cache_status clears it). */
 QVG_API qvg_status qvg_append_chunk(qvg_cache* cache, const void* X_chunk, int64_t N_chunk,
                             qvg_stream_t stream);
+
+/* Status word of the cache's workspace after the work queued on `stream`
+ * has completed (synchronises `stream`): QVG_OK, or QVG_ERR_DEVICE_TIMEOUT if
+ * a bounded device-side wait of an append gave up (that chunk's packed data
+ * is then invalid).  Clears the word. */
+QVG_API qvg_status qvg_cache_status(qvg_cache* cache, qvg_stream_t stream);
 
 /* Reconstruct the whole cache into Y[H][tokens][d] (DEVICE, cache dtype), one
  * fused launch over every (chunk, head) block. */

@@ -45,36 +45,21 @@ def e4m3_values(b: np.ndarray) -> np.ndarray:
 
 
 def compare_quantize(ora, X_np, gpu: dict, ref: dict, K, T, G, iters, dtype, init=None):
-    """Compare GPU quantisation with the oracle's.  Returns a report dict."""
-    H, N, d = X_np.shape
+    """Compare GPU quantisation with the oracle's: the agreement of every
+    packed array, then the contract of this implementation, which takes every
+    decision the oracle's way (assignments in fp64, exact centroid sums,
+    bit-exact E4M3 and rounding): the packed streams are identical.  The
+    spec tolerance (>= 99.9 % agreement, disagreements only at
+    near-ties) is looser than this, so a pass here implies it."""
+    d = X_np.shape[-1]
     rep = {}
-    exact = all(np.array_equal(gpu[k], ref[k]) for k in ("codes", "scale", "zero", "assign", "centroids"))
-    rep["bit_exact"] = exact
-    qa = unpack_codes(gpu["codes"], d)
-    qb = unpack_codes(ref["codes"], d)
-    rep["codes_agree"] = float((qa == qb).mean())
+    rep["bit_exact"] = all(np.array_equal(gpu[k], ref[k]) for k in ("codes", "scale", "zero", "assign", "centroids"))
+    rep["codes_agree"] = float((unpack_codes(gpu["codes"], d) == unpack_codes(ref["codes"], d)).mean())
     rep["scale_agree"] = float((gpu["scale"] == ref["scale"]).mean())
     rep["zero_agree"] = float((gpu["zero"] == ref["zero"]).mean())
     rep["assign_agree"] = [float((gpu["assign"][t] == ref["assign"][t]).mean()) for t in range(T)]
-    if exact:
-        return rep
-    assert rep["codes_agree"] >= 0.999, rep
-    for t in range(T):
-        assert rep["assign_agree"][t] >= 0.999, rep
-    # Stage-1 disagreements must sit at near-ties of the last iteration's
-    # assignment (oracle fp64 distance gap below 1e-5 relative).
-    if T > 0:
-        for h in range(H):
-            bad = np.nonzero(gpu["assign"][0, h] != ref["assign"][0, h])[0]
-            if len(bad) == 0:
-                continue
-            x = values(X_np[h]).astype(np.float32)
-            C0 = values(init[0, h]).astype(np.float32) if init is not None else x[:K]
-            Cp, _ = ora.kmeans(x, C0, iters - 1, dtype=dtype) if iters > 1 else (C0, None)
-            for i in bad:
-                Dg = ora.sqdist(x[i], Cp[gpu["assign"][0, h, i]])
-                Dr = ora.sqdist(x[i], Cp[ref["assign"][0, h, i]])
-                assert Dg - Dr <= 1e-5 * max(Dr, 1e-300), (h, i, Dg, Dr)
+    rep["centroids_agree"] = [float((gpu["centroids"][t] == ref["centroids"][t]).mean()) for t in range(T)]
+    assert rep["bit_exact"], rep
     return rep
 
 

@@ -47,9 +47,20 @@ def test_version_and_status_strings(q):
     (16, 1, 16, 512, 1, 1), (256, 2, 64, 4680, 12, 0), (256, 2, 64, 38000, 32, 0),
     (64, 4, 32, 38000, 32, 0), (256, 0, 64, 100, 3, 0), (7, 3, 8, 1000, 5, 1),
 ])
-def test_packed_bytes_matches_oracle_closed_form(q, ora, K, T, G, N, H, dtype):
-    cfg = q.config(K=K, T=T, group_size=G)
-    assert q.packed_bytes(cfg, N, H, 128, dtype) == ora.packed_bytes(K, T, G, N, H, 128, dtype=dtype)
+@pytest.mark.parametrize("mode", [0, 1])
+def test_packed_bytes_matches_oracle_closed_form(q, ora, K, T, G, N, H, dtype, mode):
+    cfg = q.config(K=K, T=T, group_size=G, scale_mode=mode)
+    assert q.packed_bytes(cfg, N, H, 128, dtype) == ora.packed_bytes(K, T, G, N, H, 128, dtype=dtype,
+                                                                     scale_mode=mode)
+
+
+def test_presets_are_the_closed_form_operating_points(q, ora):
+    """The named points land in the pages' ranges by the library's own size."""
+    for name, lo, hi in (("qvg", 6.94, 7.05), ("qvg-pro", 4.97, 5.20)):
+        cfg = q.preset(name)
+        ratio = 38000 * 128 * 2 / q.packed_bytes(cfg, 38000, 1)
+        assert lo <= ratio <= hi, (name, ratio)
+    assert q.packed_bytes(q.config(scale_mode=2), 100, 1) == 0
 
 
 def test_workspace_bytes_positive_and_monotone(q):
@@ -69,7 +80,7 @@ def _quantize_status(q, cfg, N=512, H=1, d=128, dtype=0, init=None, X=0x1000, ws
 @pytest.mark.parametrize("kw,expect", [
     (dict(K=0), 1), (dict(K=257), 1), (dict(T=-1), 1), (dict(bits=3), 1),
     (dict(group_size=6), 1), (dict(group_size=48), 1), (dict(iters=0), 1),
-    (dict(group_size=4), 2), (dict(T=9), 2),
+    (dict(group_size=4), 2), (dict(T=9), 2), (dict(scale_mode=2), 1), (dict(scale_mode=-1), 1),
 ])
 def test_quantize_rejects_bad_config_without_touching_the_gpu(q, kw, expect):
     args = dict(K=16, T=1, group_size=16, iters=4)
@@ -98,8 +109,11 @@ def test_dequantize_and_cache_reject_bad_arguments(q):
     assert L.qvg_dequantize(C.byref(cfg), None, 0, 10, 1, 128, 0x1000, None) == 1
     assert L.qvg_dequantize(C.byref(q.config(K=300)), C.byref(p), 0, 10, 1, 128, 0x1000, None) == 1
     h = C.c_void_p()
-    assert L.qvg_cache_create(C.byref(cfg), 0, 1, 128, 0, 4, C.byref(h)) == 1
-    assert L.qvg_cache_create(C.byref(cfg), 0, 1, 96, 100, 4, C.byref(h)) == 2
+    assert L.qvg_cache_create(C.byref(cfg), 0, 1, 128, 0, 4, 0, C.byref(h)) == 1
+    assert L.qvg_cache_create(C.byref(cfg), 0, 1, 96, 100, 4, 0, C.byref(h)) == 2
+    assert L.qvg_cache_create(C.byref(cfg), 0, 1, 128, 100, 4, -1, C.byref(h)) == 1
+    assert L.qvg_cache_create(C.byref(cfg), 0, 1, 128, 100, 4, 8, C.byref(h)) == 1    # a chunk below K
+    assert not h.value
     assert L.qvg_append_chunk(None, 0x1000, 10, None) == 1
     assert L.qvg_cache_tokens(None) == 0 and L.qvg_cache_chunks(None) == 0
 
@@ -119,3 +133,30 @@ def test_workspace_covers_two_waves_when_blocks_exceed_one(q, monkeypatch):
     assert all(sizes[H] == 2 * sizes[W] for H in range(W + 1, 400))
     monkeypatch.setenv("QVG_WAVE_LANES", "1")
     assert q.workspace_bytes(cfg, N, W + 1) == sizes[W]
+
+
+def test_fault_injection_follows_argument_checks(q, monkeypatch):
+    """QVG_FAULT_INJECT=alloc makes qvg_cache_create report NO_MEMORY before
+    any device allocation and leave no handle; arguments are checked first, so
+    an invalid call still reports INVALID_ARG.  The binding raises QvgError
+    with the status."""
+    cfg = q.config(K=16, T=1, group_size=16, iters=4, warm_iters=2)
+    L = q.lib()
+    h = C.c_void_p()
+    monkeypatch.setenv("QVG_FAULT_INJECT", "stream,alloc")
+    assert L.qvg_cache_create(C.byref(cfg), 0, 2, 128, 1000, 4, 0, C.byref(h)) == 3
+    assert not h.value
+    assert L.qvg_cache_create(C.byref(cfg), 0, 2, 128, 0, 4, 0, C.byref(h)) == 1
+    with pytest.raises(q.QvgError) as e:
+        q.Cache(cfg, H=2, max_tokens=1000, max_chunks=4)
+    assert e.value.status == 3 and "NO_MEMORY" in str(e.value)
+    # a name that is not in the list injects nothing: arguments are still checked
+    monkeypatch.setenv("QVG_FAULT_INJECT", "allocate")
+    assert L.qvg_cache_create(C.byref(cfg), 0, 2, 128, 1000, 0, 0, C.byref(h)) == 1
+    assert q.status_string(5) == "device-side wait timed out"
+
+
+def test_status_queries_reject_missing_objects(q):
+    L = q.lib()
+    assert L.qvg_cache_status(None, None) == 1
+    assert L.qvg_workspace_status(None, 0, None) == 1

@@ -67,3 +67,16 @@ def test_head_shards_partition_every_cache():
             assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
     # whole-job rate: the one cache's bytes over the slowest rank's time
     assert bench.strong_scaling_value(2e9, 1000.0) == 2.0
+
+
+def test_share_blocks_cover_the_cache_once():
+    """The ranks' block lists, in the cache's layer-major K-then-V order,
+    partition every block of the cache exactly once."""
+    from bit_kv_cache_qvg_b200.shard import share_blocks
+    for L, H in ((1, 1), (3, 7), (2, 32)):
+        for world in (1, 2, 3, min(H, 5)):
+            parts = [share_blocks(L, H, world, r) for r in range(world)]
+            flat = sorted(b for p in parts for b in p)
+            assert flat == list(range(L * 2 * H))
+            for p in parts:                       # each share keeps the cache's order
+                assert p == sorted(p)
