@@ -70,6 +70,10 @@ def lib():
         L.ref_quantize.argtypes = [i32, i32, i32, i32, i32, i32, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]
         L.ref_dequantize.restype = i32
         L.ref_dequantize.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, i32, i32, vp]
+        L.ref_rope.argtypes = [vp, i64, i32, vp, f64, vp]
+        L.ref_rope.restype = None
+        L.ref_attention.restype = i32
+        L.ref_attention.argtypes = [vp, vp, i64, vp, vp, i64, i32, f64, vp]
         L.ref_kv_cache_bytes.restype = f64
         L.ref_kv_cache_bytes.argtypes = [i64, i64, i64, i64]
         L.ref_bits_per_element.restype = f64
@@ -250,3 +254,27 @@ def bits_per_element(K, T, G, N, d, bits=2, dtype=BF16, scale_mode=0) -> float:
 
 def packed_bytes(K, T, G, N, H, d, bits=2, dtype=BF16, scale_mode=0) -> int:
     return int(lib().ref_packed_bytes(K, T, G, bits, N, H, d, dtype, scale_mode))
+
+
+# ---------------------------------------------------------------- attention
+def rope(x, pos, base=10000.0) -> np.ndarray:
+    """Rotary embedding (fp64) of x [n][d] at positions pos [n]."""
+    x = _f32(x)
+    n, d = x.shape
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    out = np.empty((n, d), np.float64)
+    lib().ref_rope(_p(x), n, d, _p(pos), float(base), _p(out))
+    return out
+
+
+def attention(Q, qpos, K, V, base=10000.0) -> np.ndarray:
+    """softmax(rope(Q) rope(K)^T / sqrt(d)) V for one head (fp64); keys at
+    positions 0 .. len(K)-1."""
+    Q, K, V = _f32(Q), _f32(K), _f32(V)
+    nq, d = Q.shape
+    nk = K.shape[0]
+    qpos = np.ascontiguousarray(qpos, dtype=np.int64)
+    O = np.empty((nq, d), np.float64)
+    if lib().ref_attention(_p(Q), _p(qpos), nq, _p(K), _p(V), nk, d, float(base), _p(O)) != 0:
+        raise ValueError("oracle attention rejected its arguments")
+    return O

@@ -637,3 +637,76 @@ int64_t ref_packed_bytes(int K, int T, int G, int bits, int64_t N, int H, int d,
     int64_t cents = (int64_t)T * H * K * d * esz;
     return codes + scales + assign + cents;
 }
+
+/* ------------------------------------------------------------------ */
+/* Attention over the reconstructed cache ([163] 五: keys are cached     */
+/* before the rotary position embedding, which is applied after         */
+/* dequantisation; the fused kernel feeds the reconstruction to          */
+/* attention without writing it out; [de] 2C "Fused Kernel").            */
+/* READINGS (the pages give no formula for either step):                */
+/*   rotary embedding in the RoFormer form: channel pair (2i, 2i+1) of a  */
+/*   token at position p is rotated by the angle p * base^(-2i/d);       */
+/*   softmax attention with scale 1/sqrt(d) and no mask: every query     */
+/*   sees every cached token.                                            */
+/* Everything in fp64, exact positions; cos and sin from libm.          */
+/* ------------------------------------------------------------------ */
+
+/* out[n][d] = rotary embedding of x[n][d] (token i at position pos[i]). */
+void ref_rope(const float* x, int64_t n, int d, const int64_t* pos, double base, double* out)
+{
+    int64_t t;
+    int i;
+    for (t = 0; t < n; ++t) {
+        for (i = 0; i < d / 2; ++i) {
+            const double theta = pow(base, -2.0 * i / (double)d);
+            const double a = (double)pos[t] * theta;
+            const double c = cos(a), s = sin(a);
+            const double x0 = x[t * d + 2 * i], x1 = x[t * d + 2 * i + 1];
+            out[t * d + 2 * i] = x0 * c - x1 * s;
+            out[t * d + 2 * i + 1] = x0 * s + x1 * c;
+        }
+    }
+}
+
+/* O[nq][d] = softmax(rope(Q) rope(K)^T / sqrt(d)) V for one head, with Q at
+ * positions qpos and the cached keys at positions 0 .. nk-1 (cache order).
+ * K and V are the reconstructed cache (the dequantised values).  Returns 0,
+ * or -1 for invalid sizes. */
+int ref_attention(const float* Q, const int64_t* qpos, int64_t nq, const float* K, const float* V,
+                  int64_t nk, int d, double base, double* O)
+{
+    double *qr, *kr, *s;
+    int64_t* kpos;
+    int64_t i, j;
+    int c;
+    if (nq < 1 || nk < 1 || d < 2 || d % 2) return -1;
+    qr = (double*)malloc((size_t)(nq * d) * sizeof(double));
+    kr = (double*)malloc((size_t)(nk * d) * sizeof(double));
+    kpos = (int64_t*)malloc((size_t)nk * sizeof(int64_t));
+    for (j = 0; j < nk; ++j) kpos[j] = j;
+    ref_rope(Q, nq, d, qpos, base, qr);
+    ref_rope(K, nk, d, kpos, base, kr);
+#pragma omp parallel for schedule(static) private(j, c, s)
+    for (i = 0; i < nq; ++i) {
+        double m = -INFINITY, l = 0.0;
+        s = (double*)malloc((size_t)nk * sizeof(double));
+        for (j = 0; j < nk; ++j) {
+            double dot = 0.0;
+            for (c = 0; c < d; ++c) dot += qr[i * d + c] * kr[j * d + c];
+            s[j] = dot / sqrt((double)d);
+            if (s[j] > m) m = s[j];
+        }
+        for (c = 0; c < d; ++c) O[i * d + c] = 0.0;
+        for (j = 0; j < nk; ++j) {
+            const double p = exp(s[j] - m);
+            l += p;
+            for (c = 0; c < d; ++c) O[i * d + c] += p * (double)V[j * d + c];
+        }
+        for (c = 0; c < d; ++c) O[i * d + c] /= l;
+        free(s);
+    }
+    free(qr);
+    free(kr);
+    free(kpos);
+    return 0;
+}
