@@ -462,8 +462,13 @@ def main():
     top = max(roof, key=lambda n: kernels[n]["ms"]) if roof else None
     dominant = dict(roof[top], kernel=top) if top else None
 
-    # quantise-path roofline: max(F / P_bf16, B / BW)
+    # quantise-path roofline: max(F / P_bf16, B / BW).  Its time is taken two
+    # ways: the device-timed step minus the dequant (which runs last in the
+    # step, so the rest is the quantise path as it runs, two waves in flight),
+    # and the sum of its kernels' event times with the waves one at a time.
     q_ms = sum(v["ms"] for n, v in kernels.items() if n != "qvg_dequant_fused")
+    dq_ms = kernels.get("qvg_dequant_fused", {}).get("ms", 0.0)
+    q_dev_ms = ms - dq_ms
     F = 2.0 * K * I * T * E
     B = E * 2 + packed.nbytes()
     q_roof_ms = max(F / (peaks["bf16_sus"] * 1e12), B / (peaks["hbm"] * 1e9)) * 1e3
@@ -480,7 +485,12 @@ def main():
                                    if strong else f"weak: {world} rank(s), independent caches")},
         "roofline": dominant,
         "rooflines": roof,
-        "quantize_path": {"ms_per_step": q_ms, "roofline_ms": q_roof_ms, "frac": q_roof_ms / q_ms if q_ms else None,
+        "quantize_path": {"ms_per_step": q_dev_ms, "roofline_ms": q_roof_ms,
+                          "frac": q_roof_ms / q_dev_ms if q_dev_ms > 0 else None,
+                          "time_is": "device-timed step minus the dequant's event time",
+                          "kernel_sum_ms": q_ms, "frac_kernel_sum": q_roof_ms / q_ms if q_ms else None,
+                          "bound": "tensor (sustained bf16)" if F / (peaks["bf16_sus"] * 1e12) > B / (peaks["hbm"] * 1e9)
+                          else "hbm",
                           "peak_source": peaks["source"]},
         "kernels": kernels,
         "gpu_launches": launches,
@@ -515,22 +525,27 @@ def stream_chunks(wl):
     return [min(cf, F - f) * hw for f in range(0, F, cf)]
 
 
-def dequant_alg_bytes(U, n, chunks, K, T, G, esz=2):
+def dequant_alg_bytes(U, n, chunks, K, T, G, esz=2, scale_bytes=2):
     """Algorithmic bytes of one fused dequant of U blocks of n tokens spread
-    over `chunks` chunks: codes + E4M3 scale/zero + assignments read, output
-    written, and every chunk's T centroid tables read once."""
-    return U * n * 128 * (2 / 8 + 2 / G + T / 128 + esz) + chunks * T * U * K * 128 * esz
+    over `chunks` chunks: codes + E4M3 scale (and zero) + assignments read,
+    output written, and every chunk's T centroid tables read once."""
+    return U * n * 128 * (2 / 8 + scale_bytes / G + T / 128 + esz) + chunks * T * U * K * 128 * esz
 
 
-def bits_per_element(K, T, G, N, d=128, bits=2, esz=2):
-    """Closed form of the packed size per element: the code, the two E4M3
-    bytes of each group, T uint8 assignments per token and T centroid tables
-    of K x d values per block."""
-    return bits + 16.0 / G + 8.0 * T / d + 8.0 * esz * T * K / N
+def bits_per_element(K, T, G, N, d=128, bits=2, esz=2, scale_bytes=2):
+    """Closed form of the packed size per element: the code, the E4M3 bytes of
+    each group (scale and zero point, or one scale), T uint8 assignments per
+    token and T centroid tables of K x d values per block."""
+    return bits + 8.0 * scale_bytes / G + 8.0 * T / d + 8.0 * esz * T * K / N
 
 
-def compression_ratio(K, T, G, N, d=128, bits=2, esz=2):
-    return 8.0 * esz / bits_per_element(K, T, G, N, d, bits, esz)
+def compression_ratio(K, T, G, N, d=128, bits=2, esz=2, scale_bytes=2):
+    return 8.0 * esz / bits_per_element(K, T, G, N, d, bits, esz, scale_bytes)
+
+
+# The pages' compression figures (m.163.com article on Quant VideoGen, section
+# 六): QVG 6.94-7.05x, QVG-Pro 4.97-5.20x, plain rounding 6.40x.
+PAGE_RATIOS = {"qvg": (6.94, 7.05), "qvg-pro": (4.97, 5.20), "rtn": (6.40, 6.40)}
 
 
 def run_sweep(args, wl, qvg, synth, dev, dist, rank, world, peaks):
@@ -555,10 +570,16 @@ def run_sweep(args, wl, qvg, synth, dev, dist, rank, world, peaks):
         return num / sum(xx[lo:hi])
 
     points = []
-    grid = [(0, G, 0) for G in (16, 32, 64)] + [(T, G, K) for T in (1, 2, 3, 4) for G in (16, 32, 64)
-                                               for K in (64, 256)]
-    for T, G, K in grid:
-        cfg = qvg.config(K=max(K, 1), T=T, group_size=G, iters=wl["iters"])
+    # scale and zero point per group (mode 0) over the whole grid; one scale
+    # per group (mode 1) at plain rounding and at every K = 256 point, which
+    # holds the named QVG (T=1, G=64) and QVG-Pro (T=4, G=16) settings
+    grid = [(0, G, 0, 0) for G in (16, 32, 64)] + [(T, G, K, 0) for T in (1, 2, 3, 4) for G in (16, 32, 64)
+                                                  for K in (64, 256)]
+    grid += [(0, G, 0, 1) for G in (16, 32, 64)] + [(T, G, 256, 1) for T in (1, 2, 3, 4) for G in (16, 32, 64)]
+    named = {(qvg.PRESETS[n]["T"], qvg.PRESETS[n]["group_size"], qvg.PRESETS[n]["K"], 1): n for n in qvg.PRESETS}
+    named[(0, 16, 0, 1)] = "rtn"
+    for T, G, K, mode in grid:
+        cfg = qvg.config(K=max(K, 1), T=T, group_size=G, iters=wl["iters"], scale_mode=mode)
         packed = qvg.alloc_packed(cfg, N, U, device=dev)
         ws = qvg.alloc_workspace(cfg, N, U, device=dev)
         with torch.cuda.stream(stream):
@@ -581,14 +602,22 @@ def run_sweep(args, wl, qvg, synth, dev, dist, rank, world, peaks):
             raise SystemExit("device-side wait timed out in the sweep")
         nbytes = packed.nbytes()
         ratio = kv_bytes / nbytes
-        closed = compression_ratio(K, T, G, N)
-        points.append({"T": T, "G": G, "K": K if T else None, "rel_mse_K": rel_err(0, Hh), "rel_mse_V": rel_err(Hh, U),
-                       "packed_bytes": nbytes, "compression": ratio, "compression_closed_form": closed,
-                       "closed_form_matches": abs(ratio - closed) < 1e-9 * closed,
-                       "quantize_ms": tq, "quantize_GBps": kv_bytes / (tq / 1e3) / 1e9,
-                       "dequant_ms": td, "dequant_GBps": dequant_alg_bytes(U, N, 1, K, T, G) / (td / 1e3) / 1e9})
+        sb = 1 if mode == 1 else 2
+        closed = compression_ratio(K, T, G, N, scale_bytes=sb)
+        pt = {"T": T, "G": G, "K": K if T else None, "scale_bytes_per_group": sb,
+              "rel_mse_K": rel_err(0, Hh), "rel_mse_V": rel_err(Hh, U),
+              "packed_bytes": nbytes, "compression": ratio, "compression_closed_form": closed,
+              "closed_form_matches": abs(ratio - closed) < 1e-9 * closed,
+              "quantize_ms": tq, "quantize_GBps": kv_bytes / (tq / 1e3) / 1e9,
+              "dequant_ms": td, "dequant_GBps": dequant_alg_bytes(U, N, 1, K, T, G, scale_bytes=sb) / (td / 1e3) / 1e9}
+        if (T, G, K, mode) in named:
+            n = named[(T, G, K, mode)]
+            pt["named"] = n
+            pt["page_ratio_range"] = PAGE_RATIOS[n]
+        points.append(pt)
         del packed, ws
-    head = next(p for p in points if (p["T"], p["G"], p["K"]) == (wl["T"], wl["G"], wl["K"]))
+    head = next(p for p in points if (p["T"], p["G"], p["K"], p["scale_bytes_per_group"]) ==
+                (wl["T"], wl["G"], wl["K"], 2))
     result = {
         "metric": SWEEP_METRIC,
         "value": head["quantize_GBps"], "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": 1,

@@ -1,0 +1,501 @@
+// kernel_attention.cu -- qvg_attention: softmax attention of a block of
+// queries over a compressed K/V cache, with the reconstruction fused into
+// the attention's K/V load (the consumer of the m.163.com article on Quant
+// VideoGen, section 五: the key cache is kept before the rotary embedding,
+// which is applied after dequantisation, and the fused kernel keeps the
+// reconstructed values on chip instead of writing them out; gist.science/de,
+// Technische Zusammenfassung 2C, "Fused Kernel").
+//
+//   O = softmax(rope(Q) rope(K^)^T / sqrt(d)) V^
+//
+// where K^ and V^ are the cache's reconstructions (the values
+// qvg_dequantize writes, bit for bit), rope is the RoFormer rotary embedding
+// (channel pair (2i, 2i+1) of a token at position p turned by
+// p * base^(-2i/d)), the cached tokens sit at positions 0 .. Nk-1 and the
+// queries at the given positions.  No mask.
+//
+// One CTA = one head x 128 queries; it walks the cache in tiles of 128
+// tokens.  Per tile:
+//   1. all 8 warps dequantise the K and V tile (unpack, scale, add every
+//      stage's centroid in reverse order, round to bf16 -- the arithmetic of
+//      qvg_dequant_fused), apply the rotary embedding to K, and store both
+//      straight into shared memory in the tensor core's K-major operand
+//      layout: K rows (keys) with the channels contiguous, V transposed
+//      (channels) with the keys contiguous, each thread an 8 x 8 block;
+//   2. one thread issues S = Q' K'^T (tcgen05.mma kind::f16, M = N = K = 128,
+//      fp32 accumulators in tensor memory);
+//   3. warps 0-3 (one per tensor-memory lane quarter, a thread per query)
+//      read S, keep the running row maximum and sum (online softmax, base-2
+//      exponentials), write P in bf16 into the K buffer (the A operand of the
+//      next product) and rescale the O accumulator in tensor memory;
+//   4. one thread issues O += P V (accumulators in tensor memory).
+// After the last tile O / l is written in fp32.  The rotary angles come from
+// two tables of (cos, sin) in fp32, p = 1024 a + b: (1024 a) theta_i and
+// b theta_i, combined by the angle-sum identity (qvg_rope_tables builds them
+// in fp64).  Every mbarrier wait is bounded; on expiry the kernel records
+// QVG_ERR_DEVICE_TIMEOUT in the status word at the start of the tables
+// buffer and stops.  No TMA and no multicast: the operands are written by the
+// threads that reconstruct them.
+#include <cuda.h>
+
+#include "qvg_common.cuh"
+#include "qvg_launch.h"
+
+namespace qvg {
+namespace {
+
+constexpr int kAtThreads = 256;                 // 8 warps
+constexpr int kAtTile = 128;                    // queries per CTA, cached tokens per tile
+constexpr int kAtOpBytes = kAtTile * kD * 2;    // one 128 x 128 bf16 operand: 32 KB
+constexpr uint64_t kAtWaitNs = 2000000000ull;   // 2 s per bounded wait
+constexpr int kRopeLo = 1024;                   // positions per low-table row block
+
+struct AttnParams {
+  const uint8_t* codes[2];        // K, V: [H][Nk][d/4]
+  const uint8_t* scale[2];        // [H][Nk][d/G]
+  const uint8_t* zero[2];         // [H][Nk][d/G] (asymmetric mode)
+  const uint8_t* assign[2];       // [T][H][Nk]
+  const __nv_bfloat16* tab[2];    // [T][H][K][d]
+  const __nv_bfloat16* Q;         // [H][Nq][d], before the rotary embedding
+  const int64_t* qpos;            // [Nq] query positions
+  const float2* rope_hi;          // [n_hi][d/2]: (cos, sin) of 1024 a theta_i
+  const float2* rope_lo;          // [1024][d/2]: (cos, sin) of b theta_i
+  float* O;                       // [H][Nq][d]
+  uint32_t* status;
+  int64_t max_pos;                // largest position the tables cover
+  int64_t Nk, Nq;
+  int H, K, T, G, sym;
+  float sl;                       // log2(e) / sqrt(d)
+};
+
+struct __align__(8) AtBars {
+  uint64_t s_done;
+  uint64_t o_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_addr(bar);
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((it & 63u) == 0u) {
+      uint64_t now;
+      asm volatile("mov.u64 %0, %globaltimer;" : "=l"(now));
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kAtWaitNs) return false;
+    }
+  }
+}
+
+// Shared-memory operand descriptor, K-major, no swizzle: 8-row x 16-byte core
+// matrices; core matrices adjacent along K are 128 bytes apart (LBO), 8-row
+// groups 2,048 bytes apart (SBO: sixteen core matrices span K = 128).
+__device__ __forceinline__ uint64_t op_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)(128 >> 4) << 16;
+  d |= (uint64_t)(2048 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+// Byte offset of element (row, k) of a 128 x 128 operand in that layout.
+__device__ __forceinline__ int op_off(int row, int k) {
+  return (row >> 3) * 2048 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2;
+}
+
+// kind::f16, A = B = bf16, D = f32, both K-major, M = N = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(128 >> 3) << 17) |
+                            ((uint32_t)(128 >> 4) << 24);
+
+__device__ __forceinline__ void mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  // the registers pass through the wait so that no use moves above it
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+        "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+        "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+        "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+__device__ __forceinline__ void tst32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// (cos, sin) of the rotary angle of pair i at position p from the two tables
+// (positions outside [0, max_pos] are clamped, so the reads stay in bounds).
+__device__ __forceinline__ float2 rope_cs(const AttnParams& p, int64_t pos, int i) {
+  pos = pos < 0 ? 0 : (pos > p.max_pos ? p.max_pos : pos);
+  const float2 a = p.rope_hi[(pos / kRopeLo) * (kD / 2) + i];
+  const float2 b = p.rope_lo[(pos % kRopeLo) * (kD / 2) + i];
+  return make_float2(__fsub_rn(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y)),
+                     __fadd_rn(__fmul_rn(a.y, b.x), __fmul_rn(a.x, b.y)));
+}
+
+// Reconstruct 8 channels (c0 .. c0+7) of token `tok` of cache `which` (0 = K,
+// 1 = V) of head h: y = s*q + m (or s*(u - 2)), plus the centroids of stages
+// T, ..., 1 in that order, each an fp32 add, then one rounding to bf16 --
+// the arithmetic of qvg_dequant_fused.  The results are returned as fp32
+// values of the rounded bf16 numbers.
+__device__ __forceinline__ void recon8(const AttnParams& p, const float* dec, int which, int h, int64_t tok, int c0,
+                                       float (&y)[8]) {
+  const int64_t row = (int64_t)h * p.Nk + tok;
+  const int ng = kD / p.G;
+  const uint16_t code = *reinterpret_cast<const uint16_t*>(p.codes[which] + row * (kD / 4) + c0 / 4);
+  const int g = c0 / p.G;
+  const float s = dec[p.scale[which][row * ng + g]];
+  if (p.sym) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(s, (float)((code >> (2 * e)) & 3u) - 2.0f);
+  } else {
+    const float m = dec[p.zero[which][row * ng + g]];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = __fmaf_rn(s, (float)((code >> (2 * e)) & 3u), m);
+  }
+  for (int t = p.T - 1; t >= 0; --t) {
+    int k = p.assign[which][((int64_t)t * p.H + h) * p.Nk + tok];
+    k = min(k, p.K - 1);
+    const uint4 w = *reinterpret_cast<const uint4*>(p.tab[which] + (((int64_t)t * p.H + h) * p.K + k) * kD + c0);
+    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      y[2 * e] = __fadd_rn(y[2 * e], __uint_as_float(x[e] << 16));
+      y[2 * e + 1] = __fadd_rn(y[2 * e + 1], __uint_as_float(x[e] & 0xFFFF0000u));
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    const uint32_t b = pack_bf16(y[e], y[e + 1]);
+    y[e] = __uint_as_float(b << 16);
+    y[e + 1] = __uint_as_float(b & 0xFFFF0000u);
+  }
+}
+
+__global__ void __launch_bounds__(kAtThreads, 1)
+qvg_attention_fused(const AttnParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;                               // A of S: queries x channels
+  uint8_t* sK = sQ + kAtOpBytes;                    // B of S: keys x channels; then A of O: queries x keys (P)
+  uint8_t* sV = sK + kAtOpBytes;                    // B of O: channels x keys
+  float* dec = reinterpret_cast<float*>(sV + kAtOpBytes);
+  AtBars* bars = reinterpret_cast<AtBars*>(dec + 256);
+
+  const int h = blockIdx.y;
+  const int64_t q0 = (int64_t)blockIdx.x * kAtTile;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the thread's 8 x 8 block of a 128 x 128 tile: rows 8*rb .. 8*rb+7, channels 8*cb .. 8*cb+7
+  const int rb = threadIdx.x >> 4, cb = threadIdx.x & 15;
+
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->s_done)));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->o_done)));
+    bars->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+                     smem_addr(&bars->tmem_base)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  for (int x = threadIdx.x; x < 256; x += blockDim.x) dec[x] = e4m3_to_f32((uint8_t)x);
+
+  // queries: rotary embedding at their positions, bf16, into the A layout
+  for (int r = 0; r < 8; ++r) {
+    const int qi = 8 * rb + r;
+    const int64_t q = q0 + qi;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (q < p.Nq) {
+      const uint4 v = *reinterpret_cast<const uint4*>(p.Q + ((int64_t)h * p.Nq + q) * kD + 8 * cb);
+      const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+      const int64_t pos = p.qpos[q];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a = __uint_as_float(x[e] << 16), b = __uint_as_float(x[e] & 0xFFFF0000u);
+        const float2 cs = rope_cs(p, pos, 4 * cb + e);
+        w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
+                         __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
+      }
+    }
+    *reinterpret_cast<uint4*>(sQ + op_off(qi, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const uint32_t tS = tmem, tO = tmem + 128;
+
+  float m_run = -3.0e38f, l_run = 0.0f;           // softmax state of this thread's query (warps 0-3)
+  const int ntiles = (int)((p.Nk + kAtTile - 1) / kAtTile);
+  bool ok = true;
+  int j_last = 0;                                 // the tile being worked on when a wait gave up
+  for (int j = 0; j < ntiles && ok; ++j) {
+    j_last = j;
+    const int64_t k0 = (int64_t)j * kAtTile;
+    // the previous product O += P V must be done before its operands are overwritten
+    if (j > 0) {
+      ok = bar_wait(&bars->o_done, (uint32_t)((j - 1) & 1));
+      if (!ok) break;
+      fence_after();
+    }
+    // 1. reconstruct the K and V tile into the operand layouts
+    {
+      float vk[8][8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int ti = 8 * rb + r;
+        const int64_t tok = k0 + ti;
+        float y[8];
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        if (tok < p.Nk) {
+          recon8(p, dec, 0, h, tok, 8 * cb, y);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 cs = rope_cs(p, tok, 4 * cb + e);
+            const float a = y[2 * e], b = y[2 * e + 1];
+            w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
+                             __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
+          }
+          recon8(p, dec, 1, h, tok, 8 * cb, vk[r]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) vk[r][e] = 0.0f;
+        }
+        *reinterpret_cast<uint4*>(sK + op_off(ti, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      // V transposed: channel 8*cb + e holds the 8 keys 8*rb .. 8*rb+7 contiguously
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint4 t = make_uint4(pack_bf16(vk[0][e], vk[1][e]), pack_bf16(vk[2][e], vk[3][e]),
+                                   pack_bf16(vk[4][e], vk[5][e]), pack_bf16(vk[6][e], vk[7][e]));
+        *reinterpret_cast<uint4*>(sV + op_off(8 * cb + e, 8 * rb)) = t;
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
+    fence_before();
+    __syncthreads();
+    fence_after();
+    // 2. S = Q' K'^T
+    if (threadIdx.x == 0) {
+      const uint32_t a0 = smem_addr(sQ), b0 = smem_addr(sK);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) mma(tS, op_desc(a0 + 256 * kk), op_desc(b0 + 256 * kk), kk > 0 ? 1u : 0u);
+      mma_commit(&bars->s_done);
+    }
+    // 3. online softmax (warps 0-3: the thread's query is row 32*warp + lane)
+    if (warp < 4) {
+      if (!bar_wait(&bars->s_done, (uint32_t)(j & 1))) {
+        *reinterpret_cast<volatile int*>(&bars->abort_flag) = 1;
+      } else {
+        fence_after();
+        const int qi = 32 * warp + lane;
+        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+        const int valid = (int)(p.Nk - k0 < kAtTile ? p.Nk - k0 : kAtTile);
+        float x[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tld32(tS + lane_base + (uint32_t)(32 * c), r);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[32 * c + e] = 32 * c + e < valid ? __uint_as_float(r[e]) * p.sl : -3.0e38f;
+        }
+        float mt = -3.0e38f;
+#pragma unroll
+        for (int e = 0; e < 128; e += 2) mt = fmaxf(mt, fmaxf(x[e], x[e + 1]));
+        const float m_new = fmaxf(m_run, mt);
+        const float alpha = exp2_approx(m_run - m_new);
+        float sum = 0.0f;
+#pragma unroll
+        for (int kg = 0; kg < 16; ++kg) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float pa = 8 * kg + 2 * e < valid ? exp2_approx(x[8 * kg + 2 * e] - m_new) : 0.0f;
+            const float pb = 8 * kg + 2 * e + 1 < valid ? exp2_approx(x[8 * kg + 2 * e + 1] - m_new) : 0.0f;
+            w[e] = pack_bf16(pa, pb);
+            // the sum takes the rounded weights, the ones the product uses
+            sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
+          }
+          *reinterpret_cast<uint4*>(sK + op_off(qi, 8 * kg)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        l_run = l_run * alpha + sum;
+        m_run = m_new;
+        // rescale O (the previous product is complete: waited for above)
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tld32(tO + lane_base + (uint32_t)(32 * c), r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tst32(tO + lane_base + (uint32_t)(32 * c), r);
+          }
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        }
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    fence_before();
+    __syncthreads();
+    fence_after();
+    if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) { ok = false; break; }
+    // 4. O += P V
+    if (threadIdx.x == 0) {
+      const uint32_t a0 = smem_addr(sK), b0 = smem_addr(sV);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) mma(tO, op_desc(a0 + 256 * kk), op_desc(b0 + 256 * kk), (j > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&bars->o_done);
+    }
+  }
+  // the last product, then O / l
+  if (ok && ntiles > 0) {
+    ok = bar_wait(&bars->o_done, (uint32_t)((ntiles - 1) & 1));
+    fence_after();
+  }
+  if (warp < 4 && ok && ntiles > 0) {
+    const int qi = 32 * warp + lane;
+    const int64_t q = q0 + qi;
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const float inv = 1.0f / l_run;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t r[32];
+      tld32(tO + lane_base + (uint32_t)(32 * c), r);
+      if (q < p.Nq) {
+        float4* dst = reinterpret_cast<float4*>(p.O + ((int64_t)h * p.Nq + q) * kD + 32 * c);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
+                               __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
+      }
+    }
+  }
+  if (!ok && threadIdx.x == 0) {
+    atomicOr(p.status, 1u);
+    // let the products already issued finish (bounded) before the tensor
+    // memory is freed: the last S product of tile j_last and the O product
+    // of the tile before it; a phase that already completed returns at once
+    bar_wait(&bars->s_done, (uint32_t)(j_last & 1));
+    if (j_last > 0) bar_wait(&bars->o_done, (uint32_t)((j_last - 1) & 1));
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem));
+  }
+}
+
+// (cos, sin) tables of the rotary angles in fp64, rounded to fp32:
+// hi[a][i] for the angle 1024 a theta_i, lo[b][i] for b theta_i.
+__global__ void qvg_rope_tables_kernel(float2* hi, float2* lo, int n_hi, double base) {
+  const int i = threadIdx.x % (kD / 2);
+  const int row = blockIdx.x * (blockDim.x / (kD / 2)) + threadIdx.x / (kD / 2);
+  if (row >= n_hi + kRopeLo) return;
+  const double theta = pow(base, -2.0 * i / (double)kD);
+  double a;
+  float2* dst;
+  if (row < n_hi) { a = (double)row * kRopeLo * theta; dst = hi + (int64_t)row * (kD / 2) + i; }
+  else { a = (double)(row - n_hi) * theta; dst = lo + (int64_t)(row - n_hi) * (kD / 2) + i; }
+  double s, c;
+  sincos(a, &s, &c);
+  *dst = make_float2(__double2float_rn(c), __double2float_rn(s));
+}
+
+}  // namespace
+
+size_t attention_smem_bytes() { return 1024 + 3 * (size_t)kAtOpBytes + 256 * sizeof(float) + sizeof(AtBars); }
+
+cudaError_t launch_rope_tables(void* tables, int n_hi, double base, cudaStream_t s) {
+  float2* hi = reinterpret_cast<float2*>(static_cast<char*>(tables) + kRopeHeaderBytes);
+  float2* lo = hi + (size_t)n_hi * (kD / 2);
+  const int rows = n_hi + kRopeLo;
+  const int per = 256 / (kD / 2);
+  qvg_rope_tables_kernel<<<(rows + per - 1) / per, 256, 0, s>>>(hi, lo, n_hi, base);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s) {
+  AttnParams p{};
+  for (int w = 0; w < 2; ++w) {
+    const qvg_packed* pk = w == 0 ? a.k : a.v;
+    p.codes[w] = pk->codes; p.scale[w] = pk->scale; p.zero[w] = pk->zero; p.assign[w] = pk->assign;
+    p.tab[w] = static_cast<const __nv_bfloat16*>(pk->centroids);
+  }
+  p.Q = static_cast<const __nv_bfloat16*>(a.Q);
+  p.qpos = a.qpos;
+  p.rope_hi = reinterpret_cast<const float2*>(static_cast<const char*>(a.tables) + kRopeHeaderBytes);
+  p.rope_lo = p.rope_hi + (size_t)a.n_hi * (kD / 2);
+  p.O = a.O;
+  p.status = reinterpret_cast<uint32_t*>(const_cast<void*>(a.tables));
+  p.max_pos = (int64_t)a.n_hi * kRopeLo - 1;
+  p.Nk = a.Nk; p.Nq = a.Nq; p.H = a.H; p.K = a.K; p.T = a.T; p.G = a.G; p.sym = a.sym;
+  p.sl = 1.4426950408889634f / sqrtf((float)kD);
+  const size_t smem = attention_smem_bytes();
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(qvg_attention_fused), smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((a.Nq + kAtTile - 1) / kAtTile), (unsigned)a.H);
+  qvg_attention_fused<<<grid, kAtThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace qvg

@@ -71,6 +71,24 @@ template <> struct Vec8<kFP32> {
 };
 
 // ---------------------------------------------------------------- packed pairs
+// Two values as a bf16 pair word (low half first), each cut to its 16 high
+// bits: exact for values that are already bf16.  For fp32 values (STICKY) the
+// cut keeps the exponent, and the lowest kept bit is set when a cut bit was
+// set, so a nonzero value never becomes zero (the channel-range checks need
+// the exponents only).
+template <bool STICKY>
+__device__ __forceinline__ uint32_t bf16_pair_bits(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+  uint32_t w = __byte_perm(a, b, 0x7632);
+  if (STICKY) w |= ((a & 0xFFFFu) != 0u ? 1u : 0u) | ((b & 0xFFFFu) != 0u ? 0x10000u : 0u);
+  return w;
+}
+// Lane-wise bf16 maximum; a NaN lane yields the other operand.
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
 // Two fp32 values operated on with the f32x2 instructions (float2 intrinsics:
 // each lane of the pair is rounded as a separate IEEE fp32 operation).
 __device__ __forceinline__ float2 f2(float lo, float hi) { return make_float2(lo, hi); }
@@ -163,7 +181,10 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
   float2* nlut = reinterpret_cast<float2*>(dec + 256);                          // nibble -> two codes
   if (i_end <= i_begin) return;                                                 // uniform over the block
   for (int x = threadIdx.x; x < 256; x += blockDim.x) dec[x] = e4m3_to_f32((uint8_t)x);
-  if (threadIdx.x < 16) nlut[threadIdx.x] = make_float2((float)(threadIdx.x & 3u), (float)(threadIdx.x >> 2));
+  // the symmetric mode reads the codes as u - 2
+  if (threadIdx.x < 16)
+    nlut[threadIdx.x] = SYM ? make_float2((float)(threadIdx.x & 3u) - 2.0f, (float)(threadIdx.x >> 2) - 2.0f)
+                            : make_float2((float)(threadIdx.x & 3u), (float)(threadIdx.x >> 2));
   for (int t = 0; t < p.t_smem; ++t) {
     const uint4* src = reinterpret_cast<const uint4*>(tables + ((int64_t)t * p.H + h) * tab_bytes);
     uint4* dst = reinterpret_cast<uint4*>(smem + (size_t)t * tab_bytes);
@@ -213,17 +234,26 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
     for (int u = 0; u < kDqU; ++u) {
       const int t = tb + u;
       // y = s*q + m (exact in fp32: E4M3 operands, q <= 3), two channels per
-      // op; the symmetric mode is the same with m = -2s (y = s*(u - 2))
+      // op; the symmetric mode multiplies, y = s*(u - 2) (exact, and with the
+      // sign of zero that product has)
       float2 y0[4], y1[4];
       {
         const float s0 = dec[sz[u] & 0xFFu], s1 = dec[(sz[u] >> 16) & 0xFFu];
-        const float m0 = SYM ? -2.0f * s0 : dec[(sz[u] >> 8) & 0xFFu];
-        const float m1 = SYM ? -2.0f * s1 : dec[sz[u] >> 24];
-        const float2 sp0 = f2(s0, s0), mp0 = f2(m0, m0), sp1 = f2(s1, s1), mp1 = f2(m1, m1);
+        const float2 sp0 = f2(s0, s0), sp1 = f2(s1, s1);
+        if (SYM) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          y0[e] = __ffma2_rn(sp0, nlut[(cb[u] >> (4 * e)) & 0xFu], mp0);
-          y1[e] = __ffma2_rn(sp1, nlut[(cb[u] >> (16 + 4 * e)) & 0xFu], mp1);
+          for (int e = 0; e < 4; ++e) {
+            y0[e] = __fmul2_rn(sp0, nlut[(cb[u] >> (4 * e)) & 0xFu]);
+            y1[e] = __fmul2_rn(sp1, nlut[(cb[u] >> (16 + 4 * e)) & 0xFu]);
+          }
+        } else {
+          const float m0 = dec[(sz[u] >> 8) & 0xFFu], m1 = dec[sz[u] >> 24];
+          const float2 mp0 = f2(m0, m0), mp1 = f2(m1, m1);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            y0[e] = __ffma2_rn(sp0, nlut[(cb[u] >> (4 * e)) & 0xFu], mp0);
+            y1[e] = __ffma2_rn(sp1, nlut[(cb[u] >> (16 + 4 * e)) & 0xFu], mp1);
+          }
         }
       }
       // centroids of stage T, T-1, ..., 1, in that order
@@ -444,10 +474,17 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
     for (int x = threadIdx.x; x < kD; x += blockDim.x) { s_chmax[x] = 0u; s_chmin[x] = 0u; }
     __syncthreads();
   }
-  const float kInf = __int_as_float(0x7f800000);
-  float mx0[8], mx1[8], mn0[8], mn1[8];
+  // Both extremes are kept on packed bf16 pairs (two channels per 32-bit
+  // word; for fp32 data the words keep each value's exponent, see
+  // bf16_pair_bits, which is all the fixed-point scale and its check use):
+  //   xw = max of |v| (bf16 max of the sign-cleared word);
+  //   nw = max of (|v| + 0x7FFF) per half: zero gives 0x7FFF, a NaN that the
+  //        max ignores, and a nonzero h gives 0x8000 | (h - 1), i.e. -(h - 1),
+  //        so the maximum is minus (smallest nonzero |v| - 1 ulp); no half
+  //        carries into the other (each sum is at most 0xFFFE).
+  uint32_t xw[8], nw[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) { mx0[e] = 0.0f; mx1[e] = 0.0f; mn0[e] = kInf; mn1[e] = kInf; }
+  for (int e = 0; e < 8; ++e) { xw[e] = 0u; nw[e] = 0x7FFF7FFFu; }
   const int j = threadIdx.x & 7;
   const int G = GT > 0 ? GT : p.G;
   const int ng = kD / G;
@@ -496,11 +533,13 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
       if (valid && j == 0 && p.rnorm2 != nullptr) p.rnorm2[(int64_t)u * p.N + i] = s2;
       if (want_max) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          mx0[e] = fmaxf(mx0[e], fabsf(r0[e]));
-          mx1[e] = fmaxf(mx1[e], fabsf(r1[e]));
-          mn0[e] = fminf(mn0[e], r0[e] != 0.0f ? fabsf(r0[e]) : kInf);
-          mn1[e] = fminf(mn1[e], r1[e] != 0.0f ? fabsf(r1[e]) : kInf);
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t a0 = bf16_pair_bits<DT == kFP32>(r0[2 * e], r0[2 * e + 1]) & 0x7FFF7FFFu;
+          const uint32_t a1 = bf16_pair_bits<DT == kFP32>(r1[2 * e], r1[2 * e + 1]) & 0x7FFF7FFFu;
+          xw[e] = bf16x2_max(xw[e], a0);
+          xw[4 + e] = bf16x2_max(xw[4 + e], a1);
+          nw[e] = bf16x2_max(nw[e], a0 + 0x7FFF7FFFu);
+          nw[4 + e] = bf16x2_max(nw[4 + e], a1 + 0x7FFF7FFFu);
         }
       }
     } else {
@@ -537,25 +576,26 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
     // valid token, so they never raise a maximum)
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      mx0[e] = fmaxf(mx0[e], __shfl_xor_sync(0xffffffffu, mx0[e], 8));
-      mx0[e] = fmaxf(mx0[e], __shfl_xor_sync(0xffffffffu, mx0[e], 16));
-      mx1[e] = fmaxf(mx1[e], __shfl_xor_sync(0xffffffffu, mx1[e], 8));
-      mx1[e] = fmaxf(mx1[e], __shfl_xor_sync(0xffffffffu, mx1[e], 16));
-      mn0[e] = fminf(mn0[e], __shfl_xor_sync(0xffffffffu, mn0[e], 8));
-      mn0[e] = fminf(mn0[e], __shfl_xor_sync(0xffffffffu, mn0[e], 16));
-      mn1[e] = fminf(mn1[e], __shfl_xor_sync(0xffffffffu, mn1[e], 8));
-      mn1[e] = fminf(mn1[e], __shfl_xor_sync(0xffffffffu, mn1[e], 16));
+      xw[e] = bf16x2_max(xw[e], __shfl_xor_sync(0xffffffffu, xw[e], 8));
+      xw[e] = bf16x2_max(xw[e], __shfl_xor_sync(0xffffffffu, xw[e], 16));
+      nw[e] = bf16x2_max(nw[e], __shfl_xor_sync(0xffffffffu, nw[e], 8));
+      nw[e] = bf16x2_max(nw[e], __shfl_xor_sync(0xffffffffu, nw[e], 16));
     }
-    // the smallest nonzero magnitude is kept as 0x7FFFFFFF minus its bits, so
-    // that an atomic maximum finds it and zero means "no nonzero value"
-    auto inv = [](float m) { return m == __int_as_float(0x7f800000) ? 0u : 0x7FFFFFFFu - __float_as_uint(m); };
+    // chmax holds fp32 bits of the largest |v|; chmin holds 0x7FFFFFFF minus
+    // the fp32 bits of the smallest nonzero |v|, so that an atomic maximum
+    // finds it and zero means "no nonzero value"
     if ((threadIdx.x & 31) < 8) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        atomicMax(&s_chmax[8 * j + e], __float_as_uint(mx0[e]));
-        atomicMax(&s_chmax[64 + 8 * j + e], __float_as_uint(mx1[e]));
-        atomicMax(&s_chmin[8 * j + e], inv(mn0[e]));
-        atomicMax(&s_chmin[64 + 8 * j + e], inv(mn1[e]));
+        const int c0 = (e < 4 ? 8 * j + 2 * e : 64 + 8 * j + 2 * (e - 4));
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t x = (xw[e] >> (16 * hf)) & 0xFFFFu;
+          const uint32_t n = (nw[e] >> (16 * hf)) & 0xFFFFu;
+          atomicMax(&s_chmax[c0 + hf], x << 16);
+          if ((n & 0x7FFFu) <= 0x7F80u)        // not the NaN of an all-zero channel
+            atomicMax(&s_chmin[c0 + hf], 0x7FFFFFFFu - ((((n & 0x7FFFu) + 1u)) << 16));
+        }
       }
     }
     __syncthreads();

@@ -481,9 +481,23 @@ qvg_update_sum(const UpdateParams p) {
   if (n <= 0) return;
   const int npairs = (n + 1) >> 1;
   float to_fix[8];
+  // For bf16 rows the scaling by 2^-L is also an integer add of -L to the
+  // exponent field of each half of a pair word, valid when L <= 0 for every
+  // channel of the lane: a normal value is scaled exactly, a zero becomes at
+  // most 2^-1 and rounds to 0, and a bf16 subnormal can only occur in a
+  // channel that the centroid kernel sums exactly instead.  The warp takes
+  // that path when all its lanes qualify (the sums are the same either way).
+  uint32_t shiftw[4];
+  bool lane_fast = true;
 #pragma unroll
-  for (int e = 0; e < 8; ++e)
-    to_fix[e] = __int_as_float((127 - fix_exponent(p.chmax[(int64_t)u * kD + 8 * hl + e], p.log2n)) << 23);
+  for (int e = 0; e < 8; ++e) {
+    const int L = fix_exponent(p.chmax[(int64_t)u * kD + 8 * hl + e], p.log2n);
+    to_fix[e] = __int_as_float((127 - L) << 23);
+    lane_fast &= L <= 0;
+    const uint32_t part = (uint32_t)(L <= 0 ? -L : 0) << ((e & 1) ? 23 : 7);
+    if ((e & 1) == 0) shiftw[e >> 1] = part; else shiftw[e >> 1] |= part;
+  }
+  const bool fast = DT == kBF16 && __all_sync(0xffffffffu, lane_fast);
   const uint32_t* list = p.list + (int64_t)u * 2 * N + e0;
   const char* Ru = static_cast<const char*>(p.R) + (int64_t)u * N * ROW + hl * LANE_BYTES;
   unsigned char* ring = smem + (size_t)warp * kSumRing * 2 * ROW + half * ROW + hl * LANE_BYTES;
@@ -536,7 +550,26 @@ qvg_update_sum(const UpdateParams p) {
     const int r = 2 * jp + half;
     const uint32_t ent = __shfl_sync(0xffffffffu, (r >> 5) & 1 ? ge1 : ge0, r & 31);
     const int slot = jp % kSumRing;
-    if (r < n) {
+    if (r < n && fast) {
+      // bf16 rows, exponent-add scaling: the sign of a subtracted row is one
+      // xor per pair word, the scaling one integer add per pair word
+      const uint4 w = *reinterpret_cast<const uint4*>(ring + slot * 2 * ROW);
+      const uint32_t key = (ent >> kEntKShift) & 0xFFu;
+      const uint32_t sgn = (ent & kEntSub) ? 0x80008000u : 0u;
+      if (key != run_key) {
+        flush();
+        run_key = key;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) run[e] = 0;
+      }
+      const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t xs = (x[e] ^ sgn) + shiftw[e];
+        run[2 * e] += __float2ll_rn(__uint_as_float(xs << 16));
+        run[2 * e + 1] += __float2ll_rn(__uint_as_float(xs & 0xFFFF0000u));
+      }
+    } else if (r < n) {
       float v[8];
       const unsigned char* src = ring + slot * 2 * ROW;
       if (DT == kBF16) {

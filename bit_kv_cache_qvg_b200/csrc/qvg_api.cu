@@ -210,12 +210,12 @@ qvg_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QVG_OK : QVG_E
 // kernel from CUDA events recorded on the launching stream around each launch.
 enum Kind {
   K_DEQUANT, K_RESIDUAL, K_RESIDUAL_QUANT, K_ROWNORM, K_INIT, K_ASSIGN_EXACT, K_ASSIGN_TC,
-  K_RECHECK, K_UPD_BUCKET, K_UPD_SUM, K_UPD_CENT, K_NKINDS
+  K_RECHECK, K_UPD_BUCKET, K_UPD_SUM, K_UPD_CENT, K_ATTN, K_ROPE, K_NKINDS
 };
 const char* const kKindNames[K_NKINDS] = {
   "qvg_dequant_fused", "qvg_residual", "qvg_residual_quant", "qvg_row_norms", "qvg_init_centroids",
   "qvg_assign_exact", "qvg_kmeans_assign", "qvg_assign_recheck", "qvg_update_bucket", "qvg_update_sum",
-  "qvg_update_centroids"};
+  "qvg_update_centroids", "qvg_attention_fused", "qvg_rope_tables"};
 
 struct Profiler {
   std::mutex mu;
@@ -517,6 +517,54 @@ qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packed, qvg_d
   p.t_smem = std::min<int>(cfg->T, (int)((160 * 1024) / table));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
   st = cuda_status(plaunch(K_DEQUANT, s, [&] { return launch_dequant(p, dt, s); }));
+  if (st == QVG_OK && fault_injected("stream")) st = QVG_ERR_CUDA;
+  return st;
+}
+
+size_t qvg_rope_tables_bytes(int32_t d, int64_t max_pos) {
+  if (d != kD || max_pos < 0 || max_pos >= (int64_t(1) << 40)) return 0;
+  const int64_t n_hi = max_pos / 1024 + 1;
+  return kRopeHeaderBytes + (size_t)(n_hi + 1024) * (kD / 2) * sizeof(float) * 2;
+}
+
+qvg_status qvg_rope_tables(double base, int32_t d, int64_t max_pos, void* tables, size_t bytes,
+                           qvg_stream_t stream_) {
+  const size_t need = qvg_rope_tables_bytes(d, max_pos);
+  if (need == 0 || !(base > 1.0) || tables == nullptr || !aligned(tables, 16)) return QVG_ERR_INVALID_ARG;
+  if (bytes < need) return QVG_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  const int n_hi = (int)(max_pos / 1024 + 1);
+  QVG_TRY(cudaMemsetAsync(tables, 0, 16, s));
+  return cuda_status(plaunch(K_ROPE, s, [&] { return launch_rope_tables(tables, n_hi, base, s); }));
+}
+
+qvg_status qvg_attention(const qvg_config* cfg, const qvg_packed* k, const qvg_packed* v, int64_t Nk, int32_t H,
+                         int32_t d, const void* Q, const int64_t* q_pos, int64_t Nq, const void* tables,
+                         size_t tables_bytes, float* O, qvg_stream_t stream_) {
+  qvg_status st = check_config(cfg, Nk, H, d, QVG_BF16);
+  if (st != QVG_OK) return st;
+  const bool sym = cfg->scale_mode == QVG_SCALE_SYM;
+  for (const qvg_packed* p : {k, v}) {
+    if (p == nullptr || p->codes == nullptr || p->scale == nullptr || (p->zero == nullptr && !sym))
+      return QVG_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (p->assign == nullptr || p->centroids == nullptr || !aligned(p->centroids, 16)))
+      return QVG_ERR_INVALID_ARG;
+    if (!aligned(p->codes, 2)) return QVG_ERR_INVALID_ARG;
+  }
+  if (Nk < 1 || Nq < 1 || Q == nullptr || q_pos == nullptr || tables == nullptr || O == nullptr ||
+      !aligned(Q, 16) || !aligned(O, 16) || !aligned(tables, 16) || Nq >= (int64_t(1) << 31) * 128)
+    return QVG_ERR_INVALID_ARG;
+  const size_t row_bytes = (kD / 2) * sizeof(float) * 2;
+  if (tables_bytes < kRopeHeaderBytes + 1024 * row_bytes + row_bytes) return QVG_ERR_INVALID_ARG;
+  const int64_t n_hi = (int64_t)((tables_bytes - kRopeHeaderBytes) / row_bytes) - 1024;
+  if (Nk - 1 > n_hi * 1024 - 1) return QVG_ERR_INVALID_ARG;        // the cache's positions must be covered
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+  st = peek_sticky(tables, s);
+  if (st != QVG_OK) return st;
+  AttentionArgs a{};
+  a.k = k; a.v = v; a.Q = Q; a.qpos = q_pos; a.tables = tables; a.n_hi = (int)n_hi; a.O = O;
+  a.Nk = Nk; a.Nq = Nq; a.H = H; a.K = cfg->K; a.T = cfg->T; a.G = cfg->group_size; a.sym = sym ? 1 : 0;
+  st = cuda_status(plaunch(K_ATTN, s, [&] { return launch_attention(a, s); }));
   if (st == QVG_OK && fault_injected("stream")) st = QVG_ERR_CUDA;
   return st;
 }

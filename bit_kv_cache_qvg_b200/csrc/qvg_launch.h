@@ -142,4 +142,24 @@ cudaError_t launch_update_bucket(const UpdateParams& p, int dtype, cudaStream_t 
 cudaError_t launch_update_sum(const UpdateParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_update_centroids(const UpdateParams& p, int dtype, cudaStream_t s);
 
+// ---- attention over the compressed cache (kernel_attention.cu)
+// Rotary tables: a 256-byte header (its first 4 bytes are the status word
+// of the attention calls that use the tables), then hi[n_hi][d/2] and
+// lo[1024][d/2] (cos, sin) pairs in fp32.
+constexpr size_t kRopeHeaderBytes = 256;
+cudaError_t launch_rope_tables(void* tables, int n_hi, double base, cudaStream_t s);
+struct AttentionArgs {
+  const qvg_packed* k;         // K cache: H blocks of Nk tokens (bf16 tables)
+  const qvg_packed* v;         // V cache, same configuration
+  const void* Q;               // [H][Nq][d] bf16, before the rotary embedding
+  const int64_t* qpos;         // [Nq]
+  const void* tables;          // rotary tables (header + hi + lo)
+  int n_hi;                    // rows of the hi table
+  float* O;                    // [H][Nq][d] fp32
+  int64_t Nk, Nq;
+  int H, K, T, G, sym;
+};
+cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s);
+size_t attention_smem_bytes();
+
 }  // namespace qvg

@@ -79,6 +79,11 @@ _SIGS = {
                                        C.POINTER(C.c_int64)]),
     "qvg_cache_device_bytes": (C.c_size_t, [C.c_void_p]),
     "qvg_cache_destroy": (None, [C.c_void_p]),
+    "qvg_rope_tables_bytes": (C.c_size_t, [C.c_int32, C.c_int64]),
+    "qvg_rope_tables": (C.c_int, [C.c_double, C.c_int32, C.c_int64, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "qvg_attention": (C.c_int, [C.POINTER(Config), C.POINTER(_Packed), C.POINTER(_Packed), C.c_int64, C.c_int32,
+                                C.c_int32, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_size_t, C.c_void_p,
+                                C.c_void_p]),
     "qvg_profile_enable": (None, [C.c_int]),
     "qvg_profile_reset": (None, []),
     "qvg_profile_launches": (C.c_int64, []),
@@ -240,6 +245,34 @@ def dequantize(p: Packed, Y: Optional[torch.Tensor] = None, stream=None) -> torc
     st = lib().qvg_dequantize(C.byref(p.cfg), C.byref(ps), p.dtype, p.N, p.H, p.d, _ptr(Y), _stream(stream))
     _check(st, "qvg_dequantize")
     return Y
+
+
+def rope_tables(max_pos: int, base: float = 10000.0, d: int = 128, device="cuda", stream=None) -> torch.Tensor:
+    """qvg_rope_tables: the rotary (cos, sin) tables for positions 0 .. max_pos
+    (a uint8 device tensor; its first 4 bytes are the attention status word)."""
+    n = int(lib().qvg_rope_tables_bytes(d, max_pos))
+    if n == 0:
+        raise QvgError(1, "qvg_rope_tables_bytes")
+    t = torch.empty(n, dtype=torch.uint8, device=device)
+    _check(lib().qvg_rope_tables(float(base), d, max_pos, _ptr(t), n, _stream(stream)), "qvg_rope_tables")
+    return t
+
+
+def attention(kp: Packed, vp: Packed, Q: torch.Tensor, q_pos: torch.Tensor, tables: torch.Tensor,
+              O: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """qvg_attention: softmax(rope(Q) rope(K^)^T / sqrt(d)) V^ per head over the
+    compressed caches kp (keys, before the rotary embedding) and vp (values);
+    Q [H][Nq][d] bf16, q_pos [Nq] int64 (device); returns O [H][Nq][d] fp32."""
+    if Q.dim() != 3 or not Q.is_contiguous() or Q.dtype != torch.bfloat16:
+        raise QvgError(1, "Q must be a contiguous bf16 [H][Nq][d] tensor")
+    H, Nq, d = Q.shape
+    if O is None:
+        O = torch.empty((H, Nq, d), dtype=torch.float32, device=Q.device)
+    ks, vs = kp.struct(), vp.struct()
+    _check(lib().qvg_attention(C.byref(kp.cfg), C.byref(ks), C.byref(vs), kp.N, H, d, _ptr(Q),
+                               _ptr(q_pos), Nq, _ptr(tables), tables.numel(), _ptr(O), _stream(stream)),
+           "qvg_attention")
+    return O
 
 
 def profile_enable(on: bool = True):

@@ -253,6 +253,52 @@ QVG_API qvg_status qvg_quantize_static(const qvg_config* cfg, const void* X, qvg
 QVG_API qvg_status qvg_static_status(qvg_stream_t stream);
 
 /* ------------------------------------------------------------------ */
+/* Attention over the compressed cache: the consumer of the m.163.com    */
+/* article, section 五 (keys are cached before the rotary position       */
+/* embedding, which is applied after dequantisation; the fused kernel     */
+/* feeds the reconstruction to attention without writing it out;         */
+/* gist.science/de, Technische Zusammenfassung 2C, "Fused Kernel").       */
+/* ------------------------------------------------------------------ */
+
+/* Bytes of the rotary tables for head dimension d and positions
+ * 0 .. max_pos: a 256-byte header, then (cos, sin) of p * theta_i in fp32
+ * for p = 1024 a and for p = b < 1024.  0 for unsupported arguments
+ * (d != 128).  Host-only. */
+QVG_API size_t qvg_rope_tables_bytes(int32_t d, int64_t max_pos);
+
+/* Fill the rotary tables (DEVICE, caller-owned, 16-byte aligned, `bytes`
+ * from qvg_rope_tables_bytes) for theta_i = base^(-2i/d), the RoFormer form:
+ * channel pair (2i, 2i+1) of a token at position p is turned by p * theta_i.
+ * The angles and their cosines and sines are formed in fp64 on the device and
+ * rounded to fp32.  The header's first 4 bytes are the status word of the
+ * qvg_attention calls that use the tables (read and cleared by
+ * qvg_workspace_status on the tables buffer).  Errors: INVALID_ARG (base
+ * <= 1, d != 128, NULL), WORKSPACE_TOO_SMALL, CUDA. */
+QVG_API qvg_status qvg_rope_tables(double base, int32_t d, int64_t max_pos, void* tables, size_t bytes,
+                           qvg_stream_t stream);
+
+/* Softmax attention of Nq queries per head over a compressed K/V cache of
+ * Nk tokens per head, with the reconstruction fused into the K/V load:
+ *   O[h] = softmax(rope(Q[h]) rope(K^[h])^T / sqrt(d)) V^[h]
+ * K^ and V^ are what qvg_dequantize would write for `k` and `v` (two
+ * qvg_quantize outputs of H blocks of Nk tokens with the same cfg; bf16),
+ * bit for bit; they are never written to memory.  Cached token i sits at
+ * position i; query n at q_pos[n] (positions outside [0, max_pos] of the
+ * tables are clamped).  No mask.
+ *   Q      DEVICE [H][Nq][d] bf16, before the rotary embedding, 16-byte aligned
+ *   q_pos  DEVICE [Nq] int64
+ *   tables DEVICE rotary tables (qvg_rope_tables); they must cover Nk - 1
+ *   O      DEVICE [H][Nq][d] fp32, 16-byte aligned
+ * The products run on the tensor cores with bf16 operands (the rotated keys
+ * and queries and the softmax weights are rounded to bf16) and fp32
+ * accumulation; the softmax uses base-2 exponentials in fp32.
+ * Errors: INVALID_ARG, UNSUPPORTED (d != 128, ...), CUDA, DEVICE_TIMEOUT (a
+ * timeout recorded in the tables' status word by earlier, completed work). */
+QVG_API qvg_status qvg_attention(const qvg_config* cfg, const qvg_packed* k, const qvg_packed* v, int64_t Nk,
+                         int32_t H, int32_t d, const void* Q, const int64_t* q_pos, int64_t Nq,
+                         const void* tables, size_t tables_bytes, float* O, qvg_stream_t stream);
+
+/* ------------------------------------------------------------------ */
 /* Diagnostics (no counterpart in the method; used by the benchmark).    */
 /* ------------------------------------------------------------------ */
 

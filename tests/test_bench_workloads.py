@@ -46,6 +46,21 @@ def test_sweep_closed_form_matches_library_packed_size():
         packed = qvg.packed_bytes(cfg, N, 1)
         ratio = N * 128 * 2 / packed
         assert abs(ratio - bench.compression_ratio(K, T, G, N)) < 1e-9 * ratio
+        packed1 = qvg.packed_bytes(qvg.config(K=K, T=T, group_size=G, scale_mode=1), N, 1)
+        ratio1 = N * 128 * 2 / packed1
+        assert abs(ratio1 - bench.compression_ratio(K, T, G, N, scale_bytes=1)) < 1e-9 * ratio1
+
+
+def test_named_points_land_in_the_pages_ranges():
+    """The sweep labels the QVG and QVG-Pro settings and plain rounding at
+    G = 16 (one scale per group) with the pages' compression figures."""
+    from bit_kv_cache_qvg_b200 import qvg
+    for name in ("qvg", "qvg-pro"):
+        P = qvg.PRESETS[name]
+        r = bench.compression_ratio(P["K"], P["T"], P["group_size"], 38000, scale_bytes=1)
+        lo, hi = bench.PAGE_RATIOS[name]
+        assert lo <= r <= hi
+    assert bench.compression_ratio(1, 0, 16, 38000, scale_bytes=1) == bench.PAGE_RATIOS["rtn"][0]
 
 
 def test_sweep_grid_covers_the_design_space():
