@@ -56,6 +56,12 @@ WORKLOADS = {
                         "tokens appended in chunks of 3 frames (4,680 tokens; last chunk 1 frame), "
                         "up to 1,092,000 tokens, d=128, bf16; K=256, T=2, G=64; warm start 3 "
                         "Lloyd iterations vs 10 cold; whole cache dequantised after every chunk"),
+    "attention": dict(layers=1, heads=32, frames=25, gh=38, gw=40, K=256, T=2, G=64, iters=10, q_frames=1,
+                      attention=True,
+                      desc="Attention over the compressed cache, one layer of the LongCat-scale cache: 32 heads, "
+                           "38,000 cached tokens per head (K=256, T=2, G=64), queries = the next frame (1,520 "
+                           "tokens per head), d=128, bf16 operands; fused dequant + RoPE + attention against "
+                           "dequantise-then-attend"),
     "sweep": dict(layers=1, heads=32, frames=25, gh=38, gw=40, K=256, T=2, G=64, iters=10, sweep=True,
                   desc="Design sweep on one layer: 32 heads x K/V, 38,000 tokens (25 frames x 38x40), "
                        "d=128, bf16; T in {0,1,2,3,4} x G in {16,32,64} x K in {64,256}, 10 Lloyd "
@@ -206,8 +212,53 @@ def oracle_stream_sample(wl, chunks: int, seed: int = 7):
     return t / chunks, o.get_threads()
 
 
+def oracle_attention_sample(wl, n_queries: int, seed: int = 5):
+    """Time the oracle's fp64 attention of `n_queries` queries over one head's
+    reconstructed cache of the workload's length (the reconstruction itself,
+    from a packed cache quantised by the oracle at T = 0, is untimed).
+    Returns (seconds, flops, threads)."""
+    import numpy as np
+    import torch
+    from bit_kv_cache_qvg_b200 import synth
+    from oracle import oracle as o
+    o.build()
+    Nk = wl["frames"] * wl["gh"] * wl["gw"]
+    Xk = synth.block_batch(1, synth.KVShape(wl["frames"], wl["gh"], wl["gw"]), seed=seed, kinds=[0])
+    Xv = synth.block_batch(1, synth.KVShape(wl["frames"], wl["gh"], wl["gw"]), seed=seed + 1, kinds=[1])
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    f32 = lambda b: (b.astype(np.uint32) << 16).view(np.float32)
+    Kh = f32(o.dequantize(o.quantize(bits(Xk), K=1, T=0, G=wl["G"], iters=0), K=1, T=0, G=wl["G"], N=Nk, H=1, d=128))
+    Vh = f32(o.dequantize(o.quantize(bits(Xv), K=1, T=0, G=wl["G"], iters=0), K=1, T=0, G=wl["G"], N=Nk, H=1, d=128))
+    rng = np.random.default_rng(seed)
+    Q = (rng.standard_normal((n_queries, 128)) * 0.05).astype(np.float32)
+    t0 = time.perf_counter()
+    o.attention(Q, np.arange(Nk, Nk + n_queries), Kh[0], Vh[0])
+    dt = time.perf_counter() - t0
+    return dt, 4.0 * n_queries * Nk * 128, o.get_threads()
+
+
 def run_reference(args, wl, rank, world):
     if rank != 0:
+        return
+    if wl.get("attention"):
+        times = []
+        nq = 32
+        for i in range(args.warmup + args.steps):
+            dt, flops, threads = oracle_attention_sample(wl, nq, seed=1000 + i)
+            if i >= args.warmup:
+                times.append(dt)
+        t = sum(times) / len(times)
+        v = flops / t / 1e12
+        sample = (f"{nq} queries of one head over the head's {wl['frames'] * wl['gh'] * wl['gw']}-token "
+                  "reconstructed cache per step (fp64 rotary embedding and softmax attention)")
+        print(json.dumps({
+            "impl": "reference", "metric": ATTN_METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl["desc"], "reference": "C oracle (fp64 attention) on host cores"},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
         return
     if "chunk_frames" in wl:
         times = []
@@ -301,6 +352,12 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks = load_peaks()
+    if wl.get("attention"):
+        run_attention(args, wl, qvg, synth, dev, dist, rank, world, local, peaks)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     if wl.get("sweep"):
         run_sweep(args, wl, qvg, synth, dev, dist, rank, world, peaks)
         if dist is not None:
@@ -628,6 +685,139 @@ def run_sweep(args, wl, qvg, synth, dev, dist, rank, world, peaks):
                    "l2": "inputs larger than L2 (no flush needed)"},
         "points": points,
     }
+    if rank == 0:
+        print(json.dumps(result))
+
+
+ATTN_METRIC = "attention over the compressed cache: fused dequant + RoPE + attention, TFLOP/s and HBM bytes"
+
+
+def rope_torch(x, pos, base=10000.0):
+    """Rotary embedding with torch ops (the dequantise-then-attend baseline):
+    pair (2i, 2i+1) turned by pos * base^(-2i/d), in fp32, back to bf16."""
+    import torch
+    d = x.shape[-1]
+    i = torch.arange(d // 2, device=x.device, dtype=torch.float64)
+    ang = (pos.to(torch.float64)[:, None] * base ** (-2.0 * i / d)[None, :])
+    c, sn = torch.cos(ang).float(), torch.sin(ang).float()
+    xf = x.float()
+    a, b = xf[..., 0::2], xf[..., 1::2]
+    out = torch.empty_like(xf)
+    out[..., 0::2] = a * c - b * sn
+    out[..., 1::2] = a * sn + b * c
+    return out.to(torch.bfloat16)
+
+
+def run_attention(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
+    """The attention consumer: one layer's compressed K and V caches (H heads of
+    Nk tokens) and the next frame's queries.  Fused: qvg_attention (dequant +
+    RoPE in shared memory, tcgen05 products, online softmax).  Baseline:
+    qvg_dequantize of K and V to bf16, RoPE with torch ops, torch's
+    scaled_dot_product_attention.  Both event-timed on the launching stream."""
+    import torch
+    H = wl["heads"]
+    Nk = wl["frames"] * wl["gh"] * wl["gw"]
+    Nq = wl["q_frames"] * wl["gh"] * wl["gw"]
+    cfg = qvg.config(K=wl["K"], T=wl["T"], group_size=wl["G"], iters=wl["iters"])
+    shape = synth.KVShape(wl["frames"], wl["gh"], wl["gw"])
+    Xk = synth.block_batch(H, shape, seed=synth.unit_seed(rank, 0, 0, 0), kinds=[0] * H, device=dev)
+    Xv = synth.block_batch(H, shape, seed=synth.unit_seed(rank, 0, 0, 1), kinds=[1] * H, device=dev)
+    kp, vp = qvg.quantize(Xk, cfg), qvg.quantize(Xv, cfg)
+    del Xk, Xv
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234 + rank)
+    Q = (torch.randn((H, Nq, 128), generator=g, device=dev) * 0.05).to(torch.bfloat16)
+    qpos = torch.arange(Nk, Nk + Nq, device=dev, dtype=torch.int64)
+    kpos = torch.arange(Nk, device=dev, dtype=torch.int64)
+    tables = qvg.rope_tables(Nk + Nq, device=dev)
+    O = torch.empty((H, Nq, 128), dtype=torch.float32, device=dev)
+    Kd = torch.empty((H, Nk, 128), dtype=torch.bfloat16, device=dev)
+    Vd = torch.empty_like(Kd)
+    stream = torch.cuda.Stream(dev)
+
+    def fused():
+        qvg.attention(kp, vp, Q, qpos, tables, O=O, stream=stream)
+
+    def unfused():
+        qvg.dequantize(kp, Kd, stream=stream)
+        qvg.dequantize(vp, Vd, stream=stream)
+        with torch.cuda.stream(stream):
+            kr = rope_torch(Kd, kpos)
+            qr = rope_torch(Q, qpos)
+            return torch.nn.functional.scaled_dot_product_attention(qr[None], kr[None], Vd[None])[0]
+
+    def timed(fn, n):
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(n):
+                fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    with ClockSampler(local) as clk:
+        ms_f = max_over_ranks(dist, timed(fused, args.steps), dev)
+        ms_u = max_over_ranks(dist, timed(unfused, args.steps), dev)
+    if qvg.workspace_status(tables) != 0:
+        raise SystemExit("device-side wait timed out in the attention kernel")
+    # agreement of the two outputs (different roundings; a sanity figure)
+    with torch.cuda.stream(stream):
+        ref = unfused()
+    torch.cuda.synchronize()
+    rel = float((O - ref.float()).norm() / ref.float().norm())
+    flops = 4.0 * H * Nq * Nk * 128
+    packed = kp.nbytes() + vp.nbytes()
+    io = Q.numel() * 2 + qpos.numel() * 8 + O.numel() * 4
+    bytes_fused = packed + io
+    # dequantise-then-attend: the packed form read, the bf16 K and V written and
+    # read back once (by the RoPE and the attention), the rotated K written and read
+    cache_bf16 = 2 * H * Nk * 128 * 2
+    bytes_unfused = packed + 2 * cache_bf16 + 2 * (H * Nk * 128 * 2) + io
+    tflops = flops / (ms_f / 1e3) / 1e12
+    result = {
+        "metric": ATTN_METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_f, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl["desc"], "heads": H, "cached_tokens": Nk, "queries": Nq,
+                   "l2": "packed caches fit in L2; the baseline's bf16 caches do not"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+                     "frac": tflops / peaks["bf16_sus"], "traffic": None, "kernel": "qvg_attention_fused",
+                     "alg_flops_per_launch": flops},
+        "fused": {"ms": ms_f, "hbm_bytes": bytes_fused},
+        "dequantise_then_attend": {"ms": ms_u, "hbm_bytes": bytes_unfused,
+                                   "parts": "qvg_dequantize x2, RoPE (torch ops), scaled_dot_product_attention"},
+        "hbm_bytes_saved": bytes_unfused - bytes_fused,
+        "speedup_vs_unfused": ms_u / ms_f,
+        "rel_diff_vs_unfused": rel,
+        "gpu_launches": 1,
+        "clocks": clk.summary(),
+    }
+    # end to end through the public API: the queries arrive from pinned host
+    # memory, the output returns to pinned host memory, every step
+    Qh = Q.cpu().pin_memory()
+    Oh = torch.empty(O.shape, dtype=torch.float32, pin_memory=True)
+    Qd = torch.empty_like(Q)
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            Qd.copy_(Qh, non_blocking=True)
+            qvg.attention(kp, vp, Qd, qpos, tables, O=O, stream=stream)
+            Oh.copy_(O, non_blocking=True)
+
+    ms_e = max_over_ranks(dist, timed(e2e_step, args.steps), dev)
+    result["e2e"] = {"value": flops / (ms_e / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e,
+                     "h2d_bytes_per_step": Qh.numel() * 2, "d2h_bytes_per_step": Oh.numel() * 4,
+                     "api": "qvg_attention with the queries copied in and the output copied out"}
+    if rank == 0 and not args.no_cpu_baseline:
+        dt, fl, threads = oracle_attention_sample(wl, 32)
+        result["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                  "sample": f"32 queries of one head over its {Nk}-token reconstructed cache, "
+                                            f"{dt:.1f} s"}
     if rank == 0:
         print(json.dumps(result))
 

@@ -291,10 +291,11 @@ qvg_attention_fused(const AttnParams p) {
   for (int j = 0; j < ntiles && ok; ++j) {
     j_last = j;
     const int64_t k0 = (int64_t)j * kAtTile;
-    // the previous product O += P V must be done before its operands are overwritten
+    // the previous product O += P V must be done before its operands are
+    // overwritten; every thread waits, and the CTA gives up together
     if (j > 0) {
-      ok = bar_wait(&bars->o_done, (uint32_t)((j - 1) & 1));
-      if (!ok) break;
+      const bool w_ok = bar_wait(&bars->o_done, (uint32_t)((j - 1) & 1));
+      if (__syncthreads_or(!w_ok)) { ok = false; break; }
       fence_after();
     }
     // 1. reconstruct the K and V tile into the operand layouts
@@ -343,7 +344,8 @@ qvg_attention_fused(const AttnParams p) {
     }
     // 3. online softmax (warps 0-3: the thread's query is row 32*warp + lane)
     if (warp < 4) {
-      if (!bar_wait(&bars->s_done, (uint32_t)(j & 1))) {
+      // warp-uniform outcome: the tensor-memory loads below are warp-collective
+      if (!__all_sync(0xffffffffu, bar_wait(&bars->s_done, (uint32_t)(j & 1)))) {
         *reinterpret_cast<volatile int*>(&bars->abort_flag) = 1;
       } else {
         fence_after();
@@ -406,9 +408,10 @@ qvg_attention_fused(const AttnParams p) {
       mma_commit(&bars->o_done);
     }
   }
-  // the last product, then O / l
+  // the last product, then O / l (ok is uniform over the CTA here)
   if (ok && ntiles > 0) {
-    ok = bar_wait(&bars->o_done, (uint32_t)((ntiles - 1) & 1));
+    const bool w_ok = bar_wait(&bars->o_done, (uint32_t)((ntiles - 1) & 1));
+    ok = !__syncthreads_or(!w_ok);
     fence_after();
   }
   if (warp < 4 && ok && ntiles > 0) {

@@ -1,0 +1,102 @@
+"""qvg_attention (the consumer of the compressed cache, with dequantisation
+and the rotary embedding fused into the K/V load) against the oracle's fp64
+attention over the oracle's reconstruction of the same packed caches.
+
+Tolerance, from the arithmetic of the kernel: the rotated queries and keys
+enter the tensor cores rounded to bf16 (relative error 2^-9 each), so a score
+s_j = q'.k'_j / sqrt(d) is off by at most eps_j = 2^-8 sum_c |q'_c k'_jc| /
+sqrt(d) (plus fp32 sums, far smaller); a perturbation of at most eps in every
+score changes the softmax weights by at most 2(e^(2 eps) - 1) in total, and
+rounding the weights to bf16 adds 2^-8 more.  So output element (i, c) is
+within max_j |v_jc| (2(e^(2 eps_i) - 1) + 2^-7) of the exact value, eps_i
+the row's largest eps_j.  The tests also check that the typical error is far
+below that bound."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import np_bits, packed_np, values
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from bit_kv_cache_qvg_b200 import build
+    build.build()
+    from bit_kv_cache_qvg_b200 import qvg
+    return qvg
+
+
+def _run_case(q, ora, cfg, H, Nk, Nq, q_scale, seed, base=10000.0):
+    from bit_kv_cache_qvg_b200 import synth
+    frames = -(-Nk // 1560)
+    Xk = synth.block_batch(H, synth.KVShape(frames, 30, 52), seed=seed, kinds=[0] * H)[:, :Nk].contiguous()
+    Xv = synth.block_batch(H, synth.KVShape(frames, 30, 52), seed=seed + 1, kinds=[1] * H)[:, :Nk].contiguous()
+    kp = q.quantize(Xk.cuda(), cfg)
+    vp = q.quantize(Xv.cuda(), cfg)
+    rng = np.random.default_rng(seed)
+    Qf = (rng.standard_normal((H, Nq, 128)) * q_scale).astype(np.float32)
+    Q = torch.from_numpy(Qf).to(torch.bfloat16)
+    qpos = np.arange(Nk, Nk + Nq, dtype=np.int64)
+    tables = q.rope_tables(Nk + Nq, base=base)
+    O = q.attention(kp, vp, Q.cuda(), torch.from_numpy(qpos).cuda(), tables)
+    torch.cuda.synchronize()
+    assert q.workspace_status(tables) == 0
+    O = O.cpu().numpy()
+    kn, vn = packed_np(kp), packed_np(vp)
+    mode = cfg.scale_mode
+    Kh = values(ora.dequantize(kn, K=cfg.K, T=cfg.T, G=cfg.group_size, N=Nk, H=H, d=128, scale_mode=mode))
+    Vh = values(ora.dequantize(vn, K=cfg.K, T=cfg.T, G=cfg.group_size, N=Nk, H=H, d=128, scale_mode=mode))
+    Qv = values(np_bits(Q))
+    worst = 0.0
+    for h in range(H):
+        ref = ora.attention(Qv[h].astype(np.float32), qpos, Kh[h].astype(np.float32), Vh[h].astype(np.float32),
+                            base=base)
+        qr = ora.rope(Qv[h].astype(np.float32), qpos, base)
+        kr = ora.rope(Kh[h].astype(np.float32), np.arange(Nk), base)
+        eps = 2.0 ** -8 * (np.abs(qr) @ np.abs(kr).T).max(axis=1) / np.sqrt(128)
+        # element (i, c): the weights' total change times channel c's largest |v|
+        bound = np.outer(2 * np.expm1(2 * eps) + 2.0 ** -7, np.abs(Vh[h]).max(axis=0)) + 1e-30
+        err = np.abs(O[h] - ref)
+        assert np.all(err <= bound), (h, float((err / bound).max()))
+        worst = max(worst, float(np.median(err / bound)))
+    return worst
+
+
+@pytest.mark.parametrize("H,Nk,Nq,T,G,K,mode,q_scale", [
+    (2, 1000, 200, 2, 64, 64, 0, 0.05),      # ragged cache and query tiles, two stages
+    (2, 256, 128, 1, 64, 256, 1, 0.05),      # the QVG point (one scale per group), whole tiles
+    (1, 77, 33, 0, 32, 1, 0, 0.2),           # plain rounding, one partial tile each
+    (2, 4680, 130, 4, 16, 256, 1, 0.02),     # the QVG-Pro point, a Self-Forcing-scale chunk
+])
+def test_attention_matches_oracle(q, ora, H, Nk, Nq, T, G, K, mode, q_scale):
+    cfg = q.config(K=K, T=T, group_size=G, iters=3, scale_mode=mode)
+    typical = _run_case(q, ora, cfg, H, Nk, Nq, q_scale, seed=Nk + T)
+    assert typical < 0.25          # the usual error is well inside the worst-case bound
+
+
+def test_attention_reports_a_stale_timeout_and_rejects_uncovered_positions(q):
+    from bit_kv_cache_qvg_b200 import synth
+    cfg = q.config(K=16, T=1, group_size=64, iters=2)
+    X = synth.block_batch(1, synth.KVShape(1, 10, 30), seed=3, kinds=[0]).cuda()
+    kp = q.quantize(X, cfg)
+    Q = torch.zeros((1, 8, 128), dtype=torch.bfloat16, device="cuda")
+    pos = torch.arange(8, dtype=torch.int64, device="cuda")
+    small = q.rope_tables(100)                       # positions 0 .. 1023 are covered
+    big = q.rope_tables(5000)
+    q.attention(kp, kp, Q, pos, big)
+    torch.cuda.synchronize()
+    X2 = synth.block_batch(1, synth.KVShape(1, 30, 52), seed=3, kinds=[0]).cuda()  # 1560 tokens
+    kp2 = q.quantize(X2, cfg)
+    with pytest.raises(q.QvgError) as e:
+        q.attention(kp2, kp2, Q, pos, small)         # token 1559 is beyond the small tables
+    assert e.value.status == 1
+    small[:4] = torch.tensor([1, 0, 0, 0], dtype=torch.uint8)   # a timeout recorded earlier
+    torch.cuda.synchronize()
+    with pytest.raises(q.QvgError) as e:
+        q.attention(kp, kp, Q, pos, small)
+    assert e.value.status == 5
+    assert q.workspace_status(small) == 5 and q.workspace_status(small) == 0
