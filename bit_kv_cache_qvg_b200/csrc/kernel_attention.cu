@@ -191,45 +191,80 @@ __device__ __forceinline__ float2 rope_cs(const AttnParams& p, int64_t pos, int 
                      __fadd_rn(__fmul_rn(a.y, b.x), __fmul_rn(a.x, b.y)));
 }
 
-// Reconstruct 8 channels (c0 .. c0+7) of token `tok` of cache `which` (0 = K,
-// 1 = V) of head h: y = s*q + m (or s*(u - 2)), plus the centroids of stages
-// T, ..., 1 in that order, each an fp32 add, then one rounding to bf16 --
-// the arithmetic of qvg_dequant_fused.  The results are returned as fp32
-// values of the rounded bf16 numbers.
-__device__ __forceinline__ void recon8(const AttnParams& p, const float* dec, int which, int h, int64_t tok, int c0,
-                                       float (&y)[8]) {
-  const int64_t row = (int64_t)h * p.Nk + tok;
+// Reconstruct channels c0 .. c0+7 of the 8 tokens tok0 .. tok0+7 (those
+// below Nk) of cache `which` (0 = K, 1 = V) of head h: y = s*q + m (or
+// s*(u - 2)), plus the centroids of stages T, ..., 1 in that order, each an
+// fp32 add, then one rounding to bf16 -- the arithmetic of qvg_dequant_fused.
+// The results are fp32 values of the rounded bf16 numbers (zero for tokens
+// past the end).  TT > 0 fixes the stage count (at most 4) so that the loads
+// of all eight tokens are issued together: first the codes, scale/zero bytes
+// and assignments, then the centroid rows they select.
+template <int TT>
+__device__ __forceinline__ void recon_block(const AttnParams& p, const float* dec, int which, int h,
+                                            int64_t tok0, int c0, float (&y)[8][8]) {
+  constexpr int TR = TT > 0 ? TT : 1;
+  const int T = TT >= 0 ? TT : p.T;
   const int ng = kD / p.G;
-  const uint16_t code = *reinterpret_cast<const uint16_t*>(p.codes[which] + row * (kD / 4) + c0 / 4);
   const int g = c0 / p.G;
-  const float s = dec[p.scale[which][row * ng + g]];
-  if (p.sym) {
+  uint32_t code[8], sz[8];
+  int kk[8][TR];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(s, (float)((code >> (2 * e)) & 3u) - 2.0f);
-  } else {
-    const float m = dec[p.zero[which][row * ng + g]];
+  for (int r = 0; r < 8; ++r) {
+    const int64_t tok = tok0 + r < p.Nk ? tok0 + r : p.Nk - 1;   // past the end: a valid token, result unused
+    const int64_t row = (int64_t)h * p.Nk + tok;
+    code[r] = *reinterpret_cast<const uint16_t*>(p.codes[which] + row * (kD / 4) + c0 / 4);
+    sz[r] = (uint32_t)p.scale[which][row * ng + g] | (p.sym ? 0u : ((uint32_t)p.zero[which][row * ng + g] << 8));
 #pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] = __fmaf_rn(s, (float)((code >> (2 * e)) & 3u), m);
+    for (int t = 0; t < TR; ++t)
+      if (TT > 0) kk[r][t] = min((int)p.assign[which][((int64_t)t * p.H + h) * p.Nk + tok], p.K - 1);
   }
-  for (int t = p.T - 1; t >= 0; --t) {
-    int k = p.assign[which][((int64_t)t * p.H + h) * p.Nk + tok];
-    k = min(k, p.K - 1);
-    const uint4 w = *reinterpret_cast<const uint4*>(p.tab[which] + (((int64_t)t * p.H + h) * p.K + k) * kD + c0);
-    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+  uint4 rows[8][TR];
+  if (TT > 0) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      y[2 * e] = __fadd_rn(y[2 * e], __uint_as_float(x[e] << 16));
-      y[2 * e + 1] = __fadd_rn(y[2 * e + 1], __uint_as_float(x[e] & 0xFFFF0000u));
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int t = 0; t < TR; ++t)
+        rows[r][t] = *reinterpret_cast<const uint4*>(p.tab[which] + (((int64_t)t * p.H + h) * p.K + kk[r][t]) * kD + c0);
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const float s = dec[sz[r] & 0xFFu];
+    if (p.sym) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[r][e] = __fmul_rn(s, (float)((code[r] >> (2 * e)) & 3u) - 2.0f);
+    } else {
+      const float m = dec[sz[r] >> 8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[r][e] = __fmaf_rn(s, (float)((code[r] >> (2 * e)) & 3u), m);
     }
-  }
+    auto add_row = [&](const uint4 w) {
+      const uint32_t x[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-  for (int e = 0; e < 8; e += 2) {
-    const uint32_t b = pack_bf16(y[e], y[e + 1]);
-    y[e] = __uint_as_float(b << 16);
-    y[e + 1] = __uint_as_float(b & 0xFFFF0000u);
+      for (int e = 0; e < 4; ++e) {
+        y[r][2 * e] = __fadd_rn(y[r][2 * e], __uint_as_float(x[e] << 16));
+        y[r][2 * e + 1] = __fadd_rn(y[r][2 * e + 1], __uint_as_float(x[e] & 0xFFFF0000u));
+      }
+    };
+    if (TT > 0) {
+#pragma unroll
+      for (int t = TR - 1; t >= 0; --t) add_row(rows[r][t]);
+    } else if (TT < 0) {
+      const int64_t tok = tok0 + r < p.Nk ? tok0 + r : p.Nk - 1;
+      for (int t = T - 1; t >= 0; --t) {
+        const int k = min((int)p.assign[which][((int64_t)t * p.H + h) * p.Nk + tok], p.K - 1);
+        add_row(*reinterpret_cast<const uint4*>(p.tab[which] + (((int64_t)t * p.H + h) * p.K + k) * kD + c0));
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const uint32_t b = pack_bf16(y[r][e], y[r][e + 1]);
+      y[r][e] = tok0 + r < p.Nk ? __uint_as_float(b << 16) : 0.0f;
+      y[r][e + 1] = tok0 + r < p.Nk ? __uint_as_float(b & 0xFFFF0000u) : 0.0f;
+    }
   }
 }
 
+template <int TT>
 __global__ void __launch_bounds__(kAtThreads, 1)
 qvg_attention_fused(const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -301,28 +336,22 @@ qvg_attention_fused(const AttnParams p) {
     // 1. reconstruct the K and V tile into the operand layouts
     {
       float vk[8][8];
+      const int64_t tok0 = k0 + 8 * rb;
+      recon_block<TT>(p, dec, 0, h, tok0, 8 * cb, vk);
+      // K rows: rotary embedding of the reconstructed values, then bf16
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        const int ti = 8 * rb + r;
-        const int64_t tok = k0 + ti;
-        float y[8];
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-        if (tok < p.Nk) {
-          recon8(p, dec, 0, h, tok, 8 * cb, y);
+        uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 cs = rope_cs(p, tok, 4 * cb + e);
-            const float a = y[2 * e], b = y[2 * e + 1];
-            w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
-                             __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
-          }
-          recon8(p, dec, 1, h, tok, 8 * cb, vk[r]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) vk[r][e] = 0.0f;
+        for (int e = 0; e < 4; ++e) {
+          const float2 cs = rope_cs(p, tok0 + r, 4 * cb + e);
+          const float a = vk[r][2 * e], b = vk[r][2 * e + 1];
+          w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
+                           __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
         }
-        *reinterpret_cast<uint4*>(sK + op_off(ti, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(sK + op_off(8 * rb + r, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
+      recon_block<TT>(p, dec, 1, h, tok0, 8 * cb, vk);
       // V transposed: channel 8*cb + e holds the 8 keys 8*rb .. 8*rb+7 contiguously
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -477,6 +506,14 @@ cudaError_t launch_rope_tables(void* tables, int n_hi, double base, cudaStream_t
   return cudaGetLastError();
 }
 
+template <int TT>
+static cudaError_t launch_attention_t(const AttnParams& p, dim3 grid, size_t smem, cudaStream_t s) {
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(qvg_attention_fused<TT>), smem);
+  if (e != cudaSuccess) return e;
+  qvg_attention_fused<TT><<<grid, kAtThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s) {
   AttnParams p{};
   for (int w = 0; w < 2; ++w) {
@@ -494,11 +531,15 @@ cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s) {
   p.Nk = a.Nk; p.Nq = a.Nq; p.H = a.H; p.K = a.K; p.T = a.T; p.G = a.G; p.sym = a.sym;
   p.sl = 1.4426950408889634f / sqrtf((float)kD);
   const size_t smem = attention_smem_bytes();
-  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(qvg_attention_fused), smem);
-  if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((a.Nq + kAtTile - 1) / kAtTile), (unsigned)a.H);
-  qvg_attention_fused<<<grid, kAtThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  switch (a.T) {
+    case 0: return launch_attention_t<0>(p, grid, smem, s);
+    case 1: return launch_attention_t<1>(p, grid, smem, s);
+    case 2: return launch_attention_t<2>(p, grid, smem, s);
+    case 3: return launch_attention_t<3>(p, grid, smem, s);
+    case 4: return launch_attention_t<4>(p, grid, smem, s);
+    default: return launch_attention_t<-1>(p, grid, smem, s);
+  }
 }
 
 }  // namespace qvg
