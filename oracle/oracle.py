@@ -68,6 +68,15 @@ def lib():
         L.ref_group_quant_sym.argtypes = [vp, i64, i32, i32, vp, vp]
         L.ref_quantize.restype = i32
         L.ref_quantize.argtypes = [i32, i32, i32, i32, i32, i32, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]
+        L.ref_quantize_ex.restype = i32
+        L.ref_quantize_ex.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, vp, i64, i32, i32, vp,
+                                      vp, vp, vp, vp, vp]
+        L.ref_range_stat.restype = C.c_uint64
+        L.ref_range_stat.argtypes = [vp, i32, i64, i32, i32, i32]
+        L.ref_adaptive_level.restype = i32
+        L.ref_adaptive_level.argtypes = [C.c_uint64, i64, vp, i32]
+        L.ref_adaptive_warm_stages.restype = i32
+        L.ref_adaptive_warm_stages.argtypes = [i32, i32, i32, i32]
         L.ref_dequantize.restype = i32
         L.ref_dequantize.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, i64, i32, i32, vp]
         L.ref_rope.argtypes = [vp, i64, i32, vp, f64, vp]
@@ -226,6 +235,47 @@ def quantize(X, K, T, G, iters, init=None, scale_mode=0):
     if rc != 0:
         raise ValueError("oracle quantize rejected its arguments")
     return out
+
+
+def quantize_ex(X, K, T, G, iters, warm_iters, warm_stages, init=None, scale_mode=0):
+    """quantize with the first warm_stages stages started from init (and
+    warm_iters iterations), the rest cold (iters)."""
+    X = np.ascontiguousarray(X)
+    dtype = _dt(X)
+    H, N, d = X.shape
+    out = dict(
+        codes=np.zeros((H, N, d // 4), np.uint8),
+        scale=np.zeros((H, N, d // G), np.uint8),
+        zero=np.zeros((H, N, d // G) if scale_mode == 0 else (0,), np.uint8),
+        assign=np.zeros((T, H, N), np.uint8),
+        centroids=np.zeros((T, H, K, d), X.dtype),
+    )
+    if init is not None:
+        init = np.ascontiguousarray(init, dtype=X.dtype)
+    rc = lib().ref_quantize_ex(K, T, G, iters, warm_iters, warm_stages, dtype, scale_mode, _p(X), N, H, d,
+                               _p(init) if init is not None else None,
+                               _p(out["codes"]), _p(out["scale"]), _p(out["zero"]) if scale_mode == 0 else None,
+                               _p(out["assign"]), _p(out["centroids"]))
+    if rc != 0:
+        raise ValueError("oracle quantize_ex rejected its arguments")
+    return out
+
+
+def range_stat(X, G) -> int:
+    """Sum of the E4M3 codes of the fp32 ranges (max - min) of every group of
+    G channels of every token of X [H][N][d]."""
+    X = np.ascontiguousarray(X)
+    H, N, d = X.shape
+    return int(lib().ref_range_stat(_p(X), _dt(X), N, H, d, G))
+
+
+def adaptive_level(S, n_groups, thresholds, levels) -> int:
+    th = np.ascontiguousarray(list(thresholds) + [0] * (3 - len(thresholds)), dtype=np.int32)
+    return int(lib().ref_adaptive_level(int(S), int(n_groups), _p(th), int(levels)))
+
+
+def adaptive_warm_stages(chunk, T_prev, T_cur, refresh_every) -> int:
+    return int(lib().ref_adaptive_warm_stages(chunk, T_prev, T_cur, refresh_every))
 
 
 def dequantize(packed, K, T, G, N, H, d, dtype=BF16, scale_mode=0) -> np.ndarray:

@@ -511,10 +511,27 @@ void ref_group_quant_sym(const float* R, int64_t N, int d, int G,
 /* centroids (READING).                                                   */
 /* Returns 0 on success, -1 on invalid arguments.                          */
 /* ------------------------------------------------------------------ */
+int ref_quantize_ex(int K, int T, int G, int iters, int warm_iters, int warm_stages, int dtype,
+                    int scale_mode, const void* X, int64_t N, int H, int d, const void* init,
+                    uint8_t* codes, uint8_t* scale, uint8_t* zero, uint8_t* assign, void* centroids);
+
 int ref_quantize(int K, int T, int G, int iters, int dtype, int scale_mode,
                  const void* X, int64_t N, int H, int d, const void* init,
                  uint8_t* codes, uint8_t* scale, uint8_t* zero,
                  uint8_t* assign, void* centroids)
+{
+    /* every stage warm-started from init when it is given, cold otherwise */
+    return ref_quantize_ex(K, T, G, iters, iters, init ? T : 0, dtype, scale_mode, X, N, H, d, init,
+                           codes, scale, zero, assign, centroids);
+}
+
+/* The codec with the first warm_stages stages started from init[t] (the
+ * previous chunk's tables, [163] 五) and run for warm_iters Lloyd
+ * iterations, the other stages started cold from the first K tokens of their
+ * input and run for iters. */
+int ref_quantize_ex(int K, int T, int G, int iters, int warm_iters, int warm_stages, int dtype,
+                    int scale_mode, const void* X, int64_t N, int H, int d, const void* init,
+                    uint8_t* codes, uint8_t* scale, uint8_t* zero, uint8_t* assign, void* centroids)
 {
     int64_t esz = dtype == REF_FP32 ? 4 : 2;
     int h, t;
@@ -522,8 +539,10 @@ int ref_quantize(int K, int T, int G, int iters, int dtype, int scale_mode,
     if (K < 1 || K > 256 || T < 0 || G < 4 || G % 4 || d % G || d % 4 || N < 1 || H < 1 || iters < 0)
         return -1;
     if (scale_mode != 0 && scale_mode != 1) return -1;
-    if (T > 0 && iters < 1) return -1;     /* assignments need one assign step */
-    if (T > 0 && init == NULL && N < K) return -1;
+    if (warm_stages < 0 || warm_stages > T || (warm_stages > 0 && init == NULL)) return -1;
+    if (T > warm_stages && iters < 1) return -1;   /* assignments need one assign step */
+    if (warm_stages > 0 && warm_iters < 1) return -1;
+    if (T > warm_stages && N < K) return -1;
     R = (float*)malloc((size_t)(N * d) * sizeof(float));
     R2 = (float*)malloc((size_t)(N * d) * sizeof(float));
     C = (float*)malloc((size_t)K * d * sizeof(float));
@@ -533,9 +552,9 @@ int ref_quantize(int K, int T, int G, int iters, int dtype, int scale_mode,
             int64_t tab = ((int64_t)t * H + h) * K * d;
             uint8_t* pi = assign + ((int64_t)t * H + h) * N;
             float* tmp;
-            if (init) load_values((const char*)init + tab * esz, dtype, (int64_t)K * d, C);
+            if (t < warm_stages) load_values((const char*)init + tab * esz, dtype, (int64_t)K * d, C);
             else memcpy(C, R, (size_t)K * d * sizeof(float));
-            ref_kmeans(R, N, d, K, iters, dtype, C, pi, NULL);
+            ref_kmeans(R, N, d, K, t < warm_stages ? warm_iters : iters, dtype, C, pi, NULL);
             store_values(C, dtype, (int64_t)K * d, (char*)centroids + tab * esz);
             ref_residual(R, N, d, C, pi, dtype, R2);
             tmp = R; R = R2; R2 = tmp;
@@ -709,4 +728,59 @@ int ref_attention(const float* Q, const int64_t* qpos, int64_t nq, const float* 
     free(kr);
     free(kpos);
     return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Adaptive per-chunk settings on the streaming path ([163] 九: adapt the */
+/* compression parameters to the content; [163] 五: the streaming        */
+/* centroid cache).  The pages give no rule; READINGS:                    */
+/*   statistic of a chunk: over every block, token and group of           */
+/*     probe_group channels, the sum of the E4M3 codes of the group's     */
+/*     range fl32(max - min) (the code grows with the range, about eight  */
+/*     codes per binade);                                                  */
+/*   level: the number of ascending thresholds theta_j (in sixteenths of */
+/*     a code) with 16 * S > theta_j * (number of groups), so a chunk of  */
+/*     wider ranges takes a later, more expensive setting of the ladder;  */
+/*   centroid reuse: chunk c > 0 starts stage t from chunk c-1's C(t) for */
+/*     t < min(T of c-1, T of c), every other stage cold (first K tokens);*/
+/*     every refresh_every-th chunk (when > 0) starts all stages cold.     */
+/* ------------------------------------------------------------------ */
+uint64_t ref_range_stat(const void* X, int dtype, int64_t N, int H, int d, int G)
+{
+    int64_t esz = dtype == REF_FP32 ? 4 : 2, i;
+    uint64_t S = 0;
+    int h, g, j;
+    float* row = (float*)malloc((size_t)d * sizeof(float));
+    for (h = 0; h < H; ++h)
+        for (i = 0; i < N; ++i) {
+            load_values((const char*)X + ((int64_t)h * N + i) * d * esz, dtype, d, row);
+            for (g = 0; g < d / G; ++g) {
+                float lo = row[g * G], hi = row[g * G];
+                for (j = 1; j < G; ++j) {
+                    if (row[g * G + j] < lo) lo = row[g * G + j];
+                    if (row[g * G + j] > hi) hi = row[g * G + j];
+                }
+                S += ref_e4m3_encode(hi - lo);
+            }
+        }
+    free(row);
+    return S;
+}
+
+/* Level of a chunk from its statistic: the count of thresholds it exceeds. */
+int ref_adaptive_level(uint64_t S, int64_t n_groups, const int* thresholds, int levels)
+{
+    int lvl = 0, j;
+    for (j = 0; j + 1 < levels; ++j)
+        if ((double)S * 16.0 > (double)thresholds[j] * (double)n_groups) lvl = j + 1;
+    return lvl;
+}
+
+/* Stages of chunk `chunk` (with T_cur stages) started from the previous
+ * chunk's tables (which had T_prev stages). */
+int ref_adaptive_warm_stages(int chunk, int T_prev, int T_cur, int refresh_every)
+{
+    if (chunk == 0) return 0;
+    if (refresh_every > 0 && chunk % refresh_every == 0) return 0;
+    return T_prev < T_cur ? T_prev : T_cur;
 }
