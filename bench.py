@@ -41,6 +41,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "KV GB/s: fused dequant + k-means/2-bit quantize, as % of B200 HBM roofline"
 STREAM_METRIC = "streaming append: per-chunk quantize latency (warm start), with whole-cache dequant GB/s"
+ADAPTIVE_METRIC = ("streaming append with per-chunk settings: per-chunk latency (statistic + level + warm "
+                   "start), with whole-cache dequant GB/s and the compression reached")
 SWEEP_METRIC = "design sweep: reconstruction error, compression ratio and per-pass rate over T, G, K"
 
 WORKLOADS = {
@@ -62,6 +64,15 @@ WORKLOADS = {
                            "38,000 cached tokens per head (K=256, T=2, G=64), queries = the next frame (1,520 "
                            "tokens per head), d=128, bf16 operands; fused dequant + RoPE + attention against "
                            "dequantise-then-attend"),
+    "adaptive": dict(layers=1, heads=32, frames=700, chunk_frames=3, gh=30, gw=52, K=256, T=1, G=64,
+                     iters=10, warm_iters=3, adaptive=True, scene_chunks=26, gains=(1.0, 8.0, 0.25),
+                     ladder=("qvg", "qvg-pro"), probe_group=16, threshold_codes=12,
+                     desc="Streaming long generation with per-chunk settings: 1 layer x 32 heads x K/V, "
+                          "700 frames of 30x52 tokens in chunks of 3 frames, scenes of 26 chunks whose "
+                          "values are scaled by 1, 8 or 1/4 in turn, d=128, bf16; one E4M3 scale per group, "
+                          "K=256; each chunk takes QVG (T=1, G=64) or QVG-Pro (T=4, G=16) by its mean "
+                          "group-range code (threshold 12 codes above the first scene's); warm start "
+                          "3 Lloyd iterations in the stages both chunks have, 10 cold"),
     "sweep": dict(layers=1, heads=32, frames=25, gh=38, gw=40, K=256, T=2, G=64, iters=10, sweep=True,
                   desc="Design sweep on one layer: 32 heads x K/V, 38,000 tokens (25 frames x 38x40), "
                        "d=128, bf16; T in {0,1,2,3,4} x G in {16,32,64} x K in {64,256}, 10 Lloyd "
@@ -201,13 +212,13 @@ def oracle_stream_sample(wl, chunks: int, seed: int = 7):
     o.build()
     s = synth.PrototypeStream(1, wl["gh"], wl["gw"], kinds=[1], seed=seed)
     bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
-    K, T, G = wl["K"], wl["T"], wl["G"]
-    prev = o.quantize(bits(s.next(wl["chunk_frames"])), K=K, T=T, G=G, iters=wl["iters"])
+    K, T, G, mode = wl["K"], wl["T"], wl["G"], wl.get("scale_mode", 0)
+    prev = o.quantize(bits(s.next(wl["chunk_frames"])), K=K, T=T, G=G, iters=wl["iters"], scale_mode=mode)
     t = 0.0
     for _ in range(chunks):
         X = bits(s.next(wl["chunk_frames"]))
         t0 = time.perf_counter()
-        prev = o.quantize(X, K=K, T=T, G=G, iters=wl["warm_iters"], init=prev["centroids"])
+        prev = o.quantize(X, K=K, T=T, G=G, iters=wl["warm_iters"], init=prev["centroids"], scale_mode=mode)
         t += time.perf_counter() - t0
     return t / chunks, o.get_threads()
 
@@ -261,6 +272,9 @@ def run_reference(args, wl, rank, world):
         }))
         return
     if "chunk_frames" in wl:
+        adaptive = bool(wl.get("adaptive"))
+        if adaptive:                       # the sample appends at the ladder's first setting
+            wl = dict(wl, T=1, G=64, scale_mode=1)
         times = []
         for i in range(args.warmup + args.steps):
             dt, threads = oracle_stream_sample(wl, 1, seed=1000 + i)
@@ -268,9 +282,10 @@ def run_reference(args, wl, rank, world):
                 times.append(dt)
         v = sum(times) / len(times) * 1e3 * 2 * wl["heads"]
         sample = ("one V block: a cold first chunk (untimed) then one warm-started 4,680-token append per "
-                  f"step; ms scaled by the {2 * wl['heads']} blocks of a chunk")
+                  f"step{' at the QVG setting' if adaptive else ''}; ms scaled by the {2 * wl['heads']} "
+                  "blocks of a chunk")
         print(json.dumps({
-            "impl": "reference", "metric": STREAM_METRIC, "value": v, "unit": "ms", "n_gpus": args.gpus,
+            "impl": "reference", "metric": ADAPTIVE_METRIC if adaptive else STREAM_METRIC, "value": v, "unit": "ms", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl["desc"], "reference": "C oracle (fp64 k-means) on host cores"},
@@ -360,6 +375,12 @@ def main():
         return
     if wl.get("sweep"):
         run_sweep(args, wl, qvg, synth, dev, dist, rank, world, peaks)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+    if wl.get("adaptive"):
+        run_stream_adaptive(args, wl, qvg, synth, dev, dist, rank, world, local, peaks)
         if dist is not None:
             dist.barrier()
             dist.destroy_process_group()
@@ -977,6 +998,157 @@ def run_stream(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
         result["cpu_baseline"] = {"value": dt * 1e3 * U, "unit": "ms", "cores": threads, "kind": "oracle",
                                   "sample": f"one warm-started {sizes[0]}-token append of one V block "
                                             f"({dt:.1f} s), scaled by the {U} blocks of a chunk"}
+    cache.close()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+def scene_gain(wl, c):
+    """Scale of chunk c's values: the scenes of the adaptive stream cycle
+    through the workload's gains (powers of two, exact in bf16)."""
+    g = wl["gains"]
+    return g[(c // wl["scene_chunks"]) % len(g)]
+
+
+def run_stream_adaptive(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
+    """Streaming cache with per-chunk settings (qvg_cache_create_adaptive):
+    every append is bracketed by CUDA events on the launching stream and
+    includes the statistic, its read-back by the host and the quantisation at
+    the chosen level; the whole cache is dequantised after every chunk by the
+    descriptor-driven fused kernel."""
+    import torch
+    Hh = wl["heads"]
+    U = 2 * Hh
+    K = wl["K"]
+    sizes = stream_chunks(wl)
+    total, nch = sum(sizes), len(sizes)
+    levels = [qvg.PRESETS[n] for n in wl["ladder"]]
+    cfg = qvg.config(K=K, T=0, iters=wl["iters"], warm_iters=wl["warm_iters"], scale_mode=qvg.SYM)
+    kinds = [0] * Hh + [1] * Hh
+    seed = synth.unit_seed(rank, 0, 0, 0)
+    stream = torch.cuda.Stream(dev)
+    ybuf = torch.empty(U * total * 128, dtype=torch.bfloat16, device=dev)
+    PG = wl["probe_group"]
+
+    def events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    # the first scene's mean range code, by the library's own statistic (a
+    # one-level cache on a warm-up chunk), sets the threshold; the same
+    # cache's appends are the warm-up
+    gen = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=kinds, seed=seed + 1, device=dev)
+    probe = qvg.policy(T=[levels[0]["T"]], group_size=[levels[0]["group_size"]], probe_group=PG)
+    nw = max(args.warmup, 1)
+    wcache = qvg.Cache(cfg, U, sum(sizes[:nw]), nw, max_chunk_tokens=max(sizes), policy=probe)
+    with torch.cuda.stream(stream):
+        for c in range(nw):
+            wcache.append(gen.next(sizes[c] // (wl["gh"] * wl["gw"])), stream=stream)
+            wcache.dequantize(ybuf[:U * wcache.tokens * 128].view(U, wcache.tokens, 128), stream=stream)
+    torch.cuda.synchronize()
+    base16 = 16 * wcache.chunk_info(0)["stat"] // (U * sizes[0] * 128 // PG)
+    wcache.close()
+    th = [base16 + 16 * wl["threshold_codes"]]
+    pol = qvg.policy(T=[lv["T"] for lv in levels], group_size=[lv["group_size"] for lv in levels],
+                     thresholds=th, probe_group=PG)
+
+    cache = qvg.Cache(cfg, U, total, nch, max_chunk_tokens=max(sizes), policy=pol)
+    gen = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=kinds, seed=seed, device=dev)
+    ea, eb, da, db = events(nch), events(nch), events(nch), events(nch)
+    quality, info = {}, []
+    with ClockSampler(local) as clk:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for c, n in enumerate(sizes):
+                X = gen.next(n // (wl["gh"] * wl["gw"]))
+                X.mul_(scene_gain(wl, c))
+                ea[c].record(stream)
+                cache.append(X, stream=stream)
+                eb[c].record(stream)
+                tok = cache.tokens
+                da[c].record(stream)
+                cache.dequantize(ybuf[:U * tok * 128].view(U, tok, 128), stream=stream)
+                db[c].record(stream)
+                if c % wl["scene_chunks"] in (1, wl["scene_chunks"] - 1):     # a chunk early and late in the scene
+                    Y = ybuf[:U * tok * 128].view(U, tok, 128)[:, tok - n:]
+                    d = Y.float() - X.float()
+                    quality[c] = float((d * d).sum() / (X.float() ** 2).sum())
+        torch.cuda.synchronize()
+    info = [cache.chunk_info(c) for c in range(nch)]
+    append_ms = [ea[c].elapsed_time(eb[c]) for c in range(nch)]
+    deq_ms = [da[c].elapsed_time(db[c]) for c in range(nch)]
+    full = [c for c in range(1, nch) if sizes[c] == sizes[0]]
+    value = max_over_ranks(dist, statistics.median(append_ms[c] for c in full), dev)
+
+    # algorithmic bytes of the whole-cache dequant and the packed size, chunk by chunk
+    def alg_bytes(last):
+        return sum(dequant_alg_bytes(U, sizes[c], 1, K, info[c]["T"], info[c]["G"], scale_bytes=1)
+                   for c in range(last + 1))
+
+    packed = sum(U * sizes[c] * 128 * bits_per_element(K, info[c]["T"], info[c]["G"], sizes[c], scale_bytes=1) / 8
+                 for c in range(nch))
+    by_level = {}
+    for lv, name in enumerate(wl["ladder"]):
+        cs = [c for c in full if info[c]["level"] == lv]
+        by_level[name] = {"chunks": sum(1 for c in range(nch) if info[c]["level"] == lv),
+                          "median_append_ms": statistics.median(append_ms[c] for c in cs) if cs else None,
+                          "relative_mse": {str(c): quality[c] for c in sorted(quality) if info[c]["level"] == lv}}
+    last = nch - 1
+    ach = alg_bytes(last) / (deq_ms[last] / 1e3) / 1e9
+    result = {
+        "metric": ADAPTIVE_METRIC, "value": value, "unit": "ms", "n_gpus": world, "steps": nch,
+        "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl["desc"], "blocks": U, "chunks": nch, "chunk_tokens": sizes[0],
+                   "cache_tokens": total, "threshold_16ths": th[0], "first_scene_mean_code_16ths": base16,
+                   "l2": "every chunk's input (76.7 MB) is freshly generated; dequant outputs up to "
+                         f"{U * total * 256 / 1e9:.1f} GB exceed L2",
+                   "parallelism": f"weak: {world} rank(s), independent caches"},
+        "levels": by_level,
+        "compression": {"reached": U * total * 256 / packed,
+                        "qvg_only": compression_ratio(K, 1, 64, sizes[0], scale_bytes=1),
+                        "qvg_pro_only": compression_ratio(K, 4, 16, sizes[0], scale_bytes=1)},
+        "dequant_vs_length": [{"chunks": c + 1, "ms": deq_ms[c], "GB/s": alg_bytes(c) / (deq_ms[c] / 1e3) / 1e9}
+                              for c in sorted({0, 25, 77, 155, last} & set(range(nch)))],
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": ach / peaks["hbm"], "traffic": None, "kernel": "qvg_dequant_fused",
+                     "at": f"full cache, {total} tokens x {U} blocks, {nch} chunks of their own T and G",
+                     "alg_bytes_per_launch": alg_bytes(last)},
+        "clocks": clk.summary(),
+    }
+    qvg.profile_reset()
+    qvg.profile_enable(True)
+    with torch.cuda.stream(stream):
+        cache.dequantize(ybuf[:U * total * 128].view(U, total, 128), stream=stream)
+    torch.cuda.synchronize()
+    qvg.profile_enable(False)
+    per_dequant = qvg.profile_launches()
+    # one append at each level into a scratch cache: its launches and kernel times
+    scache = qvg.Cache(cfg, U, 4 * sizes[0], 4, max_chunk_tokens=sizes[0], policy=pol)
+    g2 = synth.PrototypeStream(U, wl["gh"], wl["gw"], kinds=kinds, seed=seed + 2, device=dev)
+    per_append, reports = {}, {}
+    with torch.cuda.stream(stream):
+        scache.append(g2.next(wl["chunk_frames"]), stream=stream)
+        for name, gain in (("qvg", 1.0), ("qvg-pro", 8.0)):
+            torch.cuda.synchronize()
+            qvg.profile_reset()
+            qvg.profile_enable(True)
+            scache.append(g2.next(wl["chunk_frames"]).mul_(gain), stream=stream)
+            torch.cuda.synchronize()
+            qvg.profile_enable(False)
+            per_append[wl["ladder"][scache.chunk_info(scache.chunks - 1)["level"]]] = qvg.profile_launches()
+            reports[name] = qvg.profile_report()
+    scache.close()
+    result["kernels_append"] = reports
+    result["gpu_launches"] = per_dequant * nch + sum(
+        per_append.get(wl["ladder"][info[c]["level"]], 0) for c in range(nch))
+    result["gpu_launches_per_chunk"] = {"append": per_append, "dequant": per_dequant}
+    if rank == 0 and not args.no_cpu_baseline:
+        dt, threads = oracle_stream_sample(dict(wl, T=1, G=64, scale_mode=1), 1)
+        result["cpu_baseline"] = {"value": dt * 1e3 * U, "unit": "ms", "cores": threads, "kind": "oracle",
+                                  "sample": f"one warm-started {sizes[0]}-token append of one V block at the "
+                                            f"QVG setting ({dt:.1f} s), scaled by the {U} blocks of a chunk"}
     cache.close()
     if rank == 0:
         print(json.dumps(result))

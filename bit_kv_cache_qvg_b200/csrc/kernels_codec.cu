@@ -166,17 +166,32 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
   const int h = unit % p.H;
   const int c = unit / p.H;
   int64_t o_c = 0, n_c = p.N;
-  if (p.chunk_off != nullptr) {
-    o_c = p.chunk_off[c];
-    n_c = p.chunk_off[c + 1] - o_c;
+  int T = TT < 0 ? p.T : TT, G = p.G;
+  const int K = p.K;
+  const int64_t tab_elems = (int64_t)K * kD;
+  const size_t tab_bytes = (size_t)tab_elems * ESZ;
+  // where the unit's scale/zero bytes, assignments and tables start
+  int64_t sc_row0, as0, tab0;
+  if (p.desc != nullptr) {                       // per-chunk layouts (generic instance only)
+    const ChunkDesc dsc = p.desc[c];
+    o_c = dsc.o; n_c = dsc.n; T = dsc.T; G = dsc.G;
+    sc_row0 = dsc.scale_off / (kD / G) + (int64_t)h * n_c;   // in rows of d/G bytes
+    as0 = dsc.assign_off + (int64_t)h * n_c;
+    tab0 = dsc.table_off;
+  } else {
+    if (p.chunk_off != nullptr) {
+      o_c = p.chunk_off[c];
+      n_c = p.chunk_off[c + 1] - o_c;
+    }
+    sc_row0 = (int64_t)p.H * o_c + (int64_t)h * n_c;
+    as0 = (int64_t)T * p.H * o_c + (int64_t)h * n_c;
+    tab0 = (int64_t)c * T * p.H * tab_elems;
   }
+  const int t_smem = min(p.t_smem, T);
   const int64_t per = (n_c + splits - 1) / splits;
   const int64_t i_begin = (int64_t)part * per;
   const int64_t i_end = min(n_c, i_begin + per);
-  const int K = p.K, T = TT < 0 ? p.T : TT, G = p.G;
-  const int64_t tab_elems = (int64_t)K * kD;
-  const size_t tab_bytes = (size_t)tab_elems * ESZ;
-  const char* tables = static_cast<const char*>(p.centroids) + (int64_t)c * T * p.H * tab_elems * ESZ;
+  const char* tables = static_cast<const char*>(p.centroids) + tab0 * ESZ;
   float* dec = reinterpret_cast<float*>(smem + (size_t)p.t_smem * tab_bytes);   // E4M3 byte -> value
   float2* nlut = reinterpret_cast<float2*>(dec + 256);                          // nibble -> two codes
   if (i_end <= i_begin) return;                                                 // uniform over the block
@@ -185,7 +200,7 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
   if (threadIdx.x < 16)
     nlut[threadIdx.x] = SYM ? make_float2((float)(threadIdx.x & 3u) - 2.0f, (float)(threadIdx.x >> 2) - 2.0f)
                             : make_float2((float)(threadIdx.x & 3u), (float)(threadIdx.x >> 2));
-  for (int t = 0; t < p.t_smem; ++t) {
+  for (int t = 0; t < t_smem; ++t) {
     const uint4* src = reinterpret_cast<const uint4*>(tables + ((int64_t)t * p.H + h) * tab_bytes);
     uint4* dst = reinterpret_cast<uint4*>(smem + (size_t)t * tab_bytes);
     const int n16 = (int)(tab_bytes / 16);
@@ -201,9 +216,9 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
   const int64_t row0 = (int64_t)p.H * o_c + (int64_t)h * n_c + i_begin;
   // per-lane base pointers; a token t of the block is an int offset from them
   const uint16_t* cbp = reinterpret_cast<const uint16_t*>(p.codes + row0 * (kD / 4)) + ql;
-  const uint8_t* scp = p.scale + row0 * ng;
-  const uint8_t* zrp = p.zero + row0 * ng;
-  const uint8_t* ap = p.assign + (int64_t)T * p.H * o_c + (int64_t)h * n_c + i_begin;
+  const uint8_t* scp = p.scale + (sc_row0 + i_begin) * ng;
+  const uint8_t* zrp = p.zero + (sc_row0 + i_begin) * ng;
+  const uint8_t* ap = p.assign + as0 + i_begin;
   const int64_t asg_t = (int64_t)p.H * n_c;
   char* yp = static_cast<char*>(p.Y) + ((int64_t)h * p.y_head_stride + o_c + i_begin) * kD * ESZ + 8 * ql * ESZ;
   const int step = kDqStreams * kDqU;
@@ -265,7 +280,7 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
         k = min(k, K - 1);
         // shared and global rows on separate paths, so that the shared one is
         // addressed as shared memory (st < t_smem is uniform over the block)
-        if (st < p.t_smem) {
+        if (st < t_smem) {
           const char* r = reinterpret_cast<const char*>(smem) + (st * (int)tab_elems + k * kD + 8 * ql) * ESZ;
           Oct<DT>::add(r, y0);
           Oct<DT>::add(r + 64 * ESZ, y1);
@@ -606,6 +621,42 @@ qvg_residual_quant(const ResidualParams p, const int64_t per_block) {
   }
 }
 
+// ---------------------------------------------------------------- range statistic
+// The adaptive cache's per-chunk statistic: over every block, token and
+// group of G channels, the sum of the E4M3 codes of the group's range
+// fl32(max - min).  Sixteen threads per token, thread c owning channels
+// 8c .. 8c+7; a group's extremes are combined over its G/8 threads by
+// xor-shuffles, and its first thread adds the code.  Adding +0 maps a -0
+// range to +0 (the code of a zero range is 0).
+template <int DT>
+__global__ void __launch_bounds__(256)
+qvg_range_stat(const void* X, int64_t rows, int G, unsigned long long* out) {
+  constexpr int ESZ = Store<DT>::bytes;
+  const int c = threadIdx.x & 15;
+  const int64_t row = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4);
+  const bool valid = row < rows;
+  float v[8];
+  Vec8<DT>::load(static_cast<const char*>(X) + ((valid ? row : 0) * kD + 8 * c) * ESZ, v);
+  float lo, hi;
+  minmax8(v, lo, hi);
+  for (int w = 1; w < G / 8; w <<= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, w));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, w));
+  }
+  uint32_t code = 0;
+  if (valid && (c % (G / 8)) == 0) code = f32_to_e4m3(__fadd_rn(__fsub_rn(hi, lo), 0.0f));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) code += __shfl_xor_sync(0xffffffffu, code, off);
+  __shared__ uint32_t part[8];
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = code;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long sum = 0;
+    for (int w = 0; w < 8; ++w) sum += part[w];
+    atomicAdd(out, sum);
+  }
+}
+
 // ---------------------------------------------------------------- centroid init
 template <int DT>
 __global__ void __launch_bounds__(256)
@@ -649,6 +700,15 @@ cudaError_t launch_dequant(const DequantParams& p, int dtype, cudaStream_t s) {
   const size_t smem = (size_t)p.t_smem * p.K * kD * esz + 256 * sizeof(float) + 16 * sizeof(float2);
   const int units = p.n_chunks * p.H;
   if (units == 0) return cudaSuccess;
+  if (p.desc != nullptr) {                       // per-chunk layouts: the generic instance
+    DequantParams q = p;
+    q.T = -1;                                    // selects it below; the kernel reads each chunk's T
+    const int splits = 1;
+    return dtype == kBF16 ? (p.sym ? launch_dq_t<kBF16, true>(q, units * splits, splits, smem, s)
+                                   : launch_dq_t<kBF16, false>(q, units * splits, splits, smem, s))
+                          : (p.sym ? launch_dq_t<kFP32, true>(q, units * splits, splits, smem, s)
+                                   : launch_dq_t<kFP32, false>(q, units * splits, splits, smem, s));
+  }
   const int sms = device_sm_count();
   // One resident block per SM: split blocks along tokens until the grid is
   // about four waves, so that the last one is short and every block stages
@@ -722,6 +782,15 @@ cudaError_t launch_residual(const ResidualParams& p, int dtype, bool quant, cuda
                           : launch_rq<kFP32, true, false>(p, grid, per, smem, s);
   return has_c ? launch_rq<kFP32, false, true>(p, grid, per, smem, s)
                : launch_rq<kFP32, false, false>(p, grid, per, smem, s);
+}
+
+cudaError_t launch_range_stat(const void* X, int64_t rows, int G, int dtype, unsigned long long* out,
+                              cudaStream_t s) {
+  if (rows <= 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((rows + 15) / 16);
+  if (dtype == kBF16) qvg_range_stat<kBF16><<<grid, 256, 0, s>>>(X, rows, G, out);
+  else qvg_range_stat<kFP32><<<grid, 256, 0, s>>>(X, rows, G, out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_init_centroids(const void* src, int64_t src_unit_stride, void* C,

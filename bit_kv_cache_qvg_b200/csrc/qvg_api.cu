@@ -210,12 +210,12 @@ qvg_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QVG_OK : QVG_E
 // kernel from CUDA events recorded on the launching stream around each launch.
 enum Kind {
   K_DEQUANT, K_RESIDUAL, K_RESIDUAL_QUANT, K_ROWNORM, K_INIT, K_ASSIGN_EXACT, K_ASSIGN_TC,
-  K_RECHECK, K_UPD_BUCKET, K_UPD_SUM, K_UPD_CENT, K_ATTN, K_ROPE, K_NKINDS
+  K_RECHECK, K_UPD_BUCKET, K_UPD_SUM, K_UPD_CENT, K_ATTN, K_ROPE, K_STAT, K_NKINDS
 };
 const char* const kKindNames[K_NKINDS] = {
   "qvg_dequant_fused", "qvg_residual", "qvg_residual_quant", "qvg_row_norms", "qvg_init_centroids",
   "qvg_assign_exact", "qvg_kmeans_assign", "qvg_assign_recheck", "qvg_update_bucket", "qvg_update_sum",
-  "qvg_update_centroids", "qvg_attention_fused", "qvg_rope_tables"};
+  "qvg_update_centroids", "qvg_attention_fused", "qvg_rope_tables", "qvg_range_stat"};
 
 struct Profiler {
   std::mutex mu;
@@ -318,12 +318,17 @@ namespace qvg {
 
 qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, int64_t N, int32_t H,
                          int32_t d, const void* init, const qvg_packed* out, void* workspace,
-                         size_t ws_bytes, qvg_stream_t stream_, int max_lanes) {
+                         size_t ws_bytes, qvg_stream_t stream_, int max_lanes, int warm_stages) {
   qvg_status st = check_config(cfg, N, H, d, dtype);
   if (st != QVG_OK) return st;
   const qvg_config c = *cfg;
-  const bool warm = init != nullptr;
-  const int iters = warm ? c.warm_iters : c.iters;
+  // stages t < warm_stages start from init (warm_iters iterations), the
+  // others from the first K tokens of their input (iters iterations)
+  if (warm_stages < 0) warm_stages = init != nullptr ? c.T : 0;
+  if (warm_stages > c.T || (warm_stages > 0 && init == nullptr)) return QVG_ERR_INVALID_ARG;
+  const bool warm = warm_stages > 0;
+  const bool cold = warm_stages < c.T;
+  const int iters = warm ? c.warm_iters : c.iters;   // validated below for the stages that use it
   if (N < 1 || X == nullptr || out == nullptr || workspace == nullptr) return QVG_ERR_INVALID_ARG;
   const bool sym = c.scale_mode == QVG_SCALE_SYM;
   if (out->codes == nullptr || out->scale == nullptr || (out->zero == nullptr && !sym)) return QVG_ERR_INVALID_ARG;
@@ -331,8 +336,9 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
       !aligned(workspace, kAlign))
     return QVG_ERR_INVALID_ARG;
   if (c.T > 0) {
-    if (out->assign == nullptr || out->centroids == nullptr || iters < 1) return QVG_ERR_INVALID_ARG;
-    if (!warm && N < c.K) return QVG_ERR_INVALID_ARG;
+    if (out->assign == nullptr || out->centroids == nullptr) return QVG_ERR_INVALID_ARG;
+    if ((warm && c.warm_iters < 1) || (cold && c.iters < 1) || iters < 1) return QVG_ERR_INVALID_ARG;
+    if (cold && N < c.K) return QVG_ERR_INVALID_ARG;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
   const int dt = (int)dtype;
@@ -397,7 +403,9 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
         QVG_TRY(cudaMemsetAsync(chmax, 0, 2 * (size_t)plan.W * kD * sizeof(uint32_t), s));
         QVG_TRY(plaunch(K_ROWNORM, s, [&] { return launch_residual(nq, dt, false, s); }));
       }
-      if (warm) {
+      const bool stage_warm = t < warm_stages;
+      const int it_t = stage_warm ? c.warm_iters : c.iters;
+      if (stage_warm) {
         const char* src = static_cast<const char*>(init) + ((size_t)t * H + u0) * c.K * kD * esz;
         QVG_TRY(plaunch(K_INIT, s, [&] { return launch_init_centroids(src, (int64_t)c.K * kD, Ct, cn, w, c.K, dt, s); }));
       } else {
@@ -407,8 +415,8 @@ qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, 
       // that the last iteration's lands in pit and the previous one is kept
       // for the incremental update.
       uint8_t* spare = reinterpret_cast<uint8_t*>(ws + plan.off_pi);
-      for (int it = 0; it < iters; ++it) {
-        uint8_t* pi_new = ((iters - 1 - it) % 2 == 0) ? pit : spare;
+      for (int it = 0; it < it_t; ++it) {
+        uint8_t* pi_new = ((it_t - 1 - it) % 2 == 0) ? pit : spare;
         uint8_t* pi_old = it == 0 ? nullptr : (pi_new == pit ? spare : pit);
         AssignParams ap{};
         ap.R = Rin; ap.rnorm2 = rnorm; ap.C = Ct; ap.cn = cn; ap.pi = pi_new;
@@ -494,7 +502,7 @@ extern "C" {
 qvg_status qvg_quantize(const qvg_config* cfg, const void* X, qvg_dtype dtype, int64_t N,
                         int32_t H, int32_t d, const void* init, const qvg_packed* out,
                         void* workspace, size_t ws_bytes, qvg_stream_t stream_) {
-  return qvg::quantize_impl(cfg, X, dtype, N, H, d, init, out, workspace, ws_bytes, stream_, 2);
+  return qvg::quantize_impl(cfg, X, dtype, N, H, d, init, out, workspace, ws_bytes, stream_, 2, -1);
 }
 
 qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packed, qvg_dtype dtype,
@@ -655,13 +663,26 @@ struct qvg_cache {
   void* ws = nullptr;
   size_t ws_bytes = 0;
   size_t bytes = 0;
+  // adaptive caches (qvg_cache_create_adaptive): every chunk has its own
+  // stage count and group size, chosen from the policy's ladder
+  bool adaptive = false;
+  qvg_adaptive_policy pol{};
+  qvg_config level_cfg[4]{};
+  int T_max = 0;
+  ChunkDesc* d_desc = nullptr;              // device [max_chunks]
+  ChunkDesc* h_desc = nullptr;              // pinned [max_chunks], the copies' sources
+  std::vector<int32_t> level;               // per chunk
+  std::vector<uint64_t> stat;               // per chunk
+  unsigned long long* d_stat = nullptr;     // device counter of the range statistic
+  unsigned long long* h_stat = nullptr;     // pinned
+  int64_t next_scale_off = 0, next_assign_off = 0;
 };
 
 static void cache_free(qvg_cache* c) {
   if (c == nullptr) return;
   cudaFree(c->codes); cudaFree(c->scale); cudaFree(c->zero); cudaFree(c->assign);
-  cudaFree(c->tables); cudaFree(c->d_off); cudaFree(c->ws);
-  cudaFreeHost(c->h_off);
+  cudaFree(c->tables); cudaFree(c->d_off); cudaFree(c->ws); cudaFree(c->d_desc); cudaFree(c->d_stat);
+  cudaFreeHost(c->h_off); cudaFreeHost(c->h_desc); cudaFreeHost(c->h_stat);
   delete c;
 }
 
@@ -715,6 +736,15 @@ qvg_status qvg_cache_create(const qvg_config* cfg, qvg_dtype dtype, int32_t H, i
 static void chunk_view(const qvg_cache* c, int chunk, qvg_packed* v) {
   const int64_t o = c->h_off[chunk];
   const size_t esz = (size_t)esize(c->dtype);
+  if (c->adaptive) {                        // this chunk's own layout
+    const ChunkDesc& dsc = c->h_desc[chunk];
+    v->codes = c->codes + (size_t)c->H * o * (kD / 4);
+    v->scale = c->scale + dsc.scale_off;
+    v->zero = c->cfg.scale_mode == QVG_SCALE_SYM ? nullptr : c->zero + dsc.scale_off;
+    v->assign = c->assign + dsc.assign_off;
+    v->centroids = c->tables + (size_t)dsc.table_off * esz;
+    return;
+  }
   const int ng = kD / c->cfg.group_size;
   v->codes = c->codes + (size_t)c->H * o * (kD / 4);
   v->scale = c->scale + (size_t)c->H * o * ng;
@@ -723,11 +753,69 @@ static void chunk_view(const qvg_cache* c, int chunk, qvg_packed* v) {
   v->centroids = c->tables + (size_t)chunk * c->cfg.T * c->H * c->cfg.K * kD * esz;
 }
 
+// The level of a chunk from its range statistic S over n_groups groups: the
+// number of the policy's ascending thresholds (sixteenths of a code) that
+// 16 S exceeds per group.
+static int adaptive_level(const qvg_adaptive_policy& pol, uint64_t S, int64_t n_groups) {
+  int lvl = 0;
+  for (int j = 0; j + 1 < pol.levels; ++j)
+    if ((double)S * 16.0 > (double)pol.thresholds[j] * (double)n_groups) lvl = j + 1;
+  return lvl;
+}
+
+static qvg_status append_adaptive(qvg_cache* c, const void* X, int64_t n, cudaStream_t s) {
+  const int chunk = c->n_chunks;
+  // 1. the chunk's statistic (waits for the stream: the host picks the level)
+  QVG_TRY(cudaMemsetAsync(c->d_stat, 0, sizeof(unsigned long long), s));
+  QVG_TRY(plaunch(K_STAT, s, [&] {
+    return launch_range_stat(X, (int64_t)c->H * n, c->pol.probe_group, c->dtype, c->d_stat, s);
+  }));
+  QVG_TRY(cudaMemcpyAsync(c->h_stat, c->d_stat, sizeof(unsigned long long), cudaMemcpyDeviceToHost, s));
+  QVG_TRY(cudaStreamSynchronize(s));
+  const uint64_t S = *c->h_stat;
+  const int64_t n_groups = (int64_t)c->H * n * (kD / c->pol.probe_group);
+  const int lvl = adaptive_level(c->pol, S, n_groups);
+  const qvg_config& cc = c->level_cfg[lvl];
+  // 2. centroid reuse: the previous chunk's tables for the stages both have
+  int warm = 0;
+  if (chunk > 0 && !(c->pol.refresh_every > 0 && chunk % c->pol.refresh_every == 0))
+    warm = std::min(c->h_desc[chunk - 1].T, cc.T);
+  if (cc.T > warm && n < cc.K) return QVG_ERR_INVALID_ARG;   // a cold stage needs K tokens
+  // 3. this chunk's layout
+  ChunkDesc& dsc = c->h_desc[chunk];
+  dsc.o = c->h_off[chunk];
+  dsc.n = n;
+  dsc.scale_off = c->next_scale_off;
+  dsc.assign_off = c->next_assign_off;
+  dsc.table_off = (int64_t)chunk * c->T_max * c->H * cc.K * kD;
+  dsc.T = cc.T;
+  dsc.G = cc.group_size;
+  qvg_packed v;
+  chunk_view(c, chunk, &v);
+  qvg_packed prev{};
+  if (warm > 0) chunk_view(c, chunk - 1, &prev);
+  qvg_status st = quantize_impl(&cc, X, (qvg_dtype)c->dtype, n, c->H, kD, warm > 0 ? prev.centroids : nullptr, &v,
+                                c->ws, c->ws_bytes, reinterpret_cast<qvg_stream_t>(s), 2, warm);
+  if (st != QVG_OK) return st;
+  // 4. commit: offsets and the chunk's layout travel to the device in stream order
+  c->h_off[chunk + 1] = c->h_off[chunk] + n;
+  QVG_TRY(cudaMemcpyAsync(c->d_off + chunk + 1, &c->h_off[chunk + 1], sizeof(int64_t), cudaMemcpyHostToDevice, s));
+  QVG_TRY(cudaMemcpyAsync(c->d_desc + chunk, &dsc, sizeof(ChunkDesc), cudaMemcpyHostToDevice, s));
+  // scale rows of the next chunk start on a 16-byte boundary (a multiple of any row width)
+  c->next_scale_off += ((int64_t)c->H * n * (kD / cc.group_size) + 15) & ~int64_t(15);
+  c->next_assign_off += (int64_t)cc.T * c->H * n;
+  c->level[chunk] = lvl;
+  c->stat[chunk] = S;
+  c->n_chunks = chunk + 1;
+  return QVG_OK;
+}
+
 qvg_status qvg_append_chunk(qvg_cache* c, const void* X, int64_t n, qvg_stream_t stream_) {
   if (c == nullptr || X == nullptr || n < 1) return QVG_ERR_INVALID_ARG;
   const int chunk = c->n_chunks;
   if (chunk >= c->max_chunks || c->h_off[chunk] + n > c->max_tokens || n > c->max_chunk_tokens)
     return QVG_ERR_CAPACITY;
+  if (c->adaptive) return append_adaptive(c, X, n, reinterpret_cast<cudaStream_t>(stream_));
   if (chunk == 0 && c->cfg.T > 0 && n < c->cfg.K) return QVG_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
   // the workspace was sized at creation for the largest chunk: no allocation here
@@ -762,6 +850,11 @@ qvg_status qvg_cache_dequantize(const qvg_cache* c, void* Y, qvg_stream_t stream
   p.y_head_stride = c->h_off[n_chunks]; p.n_chunks = n_chunks; p.H = c->H;
   p.K = c->cfg.K; p.T = c->cfg.T; p.G = c->cfg.group_size; p.sym = c->cfg.scale_mode == QVG_SCALE_SYM;
   p.t_smem = std::min<int>(c->cfg.T, (int)((160 * 1024) / table));
+  if (c->adaptive) {                 // per-chunk stage counts and group sizes
+    p.desc = c->d_desc;
+    p.T = c->T_max;
+    p.t_smem = std::min<int>(c->T_max, (int)((160 * 1024) / table));
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
   qvg_status st = cuda_status(plaunch(K_DEQUANT, s, [&] { return launch_dequant(p, c->dtype, s); }));
   if (st == QVG_OK && fault_injected("stream")) st = QVG_ERR_CUDA;
@@ -782,6 +875,83 @@ qvg_status qvg_cache_chunk_view(const qvg_cache* c, int32_t chunk, qvg_packed* v
 }
 
 size_t qvg_cache_device_bytes(const qvg_cache* c) { return c ? c->bytes + c->ws_bytes : 0; }
+
+qvg_status qvg_cache_chunk_info(const qvg_cache* c, int32_t chunk, int32_t* level, int32_t* T, int32_t* G,
+                                uint64_t* stat) {
+  if (c == nullptr || chunk < 0 || chunk >= c->n_chunks) return QVG_ERR_INVALID_ARG;
+  if (level) *level = c->adaptive ? c->level[chunk] : 0;
+  if (T) *T = c->adaptive ? c->h_desc[chunk].T : c->cfg.T;
+  if (G) *G = c->adaptive ? c->h_desc[chunk].G : c->cfg.group_size;
+  if (stat) *stat = c->adaptive ? c->stat[chunk] : 0;
+  return QVG_OK;
+}
+
+qvg_status qvg_cache_create_adaptive(const qvg_config* cfg, const qvg_adaptive_policy* pol, qvg_dtype dtype,
+                                     int32_t H, int32_t d, int64_t max_tokens, int32_t max_chunks,
+                                     int64_t max_chunk_tokens, qvg_cache** out) {
+  if (out == nullptr || cfg == nullptr || pol == nullptr) return QVG_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (pol->levels < 1 || pol->levels > 4 || pol->refresh_every < 0) return QVG_ERR_INVALID_ARG;
+  if (!g_supported(pol->probe_group)) return QVG_ERR_INVALID_ARG;
+  for (int j = 0; j + 2 < pol->levels; ++j)
+    if (pol->thresholds[j] > pol->thresholds[j + 1]) return QVG_ERR_INVALID_ARG;
+  if (max_tokens < 1 || max_chunks < 1 || max_chunk_tokens < 0) return QVG_ERR_INVALID_ARG;
+  if (max_chunk_tokens == 0 || max_chunk_tokens > max_tokens) max_chunk_tokens = max_tokens;
+  qvg_config lc[4];
+  int T_max = 0, G_min = 128;
+  size_t ws_bytes = 0;
+  for (int l = 0; l < pol->levels; ++l) {
+    lc[l] = *cfg;
+    lc[l].T = pol->T[l];
+    lc[l].group_size = pol->group_size[l];
+    qvg_status st = check_config(&lc[l], max_tokens, H, d, dtype);
+    if (st != QVG_OK) return st;
+    if (lc[l].T > 0 && (lc[l].iters < 1 || lc[l].warm_iters < 1)) return QVG_ERR_INVALID_ARG;
+    T_max = std::max(T_max, lc[l].T);
+    G_min = std::min(G_min, lc[l].group_size);
+    ws_bytes = std::max(ws_bytes, qvg_workspace_bytes(&lc[l], max_chunk_tokens, H, d, dtype));
+  }
+  if (ws_bytes == 0) return QVG_ERR_INVALID_ARG;
+  if (fault_injected("alloc")) return QVG_ERR_NO_MEMORY;
+  qvg_cache* c = new qvg_cache();
+  c->cfg = lc[0]; c->dtype = (int)dtype; c->H = H; c->max_tokens = max_tokens; c->max_chunks = max_chunks;
+  c->max_chunk_tokens = max_chunk_tokens;
+  c->adaptive = true;
+  c->pol = *pol;
+  for (int l = 0; l < pol->levels; ++l) c->level_cfg[l] = lc[l];
+  c->T_max = T_max;
+  c->level.assign((size_t)max_chunks, 0);
+  c->stat.assign((size_t)max_chunks, 0);
+  const size_t esz = (size_t)esize(c->dtype);
+  const size_t n_codes = (size_t)H * max_tokens * (kD / 4);
+  const size_t n_sc = (size_t)H * max_tokens * (kD / G_min) + 16 * (size_t)max_chunks;
+  const size_t n_zero = cfg->scale_mode == QVG_SCALE_SYM ? 16 : n_sc;
+  const size_t n_as = std::max<size_t>(1, (size_t)T_max * H * max_tokens);
+  const size_t n_tab = std::max<size_t>(16, (size_t)max_chunks * T_max * H * cfg->K * kD * esz);
+  bool ok = cudaMalloc(&c->codes, n_codes) == cudaSuccess && cudaMalloc(&c->scale, n_sc) == cudaSuccess &&
+            cudaMalloc(&c->zero, n_zero) == cudaSuccess && cudaMalloc(&c->assign, n_as) == cudaSuccess &&
+            cudaMalloc(&c->tables, n_tab) == cudaSuccess &&
+            cudaMalloc(&c->d_off, sizeof(int64_t) * ((size_t)max_chunks + 1)) == cudaSuccess &&
+            cudaMemset(c->d_off, 0, sizeof(int64_t) * ((size_t)max_chunks + 1)) == cudaSuccess &&
+            cudaMallocHost(&c->h_off, sizeof(int64_t) * ((size_t)max_chunks + 1)) == cudaSuccess &&
+            cudaMalloc(&c->d_desc, sizeof(ChunkDesc) * (size_t)max_chunks) == cudaSuccess &&
+            cudaMallocHost(&c->h_desc, sizeof(ChunkDesc) * (size_t)max_chunks) == cudaSuccess &&
+            cudaMalloc(&c->d_stat, sizeof(unsigned long long)) == cudaSuccess &&
+            cudaMallocHost(&c->h_stat, sizeof(unsigned long long)) == cudaSuccess &&
+            cudaMalloc(&c->ws, ws_bytes) == cudaSuccess && cudaMemset(c->ws, 0, 16) == cudaSuccess &&
+            cudaDeviceSynchronize() == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    cache_free(c);
+    return QVG_ERR_NO_MEMORY;
+  }
+  c->ws_bytes = ws_bytes;
+  c->bytes = n_codes + n_sc + n_zero + n_as + n_tab + sizeof(int64_t) * ((size_t)max_chunks + 1) +
+             sizeof(ChunkDesc) * (size_t)max_chunks;
+  c->h_off[0] = 0;
+  *out = c;
+  return QVG_OK;
+}
 
 qvg_status qvg_cache_status(qvg_cache* c, qvg_stream_t stream_) {
   if (c == nullptr || c->ws == nullptr) return QVG_ERR_INVALID_ARG;

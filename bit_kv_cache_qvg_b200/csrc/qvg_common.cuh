@@ -77,6 +77,18 @@ struct UnitBatch {
   int dtype;        // kBF16 / kFP32
 };
 
+// One chunk of a cache whose chunks have their own settings (the adaptive
+// cache): its tokens, stage count, group size and where its arrays start.
+struct ChunkDesc {
+  int64_t o;            // first token of the chunk (per head)
+  int64_t n;            // tokens of the chunk (per head)
+  int64_t scale_off;    // byte offset of its [H][n][d/G] scale (and zero) bytes
+  int64_t assign_off;   // byte offset of its [T][H][n] assignments
+  int64_t table_off;    // element offset of its [T][H][K][d] centroid tables
+  int32_t T;            // stages
+  int32_t G;            // group size
+};
+
 // Dequantiser: a set of (chunk, head) units.  A unit's tokens are
 // [chunk_off[c], chunk_off[c+1]) of head h.  Packed arrays are stored chunk by
 // chunk: chunk c holds H*n_c tokens starting at token row H*chunk_off[c]
@@ -91,6 +103,7 @@ struct DequantParams {
   const void* centroids;
   void* Y;
   const int64_t* chunk_off;   // device [n_chunks+1], or nullptr: one chunk of N tokens
+  const ChunkDesc* desc;      // device [n_chunks] per-chunk layouts (adaptive cache), or nullptr
   int64_t N;                  // tokens (single-chunk case)
   int64_t y_head_stride;      // tokens between heads in Y
   int n_chunks;

@@ -12,10 +12,12 @@ namespace qvg {
 
 // ---- launch helpers (qvg_api.cu)
 // qvg_quantize with at most `max_lanes` waves of blocks in flight at once
-// (1: every wave on the caller's stream, with no side stream and no events).
+// (1: every wave on the caller's stream, with no side stream and no events)
+// and the first `warm_stages` stages started from init (-1: every stage when
+// init is given, none otherwise).
 qvg_status quantize_impl(const qvg_config* cfg, const void* X, qvg_dtype dtype, int64_t N, int32_t H,
                          int32_t d, const void* init, const qvg_packed* out, void* workspace,
-                         size_t ws_bytes, qvg_stream_t stream, int max_lanes);
+                         size_t ws_bytes, qvg_stream_t stream, int max_lanes, int warm_stages);
 // SM count of the current device (cached per device).
 int device_sm_count();
 // Host-side fault injection for tests: true when the comma-separated list in
@@ -62,6 +64,11 @@ struct ResidualParams {
   int sym;                 // 1: one E4M3 scale per group (symmetric signed INT2)
 };
 cudaError_t launch_residual(const ResidualParams& p, int dtype, bool quant, cudaStream_t s);
+
+// *out += the sum over `rows` token rows of X of the E4M3 codes of the fp32
+// ranges (max - min) of their groups of G channels (*out must start at zero).
+cudaError_t launch_range_stat(const void* X, int64_t rows, int G, int dtype, unsigned long long* out,
+                              cudaStream_t s);
 
 // C[u] = rows of src[u] (first K rows of a stage input, or given tables);
 // cn[u][k] = |c_k|^2 rounded to fp32 from an fp64 sum.

@@ -79,7 +79,8 @@ extern "C" QVG_API qvg_status qvg_quantize_static(const qvg_config* cfg, const v
   // The same checks and kernels as qvg_quantize, one wave at a time on the
   // caller's stream (no side stream, no events); a timeout recorded in the
   // reserve by earlier, completed work is returned before anything is queued.
-  return qvg::quantize_impl(cfg, X, dtype, N, H, d, init_centroids, out, scratch, kStaticScratchBytes, stream, 1);
+  return qvg::quantize_impl(cfg, X, dtype, N, H, d, init_centroids, out, scratch, kStaticScratchBytes, stream, 1,
+                           -1);
 }
 
 extern "C" QVG_API qvg_status qvg_static_status(qvg_stream_t stream) {

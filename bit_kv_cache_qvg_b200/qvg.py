@@ -46,6 +46,27 @@ class Config(C.Structure):
                 f"iters={self.iters}, warm_iters={self.warm_iters}, scale_mode={self.scale_mode})")
 
 
+class Policy(C.Structure):
+    """qvg_adaptive_policy: a ladder of (T, group_size) settings chosen per
+    chunk from the mean E4M3 code of the chunk's group ranges."""
+    _fields_ = [("levels", C.c_int32), ("T", C.c_int32 * 4), ("group_size", C.c_int32 * 4),
+                ("thresholds", C.c_int32 * 3), ("probe_group", C.c_int32), ("refresh_every", C.c_int32)]
+
+
+def policy(T, group_size, thresholds=(), probe_group=16, refresh_every=0) -> Policy:
+    """A policy of len(T) levels; thresholds in sixteenths of an E4M3 code."""
+    p = Policy()
+    p.levels = len(T)
+    if not 1 <= p.levels <= 4 or len(group_size) != p.levels or len(thresholds) != p.levels - 1:
+        raise QvgError(1, "policy: 1-4 levels, one group size per level, levels - 1 thresholds")
+    for i in range(p.levels):
+        p.T[i], p.group_size[i] = T[i], group_size[i]
+    for i, t in enumerate(thresholds):
+        p.thresholds[i] = t
+    p.probe_group, p.refresh_every = probe_group, refresh_every
+    return p
+
+
 class _Packed(C.Structure):
     _fields_ = [("codes", C.c_void_p), ("scale", C.c_void_p), ("zero", C.c_void_p),
                 ("assign", C.c_void_p), ("centroids", C.c_void_p)]
@@ -69,6 +90,10 @@ _SIGS = {
     "qvg_workspace_flagged": (C.c_int64, [C.c_void_p, C.c_size_t, C.c_void_p]),
     "qvg_cache_create": (C.c_int, [C.POINTER(Config), C.c_int, C.c_int32, C.c_int32, C.c_int64, C.c_int32,
                                    C.c_int64, C.POINTER(C.c_void_p)]),
+    "qvg_cache_create_adaptive": (C.c_int, [C.POINTER(Config), C.POINTER(Policy), C.c_int, C.c_int32, C.c_int32,
+                                            C.c_int64, C.c_int32, C.c_int64, C.POINTER(C.c_void_p)]),
+    "qvg_cache_chunk_info": (C.c_int, [C.c_void_p, C.c_int32, C.POINTER(C.c_int32), C.POINTER(C.c_int32),
+                                       C.POINTER(C.c_int32), C.POINTER(C.c_uint64)]),
     "qvg_cache_status": (C.c_int, [C.c_void_p, C.c_void_p]),
     "qvg_static_status": (C.c_int, [C.c_void_p]),
     "qvg_append_chunk": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p]),
@@ -328,16 +353,29 @@ def _view(ptr, shape, torch_dtype):
 
 class Cache:
     """Streaming compressed KV cache (qvg_cache_*): append chunks, each
-    warm-started from the previous chunk's centroids; dequantise all."""
+    warm-started from the previous chunk's centroids; dequantise all.  With a
+    Policy (qvg_cache_create_adaptive) every chunk takes its own T and G."""
 
     def __init__(self, cfg: Config, H: int, max_tokens: int, max_chunks: int, d: int = 128,
-                 dtype: int = BF16, max_chunk_tokens: int = 0):
-        self.cfg, self.H, self.d, self.dtype = cfg, H, d, dtype
+                 dtype: int = BF16, max_chunk_tokens: int = 0, policy: Optional[Policy] = None):
+        self.cfg, self.H, self.d, self.dtype, self.policy = cfg, H, d, dtype, policy
         self._h = C.c_void_p()
         h = C.c_void_p()
-        _check(lib().qvg_cache_create(C.byref(cfg), dtype, H, d, max_tokens, max_chunks, max_chunk_tokens,
-                                      C.byref(h)), "qvg_cache_create")
+        if policy is None:
+            _check(lib().qvg_cache_create(C.byref(cfg), dtype, H, d, max_tokens, max_chunks, max_chunk_tokens,
+                                          C.byref(h)), "qvg_cache_create")
+        else:
+            _check(lib().qvg_cache_create_adaptive(C.byref(cfg), C.byref(policy), dtype, H, d, max_tokens,
+                                                   max_chunks, max_chunk_tokens, C.byref(h)),
+                   "qvg_cache_create_adaptive")
         self._h = h
+
+    def chunk_info(self, c: int) -> dict:
+        """qvg_cache_chunk_info: level, T, G and statistic of chunk c."""
+        lvl, T, G, S = C.c_int32(), C.c_int32(), C.c_int32(), C.c_uint64()
+        _check(lib().qvg_cache_chunk_info(self._h, c, C.byref(lvl), C.byref(T), C.byref(G), C.byref(S)),
+               "qvg_cache_chunk_info")
+        return dict(level=lvl.value, T=T.value, G=G.value, stat=S.value)
 
     def append(self, X: torch.Tensor, stream=None):
         if X.dim() != 3 or X.shape[0] != self.H or X.shape[2] != self.d or not X.is_contiguous():
@@ -372,6 +410,10 @@ class Cache:
         _check(lib().qvg_cache_chunk_view(self._h, c, C.byref(v), C.byref(first), C.byref(n)),
                "qvg_cache_chunk_view")
         H, d, N, cfg = self.H, self.d, n.value, self.cfg
+        if self.policy is not None:             # the chunk's own settings
+            info = self.chunk_info(c)
+            cfg = config(K=cfg.K, T=info["T"], group_size=info["G"], bits=cfg.bits, iters=cfg.iters,
+                         warm_iters=cfg.warm_iters, scale_mode=cfg.scale_mode)
         G, T, K = cfg.group_size, cfg.T, cfg.K
         return Packed(codes=_view(v.codes, (H, N, d // 4), torch.uint8),
                       scale=_view(v.scale, (H, N, d // G), torch.uint8),

@@ -365,6 +365,46 @@ QVG_API int32_t qvg_cache_chunks(const qvg_cache* cache);   /* chunks so far */
 QVG_API qvg_status qvg_cache_chunk_view(const qvg_cache* cache, int32_t chunk, qvg_packed* view,
                                 int64_t* first_token, int64_t* n_tokens);
 
+/* Settings chosen chunk by chunk (the m.163.com article, section 九, names
+ * adapting the compression parameters to the content as future work; the
+ * rule below is this library's).  A ladder of up to four settings (stage
+ * count and group size; the other fields of the cache's qvg_config are
+ * shared) from the cheapest to the most expensive.  For each chunk the
+ * cache first sums, over every block, token and group of probe_group
+ * channels, the E4M3 code of the group's range fl32(max - min) (about eight
+ * codes per doubling of the range): the statistic S.  The chunk takes the
+ * level equal to the number of thresholds (ascending, in sixteenths of a
+ * code) that 16 S exceeds per group, i.e. the mean range code.  Centroid
+ * reuse: chunk c > 0 starts stage t from chunk c-1's tables when both have
+ * that stage (warm_iters iterations), every other stage from its first K
+ * tokens (iters); every refresh_every-th chunk (when > 0) starts cold. */
+typedef struct {
+    int32_t levels;          /* 1 .. 4 */
+    int32_t T[4];            /* stages of each level */
+    int32_t group_size[4];   /* G of each level */
+    int32_t thresholds[3];   /* levels - 1 ascending thresholds, sixteenths of an E4M3 code */
+    int32_t probe_group;     /* group size of the statistic */
+    int32_t refresh_every;   /* cold start every n-th chunk; 0 = never */
+} qvg_adaptive_policy;
+
+/* A cache whose chunks take their settings from `pol` (cfg gives K, bits,
+ * iters, warm_iters and scale_mode; its T and group_size are ignored).
+ * Storage is sized for the ladder's largest stage count and smallest group.
+ * qvg_append_chunk on it waits for `stream` once per chunk (the statistic
+ * is read by the host, which picks the level) and returns INVALID_ARG for a
+ * chunk with fewer than K tokens that needs a cold stage; the views of
+ * qvg_cache_chunk_view use each chunk's own T and G (qvg_cache_chunk_info).
+ * Errors as qvg_cache_create, and INVALID_ARG for a bad policy. */
+QVG_API qvg_status qvg_cache_create_adaptive(const qvg_config* cfg, const qvg_adaptive_policy* pol,
+                                     qvg_dtype dtype, int32_t H, int32_t d, int64_t max_tokens,
+                                     int32_t max_chunks, int64_t max_chunk_tokens, qvg_cache** out);
+
+/* Settings of chunk `chunk`: its level in the policy's ladder, stage count,
+ * group size and statistic (0, the cache's T and G, and 0 for a cache
+ * without a policy).  Any pointer may be NULL.  Errors: INVALID_ARG. */
+QVG_API qvg_status qvg_cache_chunk_info(const qvg_cache* cache, int32_t chunk, int32_t* level, int32_t* T,
+                                int32_t* G, uint64_t* stat);
+
 /* Bytes of device memory the cache holds (packed storage + workspace). */
 QVG_API size_t qvg_cache_device_bytes(const qvg_cache* cache);
 

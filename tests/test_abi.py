@@ -156,6 +156,45 @@ def test_fault_injection_follows_argument_checks(q, monkeypatch):
     assert q.status_string(5) == "device-side wait timed out"
 
 
+def test_adaptive_cache_rejects_bad_policies_without_touching_the_gpu(q, monkeypatch):
+    """qvg_cache_create_adaptive checks the policy and every level's setting
+    before any device work: 1-4 levels, ascending thresholds, a supported
+    probe group, a non-negative refresh period, a valid (T, G) per level.
+    With QVG_FAULT_INJECT=alloc a valid policy reaches the allocation and
+    reports NO_MEMORY, leaving no handle."""
+    cfg = q.config(K=16, T=9, group_size=7, iters=4, warm_iters=2)   # T and G come from the policy
+    L = q.lib()
+    h = C.c_void_p()
+
+    def create(pol, **kw):
+        a = dict(dtype=0, H=2, d=128, max_tokens=1000, max_chunks=4, max_chunk_tokens=0)
+        a.update(kw)
+        return L.qvg_cache_create_adaptive(C.byref(cfg), C.byref(pol), a["dtype"], a["H"], a["d"],
+                                           a["max_tokens"], a["max_chunks"], a["max_chunk_tokens"], C.byref(h))
+
+    good = q.policy(T=[1, 2], group_size=[64, 16], thresholds=[16 * 50])
+    bad = [q.policy(T=[1, 2, 4], group_size=[64, 32, 16], thresholds=[900, 800]),   # descending
+           q.policy(T=[1, 2], group_size=[64, 16], thresholds=[800], probe_group=12),
+           q.policy(T=[1, 2], group_size=[64, 16], thresholds=[800], refresh_every=-1),
+           q.policy(T=[1, 2], group_size=[64, 24], thresholds=[800]),            # G does not divide d
+           q.policy(T=[1, 9], group_size=[64, 16], thresholds=[800])]            # T above 8
+    zero = q.policy(T=[1], group_size=[64])
+    zero.levels = 0
+    five = q.policy(T=[1], group_size=[64])
+    five.levels = 5
+    for pol in bad + [zero, five]:
+        assert create(pol) in (1, 2), pol
+    assert create(good, d=96) == 1                 # 64 does not divide 96
+    assert create(good, max_tokens=0) == 1
+    assert L.qvg_cache_create_adaptive(C.byref(cfg), None, 0, 2, 128, 1000, 4, 0, C.byref(h)) == 1
+    assert not h.value
+    monkeypatch.setenv("QVG_FAULT_INJECT", "alloc")
+    assert create(good) == 3 and not h.value
+    with pytest.raises(q.QvgError):
+        q.policy(T=[1, 2], group_size=[64], thresholds=[1])
+    assert L.qvg_cache_chunk_info(None, 0, None, None, None, None) == 1
+
+
 def test_status_queries_reject_missing_objects(q):
     L = q.lib()
     assert L.qvg_cache_status(None, None) == 1

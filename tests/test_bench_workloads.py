@@ -3,6 +3,7 @@ schedule (700 frames in chunks of 3, the last chunk of 1 frame) and the
 algorithmic bytes of one fused dequant of the growing cache; the design
 sweep's closed-form compression ratio; and the oracle reference arm of both
 lines (run on the host cores)."""
+import math
 import os
 import sys
 
@@ -71,7 +72,18 @@ def test_sweep_grid_covers_the_design_space():
     assert abs(bench.bits_per_element(256, 2, 64, 38000) - (2 + 0.25 + 0.125 + 16 * 2 * 256 / 38000)) < 1e-12
 
 
-@pytest.mark.parametrize("workload", ["stream", "sweep"])
+def test_adaptive_stream_scenes_cycle_through_the_gains():
+    """Scenes of 26 chunks scaled by 1, 8 and 1/4 in turn (powers of two, so
+    the bf16 inputs are scaled exactly); the ladder is the two named points."""
+    wl = bench.WORKLOADS["adaptive"]
+    gains = [bench.scene_gain(wl, c) for c in range(len(bench.stream_chunks(wl)))]
+    assert gains[:26] == [1.0] * 26 and gains[26:52] == [8.0] * 26 and gains[52:78] == [0.25] * 26
+    assert gains[78] == 1.0 and len(gains) == 234
+    assert all(math.frexp(g)[0] == 0.5 for g in set(gains))
+    assert tuple(wl["ladder"]) == ("qvg", "qvg-pro")
+
+
+@pytest.mark.parametrize("workload", ["stream", "sweep", "adaptive"])
 def test_reference_arm_prints_one_line(workload):
     """--impl reference runs the oracle on the host cores and prints the
     workload's own metric with the reference keys (no GPU involved)."""
@@ -82,7 +94,8 @@ def test_reference_arm_prints_one_line(workload):
                          capture_output=True, text=True, timeout=600, check=True).stdout.strip().splitlines()
     line = json.loads(out[-1])
     assert line["impl"] == "reference" and line["value"] > 0
-    assert line["metric"] == (bench.STREAM_METRIC if workload == "stream" else bench.SWEEP_METRIC)
+    assert line["metric"] == {"stream": bench.STREAM_METRIC, "sweep": bench.SWEEP_METRIC,
+                              "adaptive": bench.ADAPTIVE_METRIC}[workload]
     for key in ("unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "cpu_baseline", "e2e"):
         assert key in line
     assert line["cpu_baseline"]["kind"] == "oracle"

@@ -1,6 +1,7 @@
 """qvg_attention (the consumer of the compressed cache, with dequantisation
 and the rotary embedding fused into the K/V load) against the oracle's fp64
-attention over the oracle's reconstruction of the same packed caches.
+attention over the oracle's reconstruction of the same packed caches (the
+oracle's own compression of seeded K and V blocks).
 
 Tolerance, from the arithmetic of the kernel: the rotated queries and keys
 enter the tensor cores rounded to bf16 (relative error 2^-9 each), so a score
@@ -15,7 +16,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import np_bits, packed_np, values
+from gpu_util import np_bits, to_dev, values
 
 pytestmark = pytest.mark.gpu
 
@@ -35,8 +36,13 @@ def _run_case(q, ora, cfg, H, Nk, Nq, q_scale, seed, base=10000.0):
     frames = -(-Nk // 1560)
     Xk = synth.block_batch(H, synth.KVShape(frames, 30, 52), seed=seed, kinds=[0] * H)[:, :Nk].contiguous()
     Xv = synth.block_batch(H, synth.KVShape(frames, 30, 52), seed=seed + 1, kinds=[1] * H)[:, :Nk].contiguous()
-    kp = q.quantize(Xk.cuda(), cfg)
-    vp = q.quantize(Xv.cuda(), cfg)
+    # the caches are the oracle's own packed streams of the seeded blocks
+    mode = cfg.scale_mode
+    kn = ora.quantize(np_bits(Xk), K=cfg.K, T=cfg.T, G=cfg.group_size, iters=cfg.iters, scale_mode=mode)
+    vn = ora.quantize(np_bits(Xv), K=cfg.K, T=cfg.T, G=cfg.group_size, iters=cfg.iters, scale_mode=mode)
+    kp, vp = (q.Packed(codes=to_dev(p["codes"]), scale=to_dev(p["scale"]), zero=to_dev(p["zero"]),
+                       assign=to_dev(p["assign"]), centroids=to_dev(p["centroids"]),
+                       cfg=cfg, N=Nk, H=H, d=128, dtype=0) for p in (kn, vn))
     rng = np.random.default_rng(seed)
     Qf = (rng.standard_normal((H, Nq, 128)) * q_scale).astype(np.float32)
     Q = torch.from_numpy(Qf).to(torch.bfloat16)
@@ -46,8 +52,6 @@ def _run_case(q, ora, cfg, H, Nk, Nq, q_scale, seed, base=10000.0):
     torch.cuda.synchronize()
     assert q.workspace_status(tables) == 0
     O = O.cpu().numpy()
-    kn, vn = packed_np(kp), packed_np(vp)
-    mode = cfg.scale_mode
     Kh = values(ora.dequantize(kn, K=cfg.K, T=cfg.T, G=cfg.group_size, N=Nk, H=H, d=128, scale_mode=mode))
     Vh = values(ora.dequantize(vn, K=cfg.K, T=cfg.T, G=cfg.group_size, N=Nk, H=H, d=128, scale_mode=mode))
     Qv = values(np_bits(Q))

@@ -40,6 +40,7 @@ def _rand_packed(rng, K, T, G, N, H, dtype, scale_mode=0):
 
 @pytest.mark.parametrize("dtype,T,G,K,N,H,mode", [
     (BF16, 2, 64, 256, 4680, 3, 0),
+    (BF16, 2, 64, 256, 38000, 8, 0),      # the full-size batch, in the benchmark's launch configuration
     (BF16, 0, 16, 1, 777, 2, 0),
     (BF16, 1, 8, 7, 130, 3, 0),
     (BF16, 3, 32, 256, 1000, 2, 0),       # third table read from L2
@@ -78,8 +79,8 @@ def _run(q, ora, X, K, T, G, iters, init=None, warm_iters=None, mode=0):
                        init=init, scale_mode=mode)
     H, N, d = X_np.shape
     Yr = ora.dequantize(ref, K=K, T=T, G=G, N=N, H=H, d=d, dtype=dtype, scale_mode=mode)
-    Yo = ora.dequantize(gpu, K=K, T=T, G=G, N=N, H=H, d=d, dtype=dtype, scale_mode=mode)
-    np.testing.assert_array_equal(Yg, Yo)     # GPU dequant of its own stream == oracle dequant
+    compare_quantize(ora, X_np, gpu, ref, K, T, G, iters, dtype)   # the packed streams first
+    np.testing.assert_array_equal(Yg, Yr)     # then the GPU's reconstruction of its own stream
     return X_np, gpu, ref, Yg, Yr, dtype
 
 
@@ -175,8 +176,9 @@ def test_streaming_cache_parity(q, ora, K, H, frames):
         gpu = packed_np(cache.chunk(c))
         torch.cuda.synchronize()
         compare_quantize(ora, X_np, gpu, ref, K, T, G, I if prev is None else Iw, BF16, init=prev)
-        prev = gpu["centroids"]
-        Ys.append(ora.dequantize(gpu, K=K, T=T, G=G, N=X_np.shape[1], H=H, d=128))
+        assert cache.chunk_info(c) == dict(level=0, T=T, G=G, stat=0)
+        prev = ref["centroids"]                        # the oracle chains its own chunks
+        Ys.append(ora.dequantize(ref, K=K, T=T, G=G, N=X_np.shape[1], H=H, d=128))
     assert cache.tokens == sum(frames) * 1560 and cache.chunks == len(frames)
     assert cache.status() == 0
     Y = np_bits(cache.dequantize())
@@ -187,11 +189,11 @@ def test_streaming_cache_parity(q, ora, K, H, frames):
     cache.close()
 
 
-def test_full_size_sampled(q, ora):
+def test_full_size_every_block(q, ora):
     """LongCat-scale blocks (38,000 tokens = 25 frames of 38x40, K=256, T=2,
     G=64, 10 iterations) quantised in the benchmark's batch configuration;
-    one block checked against the oracle in full, the reconstruction of every
-    block checked against the oracle's reconstruction of the GPU stream."""
+    every block (K and V kinds alternating) checked against the oracle in
+    full: packed streams bit-exact, reconstructions identical."""
     from bit_kv_cache_qvg_b200 import synth
     H = 8
     X = synth.block_batch(H, synth.KVShape(25, 38, 40), seed=1234, kinds=[h % 2 for h in range(H)],
@@ -202,15 +204,12 @@ def test_full_size_sampled(q, ora):
     torch.cuda.synchronize()
     gpu = packed_np(pg)
     X_np = np_bits(X)
-    Yo = ora.dequantize(gpu, K=256, T=2, G=64, N=38000, H=H, d=128)
-    np.testing.assert_array_equal(Yg, Yo)
-    h = 5                                            # a V block (outliers x1000)
-    sub = {k: (v[:, h:h + 1] if k in ("assign", "centroids") else v[h:h + 1]) for k, v in gpu.items()}
-    ref = ora.quantize(X_np[h:h + 1], K=256, T=2, G=64, iters=10)
-    rep = compare_quantize(ora, X_np[h:h + 1], sub, ref, 256, 2, 64, 10, BF16)
-    Yr = ora.dequantize(ref, K=256, T=2, G=64, N=38000, H=1, d=128)
-    compare_reconstruction(ora, X_np[h:h + 1], Yg[h:h + 1], Yr, sub, ref, 64)
-    print(rep)
+    for h in range(H):
+        sub = {k: (v[:, h:h + 1] if k in ("assign", "centroids") else v[h:h + 1]) for k, v in gpu.items()}
+        ref = ora.quantize(X_np[h:h + 1], K=256, T=2, G=64, iters=10)
+        compare_quantize(ora, X_np[h:h + 1], sub, ref, 256, 2, 64, 10, BF16)
+        Yr = ora.dequantize(ref, K=256, T=2, G=64, N=38000, H=1, d=128)
+        np.testing.assert_array_equal(Yg[h:h + 1], Yr)
 
 
 def _bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -475,7 +474,7 @@ def test_symmetric_streaming_cache(q, ora):
         gpu = packed_np(cache.chunk(c))
         torch.cuda.synchronize()
         compare_quantize(ora, X_np, gpu, ref, 256, 1, 64, it, BF16, init=prev)
-        prev = gpu["centroids"]
-        Ys.append(ora.dequantize(gpu, K=256, T=1, G=64, N=X_np.shape[1], H=H, d=128, scale_mode=1))
+        prev = ref["centroids"]
+        Ys.append(ora.dequantize(ref, K=256, T=1, G=64, N=X_np.shape[1], H=H, d=128, scale_mode=1))
     np.testing.assert_array_equal(np_bits(cache.dequantize()), np.concatenate(Ys, axis=1))
     cache.close()
