@@ -104,17 +104,20 @@ __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
 // half, so the shared-memory tables are read without bank conflicts, and
 // they write two coalesced 128-byte halves of the output row.  Each group of
 // eight lanes walks kDqU tokens per step and keeps the codes, scale/zero bytes
-// and assignments of the next kDqDepth steps in flight.  E4M3
-// bytes are decoded through a 256-entry shared table; a nibble of codes (two
-// channels) maps to a pair of floats through a 16-entry table.
-constexpr int kDqThreads = 768;
+// and assignments of the next kDqDepth - 1 steps in flight, every byte in a
+// register of its own, so that nothing waits on a load before the step that
+// uses it.  E4M3 bytes are decoded by the hardware conversion; a nibble of
+// codes (two channels) maps to a pair of floats through a 16-entry table.
+// Fewer threads than the SM holds leave each more registers for the bytes in
+// flight, which is what the kernel is short of.
+constexpr int kDqThreads = 640;
 constexpr int kDqWarps = kDqThreads / 32;
 constexpr int kDqStreams = 4 * kDqWarps;        // token streams per block (8 lanes each)
 
 // tokens per stream per step, and steps whose loads are in flight (fewer
 // when more assignment bytes are held per token)
 template <int TT> constexpr int dq_unroll() { return 2; }
-template <int TT> constexpr int dq_depth() { return (TT < 0 || TT >= 3) ? 3 : 4; }
+template <int TT> constexpr int dq_depth() { return 2; }
 
 template <int DT> struct Oct;                   // a lane's 8 channels of a row
 template <> struct Oct<kBF16> {
@@ -149,6 +152,18 @@ template <> struct Oct<kFP32> {
     reinterpret_cast<float4*>(row)[1] = make_float4(y[2].x, y[2].y, y[3].x, y[3].y);
   }
 };
+
+// Two E4M3 bytes (low byte first) as fp32 values, through the hardware
+// conversion to f16 (exact for every finite E4M3 value) and then to fp32.
+__device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t pair16) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 a;\n\tcvt.u16.u32 a, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\t}" : "=r"(h) : "r"(pair16));
+  float lo, hi;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h));
+  return make_float2(lo, hi);
+}
 
 // TT = number of stages when it is <= 4 (assignments fetched a step ahead
 // with the codes), or -1 for the generic runtime-T loop.
@@ -192,10 +207,8 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
   const int64_t i_begin = (int64_t)part * per;
   const int64_t i_end = min(n_c, i_begin + per);
   const char* tables = static_cast<const char*>(p.centroids) + tab0 * ESZ;
-  float* dec = reinterpret_cast<float*>(smem + (size_t)p.t_smem * tab_bytes);   // E4M3 byte -> value
-  float2* nlut = reinterpret_cast<float2*>(dec + 256);                          // nibble -> two codes
-  if (i_end <= i_begin) return;                                                 // uniform over the block
-  for (int x = threadIdx.x; x < 256; x += blockDim.x) dec[x] = e4m3_to_f32((uint8_t)x);
+  float2* nlut = reinterpret_cast<float2*>(smem + (size_t)p.t_smem * tab_bytes);  // nibble -> two codes
+  if (i_end <= i_begin) return;                                                  // uniform over the block
   // the symmetric mode reads the codes as u - 2
   if (threadIdx.x < 16)
     nlut[threadIdx.x] = SYM ? make_float2((float)(threadIdx.x & 3u) - 2.0f, (float)(threadIdx.x >> 2) - 2.0f)
@@ -225,58 +238,60 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
 
   // codes (two 16-bit words), scale/zero bytes of both halves and (TT > 0)
   // assignments of tokens t0..t0+kDqU-1 (past the block's end: token 0 again;
-  // nothing is stored for those)
-  auto load = [&](int t0, uint32_t (&cb)[kDqU], uint32_t (&sz)[kDqU], uint32_t (&ka)[kDqU]) {
+  // nothing is stored for those), each in a register of its own: they are
+  // combined only by the step that uses them
+  struct Pre {
+    uint32_t c0, c1, s0, z0, s1, z1;
+    uint32_t k[TR];
+  };
+  auto load = [&](int t0, Pre (&pr)[kDqU]) {
 #pragma unroll
     for (int u = 0; u < kDqU; ++u) {
       const int t = t0 + u < nt ? t0 + u : 0;
-      cb[u] = (uint32_t)cbp[t * (kD / 8)] | ((uint32_t)cbp[t * (kD / 8) + 8] << 16);
-      if (SYM)
-        sz[u] = (uint32_t)scp[t * ng + g0] | ((uint32_t)scp[t * ng + g1] << 16);
-      else
-        sz[u] = (uint32_t)scp[t * ng + g0] | ((uint32_t)zrp[t * ng + g0] << 8) |
-                ((uint32_t)scp[t * ng + g1] << 16) | ((uint32_t)zrp[t * ng + g1] << 24);
-      uint32_t kw = 0;
-      if (TT > 0) {
+      pr[u].c0 = cbp[t * (kD / 8)];
+      pr[u].c1 = cbp[t * (kD / 8) + 8];
+      pr[u].s0 = scp[t * ng + g0];
+      pr[u].s1 = scp[t * ng + g1];
+      pr[u].z0 = SYM ? 0u : (uint32_t)zrp[t * ng + g0];
+      pr[u].z1 = SYM ? 0u : (uint32_t)zrp[t * ng + g1];
 #pragma unroll
-        for (int tt = 0; tt < TR; ++tt) kw |= (uint32_t)ap[tt * asg_t + t] << (8 * tt);
-      }
-      ka[u] = kw;
+      for (int tt = 0; tt < TR; ++tt) pr[u].k[tt] = TT > 0 ? (uint32_t)ap[tt * asg_t + t] : 0u;
     }
   };
-  auto process = [&](int tb, const uint32_t (&cb)[kDqU], const uint32_t (&sz)[kDqU], const uint32_t (&ka)[kDqU]) {
+  auto process = [&](int tb, const Pre (&pr)[kDqU]) {
 #pragma unroll
     for (int u = 0; u < kDqU; ++u) {
       const int t = tb + u;
+      const uint32_t cb = pr[u].c0 | (pr[u].c1 << 16);
       // y = s*q + m (exact in fp32: E4M3 operands, q <= 3), two channels per
       // op; the symmetric mode multiplies, y = s*(u - 2) (exact, and with the
       // sign of zero that product has)
       float2 y0[4], y1[4];
       {
-        const float s0 = dec[sz[u] & 0xFFu], s1 = dec[(sz[u] >> 16) & 0xFFu];
-        const float2 sp0 = f2(s0, s0), sp1 = f2(s1, s1);
+        const float2 g0v = e4m3x2_to_f2(pr[u].s0 | (pr[u].z0 << 8));
+        const float2 g1v = e4m3x2_to_f2(pr[u].s1 | (pr[u].z1 << 8));
+        const float2 sp0 = f2(g0v.x, g0v.x), sp1 = f2(g1v.x, g1v.x);
         if (SYM) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            y0[e] = __fmul2_rn(sp0, nlut[(cb[u] >> (4 * e)) & 0xFu]);
-            y1[e] = __fmul2_rn(sp1, nlut[(cb[u] >> (16 + 4 * e)) & 0xFu]);
+            y0[e] = __fmul2_rn(sp0, nlut[(cb >> (4 * e)) & 0xFu]);
+            y1[e] = __fmul2_rn(sp1, nlut[(cb >> (16 + 4 * e)) & 0xFu]);
           }
         } else {
-          const float m0 = dec[(sz[u] >> 8) & 0xFFu], m1 = dec[sz[u] >> 24];
-          const float2 mp0 = f2(m0, m0), mp1 = f2(m1, m1);
+          const float2 mp0 = f2(g0v.y, g0v.y), mp1 = f2(g1v.y, g1v.y);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            y0[e] = __ffma2_rn(sp0, nlut[(cb[u] >> (4 * e)) & 0xFu], mp0);
-            y1[e] = __ffma2_rn(sp1, nlut[(cb[u] >> (16 + 4 * e)) & 0xFu], mp1);
+            y0[e] = __ffma2_rn(sp0, nlut[(cb >> (4 * e)) & 0xFu], mp0);
+            y1[e] = __ffma2_rn(sp1, nlut[(cb >> (16 + 4 * e)) & 0xFu], mp1);
           }
         }
       }
       // centroids of stage T, T-1, ..., 1, in that order
 #pragma unroll
       for (int tt = 0; tt < (TT < 0 ? kMaxT : (TT == 0 ? 0 : TR)); ++tt) {
-        const int st = T - 1 - tt;
+        const int st = (TT >= 0 ? TT : T) - 1 - tt;   // a constant in the fixed-T instances
         if (TT < 0 && st < 0) break;
-        int k = TT > 0 ? (int)((ka[u] >> (8 * st)) & 0xFFu) : (int)ap[st * asg_t + (t < nt ? t : 0)];
+        int k = TT > 0 ? (int)pr[u].k[st] : (int)ap[st * asg_t + (t < nt ? t : 0)];
         k = min(k, K - 1);
         // shared and global rows on separate paths, so that the shared one is
         // addressed as shared memory (st < t_smem is uniform over the block)
@@ -297,18 +312,18 @@ qvg_dequant_fused(const DequantParams p, const int splits) {
       }
     }
   };
-  // kDqDepth steps of per-token bytes in flight: step d of a round is loaded
+  // kDqDepth steps of per-token bytes held: step d of a round is loaded
   // kDqDepth steps before it is processed
-  uint32_t cb[kDqDepth][kDqU], sz[kDqDepth][kDqU], ka[kDqDepth][kDqU];
+  Pre pre[kDqDepth][kDqU];
   const int t_first = stream * kDqU;
 #pragma unroll
-  for (int d = 0; d < kDqDepth; ++d) load(t_first + d * step, cb[d], sz[d], ka[d]);
+  for (int d = 0; d < kDqDepth; ++d) load(t_first + d * step, pre[d]);
   for (int t0 = t_first; t0 < nt; t0 += kDqDepth * step) {
 #pragma unroll
     for (int d = 0; d < kDqDepth; ++d) {
       const int tb = t0 + d * step;
-      if (tb < nt) process(tb, cb[d], sz[d], ka[d]);
-      load(tb + kDqDepth * step, cb[d], sz[d], ka[d]);
+      if (tb < nt) process(tb, pre[d]);
+      load(tb + kDqDepth * step, pre[d]);
     }
   }
 }
@@ -697,7 +712,7 @@ cudaError_t set_smem(F* f, size_t bytes) {
 
 cudaError_t launch_dequant(const DequantParams& p, int dtype, cudaStream_t s) {
   const int esz = dtype == kBF16 ? 2 : 4;
-  const size_t smem = (size_t)p.t_smem * p.K * kD * esz + 256 * sizeof(float) + 16 * sizeof(float2);
+  const size_t smem = (size_t)p.t_smem * p.K * kD * esz + 16 * sizeof(float2);
   const int units = p.n_chunks * p.H;
   if (units == 0) return cudaSuccess;
   if (p.desc != nullptr) {                       // per-chunk layouts: the generic instance

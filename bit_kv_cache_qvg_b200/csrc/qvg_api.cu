@@ -522,7 +522,7 @@ qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packed, qvg_d
   p.assign = packed->assign; p.centroids = packed->centroids; p.Y = Y;
   p.chunk_off = nullptr; p.N = N; p.y_head_stride = N; p.n_chunks = 1; p.H = H;
   p.K = cfg->K; p.T = cfg->T; p.G = cfg->group_size; p.sym = cfg->scale_mode == QVG_SCALE_SYM;
-  p.t_smem = std::min<int>(cfg->T, (int)((160 * 1024) / table));
+  p.t_smem = std::min<int>(cfg->T, (int)((kDqTableSmemBytes) / table));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
   st = cuda_status(plaunch(K_DEQUANT, s, [&] { return launch_dequant(p, dt, s); }));
   if (st == QVG_OK && fault_injected("stream")) st = QVG_ERR_CUDA;
@@ -849,11 +849,11 @@ qvg_status qvg_cache_dequantize(const qvg_cache* c, void* Y, qvg_stream_t stream
   p.centroids = c->tables; p.Y = Y; p.chunk_off = c->d_off; p.N = 0;
   p.y_head_stride = c->h_off[n_chunks]; p.n_chunks = n_chunks; p.H = c->H;
   p.K = c->cfg.K; p.T = c->cfg.T; p.G = c->cfg.group_size; p.sym = c->cfg.scale_mode == QVG_SCALE_SYM;
-  p.t_smem = std::min<int>(c->cfg.T, (int)((160 * 1024) / table));
+  p.t_smem = std::min<int>(c->cfg.T, (int)((kDqTableSmemBytes) / table));
   if (c->adaptive) {                 // per-chunk stage counts and group sizes
     p.desc = c->d_desc;
     p.T = c->T_max;
-    p.t_smem = std::min<int>(c->T_max, (int)((160 * 1024) / table));
+    p.t_smem = std::min<int>(c->T_max, (int)((kDqTableSmemBytes) / table));
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
   qvg_status st = cuda_status(plaunch(K_DEQUANT, s, [&] { return launch_dequant(p, c->dtype, s); }));

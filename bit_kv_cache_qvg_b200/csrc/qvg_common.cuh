@@ -13,6 +13,9 @@ namespace qvg {
 constexpr int kD = 128;            // channels per token handled by the kernels
 constexpr int kMaxK = 256;         // centroids per block (uint8 assignments)
 constexpr int kMaxT = 8;           // residual stages
+// Shared memory the fused dequantisation gives to centroid tables (whole
+// stages; three of K = 256 at bf16); later stages are read through L2.
+constexpr int kDqTableSmemBytes = 200 * 1024;
 
 enum : int { kBF16 = 0, kFP32 = 1 };
 
