@@ -307,6 +307,7 @@ qvg_assign_candidates(const void* R, const void* C, const int K, const int64_t N
 //   centroids (a warp per centroid): every centroid with entries gets its new
 //             count and, if non-empty, its mean and squared norm.
 constexpr int kBucketThreads = 1024;
+constexpr size_t kBucketStageBytes = 192 * 1024;   // largest staged pair of assignment arrays
 constexpr int kScan = 8;              // assignments per thread per scan step (loads in flight)
 constexpr int kSumThreads = 256;
 constexpr int kSumWarps = kSumThreads / 32;
@@ -342,6 +343,22 @@ __device__ __forceinline__ void load_assignments(const uint8_t* piu, const uint8
   }
 }
 
+// Copy the N assignment bytes at g into shared memory at s + (g mod 16), so
+// that token t sits at s[(g mod 16) + t]: 16-byte loads over the aligned
+// middle, single bytes for the ragged ends (nothing outside [g, g + N) is
+// read).  The caller synchronises.
+__device__ __forceinline__ void stage_assignments(const uint8_t* g, int64_t N, uint8_t* s) {
+  const int off = (int)(reinterpret_cast<uintptr_t>(g) & 15u);
+  const int64_t b0 = (int64_t)((16 - off) & 15) < N ? (int64_t)((16 - off) & 15) : N;   // first aligned token
+  const int64_t n16 = (N - b0) / 16;
+  const int64_t b1 = b0 + 16 * n16;                             // first token of the tail
+  const uint4* src = reinterpret_cast<const uint4*>(g + b0);
+  uint4* dst = reinterpret_cast<uint4*>(s + off + b0);
+  for (int64_t x = threadIdx.x; x < n16; x += blockDim.x) dst[x] = src[x];
+  if (threadIdx.x < b0) s[off + threadIdx.x] = g[threadIdx.x];
+  if (threadIdx.x < N - b1) s[off + b1 + threadIdx.x] = g[b1 + threadIdx.x];
+}
+
 // Warp-aggregated shared-memory add of `v` to counter[key] (lanes with the
 // same key are combined; `key` < 0 takes part in no add).  Returns, for
 // returning adds, the slot of this lane: old value + rank among its peers.
@@ -375,6 +392,18 @@ qvg_update_bucket(const UpdateParams p) {
   __syncthreads();
   const uint8_t* piu = p.pi + (int64_t)u * N;
   const uint8_t* pio = full ? nullptr : p.pi_old + (int64_t)u * N;
+  // When the block's assignments fit in shared memory they are staged there
+  // once (a few wide loads per thread instead of a round trip per scan step
+  // and pass), and both passes read them from there.
+  extern __shared__ __align__(16) uint8_t s_pi[];
+  if (p.stage_pi) {
+    const int64_t pad = (N + 31) & ~int64_t(15);
+    stage_assignments(piu, N, s_pi);
+    if (!full) stage_assignments(pio, N, s_pi + pad);
+    piu = s_pi + (reinterpret_cast<uintptr_t>(piu) & 15u);
+    if (!full) pio = s_pi + pad + (reinterpret_cast<uintptr_t>(pio) & 15u);
+  }
+  __syncthreads();
   const int64_t step = (int64_t)kScan * blockDim.x;
   for (int64_t c = 0; c < N; c += step) {
     int kn[kScan], ko[kScan];
@@ -860,8 +889,17 @@ cudaError_t launch_assign_candidates(const void* R, const void* C, int K, int64_
 }
 
 cudaError_t launch_update_bucket(const UpdateParams& p, int dtype, cudaStream_t s) {
-  if (dtype == kBF16) qvg_update_bucket<kBF16><<<(unsigned)p.W, kBucketThreads, 0, s>>>(p);
-  else qvg_update_bucket<kFP32><<<(unsigned)p.W, kBucketThreads, 0, s>>>(p);
+  UpdateParams q = p;
+  const size_t pad = (size_t)((p.N + 31) & ~int64_t(15));
+  const size_t smem = 2 * pad;
+  q.stage_pi = smem <= kBucketStageBytes;
+  const size_t dyn = q.stage_pi ? smem : 0;
+  const void* fn = dtype == kBF16 ? reinterpret_cast<const void*>(qvg_update_bucket<kBF16>)
+                                  : reinterpret_cast<const void*>(qvg_update_bucket<kFP32>);
+  cudaError_t e = ensure_dynamic_smem(fn, dyn);
+  if (e != cudaSuccess) return e;
+  if (dtype == kBF16) qvg_update_bucket<kBF16><<<(unsigned)p.W, kBucketThreads, dyn, s>>>(q);
+  else qvg_update_bucket<kFP32><<<(unsigned)p.W, kBucketThreads, dyn, s>>>(q);
   return cudaGetLastError();
 }
 

@@ -139,6 +139,7 @@ struct UpdateParams {
   int W;
   int K;
   int log2n;              // smallest k with 2^k > N
+  int stage_pi;           // (set by the bucket launcher) assignments staged in shared memory
 };
 // Exact fixed-point centroid sums: with pi_old == nullptr every token adds its
 // row to its centroid; otherwise a token whose centroid changed adds its row
