@@ -357,6 +357,11 @@ __device__ __forceinline__ void stage_assignments(const uint8_t* g, int64_t N, u
   for (int64_t x = threadIdx.x; x < n16; x += blockDim.x) dst[x] = src[x];
   if (threadIdx.x < b0) s[off + threadIdx.x] = g[threadIdx.x];
   if (threadIdx.x < N - b1) s[off + b1 + threadIdx.x] = g[b1 + threadIdx.x];
+  // the bytes before the first token and up to the next 4-byte boundary
+  // after the last are zero, so that whole words can be compared
+  if (threadIdx.x < off) s[threadIdx.x] = 0;
+  const int64_t end = off + N, end4 = (end + 3) & ~int64_t(3);
+  if (threadIdx.x < end4 - end) s[end + threadIdx.x] = 0;
 }
 
 // Warp-aggregated shared-memory add of `v` to counter[key] (lanes with the
@@ -396,16 +401,45 @@ qvg_update_bucket(const UpdateParams p) {
   // once (a few wide loads per thread instead of a round trip per scan step
   // and pass), and both passes read them from there.
   extern __shared__ __align__(16) uint8_t s_pi[];
+  const int64_t pad = (N + 31) & ~int64_t(15);
+  const int a_off = (int)(reinterpret_cast<uintptr_t>(piu) & 15u);
+  // Incremental passes over staged arrays whose tokens sit at the same byte
+  // offset compare four tokens per 32-bit word, so that the (many) unchanged
+  // tokens cost one compare per four.
+  const bool words = p.stage_pi && !full && a_off == (int)(reinterpret_cast<uintptr_t>(pio) & 15u);
   if (p.stage_pi) {
-    const int64_t pad = (N + 31) & ~int64_t(15);
     stage_assignments(piu, N, s_pi);
     if (!full) stage_assignments(pio, N, s_pi + pad);
-    piu = s_pi + (reinterpret_cast<uintptr_t>(piu) & 15u);
+    piu = s_pi + a_off;
     if (!full) pio = s_pi + pad + (reinterpret_cast<uintptr_t>(pio) & 15u);
   }
   __syncthreads();
+  const uint32_t* wn = reinterpret_cast<const uint32_t*>(s_pi);
+  const uint32_t* wo = reinterpret_cast<const uint32_t*>(s_pi + pad);
+  const int64_t n_words = (a_off + N + 3) / 4;
+  // changed tokens of word g: calls f(token, new centroid, old centroid)
+  auto word_changes = [&](int64_t g, auto&& f) {
+    const uint32_t xn = wn[g], xo = wo[g];
+    if (xn == xo) return;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int bn = (int)((xn >> (8 * j)) & 0xFFu), bo = (int)((xo >> (8 * j)) & 0xFFu);
+      const int64_t t = 4 * g + j - a_off;
+      if (bn != bo && t >= 0 && t < N) f((uint32_t)t, min(bn, K - 1), min(bo, K - 1));
+    }
+  };
   const int64_t step = (int64_t)kScan * blockDim.x;
-  for (int64_t c = 0; c < N; c += step) {
+  if (words) {
+    for (int64_t g = threadIdx.x; g < n_words; g += blockDim.x)
+      word_changes(g, [&](uint32_t, int kn, int ko) {
+        if (kn == ko) return;
+        atomicAdd(hist + kn, 1);
+        atomicAdd(hist + ko, 1);
+        atomicAdd(dcnt + kn, 1);
+        atomicAdd(dcnt + ko, -1);
+      });
+  }
+  for (int64_t c = 0; c < N && !words; c += step) {
     int kn[kScan], ko[kScan];
     load_assignments(piu, pio, N, c, K, kn, ko);
 #pragma unroll
@@ -451,7 +485,15 @@ qvg_update_bucket(const UpdateParams p) {
     p.cnt[(int64_t)u * K + k] = full ? hist[k] : dcnt[k];
   __syncthreads();
   uint32_t* list = p.list + (int64_t)u * 2 * N;    // capacity 2N entries per block
-  for (int64_t c = 0; c < N; c += step) {
+  if (words) {
+    for (int64_t g = threadIdx.x; g < n_words; g += blockDim.x)
+      word_changes(g, [&](uint32_t t, int kn, int ko) {
+        if (kn == ko) return;
+        list[atomicAdd(cursor + kn, 1)] = t | ((uint32_t)kn << kEntKShift);
+        list[-atomicAdd(cursor_sub + ko, 1) - 1] = t | ((uint32_t)ko << kEntKShift) | kEntSub;
+      });
+  }
+  for (int64_t c = 0; c < N && !words; c += step) {
     int kn[kScan], ko[kScan];
     load_assignments(piu, pio, N, c, K, kn, ko);
 #pragma unroll
