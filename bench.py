@@ -183,23 +183,25 @@ def strong_scaling_value(total_bytes: float, ms: float) -> float:
 
 
 # ---------------------------------------------------------------- oracle arm
-def oracle_sample(wl, tokens: int, seed: int = 99, dequant: bool = True):
+def oracle_sample(wl, tokens: int, seed: int = 99, dequant: bool = True, units: int = 1):
     """Time the oracle's quantise (+ dequantise unless `dequant` is False) of
-    one block of `tokens` tokens of the workload's shape on the host cores.
-    Returns (seconds, bytes, threads)."""
+    `units` seeded blocks of `tokens` tokens of the workload's shape (V blocks,
+    or K and V alternating when there are several) on the host cores.
+    Returns (seconds, uncompressed bytes, threads)."""
     import numpy as np
     from bit_kv_cache_qvg_b200 import synth
     from oracle import oracle as o
     o.build()
     frames = max(1, math.ceil(tokens / (wl["gh"] * wl["gw"])))
-    X = synth.block_batch(1, synth.KVShape(frames, wl["gh"], wl["gw"]), seed=seed, kinds=[1])[:, :tokens]
+    kinds = [1] if units == 1 else [u % 2 for u in range(units)]
+    X = synth.block_batch(units, synth.KVShape(frames, wl["gh"], wl["gw"]), seed=seed, kinds=kinds)[:, :tokens]
     Xb = X.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
     t0 = time.perf_counter()
     p = o.quantize(Xb, K=wl["K"], T=wl["T"], G=wl["G"], iters=wl["iters"])
     if dequant:
-        o.dequantize(p, K=wl["K"], T=wl["T"], G=wl["G"], N=tokens, H=1, d=128)
+        o.dequantize(p, K=wl["K"], T=wl["T"], G=wl["G"], N=tokens, H=units, d=128)
     dt = time.perf_counter() - t0
-    return dt, tokens * 128 * 2, o.get_threads()
+    return dt, units * tokens * 128 * 2, o.get_threads()
 
 
 def oracle_stream_sample(wl, chunks: int, seed: int = 7):
@@ -328,7 +330,7 @@ def main():
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=4750)
-    ap.add_argument("--cpu-tokens", type=int, default=9500)
+    ap.add_argument("--cpu-units", type=int, default=8, help="full-size blocks of the oracle baseline")
     ap.add_argument("--frames", type=int, default=None, help="override the frame count")
     ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
                     help="weak: every rank its own cache; strong: the ranks share one cache by heads")
@@ -585,10 +587,12 @@ def main():
         result["e2e"] = e2e(args, qvg, cfg, X, Y, packed, ws, L, Hh, N, dev, world, dist,
                             total_bytes=total_bytes if strong else None)
     if rank == 0 and not args.no_cpu_baseline:
-        dt, nbytes, threads = oracle_sample(wl, args.cpu_tokens)
+        n_tok = wl["frames"] * wl["gh"] * wl["gw"]
+        dt, nbytes, threads = oracle_sample(wl, n_tok, units=args.cpu_units)
         result["cpu_baseline"] = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                                  "sample": f"one V block of {args.cpu_tokens} tokens of the workload's shape "
-                                            f"(quantise + dequantise), {dt:.1f} s"}
+                                  "sample": f"{args.cpu_units} seeded full-size blocks ({n_tok} tokens, K and V "
+                                            f"alternating) quantised and dequantised in {dt:.1f} s; the rate is "
+                                            "extrapolated linearly to the workload (blocks are independent)"}
     if rank == 0:
         print(json.dumps(result))
     if dist is not None:
