@@ -20,8 +20,9 @@
 //      stage's centroid in reverse order, round to bf16 -- the arithmetic of
 //      qvg_dequant_fused), apply the rotary embedding to K, and store both
 //      straight into shared memory in the tensor core's K-major operand
-//      layout: K rows (keys) with the channels contiguous, V transposed
-//      (channels) with the keys contiguous, each thread an 8 x 8 block;
+//      layout (128-byte swizzle): K rows (keys) with the channels contiguous,
+//      V transposed (channels) with the keys contiguous, each thread an
+//      8 x 8 block;
 //   2. one thread issues S = Q' K'^T (tcgen05.mma kind::f16, M = N = K = 128,
 //      fp32 accumulators in tensor memory);
 //   3. warps 0-3 (one per tensor-memory lane quarter, a thread per query)
@@ -101,20 +102,29 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Shared-memory operand descriptor, K-major, no swizzle: 8-row x 16-byte core
-// matrices; core matrices adjacent along K are 128 bytes apart (LBO), 8-row
-// groups 2,048 bytes apart (SBO: sixteen core matrices span K = 128).
+// Shared-memory operand descriptor, K-major, 128-byte swizzle: a 128 x 128
+// bf16 operand is two 64-column halves of 128 rows x 128 bytes (16 KB apart),
+// and in each 8-row group of 1,024 bytes (SBO) the 16-byte chunk c of row r
+// sits at chunk position c ^ (r mod 8).  The swizzle spreads a warp's stores
+// of one chunk column over all banks.
 __device__ __forceinline__ uint64_t op_desc(uint32_t saddr) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFF);
-  d |= (uint64_t)(128 >> 4) << 16;
-  d |= (uint64_t)(2048 >> 4) << 32;
-  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)1 << 16;                 // LBO (unused with this swizzle)
+  d |= (uint64_t)(1024 >> 4) << 32;       // SBO
+  d |= (uint64_t)1 << 46;                 // version
+  d |= (uint64_t)2 << 61;                 // SWIZZLE_128B
   return d;
 }
-// Byte offset of element (row, k) of a 128 x 128 operand in that layout.
+constexpr int kAtHalfBytes = kAtTile * 128;     // one 64-column half of an operand
+// Byte offset of element (row, k) (k a multiple of 4 within its chunk is
+// enough for the 8- and 16-byte stores below) of a 128 x 128 operand.
 __device__ __forceinline__ int op_off(int row, int k) {
-  return (row >> 3) * 2048 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2;
+  return (k >> 6) * kAtHalfBytes + row * 128 + ((((k & 63) >> 3) ^ (row & 7)) << 4) + (k & 7) * 2;
+}
+// Descriptor of K-step kk (16 columns) of the operand at saddr.
+__device__ __forceinline__ uint64_t op_desc_k(uint32_t saddr, int kk) {
+  return op_desc(saddr + (uint32_t)((kk >> 2) * kAtHalfBytes + (kk & 3) * 32));
 }
 
 // kind::f16, A = B = bf16, D = f32, both K-major, M = N = 128.
@@ -181,35 +191,52 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
+// Two E4M3 bytes (low byte first) as fp32 values, through the hardware
+// conversion to f16 (exact for every finite E4M3 value) and then to fp32.
+__device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t pair16) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 a;\n\tcvt.u16.u32 a, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\t}" : "=r"(h) : "r"(pair16));
+  float lo, hi;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h));
+  return make_float2(lo, hi);
+}
+
 // (cos, sin) of the rotary angle of pair i at position p from the two tables
 // (positions outside [0, max_pos] are clamped, so the reads stay in bounds).
-__device__ __forceinline__ float2 rope_cs(const AttnParams& p, int64_t pos, int i) {
-  pos = pos < 0 ? 0 : (pos > p.max_pos ? p.max_pos : pos);
-  const float2 a = p.rope_hi[(pos / kRopeLo) * (kD / 2) + i];
-  const float2 b = p.rope_lo[(pos % kRopeLo) * (kD / 2) + i];
+__device__ __forceinline__ int64_t rope_pos(const AttnParams& p, int64_t pos) {
+  return pos < 0 ? 0 : (pos > p.max_pos ? p.max_pos : pos);
+}
+// the angle sum from the high-table entry a and the low-table entry b
+__device__ __forceinline__ float2 rope_combine(float2 a, float2 b) {
   return make_float2(__fsub_rn(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y)),
                      __fadd_rn(__fmul_rn(a.y, b.x), __fmul_rn(a.x, b.y)));
 }
+__device__ __forceinline__ float2 rope_cs(const AttnParams& p, int64_t pos, int i) {
+  pos = rope_pos(p, pos);
+  return rope_combine(p.rope_hi[(pos / kRopeLo) * (kD / 2) + i], p.rope_lo[(pos % kRopeLo) * (kD / 2) + i]);
+}
 
-// Reconstruct channels c0 .. c0+7 of the 8 tokens tok0 .. tok0+7 (those
+// Reconstruct channels c0 .. c0+7 of the NR tokens tok0 .. tok0+NR-1 (those
 // below Nk) of cache `which` (0 = K, 1 = V) of head h: y = s*q + m (or
 // s*(u - 2)), plus the centroids of stages T, ..., 1 in that order, each an
 // fp32 add, then one rounding to bf16 -- the arithmetic of qvg_dequant_fused.
 // The results are fp32 values of the rounded bf16 numbers (zero for tokens
 // past the end).  TT > 0 fixes the stage count (at most 4) so that the loads
-// of all eight tokens are issued together: first the codes, scale/zero bytes
+// of all NR tokens are issued together: first the codes, scale/zero bytes
 // and assignments, then the centroid rows they select.
-template <int TT>
-__device__ __forceinline__ void recon_block(const AttnParams& p, const float* dec, int which, int h,
-                                            int64_t tok0, int c0, float (&y)[8][8]) {
+template <int TT, int NR>
+__device__ __forceinline__ void recon_block(const AttnParams& p, const float2* nlut, int which, int h,
+                                            int64_t tok0, int c0, float (&y)[NR][8]) {
   constexpr int TR = TT > 0 ? TT : 1;
   const int T = TT >= 0 ? TT : p.T;
   const int ng = kD / p.G;
   const int g = c0 / p.G;
-  uint32_t code[8], sz[8];
-  int kk[8][TR];
+  uint32_t code[NR], sz[NR];
+  int kk[NR][TR];
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
+  for (int r = 0; r < NR; ++r) {
     const int64_t tok = tok0 + r < p.Nk ? tok0 + r : p.Nk - 1;   // past the end: a valid token, result unused
     const int64_t row = (int64_t)h * p.Nk + tok;
     code[r] = *reinterpret_cast<const uint16_t*>(p.codes[which] + row * (kD / 4) + c0 / 4);
@@ -218,32 +245,30 @@ __device__ __forceinline__ void recon_block(const AttnParams& p, const float* de
     for (int t = 0; t < TR; ++t)
       if (TT > 0) kk[r][t] = min((int)p.assign[which][((int64_t)t * p.H + h) * p.Nk + tok], p.K - 1);
   }
-  uint4 rows[8][TR];
+  uint4 rows[NR][TR];
   if (TT > 0) {
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
+    for (int r = 0; r < NR; ++r)
 #pragma unroll
       for (int t = 0; t < TR; ++t)
         rows[r][t] = *reinterpret_cast<const uint4*>(p.tab[which] + (((int64_t)t * p.H + h) * p.K + kk[r][t]) * kD + c0);
   }
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const float s = dec[sz[r] & 0xFFu];
-    if (p.sym) {
+  for (int r = 0; r < NR; ++r) {
+    // y = s*q + m (or s*(u - 2)), exact in fp32, two channels per op through
+    // the nibble table (which holds q, or u - 2 in the symmetric mode)
+    const float2 sm = e4m3x2_to_f2(sz[r]);
+    const float2 s2 = make_float2(sm.x, sm.x), m2 = make_float2(sm.y, sm.y);
+    float2 y2[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[r][e] = __fmul_rn(s, (float)((code[r] >> (2 * e)) & 3u) - 2.0f);
-    } else {
-      const float m = dec[sz[r] >> 8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) y[r][e] = __fmaf_rn(s, (float)((code[r] >> (2 * e)) & 3u), m);
-    }
+    for (int e = 0; e < 4; ++e)
+      y2[e] = p.sym ? __fmul2_rn(s2, nlut[(code[r] >> (4 * e)) & 0xFu])
+                    : __ffma2_rn(s2, nlut[(code[r] >> (4 * e)) & 0xFu], m2);
     auto add_row = [&](const uint4 w) {
-      const uint32_t x[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        y[r][2 * e] = __fadd_rn(y[r][2 * e], __uint_as_float(x[e] << 16));
-        y[r][2 * e + 1] = __fadd_rn(y[r][2 * e + 1], __uint_as_float(x[e] & 0xFFFF0000u));
-      }
+      y2[0] = __fadd2_rn(y2[0], make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u)));
+      y2[1] = __fadd2_rn(y2[1], make_float2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u)));
+      y2[2] = __fadd2_rn(y2[2], make_float2(__uint_as_float(w.z << 16), __uint_as_float(w.z & 0xFFFF0000u)));
+      y2[3] = __fadd2_rn(y2[3], make_float2(__uint_as_float(w.w << 16), __uint_as_float(w.w & 0xFFFF0000u)));
     };
     if (TT > 0) {
 #pragma unroll
@@ -256,6 +281,8 @@ __device__ __forceinline__ void recon_block(const AttnParams& p, const float* de
       }
     }
 #pragma unroll
+    for (int e = 0; e < 4; ++e) { y[r][2 * e] = y2[e].x; y[r][2 * e + 1] = y2[e].y; }
+#pragma unroll
     for (int e = 0; e < 8; e += 2) {
       const uint32_t b = pack_bf16(y[r][e], y[r][e + 1]);
       y[r][e] = tok0 + r < p.Nk ? __uint_as_float(b << 16) : 0.0f;
@@ -265,21 +292,22 @@ __device__ __forceinline__ void recon_block(const AttnParams& p, const float* de
 }
 
 template <int TT>
-__global__ void __launch_bounds__(kAtThreads, 1)
+__global__ void __launch_bounds__(kAtThreads, 2)
 qvg_attention_fused(const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                               // A of S: queries x channels
   uint8_t* sK = sQ + kAtOpBytes;                    // B of S: keys x channels; then A of O: queries x keys (P)
   uint8_t* sV = sK + kAtOpBytes;                    // B of O: channels x keys
-  float* dec = reinterpret_cast<float*>(sV + kAtOpBytes);
-  AtBars* bars = reinterpret_cast<AtBars*>(dec + 256);
+  float2* nlut = reinterpret_cast<float2*>(sV + kAtOpBytes);    // nibble -> two codes (q, or u - 2)
+  AtBars* bars = reinterpret_cast<AtBars*>(nlut + 32);
 
   const int h = blockIdx.y;
   const int64_t q0 = (int64_t)blockIdx.x * kAtTile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // the thread's 8 x 8 block of a 128 x 128 tile: rows 8*rb .. 8*rb+7, channels 8*cb .. 8*cb+7
   const int rb = threadIdx.x >> 4, cb = threadIdx.x & 15;
+  const int rbv = threadIdx.x & 15, cbv = threadIdx.x >> 4;   // the same blocks, transposed, for V
 
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->s_done)));
@@ -292,7 +320,10 @@ qvg_attention_fused(const AttnParams p) {
                      smem_addr(&bars->tmem_base)));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  for (int x = threadIdx.x; x < 256; x += blockDim.x) dec[x] = e4m3_to_f32((uint8_t)x);
+  if (threadIdx.x < 16) {
+    const float off = p.sym ? 2.0f : 0.0f;
+    nlut[threadIdx.x] = make_float2((float)(threadIdx.x & 3u) - off, (float)(threadIdx.x >> 2) - off);
+  }
 
   // queries: rotary embedding at their positions, bf16, into the A layout
   for (int r = 0; r < 8; ++r) {
@@ -333,32 +364,43 @@ qvg_attention_fused(const AttnParams p) {
       if (__syncthreads_or(!w_ok)) { ok = false; break; }
       fence_after();
     }
-    // 1. reconstruct the K and V tile into the operand layouts
-    {
-      float vk[8][8];
-      const int64_t tok0 = k0 + 8 * rb;
-      recon_block<TT>(p, dec, 0, h, tok0, 8 * cb, vk);
+    // 1. reconstruct the K and V tile into the operand layouts, four of the
+    // thread's eight tokens at a time (registers: two CTAs share an SM)
+#pragma unroll 1
+    for (int half = 0; half < 2; ++half) {
+      float vk[4][8];
+      const int r0 = 8 * rb + 4 * half;
+      const int64_t tok0 = k0 + r0;
+      recon_block<TT, 4>(p, nlut, 0, h, tok0, 8 * cb, vk);
       // K rows: rotary embedding of the reconstructed values, then bf16
+      const int64_t pa = rope_pos(p, tok0), pz = rope_pos(p, tok0 + 3);
+      const bool one_hi = pa / kRopeLo == pz / kRopeLo;   // the four positions share the high entry
+      float2 hi[4];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
+      for (int e = 0; e < 4; ++e) hi[e] = p.rope_hi[(pa / kRopeLo) * (kD / 2) + 4 * cb + e];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
         uint32_t w[4];
+        const int64_t pr = rope_pos(p, tok0 + r);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float2 cs = rope_cs(p, tok0 + r, 4 * cb + e);
+          const float2 cs = one_hi ? rope_combine(hi[e], p.rope_lo[(pr % kRopeLo) * (kD / 2) + 4 * cb + e])
+                                   : rope_cs(p, tok0 + r, 4 * cb + e);
           const float a = vk[r][2 * e], b = vk[r][2 * e + 1];
           w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
                            __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
         }
-        *reinterpret_cast<uint4*>(sK + op_off(8 * rb + r, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(sK + op_off(r0 + r, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      recon_block<TT>(p, dec, 1, h, tok0, 8 * cb, vk);
-      // V transposed: channel 8*cb + e holds the 8 keys 8*rb .. 8*rb+7 contiguously
+      // V, transposed (channel 8*cbv + e holds keys rv .. rv+3 in 8 contiguous
+      // bytes), with the thread's key and channel blocks swapped: the eight
+      // lanes of a store phase then write eight key chunks of one channel row
+      const int rv = 8 * rbv + 4 * half;
+      recon_block<TT, 4>(p, nlut, 1, h, k0 + rv, 8 * cbv, vk);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const uint4 t = make_uint4(pack_bf16(vk[0][e], vk[1][e]), pack_bf16(vk[2][e], vk[3][e]),
-                                   pack_bf16(vk[4][e], vk[5][e]), pack_bf16(vk[6][e], vk[7][e]));
-        *reinterpret_cast<uint4*>(sV + op_off(8 * cb + e, 8 * rb)) = t;
-      }
+      for (int e = 0; e < 8; ++e)
+        *reinterpret_cast<uint2*>(sV + op_off(8 * cbv + e, rv)) =
+            make_uint2(pack_bf16(vk[0][e], vk[1][e]), pack_bf16(vk[2][e], vk[3][e]));
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
     fence_before();
@@ -368,7 +410,7 @@ qvg_attention_fused(const AttnParams p) {
     if (threadIdx.x == 0) {
       const uint32_t a0 = smem_addr(sQ), b0 = smem_addr(sK);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) mma(tS, op_desc(a0 + 256 * kk), op_desc(b0 + 256 * kk), kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < 8; ++kk) mma(tS, op_desc_k(a0, kk), op_desc_k(b0, kk), kk > 0 ? 1u : 0u);
       mma_commit(&bars->s_done);
     }
     // 3. online softmax (warps 0-3: the thread's query is row 32*warp + lane)
@@ -381,32 +423,38 @@ qvg_attention_fused(const AttnParams p) {
         const int qi = 32 * warp + lane;
         const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
         const int valid = (int)(p.Nk - k0 < kAtTile ? p.Nk - k0 : kAtTile);
-        float x[128];
-#pragma unroll
+        // pass 1: the row maximum, 32 columns at a time
+        float mt = -3.0e38f;
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
           tld32(tS + lane_base + (uint32_t)(32 * c), r);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[32 * c + e] = 32 * c + e < valid ? __uint_as_float(r[e]) * p.sl : -3.0e38f;
+          for (int e = 0; e < 32; ++e)
+            if (32 * c + e < valid) mt = fmaxf(mt, __uint_as_float(r[e]) * p.sl);
         }
-        float mt = -3.0e38f;
-#pragma unroll
-        for (int e = 0; e < 128; e += 2) mt = fmaxf(mt, fmaxf(x[e], x[e + 1]));
         const float m_new = fmaxf(m_run, mt);
         const float alpha = exp2_approx(m_run - m_new);
+        // pass 2: the weights, rounded to bf16 into the P operand, and their sum
         float sum = 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tld32(tS + lane_base + (uint32_t)(32 * c), r);
 #pragma unroll
-        for (int kg = 0; kg < 16; ++kg) {
-          uint32_t w[4];
+          for (int kg = 0; kg < 4; ++kg) {
+            uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float pa = 8 * kg + 2 * e < valid ? exp2_approx(x[8 * kg + 2 * e] - m_new) : 0.0f;
-            const float pb = 8 * kg + 2 * e + 1 < valid ? exp2_approx(x[8 * kg + 2 * e + 1] - m_new) : 0.0f;
-            w[e] = pack_bf16(pa, pb);
-            // the sum takes the rounded weights, the ones the product uses
-            sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
+            for (int e = 0; e < 4; ++e) {
+              const int j0 = 32 * c + 8 * kg + 2 * e;
+              const float pa = j0 < valid ? exp2_approx(__uint_as_float(r[8 * kg + 2 * e]) * p.sl - m_new) : 0.0f;
+              const float pb = j0 + 1 < valid ? exp2_approx(__uint_as_float(r[8 * kg + 2 * e + 1]) * p.sl - m_new) : 0.0f;
+              w[e] = pack_bf16(pa, pb);
+              // the sum takes the rounded weights, the ones the product uses
+              sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
+            }
+            *reinterpret_cast<uint4*>(sK + op_off(qi, 32 * c + 8 * kg)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          *reinterpret_cast<uint4*>(sK + op_off(qi, 8 * kg)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         l_run = l_run * alpha + sum;
         m_run = m_new;
@@ -433,7 +481,7 @@ qvg_attention_fused(const AttnParams p) {
     if (threadIdx.x == 0) {
       const uint32_t a0 = smem_addr(sK), b0 = smem_addr(sV);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) mma(tO, op_desc(a0 + 256 * kk), op_desc(b0 + 256 * kk), (j > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < 8; ++kk) mma(tO, op_desc_k(a0, kk), op_desc_k(b0, kk), (j > 0 || kk > 0) ? 1u : 0u);
       mma_commit(&bars->o_done);
     }
   }
