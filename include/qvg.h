@@ -37,11 +37,14 @@
  *     qvg_static_status wait for the stream, read the word and clear it.
  *   - Fault injection for tests (host side; unset in normal use): the
  *     environment variable QVG_FAULT_INJECT holds a comma-separated list of
- *       alloc    every device allocation of qvg_cache_create fails
- *                (QVG_ERR_NO_MEMORY, nothing allocated);
- *       stream   qvg_quantize, qvg_dequantize and qvg_cache_dequantize report
- *                QVG_ERR_CUDA after queueing, as a failed launch would (an
- *                append then leaves the cache unchanged);
+ *       alloc    every device allocation of qvg_cache_create and
+ *                qvg_cache_create_adaptive fails (QVG_ERR_NO_MEMORY, nothing
+ *                allocated);
+ *       stream   the quantising calls (qvg_quantize, qvg_quantize_static,
+ *                both appends), qvg_dequantize, qvg_cache_dequantize and
+ *                qvg_attention report QVG_ERR_CUDA after queueing, as a
+ *                failed launch would (an append then leaves the cache
+ *                unchanged);
  *       timeout  the first CTA of the tensor-core assignment withholds one
  *                tile load and its waits give up after 1 ms, so that the
  *                bounded waits run out and record a device-side timeout.
