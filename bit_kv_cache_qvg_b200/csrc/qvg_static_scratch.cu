@@ -25,7 +25,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "qvg.h"
 #include "qvg_launch.h"
@@ -33,32 +32,23 @@
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(32) << 20;
-constexpr int kMaxDevices = 64;
 
 // One reserve per device (a __device__ variable has one instance per device
 // on which the library's device code is loaded).  256-byte alignment is the
 // alignment qvg_quantize requires of a workspace.
 __device__ __align__(256) unsigned char g_qvg_static_scratch[kStaticScratchBytes];
 
-std::mutex g_setup_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the reserve on the current device, looked up once per
-// device (the lookup may load this file's device code on first use).
+// Device address of the reserve on the current device.  It is looked up on
+// every call (cheap once the module is loaded; the first lookup may load this
+// file's device code), so that it stays right after a context teardown
+// reloads the module at another address.
 qvg_status scratch_on_current_device(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return QVG_ERR_CUDA; }
-  if (dev < 0 || dev >= kMaxDevices) return QVG_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_qvg_static_scratch) != cudaSuccess || p == nullptr) {
-      cudaGetLastError();       // leave no error pending for a later launch check
-      return QVG_ERR_CUDA;
-    }
-    g_scratch_ptr[dev] = p;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_qvg_static_scratch) != cudaSuccess || p == nullptr) {
+    cudaGetLastError();       // leave no error pending for a later launch check
+    return QVG_ERR_CUDA;
   }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return QVG_OK;
 }
 
