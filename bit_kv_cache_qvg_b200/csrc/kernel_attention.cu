@@ -45,7 +45,8 @@
 namespace qvg {
 namespace {
 
-constexpr int kAtThreads = 256;                 // 8 warps
+constexpr int kAtThreads = 512;                 // 16 warps
+constexpr int kAtQTiles = 2;                    // query tiles per CTA (each reconstructed K/V tile serves both)
 constexpr int kAtTile = 128;                    // queries per CTA, cached tokens per tile
 constexpr int kAtOpBytes = kAtTile * kD * 2;    // one 128 x 128 bf16 operand: 32 KB
 constexpr uint64_t kAtWaitNs = 2000000000ull;   // 2 s per bounded wait
@@ -292,22 +293,23 @@ __device__ __forceinline__ void recon_block(const AttnParams& p, const float2* n
 }
 
 template <int TT>
-__global__ void __launch_bounds__(kAtThreads, 2)
+__global__ void __launch_bounds__(kAtThreads, 1)
 qvg_attention_fused(const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                               // A of S: queries x channels
-  uint8_t* sK = sQ + kAtOpBytes;                    // B of S: keys x channels; then A of O: queries x keys (P)
+  uint8_t* sQ = smem;                               // A of S: two query tiles x channels
+  uint8_t* sK = sQ + kAtQTiles * kAtOpBytes;        // B of S: keys x channels; then A of O for query tile 0 (P)
   uint8_t* sV = sK + kAtOpBytes;                    // B of O: channels x keys
-  float2* nlut = reinterpret_cast<float2*>(sV + kAtOpBytes);    // nibble -> two codes (q, or u - 2)
+  uint8_t* sP1 = sV + kAtOpBytes;                   // A of O for query tile 1 (P)
+  float2* nlut = reinterpret_cast<float2*>(sP1 + kAtOpBytes);   // nibble -> two codes (q, or u - 2)
   AtBars* bars = reinterpret_cast<AtBars*>(nlut + 32);
 
   const int h = blockIdx.y;
-  const int64_t q0 = (int64_t)blockIdx.x * kAtTile;
+  const int64_t q0 = (int64_t)blockIdx.x * (kAtQTiles * kAtTile);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // the thread's 8 x 8 block of a 128 x 128 tile: rows 8*rb .. 8*rb+7, channels 8*cb .. 8*cb+7
+  // the thread's 4 x 8 block of a 128 x 128 tile: rows 4*rb .. 4*rb+3, channels 8*cb .. 8*cb+7
   const int rb = threadIdx.x >> 4, cb = threadIdx.x & 15;
-  const int rbv = threadIdx.x & 15, cbv = threadIdx.x >> 4;   // the same blocks, transposed, for V
+  const int rbv = threadIdx.x & 31, cbv = threadIdx.x >> 5;   // the same blocks, transposed, for V
 
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->s_done)));
@@ -316,7 +318,7 @@ qvg_attention_fused(const AttnParams p) {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
                      smem_addr(&bars->tmem_base)));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
@@ -326,50 +328,56 @@ qvg_attention_fused(const AttnParams p) {
   }
 
   // queries: rotary embedding at their positions, bf16, into the A layout
-  for (int r = 0; r < 8; ++r) {
-    const int qi = 8 * rb + r;
-    const int64_t q = q0 + qi;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (q < p.Nq) {
-      const uint4 v = *reinterpret_cast<const uint4*>(p.Q + ((int64_t)h * p.Nq + q) * kD + 8 * cb);
-      const uint32_t x[4] = {v.x, v.y, v.z, v.w};
-      const int64_t pos = p.qpos[q];
+  for (int qt = 0; qt < kAtQTiles; ++qt) {
+    for (int r = 0; r < 4; ++r) {
+      const int qi = 4 * rb + r;
+      const int64_t q = q0 + qt * kAtTile + qi;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if (q < p.Nq) {
+        const uint4 v = *reinterpret_cast<const uint4*>(p.Q + ((int64_t)h * p.Nq + q) * kD + 8 * cb);
+        const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+        const int64_t pos = p.qpos[q];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float a = __uint_as_float(x[e] << 16), b = __uint_as_float(x[e] & 0xFFFF0000u);
-        const float2 cs = rope_cs(p, pos, 4 * cb + e);
-        w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
-                         __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
+        for (int e = 0; e < 4; ++e) {
+          const float a = __uint_as_float(x[e] << 16), b = __uint_as_float(x[e] & 0xFFFF0000u);
+          const float2 cs = rope_cs(p, pos, 4 * cb + e);
+          w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
+                           __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
+        }
       }
+      *reinterpret_cast<uint4*>(sQ + qt * kAtOpBytes + op_off(qi, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    *reinterpret_cast<uint4*>(sQ + op_off(qi, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const uint32_t tS = tmem, tO = tmem + 128;
+  // S of query tile t at column 128 t, O of query tile t at column 256 + 128 t
+  const uint32_t tS = tmem, tO = tmem + 256;
 
-  float m_run = -3.0e38f, l_run = 0.0f;           // softmax state of this thread's query (warps 0-3)
+  // warps 0-3 hold the softmax state of query tile 0, warps 4-7 of tile 1
+  // (row 32 * (warp mod 4) + lane of the tile: the warp's tensor-memory lanes)
+  const bool sm_warp = warp < 4 * kAtQTiles;
+  const int sm_tile = warp >> 2;
+  float m_run = -3.0e38f, l_run = 0.0f;
   const int ntiles = (int)((p.Nk + kAtTile - 1) / kAtTile);
   bool ok = true;
   int j_last = 0;                                 // the tile being worked on when a wait gave up
   for (int j = 0; j < ntiles && ok; ++j) {
     j_last = j;
     const int64_t k0 = (int64_t)j * kAtTile;
-    // the previous product O += P V must be done before its operands are
+    // the previous products O += P V must be done before their operands are
     // overwritten; every thread waits, and the CTA gives up together
     if (j > 0) {
       const bool w_ok = bar_wait(&bars->o_done, (uint32_t)((j - 1) & 1));
       if (__syncthreads_or(!w_ok)) { ok = false; break; }
       fence_after();
     }
-    // 1. reconstruct the K and V tile into the operand layouts, four of the
-    // thread's eight tokens at a time (registers: two CTAs share an SM)
-#pragma unroll 1
-    for (int half = 0; half < 2; ++half) {
+    // 1. reconstruct the K and V tile into the operand layouts (once for
+    // both query tiles)
+    {
       float vk[4][8];
-      const int r0 = 8 * rb + 4 * half;
+      const int r0 = 4 * rb;
       const int64_t tok0 = k0 + r0;
       recon_block<TT, 4>(p, nlut, 0, h, tok0, 8 * cb, vk);
       // K rows: rotary embedding of the reconstructed values, then bf16
@@ -393,9 +401,9 @@ qvg_attention_fused(const AttnParams p) {
         *reinterpret_cast<uint4*>(sK + op_off(r0 + r, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       // V, transposed (channel 8*cbv + e holds keys rv .. rv+3 in 8 contiguous
-      // bytes), with the thread's key and channel blocks swapped: the eight
-      // lanes of a store phase then write eight key chunks of one channel row
-      const int rv = 8 * rbv + 4 * half;
+      // bytes), with the thread's key and channel blocks swapped: the lanes of
+      // a store phase then write distinct key chunks of one channel row
+      const int rv = 4 * rbv;
       recon_block<TT, 4>(p, nlut, 1, h, k0 + rv, 8 * cbv, vk);
 #pragma unroll
       for (int e = 0; e < 8; ++e)
@@ -406,29 +414,36 @@ qvg_attention_fused(const AttnParams p) {
     fence_before();
     __syncthreads();
     fence_after();
-    // 2. S = Q' K'^T
+    // 2. S_t = Q_t' K'^T for both query tiles
     if (threadIdx.x == 0) {
-      const uint32_t a0 = smem_addr(sQ), b0 = smem_addr(sK);
+      const uint32_t b0 = smem_addr(sK);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) mma(tS, op_desc_k(a0, kk), op_desc_k(b0, kk), kk > 0 ? 1u : 0u);
+      for (int qt = 0; qt < kAtQTiles; ++qt) {
+        const uint32_t a0 = smem_addr(sQ + qt * kAtOpBytes);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma(tS + 128 * qt, op_desc_k(a0, kk), op_desc_k(b0, kk), kk > 0 ? 1u : 0u);
+      }
       mma_commit(&bars->s_done);
     }
-    // 3. online softmax (warps 0-3: the thread's query is row 32*warp + lane)
-    if (warp < 4) {
+    // 3. online softmax (warps 0-7: the thread's query is row 32*(warp mod 4) + lane of tile warp/4)
+    if (sm_warp) {
       // warp-uniform outcome: the tensor-memory loads below are warp-collective
       if (!__all_sync(0xffffffffu, bar_wait(&bars->s_done, (uint32_t)(j & 1)))) {
         *reinterpret_cast<volatile int*>(&bars->abort_flag) = 1;
       } else {
         fence_after();
-        const int qi = 32 * warp + lane;
-        const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+        const int qi = 32 * (warp & 3) + lane;
+        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        const uint32_t tSt = tS + 128 * sm_tile, tOt = tO + 128 * sm_tile;
+        uint8_t* sP = sm_tile == 0 ? sK : sP1;
         const int valid = (int)(p.Nk - k0 < kAtTile ? p.Nk - k0 : kAtTile);
         // pass 1: the row maximum, 32 columns at a time
         float mt = -3.0e38f;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
-          tld32(tS + lane_base + (uint32_t)(32 * c), r);
+          tld32(tSt + lane_base + (uint32_t)(32 * c), r);
 #pragma unroll
           for (int e = 0; e < 32; ++e)
             if (32 * c + e < valid) mt = fmaxf(mt, __uint_as_float(r[e]) * p.sl);
@@ -440,7 +455,7 @@ qvg_attention_fused(const AttnParams p) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
-          tld32(tS + lane_base + (uint32_t)(32 * c), r);
+          tld32(tSt + lane_base + (uint32_t)(32 * c), r);
 #pragma unroll
           for (int kg = 0; kg < 4; ++kg) {
             uint32_t w[4];
@@ -453,20 +468,20 @@ qvg_attention_fused(const AttnParams p) {
               // the sum takes the rounded weights, the ones the product uses
               sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
             }
-            *reinterpret_cast<uint4*>(sK + op_off(qi, 32 * c + 8 * kg)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(sP + op_off(qi, 32 * c + 8 * kg)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
         l_run = l_run * alpha + sum;
         m_run = m_new;
-        // rescale O (the previous product is complete: waited for above)
+        // rescale O (the previous products are complete: waited for above)
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t r[32];
-            tld32(tO + lane_base + (uint32_t)(32 * c), r);
+            tld32(tOt + lane_base + (uint32_t)(32 * c), r);
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tst32(tO + lane_base + (uint32_t)(32 * c), r);
+            tst32(tOt + lane_base + (uint32_t)(32 * c), r);
           }
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         }
@@ -477,29 +492,35 @@ qvg_attention_fused(const AttnParams p) {
     __syncthreads();
     fence_after();
     if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) { ok = false; break; }
-    // 4. O += P V
+    // 4. O_t += P_t V for both query tiles
     if (threadIdx.x == 0) {
-      const uint32_t a0 = smem_addr(sK), b0 = smem_addr(sV);
+      const uint32_t b0 = smem_addr(sV);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) mma(tO, op_desc_k(a0, kk), op_desc_k(b0, kk), (j > 0 || kk > 0) ? 1u : 0u);
+      for (int qt = 0; qt < kAtQTiles; ++qt) {
+        const uint32_t a0 = smem_addr(qt == 0 ? sK : sP1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma(tO + 128 * qt, op_desc_k(a0, kk), op_desc_k(b0, kk), (j > 0 || kk > 0) ? 1u : 0u);
+      }
       mma_commit(&bars->o_done);
     }
   }
-  // the last product, then O / l (ok is uniform over the CTA here)
+  // the last products, then O / l (ok is uniform over the CTA here)
   if (ok && ntiles > 0) {
     const bool w_ok = bar_wait(&bars->o_done, (uint32_t)((ntiles - 1) & 1));
     ok = !__syncthreads_or(!w_ok);
     fence_after();
   }
-  if (warp < 4 && ok && ntiles > 0) {
-    const int qi = 32 * warp + lane;
-    const int64_t q = q0 + qi;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+  if (sm_warp && ok && ntiles > 0) {
+    const int qi = 32 * (warp & 3) + lane;
+    const int64_t q = q0 + sm_tile * kAtTile + qi;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tOt = tO + 128 * sm_tile;
     const float inv = 1.0f / l_run;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t r[32];
-      tld32(tO + lane_base + (uint32_t)(32 * c), r);
+      tld32(tOt + lane_base + (uint32_t)(32 * c), r);
       if (q < p.Nq) {
         float4* dst = reinterpret_cast<float4*>(p.O + ((int64_t)h * p.Nq + q) * kD + 32 * c);
 #pragma unroll
@@ -512,7 +533,7 @@ qvg_attention_fused(const AttnParams p) {
   if (!ok && threadIdx.x == 0) {
     atomicOr(p.status, 1u);
     // let the products already issued finish (bounded) before the tensor
-    // memory is freed: the last S product of tile j_last and the O product
+    // memory is freed: the last S products of tile j_last and the O products
     // of the tile before it; a phase that already completed returns at once
     bar_wait(&bars->s_done, (uint32_t)(j_last & 1));
     if (j_last > 0) bar_wait(&bars->o_done, (uint32_t)((j_last - 1) & 1));
@@ -521,7 +542,7 @@ qvg_attention_fused(const AttnParams p) {
   __syncthreads();
   if (warp == 0) {
     fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
   }
 }
 
@@ -543,7 +564,9 @@ __global__ void qvg_rope_tables_kernel(float2* hi, float2* lo, int n_hi, double 
 
 }  // namespace
 
-size_t attention_smem_bytes() { return 1024 + 3 * (size_t)kAtOpBytes + 256 * sizeof(float) + sizeof(AtBars); }
+size_t attention_smem_bytes() {
+  return 1024 + (size_t)(kAtQTiles + 3) * kAtOpBytes + 32 * sizeof(float2) + sizeof(AtBars);
+}
 
 cudaError_t launch_rope_tables(void* tables, int n_hi, double base, cudaStream_t s) {
   float2* hi = reinterpret_cast<float2*>(static_cast<char*>(tables) + kRopeHeaderBytes);
@@ -579,7 +602,7 @@ cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s) {
   p.Nk = a.Nk; p.Nq = a.Nq; p.H = a.H; p.K = a.K; p.T = a.T; p.G = a.G; p.sym = a.sym;
   p.sl = 1.4426950408889634f / sqrtf((float)kD);
   const size_t smem = attention_smem_bytes();
-  const dim3 grid((unsigned)((a.Nq + kAtTile - 1) / kAtTile), (unsigned)a.H);
+  const dim3 grid((unsigned)((a.Nq + kAtQTiles * kAtTile - 1) / (kAtQTiles * kAtTile)), (unsigned)a.H);
   switch (a.T) {
     case 0: return launch_attention_t<0>(p, grid, smem, s);
     case 1: return launch_attention_t<1>(p, grid, smem, s);
