@@ -47,6 +47,8 @@ namespace {
 
 constexpr int kAtThreads = 512;                 // 16 warps
 constexpr int kAtQTiles = 2;                    // query tiles per CTA (each reconstructed K/V tile serves both)
+constexpr int kAtSoftmaxThreads = 256;          // warps 0-7: softmax of the two query tiles (thread 0 issues the MMAs)
+constexpr int kAtReconThreads = 256;            // warps 8-15: reconstruction into the K/V ring
 constexpr int kAtTile = 128;                    // queries per CTA, cached tokens per tile
 constexpr int kAtOpBytes = kAtTile * kD * 2;    // one 128 x 128 bf16 operand: 32 KB
 constexpr uint64_t kAtWaitNs = 2000000000ull;   // 2 s per bounded wait
@@ -71,8 +73,10 @@ struct AttnParams {
 };
 
 struct __align__(8) AtBars {
-  uint64_t s_done;
-  uint64_t o_done;
+  uint64_t s_done;          // S products of a tile complete (tcgen05.commit)
+  uint64_t o_done;          // O products of a tile complete (tcgen05.commit)
+  uint64_t kv_full[2];      // ring stage reconstructed (the 256 reconstruction threads arrive)
+  uint64_t kv_empty[2];     // ring stage free again: the O products that read it completed
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -101,6 +105,49 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity) {
       else if (now - t0 > kAtWaitNs) return false;
     }
   }
+}
+
+// bar_wait that also gives up as soon as another role of the CTA has
+// recorded an abort (so that no role waits out the full limit for a
+// partner that has stopped).
+__device__ __forceinline__ bool bar_wait_or_abort(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
+  const uint32_t addr = smem_addr(bar);
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort_flag) return false;
+      uint64_t now;
+      asm volatile("mov.u64 %0, %globaltimer;" : "=l"(now));
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kAtWaitNs) return false;
+    }
+  }
+}
+// Named barrier over `count` threads with an OR of `pred` (every participant
+// gets the same answer).
+__device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 // Shared-memory operand descriptor, K-major, 128-byte swizzle: a 128 x 128
@@ -298,22 +345,25 @@ qvg_attention_fused(const AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                               // A of S: two query tiles x channels
-  uint8_t* sK = sQ + kAtQTiles * kAtOpBytes;        // B of S: keys x channels; then A of O for query tile 0 (P)
-  uint8_t* sV = sK + kAtOpBytes;                    // B of O: channels x keys
-  uint8_t* sP1 = sV + kAtOpBytes;                   // A of O for query tile 1 (P)
+  uint8_t* sK0 = sQ + kAtQTiles * kAtOpBytes;       // ring stage s: K at sK0 + 2s tiles, V after it
+  uint8_t* sP1 = sK0 + 4 * kAtOpBytes;              // A of O for query tile 1 (P)
   float2* nlut = reinterpret_cast<float2*>(sP1 + kAtOpBytes);   // nibble -> two codes (q, or u - 2)
   AtBars* bars = reinterpret_cast<AtBars*>(nlut + 32);
+  volatile int* abort_flag = &bars->abort_flag;
+  auto stage_k = [&](int st) { return sK0 + (2 * st) * kAtOpBytes; };   // B of S; then A of O for tile 0 (P)
+  auto stage_v = [&](int st) { return sK0 + (2 * st + 1) * kAtOpBytes; };
 
   const int h = blockIdx.y;
   const int64_t q0 = (int64_t)blockIdx.x * (kAtQTiles * kAtTile);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // the thread's 4 x 8 block of a 128 x 128 tile: rows 4*rb .. 4*rb+3, channels 8*cb .. 8*cb+7
-  const int rb = threadIdx.x >> 4, cb = threadIdx.x & 15;
-  const int rbv = threadIdx.x & 31, cbv = threadIdx.x >> 5;   // the same blocks, transposed, for V
 
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->s_done)));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->o_done)));
+    for (int st = 0; st < 2; ++st) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&bars->kv_full[st])), "r"(kAtReconThreads));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->kv_empty[st])));
+    }
     bars->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -326,26 +376,29 @@ qvg_attention_fused(const AttnParams p) {
     const float off = p.sym ? 2.0f : 0.0f;
     nlut[threadIdx.x] = make_float2((float)(threadIdx.x & 3u) - off, (float)(threadIdx.x >> 2) - off);
   }
-
   // queries: rotary embedding at their positions, bf16, into the A layout
-  for (int qt = 0; qt < kAtQTiles; ++qt) {
-    for (int r = 0; r < 4; ++r) {
-      const int qi = 4 * rb + r;
-      const int64_t q = q0 + qt * kAtTile + qi;
-      uint32_t w[4] = {0u, 0u, 0u, 0u};
-      if (q < p.Nq) {
-        const uint4 v = *reinterpret_cast<const uint4*>(p.Q + ((int64_t)h * p.Nq + q) * kD + 8 * cb);
-        const uint32_t x[4] = {v.x, v.y, v.z, v.w};
-        const int64_t pos = p.qpos[q];
+  // (all 512 threads: rows 4*rb .. 4*rb+3 of each tile, channels 8*cb ..)
+  {
+    const int rb = threadIdx.x >> 4, cb = threadIdx.x & 15;
+    for (int qt = 0; qt < kAtQTiles; ++qt) {
+      for (int r = 0; r < 4; ++r) {
+        const int qi = 4 * rb + r;
+        const int64_t q = q0 + qt * kAtTile + qi;
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        if (q < p.Nq) {
+          const uint4 v = *reinterpret_cast<const uint4*>(p.Q + ((int64_t)h * p.Nq + q) * kD + 8 * cb);
+          const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+          const int64_t pos = p.qpos[q];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = __uint_as_float(x[e] << 16), b = __uint_as_float(x[e] & 0xFFFF0000u);
-          const float2 cs = rope_cs(p, pos, 4 * cb + e);
-          w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
-                           __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
+          for (int e = 0; e < 4; ++e) {
+            const float a = __uint_as_float(x[e] << 16), b = __uint_as_float(x[e] & 0xFFFF0000u);
+            const float2 cs = rope_cs(p, pos, 4 * cb + e);
+            w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
+                             __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
+          }
         }
+        *reinterpret_cast<uint4*>(sQ + qt * kAtOpBytes + op_off(qi, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      *reinterpret_cast<uint4*>(sQ + qt * kAtOpBytes + op_off(qi, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
   fence_before();
@@ -354,116 +407,131 @@ qvg_attention_fused(const AttnParams p) {
   const uint32_t tmem = bars->tmem_base;
   // S of query tile t at column 128 t, O of query tile t at column 256 + 128 t
   const uint32_t tS = tmem, tO = tmem + 256;
-
-  // warps 0-3 hold the softmax state of query tile 0, warps 4-7 of tile 1
-  // (row 32 * (warp mod 4) + lane of the tile: the warp's tensor-memory lanes)
-  const bool sm_warp = warp < 4 * kAtQTiles;
-  const int sm_tile = warp >> 2;
-  float m_run = -3.0e38f, l_run = 0.0f;
   const int ntiles = (int)((p.Nk + kAtTile - 1) / kAtTile);
-  bool ok = true;
-  int j_last = 0;                                 // the tile being worked on when a wait gave up
-  for (int j = 0; j < ntiles && ok; ++j) {
-    j_last = j;
-    const int64_t k0 = (int64_t)j * kAtTile;
-    // the previous products O += P V must be done before their operands are
-    // overwritten; every thread waits, and the CTA gives up together
-    if (j > 0) {
-      const bool w_ok = bar_wait(&bars->o_done, (uint32_t)((j - 1) & 1));
-      if (__syncthreads_or(!w_ok)) { ok = false; break; }
+  int s_issued = 0, o_issued = 0;                   // products committed (thread 0)
+
+  if (warp >= 8) {
+    // ---------------------------------------------------------------- reconstruction warps
+    // tile j goes to ring stage j mod 2 once the O products of tile j - 2
+    // (the stage's last readers) have completed
+    const int r = threadIdx.x - kAtSoftmaxThreads;
+    const int rb = r >> 4, cb = r & 15;             // K: rows 8*rb .. 8*rb+7, channels 8*cb ..
+    const int rbv = r & 15, cbv = r >> 4;           // V: the same blocks, transposed
+    for (int j = 0; j < ntiles; ++j) {
+      const int st = j & 1;
+      if (j >= 2 && !bar_wait_or_abort(&bars->kv_empty[st], (uint32_t)(((j >> 1) - 1) & 1), abort_flag)) {
+        *abort_flag = 1;
+        break;
+      }
       fence_after();
-    }
-    // 1. reconstruct the K and V tile into the operand layouts (once for
-    // both query tiles)
-    {
-      float vk[4][8];
-      const int r0 = 4 * rb;
-      const int64_t tok0 = k0 + r0;
-      recon_block<TT, 4>(p, nlut, 0, h, tok0, 8 * cb, vk);
-      // K rows: rotary embedding of the reconstructed values, then bf16
-      const int64_t pa = rope_pos(p, tok0), pz = rope_pos(p, tok0 + 3);
-      const bool one_hi = pa / kRopeLo == pz / kRopeLo;   // the four positions share the high entry
-      float2 hi[4];
+      uint8_t* sK = stage_k(st);
+      uint8_t* sV = stage_v(st);
+      const int64_t k0 = (int64_t)j * kAtTile;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        float vk[4][8];
+        const int r0 = 8 * rb + 4 * half;
+        const int64_t tok0 = k0 + r0;
+        recon_block<TT, 4>(p, nlut, 0, h, tok0, 8 * cb, vk);
+        // K rows: rotary embedding of the reconstructed values, then bf16
+        const int64_t pa = rope_pos(p, tok0), pz = rope_pos(p, tok0 + 3);
+        const bool one_hi = pa / kRopeLo == pz / kRopeLo;   // the four positions share the high entry
+        float2 hi[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) hi[e] = p.rope_hi[(pa / kRopeLo) * (kD / 2) + 4 * cb + e];
+        for (int e = 0; e < 4; ++e) hi[e] = p.rope_hi[(pa / kRopeLo) * (kD / 2) + 4 * cb + e];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        uint32_t w[4];
-        const int64_t pr = rope_pos(p, tok0 + r);
+        for (int rr = 0; rr < 4; ++rr) {
+          uint32_t w[4];
+          const int64_t pr = rope_pos(p, tok0 + rr);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 cs = one_hi ? rope_combine(hi[e], p.rope_lo[(pr % kRopeLo) * (kD / 2) + 4 * cb + e])
-                                   : rope_cs(p, tok0 + r, 4 * cb + e);
-          const float a = vk[r][2 * e], b = vk[r][2 * e + 1];
-          w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
-                           __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
+          for (int e = 0; e < 4; ++e) {
+            const float2 cs = one_hi ? rope_combine(hi[e], p.rope_lo[(pr % kRopeLo) * (kD / 2) + 4 * cb + e])
+                                     : rope_cs(p, tok0 + rr, 4 * cb + e);
+            const float a = vk[rr][2 * e], b = vk[rr][2 * e + 1];
+            w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
+                             __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
+          }
+          *reinterpret_cast<uint4*>(sK + op_off(r0 + rr, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        *reinterpret_cast<uint4*>(sK + op_off(r0 + r, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
+        // V, transposed (channel 8*cbv + e holds keys rv .. rv+3 in 8 contiguous
+        // bytes), with the key and channel blocks swapped: the eight lanes of a
+        // store phase write eight key chunks of one channel row
+        const int rv = 8 * rbv + 4 * half;
+        recon_block<TT, 4>(p, nlut, 1, h, k0 + rv, 8 * cbv, vk);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          *reinterpret_cast<uint2*>(sV + op_off(8 * cbv + e, rv)) =
+              make_uint2(pack_bf16(vk[0][e], vk[1][e]), pack_bf16(vk[2][e], vk[3][e]));
       }
-      // V, transposed (channel 8*cbv + e holds keys rv .. rv+3 in 8 contiguous
-      // bytes), with the thread's key and channel blocks swapped: the lanes of
-      // a store phase then write distinct key chunks of one channel row
-      const int rv = 4 * rbv;
-      recon_block<TT, 4>(p, nlut, 1, h, k0 + rv, 8 * cbv, vk);
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        *reinterpret_cast<uint2*>(sV + op_off(8 * cbv + e, rv)) =
-            make_uint2(pack_bf16(vk[0][e], vk[1][e]), pack_bf16(vk[2][e], vk[3][e]));
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
+      mbar_arrive(&bars->kv_full[st]);
+      if (*abort_flag) break;
     }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
-    fence_before();
-    __syncthreads();
-    fence_after();
-    // 2. S_t = Q_t' K'^T for both query tiles
-    if (threadIdx.x == 0) {
-      const uint32_t b0 = smem_addr(sK);
+  } else {
+    // ---------------------------------------------------------------- softmax warps (thread 0 issues the products)
+    // warps 0-3 hold query tile 0, warps 4-7 tile 1: row 32*(warp mod 4) + lane,
+    // the warp's tensor-memory lane quarter
+    const int sm_tile = warp >> 2;
+    const int qi = 32 * (warp & 3) + lane;
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tSt = tS + 128 * sm_tile, tOt = tO + 128 * sm_tile;
+    float m_run = -3.0e38f, l_run = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int st = j & 1;
+      const int64_t k0 = (int64_t)j * kAtTile;
+      uint8_t* sK = stage_k(st);
+      // 1. S_t = Q_t' K'^T for both query tiles, once the stage is reconstructed
+      if (threadIdx.x == 0) {
+        if (bar_wait_or_abort(&bars->kv_full[st], (uint32_t)((j >> 1) & 1), abort_flag)) {
+          fence_after();
+          const uint32_t b0 = smem_addr(sK);
 #pragma unroll
-      for (int qt = 0; qt < kAtQTiles; ++qt) {
-        const uint32_t a0 = smem_addr(sQ + qt * kAtOpBytes);
+          for (int qt = 0; qt < kAtQTiles; ++qt) {
+            const uint32_t a0 = smem_addr(sQ + qt * kAtOpBytes);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma(tS + 128 * qt, op_desc_k(a0, kk), op_desc_k(b0, kk), kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk)
+              mma(tS + 128 * qt, op_desc_k(a0, kk), op_desc_k(b0, kk), kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars->s_done);
+          ++s_issued;
+        } else {
+          *abort_flag = 1;
+        }
       }
-      mma_commit(&bars->s_done);
-    }
-    // 3. online softmax (warps 0-7: the thread's query is row 32*(warp mod 4) + lane of tile warp/4)
-    if (sm_warp) {
-      // warp-uniform outcome: the tensor-memory loads below are warp-collective
-      if (!__all_sync(0xffffffffu, bar_wait(&bars->s_done, (uint32_t)(j & 1)))) {
-        *reinterpret_cast<volatile int*>(&bars->abort_flag) = 1;
-      } else {
-        fence_after();
-        const int qi = 32 * (warp & 3) + lane;
-        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-        const uint32_t tSt = tS + 128 * sm_tile, tOt = tO + 128 * sm_tile;
+      // 2. the scores, and the previous tile's products (O rescale, P_1 buffer)
+      bool w_ok = bar_wait_or_abort(&bars->s_done, (uint32_t)(j & 1), abort_flag);
+      if (w_ok && j > 0) w_ok = bar_wait_or_abort(&bars->o_done, (uint32_t)((j - 1) & 1), abort_flag);
+      if (named_bar_or(1, kAtSoftmaxThreads, !w_ok)) { ok = false; break; }
+      fence_after();
+      // 3. online softmax of the thread's query row
+      {
         uint8_t* sP = sm_tile == 0 ? sK : sP1;
         const int valid = (int)(p.Nk - k0 < kAtTile ? p.Nk - k0 : kAtTile);
-        // pass 1: the row maximum, 32 columns at a time
-        float mt = -3.0e38f;
+        float mt = -3.0e38f;                          // pass 1: the row maximum, 32 columns at a time
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tld32(tSt + lane_base + (uint32_t)(32 * c), r);
+          uint32_t rg[32];
+          tld32(tSt + lane_base + (uint32_t)(32 * c), rg);
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            if (32 * c + e < valid) mt = fmaxf(mt, __uint_as_float(r[e]) * p.sl);
+            if (32 * c + e < valid) mt = fmaxf(mt, __uint_as_float(rg[e]) * p.sl);
         }
         const float m_new = fmaxf(m_run, mt);
         const float alpha = exp2_approx(m_run - m_new);
-        // pass 2: the weights, rounded to bf16 into the P operand, and their sum
-        float sum = 0.0f;
+        float sum = 0.0f;                             // pass 2: bf16 weights into P, and their sum
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tld32(tSt + lane_base + (uint32_t)(32 * c), r);
+          uint32_t rg[32];
+          tld32(tSt + lane_base + (uint32_t)(32 * c), rg);
 #pragma unroll
           for (int kg = 0; kg < 4; ++kg) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int j0 = 32 * c + 8 * kg + 2 * e;
-              const float pa = j0 < valid ? exp2_approx(__uint_as_float(r[8 * kg + 2 * e]) * p.sl - m_new) : 0.0f;
-              const float pb = j0 + 1 < valid ? exp2_approx(__uint_as_float(r[8 * kg + 2 * e + 1]) * p.sl - m_new) : 0.0f;
+              const float pa = j0 < valid ? exp2_approx(__uint_as_float(rg[8 * kg + 2 * e]) * p.sl - m_new) : 0.0f;
+              const float pb = j0 + 1 < valid ? exp2_approx(__uint_as_float(rg[8 * kg + 2 * e + 1]) * p.sl - m_new) : 0.0f;
               w[e] = pack_bf16(pa, pb);
               // the sum takes the rounded weights, the ones the product uses
               sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
@@ -473,72 +541,70 @@ qvg_attention_fused(const AttnParams p) {
         }
         l_run = l_run * alpha + sum;
         m_run = m_new;
-        // rescale O (the previous products are complete: waited for above)
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {   // rescale O
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tld32(tOt + lane_base + (uint32_t)(32 * c), r);
+            uint32_t rg[32];
+            tld32(tOt + lane_base + (uint32_t)(32 * c), rg);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tst32(tOt + lane_base + (uint32_t)(32 * c), r);
+            for (int e = 0; e < 32; ++e) rg[e] = __float_as_uint(__uint_as_float(rg[e]) * alpha);
+            tst32(tOt + lane_base + (uint32_t)(32 * c), rg);
           }
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         }
       }
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    fence_before();
-    __syncthreads();
-    fence_after();
-    if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) { ok = false; break; }
-    // 4. O_t += P_t V for both query tiles
-    if (threadIdx.x == 0) {
-      const uint32_t b0 = smem_addr(sV);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      fence_before();
+      named_bar_or(1, kAtSoftmaxThreads, false);       // P of both tiles written, O rescaled
+      // 4. O_t += P_t V for both query tiles; the stage is free once they complete
+      if (threadIdx.x == 0) {
+        fence_after();
+        const uint32_t b0 = smem_addr(stage_v(st));
 #pragma unroll
-      for (int qt = 0; qt < kAtQTiles; ++qt) {
-        const uint32_t a0 = smem_addr(qt == 0 ? sK : sP1);
+        for (int qt = 0; qt < kAtQTiles; ++qt) {
+          const uint32_t a0 = smem_addr(qt == 0 ? sK : sP1);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma(tO + 128 * qt, op_desc_k(a0, kk), op_desc_k(b0, kk), (j > 0 || kk > 0) ? 1u : 0u);
-      }
-      mma_commit(&bars->o_done);
-    }
-  }
-  // the last products, then O / l (ok is uniform over the CTA here)
-  if (ok && ntiles > 0) {
-    const bool w_ok = bar_wait(&bars->o_done, (uint32_t)((ntiles - 1) & 1));
-    ok = !__syncthreads_or(!w_ok);
-    fence_after();
-  }
-  if (sm_warp && ok && ntiles > 0) {
-    const int qi = 32 * (warp & 3) + lane;
-    const int64_t q = q0 + sm_tile * kAtTile + qi;
-    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tOt = tO + 128 * sm_tile;
-    const float inv = 1.0f / l_run;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t r[32];
-      tld32(tOt + lane_base + (uint32_t)(32 * c), r);
-      if (q < p.Nq) {
-        float4* dst = reinterpret_cast<float4*>(p.O + ((int64_t)h * p.Nq + q) * kD + 32 * c);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          dst[e] = make_float4(__uint_as_float(r[4 * e]) * inv, __uint_as_float(r[4 * e + 1]) * inv,
-                               __uint_as_float(r[4 * e + 2]) * inv, __uint_as_float(r[4 * e + 3]) * inv);
+          for (int kk = 0; kk < 8; ++kk)
+            mma(tO + 128 * qt, op_desc_k(a0, kk), op_desc_k(b0, kk), (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&bars->o_done);
+        mma_commit(&bars->kv_empty[st]);
+        ++o_issued;
       }
     }
-  }
-  if (!ok && threadIdx.x == 0) {
-    atomicOr(p.status, 1u);
-    // let the products already issued finish (bounded) before the tensor
-    // memory is freed: the last S products of tile j_last and the O products
-    // of the tile before it; a phase that already completed returns at once
-    bar_wait(&bars->s_done, (uint32_t)(j_last & 1));
-    if (j_last > 0) bar_wait(&bars->o_done, (uint32_t)((j_last - 1) & 1));
+    // the last products, then O / l
+    if (ok && ntiles > 0) {
+      const bool w_ok = bar_wait_or_abort(&bars->o_done, (uint32_t)((ntiles - 1) & 1), abort_flag);
+      ok = !named_bar_or(1, kAtSoftmaxThreads, !w_ok);
+      fence_after();
+    }
+    if (!ok) *abort_flag = 1;
+    if (ok && ntiles > 0) {
+      const int64_t q = q0 + sm_tile * kAtTile + qi;
+      const float inv = 1.0f / l_run;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rg[32];
+        tld32(tOt + lane_base + (uint32_t)(32 * c), rg);
+        if (q < p.Nq) {
+          float4* dst = reinterpret_cast<float4*>(p.O + ((int64_t)h * p.Nq + q) * kD + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(rg[4 * e]) * inv, __uint_as_float(rg[4 * e + 1]) * inv,
+                                 __uint_as_float(rg[4 * e + 2]) * inv, __uint_as_float(rg[4 * e + 3]) * inv);
+        }
+      }
+    }
   }
   fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    atomicOr(p.status, 1u);
+    // let the products already issued finish (bounded) before the tensor
+    // memory is freed; a phase that already completed returns at once
+    if (s_issued > 0) bar_wait(&bars->s_done, (uint32_t)((s_issued - 1) & 1));
+    if (o_issued > 0) bar_wait(&bars->o_done, (uint32_t)((o_issued - 1) & 1));
+  }
   __syncthreads();
   if (warp == 0) {
     fence_after();
@@ -565,7 +631,7 @@ __global__ void qvg_rope_tables_kernel(float2* hi, float2* lo, int n_hi, double 
 }  // namespace
 
 size_t attention_smem_bytes() {
-  return 1024 + (size_t)(kAtQTiles + 3) * kAtOpBytes + 32 * sizeof(float2) + sizeof(AtBars);
+  return 1024 + (size_t)(kAtQTiles + 5) * kAtOpBytes + 32 * sizeof(float2) + sizeof(AtBars);
 }
 
 cudaError_t launch_rope_tables(void* tables, int n_hi, double base, cudaStream_t s) {
