@@ -263,7 +263,7 @@ __device__ __forceinline__ float2 rope_combine(float2 a, float2 b) {
 }
 __device__ __forceinline__ float2 rope_cs(const AttnParams& p, int64_t pos, int i) {
   pos = rope_pos(p, pos);
-  return rope_combine(p.rope_hi[(pos / kRopeLo) * (kD / 2) + i], p.rope_lo[(pos % kRopeLo) * (kD / 2) + i]);
+  return rope_combine(__ldg(p.rope_hi + (pos / kRopeLo) * (kD / 2) + i), __ldg(p.rope_lo + (pos % kRopeLo) * (kD / 2) + i));
 }
 
 // Reconstruct channels c0 .. c0+7 of the NR tokens tok0 .. tok0+NR-1 (those
@@ -287,11 +287,12 @@ __device__ __forceinline__ void recon_block(const AttnParams& p, const float2* n
   for (int r = 0; r < NR; ++r) {
     const int64_t tok = tok0 + r < p.Nk ? tok0 + r : p.Nk - 1;   // past the end: a valid token, result unused
     const int64_t row = (int64_t)h * p.Nk + tok;
-    code[r] = *reinterpret_cast<const uint16_t*>(p.codes[which] + row * (kD / 4) + c0 / 4);
-    sz[r] = (uint32_t)p.scale[which][row * ng + g] | (p.sym ? 0u : ((uint32_t)p.zero[which][row * ng + g] << 8));
+    code[r] = __ldg(reinterpret_cast<const unsigned short*>(p.codes[which] + row * (kD / 4) + c0 / 4));
+    sz[r] = (uint32_t)__ldg(p.scale[which] + row * ng + g) |
+            (p.sym ? 0u : ((uint32_t)__ldg(p.zero[which] + row * ng + g) << 8));
 #pragma unroll
     for (int t = 0; t < TR; ++t)
-      if (TT > 0) kk[r][t] = min((int)p.assign[which][((int64_t)t * p.H + h) * p.Nk + tok], p.K - 1);
+      if (TT > 0) kk[r][t] = min((int)__ldg(p.assign[which] + ((int64_t)t * p.H + h) * p.Nk + tok), p.K - 1);
   }
   uint4 rows[NR][TR];
   if (TT > 0) {
@@ -299,7 +300,7 @@ __device__ __forceinline__ void recon_block(const AttnParams& p, const float2* n
     for (int r = 0; r < NR; ++r)
 #pragma unroll
       for (int t = 0; t < TR; ++t)
-        rows[r][t] = *reinterpret_cast<const uint4*>(p.tab[which] + (((int64_t)t * p.H + h) * p.K + kk[r][t]) * kD + c0);
+        rows[r][t] = __ldg(reinterpret_cast<const uint4*>(p.tab[which] + (((int64_t)t * p.H + h) * p.K + kk[r][t]) * kD + c0));
   }
 #pragma unroll
   for (int r = 0; r < NR; ++r) {
@@ -438,14 +439,14 @@ qvg_attention_fused(const AttnParams p) {
         const bool one_hi = pa / kRopeLo == pz / kRopeLo;   // the four positions share the high entry
         float2 hi[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) hi[e] = p.rope_hi[(pa / kRopeLo) * (kD / 2) + 4 * cb + e];
+        for (int e = 0; e < 4; ++e) hi[e] = __ldg(p.rope_hi + (pa / kRopeLo) * (kD / 2) + 4 * cb + e);
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
           uint32_t w[4];
           const int64_t pr = rope_pos(p, tok0 + rr);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 cs = one_hi ? rope_combine(hi[e], p.rope_lo[(pr % kRopeLo) * (kD / 2) + 4 * cb + e])
+            const float2 cs = one_hi ? rope_combine(hi[e], __ldg(p.rope_lo + (pr % kRopeLo) * (kD / 2) + 4 * cb + e))
                                      : rope_cs(p, tok0 + rr, 4 * cb + e);
             const float a = vk[rr][2 * e], b = vk[rr][2 * e + 1];
             w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
