@@ -817,26 +817,34 @@ qvg_update_centroids(const UpdateParams p) {
   if (k >= p.K) return;
   const bool full = p.pi_old == nullptr;
   const int* off_u = p.off + (int64_t)u * (p.K + 1);
-  if (!full && off_u[k + 1] == off_u[k]) return;   // no entries: unchanged
-  int n = p.cnt[(int64_t)u * p.K + k];
-  if (!full) n += p.n[(int64_t)u * p.K + k];
-  if (lane == 0) p.n[(int64_t)u * p.K + k] = n;
-  if (n <= 0) return;                                // an empty centroid keeps its value
+  // every load of the warp is issued before any of them is used: the bucket
+  // bounds, the count (change), the 128 sums and the channel ranges
+  const int o0 = off_u[k], o1 = off_u[k + 1];
+  const int cnt = p.cnt[(int64_t)u * p.K + k];
+  const int n_old = full ? 0 : p.n[(int64_t)u * p.K + k];
   // channel c = 4 * lane + e sits at (c % 8) * 16 + c / 8 of the centroid's sums
   const long long* Sg = p.S + ((int64_t)u * p.K + k) * kD + (4 * (lane & 1)) * 16 + (lane >> 1);
   const long long sum[4] = {Sg[0], Sg[16], Sg[32], Sg[48]};
+  const uint4 cmax = *reinterpret_cast<const uint4*>(p.chmax + (int64_t)u * kD + 4 * lane);
+  const uint4 cmin = *reinterpret_cast<const uint4*>(p.chmin + (int64_t)u * kD + 4 * lane);
+  if (!full && o1 == o0) return;                     // no entries: unchanged
+  const int n = cnt + n_old;
+  if (lane == 0) p.n[(int64_t)u * p.K + k] = n;
+  if (n <= 0) return;                                // an empty centroid keeps its value
+  const uint32_t cmax_e[4] = {cmax.x, cmax.y, cmax.z, cmax.w};
+  const uint32_t cmin_e[4] = {cmin.x, cmin.y, cmin.z, cmin.w};
   const double dn = (double)n;
   double sq = 0.0;
   double mean[4];
   uint32_t wide = 0;                     // this lane's channels outside the fixed-point window
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const int L = fix_exponent(p.chmax[(int64_t)u * kD + 4 * lane + e], p.log2n);
+    const int L = fix_exponent(cmax_e[e], p.log2n);
     const double scale = __longlong_as_double((long long)(1023 + L) << 52);
     mean[e] = __ddiv_rn(__dmul_rn(__ll2double_rn(sum[e]), scale), dn);
     // the quantum of the smallest nonzero value, 2^(e_min - p) with p the
     // stored fraction bits, must be at least 2^L for the sum to be exact
-    const uint32_t inv = p.chmin[(int64_t)u * kD + 4 * lane + e];
+    const uint32_t inv = cmin_e[e];
     if (inv != 0u) {
       const uint32_t mb = 0x7FFFFFFFu - inv;
       const int emin = (int)((mb >> 23) & 0xFFu) == 0 ? -126 : (int)((mb >> 23) & 0xFFu) - 127;
