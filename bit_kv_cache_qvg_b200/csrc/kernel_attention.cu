@@ -45,10 +45,10 @@
 namespace qvg {
 namespace {
 
-constexpr int kAtThreads = 512;                 // 16 warps
+constexpr int kAtThreads = 768;                 // 24 warps
 constexpr int kAtQTiles = 2;                    // query tiles per CTA (each reconstructed K/V tile serves both)
 constexpr int kAtSoftmaxThreads = 256;          // warps 0-7: softmax of the two query tiles (thread 0 issues the MMAs)
-constexpr int kAtReconThreads = 256;            // warps 8-15: reconstruction into the K/V ring
+constexpr int kAtReconThreads = 512;            // warps 8-23: reconstruction into the K/V ring
 constexpr int kAtTile = 128;                    // queries per CTA, cached tokens per tile
 constexpr int kAtOpBytes = kAtTile * kD * 2;    // one 128 x 128 bf16 operand: 32 KB
 constexpr uint64_t kAtWaitNs = 2000000000ull;   // 2 s per bounded wait
@@ -165,8 +165,8 @@ __device__ __forceinline__ uint64_t op_desc(uint32_t saddr) {
   return d;
 }
 constexpr int kAtHalfBytes = kAtTile * 128;     // one 64-column half of an operand
-// Byte offset of element (row, k) (k a multiple of 4 within its chunk is
-// enough for the 8- and 16-byte stores below) of a 128 x 128 operand.
+// Byte offset of element (row, k) of a 128 x 128 operand (k even for the
+// 4-byte stores, a multiple of 8 for the 16-byte ones).
 __device__ __forceinline__ int op_off(int row, int k) {
   return (k >> 6) * kAtHalfBytes + row * 128 + ((((k & 63) >> 3) ^ (row & 7)) << 4) + (k & 7) * 2;
 }
@@ -379,7 +379,7 @@ qvg_attention_fused(const AttnParams p) {
   }
   // queries: rotary embedding at their positions, bf16, into the A layout
   // (all 512 threads: rows 4*rb .. 4*rb+3 of each tile, channels 8*cb ..)
-  {
+  if (threadIdx.x < 512) {
     const int rb = threadIdx.x >> 4, cb = threadIdx.x & 15;
     for (int qt = 0; qt < kAtQTiles; ++qt) {
       for (int r = 0; r < 4; ++r) {
@@ -416,8 +416,8 @@ qvg_attention_fused(const AttnParams p) {
     // tile j goes to ring stage j mod 2 once the O products of tile j - 2
     // (the stage's last readers) have completed
     const int r = threadIdx.x - kAtSoftmaxThreads;
-    const int rb = r >> 4, cb = r & 15;             // K: rows 8*rb .. 8*rb+7, channels 8*cb ..
-    const int rbv = r & 15, cbv = r >> 4;           // V: the same blocks, transposed
+    const int rb = r >> 4, cb = r & 15;             // K: rows 4*rb .. 4*rb+3, channels 8*cb ..
+    const int rbv = r & 31, cbv = r >> 5;           // V: the same blocks, transposed
     for (int j = 0; j < ntiles; ++j) {
       const int st = j & 1;
       if (j >= 2 && !bar_wait_or_abort(&bars->kv_empty[st], (uint32_t)(((j >> 1) - 1) & 1), abort_flag)) {
@@ -430,18 +430,18 @@ qvg_attention_fused(const AttnParams p) {
       const int64_t k0 = (int64_t)j * kAtTile;
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
-        float vk[4][8];
-        const int r0 = 8 * rb + 4 * half;
+        float vk[2][8];
+        const int r0 = 4 * rb + 2 * half;
         const int64_t tok0 = k0 + r0;
-        recon_block<TT, 4>(p, nlut, 0, h, tok0, 8 * cb, vk);
+        recon_block<TT, 2>(p, nlut, 0, h, tok0, 8 * cb, vk);
         // K rows: rotary embedding of the reconstructed values, then bf16
-        const int64_t pa = rope_pos(p, tok0), pz = rope_pos(p, tok0 + 3);
-        const bool one_hi = pa / kRopeLo == pz / kRopeLo;   // the four positions share the high entry
+        const int64_t pa = rope_pos(p, tok0), pz = rope_pos(p, tok0 + 1);
+        const bool one_hi = pa / kRopeLo == pz / kRopeLo;   // the two positions share the high entry
         float2 hi[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) hi[e] = __ldg(p.rope_hi + (pa / kRopeLo) * (kD / 2) + 4 * cb + e);
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
+        for (int rr = 0; rr < 2; ++rr) {
           uint32_t w[4];
           const int64_t pr = rope_pos(p, tok0 + rr);
 #pragma unroll
@@ -454,15 +454,14 @@ qvg_attention_fused(const AttnParams p) {
           }
           *reinterpret_cast<uint4*>(sK + op_off(r0 + rr, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        // V, transposed (channel 8*cbv + e holds keys rv .. rv+3 in 8 contiguous
-        // bytes), with the key and channel blocks swapped: the eight lanes of a
-        // store phase write eight key chunks of one channel row
-        const int rv = 8 * rbv + 4 * half;
-        recon_block<TT, 4>(p, nlut, 1, h, k0 + rv, 8 * cbv, vk);
+        // V, transposed (channel 8*cbv + e holds keys rv, rv+1 in 4 contiguous
+        // bytes), with the key and channel blocks swapped: the lanes of a store
+        // phase write distinct key chunks of one channel row
+        const int rv = 4 * rbv + 2 * half;
+        recon_block<TT, 2>(p, nlut, 1, h, k0 + rv, 8 * cbv, vk);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          *reinterpret_cast<uint2*>(sV + op_off(8 * cbv + e, rv)) =
-              make_uint2(pack_bf16(vk[0][e], vk[1][e]), pack_bf16(vk[2][e], vk[3][e]));
+          *reinterpret_cast<uint32_t*>(sV + op_off(8 * cbv + e, rv)) = pack_bf16(vk[0][e], vk[1][e]);
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
       mbar_arrive(&bars->kv_full[st]);
