@@ -73,10 +73,10 @@ struct AttnParams {
 };
 
 struct __align__(8) AtBars {
-  uint64_t s_done;          // S products of a tile complete (tcgen05.commit)
-  uint64_t o_done;          // O products of a tile complete (tcgen05.commit)
-  uint64_t kv_full[2];      // ring stage reconstructed (the 256 reconstruction threads arrive)
-  uint64_t kv_empty[2];     // ring stage free again: the O products that read it completed
+  uint64_t s_done[2];       // S product of query tile g complete (tcgen05.commit)
+  uint64_t o_done[2];       // O product of query tile g complete (tcgen05.commit)
+  uint64_t kv_full[2];      // ring stage reconstructed (the reconstruction threads arrive)
+  uint64_t kv_empty[2];     // ring stage free again: both O products that read it completed
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -187,6 +187,16 @@ __device__ __forceinline__ void mma(uint32_t tmem_d, uint64_t a, uint64_t b, uin
       "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
       : "memory");
 }
+// The same product with A read from tensor memory (lane i = row i, K
+// elements packed two per 32-bit column, the lower half first).
+__device__ __forceinline__ void mma_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(b), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
                : "memory");
@@ -226,6 +236,35 @@ __device__ __forceinline__ void tst32(uint32_t taddr, const uint32_t (&r)[32]) {
         "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
         "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
+}
+
+__device__ __forceinline__ void tld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  // the registers pass through the wait so that no use moves above it
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+      :
+      : "memory");
+}
+__device__ __forceinline__ void tst16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tst8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 
 __device__ __forceinline__ float exp2_approx(float x) {
@@ -347,11 +386,10 @@ qvg_attention_fused(const AttnParams p) {
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                               // A of S: two query tiles x channels
   uint8_t* sK0 = sQ + kAtQTiles * kAtOpBytes;       // ring stage s: K at sK0 + 2s tiles, V after it
-  uint8_t* sP1 = sK0 + 4 * kAtOpBytes;              // A of O for query tile 1 (P)
-  float2* nlut = reinterpret_cast<float2*>(sP1 + kAtOpBytes);   // nibble -> two codes (q, or u - 2)
+  float2* nlut = reinterpret_cast<float2*>(sK0 + 4 * kAtOpBytes);   // nibble -> two codes (q, or u - 2)
   AtBars* bars = reinterpret_cast<AtBars*>(nlut + 32);
   volatile int* abort_flag = &bars->abort_flag;
-  auto stage_k = [&](int st) { return sK0 + (2 * st) * kAtOpBytes; };   // B of S; then A of O for tile 0 (P)
+  auto stage_k = [&](int st) { return sK0 + (2 * st) * kAtOpBytes; };   // B of S
   auto stage_v = [&](int st) { return sK0 + (2 * st + 1) * kAtOpBytes; };
 
   const int h = blockIdx.y;
@@ -359,11 +397,11 @@ qvg_attention_fused(const AttnParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->s_done)));
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->o_done)));
-    for (int st = 0; st < 2; ++st) {
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&bars->kv_full[st])), "r"(kAtReconThreads));
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->kv_empty[st])));
+    for (int i = 0; i < 2; ++i) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->s_done[i])));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->o_done[i])));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&bars->kv_full[i])), "r"(kAtReconThreads));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 2;" ::"r"(smem_addr(&bars->kv_empty[i])));   // one commit per query tile
     }
     bars->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -409,7 +447,7 @@ qvg_attention_fused(const AttnParams p) {
   // S of query tile t at column 128 t, O of query tile t at column 256 + 128 t
   const uint32_t tS = tmem, tO = tmem + 256;
   const int ntiles = (int)((p.Nk + kAtTile - 1) / kAtTile);
-  int s_issued = 0, o_issued = 0;                   // products committed (thread 0)
+  int s_issued = 0, o_issued = 0;                   // products committed (the issuing threads 0 and 128)
 
   if (warp >= 8) {
     // ---------------------------------------------------------------- reconstruction warps
@@ -468,119 +506,113 @@ qvg_attention_fused(const AttnParams p) {
       if (*abort_flag) break;
     }
   } else {
-    // ---------------------------------------------------------------- softmax warps (thread 0 issues the products)
-    // warps 0-3 hold query tile 0, warps 4-7 tile 1: row 32*(warp mod 4) + lane,
-    // the warp's tensor-memory lane quarter
-    const int sm_tile = warp >> 2;
+    // ---------------------------------------------------------------- softmax warps, two independent groups
+    // Group g (warps 4g .. 4g+3) owns query tile g: row 32*(warp mod 4) + lane,
+    // the warp's tensor-memory lane quarter.  Its first thread issues the
+    // group's products: S_g = Q_g'K'^T when a stage is full, then, after the
+    // group's softmax has written P_g over the first 64 columns of S_g (bf16,
+    // two per column), O_g += P_g V with A read from tensor memory.  The two
+    // groups run independently, so one group's softmax overlaps the other's
+    // products.
+    const int g = warp >> 2;
+    const bool issuer = threadIdx.x == 128 * g;
     const int qi = 32 * (warp & 3) + lane;
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    const uint32_t tSt = tS + 128 * sm_tile, tOt = tO + 128 * sm_tile;
+    const uint32_t tSt = tS + 128 * g, tOt = tO + 128 * g;
     float m_run = -3.0e38f, l_run = 0.0f;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int st = j & 1;
       const int64_t k0 = (int64_t)j * kAtTile;
-      uint8_t* sK = stage_k(st);
-      // 1. S_t = Q_t' K'^T for both query tiles, once the stage is reconstructed
-      if (threadIdx.x == 0) {
-        if (bar_wait_or_abort(&bars->kv_full[st], (uint32_t)((j >> 1) & 1), abort_flag)) {
+      // 1. S_g once the stage is reconstructed and the previous O_g (which
+      // read P_g from these columns) has completed
+      if (issuer) {
+        bool w = bar_wait_or_abort(&bars->kv_full[st], (uint32_t)((j >> 1) & 1), abort_flag);
+        if (w && j > 0) w = bar_wait_or_abort(&bars->o_done[g], (uint32_t)((j - 1) & 1), abort_flag);
+        if (w) {
           fence_after();
-          const uint32_t b0 = smem_addr(sK);
+          const uint32_t a0 = smem_addr(sQ + g * kAtOpBytes), b0 = smem_addr(stage_k(st));
 #pragma unroll
-          for (int qt = 0; qt < kAtQTiles; ++qt) {
-            const uint32_t a0 = smem_addr(sQ + qt * kAtOpBytes);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma(tS + 128 * qt, op_desc_k(a0, kk), op_desc_k(b0, kk), kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars->s_done);
+          for (int kk = 0; kk < 8; ++kk) mma(tSt, op_desc_k(a0, kk), op_desc_k(b0, kk), kk > 0 ? 1u : 0u);
+          mma_commit(&bars->s_done[g]);
           ++s_issued;
         } else {
           *abort_flag = 1;
         }
       }
-      // 2. the scores, and the previous tile's products (O rescale, P_1 buffer)
-      bool w_ok = bar_wait_or_abort(&bars->s_done, (uint32_t)(j & 1), abort_flag);
-      if (w_ok && j > 0) w_ok = bar_wait_or_abort(&bars->o_done, (uint32_t)((j - 1) & 1), abort_flag);
-      if (named_bar_or(1, kAtSoftmaxThreads, !w_ok)) { ok = false; break; }
+      // 2. the scores (the previous O_g is complete too: the issuer waited for it)
+      bool w_ok = bar_wait_or_abort(&bars->s_done[g], (uint32_t)(j & 1), abort_flag);
+      if (named_bar_or(1 + g, 128, !w_ok)) { ok = false; break; }
       fence_after();
-      // 3. online softmax of the thread's query row
+      // 3. online softmax of the thread's query row; P_g into tensor memory
       {
-        uint8_t* sP = sm_tile == 0 ? sK : sP1;
         const int valid = (int)(p.Nk - k0 < kAtTile ? p.Nk - k0 : kAtTile);
-        float mt = -3.0e38f;                          // pass 1: the row maximum, 32 columns at a time
+        float mt = -3.0e38f;                          // pass 1: the row maximum, 16 columns at a time
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t rg[32];
-          tld32(tSt + lane_base + (uint32_t)(32 * c), rg);
+        for (int c = 0; c < 8; ++c) {
+          uint32_t rg[16];
+          tld16(tSt + lane_base + (uint32_t)(16 * c), rg);
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (32 * c + e < valid) mt = fmaxf(mt, __uint_as_float(rg[e]) * p.sl);
+          for (int e = 0; e < 16; ++e)
+            if (16 * c + e < valid) mt = fmaxf(mt, __uint_as_float(rg[e]) * p.sl);
         }
         const float m_new = fmaxf(m_run, mt);
         const float alpha = exp2_approx(m_run - m_new);
-        float sum = 0.0f;                             // pass 2: bf16 weights into P, and their sum
+        float sum = 0.0f;                             // pass 2: bf16 weights, and their sum
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t rg[32];
-          tld32(tSt + lane_base + (uint32_t)(32 * c), rg);
+        for (int c = 0; c < 8; ++c) {
+          uint32_t rg[16];
+          tld16(tSt + lane_base + (uint32_t)(16 * c), rg);
+          uint32_t w[8];
 #pragma unroll
-          for (int kg = 0; kg < 4; ++kg) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int j0 = 32 * c + 8 * kg + 2 * e;
-              const float pa = j0 < valid ? exp2_approx(__uint_as_float(rg[8 * kg + 2 * e]) * p.sl - m_new) : 0.0f;
-              const float pb = j0 + 1 < valid ? exp2_approx(__uint_as_float(rg[8 * kg + 2 * e + 1]) * p.sl - m_new) : 0.0f;
-              w[e] = pack_bf16(pa, pb);
-              // the sum takes the rounded weights, the ones the product uses
-              sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
-            }
-            *reinterpret_cast<uint4*>(sP + op_off(qi, 32 * c + 8 * kg)) = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int e = 0; e < 8; ++e) {
+            const int j0 = 16 * c + 2 * e;
+            const float pa = j0 < valid ? exp2_approx(__uint_as_float(rg[2 * e]) * p.sl - m_new) : 0.0f;
+            const float pb = j0 + 1 < valid ? exp2_approx(__uint_as_float(rg[2 * e + 1]) * p.sl - m_new) : 0.0f;
+            w[e] = pack_bf16(pa, pb);
+            // the sum takes the rounded weights, the ones the product uses
+            sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
           }
+          // keys 16c .. 16c+15 -> columns 8c .. 8c+7, already read
+          tst8(tSt + lane_base + (uint32_t)(8 * c), w);
         }
         l_run = l_run * alpha + sum;
         m_run = m_new;
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {   // rescale O
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {   // rescale O_g
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t rg[16];
+            tld16(tOt + lane_base + (uint32_t)(16 * c), rg);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t rg[32];
-            tld32(tOt + lane_base + (uint32_t)(32 * c), rg);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) rg[e] = __float_as_uint(__uint_as_float(rg[e]) * alpha);
-            tst32(tOt + lane_base + (uint32_t)(32 * c), rg);
+            for (int e = 0; e < 16; ++e) rg[e] = __float_as_uint(__uint_as_float(rg[e]) * alpha);
+            tst16(tOt + lane_base + (uint32_t)(16 * c), rg);
           }
-          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       fence_before();
-      named_bar_or(1, kAtSoftmaxThreads, false);       // P of both tiles written, O rescaled
-      // 4. O_t += P_t V for both query tiles; the stage is free once they complete
-      if (threadIdx.x == 0) {
+      named_bar_or(1 + g, 128, false);                 // P_g written, O_g rescaled
+      // 4. O_g += P_g V; the stage is free once both query tiles' products complete
+      if (issuer) {
         fence_after();
         const uint32_t b0 = smem_addr(stage_v(st));
 #pragma unroll
-        for (int qt = 0; qt < kAtQTiles; ++qt) {
-          const uint32_t a0 = smem_addr(qt == 0 ? sK : sP1);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma(tO + 128 * qt, op_desc_k(a0, kk), op_desc_k(b0, kk), (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&bars->o_done);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ta(tOt, tSt + (uint32_t)(8 * kk), op_desc_k(b0, kk), (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars->o_done[g]);
         mma_commit(&bars->kv_empty[st]);
         ++o_issued;
       }
     }
-    // the last products, then O / l
+    // the last product, then O / l
     if (ok && ntiles > 0) {
-      const bool w_ok = bar_wait_or_abort(&bars->o_done, (uint32_t)((ntiles - 1) & 1), abort_flag);
-      ok = !named_bar_or(1, kAtSoftmaxThreads, !w_ok);
+      const bool w_ok = bar_wait_or_abort(&bars->o_done[g], (uint32_t)((ntiles - 1) & 1), abort_flag);
+      ok = !named_bar_or(1 + g, 128, !w_ok);
       fence_after();
     }
     if (!ok) *abort_flag = 1;
     if (ok && ntiles > 0) {
-      const int64_t q = q0 + sm_tile * kAtTile + qi;
+      const int64_t q = q0 + g * kAtTile + qi;
       const float inv = 1.0f / l_run;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -598,12 +630,13 @@ qvg_attention_fused(const AttnParams p) {
   }
   fence_before();
   __syncthreads();
-  if (*abort_flag && threadIdx.x == 0) {
-    atomicOr(p.status, 1u);
-    // let the products already issued finish (bounded) before the tensor
+  if (*abort_flag && (threadIdx.x == 0 || threadIdx.x == 128)) {
+    const int g = threadIdx.x >> 7;
+    if (g == 0) atomicOr(p.status, 1u);
+    // let the products this thread issued finish (bounded) before the tensor
     // memory is freed; a phase that already completed returns at once
-    if (s_issued > 0) bar_wait(&bars->s_done, (uint32_t)((s_issued - 1) & 1));
-    if (o_issued > 0) bar_wait(&bars->o_done, (uint32_t)((o_issued - 1) & 1));
+    if (s_issued > 0) bar_wait(&bars->s_done[g], (uint32_t)((s_issued - 1) & 1));
+    if (o_issued > 0) bar_wait(&bars->o_done[g], (uint32_t)((o_issued - 1) & 1));
   }
   __syncthreads();
   if (warp == 0) {
@@ -631,7 +664,7 @@ __global__ void qvg_rope_tables_kernel(float2* hi, float2* lo, int n_hi, double 
 }  // namespace
 
 size_t attention_smem_bytes() {
-  return 1024 + (size_t)(kAtQTiles + 5) * kAtOpBytes + 32 * sizeof(float2) + sizeof(AtBars);
+  return 1024 + (size_t)(kAtQTiles + 4) * kAtOpBytes + 32 * sizeof(float2) + sizeof(AtBars);
 }
 
 cudaError_t launch_rope_tables(void* tables, int n_hi, double base, cudaStream_t s) {
