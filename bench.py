@@ -332,6 +332,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=4750)
     ap.add_argument("--cpu-units", type=int, default=8, help="full-size blocks of the oracle baseline")
     ap.add_argument("--frames", type=int, default=None, help="override the frame count")
+    ap.add_argument("--attention-split", type=int, default=0,
+                    help="CTAs per cluster over the cache in qvg_attention (0 = the library's choice)")
     ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
                     help="weak: every rank its own cache; strong: the ranks share one cache by heads")
     args = ap.parse_args()
@@ -755,6 +757,8 @@ def run_attention(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
     qpos = torch.arange(Nk, Nk + Nq, device=dev, dtype=torch.int64)
     kpos = torch.arange(Nk, device=dev, dtype=torch.int64)
     tables = qvg.rope_tables(Nk + Nq, device=dev)
+    qvg.attention_set_split(args.attention_split)
+    split = qvg.attention_split(cfg, Nk, H, Nq)
     O = torch.empty((H, Nq, 128), dtype=torch.float32, device=dev)
     Kd = torch.empty((H, Nk, 128), dtype=torch.bfloat16, device=dev)
     Vd = torch.empty_like(Kd)
@@ -809,6 +813,7 @@ def run_attention(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
         "warmup": args.warmup, "ms_per_step": ms_f, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl["desc"], "heads": H, "cached_tokens": Nk, "queries": Nq,
+                   "cluster_split": split,
                    "l2": "packed caches fit in L2; the baseline's bf16 caches do not"},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
                      "frac": tflops / peaks["bf16_sus"], "traffic": None, "kernel": "qvg_attention_fused",

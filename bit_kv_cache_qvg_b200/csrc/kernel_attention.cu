@@ -14,30 +14,37 @@
 // p * base^(-2i/d)), the cached tokens sit at positions 0 .. Nk-1 and the
 // queries at the given positions.  No mask.
 //
-// One CTA = one head x 128 queries; it walks the cache in tiles of 128
-// tokens.  Per tile:
-//   1. all 8 warps dequantise the K and V tile (unpack, scale, add every
-//      stage's centroid in reverse order, round to bf16 -- the arithmetic of
-//      qvg_dequant_fused), apply the rotary embedding to K, and store both
-//      straight into shared memory in the tensor core's K-major operand
-//      layout (128-byte swizzle): K rows (keys) with the channels contiguous,
-//      V transposed (channels) with the keys contiguous, each thread an
-//      8 x 8 block;
-//   2. one thread issues S = Q' K'^T (tcgen05.mma kind::f16, M = N = K = 128,
-//      fp32 accumulators in tensor memory);
-//   3. warps 0-3 (one per tensor-memory lane quarter, a thread per query)
-//      read S, keep the running row maximum and sum (online softmax, base-2
-//      exponentials), write P in bf16 into the K buffer (the A operand of the
-//      next product) and rescale the O accumulator in tensor memory;
-//   4. one thread issues O += P V (accumulators in tensor memory).
-// After the last tile O / l is written in fp32.  The rotary angles come from
-// two tables of (cos, sin) in fp32, p = 1024 a + b: (1024 a) theta_i and
-// b theta_i, combined by the angle-sum identity (qvg_rope_tables builds them
-// in fp64).  Every mbarrier wait is bounded; on expiry the kernel records
-// QVG_ERR_DEVICE_TIMEOUT in the status word at the start of the tables
-// buffer and stops.  No TMA and no multicast: the operands are written by the
-// threads that reconstruct them.
+// One CTA = one head x 256 queries (two query tiles of 128) x a range of the
+// cache's tiles of 128 tokens; 24 warps in three roles:
+//   * warps 8-23 dequantise each K and V tile (unpack, scale, add every
+//     stage's centroid in reverse order, round to bf16 -- the arithmetic of
+//     qvg_dequant_fused), apply the rotary embedding to K, and store both
+//     into a two-stage ring in shared memory in the tensor core's K-major
+//     operand layout (128-byte swizzle): K rows (keys) with the channels
+//     contiguous, V transposed (channels) with the keys contiguous;
+//   * the first thread of each query tile's group issues S = Q' K'^T
+//     (tcgen05.mma kind::f16, M = N = K = 128, fp32 accumulators in tensor
+//     memory) when a stage is full, and O += P V (P read from tensor memory)
+//     when the group's softmax is done;
+//   * warps 0-3 and 4-7 (one per tensor-memory lane quarter, a thread per
+//     query) run the online softmax of the two query tiles (running row
+//     maximum and sum, base-2 exponentials), write P in bf16 over their S
+//     columns and rescale O in tensor memory.
+// The two query tiles' groups run independently, so one group's softmax
+// overlaps the other's products.  When the cache is split over a cluster of
+// S CTAs (one key range each, so that the grid fills the SMs), each CTA
+// leaves its unnormalised O with its row maximum and sum in shared memory and
+// the cluster merges them through distributed shared memory (the usual
+// rescaling of partial softmax sums); otherwise O / l is written directly.
+// The rotary angles come from two tables of (cos, sin) in fp32, p = 1024 a + b:
+// (1024 a) theta_i and b theta_i, combined by the angle-sum identity
+// (qvg_rope_tables builds them in fp64).  Every mbarrier wait is bounded; on
+// expiry the kernel records QVG_ERR_DEVICE_TIMEOUT in the status word at the
+// start of the tables buffer and stops.  No TMA and no multicast: the
+// operands are written by the threads that reconstruct them.
 #include <cuda.h>
+
+#include <atomic>
 
 #include "qvg_common.cuh"
 #include "qvg_launch.h"
@@ -53,6 +60,8 @@ constexpr int kAtTile = 128;                    // queries per CTA, cached token
 constexpr int kAtOpBytes = kAtTile * kD * 2;    // one 128 x 128 bf16 operand: 32 KB
 constexpr uint64_t kAtWaitNs = 2000000000ull;   // 2 s per bounded wait
 constexpr int kRopeLo = 1024;                   // positions per low-table row block
+constexpr int kAtMaxSplit = 8;                  // CTAs per cluster, at most (the portable cluster size)
+constexpr int kMaxDevices = 64;
 
 struct AttnParams {
   const uint8_t* codes[2];        // K, V: [H][Nk][d/4]
@@ -69,6 +78,7 @@ struct AttnParams {
   int64_t max_pos;                // largest position the tables cover
   int64_t Nk, Nq;
   int H, K, T, G, sym;
+  int split;                      // CTAs per cluster, each over one range of the cache's tiles
   float sl;                       // log2(e) / sqrt(d)
 };
 
@@ -273,6 +283,30 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
+// Distributed shared memory of the CTA's cluster: the address of the same
+// shared-memory location in CTA `rank`, loads from it, and the cluster-wide
+// barrier (every thread of every CTA arrives; release/acquire order the
+// shared-memory writes before it with the reads after it).
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ float2 ld_cluster_f2(uint32_t a) {
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&b);
@@ -393,7 +427,10 @@ qvg_attention_fused(const AttnParams p) {
   auto stage_v = [&](int st) { return sK0 + (2 * st + 1) * kAtOpBytes; };
 
   const int h = blockIdx.y;
-  const int64_t q0 = (int64_t)blockIdx.x * (kAtQTiles * kAtTile);
+  // the cluster's CTAs share the query block; CTA `rank` takes tiles
+  // j_begin .. j_begin + n_loc - 1 of the cache (at least one each)
+  const int rank = (int)(blockIdx.x % (unsigned)p.split);
+  const int64_t q0 = (int64_t)(blockIdx.x / (unsigned)p.split) * (kAtQTiles * kAtTile);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -446,8 +483,11 @@ qvg_attention_fused(const AttnParams p) {
   const uint32_t tmem = bars->tmem_base;
   // S of query tile t at column 128 t, O of query tile t at column 256 + 128 t
   const uint32_t tS = tmem, tO = tmem + 256;
-  const int ntiles = (int)((p.Nk + kAtTile - 1) / kAtTile);
+  const int64_t ntot = (p.Nk + kAtTile - 1) / kAtTile;
+  const int j_begin = (int)(ntot * rank / p.split);
+  const int ntiles = (int)(ntot * (rank + 1) / p.split) - j_begin;   // this CTA's tiles
   int s_issued = 0, o_issued = 0;                   // products committed (the issuing threads 0 and 128)
+  float m_fin = 0.0f, l_fin = 0.0f;                 // the softmax thread's row maximum and sum at the end
 
   if (warp >= 8) {
     // ---------------------------------------------------------------- reconstruction warps
@@ -465,7 +505,7 @@ qvg_attention_fused(const AttnParams p) {
       fence_after();
       uint8_t* sK = stage_k(st);
       uint8_t* sV = stage_v(st);
-      const int64_t k0 = (int64_t)j * kAtTile;
+      const int64_t k0 = (int64_t)(j_begin + j) * kAtTile;
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         float vk[2][8];
@@ -523,7 +563,7 @@ qvg_attention_fused(const AttnParams p) {
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int st = j & 1;
-      const int64_t k0 = (int64_t)j * kAtTile;
+      const int64_t k0 = (int64_t)(j_begin + j) * kAtTile;
       // 1. S_g once the stage is reconstructed and the previous O_g (which
       // read P_g from these columns) has completed
       if (issuer) {
@@ -611,7 +651,9 @@ qvg_attention_fused(const AttnParams p) {
       fence_after();
     }
     if (!ok) *abort_flag = 1;
-    if (ok && ntiles > 0) {
+    m_fin = m_run;
+    l_fin = l_run;
+    if (ok && ntiles > 0 && p.split == 1) {
       const int64_t q = q0 + g * kAtTile + qi;
       const float inv = 1.0f / l_run;
 #pragma unroll
@@ -639,6 +681,64 @@ qvg_attention_fused(const AttnParams p) {
     if (o_issued > 0) bar_wait(&bars->o_done[g], (uint32_t)((o_issued - 1) & 1));
   }
   __syncthreads();
+  if (p.split > 1) {
+    // The products are complete and the query and ring buffers free: leave
+    // this CTA's unnormalised O rows there (row R = query q0 + R, channel
+    // chunk c of 4 at chunk c ^ (R mod 8), so that a warp's stores hit
+    // distinct banks) with the rows' maximum and sum after them.
+    float* sX = reinterpret_cast<float*>(smem);
+    float2* sML = reinterpret_cast<float2*>(smem + kAtQTiles * kAtTile * kD * sizeof(float));
+    if (warp < 8) {
+      const int R = threadIdx.x;
+      const uint32_t tOt = tO + 128 * (warp >> 2), lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t rg[32];
+        tld32(tOt + lane_base + (uint32_t)(32 * c), rg);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          *reinterpret_cast<float4*>(sX + R * kD + 4 * ((8 * c + e) ^ (R & 7))) =
+              make_float4(__uint_as_float(rg[4 * e]), __uint_as_float(rg[4 * e + 1]),
+                          __uint_as_float(rg[4 * e + 2]), __uint_as_float(rg[4 * e + 3]));
+      }
+      sML[R] = make_float2(m_fin, l_fin);
+    }
+    fence_before();
+    cluster_sync();
+    // CTA `rank` merges rows [R0, R1) of the block from every CTA of the
+    // cluster: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s
+    // (a CTA with no tiles has l = 0 and takes no part); a warp per row, a
+    // lane per chunk of four channels.
+    const int R0 = kAtQTiles * kAtTile * rank / p.split, R1 = kAtQTiles * kAtTile * (rank + 1) / p.split;
+    for (int t = threadIdx.x; t < (R1 - R0) * 32; t += kAtThreads) {
+      const int R = R0 + (t >> 5), c = t & 31;
+      const uint32_t ml_a = smem_addr(sML + R), x_a = smem_addr(sX + R * kD + 4 * (c ^ (R & 7)));
+      float M = -3.0e38f;
+      for (int r = 0; r < p.split; ++r) {
+        const float2 ml = ld_cluster_f2(cluster_addr(ml_a, (uint32_t)r));
+        if (ml.y > 0.0f) M = fmaxf(M, ml.x);
+      }
+      float L = 0.0f;
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (int r = 0; r < p.split; ++r) {
+        const float2 ml = ld_cluster_f2(cluster_addr(ml_a, (uint32_t)r));
+        const float w = ml.y > 0.0f ? exp2_approx(ml.x - M) : 0.0f;
+        if (w > 0.0f) {
+          const float4 x = ld_cluster_f4(cluster_addr(x_a, (uint32_t)r));
+          acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
+          L += w * ml.y;
+        }
+      }
+      const int64_t q = q0 + R;
+      if (q < p.Nq && !*abort_flag) {
+        const float inv = 1.0f / L;
+        *reinterpret_cast<float4*>(p.O + ((int64_t)h * p.Nq + q) * kD + 4 * c) =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      }
+    }
+    // no CTA leaves while another still reads its shared memory
+    cluster_sync();
+  }
   if (warp == 0) {
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
@@ -680,8 +780,103 @@ template <int TT>
 static cudaError_t launch_attention_t(const AttnParams& p, dim3 grid, size_t smem, cudaStream_t s) {
   cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(qvg_attention_fused<TT>), smem);
   if (e != cudaSuccess) return e;
-  qvg_attention_fused<TT><<<grid, kAtThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  if (p.split == 1) {
+    qvg_attention_fused<TT><<<grid, kAtThreads, smem, s>>>(p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kAtThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)p.split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, qvg_attention_fused<TT>, p);
+}
+
+// Clusters of `split` attention CTAs that fit on the device at once (CTAs
+// per SM times SMs for split = 1); 0 if none fits.  Cached per device,
+// kernel instance and split.
+template <int TT>
+static int resident_clusters(int split) {
+  static std::atomic<int> cache[kMaxDevices][kAtMaxSplit + 1];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  const int known = cache[dev][split].load(std::memory_order_relaxed);
+  if (known > 0) return known - 1;
+  const size_t smem = attention_smem_bytes();
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(qvg_attention_fused<TT>), smem) != cudaSuccess) return 0;
+  int n = 0;
+  if (split == 1) {
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qvg_attention_fused<TT>, kAtThreads, smem) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 0;
+    n = per_sm * sms;
+  } else {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)split, 1, 1);
+    cfg.blockDim = dim3(kAtThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, qvg_attention_fused<TT>, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+  }
+  cache[dev][split].store(n + 1, std::memory_order_relaxed);
+  return n;
+}
+
+// The split of the cache over a cluster: the one with the least estimated
+// time, (waves of resident clusters) x (tiles per CTA + the fixed cost of a
+// CTA, about two tiles), over 1 .. 4 CTAs per cluster; a positive `forced`
+// is taken as it is.  Never more CTAs than the cache has tiles.
+template <int TT>
+static int choose_split(int64_t Nk, int64_t Nq, int H, int forced) {
+  const int64_t ntot = (Nk + kAtTile - 1) / kAtTile;
+  const int smax = (int)(ntot < kAtMaxSplit ? ntot : kAtMaxSplit);
+  if (forced > 0) return forced < smax ? forced : smax;
+  const int64_t units = (Nq + kAtQTiles * kAtTile - 1) / (kAtQTiles * kAtTile) * H;
+  int best = 1;
+  double best_cost = 0.0;
+  for (int sp = 1; sp <= (smax < 4 ? smax : 4); ++sp) {
+    const int n = resident_clusters<TT>(sp);
+    if (n <= 0) continue;
+    const double waves = (double)((units + n - 1) / n);
+    const double cost = waves * (double)((ntot + sp - 1) / sp + 2);
+    if (sp == 1 || cost < best_cost) { best = sp; best_cost = cost; }
+  }
+  return best;
+}
+
+template <int TT>
+static cudaError_t launch_attention_split(AttnParams& p, int64_t Nq, size_t smem, int forced, cudaStream_t s) {
+  p.split = choose_split<TT>(p.Nk, Nq, p.H, forced);
+  const dim3 grid((unsigned)(p.split * ((Nq + kAtQTiles * kAtTile - 1) / (kAtQTiles * kAtTile))), (unsigned)p.H);
+  return launch_attention_t<TT>(p, grid, smem, s);
+}
+
+int attention_split(int T, int64_t Nk, int64_t Nq, int H, int forced) {
+  switch (T) {
+    case 0: return choose_split<0>(Nk, Nq, H, forced);
+    case 1: return choose_split<1>(Nk, Nq, H, forced);
+    case 2: return choose_split<2>(Nk, Nq, H, forced);
+    case 3: return choose_split<3>(Nk, Nq, H, forced);
+    case 4: return choose_split<4>(Nk, Nq, H, forced);
+    default: return choose_split<-1>(Nk, Nq, H, forced);
+  }
 }
 
 cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s) {
@@ -701,14 +896,13 @@ cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s) {
   p.Nk = a.Nk; p.Nq = a.Nq; p.H = a.H; p.K = a.K; p.T = a.T; p.G = a.G; p.sym = a.sym;
   p.sl = 1.4426950408889634f / sqrtf((float)kD);
   const size_t smem = attention_smem_bytes();
-  const dim3 grid((unsigned)((a.Nq + kAtQTiles * kAtTile - 1) / (kAtQTiles * kAtTile)), (unsigned)a.H);
   switch (a.T) {
-    case 0: return launch_attention_t<0>(p, grid, smem, s);
-    case 1: return launch_attention_t<1>(p, grid, smem, s);
-    case 2: return launch_attention_t<2>(p, grid, smem, s);
-    case 3: return launch_attention_t<3>(p, grid, smem, s);
-    case 4: return launch_attention_t<4>(p, grid, smem, s);
-    default: return launch_attention_t<-1>(p, grid, smem, s);
+    case 0: return launch_attention_split<0>(p, a.Nq, smem, a.split, s);
+    case 1: return launch_attention_split<1>(p, a.Nq, smem, a.split, s);
+    case 2: return launch_attention_split<2>(p, a.Nq, smem, a.split, s);
+    case 3: return launch_attention_split<3>(p, a.Nq, smem, a.split, s);
+    case 4: return launch_attention_split<4>(p, a.Nq, smem, a.split, s);
+    default: return launch_attention_split<-1>(p, a.Nq, smem, a.split, s);
   }
 }
 

@@ -50,13 +50,18 @@ bool fault_injected(const char* what) {
 
 cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
+  // the attribute is per device: remember (kernel, device) pairs
+  struct Done { const void* kernel; int dev; size_t bytes; };
   static std::mutex mu;
-  static std::vector<std::pair<const void*, size_t>> done;
+  static std::vector<Done> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> g(mu);
   for (auto& d : done)
-    if (d.first == kernel && d.second >= bytes) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess) done.emplace_back(kernel, bytes);
+    if (d.kernel == kernel && d.dev == dev && d.bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done.push_back(Done{kernel, dev, bytes});
   return e;
 }
 
@@ -546,6 +551,21 @@ qvg_status qvg_rope_tables(double base, int32_t d, int64_t max_pos, void* tables
   return cuda_status(plaunch(K_ROPE, s, [&] { return launch_rope_tables(tables, n_hi, base, s); }));
 }
 
+// The split of qvg_attention_set_split (0 = the library's choice).
+static std::atomic<int> g_attention_split{0};
+
+int32_t qvg_attention_set_split(int32_t split) {
+  if (split < 0 || split > 8) return -1;
+  return g_attention_split.exchange(split);
+}
+
+int32_t qvg_attention_split(const qvg_config* cfg, int64_t Nk, int32_t H, int64_t Nq) {
+  if (check_config(cfg, Nk, H, kD, QVG_BF16) != QVG_OK || Nk < 1 || Nq < 1) return -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { (void)cudaGetLastError(); return -1; }
+  return attention_split(cfg->T, Nk, Nq, H, g_attention_split.load(std::memory_order_relaxed));
+}
+
 qvg_status qvg_attention(const qvg_config* cfg, const qvg_packed* k, const qvg_packed* v, int64_t Nk, int32_t H,
                          int32_t d, const void* Q, const int64_t* q_pos, int64_t Nq, const void* tables,
                          size_t tables_bytes, float* O, qvg_stream_t stream_) {
@@ -572,6 +592,7 @@ qvg_status qvg_attention(const qvg_config* cfg, const qvg_packed* k, const qvg_p
   AttentionArgs a{};
   a.k = k; a.v = v; a.Q = Q; a.qpos = q_pos; a.tables = tables; a.n_hi = (int)n_hi; a.O = O;
   a.Nk = Nk; a.Nq = Nq; a.H = H; a.K = cfg->K; a.T = cfg->T; a.G = cfg->group_size; a.sym = sym ? 1 : 0;
+  a.split = g_attention_split.load(std::memory_order_relaxed);
   st = cuda_status(plaunch(K_ATTN, s, [&] { return launch_attention(a, s); }));
   if (st == QVG_OK && fault_injected("stream")) st = QVG_ERR_CUDA;
   return st;

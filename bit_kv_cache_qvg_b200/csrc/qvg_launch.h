@@ -166,8 +166,12 @@ struct AttentionArgs {
   float* O;                    // [H][Nq][d] fp32
   int64_t Nk, Nq;
   int H, K, T, G, sym;
+  int split;                   // CTAs per cluster over the cache of a query block; 0 = chosen here
 };
 cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s);
+// The split launch_attention uses for these sizes (forced > 0: that one,
+// capped at the cache's tile count and the cluster limit).
+int attention_split(int T, int64_t Nk, int64_t Nq, int H, int forced);
 size_t attention_smem_bytes();
 
 }  // namespace qvg

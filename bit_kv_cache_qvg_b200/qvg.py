@@ -109,6 +109,8 @@ _SIGS = {
     "qvg_attention": (C.c_int, [C.POINTER(Config), C.POINTER(_Packed), C.POINTER(_Packed), C.c_int64, C.c_int32,
                                 C.c_int32, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_size_t, C.c_void_p,
                                 C.c_void_p]),
+    "qvg_attention_set_split": (C.c_int32, [C.c_int32]),
+    "qvg_attention_split": (C.c_int32, [C.POINTER(Config), C.c_int64, C.c_int32, C.c_int64]),
     "qvg_profile_enable": (None, [C.c_int]),
     "qvg_profile_reset": (None, []),
     "qvg_profile_launches": (C.c_int64, []),
@@ -298,6 +300,24 @@ def attention(kp: Packed, vp: Packed, Q: torch.Tensor, q_pos: torch.Tensor, tabl
                                _ptr(q_pos), Nq, _ptr(tables), tables.numel(), _ptr(O), _stream(stream)),
            "qvg_attention")
     return O
+
+
+def attention_set_split(split: int) -> int:
+    """qvg_attention_set_split: fix the cluster split of qvg_attention for the
+    process (1 .. 8; 0 = the library's choice); returns the previous setting."""
+    prev = int(lib().qvg_attention_set_split(int(split)))
+    if prev < 0:
+        raise QvgError(1, "qvg_attention_set_split")
+    return prev
+
+
+def attention_split(cfg: Config, Nk: int, H: int, Nq: int) -> int:
+    """qvg_attention_split: the split a qvg_attention call with these sizes
+    would use on the current device."""
+    n = int(lib().qvg_attention_split(C.byref(cfg), Nk, H, Nq))
+    if n < 0:
+        raise QvgError(1, "qvg_attention_split")
+    return n
 
 
 def profile_enable(on: bool = True):

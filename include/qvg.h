@@ -301,6 +301,22 @@ QVG_API qvg_status qvg_attention(const qvg_config* cfg, const qvg_packed* k, con
                          int32_t H, int32_t d, const void* Q, const int64_t* q_pos, int64_t Nq,
                          const void* tables, size_t tables_bytes, float* O, qvg_stream_t stream);
 
+/* qvg_attention splits the cache of each head and block of 256 queries over
+ * a thread-block cluster of `split` CTAs, each over one range of the cache's
+ * tiles of 128 tokens; the cluster merges their partial softmax sums through
+ * distributed shared memory.  Each CTA rounds its softmax weights to bf16
+ * against its own running maximum, so splits differ by such roundings (the
+ * error bound of qvg_attention holds for every split).
+ * By default (0) the library picks it from the device's cluster occupancy so
+ * that the grid fills the SMs.  qvg_attention_set_split fixes it for the
+ * process (1 .. 8, capped at the cache's tile count; 0 = automatic again) and
+ * returns the previous setting, or -1 (nothing changed) for other values.
+ * qvg_attention_split returns the split a qvg_attention call with these
+ * sizes would use on the current device, or -1 for invalid arguments or no
+ * device.  Host-only; neither launches work. */
+QVG_API int32_t qvg_attention_set_split(int32_t split);
+QVG_API int32_t qvg_attention_split(const qvg_config* cfg, int64_t Nk, int32_t H, int64_t Nq);
+
 /* ------------------------------------------------------------------ */
 /* Diagnostics (no counterpart in the method; used by the benchmark).    */
 /* ------------------------------------------------------------------ */

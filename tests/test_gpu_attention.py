@@ -82,6 +82,66 @@ def test_attention_matches_oracle(q, ora, H, Nk, Nq, T, G, K, mode, q_scale):
     assert typical < 0.25          # the usual error is well inside the worst-case bound
 
 
+@pytest.mark.parametrize("split", [2, 3, 4, 8])
+def test_attention_split_over_a_cluster_matches_oracle(q, ora, split):
+    """The cache of each query block split over a cluster of `split` CTAs
+    (ragged ranges: 8 tiles over 3 CTAs; 8 CTAs of one tile each) stays
+    within the bound."""
+    cfg = q.config(K=64, T=2, group_size=64, iters=3, scale_mode=0)
+    prev = q.attention_set_split(split)
+    try:
+        assert q.attention_split(cfg, 1000, 2, 300) == min(split, 8)
+        typical = _run_case(q, ora, cfg, 2, 1000, 300, 0.05, seed=1002)
+    finally:
+        q.attention_set_split(prev)
+    assert typical < 0.25
+
+
+def test_attention_splits_agree(q):
+    """Each CTA of a split rounds its weights to bf16 against its own running
+    maximum (as the unsplit kernel does against the maximum so far), so the
+    splits differ by weight roundings of 2^-9 relative, far inside the
+    bound, and never by more than 2^-7 of the largest output."""
+    from bit_kv_cache_qvg_b200 import synth
+    cfg = q.config(K=32, T=1, group_size=64, iters=2)
+    H, Nk, Nq = 2, 3000, 520
+    X = synth.block_batch(H, synth.KVShape(2, 30, 52), seed=9, kinds=[0, 1])[:, :Nk].contiguous().cuda()
+    kp = q.quantize(X, cfg)
+    Q = (torch.randn((H, Nq, 128), generator=torch.Generator().manual_seed(4)) * 0.1).to(torch.bfloat16).cuda()
+    pos = torch.arange(Nk, Nk + Nq, dtype=torch.int64, device="cuda")
+    tables = q.rope_tables(Nk + Nq)
+    outs = {}
+    for split in (1, 2, 3, 5, 8):
+        prev = q.attention_set_split(split)
+        try:
+            outs[split] = q.attention(kp, kp, Q, pos, tables).cpu()
+        finally:
+            q.attention_set_split(prev)
+    torch.cuda.synchronize()
+    assert q.workspace_status(tables) == 0
+    scale = outs[1].abs().max().item()
+    for split, O in outs.items():
+        assert torch.isfinite(O).all()
+        assert (O - outs[1]).abs().max().item() <= 2.0 ** -7 * scale, split
+
+
+def test_attention_split_setting_is_checked(q):
+    cfg = q.config(K=256, T=2, group_size=64)
+    with pytest.raises(q.QvgError):
+        q.attention_set_split(9)
+    with pytest.raises(q.QvgError):
+        q.attention_set_split(-1)
+    auto = q.attention_split(cfg, 38000, 32, 1520)
+    assert 1 <= auto <= 4
+    assert q.attention_split(cfg, 100, 32, 1520) == 1      # one tile: nothing to split
+    prev = q.attention_set_split(3)
+    try:
+        assert q.attention_split(cfg, 38000, 32, 1520) == 3
+        assert q.attention_split(cfg, 200, 32, 1520) == 2   # capped at the two tiles
+    finally:
+        assert q.attention_set_split(prev) == 3
+
+
 def test_attention_reports_a_stale_timeout_and_rejects_uncovered_positions(q):
     from bit_kv_cache_qvg_b200 import synth
     cfg = q.config(K=16, T=1, group_size=64, iters=2)
