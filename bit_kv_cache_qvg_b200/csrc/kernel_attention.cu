@@ -45,6 +45,7 @@
 #include <cuda.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "qvg_common.cuh"
 #include "qvg_launch.h"
@@ -60,6 +61,7 @@ constexpr int kAtTile = 128;                    // queries per CTA, cached token
 constexpr int kAtOpBytes = kAtTile * kD * 2;    // one 128 x 128 bf16 operand: 32 KB
 constexpr uint64_t kAtWaitNs = 2000000000ull;   // 2 s per bounded wait
 constexpr int kRopeLo = 1024;                   // positions per low-table row block
+static_assert(kRopeLo == 1 << 10, "key positions split by shifts");
 constexpr int kAtMaxSplit = 8;                  // CTAs per cluster, at most (the portable cluster size)
 constexpr int kMaxDevices = 64;
 
@@ -236,17 +238,6 @@ __device__ __forceinline__ void tld32(uint32_t taddr, uint32_t (&r)[32]) {
       :
       : "memory");
 }
-__device__ __forceinline__ void tst32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
-        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
-        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
 
 __device__ __forceinline__ void tld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -349,23 +340,31 @@ __device__ __forceinline__ float2 rope_cs(const AttnParams& p, int64_t pos, int 
 // and assignments, then the centroid rows they select.
 template <int TT, int NR>
 __device__ __forceinline__ void recon_block(const AttnParams& p, const float2* nlut, int which, int h,
-                                            int64_t tok0, int c0, float (&y)[NR][8]) {
+                                            int tok0, int c0, float (&y)[NR][8]) {
   constexpr int TR = TT > 0 ? TT : 1;
   const int T = TT >= 0 ? TT : p.T;
   const int ng = kD / p.G;
   const int g = c0 / p.G;
+  // the head's streams (the same for the whole CTA), then 32-bit offsets
+  // within them (a block has fewer than 2^23 tokens)
+  const int64_t hN = (int64_t)h * p.Nk;
+  const uint8_t* codes = p.codes[which] + hN * (kD / 4) + c0 / 4;
+  const uint8_t* scl = p.scale[which] + hN * ng + g;
+  const uint8_t* zr = p.zero[which] + hN * ng + g;
+  const uint8_t* asg = p.assign[which] + hN;
+  const int64_t asg_stage = (int64_t)p.H * p.Nk;
+  const __nv_bfloat16* tab = p.tab[which] + (int64_t)h * p.K * kD + c0;
+  const int64_t tab_stage = (int64_t)p.H * p.K * kD;
   uint32_t code[NR], sz[NR];
   int kk[NR][TR];
 #pragma unroll
   for (int r = 0; r < NR; ++r) {
-    const int64_t tok = tok0 + r < p.Nk ? tok0 + r : p.Nk - 1;   // past the end: a valid token, result unused
-    const int64_t row = (int64_t)h * p.Nk + tok;
-    code[r] = __ldg(reinterpret_cast<const unsigned short*>(p.codes[which] + row * (kD / 4) + c0 / 4));
-    sz[r] = (uint32_t)__ldg(p.scale[which] + row * ng + g) |
-            (p.sym ? 0u : ((uint32_t)__ldg(p.zero[which] + row * ng + g) << 8));
+    const uint32_t tok = (uint32_t)(tok0 + r < p.Nk ? tok0 + r : p.Nk - 1);   // past the end: a valid token, result unused
+    code[r] = __ldg(reinterpret_cast<const unsigned short*>(codes + tok * (kD / 4)));
+    sz[r] = (uint32_t)__ldg(scl + tok * (uint32_t)ng) | (p.sym ? 0u : ((uint32_t)__ldg(zr + tok * (uint32_t)ng) << 8));
 #pragma unroll
     for (int t = 0; t < TR; ++t)
-      if (TT > 0) kk[r][t] = min((int)__ldg(p.assign[which] + ((int64_t)t * p.H + h) * p.Nk + tok), p.K - 1);
+      if (TT > 0) kk[r][t] = min((int)__ldg(asg + t * asg_stage + tok), p.K - 1);
   }
   uint4 rows[NR][TR];
   if (TT > 0) {
@@ -373,7 +372,7 @@ __device__ __forceinline__ void recon_block(const AttnParams& p, const float2* n
     for (int r = 0; r < NR; ++r)
 #pragma unroll
       for (int t = 0; t < TR; ++t)
-        rows[r][t] = __ldg(reinterpret_cast<const uint4*>(p.tab[which] + (((int64_t)t * p.H + h) * p.K + kk[r][t]) * kD + c0));
+        rows[r][t] = __ldg(reinterpret_cast<const uint4*>(tab + t * tab_stage + (uint32_t)kk[r][t] * kD));
   }
 #pragma unroll
   for (int r = 0; r < NR; ++r) {
@@ -396,10 +395,10 @@ __device__ __forceinline__ void recon_block(const AttnParams& p, const float2* n
 #pragma unroll
       for (int t = TR - 1; t >= 0; --t) add_row(rows[r][t]);
     } else if (TT < 0) {
-      const int64_t tok = tok0 + r < p.Nk ? tok0 + r : p.Nk - 1;
+      const uint32_t tok = (uint32_t)(tok0 + r < p.Nk ? tok0 + r : p.Nk - 1);
       for (int t = T - 1; t >= 0; --t) {
-        const int k = min((int)p.assign[which][((int64_t)t * p.H + h) * p.Nk + tok], p.K - 1);
-        add_row(*reinterpret_cast<const uint4*>(p.tab[which] + (((int64_t)t * p.H + h) * p.K + k) * kD + c0));
+        const int k = min((int)__ldg(asg + t * asg_stage + tok), p.K - 1);
+        add_row(__ldg(reinterpret_cast<const uint4*>(tab + t * tab_stage + (uint32_t)k * kD)));
       }
     }
 #pragma unroll
@@ -505,27 +504,29 @@ qvg_attention_fused(const AttnParams p) {
       fence_after();
       uint8_t* sK = stage_k(st);
       uint8_t* sV = stage_v(st);
-      const int64_t k0 = (int64_t)(j_begin + j) * kAtTile;
+      const int k0 = (j_begin + j) * kAtTile;         // a block has fewer than 2^23 tokens
+      const int last = (int)p.Nk - 1;                 // the host checked that the tables cover it
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         float vk[2][8];
         const int r0 = 4 * rb + 2 * half;
-        const int64_t tok0 = k0 + r0;
+        const int tok0 = k0 + r0;
         recon_block<TT, 2>(p, nlut, 0, h, tok0, 8 * cb, vk);
-        // K rows: rotary embedding of the reconstructed values, then bf16
-        const int64_t pa = rope_pos(p, tok0), pz = rope_pos(p, tok0 + 1);
-        const bool one_hi = pa / kRopeLo == pz / kRopeLo;   // the two positions share the high entry
+        // K rows: rotary embedding of the reconstructed values at their
+        // positions (past the end: the last token's, result unused), then bf16
+        const int pa = min(tok0, last), pz = min(tok0 + 1, last);
+        const bool one_hi = (pa >> 10) == (pz >> 10);   // the two positions share the high entry
         float2 hi[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) hi[e] = __ldg(p.rope_hi + (pa / kRopeLo) * (kD / 2) + 4 * cb + e);
+        for (int e = 0; e < 4; ++e) hi[e] = __ldg(p.rope_hi + (pa >> 10) * (kD / 2) + 4 * cb + e);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
           uint32_t w[4];
-          const int64_t pr = rope_pos(p, tok0 + rr);
+          const int pr = rr == 0 ? pa : pz;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 cs = one_hi ? rope_combine(hi[e], __ldg(p.rope_lo + (pr % kRopeLo) * (kD / 2) + 4 * cb + e))
-                                     : rope_cs(p, tok0 + rr, 4 * cb + e);
+            const float2 h2 = one_hi ? hi[e] : __ldg(p.rope_hi + (pr >> 10) * (kD / 2) + 4 * cb + e);
+            const float2 cs = rope_combine(h2, __ldg(p.rope_lo + (pr & (kRopeLo - 1)) * (kD / 2) + 4 * cb + e));
             const float a = vk[rr][2 * e], b = vk[rr][2 * e + 1];
             w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
                              __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
@@ -587,35 +588,50 @@ qvg_attention_fused(const AttnParams p) {
       // 3. online softmax of the thread's query row; P_g into tensor memory
       {
         const int valid = (int)(p.Nk - k0 < kAtTile ? p.Nk - k0 : kAtTile);
-        float mt = -3.0e38f;                          // pass 1: the row maximum, 16 columns at a time
+        // pass 1: the largest raw score, 16 columns at a time (fp32 rounding is
+        // monotonic, so sl times it is the largest scaled score); the keys past
+        // the end of the cache take no part
+        float mt = -3.0e38f;
+        auto pass1 = [&](auto full) {
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t rg[16];
-          tld16(tSt + lane_base + (uint32_t)(16 * c), rg);
+          for (int c = 0; c < 8; ++c) {
+            uint32_t rg[16];
+            tld16(tSt + lane_base + (uint32_t)(16 * c), rg);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (16 * c + e < valid) mt = fmaxf(mt, __uint_as_float(rg[e]) * p.sl);
-        }
-        const float m_new = fmaxf(m_run, mt);
-        const float alpha = exp2_approx(m_run - m_new);
-        float sum = 0.0f;                             // pass 2: bf16 weights, and their sum
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t rg[16];
-          tld16(tSt + lane_base + (uint32_t)(16 * c), rg);
-          uint32_t w[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int j0 = 16 * c + 2 * e;
-            const float pa = j0 < valid ? exp2_approx(__uint_as_float(rg[2 * e]) * p.sl - m_new) : 0.0f;
-            const float pb = j0 + 1 < valid ? exp2_approx(__uint_as_float(rg[2 * e + 1]) * p.sl - m_new) : 0.0f;
-            w[e] = pack_bf16(pa, pb);
-            // the sum takes the rounded weights, the ones the product uses
-            sum += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
+            for (int e = 0; e < 16; ++e)
+              if (decltype(full)::value || 16 * c + e < valid) mt = fmaxf(mt, __uint_as_float(rg[e]));
           }
-          // keys 16c .. 16c+15 -> columns 8c .. 8c+7, already read
-          tst8(tSt + lane_base + (uint32_t)(8 * c), w);
-        }
+        };
+        if (valid == kAtTile) pass1(std::true_type{}); else pass1(std::false_type{});
+        const float m_new = fmaxf(m_run, mt * p.sl);
+        const float alpha = exp2_approx(m_run - m_new);
+        // pass 2: bf16 weights 2^(sl s - m), two columns per packed op, and
+        // their sum (of the rounded weights, the ones the product uses)
+        const float2 sl2 = make_float2(p.sl, p.sl), nm2 = make_float2(-m_new, -m_new);
+        float2 sum2 = make_float2(0.0f, 0.0f);
+        auto pass2 = [&](auto full) {
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t rg[16];
+            tld16(tSt + lane_base + (uint32_t)(16 * c), rg);
+            uint32_t w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float2 x = __ffma2_rn(make_float2(__uint_as_float(rg[2 * e]), __uint_as_float(rg[2 * e + 1])), sl2, nm2);
+              float pa = exp2_approx(x.x), pb = exp2_approx(x.y);
+              if (!decltype(full)::value) {
+                if (16 * c + 2 * e >= valid) pa = 0.0f;
+                if (16 * c + 2 * e + 1 >= valid) pb = 0.0f;
+              }
+              w[e] = pack_bf16(pa, pb);
+              sum2 = __fadd2_rn(sum2, make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u)));
+            }
+            // keys 16c .. 16c+15 -> columns 8c .. 8c+7, already read
+            tst8(tSt + lane_base + (uint32_t)(8 * c), w);
+          }
+        };
+        if (valid == kAtTile) pass2(std::true_type{}); else pass2(std::false_type{});
+        const float sum = sum2.x + sum2.y;
         l_run = l_run * alpha + sum;
         m_run = m_new;
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {   // rescale O_g
@@ -624,7 +640,12 @@ qvg_attention_fused(const AttnParams p) {
             uint32_t rg[16];
             tld16(tOt + lane_base + (uint32_t)(16 * c), rg);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) rg[e] = __float_as_uint(__uint_as_float(rg[e]) * alpha);
+            for (int e = 0; e < 16; e += 2) {
+              const float2 v = __fmul2_rn(make_float2(__uint_as_float(rg[e]), __uint_as_float(rg[e + 1])),
+                                          make_float2(alpha, alpha));
+              rg[e] = __float_as_uint(v.x);
+              rg[e + 1] = __float_as_uint(v.y);
+            }
             tst16(tOt + lane_base + (uint32_t)(16 * c), rg);
           }
         }
