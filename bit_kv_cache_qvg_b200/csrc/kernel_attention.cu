@@ -80,7 +80,8 @@ struct AttnParams {
   int64_t max_pos;                // largest position the tables cover
   int64_t Nk, Nq;
   int H, K, T, G, sym;
-  int split;                      // CTAs per cluster, each over one range of the cache's tiles
+  int split;                      // cluster CTAs (per query block) over ranges of the cache's tiles
+  int pair;                       // 2: two CTAs (two query blocks) share each tile's reconstruction
   float sl;                       // log2(e) / sqrt(d)
 };
 
@@ -144,6 +145,30 @@ __device__ __forceinline__ bool bar_wait_or_abort(uint64_t* bar, uint32_t parity
     }
   }
 }
+// bar_wait_or_abort with acquire at cluster scope: the barrier also takes
+// arrivals (and the writes they release) from the other CTA of a pair.
+__device__ __forceinline__ bool bar_wait_cluster(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
+  const uint32_t addr = smem_addr(bar);
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort_flag) return false;
+      uint64_t now;
+      asm volatile("mov.u64 %0, %globaltimer;" : "=l"(now));
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > kAtWaitNs) return false;
+    }
+  }
+}
 // Named barrier over `count` threads with an OR of `pred` (every participant
 // gets the same answer).
 __device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
@@ -160,6 +185,21 @@ __device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+// arrive on a barrier of another CTA of the cluster (shared::cluster
+// address), releasing this thread's earlier writes at cluster scope
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr_of_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr_of_bar) : "memory");
+}
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t a, uint4 v) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_b32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 
 // Shared-memory operand descriptor, K-major, 128-byte swizzle: a 128 x 128
@@ -212,6 +252,15 @@ __device__ __forceinline__ void mma_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
                : "memory");
+}
+// the same arrival on the barrier at this offset in every CTA of `mask`
+// (bit i = cluster rank i)
+__device__ __forceinline__ void mma_commit_mc(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_addr(bar)),
+      "h"(mask)
+      : "memory");
 }
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -426,18 +475,25 @@ qvg_attention_fused(const AttnParams p) {
   auto stage_v = [&](int st) { return sK0 + (2 * st + 1) * kAtOpBytes; };
 
   const int h = blockIdx.y;
-  // the cluster's CTAs share the query block; CTA `rank` takes tiles
-  // j_begin .. j_begin + n_loc - 1 of the cache (at least one each)
-  const int rank = (int)(blockIdx.x % (unsigned)p.split);
-  const int64_t q0 = (int64_t)(blockIdx.x / (unsigned)p.split) * (kAtQTiles * kAtTile);
+  // A cluster = pair x split CTAs.  Cluster rank = sr * pair + pr: the pair
+  // (pr = 0, 1) holds two neighbouring blocks of 256 queries and shares the
+  // reconstruction of every tile; split rank sr takes tiles
+  // j_begin .. j_begin + ntiles - 1 of the cache (at least one each).
+  const int csize = p.pair * p.split;
+  const int rank = (int)(blockIdx.x % (unsigned)csize);
+  const int pr = rank % p.pair, sr = rank / p.pair;
+  const int64_t q0 = ((int64_t)(blockIdx.x / (unsigned)csize) * p.pair + pr) * (kAtQTiles * kAtTile);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->s_done[i])));
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->o_done[i])));
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&bars->kv_full[i])), "r"(kAtReconThreads));
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 2;" ::"r"(smem_addr(&bars->kv_empty[i])));   // one commit per query tile
+      // kv_full: every reconstruction thread, or (paired) one thread of each CTA
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&bars->kv_full[i])),
+                   "r"(p.pair > 1 ? 2 : kAtReconThreads));
+      // kv_empty: one commit per query tile of each CTA that reads the stage's contents
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&bars->kv_empty[i])), "r"(2 * p.pair));
     }
     bars->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -479,25 +535,36 @@ qvg_attention_fused(const AttnParams p) {
   fence_before();
   __syncthreads();
   fence_after();
+  // every CTA of the cluster has initialised its barriers before any remote
+  // store or arrival
+  if (csize > 1) cluster_sync();
   const uint32_t tmem = bars->tmem_base;
   // S of query tile t at column 128 t, O of query tile t at column 256 + 128 t
   const uint32_t tS = tmem, tO = tmem + 256;
   const int64_t ntot = (p.Nk + kAtTile - 1) / kAtTile;
-  const int j_begin = (int)(ntot * rank / p.split);
-  const int ntiles = (int)(ntot * (rank + 1) / p.split) - j_begin;   // this CTA's tiles
+  const int j_begin = (int)(ntot * sr / p.split);
+  const int ntiles = (int)(ntot * (sr + 1) / p.split) - j_begin;   // this CTA's tiles
   int s_issued = 0, o_issued = 0;                   // products committed (the issuing threads 0 and 128)
   float m_fin = 0.0f, l_fin = 0.0f;                 // the softmax thread's row maximum and sum at the end
 
   if (warp >= 8) {
     // ---------------------------------------------------------------- reconstruction warps
     // tile j goes to ring stage j mod 2 once the O products of tile j - 2
-    // (the stage's last readers) have completed
+    // (the stage's last readers, in both CTAs of a pair) have completed.
+    // Alone, the CTA reconstructs the whole tile (two passes of 64 keys);
+    // paired, keys 64 pr .. 64 pr + 63 only, stored into both CTAs' stage.
+    // The threads take the abort decision together, so that all of them
+    // reach every barrier of the loop.
     const int r = threadIdx.x - kAtSoftmaxThreads;
-    const int rb = r >> 4, cb = r & 15;             // K: rows 4*rb .. 4*rb+3, channels 8*cb ..
+    const int rb = r >> 4, cb = r & 15;             // K: two rows from 2*rb (4*rb alone), channels 8*cb ..
     const int rbv = r & 31, cbv = r >> 5;           // V: the same blocks, transposed
+    const bool paired = p.pair > 1;
+    const uint32_t own_base = smem_addr(smem);
+    const uint32_t peer_base = paired ? cluster_addr(own_base, (uint32_t)(rank ^ 1)) : 0u;
     for (int j = 0; j < ntiles; ++j) {
       const int st = j & 1;
-      if (j >= 2 && !bar_wait_or_abort(&bars->kv_empty[st], (uint32_t)(((j >> 1) - 1) & 1), abort_flag)) {
+      const bool w = j < 2 || bar_wait_cluster(&bars->kv_empty[st], (uint32_t)(((j >> 1) - 1) & 1), abort_flag);
+      if (named_bar_or(3, kAtReconThreads, !w || *abort_flag)) {
         *abort_flag = 1;
         break;
       }
@@ -507,9 +574,9 @@ qvg_attention_fused(const AttnParams p) {
       const int k0 = (j_begin + j) * kAtTile;         // a block has fewer than 2^23 tokens
       const int last = (int)p.Nk - 1;                 // the host checked that the tables cover it
 #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < 2 / p.pair; ++half) {
         float vk[2][8];
-        const int r0 = 4 * rb + 2 * half;
+        const int r0 = paired ? 64 * pr + 2 * rb : 4 * rb + 2 * half;
         const int tok0 = k0 + r0;
         recon_block<TT, 2>(p, nlut, 0, h, tok0, 8 * cb, vk);
         // K rows: rotary embedding of the reconstructed values at their
@@ -521,31 +588,54 @@ qvg_attention_fused(const AttnParams p) {
         for (int e = 0; e < 4; ++e) hi[e] = __ldg(p.rope_hi + (pa >> 10) * (kD / 2) + 4 * cb + e);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
-          uint32_t w[4];
-          const int pr = rr == 0 ? pa : pz;
+          uint32_t w4[4];
+          const int pos = rr == 0 ? pa : pz;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 h2 = one_hi ? hi[e] : __ldg(p.rope_hi + (pr >> 10) * (kD / 2) + 4 * cb + e);
-            const float2 cs = rope_combine(h2, __ldg(p.rope_lo + (pr & (kRopeLo - 1)) * (kD / 2) + 4 * cb + e));
+            const float2 h2 = one_hi ? hi[e] : __ldg(p.rope_hi + (pos >> 10) * (kD / 2) + 4 * cb + e);
+            const float2 cs = rope_combine(h2, __ldg(p.rope_lo + (pos & (kRopeLo - 1)) * (kD / 2) + 4 * cb + e));
             const float a = vk[rr][2 * e], b = vk[rr][2 * e + 1];
-            w[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
-                             __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
+            w4[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
+                              __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
           }
-          *reinterpret_cast<uint4*>(sK + op_off(r0 + rr, 8 * cb)) = make_uint4(w[0], w[1], w[2], w[3]);
+          const uint4 v4 = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          uint8_t* dst = sK + op_off(r0 + rr, 8 * cb);
+          *reinterpret_cast<uint4*>(dst) = v4;
+          if (paired) st_cluster_v4(peer_base + (smem_addr(dst) - own_base), v4);
         }
         // V, transposed (channel 8*cbv + e holds keys rv, rv+1 in 4 contiguous
         // bytes), with the key and channel blocks swapped: the lanes of a store
         // phase write distinct key chunks of one channel row
-        const int rv = 4 * rbv + 2 * half;
+        const int rv = paired ? 64 * pr + 2 * rbv : 4 * rbv + 2 * half;
         recon_block<TT, 2>(p, nlut, 1, h, k0 + rv, 8 * cbv, vk);
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          *reinterpret_cast<uint32_t*>(sV + op_off(8 * cbv + e, rv)) = pack_bf16(vk[0][e], vk[1][e]);
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t v2 = pack_bf16(vk[0][e], vk[1][e]);
+          uint8_t* dst = sV + op_off(8 * cbv + e, rv);
+          *reinterpret_cast<uint32_t*>(dst) = v2;
+          if (paired) st_cluster_b32(peer_base + (smem_addr(dst) - own_base), v2);
+        }
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
-      mbar_arrive(&bars->kv_full[st]);
-      if (*abort_flag) break;
+      if (paired) {
+        // both halves of the stage are written into both CTAs: one thread of
+        // each CTA arrives on both CTAs' barrier
+        asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");   // visible to the tensor cores
+        named_bar_sync(3, kAtReconThreads);
+        if (r == 0) {
+          mbar_arrive(&bars->kv_full[st]);
+          mbar_arrive_remote(cluster_addr(smem_addr(&bars->kv_full[st]), (uint32_t)(rank ^ 1)));
+        }
+      } else {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
+        mbar_arrive(&bars->kv_full[st]);
+      }
     }
+    // Paired, the other CTA's commits arrive here too: the last use of each
+    // stage must have completed before this CTA may leave (bounded; skipped
+    // once a role has aborted).
+    if (paired && r == 0 && !*abort_flag)
+      for (int j = ntiles - 2 > 0 ? ntiles - 2 : 0; j < ntiles; ++j)
+        if (!bar_wait_cluster(&bars->kv_empty[j & 1], (uint32_t)((j >> 1) & 1), abort_flag)) *abort_flag = 1;
   } else {
     // ---------------------------------------------------------------- softmax warps, two independent groups
     // Group g (warps 4g .. 4g+3) owns query tile g: row 32*(warp mod 4) + lane,
@@ -568,10 +658,11 @@ qvg_attention_fused(const AttnParams p) {
       // 1. S_g once the stage is reconstructed and the previous O_g (which
       // read P_g from these columns) has completed
       if (issuer) {
-        bool w = bar_wait_or_abort(&bars->kv_full[st], (uint32_t)((j >> 1) & 1), abort_flag);
+        bool w = bar_wait_cluster(&bars->kv_full[st], (uint32_t)((j >> 1) & 1), abort_flag);
         if (w && j > 0) w = bar_wait_or_abort(&bars->o_done[g], (uint32_t)((j - 1) & 1), abort_flag);
         if (w) {
           fence_after();
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           const uint32_t a0 = smem_addr(sQ + g * kAtOpBytes), b0 = smem_addr(stage_k(st));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) mma(tSt, op_desc_k(a0, kk), op_desc_k(b0, kk), kk > 0 ? 1u : 0u);
@@ -661,7 +752,8 @@ qvg_attention_fused(const AttnParams p) {
         for (int kk = 0; kk < 8; ++kk)
           mma_ta(tOt, tSt + (uint32_t)(8 * kk), op_desc_k(b0, kk), (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->o_done[g]);
-        mma_commit(&bars->kv_empty[st]);
+        if (p.pair > 1) mma_commit_mc(&bars->kv_empty[st], (uint16_t)((1u << rank) | (1u << (rank ^ 1))));
+        else mma_commit(&bars->kv_empty[st]);
         ++o_issued;
       }
     }
@@ -726,26 +818,28 @@ qvg_attention_fused(const AttnParams p) {
     }
     fence_before();
     cluster_sync();
-    // CTA `rank` merges rows [R0, R1) of the block from every CTA of the
-    // cluster: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s
-    // (a CTA with no tiles has l = 0 and takes no part); a warp per row, a
-    // lane per chunk of four channels.
-    const int R0 = kAtQTiles * kAtTile * rank / p.split, R1 = kAtQTiles * kAtTile * (rank + 1) / p.split;
+    // Split rank sr merges rows [R0, R1) of its query block from the CTAs
+    // that hold the block (cluster ranks m * pair + pr): O = sum_s 2^(m_s - M)
+    // O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s (a CTA with no tiles has
+    // l = 0 and takes no part); a warp per row, a lane per chunk of four
+    // channels.
+    const int R0 = kAtQTiles * kAtTile * sr / p.split, R1 = kAtQTiles * kAtTile * (sr + 1) / p.split;
     for (int t = threadIdx.x; t < (R1 - R0) * 32; t += kAtThreads) {
       const int R = R0 + (t >> 5), c = t & 31;
       const uint32_t ml_a = smem_addr(sML + R), x_a = smem_addr(sX + R * kD + 4 * (c ^ (R & 7)));
       float M = -3.0e38f;
-      for (int r = 0; r < p.split; ++r) {
-        const float2 ml = ld_cluster_f2(cluster_addr(ml_a, (uint32_t)r));
+      for (int m = 0; m < p.split; ++m) {
+        const float2 ml = ld_cluster_f2(cluster_addr(ml_a, (uint32_t)(m * p.pair + pr)));
         if (ml.y > 0.0f) M = fmaxf(M, ml.x);
       }
       float L = 0.0f;
       float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      for (int r = 0; r < p.split; ++r) {
-        const float2 ml = ld_cluster_f2(cluster_addr(ml_a, (uint32_t)r));
+      for (int m = 0; m < p.split; ++m) {
+        const uint32_t src = (uint32_t)(m * p.pair + pr);
+        const float2 ml = ld_cluster_f2(cluster_addr(ml_a, src));
         const float w = ml.y > 0.0f ? exp2_approx(ml.x - M) : 0.0f;
         if (w > 0.0f) {
-          const float4 x = ld_cluster_f4(cluster_addr(x_a, (uint32_t)r));
+          const float4 x = ld_cluster_f4(cluster_addr(x_a, src));
           acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
           L += w * ml.y;
         }
@@ -757,9 +851,9 @@ qvg_attention_fused(const AttnParams p) {
             make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
       }
     }
-    // no CTA leaves while another still reads its shared memory
-    cluster_sync();
   }
+  // no CTA leaves while another still reads or writes its shared memory
+  if (csize > 1) cluster_sync();
   if (warp == 0) {
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
@@ -801,7 +895,7 @@ template <int TT>
 static cudaError_t launch_attention_t(const AttnParams& p, dim3 grid, size_t smem, cudaStream_t s) {
   cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(qvg_attention_fused<TT>), smem);
   if (e != cudaSuccess) return e;
-  if (p.split == 1) {
+  if (p.split * p.pair == 1) {
     qvg_attention_fused<TT><<<grid, kAtThreads, smem, s>>>(p);
     return cudaGetLastError();
   }
@@ -812,7 +906,7 @@ static cudaError_t launch_attention_t(const AttnParams& p, dim3 grid, size_t sme
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)p.split;
+  attr[0].val.clusterDim.x = (unsigned)(p.split * p.pair);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
@@ -860,43 +954,53 @@ static int resident_clusters(int split) {
   return n;
 }
 
-// The split of the cache over a cluster: the one with the least estimated
-// time, (waves of resident clusters) x (tiles per CTA + the fixed cost of a
-// CTA, about two tiles), over 1 .. 4 CTAs per cluster; a positive `forced`
-// is taken as it is.  Never more CTAs than the cache has tiles.
+// The cluster shape: pair = 2 when there are at least two blocks of 256
+// queries (two CTAs share every tile's reconstruction), and the split of the
+// cache with the least estimated time, (waves of resident clusters) x
+// (tiles per CTA + the fixed cost of a CTA, about two tiles), over 1 .. 4
+// ranges (cluster size pair x split at most 8); a positive `forced` split is
+// taken as it is.  Never more ranges than the cache has tiles.
+struct SplitPlan { int pair, split; };
 template <int TT>
-static int choose_split(int64_t Nk, int64_t Nq, int H, int forced) {
+static SplitPlan choose_split(int64_t Nk, int64_t Nq, int H, int forced) {
   const int64_t ntot = (Nk + kAtTile - 1) / kAtTile;
-  const int smax = (int)(ntot < kAtMaxSplit ? ntot : kAtMaxSplit);
-  if (forced > 0) return forced < smax ? forced : smax;
-  const int64_t units = (Nq + kAtQTiles * kAtTile - 1) / (kAtQTiles * kAtTile) * H;
+  const int64_t qblocks = (Nq + kAtQTiles * kAtTile - 1) / (kAtQTiles * kAtTile);
+  const int pair = qblocks >= 2 ? 2 : 1;
+  const int cap = kAtMaxSplit / pair;
+  const int smax = (int)(ntot < cap ? ntot : cap);
+  if (forced > 0) return SplitPlan{pair, forced < smax ? forced : smax};
+  const int64_t units = (qblocks + pair - 1) / pair * H;
   int best = 1;
   double best_cost = 0.0;
   for (int sp = 1; sp <= (smax < 4 ? smax : 4); ++sp) {
-    const int n = resident_clusters<TT>(sp);
+    const int n = resident_clusters<TT>(pair * sp);
     if (n <= 0) continue;
     const double waves = (double)((units + n - 1) / n);
     const double cost = waves * (double)((ntot + sp - 1) / sp + 2);
     if (sp == 1 || cost < best_cost) { best = sp; best_cost = cost; }
   }
-  return best;
+  return SplitPlan{pair, best};
 }
 
 template <int TT>
 static cudaError_t launch_attention_split(AttnParams& p, int64_t Nq, size_t smem, int forced, cudaStream_t s) {
-  p.split = choose_split<TT>(p.Nk, Nq, p.H, forced);
-  const dim3 grid((unsigned)(p.split * ((Nq + kAtQTiles * kAtTile - 1) / (kAtQTiles * kAtTile))), (unsigned)p.H);
+  const SplitPlan plan = choose_split<TT>(p.Nk, Nq, p.H, forced);
+  p.split = plan.split;
+  p.pair = plan.pair;
+  const int64_t qblocks = (Nq + kAtQTiles * kAtTile - 1) / (kAtQTiles * kAtTile);
+  const int64_t units = (qblocks + plan.pair - 1) / plan.pair;
+  const dim3 grid((unsigned)(units * plan.pair * plan.split), (unsigned)p.H);
   return launch_attention_t<TT>(p, grid, smem, s);
 }
 
 int attention_split(int T, int64_t Nk, int64_t Nq, int H, int forced) {
   switch (T) {
-    case 0: return choose_split<0>(Nk, Nq, H, forced);
-    case 1: return choose_split<1>(Nk, Nq, H, forced);
-    case 2: return choose_split<2>(Nk, Nq, H, forced);
-    case 3: return choose_split<3>(Nk, Nq, H, forced);
-    case 4: return choose_split<4>(Nk, Nq, H, forced);
-    default: return choose_split<-1>(Nk, Nq, H, forced);
+    case 0: return choose_split<0>(Nk, Nq, H, forced).split;
+    case 1: return choose_split<1>(Nk, Nq, H, forced).split;
+    case 2: return choose_split<2>(Nk, Nq, H, forced).split;
+    case 3: return choose_split<3>(Nk, Nq, H, forced).split;
+    case 4: return choose_split<4>(Nk, Nq, H, forced).split;
+    default: return choose_split<-1>(Nk, Nq, H, forced).split;
   }
 }
 

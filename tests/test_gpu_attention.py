@@ -75,6 +75,8 @@ def _run_case(q, ora, cfg, H, Nk, Nq, q_scale, seed, base=10000.0):
     (2, 256, 128, 1, 64, 256, 1, 0.05),      # the QVG point (one scale per group), whole tiles
     (1, 77, 33, 0, 32, 1, 0, 0.2),           # plain rounding, one partial tile each
     (2, 4680, 130, 4, 16, 256, 1, 0.02),     # the QVG-Pro point, a Self-Forcing-scale chunk
+    (2, 2900, 600, 2, 64, 128, 0, 0.05),     # three query blocks: two CTAs share each tile, one CTA has no queries
+    (1, 1300, 512, 1, 32, 64, 1, 0.05),      # two whole query blocks, one pair
 ])
 def test_attention_matches_oracle(q, ora, H, Nk, Nq, T, G, K, mode, q_scale):
     cfg = q.config(K=K, T=T, group_size=G, iters=3, scale_mode=mode)
@@ -83,15 +85,18 @@ def test_attention_matches_oracle(q, ora, H, Nk, Nq, T, G, K, mode, q_scale):
 
 
 @pytest.mark.parametrize("split", [2, 3, 4, 8])
-def test_attention_split_over_a_cluster_matches_oracle(q, ora, split):
+@pytest.mark.parametrize("Nq", [200, 300])
+def test_attention_split_over_a_cluster_matches_oracle(q, ora, split, Nq):
     """The cache of each query block split over a cluster of `split` CTAs
     (ragged ranges: 8 tiles over 3 CTAs; 8 CTAs of one tile each) stays
-    within the bound."""
+    within the bound.  With one block of 256 queries (Nq = 200) the CTAs
+    are alone; with two (Nq = 300) they come in pairs that share the
+    reconstruction, and a cluster holds at most 4 ranges."""
     cfg = q.config(K=64, T=2, group_size=64, iters=3, scale_mode=0)
     prev = q.attention_set_split(split)
     try:
-        assert q.attention_split(cfg, 1000, 2, 300) == min(split, 8)
-        typical = _run_case(q, ora, cfg, 2, 1000, 300, 0.05, seed=1002)
+        assert q.attention_split(cfg, 1000, 2, Nq) == min(split, 8 if Nq <= 256 else 4)
+        typical = _run_case(q, ora, cfg, 2, 1000, Nq, 0.05, seed=1002)
     finally:
         q.attention_set_split(prev)
     assert typical < 0.25
