@@ -379,87 +379,96 @@ __device__ __forceinline__ float2 rope_cs(const AttnParams& p, int64_t pos, int 
   return rope_combine(__ldg(p.rope_hi + (pos / kRopeLo) * (kD / 2) + i), __ldg(p.rope_lo + (pos % kRopeLo) * (kD / 2) + i));
 }
 
-// Reconstruct channels c0 .. c0+7 of the NR tokens tok0 .. tok0+NR-1 (those
-// below Nk) of cache `which` (0 = K, 1 = V) of head h: y = s*q + m (or
-// s*(u - 2)), plus the centroids of stages T, ..., 1 in that order, each an
-// fp32 add, then one rounding to bf16 -- the arithmetic of qvg_dequant_fused.
-// The results are fp32 values of the rounded bf16 numbers (zero for tokens
-// past the end).  TT > 0 fixes the stage count (at most 4) so that the loads
-// of all NR tokens are issued together: first the codes, scale/zero bytes
-// and assignments, then the centroid rows they select.
+// Reconstruction of channels c0 .. c0+7 of the NR tokens tok0 .. tok0+NR-1
+// (those below Nk) of cache `which` (0 = K, 1 = V) of head h: y = s*q + m
+// (or s*(u - 2)), plus the centroids of stages T, ..., 1 in that order, each
+// an fp32 add, then one rounding to bf16 -- the arithmetic of
+// qvg_dequant_fused.  The results are fp32 values of the rounded bf16
+// numbers (zero for tokens past the end).  In three steps, so that a thread
+// can issue the loads of several blocks before it waits for any: the
+// per-token codes, scale/zero bytes and assignments; the centroid rows they
+// select (TT > 0, a fixed stage count of at most 4); the arithmetic.
 template <int TT, int NR>
-__device__ __forceinline__ void recon_block(const AttnParams& p, const float2* nlut, int which, int h,
-                                            int tok0, int c0, float (&y)[NR][8]) {
-  constexpr int TR = TT > 0 ? TT : 1;
-  const int T = TT >= 0 ? TT : p.T;
-  const int ng = kD / p.G;
-  const int g = c0 / p.G;
-  // the head's streams (the same for the whole CTA), then 32-bit offsets
-  // within them (a block has fewer than 2^23 tokens)
-  const int64_t hN = (int64_t)h * p.Nk;
-  const uint8_t* codes = p.codes[which] + hN * (kD / 4) + c0 / 4;
-  const uint8_t* scl = p.scale[which] + hN * ng + g;
-  const uint8_t* zr = p.zero[which] + hN * ng + g;
-  const uint8_t* asg = p.assign[which] + hN;
-  const int64_t asg_stage = (int64_t)p.H * p.Nk;
-  const __nv_bfloat16* tab = p.tab[which] + (int64_t)h * p.K * kD + c0;
-  const int64_t tab_stage = (int64_t)p.H * p.K * kD;
+struct ReconBlock {
+  static constexpr int TR = TT > 0 ? TT : 1;
+  int tok0, c0, which;
   uint32_t code[NR], sz[NR];
   int kk[NR][TR];
-#pragma unroll
-  for (int r = 0; r < NR; ++r) {
-    const uint32_t tok = (uint32_t)(tok0 + r < p.Nk ? tok0 + r : p.Nk - 1);   // past the end: a valid token, result unused
-    code[r] = __ldg(reinterpret_cast<const unsigned short*>(codes + tok * (kD / 4)));
-    sz[r] = (uint32_t)__ldg(scl + tok * (uint32_t)ng) | (p.sym ? 0u : ((uint32_t)__ldg(zr + tok * (uint32_t)ng) << 8));
-#pragma unroll
-    for (int t = 0; t < TR; ++t)
-      if (TT > 0) kk[r][t] = min((int)__ldg(asg + t * asg_stage + tok), p.K - 1);
-  }
   uint4 rows[NR][TR];
-  if (TT > 0) {
+
+  // the head's streams (the same for the whole CTA), then 32-bit offsets
+  // within them (a block has fewer than 2^23 tokens)
+  __device__ __forceinline__ void load_tokens(const AttnParams& p, int w, int h, int t0, int ch) {
+    which = w; tok0 = t0; c0 = ch;
+    const int ng = kD / p.G;
+    const int64_t hN = (int64_t)h * p.Nk;
+    const uint8_t* codes = p.codes[w] + hN * (kD / 4) + c0 / 4;
+    const uint8_t* scl = p.scale[w] + hN * ng + c0 / p.G;
+    const uint8_t* zr = p.zero[w] + hN * ng + c0 / p.G;
+    const uint8_t* asg = p.assign[w] + hN;
+    const int64_t asg_stage = (int64_t)p.H * p.Nk;
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      const uint32_t tok = (uint32_t)(tok0 + r < p.Nk ? tok0 + r : p.Nk - 1);   // past the end: a valid token, result unused
+      code[r] = __ldg(reinterpret_cast<const unsigned short*>(codes + tok * (kD / 4)));
+      sz[r] = (uint32_t)__ldg(scl + tok * (uint32_t)ng) | (p.sym ? 0u : ((uint32_t)__ldg(zr + tok * (uint32_t)ng) << 8));
+#pragma unroll
+      for (int t = 0; t < TR; ++t)
+        if (TT > 0) kk[r][t] = min((int)__ldg(asg + t * asg_stage + tok), p.K - 1);
+    }
+  }
+  __device__ __forceinline__ void load_rows(const AttnParams& p, int h) {
+    if (TT <= 0) return;
+    const __nv_bfloat16* tab = p.tab[which] + (int64_t)h * p.K * kD + c0;
+    const int64_t tab_stage = (int64_t)p.H * p.K * kD;
 #pragma unroll
     for (int r = 0; r < NR; ++r)
 #pragma unroll
       for (int t = 0; t < TR; ++t)
         rows[r][t] = __ldg(reinterpret_cast<const uint4*>(tab + t * tab_stage + (uint32_t)kk[r][t] * kD));
   }
+  __device__ __forceinline__ void finish(const AttnParams& p, const float2* nlut, int h, float (&y)[NR][8]) const {
+    const int T = TT >= 0 ? TT : p.T;
 #pragma unroll
-  for (int r = 0; r < NR; ++r) {
-    // y = s*q + m (or s*(u - 2)), exact in fp32, two channels per op through
-    // the nibble table (which holds q, or u - 2 in the symmetric mode)
-    const float2 sm = e4m3x2_to_f2(sz[r]);
-    const float2 s2 = make_float2(sm.x, sm.x), m2 = make_float2(sm.y, sm.y);
-    float2 y2[4];
+    for (int r = 0; r < NR; ++r) {
+      // y = s*q + m (or s*(u - 2)), exact in fp32, two channels per op through
+      // the nibble table (which holds q, or u - 2 in the symmetric mode)
+      const float2 sm = e4m3x2_to_f2(sz[r]);
+      const float2 s2 = make_float2(sm.x, sm.x), m2 = make_float2(sm.y, sm.y);
+      float2 y2[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      y2[e] = p.sym ? __fmul2_rn(s2, nlut[(code[r] >> (4 * e)) & 0xFu])
-                    : __ffma2_rn(s2, nlut[(code[r] >> (4 * e)) & 0xFu], m2);
-    auto add_row = [&](const uint4 w) {
-      y2[0] = __fadd2_rn(y2[0], make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u)));
-      y2[1] = __fadd2_rn(y2[1], make_float2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u)));
-      y2[2] = __fadd2_rn(y2[2], make_float2(__uint_as_float(w.z << 16), __uint_as_float(w.z & 0xFFFF0000u)));
-      y2[3] = __fadd2_rn(y2[3], make_float2(__uint_as_float(w.w << 16), __uint_as_float(w.w & 0xFFFF0000u)));
-    };
-    if (TT > 0) {
+      for (int e = 0; e < 4; ++e)
+        y2[e] = p.sym ? __fmul2_rn(s2, nlut[(code[r] >> (4 * e)) & 0xFu])
+                      : __ffma2_rn(s2, nlut[(code[r] >> (4 * e)) & 0xFu], m2);
+      auto add_row = [&](const uint4 w) {
+        y2[0] = __fadd2_rn(y2[0], make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u)));
+        y2[1] = __fadd2_rn(y2[1], make_float2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u)));
+        y2[2] = __fadd2_rn(y2[2], make_float2(__uint_as_float(w.z << 16), __uint_as_float(w.z & 0xFFFF0000u)));
+        y2[3] = __fadd2_rn(y2[3], make_float2(__uint_as_float(w.w << 16), __uint_as_float(w.w & 0xFFFF0000u)));
+      };
+      if (TT > 0) {
 #pragma unroll
-      for (int t = TR - 1; t >= 0; --t) add_row(rows[r][t]);
-    } else if (TT < 0) {
-      const uint32_t tok = (uint32_t)(tok0 + r < p.Nk ? tok0 + r : p.Nk - 1);
-      for (int t = T - 1; t >= 0; --t) {
-        const int k = min((int)__ldg(asg + t * asg_stage + tok), p.K - 1);
-        add_row(__ldg(reinterpret_cast<const uint4*>(tab + t * tab_stage + (uint32_t)k * kD)));
+        for (int t = TR - 1; t >= 0; --t) add_row(rows[r][t]);
+      } else if (TT < 0) {
+        const uint32_t tok = (uint32_t)(tok0 + r < p.Nk ? tok0 + r : p.Nk - 1);
+        const uint8_t* asg = p.assign[which] + (int64_t)h * p.Nk;
+        const __nv_bfloat16* tab = p.tab[which] + (int64_t)h * p.K * kD + c0;
+        for (int t = T - 1; t >= 0; --t) {
+          const int k = min((int)__ldg(asg + t * (int64_t)p.H * p.Nk + tok), p.K - 1);
+          add_row(__ldg(reinterpret_cast<const uint4*>(tab + t * (int64_t)p.H * p.K * kD + (uint32_t)k * kD)));
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) { y[r][2 * e] = y2[e].x; y[r][2 * e + 1] = y2[e].y; }
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const uint32_t b = pack_bf16(y[r][e], y[r][e + 1]);
+        y[r][e] = tok0 + r < p.Nk ? __uint_as_float(b << 16) : 0.0f;
+        y[r][e + 1] = tok0 + r < p.Nk ? __uint_as_float(b & 0xFFFF0000u) : 0.0f;
       }
     }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) { y[r][2 * e] = y2[e].x; y[r][2 * e + 1] = y2[e].y; }
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      const uint32_t b = pack_bf16(y[r][e], y[r][e + 1]);
-      y[r][e] = tok0 + r < p.Nk ? __uint_as_float(b << 16) : 0.0f;
-      y[r][e + 1] = tok0 + r < p.Nk ? __uint_as_float(b & 0xFFFF0000u) : 0.0f;
-    }
   }
-}
+};
 
 template <int TT>
 __global__ void __launch_bounds__(kAtThreads, 1)
@@ -489,9 +498,9 @@ qvg_attention_fused(const AttnParams p) {
     for (int i = 0; i < 2; ++i) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->s_done[i])));
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars->o_done[i])));
-      // kv_full: every reconstruction thread, or (paired) one thread of each CTA
+      // kv_full: one lane of every reconstruction warp of each CTA that writes the stage
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&bars->kv_full[i])),
-                   "r"(p.pair > 1 ? 2 : kAtReconThreads));
+                   "r"(kAtReconThreads / 32 * p.pair));
       // kv_empty: one commit per query tile of each CTA that reads the stage's contents
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(&bars->kv_empty[i])), "r"(2 * p.pair));
     }
@@ -553,8 +562,8 @@ qvg_attention_fused(const AttnParams p) {
     // (the stage's last readers, in both CTAs of a pair) have completed.
     // Alone, the CTA reconstructs the whole tile (two passes of 64 keys);
     // paired, keys 64 pr .. 64 pr + 63 only, stored into both CTAs' stage.
-    // The threads take the abort decision together, so that all of them
-    // reach every barrier of the loop.
+    // Each warp arrives for itself once its lanes have stored their blocks,
+    // so that the warps drift apart and their memory latencies overlap.
     const int r = threadIdx.x - kAtSoftmaxThreads;
     const int rb = r >> 4, cb = r & 15;             // K: two rows from 2*rb (4*rb alone), channels 8*cb ..
     const int rbv = r & 31, cbv = r >> 5;           // V: the same blocks, transposed
@@ -564,7 +573,7 @@ qvg_attention_fused(const AttnParams p) {
     for (int j = 0; j < ntiles; ++j) {
       const int st = j & 1;
       const bool w = j < 2 || bar_wait_cluster(&bars->kv_empty[st], (uint32_t)(((j >> 1) - 1) & 1), abort_flag);
-      if (named_bar_or(3, kAtReconThreads, !w || *abort_flag)) {
+      if (__any_sync(0xffffffffu, !w || *abort_flag)) {
         *abort_flag = 1;
         break;
       }
@@ -578,7 +587,16 @@ qvg_attention_fused(const AttnParams p) {
         float vk[2][8];
         const int r0 = paired ? 64 * pr + 2 * rb : 4 * rb + 2 * half;
         const int tok0 = k0 + r0;
-        recon_block<TT, 2>(p, nlut, 0, h, tok0, 8 * cb, vk);
+        // V, transposed (channel 8*cbv + e holds keys rv, rv+1 in 4 contiguous
+        // bytes), with the key and channel blocks swapped: the lanes of a store
+        // phase write distinct key chunks of one channel row
+        const int rv = paired ? 64 * pr + 2 * rbv : 4 * rbv + 2 * half;
+        ReconBlock<TT, 2> bk, bv;
+        bk.load_tokens(p, 0, h, tok0, 8 * cb);
+        bv.load_tokens(p, 1, h, k0 + rv, 8 * cbv);
+        bk.load_rows(p, h);
+        bv.load_rows(p, h);
+        bk.finish(p, nlut, h, vk);
         // K rows: rotary embedding of the reconstructed values at their
         // positions (past the end: the last token's, result unused), then bf16
         const int pa = min(tok0, last), pz = min(tok0 + 1, last);
@@ -603,11 +621,7 @@ qvg_attention_fused(const AttnParams p) {
           *reinterpret_cast<uint4*>(dst) = v4;
           if (paired) st_cluster_v4(peer_base + (smem_addr(dst) - own_base), v4);
         }
-        // V, transposed (channel 8*cbv + e holds keys rv, rv+1 in 4 contiguous
-        // bytes), with the key and channel blocks swapped: the lanes of a store
-        // phase write distinct key chunks of one channel row
-        const int rv = paired ? 64 * pr + 2 * rbv : 4 * rbv + 2 * half;
-        recon_block<TT, 2>(p, nlut, 1, h, k0 + rv, 8 * cbv, vk);
+        bv.finish(p, nlut, h, vk);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const uint32_t v2 = pack_bf16(vk[0][e], vk[1][e]);
@@ -616,18 +630,14 @@ qvg_attention_fused(const AttnParams p) {
           if (paired) st_cluster_b32(peer_base + (smem_addr(dst) - own_base), v2);
         }
       }
-      if (paired) {
-        // both halves of the stage are written into both CTAs: one thread of
-        // each CTA arrives on both CTAs' barrier
-        asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");   // visible to the tensor cores
-        named_bar_sync(3, kAtReconThreads);
-        if (r == 0) {
-          mbar_arrive(&bars->kv_full[st]);
-          mbar_arrive_remote(cluster_addr(smem_addr(&bars->kv_full[st]), (uint32_t)(rank ^ 1)));
-        }
-      } else {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
+      // visible to the tensor cores (of both CTAs when paired), then one
+      // lane arrives for the warp (on both CTAs' barrier when paired)
+      if (paired) asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+      else asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
         mbar_arrive(&bars->kv_full[st]);
+        if (paired) mbar_arrive_remote(cluster_addr(smem_addr(&bars->kv_full[st]), (uint32_t)(rank ^ 1)));
       }
     }
     // Paired, the other CTA's commits arrive here too: the last use of each
