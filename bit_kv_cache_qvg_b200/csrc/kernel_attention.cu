@@ -417,6 +417,17 @@ struct ReconBlock {
         if (TT > 0) kk[r][t] = min((int)__ldg(asg + t * asg_stage + tok), p.K - 1);
     }
   }
+  // the per-token part of another block (loaded one step ahead)
+  __device__ __forceinline__ void take_tokens(const ReconBlock& o) {
+    which = o.which; tok0 = o.tok0; c0 = o.c0;
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      code[r] = o.code[r];
+      sz[r] = o.sz[r];
+#pragma unroll
+      for (int t = 0; t < TR; ++t) kk[r][t] = o.kk[r][t];
+    }
+  }
   __device__ __forceinline__ void load_rows(const AttnParams& p, int h) {
     if (TT <= 0) return;
     const __nv_bfloat16* tab = p.tab[which] + (int64_t)h * p.K * kD + c0;
@@ -558,6 +569,9 @@ qvg_attention_fused(const AttnParams p) {
 
   if (warp >= 8) {
     // ---------------------------------------------------------------- reconstruction warps
+    // Registers move from the softmax warpgroups (48 each thread) to these
+    // four (96): 256 x 48 + 512 x 96 = 768 x 80, the launch's allocation.
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 96;");
     // tile j goes to ring stage j mod 2 once the O products of tile j - 2
     // (the stage's last readers, in both CTAs of a pair) have completed.
     // Alone, the CTA reconstructs the whole tile (two passes of 64 keys);
@@ -570,32 +584,53 @@ qvg_attention_fused(const AttnParams p) {
     const bool paired = p.pair > 1;
     const uint32_t own_base = smem_addr(smem);
     const uint32_t peer_base = paired ? cluster_addr(own_base, (uint32_t)(rank ^ 1)) : 0u;
-    for (int j = 0; j < ntiles; ++j) {
+    // Steps of 64 keys (two per tile alone, one paired).  With at most two
+    // stages a thread's per-token bytes of the next step are loaded while it
+    // works on this one (more stages' centroid rows leave no registers for it).
+    constexpr bool kAhead = TT >= 0 && TT <= 2;
+    const int nh = 2 / p.pair;
+    const int nsteps = ntiles * nh;
+    auto row_k = [&](int half) { return paired ? 64 * pr + 2 * rb : 4 * rb + 2 * half; };
+    auto row_v = [&](int half) { return paired ? 64 * pr + 2 * rbv : 4 * rbv + 2 * half; };
+    const int last = (int)p.Nk - 1;                   // the host checked that the tables cover it
+    ReconBlock<TT, 2> bk, bv;
+    if (kAhead && nsteps > 0) {
+      bk.load_tokens(p, 0, h, j_begin * kAtTile + row_k(0), 8 * cb);
+      bv.load_tokens(p, 1, h, j_begin * kAtTile + row_v(0), 8 * cbv);
+    }
+#pragma unroll 1
+    for (int s = 0; s < nsteps; ++s) {
+      const int j = nh == 1 ? s : s >> 1, half = s - j * nh;
       const int st = j & 1;
-      const bool w = j < 2 || bar_wait_cluster(&bars->kv_empty[st], (uint32_t)(((j >> 1) - 1) & 1), abort_flag);
-      if (__any_sync(0xffffffffu, !w || *abort_flag)) {
-        *abort_flag = 1;
-        break;
+      if (half == 0) {
+        const bool w = j < 2 || bar_wait_cluster(&bars->kv_empty[st], (uint32_t)(((j >> 1) - 1) & 1), abort_flag);
+        if (__any_sync(0xffffffffu, !w || *abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        fence_after();
       }
-      fence_after();
       uint8_t* sK = stage_k(st);
       uint8_t* sV = stage_v(st);
-      const int k0 = (j_begin + j) * kAtTile;         // a block has fewer than 2^23 tokens
-      const int last = (int)p.Nk - 1;                 // the host checked that the tables cover it
-#pragma unroll 1
-      for (int half = 0; half < 2 / p.pair; ++half) {
+      {
         float vk[2][8];
-        const int r0 = paired ? 64 * pr + 2 * rb : 4 * rb + 2 * half;
-        const int tok0 = k0 + r0;
+        const int r0 = row_k(half), tok0 = (j_begin + j) * kAtTile + r0;
         // V, transposed (channel 8*cbv + e holds keys rv, rv+1 in 4 contiguous
         // bytes), with the key and channel blocks swapped: the lanes of a store
         // phase write distinct key chunks of one channel row
-        const int rv = paired ? 64 * pr + 2 * rbv : 4 * rbv + 2 * half;
-        ReconBlock<TT, 2> bk, bv;
-        bk.load_tokens(p, 0, h, tok0, 8 * cb);
-        bv.load_tokens(p, 1, h, k0 + rv, 8 * cbv);
+        const int rv = row_v(half);
+        if (!kAhead) {
+          bk.load_tokens(p, 0, h, (j_begin + j) * kAtTile + r0, 8 * cb);
+          bv.load_tokens(p, 1, h, (j_begin + j) * kAtTile + rv, 8 * cbv);
+        }
         bk.load_rows(p, h);
         bv.load_rows(p, h);
+        ReconBlock<TT, 2> nk, nv;
+        if (kAhead && s + 1 < nsteps) {
+          const int j1 = nh == 1 ? s + 1 : (s + 1) >> 1, half1 = s + 1 - j1 * nh;
+          nk.load_tokens(p, 0, h, (j_begin + j1) * kAtTile + row_k(half1), 8 * cb);
+          nv.load_tokens(p, 1, h, (j_begin + j1) * kAtTile + row_v(half1), 8 * cbv);
+        }
         bk.finish(p, nlut, h, vk);
         // K rows: rotary embedding of the reconstructed values at their
         // positions (past the end: the last token's, result unused), then bf16
@@ -629,7 +664,12 @@ qvg_attention_fused(const AttnParams p) {
           *reinterpret_cast<uint32_t*>(dst) = v2;
           if (paired) st_cluster_b32(peer_base + (smem_addr(dst) - own_base), v2);
         }
+        if (kAhead) {
+          bk.take_tokens(nk);
+          bv.take_tokens(nv);
+        }
       }
+      if (half < nh - 1) continue;
       // visible to the tensor cores (of both CTAs when paired), then one
       // lane arrives for the warp (on both CTAs' barrier when paired)
       if (paired) asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
@@ -648,6 +688,7 @@ qvg_attention_fused(const AttnParams p) {
         if (!bar_wait_cluster(&bars->kv_empty[j & 1], (uint32_t)((j >> 1) & 1), abort_flag)) *abort_flag = 1;
   } else {
     // ---------------------------------------------------------------- softmax warps, two independent groups
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 48;");
     // Group g (warps 4g .. 4g+3) owns query tile g: row 32*(warp mod 4) + lane,
     // the warp's tensor-memory lane quarter.  Its first thread issues the
     // group's products: S_g = Q_g'K'^T when a stage is full, then, after the
