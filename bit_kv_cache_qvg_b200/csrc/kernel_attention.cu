@@ -36,9 +36,8 @@
 // leaves its unnormalised O with its row maximum and sum in shared memory and
 // the cluster merges them through distributed shared memory (the usual
 // rescaling of partial softmax sums); otherwise O / l is written directly.
-// The rotary angles come from two tables of (cos, sin) in fp32, p = 1024 a + b:
-// (1024 a) theta_i and b theta_i, combined by the angle-sum identity
-// (qvg_rope_tables builds them in fp64).  Every mbarrier wait is bounded; on
+// The rotary (cos, sin) pairs come from a table of every position, formed
+// in fp64 and rounded to fp32 (qvg_rope_tables).  Every mbarrier wait is bounded; on
 // expiry the kernel records QVG_ERR_DEVICE_TIMEOUT in the status word at the
 // start of the tables buffer and stops.  No TMA and no multicast: the
 // operands are written by the threads that reconstruct them.
@@ -60,8 +59,6 @@ constexpr int kAtReconThreads = 512;            // warps 8-23: reconstruction in
 constexpr int kAtTile = 128;                    // queries per CTA, cached tokens per tile
 constexpr int kAtOpBytes = kAtTile * kD * 2;    // one 128 x 128 bf16 operand: 32 KB
 constexpr uint64_t kAtWaitNs = 2000000000ull;   // 2 s per bounded wait
-constexpr int kRopeLo = 1024;                   // positions per low-table row block
-static_assert(kRopeLo == 1 << 10, "key positions split by shifts");
 constexpr int kAtMaxSplit = 8;                  // CTAs per cluster, at most (the portable cluster size)
 constexpr int kMaxDevices = 64;
 
@@ -73,8 +70,7 @@ struct AttnParams {
   const __nv_bfloat16* tab[2];    // [T][H][K][d]
   const __nv_bfloat16* Q;         // [H][Nq][d], before the rotary embedding
   const int64_t* qpos;            // [Nq] query positions
-  const float2* rope_hi;          // [n_hi][d/2]: (cos, sin) of 1024 a theta_i
-  const float2* rope_lo;          // [1024][d/2]: (cos, sin) of b theta_i
+  const float2* rope;             // [max_pos + 1][d/2]: (cos, sin) of p theta_i
   float* O;                       // [H][Nq][d]
   uint32_t* status;
   int64_t max_pos;                // largest position the tables cover
@@ -364,19 +360,11 @@ __device__ __forceinline__ float2 e4m3x2_to_f2(uint32_t pair16) {
   return make_float2(lo, hi);
 }
 
-// (cos, sin) of the rotary angle of pair i at position p from the two tables
-// (positions outside [0, max_pos] are clamped, so the reads stay in bounds).
-__device__ __forceinline__ int64_t rope_pos(const AttnParams& p, int64_t pos) {
-  return pos < 0 ? 0 : (pos > p.max_pos ? p.max_pos : pos);
-}
-// the angle sum from the high-table entry a and the low-table entry b
-__device__ __forceinline__ float2 rope_combine(float2 a, float2 b) {
-  return make_float2(__fsub_rn(__fmul_rn(a.x, b.x), __fmul_rn(a.y, b.y)),
-                     __fadd_rn(__fmul_rn(a.y, b.x), __fmul_rn(a.x, b.y)));
-}
+// (cos, sin) of the rotary angle of pair i at position pos (positions outside
+// [0, max_pos] are clamped, so the reads stay in bounds).
 __device__ __forceinline__ float2 rope_cs(const AttnParams& p, int64_t pos, int i) {
-  pos = rope_pos(p, pos);
-  return rope_combine(__ldg(p.rope_hi + (pos / kRopeLo) * (kD / 2) + i), __ldg(p.rope_lo + (pos % kRopeLo) * (kD / 2) + i));
+  pos = pos < 0 ? 0 : (pos > p.max_pos ? p.max_pos : pos);
+  return __ldg(p.rope + pos * (kD / 2) + i);
 }
 
 // Reconstruction of channels c0 .. c0+7 of the NR tokens tok0 .. tok0+NR-1
@@ -614,7 +602,7 @@ qvg_attention_fused(const AttnParams p) {
       uint8_t* sV = stage_v(st);
       {
         float vk[2][8];
-        const int r0 = row_k(half), tok0 = (j_begin + j) * kAtTile + r0;
+        const int r0 = row_k(half), tok0 = kAhead ? bk.tok0 : (j_begin + j) * kAtTile + r0;
         // V, transposed (channel 8*cbv + e holds keys rv, rv+1 in 4 contiguous
         // bytes), with the key and channel blocks swapped: the lanes of a store
         // phase write distinct key chunks of one channel row
@@ -634,19 +622,16 @@ qvg_attention_fused(const AttnParams p) {
         bk.finish(p, nlut, h, vk);
         // K rows: rotary embedding of the reconstructed values at their
         // positions (past the end: the last token's, result unused), then bf16
-        const int pa = min(tok0, last), pz = min(tok0 + 1, last);
-        const bool one_hi = (pa >> 10) == (pz >> 10);   // the two positions share the high entry
-        float2 hi[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) hi[e] = __ldg(p.rope_hi + (pa >> 10) * (kD / 2) + 4 * cb + e);
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
           uint32_t w4[4];
-          const int pos = rr == 0 ? pa : pz;
+          const float4* cs4 = reinterpret_cast<const float4*>(p.rope + (int64_t)min(tok0 + rr, last) * (kD / 2) + 4 * cb);
+          const float4 c01 = __ldg(cs4), c23 = __ldg(cs4 + 1);
+          const float2 csv[4] = {make_float2(c01.x, c01.y), make_float2(c01.z, c01.w), make_float2(c23.x, c23.y),
+                                 make_float2(c23.z, c23.w)};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 h2 = one_hi ? hi[e] : __ldg(p.rope_hi + (pos >> 10) * (kD / 2) + 4 * cb + e);
-            const float2 cs = rope_combine(h2, __ldg(p.rope_lo + (pos & (kRopeLo - 1)) * (kD / 2) + 4 * cb + e));
+            const float2 cs = csv[e];
             const float a = vk[rr][2 * e], b = vk[rr][2 * e + 1];
             w4[e] = pack_bf16(__fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y)),
                               __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x)));
@@ -911,20 +896,16 @@ qvg_attention_fused(const AttnParams p) {
   }
 }
 
-// (cos, sin) tables of the rotary angles in fp64, rounded to fp32:
-// hi[a][i] for the angle 1024 a theta_i, lo[b][i] for b theta_i.
-__global__ void qvg_rope_tables_kernel(float2* hi, float2* lo, int n_hi, double base) {
+// The (cos, sin) table of the rotary angles, formed in fp64 and rounded to
+// fp32: rope[p][i] for the angle p theta_i, theta_i = base^(-2i/d).
+__global__ void qvg_rope_tables_kernel(float2* rope, int64_t rows, double base) {
   const int i = threadIdx.x % (kD / 2);
-  const int row = blockIdx.x * (blockDim.x / (kD / 2)) + threadIdx.x / (kD / 2);
-  if (row >= n_hi + kRopeLo) return;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / (kD / 2)) + threadIdx.x / (kD / 2);
+  if (row >= rows) return;
   const double theta = pow(base, -2.0 * i / (double)kD);
-  double a;
-  float2* dst;
-  if (row < n_hi) { a = (double)row * kRopeLo * theta; dst = hi + (int64_t)row * (kD / 2) + i; }
-  else { a = (double)(row - n_hi) * theta; dst = lo + (int64_t)(row - n_hi) * (kD / 2) + i; }
-  double s, c;
-  sincos(a, &s, &c);
-  *dst = make_float2(__double2float_rn(c), __double2float_rn(s));
+  double sn, cs;
+  sincos((double)row * theta, &sn, &cs);
+  rope[row * (kD / 2) + i] = make_float2(__double2float_rn(cs), __double2float_rn(sn));
 }
 
 }  // namespace
@@ -933,12 +914,11 @@ size_t attention_smem_bytes() {
   return 1024 + (size_t)(kAtQTiles + 4) * kAtOpBytes + 32 * sizeof(float2) + sizeof(AtBars);
 }
 
-cudaError_t launch_rope_tables(void* tables, int n_hi, double base, cudaStream_t s) {
-  float2* hi = reinterpret_cast<float2*>(static_cast<char*>(tables) + kRopeHeaderBytes);
-  float2* lo = hi + (size_t)n_hi * (kD / 2);
-  const int rows = n_hi + kRopeLo;
+cudaError_t launch_rope_tables(void* tables, int64_t max_pos, double base, cudaStream_t s) {
+  float2* rope = reinterpret_cast<float2*>(static_cast<char*>(tables) + kRopeHeaderBytes);
+  const int64_t rows = max_pos + 1;
   const int per = 256 / (kD / 2);
-  qvg_rope_tables_kernel<<<(rows + per - 1) / per, 256, 0, s>>>(hi, lo, n_hi, base);
+  qvg_rope_tables_kernel<<<(unsigned)((rows + per - 1) / per), 256, 0, s>>>(rope, rows, base);
   return cudaGetLastError();
 }
 
@@ -1064,11 +1044,10 @@ cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s) {
   }
   p.Q = static_cast<const __nv_bfloat16*>(a.Q);
   p.qpos = a.qpos;
-  p.rope_hi = reinterpret_cast<const float2*>(static_cast<const char*>(a.tables) + kRopeHeaderBytes);
-  p.rope_lo = p.rope_hi + (size_t)a.n_hi * (kD / 2);
+  p.rope = reinterpret_cast<const float2*>(static_cast<const char*>(a.tables) + kRopeHeaderBytes);
   p.O = a.O;
   p.status = reinterpret_cast<uint32_t*>(const_cast<void*>(a.tables));
-  p.max_pos = (int64_t)a.n_hi * kRopeLo - 1;
+  p.max_pos = a.max_pos;
   p.Nk = a.Nk; p.Nq = a.Nq; p.H = a.H; p.K = a.K; p.T = a.T; p.G = a.G; p.sym = a.sym;
   p.sl = 1.4426950408889634f / sqrtf((float)kD);
   const size_t smem = attention_smem_bytes();

@@ -535,9 +535,8 @@ qvg_status qvg_dequantize(const qvg_config* cfg, const qvg_packed* packed, qvg_d
 }
 
 size_t qvg_rope_tables_bytes(int32_t d, int64_t max_pos) {
-  if (d != kD || max_pos < 0 || max_pos >= (int64_t(1) << 40)) return 0;
-  const int64_t n_hi = max_pos / 1024 + 1;
-  return kRopeHeaderBytes + (size_t)(n_hi + 1024) * (kD / 2) * sizeof(float) * 2;
+  if (d != kD || max_pos < 0 || max_pos >= kRopeMaxPositions) return 0;
+  return kRopeHeaderBytes + (size_t)(max_pos + 1) * kRopeRowBytes;
 }
 
 qvg_status qvg_rope_tables(double base, int32_t d, int64_t max_pos, void* tables, size_t bytes,
@@ -546,9 +545,8 @@ qvg_status qvg_rope_tables(double base, int32_t d, int64_t max_pos, void* tables
   if (need == 0 || !(base > 1.0) || tables == nullptr || !aligned(tables, 16)) return QVG_ERR_INVALID_ARG;
   if (bytes < need) return QVG_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
-  const int n_hi = (int)(max_pos / 1024 + 1);
   QVG_TRY(cudaMemsetAsync(tables, 0, 16, s));
-  return cuda_status(plaunch(K_ROPE, s, [&] { return launch_rope_tables(tables, n_hi, base, s); }));
+  return cuda_status(plaunch(K_ROPE, s, [&] { return launch_rope_tables(tables, max_pos, base, s); }));
 }
 
 // The split of qvg_attention_set_split (0 = the library's choice).
@@ -582,15 +580,15 @@ qvg_status qvg_attention(const qvg_config* cfg, const qvg_packed* k, const qvg_p
   if (Nk < 1 || Nq < 1 || Q == nullptr || q_pos == nullptr || tables == nullptr || O == nullptr ||
       !aligned(Q, 16) || !aligned(O, 16) || !aligned(tables, 16) || Nq >= (int64_t(1) << 31) * 128)
     return QVG_ERR_INVALID_ARG;
-  const size_t row_bytes = (kD / 2) * sizeof(float) * 2;
-  if (tables_bytes < kRopeHeaderBytes + 1024 * row_bytes + row_bytes) return QVG_ERR_INVALID_ARG;
-  const int64_t n_hi = (int64_t)((tables_bytes - kRopeHeaderBytes) / row_bytes) - 1024;
-  if (Nk - 1 > n_hi * 1024 - 1) return QVG_ERR_INVALID_ARG;        // the cache's positions must be covered
+  if (tables_bytes < kRopeHeaderBytes + kRopeRowBytes) return QVG_ERR_INVALID_ARG;
+  const int64_t max_pos = std::min<int64_t>((int64_t)((tables_bytes - kRopeHeaderBytes) / kRopeRowBytes),
+                                            kRopeMaxPositions) - 1;
+  if (Nk - 1 > max_pos) return QVG_ERR_INVALID_ARG;                // the cache's positions must be covered
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
   st = peek_sticky(tables, s);
   if (st != QVG_OK) return st;
   AttentionArgs a{};
-  a.k = k; a.v = v; a.Q = Q; a.qpos = q_pos; a.tables = tables; a.n_hi = (int)n_hi; a.O = O;
+  a.k = k; a.v = v; a.Q = Q; a.qpos = q_pos; a.tables = tables; a.max_pos = max_pos; a.O = O;
   a.Nk = Nk; a.Nq = Nq; a.H = H; a.K = cfg->K; a.T = cfg->T; a.G = cfg->group_size; a.sym = sym ? 1 : 0;
   a.split = g_attention_split.load(std::memory_order_relaxed);
   st = cuda_status(plaunch(K_ATTN, s, [&] { return launch_attention(a, s); }));

@@ -152,17 +152,19 @@ cudaError_t launch_update_centroids(const UpdateParams& p, int dtype, cudaStream
 
 // ---- attention over the compressed cache (kernel_attention.cu)
 // Rotary tables: a 256-byte header (its first 4 bytes are the status word
-// of the attention calls that use the tables), then hi[n_hi][d/2] and
-// lo[1024][d/2] (cos, sin) pairs in fp32.
+// of the attention calls that use the tables), then (cos, sin) in fp32 of
+// p theta_i for every position p = 0 .. max_pos and pair i < d/2.
 constexpr size_t kRopeHeaderBytes = 256;
-cudaError_t launch_rope_tables(void* tables, int n_hi, double base, cudaStream_t s);
+constexpr size_t kRopeRowBytes = (kD / 2) * 2 * sizeof(float);
+constexpr int64_t kRopeMaxPositions = int64_t(1) << 24;
+cudaError_t launch_rope_tables(void* tables, int64_t max_pos, double base, cudaStream_t s);
 struct AttentionArgs {
   const qvg_packed* k;         // K cache: H blocks of Nk tokens (bf16 tables)
   const qvg_packed* v;         // V cache, same configuration
   const void* Q;               // [H][Nq][d] bf16, before the rotary embedding
   const int64_t* qpos;         // [Nq]
   const void* tables;          // rotary tables (header + hi + lo)
-  int n_hi;                    // rows of the hi table
+  int64_t max_pos;             // largest position the tables cover
   float* O;                    // [H][Nq][d] fp32
   int64_t Nk, Nq;
   int H, K, T, G, sym;

@@ -265,15 +265,16 @@ QVG_API qvg_status qvg_static_status(qvg_stream_t stream);
 
 /* Bytes of the rotary tables for head dimension d and positions
  * 0 .. max_pos: a 256-byte header, then (cos, sin) of p * theta_i in fp32
- * for p = 1024 a and for p = b < 1024.  0 for unsupported arguments
- * (d != 128).  Host-only. */
+ * for every position p and pair i < d/2 (512 bytes a position at d = 128).
+ * 0 for unsupported arguments (d != 128, max_pos < 0 or >= 2^24).
+ * Host-only. */
 QVG_API size_t qvg_rope_tables_bytes(int32_t d, int64_t max_pos);
 
 /* Fill the rotary tables (DEVICE, caller-owned, 16-byte aligned, `bytes`
  * from qvg_rope_tables_bytes) for theta_i = base^(-2i/d), the RoFormer form:
  * channel pair (2i, 2i+1) of a token at position p is turned by p * theta_i.
  * The angles and their cosines and sines are formed in fp64 on the device and
- * rounded to fp32.  The header's first 4 bytes are the status word of the
+ * rounded once to fp32.  The header's first 4 bytes are the status word of the
  * qvg_attention calls that use the tables (read and cleared by
  * qvg_workspace_status on the tables buffer).  Errors: INVALID_ARG (base
  * <= 1, d != 128, NULL), WORKSPACE_TOO_SMALL, CUDA. */

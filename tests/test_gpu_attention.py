@@ -154,7 +154,7 @@ def test_attention_reports_a_stale_timeout_and_rejects_uncovered_positions(q):
     kp = q.quantize(X, cfg)
     Q = torch.zeros((1, 8, 128), dtype=torch.bfloat16, device="cuda")
     pos = torch.arange(8, dtype=torch.int64, device="cuda")
-    small = q.rope_tables(100)                       # positions 0 .. 1023 are covered
+    small = q.rope_tables(400)                       # positions 0 .. 400 are covered
     big = q.rope_tables(5000)
     q.attention(kp, kp, Q, pos, big)
     torch.cuda.synchronize()
