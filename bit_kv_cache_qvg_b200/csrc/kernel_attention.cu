@@ -60,6 +60,7 @@ constexpr int kAtTile = 128;                    // queries per CTA, cached token
 constexpr int kAtOpBytes = kAtTile * kD * 2;    // one 128 x 128 bf16 operand: 32 KB
 constexpr uint64_t kAtWaitNs = 2000000000ull;   // 2 s per bounded wait
 constexpr int kAtMaxSplit = 8;                  // CTAs per cluster, at most (the portable cluster size)
+constexpr int kAtMaxGlobalSplit = 16;           // ranges of a global split, at most
 constexpr int kMaxDevices = 64;
 
 struct AttnParams {
@@ -78,6 +79,9 @@ struct AttnParams {
   int H, K, T, G, sym;
   int split;                      // cluster CTAs (per query block) over ranges of the cache's tiles
   int pair;                       // 2: two CTAs (two query blocks) share each tile's reconstruction
+  int gsplit;                     // ranges of the cache merged through global memory (1: none)
+  float* part_O;                  // [gsplit][H][Nq][d]: unnormalised O of each range
+  float2* part_ml;                // [gsplit][H][Nq]: (row maximum, row sum) of each range
   float sl;                       // log2(e) / sqrt(d)
 };
 
@@ -485,12 +489,15 @@ qvg_attention_fused(const AttnParams p) {
   const int h = blockIdx.y;
   // A cluster = pair x split CTAs.  Cluster rank = sr * pair + pr: the pair
   // (pr = 0, 1) holds two neighbouring blocks of 256 queries and shares the
-  // reconstruction of every tile; split rank sr takes tiles
-  // j_begin .. j_begin + ntiles - 1 of the cache (at least one each).
+  // reconstruction of every tile; split rank sr takes one range of the
+  // cache's tiles.  Clusters x = unit * gsplit + gs take range gs of a
+  // global split (merged through global memory by qvg_attention_merge).
   const int csize = p.pair * p.split;
   const int rank = (int)(blockIdx.x % (unsigned)csize);
   const int pr = rank % p.pair, sr = rank / p.pair;
-  const int64_t q0 = ((int64_t)(blockIdx.x / (unsigned)csize) * p.pair + pr) * (kAtQTiles * kAtTile);
+  const unsigned ug = blockIdx.x / (unsigned)csize;
+  const int gs = (int)(ug % (unsigned)p.gsplit);
+  const int64_t q0 = ((int64_t)(ug / (unsigned)p.gsplit) * p.pair + pr) * (kAtQTiles * kAtTile);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -550,8 +557,11 @@ qvg_attention_fused(const AttnParams p) {
   // S of query tile t at column 128 t, O of query tile t at column 256 + 128 t
   const uint32_t tS = tmem, tO = tmem + 256;
   const int64_t ntot = (p.Nk + kAtTile - 1) / kAtTile;
-  const int j_begin = (int)(ntot * sr / p.split);
-  const int ntiles = (int)(ntot * (sr + 1) / p.split) - j_begin;   // this CTA's tiles
+  // range gs * split + sr of gsplit * split (one of the two is 1): tiles
+  // j_begin .. j_begin + ntiles - 1, at least one
+  const int parts = p.gsplit * p.split, part = gs * p.split + sr;
+  const int j_begin = (int)(ntot * part / parts);
+  const int ntiles = (int)(ntot * (part + 1) / parts) - j_begin;   // this CTA's tiles
   int s_issued = 0, o_issued = 0;                   // products committed (the issuing threads 0 and 128)
   float m_fin = 0.0f, l_fin = 0.0f;                 // the softmax thread's row maximum and sum at the end
 
@@ -803,14 +813,19 @@ qvg_attention_fused(const AttnParams p) {
     m_fin = m_run;
     l_fin = l_run;
     if (ok && ntiles > 0 && p.split == 1) {
+      // O / l, or (a range of a global split) the unnormalised O with the
+      // row's maximum and sum
       const int64_t q = q0 + g * kAtTile + qi;
-      const float inv = 1.0f / l_run;
+      const bool partial = p.gsplit > 1;
+      const float inv = partial ? 1.0f : 1.0f / l_run;
+      float* orow = partial ? p.part_O + (((int64_t)gs * p.H + h) * p.Nq + q) * kD : p.O + ((int64_t)h * p.Nq + q) * kD;
+      if (partial && q < p.Nq) p.part_ml[((int64_t)gs * p.H + h) * p.Nq + q] = make_float2(m_run, l_run);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t rg[32];
         tld32(tOt + lane_base + (uint32_t)(32 * c), rg);
         if (q < p.Nq) {
-          float4* dst = reinterpret_cast<float4*>(p.O + ((int64_t)h * p.Nq + q) * kD + 32 * c);
+          float4* dst = reinterpret_cast<float4*>(orow + 32 * c);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             dst[e] = make_float4(__uint_as_float(rg[4 * e]) * inv, __uint_as_float(rg[4 * e + 1]) * inv,
@@ -894,6 +909,34 @@ qvg_attention_fused(const AttnParams p) {
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
   }
+}
+
+// The ranges of a global split merged, a warp per query row (a lane per four
+// channels): O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, M = max_s m_s,
+// the rescaling of the cluster merge.
+__global__ void __launch_bounds__(256)
+qvg_attention_merge(const float* part_O, const float2* part_ml, float* O, int64_t rows, int S) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float M = -3.0e38f;
+  for (int s = 0; s < S; ++s) {
+    const float2 ml = __ldg(part_ml + s * rows + row);
+    if (ml.y > 0.0f) M = fmaxf(M, ml.x);
+  }
+  float L = 0.0f;
+  float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int s = 0; s < S; ++s) {
+    const float2 ml = __ldg(part_ml + s * rows + row);
+    const float w = ml.y > 0.0f ? exp2_approx(ml.x - M) : 0.0f;
+    if (w > 0.0f) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(part_O + (s * rows + row) * kD) + lane);
+      acc.x += w * x.x; acc.y += w * x.y; acc.z += w * x.z; acc.w += w * x.w;
+      L += w * ml.y;
+    }
+  }
+  const float inv = 1.0f / L;
+  reinterpret_cast<float4*>(O + row * kD)[lane] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
 }
 
 // The (cos, sin) table of the rotary angles, formed in fp64 and rounded to
@@ -985,54 +1028,91 @@ static int resident_clusters(int split) {
   return n;
 }
 
-// The cluster shape: pair = 2 when there are at least two blocks of 256
-// queries (two CTAs share every tile's reconstruction), and the split of the
-// cache with the least estimated time, (waves of resident clusters) x
-// (tiles per CTA + the fixed cost of a CTA, about two tiles), over 1 .. 4
-// ranges (cluster size pair x split at most 8); a positive `forced` split is
-// taken as it is.  Never more ranges than the cache has tiles.
-struct SplitPlan { int pair, split; };
+// Bytes of the partial results of a global split into S ranges.
+static size_t partial_bytes(int S, int H, int64_t Nq) {
+  return (size_t)S * H * Nq * (kD * sizeof(float) + sizeof(float2));
+}
+
+// The launch shape.  pair = 2 when there are at least two blocks of 256
+// queries (two CTAs share every tile's reconstruction).  The cache of a
+// query block is cut into ranges either inside the cluster (split 1 .. 4,
+// cluster size pair x split at most 8, merged through distributed shared
+// memory) or, when the workspace holds the partial results, over clusters
+// (gsplit 2 .. 16, merged by a second kernel).  The plan with the least
+// estimated time wins: (waves of resident clusters) x (tiles per CTA + the
+// fixed cost of a CTA, about two tiles), plus one tile for a merge kernel.
+// A positive `forced` split is a cluster split, taken as it is.  Never more
+// ranges than the cache has tiles.
+struct SplitPlan { int pair, split, gsplit; };
 template <int TT>
-static SplitPlan choose_split(int64_t Nk, int64_t Nq, int H, int forced) {
+static SplitPlan choose_split(int64_t Nk, int64_t Nq, int H, int forced, size_t ws_bytes) {
   const int64_t ntot = (Nk + kAtTile - 1) / kAtTile;
   const int64_t qblocks = (Nq + kAtQTiles * kAtTile - 1) / (kAtQTiles * kAtTile);
   const int pair = qblocks >= 2 ? 2 : 1;
   const int cap = kAtMaxSplit / pair;
   const int smax = (int)(ntot < cap ? ntot : cap);
-  if (forced > 0) return SplitPlan{pair, forced < smax ? forced : smax};
+  if (forced > 0) return SplitPlan{pair, forced < smax ? forced : smax, 1};
   const int64_t units = (qblocks + pair - 1) / pair * H;
-  int best = 1;
-  double best_cost = 0.0;
+  SplitPlan best{pair, 1, 1};
+  double best_cost = -1.0;
   for (int sp = 1; sp <= (smax < 4 ? smax : 4); ++sp) {
     const int n = resident_clusters<TT>(pair * sp);
     if (n <= 0) continue;
-    const double waves = (double)((units + n - 1) / n);
-    const double cost = waves * (double)((ntot + sp - 1) / sp + 2);
-    if (sp == 1 || cost < best_cost) { best = sp; best_cost = cost; }
+    const double cost = (double)((units + n - 1) / n) * (double)((ntot + sp - 1) / sp + 2);
+    if (best_cost < 0.0 || cost < best_cost) { best = SplitPlan{pair, sp, 1}; best_cost = cost; }
   }
-  return SplitPlan{pair, best};
+  const int n = resident_clusters<TT>(pair);
+  const int gmax = (int)(ntot < kAtMaxGlobalSplit ? ntot : kAtMaxGlobalSplit);
+  for (int gs = 2; n > 0 && gs <= gmax; ++gs) {
+    if (partial_bytes(gs, H, Nq) > ws_bytes) break;
+    const double cost = (double)((units * gs + n - 1) / n) * (double)((ntot + gs - 1) / gs + 2) + 1.0;
+    if (best_cost < 0.0 || cost < best_cost) { best = SplitPlan{pair, 1, gs}; best_cost = cost; }
+  }
+  return best;
 }
 
 template <int TT>
-static cudaError_t launch_attention_split(AttnParams& p, int64_t Nq, size_t smem, int forced, cudaStream_t s) {
-  const SplitPlan plan = choose_split<TT>(p.Nk, Nq, p.H, forced);
+static cudaError_t launch_attention_plan(AttnParams& p, int64_t Nq, size_t smem, int forced, size_t ws_bytes,
+                                         cudaStream_t s) {
+  const SplitPlan plan = choose_split<TT>(p.Nk, Nq, p.H, forced, ws_bytes);
   p.split = plan.split;
   p.pair = plan.pair;
+  p.gsplit = plan.gsplit;
+  // the partial results of a global split: O rows, then (maximum, sum) pairs
+  if (plan.gsplit > 1) p.part_ml = reinterpret_cast<float2*>(p.part_O + (size_t)plan.gsplit * p.H * Nq * kD);
   const int64_t qblocks = (Nq + kAtQTiles * kAtTile - 1) / (kAtQTiles * kAtTile);
   const int64_t units = (qblocks + plan.pair - 1) / plan.pair;
-  const dim3 grid((unsigned)(units * plan.pair * plan.split), (unsigned)p.H);
-  return launch_attention_t<TT>(p, grid, smem, s);
+  const dim3 grid((unsigned)(units * plan.gsplit * plan.pair * plan.split), (unsigned)p.H);
+  cudaError_t e = launch_attention_t<TT>(p, grid, smem, s);
+  if (e != cudaSuccess || plan.gsplit == 1) return e;
+  const int64_t rows = (int64_t)p.H * Nq;
+  qvg_attention_merge<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(p.part_O, p.part_ml, p.O, rows, plan.gsplit);
+  return cudaGetLastError();
 }
 
-int attention_split(int T, int64_t Nk, int64_t Nq, int H, int forced) {
+template <int TT>
+static SplitPlan plan_for(int64_t Nk, int64_t Nq, int H, int forced, size_t ws_bytes) {
+  return choose_split<TT>(Nk, Nq, H, forced, ws_bytes);
+}
+static SplitPlan plan_any(int T, int64_t Nk, int64_t Nq, int H, int forced, size_t ws_bytes) {
   switch (T) {
-    case 0: return choose_split<0>(Nk, Nq, H, forced).split;
-    case 1: return choose_split<1>(Nk, Nq, H, forced).split;
-    case 2: return choose_split<2>(Nk, Nq, H, forced).split;
-    case 3: return choose_split<3>(Nk, Nq, H, forced).split;
-    case 4: return choose_split<4>(Nk, Nq, H, forced).split;
-    default: return choose_split<-1>(Nk, Nq, H, forced).split;
+    case 0: return plan_for<0>(Nk, Nq, H, forced, ws_bytes);
+    case 1: return plan_for<1>(Nk, Nq, H, forced, ws_bytes);
+    case 2: return plan_for<2>(Nk, Nq, H, forced, ws_bytes);
+    case 3: return plan_for<3>(Nk, Nq, H, forced, ws_bytes);
+    case 4: return plan_for<4>(Nk, Nq, H, forced, ws_bytes);
+    default: return plan_for<-1>(Nk, Nq, H, forced, ws_bytes);
   }
+}
+
+int attention_split(int T, int64_t Nk, int64_t Nq, int H, int forced, size_t ws_bytes) {
+  const SplitPlan plan = plan_any(T, Nk, Nq, H, forced, ws_bytes);
+  return plan.split * plan.gsplit;
+}
+
+size_t attention_workspace_bytes(int T, int64_t Nk, int64_t Nq, int H, int forced) {
+  const SplitPlan plan = plan_any(T, Nk, Nq, H, forced, ~size_t(0));
+  return plan.gsplit > 1 ? partial_bytes(plan.gsplit, H, Nq) : 0;
 }
 
 cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s) {
@@ -1050,14 +1130,16 @@ cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s) {
   p.max_pos = a.max_pos;
   p.Nk = a.Nk; p.Nq = a.Nq; p.H = a.H; p.K = a.K; p.T = a.T; p.G = a.G; p.sym = a.sym;
   p.sl = 1.4426950408889634f / sqrtf((float)kD);
+  const size_t ws = a.workspace != nullptr ? a.ws_bytes : 0;
+  p.part_O = static_cast<float*>(a.workspace);
   const size_t smem = attention_smem_bytes();
   switch (a.T) {
-    case 0: return launch_attention_split<0>(p, a.Nq, smem, a.split, s);
-    case 1: return launch_attention_split<1>(p, a.Nq, smem, a.split, s);
-    case 2: return launch_attention_split<2>(p, a.Nq, smem, a.split, s);
-    case 3: return launch_attention_split<3>(p, a.Nq, smem, a.split, s);
-    case 4: return launch_attention_split<4>(p, a.Nq, smem, a.split, s);
-    default: return launch_attention_split<-1>(p, a.Nq, smem, a.split, s);
+    case 0: return launch_attention_plan<0>(p, a.Nq, smem, a.split, ws, s);
+    case 1: return launch_attention_plan<1>(p, a.Nq, smem, a.split, ws, s);
+    case 2: return launch_attention_plan<2>(p, a.Nq, smem, a.split, ws, s);
+    case 3: return launch_attention_plan<3>(p, a.Nq, smem, a.split, ws, s);
+    case 4: return launch_attention_plan<4>(p, a.Nq, smem, a.split, ws, s);
+    default: return launch_attention_plan<-1>(p, a.Nq, smem, a.split, ws, s);
   }
 }
 

@@ -557,16 +557,23 @@ int32_t qvg_attention_set_split(int32_t split) {
   return g_attention_split.exchange(split);
 }
 
-int32_t qvg_attention_split(const qvg_config* cfg, int64_t Nk, int32_t H, int64_t Nq) {
+int32_t qvg_attention_split(const qvg_config* cfg, int64_t Nk, int32_t H, int64_t Nq, size_t ws_bytes) {
   if (check_config(cfg, Nk, H, kD, QVG_BF16) != QVG_OK || Nk < 1 || Nq < 1) return -1;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) { (void)cudaGetLastError(); return -1; }
-  return attention_split(cfg->T, Nk, Nq, H, g_attention_split.load(std::memory_order_relaxed));
+  return attention_split(cfg->T, Nk, Nq, H, g_attention_split.load(std::memory_order_relaxed), ws_bytes);
+}
+
+size_t qvg_attention_workspace_bytes(const qvg_config* cfg, int64_t Nk, int32_t H, int64_t Nq) {
+  if (check_config(cfg, Nk, H, kD, QVG_BF16) != QVG_OK || Nk < 1 || Nq < 1) return 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) { (void)cudaGetLastError(); return 0; }
+  return attention_workspace_bytes(cfg->T, Nk, Nq, H, g_attention_split.load(std::memory_order_relaxed));
 }
 
 qvg_status qvg_attention(const qvg_config* cfg, const qvg_packed* k, const qvg_packed* v, int64_t Nk, int32_t H,
                          int32_t d, const void* Q, const int64_t* q_pos, int64_t Nq, const void* tables,
-                         size_t tables_bytes, float* O, qvg_stream_t stream_) {
+                         size_t tables_bytes, float* O, void* workspace, size_t ws_bytes, qvg_stream_t stream_) {
   qvg_status st = check_config(cfg, Nk, H, d, QVG_BF16);
   if (st != QVG_OK) return st;
   const bool sym = cfg->scale_mode == QVG_SCALE_SYM;
@@ -578,7 +585,8 @@ qvg_status qvg_attention(const qvg_config* cfg, const qvg_packed* k, const qvg_p
     if (!aligned(p->codes, 2)) return QVG_ERR_INVALID_ARG;
   }
   if (Nk < 1 || Nq < 1 || Q == nullptr || q_pos == nullptr || tables == nullptr || O == nullptr ||
-      !aligned(Q, 16) || !aligned(O, 16) || !aligned(tables, 16) || Nq >= (int64_t(1) << 31) * 128)
+      !aligned(Q, 16) || !aligned(O, 16) || !aligned(tables, 16) || !aligned(workspace, 16) ||
+      Nq >= (int64_t(1) << 31) * 128)
     return QVG_ERR_INVALID_ARG;
   if (tables_bytes < kRopeHeaderBytes + kRopeRowBytes) return QVG_ERR_INVALID_ARG;
   const int64_t max_pos = std::min<int64_t>((int64_t)((tables_bytes - kRopeHeaderBytes) / kRopeRowBytes),
@@ -591,6 +599,8 @@ qvg_status qvg_attention(const qvg_config* cfg, const qvg_packed* k, const qvg_p
   a.k = k; a.v = v; a.Q = Q; a.qpos = q_pos; a.tables = tables; a.max_pos = max_pos; a.O = O;
   a.Nk = Nk; a.Nq = Nq; a.H = H; a.K = cfg->K; a.T = cfg->T; a.G = cfg->group_size; a.sym = sym ? 1 : 0;
   a.split = g_attention_split.load(std::memory_order_relaxed);
+  a.workspace = workspace;
+  a.ws_bytes = workspace != nullptr ? ws_bytes : 0;
   st = cuda_status(plaunch(K_ATTN, s, [&] { return launch_attention(a, s); }));
   if (st == QVG_OK && fault_injected("stream")) st = QVG_ERR_CUDA;
   return st;

@@ -169,11 +169,16 @@ struct AttentionArgs {
   int64_t Nk, Nq;
   int H, K, T, G, sym;
   int split;                   // CTAs per cluster over the cache of a query block; 0 = chosen here
+  void* workspace;             // partial results of a split over clusters (may be null)
+  size_t ws_bytes;
 };
 cudaError_t launch_attention(const AttentionArgs& a, cudaStream_t s);
-// The split launch_attention uses for these sizes (forced > 0: that one,
-// capped at the cache's tile count and the cluster limit).
-int attention_split(int T, int64_t Nk, int64_t Nq, int H, int forced);
+// The ranges the cache of a query block is cut into for these sizes and this
+// workspace (forced > 0: a cluster split of that many CTAs, capped at the
+// cache's tile count and the cluster limit).
+int attention_split(int T, int64_t Nk, int64_t Nq, int H, int forced, size_t ws_bytes);
+// The workspace the preferred plan needs (0: none).
+size_t attention_workspace_bytes(int T, int64_t Nk, int64_t Nq, int H, int forced);
 size_t attention_smem_bytes();
 
 }  // namespace qvg

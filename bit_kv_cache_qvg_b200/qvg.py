@@ -108,9 +108,10 @@ _SIGS = {
     "qvg_rope_tables": (C.c_int, [C.c_double, C.c_int32, C.c_int64, C.c_void_p, C.c_size_t, C.c_void_p]),
     "qvg_attention": (C.c_int, [C.POINTER(Config), C.POINTER(_Packed), C.POINTER(_Packed), C.c_int64, C.c_int32,
                                 C.c_int32, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_size_t, C.c_void_p,
-                                C.c_void_p]),
+                                C.c_void_p, C.c_size_t, C.c_void_p]),
     "qvg_attention_set_split": (C.c_int32, [C.c_int32]),
-    "qvg_attention_split": (C.c_int32, [C.POINTER(Config), C.c_int64, C.c_int32, C.c_int64]),
+    "qvg_attention_split": (C.c_int32, [C.POINTER(Config), C.c_int64, C.c_int32, C.c_int64, C.c_size_t]),
+    "qvg_attention_workspace_bytes": (C.c_size_t, [C.POINTER(Config), C.c_int64, C.c_int32, C.c_int64]),
     "qvg_profile_enable": (None, [C.c_int]),
     "qvg_profile_reset": (None, []),
     "qvg_profile_launches": (C.c_int64, []),
@@ -286,18 +287,25 @@ def rope_tables(max_pos: int, base: float = 10000.0, d: int = 128, device="cuda"
 
 
 def attention(kp: Packed, vp: Packed, Q: torch.Tensor, q_pos: torch.Tensor, tables: torch.Tensor,
-              O: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+              O: Optional[torch.Tensor] = None, stream=None, workspace=True) -> torch.Tensor:
     """qvg_attention: softmax(rope(Q) rope(K^)^T / sqrt(d)) V^ per head over the
     compressed caches kp (keys, before the rotary embedding) and vp (values);
-    Q [H][Nq][d] bf16, q_pos [Nq] int64 (device); returns O [H][Nq][d] fp32."""
+    Q [H][Nq][d] bf16, q_pos [Nq] int64 (device); returns O [H][Nq][d] fp32.
+    `workspace`: a uint8 device tensor, True (one of
+    qvg_attention_workspace_bytes is allocated) or None (no workspace)."""
     if Q.dim() != 3 or not Q.is_contiguous() or Q.dtype != torch.bfloat16:
         raise QvgError(1, "Q must be a contiguous bf16 [H][Nq][d] tensor")
     H, Nq, d = Q.shape
     if O is None:
         O = torch.empty((H, Nq, d), dtype=torch.float32, device=Q.device)
+    if workspace is True:
+        n = attention_workspace_bytes(kp.cfg, kp.N, H, Nq)
+        workspace = torch.empty(n, dtype=torch.uint8, device=Q.device) if n > 0 else None
+    ws_ptr, ws_n = (_ptr(workspace), workspace.numel()) if workspace is not None else (None, 0)
     ks, vs = kp.struct(), vp.struct()
     _check(lib().qvg_attention(C.byref(kp.cfg), C.byref(ks), C.byref(vs), kp.N, H, d, _ptr(Q),
-                               _ptr(q_pos), Nq, _ptr(tables), tables.numel(), _ptr(O), _stream(stream)),
+                               _ptr(q_pos), Nq, _ptr(tables), tables.numel(), _ptr(O), ws_ptr, ws_n,
+                               _stream(stream)),
            "qvg_attention")
     return O
 
@@ -311,13 +319,18 @@ def attention_set_split(split: int) -> int:
     return prev
 
 
-def attention_split(cfg: Config, Nk: int, H: int, Nq: int) -> int:
-    """qvg_attention_split: the split a qvg_attention call with these sizes
-    would use on the current device."""
-    n = int(lib().qvg_attention_split(C.byref(cfg), Nk, H, Nq))
+def attention_split(cfg: Config, Nk: int, H: int, Nq: int, ws_bytes: int = 0) -> int:
+    """qvg_attention_split: the ranges the cache of a query block is cut into
+    by a qvg_attention call with these sizes and a workspace of ws_bytes."""
+    n = int(lib().qvg_attention_split(C.byref(cfg), Nk, H, Nq, ws_bytes))
     if n < 0:
         raise QvgError(1, "qvg_attention_split")
     return n
+
+
+def attention_workspace_bytes(cfg: Config, Nk: int, H: int, Nq: int) -> int:
+    """qvg_attention_workspace_bytes: the workspace the preferred cut needs."""
+    return int(lib().qvg_attention_workspace_bytes(C.byref(cfg), Nk, H, Nq))
 
 
 def profile_enable(on: bool = True):

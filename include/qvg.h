@@ -293,6 +293,10 @@ QVG_API qvg_status qvg_rope_tables(double base, int32_t d, int64_t max_pos, void
  *   q_pos  DEVICE [Nq] int64
  *   tables DEVICE rotary tables (qvg_rope_tables); they must cover Nk - 1
  *   O      DEVICE [H][Nq][d] fp32, 16-byte aligned
+ *   workspace, ws_bytes  DEVICE scratch for the partial results of a cache
+ *          split over clusters (qvg_attention_workspace_bytes), 16-byte
+ *          aligned, caller-owned; NULL (or too small) keeps every split
+ *          inside one thread-block cluster
  * The products run on the tensor cores with bf16 operands (the rotated keys
  * and queries and the softmax weights are rounded to bf16) and fp32
  * accumulation; the softmax uses base-2 exponentials in fp32.
@@ -300,23 +304,31 @@ QVG_API qvg_status qvg_rope_tables(double base, int32_t d, int64_t max_pos, void
  * timeout recorded in the tables' status word by earlier, completed work). */
 QVG_API qvg_status qvg_attention(const qvg_config* cfg, const qvg_packed* k, const qvg_packed* v, int64_t Nk,
                          int32_t H, int32_t d, const void* Q, const int64_t* q_pos, int64_t Nq,
-                         const void* tables, size_t tables_bytes, float* O, qvg_stream_t stream);
+                         const void* tables, size_t tables_bytes, float* O, void* workspace, size_t ws_bytes,
+                         qvg_stream_t stream);
 
-/* qvg_attention splits the cache of each head and block of 256 queries over
- * a thread-block cluster of `split` CTAs, each over one range of the cache's
- * tiles of 128 tokens; the cluster merges their partial softmax sums through
- * distributed shared memory.  Each CTA rounds its softmax weights to bf16
- * against its own running maximum, so splits differ by such roundings (the
- * error bound of qvg_attention holds for every split).
- * By default (0) the library picks it from the device's cluster occupancy so
- * that the grid fills the SMs.  qvg_attention_set_split fixes it for the
- * process (1 .. 8, capped at the cache's tile count; 0 = automatic again) and
- * returns the previous setting, or -1 (nothing changed) for other values.
- * qvg_attention_split returns the split a qvg_attention call with these
- * sizes would use on the current device, or -1 for invalid arguments or no
- * device.  Host-only; neither launches work. */
+/* qvg_attention cuts the cache of each head and block of 256 queries into
+ * ranges of its tiles of 128 tokens, one CTA (or pair of CTAs, which share
+ * the reconstruction of two query blocks) per range, so that the grid fills
+ * the SMs.  The ranges are merged by the usual rescaling of partial softmax
+ * sums: inside a thread-block cluster (up to 4 ranges, through distributed
+ * shared memory), or, with a workspace, over clusters (up to 16 ranges,
+ * through the workspace and a second kernel).  Each range rounds its softmax
+ * weights to bf16 against its own running maximum, so cuts differ by such
+ * roundings (the error bound of qvg_attention holds for every cut).  By
+ * default the library picks the cut from the device's cluster occupancy.
+ *   qvg_attention_set_split fixes a cluster split for the process (1 .. 8
+ *     CTAs, capped at the cache's tile count and 4 for pairs; 0 = automatic
+ *     again) and returns the previous setting, or -1 (nothing changed).
+ *   qvg_attention_split returns the number of ranges a qvg_attention call
+ *     with these sizes and a workspace of ws_bytes would use on the current
+ *     device, or -1 for invalid arguments or no device.
+ *   qvg_attention_workspace_bytes returns the workspace the preferred cut
+ *     needs (0: none), or 0 for invalid arguments.
+ * Host-only; none launches work. */
 QVG_API int32_t qvg_attention_set_split(int32_t split);
-QVG_API int32_t qvg_attention_split(const qvg_config* cfg, int64_t Nk, int32_t H, int64_t Nq);
+QVG_API int32_t qvg_attention_split(const qvg_config* cfg, int64_t Nk, int32_t H, int64_t Nq, size_t ws_bytes);
+QVG_API size_t qvg_attention_workspace_bytes(const qvg_config* cfg, int64_t Nk, int32_t H, int64_t Nq);
 
 /* ------------------------------------------------------------------ */
 /* Diagnostics (no counterpart in the method; used by the benchmark).    */

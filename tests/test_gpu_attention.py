@@ -102,6 +102,19 @@ def test_attention_split_over_a_cluster_matches_oracle(q, ora, split, Nq):
     assert typical < 0.25
 
 
+def test_attention_split_over_clusters_matches_oracle(q, ora):
+    """With a workspace the cache of a query block is cut into up to 16
+    ranges over clusters, merged by a second kernel: here 32 tiles into 16
+    ranges for each of four pairs of query blocks."""
+    cfg = q.config(K=64, T=2, group_size=64, iters=3, scale_mode=0)
+    ws = q.attention_workspace_bytes(cfg, 4000, 2, 600)
+    assert ws == 16 * 2 * 600 * (128 * 4 + 8)
+    assert q.attention_split(cfg, 4000, 2, 600, ws) == 16
+    assert q.attention_split(cfg, 4000, 2, 600, ws - 1) < 16
+    typical = _run_case(q, ora, cfg, 2, 4000, 600, 0.05, seed=4004)
+    assert typical < 0.25
+
+
 def test_attention_splits_agree(q):
     """Each CTA of a split rounds its weights to bf16 against its own running
     maximum (as the unsplit kernel does against the maximum so far), so the
@@ -122,6 +135,8 @@ def test_attention_splits_agree(q):
             outs[split] = q.attention(kp, kp, Q, pos, tables).cpu()
         finally:
             q.attention_set_split(prev)
+    outs["clusters"] = q.attention(kp, kp, Q, pos, tables, workspace=None).cpu()
+    outs["global"] = q.attention(kp, kp, Q, pos, tables).cpu()
     torch.cuda.synchronize()
     assert q.workspace_status(tables) == 0
     scale = outs[1].abs().max().item()
@@ -138,6 +153,8 @@ def test_attention_split_setting_is_checked(q):
         q.attention_set_split(-1)
     auto = q.attention_split(cfg, 38000, 32, 1520)
     assert 1 <= auto <= 4
+    ws = q.attention_workspace_bytes(cfg, 38000, 32, 1520)
+    assert 1 <= q.attention_split(cfg, 38000, 32, 1520, ws) <= 16
     assert q.attention_split(cfg, 100, 32, 1520) == 1      # one tile: nothing to split
     prev = q.attention_set_split(3)
     try:
