@@ -150,3 +150,16 @@ def test_injected_allocation_and_stream_errors(q, monkeypatch):
         err = ((Y[:, c * 1560:(c + 1) * 1560].float() - x) ** 2).mean() / (x ** 2).mean()
         assert float(err) < 1e-2
     cache.close()
+    # attention over a compressed cache: the injected stream error, then a clean call
+    kp = q.quantize(X, cfg)
+    Q = torch.zeros((X.shape[0], 8, 128), dtype=torch.bfloat16, device="cuda")
+    pos = torch.arange(8, dtype=torch.int64, device="cuda")
+    tables = q.rope_tables(X.shape[1])
+    monkeypatch.setenv("QVG_FAULT_INJECT", "stream")
+    with pytest.raises(q.QvgError) as e:
+        q.attention(kp, kp, Q, pos, tables)
+    assert e.value.status == CUDA
+    monkeypatch.delenv("QVG_FAULT_INJECT")
+    O = q.attention(kp, kp, Q, pos, tables)
+    torch.cuda.synchronize()
+    assert torch.isfinite(O).all() and q.workspace_status(tables) == 0
