@@ -737,7 +737,12 @@ qvg_attention_fused(const AttnParams p) {
           }
         };
         if (valid == kAtTile) pass1(std::true_type{}); else pass1(std::false_type{});
-        const float m_new = fmaxf(m_run, mt * p.sl);
+        // The weights are taken against a reference maximum m_run, raised only
+        // when the row's maximum exceeds it by more than 8: the weights stay
+        // below 2^8 (exact in bf16 and fp32 alike), and O and l are rescaled
+        // rarely.  O / l is the same for any reference.
+        const float m_row = fmaxf(m_run, mt * p.sl);
+        const float m_new = m_row > m_run + 8.0f ? m_row : m_run;
         const float alpha = exp2_approx(m_run - m_new);
         // pass 2: bf16 weights 2^(sl s - m), two columns per packed op, and
         // their sum (of the rounded weights, the ones the product uses)
