@@ -77,6 +77,9 @@ def _run_case(q, ora, cfg, H, Nk, Nq, q_scale, seed, base=10000.0):
     (2, 4680, 130, 4, 16, 256, 1, 0.02),     # the QVG-Pro point, a Self-Forcing-scale chunk
     (2, 2900, 600, 2, 64, 128, 0, 0.05),     # three query blocks: two CTAs share each tile, one CTA has no queries
     (1, 1300, 512, 1, 32, 64, 1, 0.05),      # two whole query blocks, one pair
+    (2, 3000, 600, 4, 16, 256, 1, 0.02),     # the QVG-Pro point, paired (four stages: no prefetch of the next step)
+    (1, 2000, 300, 3, 32, 128, 0, 0.05),     # three stages, paired
+    (1, 700, 260, 5, 64, 32, 0, 0.05),       # five stages: the instance with the stage count at run time
 ])
 def test_attention_matches_oracle(q, ora, H, Nk, Nq, T, G, K, mode, q_scale):
     cfg = q.config(K=K, T=T, group_size=G, iters=3, scale_mode=mode)
