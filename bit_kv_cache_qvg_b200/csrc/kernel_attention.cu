@@ -16,31 +16,46 @@
 //
 // One CTA = one head x 256 queries (two query tiles of 128) x a range of the
 // cache's tiles of 128 tokens; 24 warps in three roles:
-//   * warps 8-23 dequantise each K and V tile (unpack, scale, add every
+//   * warps 8-23 (96 registers each, moved from the softmax warps by
+//     setmaxnreg) dequantise each K and V tile (unpack, scale, add every
 //     stage's centroid in reverse order, round to bf16 -- the arithmetic of
 //     qvg_dequant_fused), apply the rotary embedding to K, and store both
 //     into a two-stage ring in shared memory in the tensor core's K-major
 //     operand layout (128-byte swizzle): K rows (keys) with the channels
-//     contiguous, V transposed (channels) with the keys contiguous;
+//     contiguous, V transposed (channels) with the keys contiguous.  A
+//     thread's per-token bytes of the next step are loaded during the
+//     current one (at most two stages);
 //   * the first thread of each query tile's group issues S = Q' K'^T
 //     (tcgen05.mma kind::f16, M = N = K = 128, fp32 accumulators in tensor
 //     memory) when a stage is full, and O += P V (P read from tensor memory)
 //     when the group's softmax is done;
-//   * warps 0-3 and 4-7 (one per tensor-memory lane quarter, a thread per
-//     query) run the online softmax of the two query tiles (running row
-//     maximum and sum, base-2 exponentials), write P in bf16 over their S
-//     columns and rescale O in tensor memory.
+//   * warps 0-3 and 4-7 (48 registers each; one per tensor-memory lane
+//     quarter, a thread per query) run the online softmax of the two query
+//     tiles (base-2 exponentials against a reference maximum that rises only
+//     when a row's maximum exceeds it by more than 8), write P in bf16 over
+//     their S columns and, rarely, rescale O in tensor memory.
 // The two query tiles' groups run independently, so one group's softmax
-// overlaps the other's products.  When the cache is split over a cluster of
-// S CTAs (one key range each, so that the grid fills the SMs), each CTA
-// leaves its unnormalised O with its row maximum and sum in shared memory and
-// the cluster merges them through distributed shared memory (the usual
-// rescaling of partial softmax sums); otherwise O / l is written directly.
+// overlaps the other's products.
+//
+// Pairs: two CTAs of a cluster hold neighbouring blocks of 256 queries; each
+// reconstructs 64 keys of every tile and stores them into both CTAs' ring
+// stage through distributed shared memory, and a stage is freed by a commit
+// multicast to the pair once the products of both CTAs have read it.
+//
+// Cuts: the cache of a query block is cut into ranges so that the grid fills
+// the SMs.  Inside a cluster (split CTAs per query block) each CTA leaves its
+// unnormalised O with its row maximum and sum in shared memory and the
+// cluster merges them through distributed shared memory; over clusters
+// (gsplit ranges) they go to the caller's workspace and qvg_attention_merge
+// combines them (the usual rescaling of partial softmax sums).  With no cut,
+// O / l is written directly.
+//
 // The rotary (cos, sin) pairs come from a table of every position, formed
-// in fp64 and rounded to fp32 (qvg_rope_tables).  Every mbarrier wait is bounded; on
-// expiry the kernel records QVG_ERR_DEVICE_TIMEOUT in the status word at the
-// start of the tables buffer and stops.  No TMA and no multicast: the
-// operands are written by the threads that reconstruct them.
+// in fp64 and rounded to fp32 (qvg_rope_tables).  Every mbarrier wait is
+// bounded; on expiry the kernel records QVG_ERR_DEVICE_TIMEOUT in the status
+// word at the start of the tables buffer and stops.  No TMA and no
+// multicast loads: the operands are written by the threads that reconstruct
+// them.
 #include <cuda.h>
 
 #include <atomic>
@@ -54,9 +69,9 @@ namespace {
 
 constexpr int kAtThreads = 768;                 // 24 warps
 constexpr int kAtQTiles = 2;                    // query tiles per CTA (each reconstructed K/V tile serves both)
-constexpr int kAtSoftmaxThreads = 256;          // warps 0-7: softmax of the two query tiles (thread 0 issues the MMAs)
+constexpr int kAtSoftmaxThreads = 256;          // warps 0-7: softmax of the two query tiles (threads 0 and 128 issue the MMAs)
 constexpr int kAtReconThreads = 512;            // warps 8-23: reconstruction into the K/V ring
-constexpr int kAtTile = 128;                    // queries per CTA, cached tokens per tile
+constexpr int kAtTile = 128;                    // queries per query tile, cached tokens per tile
 constexpr int kAtOpBytes = kAtTile * kD * 2;    // one 128 x 128 bf16 operand: 32 KB
 constexpr uint64_t kAtWaitNs = 2000000000ull;   // 2 s per bounded wait
 constexpr int kAtMaxSplit = 8;                  // CTAs per cluster, at most (the portable cluster size)
