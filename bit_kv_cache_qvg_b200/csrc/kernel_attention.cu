@@ -103,8 +103,8 @@ struct AttnParams {
 struct __align__(8) AtBars {
   uint64_t s_done[2];       // S product of query tile g complete (tcgen05.commit)
   uint64_t o_done[2];       // O product of query tile g complete (tcgen05.commit)
-  uint64_t kv_full[2];      // ring stage reconstructed (the reconstruction threads arrive)
-  uint64_t kv_empty[2];     // ring stage free again: both O products that read it completed
+  uint64_t kv_full[2];      // ring stage reconstructed (lane 0 of every reconstruction warp of each CTA that writes it)
+  uint64_t kv_empty[2];     // ring stage free again: the O products of every CTA that read it completed
   uint32_t tmem_base;
   int abort_flag;
 };
