@@ -199,3 +199,44 @@ def test_status_queries_reject_missing_objects(q):
     L = q.lib()
     assert L.qvg_cache_status(None, None) == 1
     assert L.qvg_workspace_status(None, 0, None) == 1
+
+
+def test_attention_host_calls_without_a_gpu(q):
+    """qvg_rope_tables_bytes is the closed form 256 + (max_pos + 1) * 512 bytes
+    (d = 128, positions below 2^24); qvg_attention rejects missing or
+    misaligned arguments, and caches whose positions the tables do not cover,
+    before it touches the GPU; qvg_attention_set_split takes 0 .. 8 only; the
+    planner queries answer -1 and 0 without a device."""
+    import torch
+    L = q.lib()
+    assert L.qvg_rope_tables_bytes(128, 0) == 256 + 512
+    assert L.qvg_rope_tables_bytes(128, 39519) == 256 + 39520 * 512
+    assert L.qvg_rope_tables_bytes(128, (1 << 24) - 1) == 256 + (1 << 24) * 512
+    assert L.qvg_rope_tables_bytes(128, 1 << 24) == 0
+    assert L.qvg_rope_tables_bytes(128, -1) == 0
+    assert L.qvg_rope_tables_bytes(96, 100) == 0
+    cfg = q.config(K=16, T=1, group_size=64, iters=2)
+    p = q._Packed(0x2000, 0x3000, 0x4000, 0x5000, 0x6000)
+    tb = L.qvg_rope_tables_bytes(128, 999)                    # positions 0 .. 999
+
+    def att(Nk=1000, d=128, Q=0x10000, Nq=8, tbytes=tb, O=0x40000, ws=None, wsn=0, kp=p):
+        return L.qvg_attention(C.byref(cfg), C.byref(kp) if kp is not None else None, C.byref(p), Nk, 1, d, Q,
+                               0x20000, Nq, 0x30000, tbytes, O, ws, wsn, None)
+
+    assert att(Q=None) == 1
+    assert att(O=None) == 1
+    assert att(Q=0x10008) == 1                 # Q must be 16-byte aligned
+    assert att(ws=0x50008, wsn=4096) == 1      # and so must a workspace
+    assert att(Nq=0) == 1
+    assert att(Nk=1001) == 1                   # token 1000 lies beyond the tables
+    assert att(tbytes=256) == 1                # tables with no position
+    assert att(kp=None) == 1
+    assert att(d=96) != 0
+    assert L.qvg_attention_set_split(9) == -1 and L.qvg_attention_set_split(-1) == -1
+    prev = L.qvg_attention_set_split(3)
+    assert L.qvg_attention_set_split(prev) == 3
+    if not torch.cuda.is_available():
+        assert L.qvg_attention_split(C.byref(cfg), 1000, 1, 8, 0) == -1
+        assert L.qvg_attention_workspace_bytes(C.byref(cfg), 1000, 1, 8) == 0
+    assert L.qvg_attention_split(C.byref(q.config(K=300)), 1000, 1, 8, 0) == -1
+    assert L.qvg_attention_workspace_bytes(C.byref(cfg), 0, 1, 8) == 0
