@@ -803,6 +803,10 @@ def run_attention(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
     torch.cuda.synchronize()
     rel = float((O - ref.float()).norm() / ref.float().norm())
     flops = 4.0 * H * Nq * Nk * 128
+    # DRAM bytes of one qvg_attention_fused launch from the committed ncu table
+    # (captured at this workload; the table's units are heads)
+    tr = load_traffic().get("qvg_attention_fused")
+    traffic = tr[0] * H / tr[1] if tr else None
     packed = kp.nbytes() + vp.nbytes()
     io = Q.numel() * 2 + qpos.numel() * 8 + O.numel() * 4
     bytes_fused = packed + io + 2 * ws_n        # the partial results written and read back
@@ -819,7 +823,7 @@ def run_attention(args, wl, qvg, synth, dev, dist, rank, world, local, peaks):
                    "key_ranges": split, "workspace_bytes": ws_n,
                    "l2": "packed caches fit in L2; the baseline's bf16 caches do not"},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
-                     "frac": tflops / peaks["bf16_sus"], "traffic": None, "kernel": "qvg_attention_fused",
+                     "frac": tflops / peaks["bf16_sus"], "traffic": traffic, "kernel": "qvg_attention_fused",
                      "alg_flops_per_launch": flops},
         "fused": {"ms": ms_f, "hbm_bytes": bytes_fused},
         "dequantise_then_attend": {"ms": ms_u, "hbm_bytes": bytes_unfused,
